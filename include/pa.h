@@ -1,0 +1,219 @@
+/*
+ * pa.h — C ABI of the paged KV-cache decode library (sm_100a, one GPU).
+ *
+ * Three operations make up the decode hot path of PagedAttention:
+ *
+ *   pa_kv_append   scatter each step's new K/V vectors into their cache slots
+ *   pa_decode      single-query attention over K/V that a per-sequence block
+ *                  table gathers from fixed-size physical blocks
+ *   pa_block_copy  copy whole physical blocks (copy-on-write at a fork)
+ *
+ * Sources for what each call computes (page title, section):
+ *   [P1] "PagedAttention：大模型推理性能优化的核心技术解析" (bmjup.com),
+ *        § "PagedAttention 的核心工作机制与创新" (1 页表式管理, 2 写入时拷贝).
+ *   [P2] "AI 推理系列（十六）：PagedAttention——为什么 vLLM 能把 GPU 显存
+ *        “像操作系统一样”管理？" (wiblog.cn), § "PagedAttention 如何把连续
+ *        序列映射到离散显存块" (block table, flowchart), § "Copy-on-Write、
+ *        并行采样与 Prefix Caching 不是同一件事", § "非连续 KV 为什么需要
+ *        专门的 Attention Kernel".
+ *   [P3] "PagedAttention原理详解：GPU显存优化与模型路由技术" (kongchang.com),
+ *        § "显存消耗的三大来源" (single-query attention over cached K/V),
+ *        § "PagedAttention的三大核心优势" (reference counts, copy-on-write).
+ *   [P4] "vLLM的Paged Attention技术：高效注意力机制解析" (intelliparadigm.com),
+ *        § 2.2 内存布局优化, § 3.1 核函数签名解析, § 3.2 执行层次结构.
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions shared by every call
+ * ---------------------------------------------------------------------------
+ * Memory.  Every tensor pointer is a DEVICE pointer owned by the caller. The
+ *   library never allocates, frees or retains caller memory; it keeps only a
+ *   per-device 4-byte status word (see pa_sync_check).
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *   default stream). Every call only enqueues work on that stream and returns;
+ *   results are ready when the stream reaches that point.
+ * Status.  Every int-returning call returns PA_OK (0) or a negative PA_ERR_*
+ *   code. Argument errors are detected on the host before anything is
+ *   enqueued; pa_get_last_error() then returns a message for the calling
+ *   thread. Data-dependent errors (a block id or slot outside the pool, a
+ *   context longer than its block-table row) are detected by the kernels,
+ *   which skip the offending access, never fault, and record PA_ERR_BAD_INDEX
+ *   in the device status word that pa_sync_check reads.
+ * Element type.  PA_F32 (IEEE binary32) or PA_BF16 (bfloat16). q, out, k, v
+ *   and both caches of one call share that type. Attention arithmetic is
+ *   fp32 internally; outputs are rounded to nearest-even into the type.
+ *
+ * Cache layout (identical for k_cache and v_cache):
+ *
+ *   cache[num_blocks][num_kv_heads][block_size][head_dim], head_dim fastest.
+ *
+ *   Element (block b, kv head h, slot o, dim i) sits at linear index
+ *   ((b * num_kv_heads + h) * block_size + o) * head_dim + i.
+ *   Token position t of a sequence whose block table row is `tbl` lives in
+ *   block tbl[t / block_size], slot t % block_size [P2 block-table example:
+ *   logical blocks 0,1,2 -> physical 17,4,29]. Only the last block of a
+ *   sequence is partly filled [P2 same section, closing paragraph].
+ *   A slot index encodes (block, offset) as block * block_size + offset.
+ *   This replaces the 5-D [blocks, kv_heads, head_dim/x, block_size, x] key
+ *   layout of [P4 § 2.2]: here each (block, kv head) tile of one cache is one
+ *   contiguous, 16-byte aligned span of block_size * head_dim elements.
+ *
+ * Supported shapes: head_dim in {64, 128}; block_size a power of two in
+ *   [16, 256]; num_heads % num_kv_heads == 0 (query head h reads kv head
+ *   h / (num_heads / num_kv_heads), contiguous groups). All pointers must be
+ *   16-byte aligned.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+#define PA_OK               0
+#define PA_ERR_INVALID_ARG (-1) /* null pointer, negative size, bad shape     */
+#define PA_ERR_DTYPE       (-2) /* dtype not PA_F32 / PA_BF16                 */
+#define PA_ERR_ALIGN       (-3) /* a pointer is not 16-byte aligned           */
+#define PA_ERR_UNSUPPORTED (-4) /* head_dim / block_size not compiled         */
+#define PA_ERR_CUDA        (-5) /* a CUDA runtime call or launch failed       */
+#define PA_ERR_BAD_INDEX   (-6) /* a kernel met an out-of-range index         */
+#define PA_ERR_WORKSPACE   (-7) /* workspace missing or smaller than needed   */
+
+/* ---- element types ------------------------------------------------------ */
+#define PA_F32  0
+#define PA_BF16 1
+
+/* Shape of one physical KV pool (both k_cache and v_cache). */
+typedef struct pa_cache_desc {
+    int32_t num_blocks;   /* physical blocks in the pool                    */
+    int32_t num_kv_heads; /* KV heads stored per block                      */
+    int32_t block_size;   /* token slots per block                          */
+    int32_t head_dim;     /* elements per K or V vector                     */
+    int32_t dtype;        /* PA_F32 or PA_BF16                              */
+} pa_cache_desc;
+
+/*
+ * pa_kv_append — write this step's new K/V vectors into their slots.
+ *
+ * Computes the flowchart node "追加 KV" of [P2 § PagedAttention 如何把连续序列
+ * 映射到离散显存块]: for every token i in [0, num_tokens) with
+ * slot_mapping[i] >= 0, and every kv head h,
+ *     k_cache[slot / block_size][h][slot % block_size][:] = k[i][h][:]
+ *     v_cache[slot / block_size][h][slot % block_size][:] = v[i][h][:]
+ * as a bit-exact copy. slot_mapping[i] < 0 marks a padding token: skipped.
+ * Allocating a new block when the current one is full is the caller's job.
+ *
+ *   k, v          device, [num_tokens][num_kv_heads][head_dim], contiguous.
+ *   slot_mapping  device, int64 [num_tokens].
+ *   k_cache, v_cache  device pools in the layout above.
+ *   cache         host pointer to the pool's shape.
+ * Non-negative slots within one call must be distinct (otherwise which token
+ * lands in a slot is unspecified). A slot >= num_blocks * block_size is
+ * skipped and recorded as PA_ERR_BAD_INDEX. num_tokens == 0 is a no-op.
+ */
+int pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping,
+                 int32_t num_tokens, void* k_cache, void* v_cache,
+                 const pa_cache_desc* cache, void* stream);
+
+/*
+ * pa_decode — single-query paged attention for one decode step.
+ *
+ * For every sequence s, query head h (kh = h / (num_heads / num_kv_heads)):
+ *     n      = context_lens[s]
+ *     K_t    = k_cache[block_tables[s][t / block_size]][kh][t % block_size]
+ *     V_t    = v_cache[ ... same ... ],                  t = 0 .. n-1
+ *     out[s][h] = softmax_t(scale * q[s][h] . K_t) . V
+ * i.e. the unchanged attention of [P2 § 非连续 KV 为什么需要专门的 Attention
+ * Kernel] and [P3 § 显存消耗的三大来源] (one query against all cached K/V),
+ * read through the block table. n == 0 gives out[s][h] = 0.
+ * Long contexts are split into partitions of `partition_size` tokens, each
+ * producing (running max, running sum, normalised partial output) in the
+ * workspace, then merged by a log-sum-exp reduction (grid dimension
+ * "分区" of [P4 § 3.2]; the merge itself is not on the pages).
+ *
+ *   out           device, [num_seqs][num_heads][head_dim], type of the cache.
+ *   q             device, [num_seqs][num_heads][head_dim], type of the cache.
+ *   block_tables  device, int32 [num_seqs][block_table_stride]; entries past
+ *                 ceil(n / block_size) are never read.
+ *   context_lens  device, int32 [num_seqs], each in [0, max_context_len].
+ *   max_context_len  host bound on context_lens; must not exceed
+ *                 block_table_stride * block_size. A larger context is
+ *                 clipped to the bound and recorded as PA_ERR_BAD_INDEX.
+ *   scale         softmax scale (commonly 1/sqrt(head_dim)).
+ *   cache         host pointer; cache->num_kv_heads is the kv-head count.
+ *   partition_size  0 = library policy; -1 = never split; otherwise the
+ *                 tokens per partition, a positive multiple of 16.
+ *   workspace     device scratch of at least pa_decode_workspace_size(...)
+ *                 bytes (same arguments); may be NULL when that size is 0.
+ * The result does not depend on the physical placement of blocks: the
+ * arithmetic order depends only on logical token positions.
+ */
+int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+              const int32_t* block_tables, int32_t block_table_stride,
+              const int32_t* context_lens, int32_t max_context_len,
+              int32_t num_seqs, int32_t num_heads, float scale,
+              const pa_cache_desc* cache, int32_t partition_size,
+              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * pa_decode_workspace_size — bytes of device scratch pa_decode needs for the
+ * same (num_seqs, num_heads, max_context_len, cache, partition_size); 0 when
+ * the call will not split. Returns 0 and sets the last error on bad
+ * arguments. Queries the current device's SM count (cached per device).
+ */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads,
+                                int32_t max_context_len,
+                                const pa_cache_desc* cache,
+                                int32_t partition_size);
+
+/*
+ * pa_decode_num_partitions — number of context partitions pa_decode will use
+ * for these arguments (1 = no split); negative PA_ERR_* on bad arguments.
+ */
+int pa_decode_num_partitions(int32_t num_seqs, int32_t num_heads,
+                             int32_t max_context_len,
+                             const pa_cache_desc* cache,
+                             int32_t partition_size);
+
+/*
+ * pa_block_copy — copy whole physical blocks, the copy-on-write step that
+ * [P1 § 2 写入时拷贝], [P2 § Copy-on-Write、并行采样与 Prefix Caching] and
+ * [P3 § PagedAttention的三大核心优势] describe: when a sequence is about to
+ * write into a block that other sequences still share, the block is first
+ * copied to a private one.
+ *
+ * For every pair p: block dst = src_dst_pairs[2p+1] receives all slots of all
+ * kv heads of block src = src_dst_pairs[2p], in both k_cache and v_cache, as
+ * a bit-exact copy.
+ *   src_dst_pairs  device, int64 [num_pairs][2] = (src, dst).
+ * Within one call the dst ids must be distinct and no dst may also appear as
+ * a src (the result is then independent of copy order). Ids outside
+ * [0, num_blocks) are skipped and recorded as PA_ERR_BAD_INDEX. Deciding WHICH
+ * blocks to copy (reference counts) is the caller's host-side job.
+ */
+int pa_block_copy(const int64_t* src_dst_pairs, int32_t num_pairs,
+                  void* k_cache, void* v_cache, const pa_cache_desc* cache,
+                  void* stream);
+
+/*
+ * pa_sync_check — wait for `stream`, then read and clear the current device's
+ * status word. Returns PA_OK, PA_ERR_BAD_INDEX if any kernel since the last
+ * check met an out-of-range index, or PA_ERR_CUDA if the stream reported an
+ * error.
+ */
+int pa_sync_check(void* stream);
+
+/* Message describing the last failed call on this host thread ("" if none). */
+const char* pa_get_last_error(void);
+
+/* Constant name of a status code, e.g. "PA_ERR_ALIGN". */
+const char* pa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

@@ -1,0 +1,181 @@
+"""fp64 CPU oracle for the paged KV-cache decode path.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline leg and reference arm import this package. The
+product package ``paged_kv_cache_335_b200`` never imports it, and the C source
+``pa_oracle.c`` shares no code with the CUDA sources.
+
+What each function computes is documented in ``pa_oracle.c`` with the page and
+section it follows. Arrays are numpy: element type ``float32`` for binary32
+caches and ``uint16`` (raw bit patterns) for bfloat16 caches.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against
+something other than itself (a library attention routine, hand-written golden
+layouts, invariants and closed forms); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import contextlib
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+F32 = 0
+BF16 = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile ``pa_oracle.c`` into ``liboracle.so`` next to it (gcc, OpenMP).
+
+    No fast-math: the oracle keeps IEEE double semantics and source order.
+    """
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    compile_source(_SRC, tmp)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    p, i32 = ctypes.c_void_p, ctypes.c_int32
+    lib.oracle_kv_append.argtypes = [p, p, p, i32, p, p, i32, i32, i32, i32, i32]
+    lib.oracle_block_copy.argtypes = [p, i32, p, p, i32, i32, i32, i32, i32]
+    lib.oracle_decode.argtypes = [p, p, p, p, p, i32, p, i32, i32, i32, i32, i32,
+                                  i32, i32, ctypes.c_float, i32]
+    for f in (lib.oracle_kv_append, lib.oracle_block_copy, lib.oracle_decode,
+              lib.oracle_max_threads):
+        f.restype = ctypes.c_int
+    lib.oracle_max_threads.argtypes = []
+    return lib
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Temporarily route every call to another build of the oracle source (the
+    mutation tests use it to check that planted slips fail the pins)."""
+    global _lib
+    with _lock:
+        saved = _lib
+        _lib = _bind(path)
+    try:
+        yield
+    finally:
+        with _lock:
+            _lib = saved
+
+
+def compile_source(src_path: str, out_path: str) -> str:
+    """Compile an oracle C source with the same flags as ``build``."""
+    cmd = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-shared",
+           "-fPIC", "-std=c11", src_path, "-o", out_path, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out_path
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            _lib = _bind(_LIB_PATH)
+    return _lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.float32:
+        return F32
+    if a.dtype == np.uint16:
+        return BF16
+    raise TypeError(f"cache element type must be float32 or uint16 (bf16 bits), got {a.dtype}")
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        reason = {-1: "invalid argument", -2: "index outside the pool",
+                  -3: "out of memory"}.get(rc, str(rc))
+        raise OracleError(f"oracle {what}: {reason}")
+
+
+def _contig(a: np.ndarray, dtype=None) -> np.ndarray:
+    a = np.asarray(a)
+    if dtype is not None and a.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {a.dtype}")
+    if not a.flags.c_contiguous:
+        raise ValueError("arrays passed to the oracle must be C-contiguous")
+    return a
+
+
+def kv_append(k: np.ndarray, v: np.ndarray, slot_mapping: np.ndarray,
+              k_cache: np.ndarray, v_cache: np.ndarray) -> None:
+    """In place: write k[i], v[i] ([T][Hkv][d]) into slot_mapping[i] (int64)."""
+    k_cache = _contig(k_cache)
+    v_cache = _contig(v_cache, k_cache.dtype)
+    nb, hkv, bs, d = k_cache.shape
+    k = _contig(k, k_cache.dtype)
+    v = _contig(v, k_cache.dtype)
+    slot = _contig(slot_mapping, np.int64)
+    t = slot.shape[0]
+    if k.shape != (t, hkv, d) or v.shape != (t, hkv, d):
+        raise ValueError("k/v must be [num_tokens][num_kv_heads][head_dim]")
+    rc = _load().oracle_kv_append(_ptr(k), _ptr(v), _ptr(slot), t, _ptr(k_cache),
+                                  _ptr(v_cache), nb, hkv, bs, d, _dtype_code(k_cache))
+    _check(rc, "kv_append")
+
+
+def block_copy(pairs: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray) -> None:
+    """In place: for every (src, dst) row of ``pairs`` (int64 [P][2]) copy block src to dst."""
+    k_cache = _contig(k_cache)
+    v_cache = _contig(v_cache, k_cache.dtype)
+    nb, hkv, bs, d = k_cache.shape
+    pairs = _contig(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+    rc = _load().oracle_block_copy(_ptr(pairs), pairs.shape[0], _ptr(k_cache), _ptr(v_cache),
+                                   nb, hkv, bs, d, _dtype_code(k_cache))
+    _check(rc, "block_copy")
+
+
+def decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+           block_tables: np.ndarray, context_lens: np.ndarray, scale: float,
+           num_threads: int = 1) -> np.ndarray:
+    """Return out (float64 [S][H][d]) = softmax(scale q K^T) V over the paged context."""
+    k_cache = _contig(k_cache)
+    v_cache = _contig(v_cache, k_cache.dtype)
+    nb, hkv, bs, d = k_cache.shape
+    q = _contig(q, k_cache.dtype)
+    s, h, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the cache's")
+    tables = _contig(block_tables, np.int32)
+    ctx = _contig(context_lens, np.int32)
+    if tables.ndim != 2 or tables.shape[0] != s or ctx.shape != (s,):
+        raise ValueError("block_tables must be [S][stride], context_lens [S]")
+    out = np.zeros((s, h, d), dtype=np.float64)
+    rc = _load().oracle_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                               _ptr(tables), tables.shape[1], _ptr(ctx), s, h, hkv, nb, bs, d,
+                               _dtype_code(k_cache), float(np.float32(scale)), int(num_threads))
+    _check(rc, "decode")
+    return out
+
+
+def max_threads() -> int:
+    """Threads the oracle's OpenMP runtime would use by default."""
+    return int(_load().oracle_max_threads())

@@ -1,0 +1,373 @@
+"""Seeded synthetic decode workloads shared by the tests, the smoke check and
+the bench. Input construction only: it holds no attention arithmetic, and both
+the CUDA path and the CPU oracle consume exactly the bits it produces.
+
+Shapes follow the pages' workloads (LLaMA-shaped head counts, prompts around
+1024 tokens, contexts up to 32K, beam width 4 sharing a prompt):
+
+* "PagedAttention：大模型推理性能优化的核心技术解析", § 实际性能对比与量化数据:
+  LLaMA-2-13B, prompt 1024, 256 generated tokens.
+* "PagedAttention原理详解：GPU显存优化与模型路由技术", § 显存消耗的三大来源
+  (70B-shaped heads) and § PagedAttention的三大核心优势 (beam_width = 4 sharing).
+* "vLLM的Paged Attention技术：高效注意力机制解析", § 3.1 (HEAD_SIZE 128,
+  BLOCK_SIZE 16/32).
+
+Structure (context lengths, the shuffled pool, block tables, slots, copy
+pairs) is drawn on the host with ``numpy.random.default_rng(seed)``. Values
+(q, new k/v, both pools) are N(0, 1) drawn with a seeded ``torch.Generator`` on
+the device that will hold them; a test that needs them on the host copies them.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+from .block_manager import BlockManager
+
+DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@dataclass
+class Workload:
+    name: str
+    dtype: str
+    num_seqs: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    scale: float
+    seed: int
+    context_lens: np.ndarray          # int32 [S], includes this step's appended tokens
+    history_lens: np.ndarray          # int32 [S], tokens already in the cache before the step
+    block_tables: np.ndarray          # int32 [S][MB]; padding entries = poison_block
+    slot_mapping: np.ndarray          # int64 [T], this step's appended tokens
+    token_seq: np.ndarray             # int32 [T], sequence of each appended token
+    copy_pairs: np.ndarray            # int64 [P][2], this step's copy-on-write pairs
+    poison_block: int
+    partition_size: int = 0           # 0 = library policy
+    description: str = ""
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def torch_dtype(self):
+        return DTYPES[self.dtype]
+
+    @property
+    def elem_bytes(self) -> int:
+        return 4 if self.dtype == "f32" else 2
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.slot_mapping.shape[0])
+
+    @property
+    def max_context_len(self) -> int:
+        return int(self.context_lens.max()) if self.num_seqs else 0
+
+    def kv_bytes(self) -> int:
+        """Logical K+V bytes one decode call reads: every context token, K and V."""
+        return int(self.context_lens.astype(np.int64).sum()) * self.num_kv_heads * \
+            self.head_dim * 2 * self.elem_bytes
+
+    def decode_bytes(self) -> int:
+        """Algorithmic bytes of one decode call: K/V of every context token + q + out."""
+        qo = 2 * self.num_seqs * self.num_heads * self.head_dim * self.elem_bytes
+        return self.kv_bytes() + qo
+
+    def append_bytes(self) -> int:
+        """Bytes one append call moves: new k, v read and written once each."""
+        return 2 * 2 * self.num_tokens * self.num_kv_heads * self.head_dim * self.elem_bytes
+
+    def copy_bytes(self) -> int:
+        """Bytes one block-copy call moves: K and V block read + written per pair."""
+        blk = self.num_kv_heads * self.block_size * self.head_dim * self.elem_bytes
+        return 2 * 2 * int(self.copy_pairs.shape[0]) * blk
+
+    def unique_kv_bytes(self) -> int:
+        """K+V bytes of distinct (block, filled slot) pairs the decode reads."""
+        seen = {}
+        for s in range(self.num_seqs):
+            n = int(self.context_lens[s])
+            nb = -(-n // self.block_size)
+            for j in range(nb):
+                b = int(self.block_tables[s, j])
+                fill = min(self.block_size, n - j * self.block_size)
+                seen[b] = max(seen.get(b, 0), fill)
+        toks = sum(seen.values())
+        return toks * self.num_kv_heads * self.head_dim * 2 * self.elem_bytes
+
+
+# ---------------------------------------------------------------------------
+# structure
+# ---------------------------------------------------------------------------
+def _decode_structure(name, dtype, ctx, num_heads, num_kv_heads, head_dim, block_size,
+                      num_blocks, scale, seed, rng, partition_size=0, description=""):
+    """Sequences of the given final context lengths, each holding ctx-1 tokens
+    before the step and appending one token (position ctx-1) in it."""
+    ctx = np.asarray(ctx, dtype=np.int64)
+    s_count = ctx.shape[0]
+    order = rng.permutation(num_blocks)
+    poison = int(order[-1])                      # a valid id that no sequence owns
+    bm = BlockManager(num_blocks, block_size, order=order, reserved=(poison,))
+    seqs, slots, token_seq = [], [], []
+    for s in range(s_count):
+        n = int(ctx[s])
+        seq = bm.new_sequence(max(n - 1, 0))
+        if n >= 1:
+            slots.append(bm.append_slot(seq))
+            token_seq.append(s)
+        seqs.append(seq)
+    width = max(1, max(len(q.table) for q in seqs) if seqs else 1)
+    tables = bm.tables_array(seqs, width, poison)
+    return Workload(
+        name=name, dtype=dtype, num_seqs=s_count, num_heads=num_heads,
+        num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=block_size,
+        num_blocks=num_blocks, scale=float(np.float32(scale)), seed=seed,
+        context_lens=ctx.astype(np.int32), history_lens=np.maximum(ctx - 1, 0).astype(np.int32),
+        block_tables=tables, slot_mapping=np.asarray(slots, dtype=np.int64),
+        token_seq=np.asarray(token_seq, dtype=np.int32),
+        copy_pairs=np.zeros((0, 2), dtype=np.int64), poison_block=poison,
+        partition_size=partition_size, description=description)
+
+
+def _pool_size(ctx, block_size, factor=1.2):
+    demand = int(sum(-(-int(n) // block_size) for n in ctx))
+    return int(math.ceil(factor * demand)) + 1
+
+
+def tiny(seed: int = 0) -> Workload:
+    """4 seqs, 4 heads = 4 kv heads, d 64, bs 16, fp32, ctx U[1,200], 64-block
+    permuted pool, scale 1/8."""
+    rng = np.random.default_rng(seed)
+    ctx = rng.integers(1, 201, size=4)
+    return _decode_structure("tiny", "f32", ctx, 4, 4, 64, 16, 64, 0.125, seed, rng,
+                             description="4 seqs, 4/4 heads, d64, bs16, fp32, ctx U[1,200]")
+
+
+def llama7b(seed: int = 1, block_size: int = 16) -> Workload:
+    """LLaMA-7B-shaped layer: 64 seqs, 32 heads = 32 kv heads, d 128, bf16,
+    ctx U[512,2048] (including the token appended this step), pool 1.2x demand."""
+    rng = np.random.default_rng(seed)
+    ctx = rng.integers(512, 2049, size=64)
+    nb = _pool_size(ctx, block_size)
+    return _decode_structure("llama7b", "bf16", ctx, 32, 32, 128, block_size, nb,
+                             1.0 / math.sqrt(128), seed, rng,
+                             description="64 seqs, 32/32 heads, d128, bs16, bf16, ctx U[512,2048]")
+
+
+def llama13b(seed: int = 2, block_size: int = 16, sigma: float = 0.5) -> Workload:
+    """LLaMA-13B-shaped layer: 256 seqs, 40 heads = 40 kv heads, d 128, bf16,
+    ctx = clip(round(LogNormal(ln 1152, sigma)), 16, 4096): median = prompt 1024
+    + 128 generated. sigma is not given by the pages; 0.5 is this build's reading."""
+    rng = np.random.default_rng(seed)
+    ctx = np.clip(np.rint(rng.lognormal(math.log(1152.0), sigma, size=256)), 16, 4096)
+    ctx = ctx.astype(np.int64)
+    nb = _pool_size(ctx, block_size)
+    return _decode_structure(f"llama13b_bs{block_size}", "bf16", ctx, 40, 40, 128, block_size,
+                             nb, 1.0 / math.sqrt(128), seed, rng,
+                             description=f"256 seqs, 40/40 heads, d128, bs{block_size}, bf16, "
+                                         "ctx lognormal(median 1152, sigma 0.5) in [16,4096]")
+
+
+def llama70b_gqa(seed: int = 3, num_seqs: int = 8, context_len: int = 32768) -> Workload:
+    """70B-GQA long context: 8 seqs, 64 q heads / 8 kv heads, d 128, bs 16, bf16,
+    ctx 32768 each, split into partitions of 512 tokens."""
+    rng = np.random.default_rng(seed)
+    ctx = np.full(num_seqs, context_len, dtype=np.int64)
+    nb = _pool_size(ctx, 16)
+    return _decode_structure("llama70b_gqa", "bf16", ctx, 64, 8, 128, 16, nb,
+                             1.0 / math.sqrt(128), seed, rng, partition_size=512,
+                             description=f"{num_seqs} seqs, 64/8 heads, d128, bs16, bf16, "
+                                         f"ctx {context_len}, partitions of 512")
+
+
+def cow_beam4(seed: int = 4, num_prompts: int = 32, beam_width: int = 4,
+              prompt_len: int = 2048, aligned: bool = False, max_suffix: int = 256,
+              num_heads: int = 64, num_kv_heads: int = 8, head_dim: int = 128,
+              block_size: int = 16, dtype: str = "bf16") -> Workload:
+    """Copy-on-write parallel sampling: each prompt is prefilled once and shared
+    by ``beam_width`` beams through reference counts; in this step every beam
+    appends its own suffix of U[1, max_suffix] tokens. The first suffix token of
+    a beam falls into the prompt's partly filled tail block, which is still
+    shared, so beams 0..W-2 get a private copy (a ``pa_block_copy`` pair) and the
+    last beam, then the tail's only owner, writes in place.
+
+    A 2048-token prompt fills its last block exactly at block_size 16, leaving
+    nothing to copy; the reading used here shortens each prompt by U{1..15}
+    tokens (``aligned=False``). ``aligned=True`` keeps prompt_len exactly and
+    must give zero copies."""
+    rng = np.random.default_rng(seed)
+    if aligned:
+        plen = np.full(num_prompts, prompt_len, dtype=np.int64)
+    else:
+        plen = prompt_len - rng.integers(1, block_size, size=num_prompts)
+    suffix = rng.integers(1, max_suffix + 1, size=num_prompts * beam_width)
+    demand = sum(-(-int(p) // block_size) for p in plen)
+    for i in range(num_prompts):
+        for b in range(beam_width):
+            total = int(plen[i] + suffix[i * beam_width + b])
+            demand += -(-total // block_size) - int(plen[i]) // block_size
+    nb = int(math.ceil(1.2 * demand)) + 1
+    order = rng.permutation(nb)
+    poison = int(order[-1])
+    bm = BlockManager(nb, block_size, order=order, reserved=(poison,))
+    seqs, hist, ctx, slots, token_seq = [], [], [], [], []
+    for i in range(num_prompts):
+        prompt = bm.new_sequence(int(plen[i]))
+        beams = [bm.fork(prompt) for _ in range(beam_width)]
+        bm.free(prompt)                       # the prompt itself is no longer a sequence
+        for b, beam in enumerate(beams):
+            s = len(seqs)
+            n_new = int(suffix[i * beam_width + b])
+            hist.append(beam.length)
+            for _ in range(n_new):
+                slots.append(bm.append_slot(beam))
+                token_seq.append(s)
+            ctx.append(beam.length)
+            seqs.append(beam)
+    pairs = bm.take_copies()
+    width = max(len(s.table) for s in seqs)
+    tables = bm.tables_array(seqs, width, poison)
+    name = "cow_beam4_aligned" if aligned else "cow_beam4"
+    return Workload(
+        name=name, dtype=dtype, num_seqs=len(seqs), num_heads=num_heads,
+        num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=block_size, num_blocks=nb,
+        scale=float(np.float32(1.0 / math.sqrt(head_dim))), seed=seed,
+        context_lens=np.asarray(ctx, dtype=np.int32), history_lens=np.asarray(hist, np.int32),
+        block_tables=tables, slot_mapping=np.asarray(slots, dtype=np.int64),
+        token_seq=np.asarray(token_seq, dtype=np.int32), copy_pairs=pairs, poison_block=poison,
+        description=f"{num_prompts} prompts x beam {beam_width}, prompt ~{prompt_len} shared, "
+                    f"suffix U[1,{max_suffix}], {num_heads}/{num_kv_heads} heads, d{head_dim}, "
+                    f"bs{block_size}, {dtype}",
+        extra={"prompt_lens": plen.astype(np.int32), "suffix_lens": suffix.astype(np.int32),
+               "beam_width": beam_width, "refcount": bm.refcount.copy()})
+
+
+CONFIGS = {
+    "tiny": tiny,
+    "llama7b": llama7b,
+    "llama13b_bs16": lambda seed=2: llama13b(seed, 16),
+    "llama13b_bs32": lambda seed=2: llama13b(seed, 32),
+    "llama70b_gqa": llama70b_gqa,
+    "cow_beam4": cow_beam4,
+}
+
+
+def make(name: str, **kw) -> Workload:
+    if name not in CONFIGS:
+        raise KeyError(f"unknown workload {name!r}; known: {sorted(CONFIGS)}")
+    return CONFIGS[name](**kw)
+
+
+# ---------------------------------------------------------------------------
+# values
+# ---------------------------------------------------------------------------
+def make_values(wl: Workload, device="cpu", poison: bool = False, seed_offset: int = 0):
+    """q, new k/v and both pools, N(0,1) in the workload's dtype on ``device``.
+
+    With ``poison``, every cache slot that no sequence may read before this
+    step's writes is set to NaN: blocks no table references, the slots of each
+    sequence from its history length to the end of its last block (including
+    the slots this step's append must fill), and every copy destination. A
+    read of any of them, or a missed append or copy, turns outputs into NaN.
+    """
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(wl.seed * 1000003 + seed_offset)
+    dt = wl.torch_dtype
+    S, H, Hkv, d = wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim
+    q = torch.randn((S, H, d), generator=g, device=device, dtype=dt)
+    k_new = torch.randn((wl.num_tokens, Hkv, d), generator=g, device=device, dtype=dt)
+    v_new = torch.randn((wl.num_tokens, Hkv, d), generator=g, device=device, dtype=dt)
+    shape = (wl.num_blocks, Hkv, wl.block_size, d)
+    k_cache = torch.randn(shape, generator=g, device=device, dtype=dt)
+    v_cache = torch.randn(shape, generator=g, device=device, dtype=dt)
+    if poison:
+        blocks, offs, whole = poison_slots(wl)
+        if blocks.size:
+            bi = torch.as_tensor(blocks, device=device)
+            oi = torch.as_tensor(offs, device=device)
+            k_cache[bi, :, oi, :] = float("nan")
+            v_cache[bi, :, oi, :] = float("nan")
+        if whole.size:
+            wi = torch.as_tensor(whole, device=device)
+            k_cache[wi] = float("nan")
+            v_cache[wi] = float("nan")
+    return {"q": q, "k_new": k_new, "v_new": v_new, "k_cache": k_cache, "v_cache": v_cache}
+
+
+def poison_slots(wl: Workload):
+    """(block ids, slot offsets) of per-sequence unfilled slots, and ids of
+    whole blocks to poison (unreferenced blocks and copy destinations)."""
+    B = wl.block_size
+    blocks, offs = [], []
+    referenced = np.zeros(wl.num_blocks, dtype=bool)
+    for s in range(wl.num_seqs):
+        n = int(wl.context_lens[s])
+        h = int(wl.history_lens[s])
+        nb = -(-n // B)
+        referenced[wl.block_tables[s, :nb]] = True
+        for pos in range(h, nb * B):
+            blocks.append(int(wl.block_tables[s, pos // B]))
+            offs.append(pos % B)
+    whole = set(np.nonzero(~referenced)[0].tolist())
+    whole.update(int(x) for x in wl.copy_pairs[:, 1].tolist())
+    whole.add(wl.poison_block)
+    return (np.asarray(blocks, dtype=np.int64), np.asarray(offs, dtype=np.int64),
+            np.asarray(sorted(whole), dtype=np.int64))
+
+
+def to_numpy(t: torch.Tensor) -> np.ndarray:
+    """Host numpy view of a tensor: float32 stays float32; bfloat16 becomes its
+    uint16 bit patterns (the oracle's bf16 representation)."""
+    t = t.detach().contiguous().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float32:
+        return t.numpy()
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def subproblem(wl: Workload, k_cache: torch.Tensor, v_cache: torch.Tensor,
+               seq_ids, q: torch.Tensor | None = None):
+    """Host copy of the part of a (possibly device-resident) pool that the
+    sequences ``seq_ids`` read, with their block tables renumbered onto the
+    compact copy. Renumbering is a change of physical placement only.
+
+    Returns dict(q, k_cache, v_cache, block_tables, context_lens) as numpy.
+    """
+    seq_ids = [int(s) for s in seq_ids]
+    B = wl.block_size
+    used = []
+    index = {}
+    rows = []
+    for s in seq_ids:
+        n = int(wl.context_lens[s])
+        nb = -(-n // B)
+        row = []
+        for j in range(nb):
+            b = int(wl.block_tables[s, j])
+            if b not in index:
+                index[b] = len(used)
+                used.append(b)
+            row.append(index[b])
+        rows.append(row)
+    width = max([1] + [len(r) for r in rows])
+    tables = np.zeros((len(seq_ids), width), dtype=np.int32)
+    for i, r in enumerate(rows):
+        tables[i, :len(r)] = r
+    ids = torch.as_tensor(used if used else [0], dtype=torch.long, device=k_cache.device)
+    out = {
+        "k_cache": to_numpy(k_cache.index_select(0, ids)),
+        "v_cache": to_numpy(v_cache.index_select(0, ids)),
+        "block_tables": tables,
+        "context_lens": wl.context_lens[seq_ids].astype(np.int32),
+    }
+    if q is not None:
+        qi = torch.as_tensor(seq_ids, dtype=torch.long, device=q.device)
+        out["q"] = to_numpy(q.index_select(0, qi))
+    return out

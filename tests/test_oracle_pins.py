@@ -1,0 +1,369 @@
+"""Pins of the fp64 oracle against things other than itself.
+
+Each test names what fixes the expected value: a hand-written golden fixture,
+a library attention routine (torch's scaled_dot_product_attention in float64
+on the logically ordered, contiguous K/V), an invariant the pages state, or a
+closed form. Together they are chosen so that a plausible slip in the oracle
+(a dropped scale, a wrong kv-head grouping, a swapped block / offset, a
+transposed layout, an off-by-one context, a missing max shift, a wrong bf16
+widening) fails at least one of them.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_335_b200 import block_manager as bmod
+from paged_kv_cache_335_b200 import workloads as W
+from tests.conftest import read_golden
+
+
+def _bits_bf16(x: torch.Tensor) -> np.ndarray:
+    return x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _paged_from_stream(K, V, ctx, block_size, num_blocks, rng, dtype):
+    """Build a permuted paged pool from logical token streams K, V [S][Tmax][Hkv][d]
+    (float64 holding representable values) through the oracle's append and a block
+    manager; returns (k_cache, v_cache, tables)."""
+    S, Tmax, Hkv, d = K.shape
+    order = rng.permutation(num_blocks)
+    bm = bmod.BlockManager(num_blocks, block_size, order=order)
+    seqs, slots, toks = [], [], []
+    for s in range(S):
+        seq = bm.new_sequence(0)
+        for t in range(int(ctx[s])):
+            slots.append(bm.append_slot(seq))
+            toks.append((s, t))
+        seqs.append(seq)
+    width = max(1, max(len(q.table) for q in seqs))
+    tables = bm.tables_array(seqs, width, 0)
+    conv = (lambda a: a.astype(np.float32)) if dtype == "f32" else \
+        (lambda a: _bits_bf16(torch.from_numpy(a)))
+    kc = np.zeros((num_blocks, Hkv, block_size, d), dtype=np.float32 if dtype == "f32" else np.uint16)
+    vc = np.zeros_like(kc)
+    if toks:
+        kt = np.stack([K[s, t] for s, t in toks])
+        vt = np.stack([V[s, t] for s, t in toks])
+        oracle.kv_append(np.ascontiguousarray(conv(kt)), np.ascontiguousarray(conv(vt)),
+                         np.asarray(slots, dtype=np.int64), kc, vc)
+    return kc, vc, tables
+
+
+def _sdpa_reference(q, K, V, ctx, scale, num_kv_heads):
+    """torch float64 scaled_dot_product_attention on the contiguous context."""
+    S, H, d = q.shape
+    out = np.zeros((S, H, d))
+    for s in range(S):
+        n = int(ctx[s])
+        if n == 0:
+            continue
+        qs = torch.from_numpy(q[s]).view(1, H, 1, d)
+        ks = torch.from_numpy(np.ascontiguousarray(K[s, :n].transpose(1, 0, 2))).view(1, num_kv_heads, n, d)
+        vs = torch.from_numpy(np.ascontiguousarray(V[s, :n].transpose(1, 0, 2))).view(1, num_kv_heads, n, d)
+        o = torch.nn.functional.scaled_dot_product_attention(
+            qs, ks, vs, scale=scale, enable_gqa=(H != num_kv_heads))
+        out[s] = o.view(H, d).numpy()
+    return out
+
+
+def _random_case(seed, S, H, Hkv, d, B, max_ctx, dtype, num_blocks=None, qmul=1.0):
+    rng = np.random.default_rng(seed)
+    ctx = rng.integers(1, max_ctx + 1, size=S)
+    Tmax = int(ctx.max())
+    g = torch.Generator().manual_seed(seed)
+    qf = torch.randn((S, H, d), generator=g, dtype=torch.float64) * qmul
+    Kf = torch.randn((S, Tmax, Hkv, d), generator=g, dtype=torch.float64)
+    Vf = torch.randn((S, Tmax, Hkv, d), generator=g, dtype=torch.float64)
+    if dtype == "f32":
+        q_store = qf.to(torch.float32).numpy()
+        q_val = q_store.astype(np.float64)
+        K = Kf.to(torch.float32).double().numpy()
+        V = Vf.to(torch.float32).double().numpy()
+    else:
+        q_store = _bits_bf16(qf)
+        q_val = qf.to(torch.bfloat16).double().numpy()
+        K = Kf.to(torch.bfloat16).double().numpy()
+        V = Vf.to(torch.bfloat16).double().numpy()
+    demand = int(sum(-(-int(n) // B) for n in ctx))
+    nb = num_blocks or demand + 5
+    kc, vc, tables = _paged_from_stream(K, V, ctx, B, nb, rng, dtype)
+    return dict(ctx=ctx.astype(np.int32), q_store=q_store, q_val=q_val, K=K, V=V,
+                kc=kc, vc=vc, tables=tables)
+
+
+# ---------------------------------------------------------------------------
+# golden fixtures
+# ---------------------------------------------------------------------------
+def test_golden_append_layout():
+    g = read_golden("append_layout.txt")
+    nb, hkv, bs, d = (int(x) for x in g["shape"][0])
+    slots = np.asarray([int(x) for x in g["slots"][0]], dtype=np.int64)
+    T = slots.shape[0]
+    k = np.zeros((T, hkv, d), dtype=np.float32)
+    for i in range(T):
+        for h in range(hkv):
+            for j in range(d):
+                k[i, h, j] = 100 * i + 10 * h + j + 1
+    v = -k
+    kc = np.zeros((nb, hkv, bs, d), dtype=np.float32)
+    vc = np.zeros_like(kc)
+    oracle.kv_append(k, v, slots, kc, vc)
+    expect = np.asarray([float(x) for x in g["k"][0]], dtype=np.float32)
+    np.testing.assert_array_equal(kc.reshape(-1), expect)
+    np.testing.assert_array_equal(vc.reshape(-1), -expect)
+
+
+def test_golden_block_copy():
+    g = read_golden("block_copy.txt")
+    nb, hkv, bs, d = (int(x) for x in g["shape"][0])
+    pairs = np.asarray([int(x) for x in g["pairs"][0]], dtype=np.int64).reshape(-1, 2)
+    before = np.asarray([float(x) for x in g["before"][0]], dtype=np.float32)
+    after = np.asarray([float(x) for x in g["after"][0]], dtype=np.float32)
+    kc = before.reshape(nb, hkv, bs, d).copy()
+    vc = -kc
+    oracle.block_copy(pairs, kc, vc)
+    np.testing.assert_array_equal(kc.reshape(-1), after)
+    np.testing.assert_array_equal(vc.reshape(-1), -after)
+
+
+@pytest.mark.parametrize("ctx_len", [48, 40, 33])
+def test_block_table_worked_example(ctx_len):
+    """Logical blocks 0,1,2 in physical 17,4,29: decode through that table equals
+    attention over the contiguous K/V (torch SDPA, float64)."""
+    table = [int(x) for x in read_golden("block_table_17_4_29.txt")["table"][0]]
+    B, d, Hkv, H, nb = 16, 8, 2, 2, 32
+    g = torch.Generator().manual_seed(7)
+    K = torch.randn((1, ctx_len, Hkv, d), generator=g).float().double().numpy()
+    V = torch.randn((1, ctx_len, Hkv, d), generator=g).float().double().numpy()
+    q = torch.randn((1, H, d), generator=g).float().numpy()
+    kc = np.full((nb, Hkv, B, d), np.nan, dtype=np.float32)
+    vc = np.full_like(kc, np.nan)
+    slots = np.asarray([table[t // B] * B + t % B for t in range(ctx_len)], dtype=np.int64)
+    oracle.kv_append(np.ascontiguousarray(K[0].astype(np.float32)),
+                     np.ascontiguousarray(V[0].astype(np.float32)), slots, kc, vc)
+    out = oracle.decode(q, kc, vc, np.asarray([table], dtype=np.int32),
+                        np.asarray([ctx_len], dtype=np.int32), 0.25)
+    ref = _sdpa_reference(q.astype(np.float64), K, V, [ctx_len], float(np.float32(0.25)), Hkv)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-13)
+
+
+def test_golden_closed_form():
+    g = read_golden("decode_closed_form.txt")
+    qv, k0, k1, v0, v1, expect, tol = (float(x) for x in g["case"][0])
+    kc = np.asarray([k0, k1], dtype=np.float32).reshape(1, 1, 2, 1)
+    vc = np.asarray([v0, v1], dtype=np.float32).reshape(1, 1, 2, 1)
+    q = np.asarray([qv], dtype=np.float32).reshape(1, 1, 1)
+    out = oracle.decode(q, kc, vc, np.zeros((1, 1), np.int32), np.asarray([2], np.int32), 1.0)
+    assert abs(out[0, 0, 0] - expect) <= tol
+    vals = [float(x) for x in g["case3"][0]]
+    qv, k0, k1, k2, a, b, c, expect, tol = vals
+    kc = np.asarray([k0, k1, k2, 0], dtype=np.float32).reshape(1, 1, 4, 1)
+    vc = np.asarray([a, b, c, 0], dtype=np.float32).reshape(1, 1, 4, 1)
+    q = np.asarray([qv], dtype=np.float32).reshape(1, 1, 1)
+    out = oracle.decode(q, kc, vc, np.zeros((1, 1), np.int32), np.asarray([3], np.int32), 1.0)
+    assert abs(out[0, 0, 0] - expect) <= tol
+
+
+# ---------------------------------------------------------------------------
+# library routine: contiguous attention
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("B", [1, 2, 16])
+@pytest.mark.parametrize("H,Hkv", [(4, 4), (4, 2), (8, 2)])
+def test_decode_equals_contiguous_sdpa(dtype, B, H, Hkv):
+    c = _random_case(seed=100 + B + 10 * H + Hkv, S=4, H=H, Hkv=Hkv, d=16, B=B,
+                     max_ctx=40, dtype=dtype)
+    scale = float(np.float32(1 / 4))
+    out = oracle.decode(c["q_store"], c["kc"], c["vc"], c["tables"], c["ctx"], scale)
+    ref = _sdpa_reference(c["q_val"], c["K"], c["V"], c["ctx"], scale, Hkv)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_large_logits_stable():
+    """Scores of order 1e3: exp without the max shift overflows; SDPA does not."""
+    c = _random_case(seed=5, S=2, H=2, Hkv=2, d=16, B=4, max_ctx=30, dtype="f32", qmul=300.0)
+    out = oracle.decode(c["q_store"], c["kc"], c["vc"], c["tables"], c["ctx"], 1.0)
+    ref = _sdpa_reference(c["q_val"], c["K"], c["V"], c["ctx"], 1.0, 2)
+    assert np.all(np.isfinite(out))
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-9)
+
+
+# ---------------------------------------------------------------------------
+# invariants and closed forms
+# ---------------------------------------------------------------------------
+def test_placement_invariance_bitwise():
+    """Two different physical placements of the same logical K/V: identical bits."""
+    outs = []
+    for perm_seed in (11, 12):
+        rng = np.random.default_rng(3)
+        ctx = rng.integers(1, 60, size=3)
+        g = torch.Generator().manual_seed(3)
+        K = torch.randn((3, 60, 2, 16), generator=g).float().double().numpy()
+        V = torch.randn((3, 60, 2, 16), generator=g).float().double().numpy()
+        q = torch.randn((3, 4, 16), generator=g).float().numpy()
+        kc, vc, tables = _paged_from_stream(K, V, ctx, 8, 40, np.random.default_rng(perm_seed), "f32")
+        outs.append((oracle.decode(q, kc, vc, tables, ctx.astype(np.int32), 0.3), tables))
+    assert not np.array_equal(outs[0][1], outs[1][1]), "placements should differ"
+    assert np.array_equal(outs[0][0], outs[1][0])
+
+
+def test_prefix_sharing_bitwise():
+    """Sequences sharing prefix blocks through reference counts decode exactly like
+    sequences holding private copies of the same tokens."""
+    B, Hkv, d, H = 4, 2, 8, 4
+    g = torch.Generator().manual_seed(9)
+    prefix = torch.randn((10, Hkv, d), generator=g).float().numpy()
+    suffix = [torch.randn((n, Hkv, d), generator=g).float().numpy() for n in (3, 6)]
+    q = torch.randn((2, H, d), generator=g).float().numpy()
+    vscale = np.float32(-0.5)
+
+    # shared: one prefix, two forks, copy-on-write of the partly filled tail
+    bm = bmod.BlockManager(32, B, order=np.random.default_rng(1).permutation(32))
+    kc = np.full((32, Hkv, B, d), np.nan, np.float32)
+    vc = np.full_like(kc, np.nan)
+    parent = bm.new_sequence(0)
+    pslots = np.asarray([bm.append_slot(parent) for _ in range(10)], np.int64)
+    oracle.kv_append(prefix, prefix * vscale, pslots, kc, vc)
+    kids = [bm.fork(parent) for _ in range(2)]
+    bm.free(parent)
+    slots, ks = [], []
+    for kid, suf in zip(kids, suffix):
+        for t in range(suf.shape[0]):
+            slots.append(bm.append_slot(kid))
+            ks.append(suf[t])
+    pairs = bm.take_copies()
+    assert pairs.shape[0] == 1          # first fork copies the shared tail, second writes in place
+    oracle.block_copy(pairs, kc, vc)
+    kt = np.stack(ks)
+    oracle.kv_append(kt, kt * vscale, np.asarray(slots, np.int64), kc, vc)
+    tables = bm.tables_array(kids, 4, 0)
+    ctx = np.asarray([13, 16], np.int32)
+    shared_out = oracle.decode(q, kc, vc, tables, ctx, 0.35)
+    assert len(set(tables[0, :2]) & set(tables[1, :2])) == 2   # prefix blocks really shared
+
+    # private: each sequence written separately into its own blocks
+    bm2 = bmod.BlockManager(32, B, order=np.random.default_rng(2).permutation(32))
+    kc2 = np.full((32, Hkv, B, d), np.nan, np.float32)
+    vc2 = np.full_like(kc2, np.nan)
+    seqs = []
+    for suf in suffix:
+        s = bm2.new_sequence(0)
+        toks = np.concatenate([prefix, suf])
+        sl = np.asarray([bm2.append_slot(s) for _ in range(toks.shape[0])], np.int64)
+        oracle.kv_append(np.ascontiguousarray(toks), np.ascontiguousarray(toks * vscale), sl, kc2, vc2)
+        seqs.append(s)
+    private_out = oracle.decode(q, kc2, vc2, bm2.tables_array(seqs, 4, 0), ctx, 0.35)
+    assert np.array_equal(shared_out, private_out)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_ctx1_returns_v_exactly(dtype):
+    c = _random_case(seed=21, S=4, H=4, Hkv=2, d=16, B=2, max_ctx=1, dtype=dtype)
+    out = oracle.decode(c["q_store"], c["kc"], c["vc"], c["tables"], c["ctx"], 0.5)
+    for s in range(4):
+        for h in range(4):
+            assert np.array_equal(out[s, h], c["V"][s, 0, h // 2])
+
+
+def test_bf16_widening_known_bits():
+    """ctx = 1 returns V exactly, so known bf16 bit patterns must come back as their values."""
+    bits = np.asarray([0x3F80, 0xC000, 0x4049, 0x0001, 0x7F7F, 0xBF00, 0x0000, 0x3E80], np.uint16)
+    expect = np.asarray([1.0, -2.0, 3.140625, 2.0 ** -133, 3.3895313892515355e38, -0.5, 0.0, 0.25])
+    kc = np.zeros((1, 1, 16, 8), np.uint16)
+    vc = np.zeros_like(kc)
+    vc[0, 0, 0, :] = bits
+    q = np.zeros((1, 1, 8), np.uint16)
+    out = oracle.decode(q, kc, vc, np.zeros((1, 1), np.int32), np.asarray([1], np.int32), 1.0)
+    np.testing.assert_array_equal(out[0, 0], expect)
+
+
+def test_zero_query_gives_mean_of_v():
+    c = _random_case(seed=31, S=3, H=2, Hkv=2, d=16, B=4, max_ctx=37, dtype="f32")
+    q0 = np.zeros_like(c["q_store"])
+    out = oracle.decode(q0, c["kc"], c["vc"], c["tables"], c["ctx"], 0.7)
+    for s in range(3):
+        n = int(c["ctx"][s])
+        mean = c["V"][s, :n].mean(axis=0)            # [Hkv][d]
+        np.testing.assert_allclose(out[s], mean, rtol=0, atol=1e-14)
+
+
+def test_linear_in_v():
+    """V1, V2 small integers (exact in float32): out(V1 + V2) = out(V1) + out(V2)."""
+    rng = np.random.default_rng(41)
+    ctx = np.asarray([5, 17, 33], np.int32)
+    nb, B, Hkv, d = 40, 4, 2, 8
+    kc = rng.standard_normal((nb, Hkv, B, d)).astype(np.float32)
+    v1 = rng.integers(-8, 9, size=(nb, Hkv, B, d)).astype(np.float32)
+    v2 = rng.integers(-8, 9, size=(nb, Hkv, B, d)).astype(np.float32)
+    tables = rng.permutation(nb)[:27].reshape(3, 9).astype(np.int32)
+    q = rng.standard_normal((3, 2, d)).astype(np.float32)
+    o1 = oracle.decode(q, kc, v1, tables, ctx, 0.4)
+    o2 = oracle.decode(q, kc, v2, tables, ctx, 0.4)
+    o12 = oracle.decode(q, kc, v1 + v2, tables, ctx, 0.4)
+    np.testing.assert_allclose(o12, o1 + o2, rtol=0, atol=1e-12)
+    o3 = oracle.decode(q, kc, 2 * v1, tables, ctx, 0.4)
+    assert np.array_equal(o3, 2 * o1)
+
+
+def test_ctx0_gives_zeros():
+    kc = np.full((2, 1, 16, 8), np.nan, np.float32)
+    out = oracle.decode(np.ones((2, 1, 8), np.float32), kc, kc.copy(),
+                        np.zeros((2, 1), np.int32), np.asarray([0, 0], np.int32), 1.0)
+    assert np.array_equal(out, np.zeros_like(out))
+
+
+def test_scale_is_applied():
+    """scale 0 makes every weight equal: out = mean(V), unlike scale 1."""
+    c = _random_case(seed=51, S=2, H=2, Hkv=2, d=16, B=4, max_ctx=20, dtype="f32")
+    out0 = oracle.decode(c["q_store"], c["kc"], c["vc"], c["tables"], c["ctx"], 0.0)
+    for s in range(2):
+        n = int(c["ctx"][s])
+        np.testing.assert_allclose(out0[s], c["V"][s, :n].mean(axis=0), rtol=0, atol=1e-14)
+
+
+def test_threads_do_not_change_bits():
+    c = _random_case(seed=61, S=4, H=8, Hkv=2, d=16, B=16, max_ctx=40, dtype="bf16")
+    o1 = oracle.decode(c["q_store"], c["kc"], c["vc"], c["tables"], c["ctx"], 0.25, num_threads=1)
+    o8 = oracle.decode(c["q_store"], c["kc"], c["vc"], c["tables"], c["ctx"], 0.25, num_threads=8)
+    assert np.array_equal(o1, o8)
+
+
+def test_rejects_block_outside_pool():
+    kc = np.zeros((4, 1, 2, 4), np.float32)
+    with pytest.raises(oracle.OracleError):
+        oracle.decode(np.zeros((1, 1, 4), np.float32), kc, kc.copy(),
+                      np.asarray([[0, 9]], np.int32), np.asarray([3], np.int32), 1.0)
+    with pytest.raises(oracle.OracleError):
+        oracle.kv_append(np.zeros((1, 1, 4), np.float32), np.zeros((1, 1, 4), np.float32),
+                         np.asarray([8], np.int64), kc, kc.copy())
+
+
+# ---------------------------------------------------------------------------
+# the seeded workloads feed the oracle consistently
+# ---------------------------------------------------------------------------
+def test_tiny_workload_step_matches_sdpa():
+    """The tiny configuration end to end on the oracle (append, then decode) equals
+    SDPA on the logical token streams rebuilt from the pool."""
+    wl = W.tiny()
+    vals = W.make_values(wl, "cpu", poison=True)
+    kc = W.to_numpy(vals["k_cache"]).copy()
+    vc = W.to_numpy(vals["v_cache"]).copy()
+    oracle.kv_append(W.to_numpy(vals["k_new"]), W.to_numpy(vals["v_new"]), wl.slot_mapping, kc, vc)
+    out = oracle.decode(W.to_numpy(vals["q"]), kc, vc, wl.block_tables, wl.context_lens, wl.scale)
+    assert np.all(np.isfinite(out))
+    # rebuild logical streams by walking tables in the test (independent of the oracle)
+    S, B = wl.num_seqs, wl.block_size
+    Tmax = wl.max_context_len
+    K = np.zeros((S, Tmax, wl.num_kv_heads, wl.head_dim))
+    V = np.zeros_like(K)
+    for s in range(S):
+        for t in range(int(wl.context_lens[s])):
+            b = wl.block_tables[s, t // B]
+            K[s, t] = kc[b, :, t % B, :]
+            V[s, t] = vc[b, :, t % B, :]
+    ref = _sdpa_reference(W.to_numpy(vals["q"]).astype(np.float64), K, V, wl.context_lens,
+                          wl.scale, wl.num_kv_heads)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
