@@ -1,0 +1,295 @@
+// pa_api.cpp — the C ABI declared in include/pa.h: argument validation,
+// partition policy, workspace carving and dispatch to the kernels.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace {
+
+thread_local std::string t_last_error;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return code;
+}
+
+int fail_cuda(cudaError_t e, const char* what) {
+    return fail(PA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int ilog2_exact(int x) {
+    int l = 0;
+    while ((1 << l) < x) ++l;
+    return (1 << l) == x ? l : -1;
+}
+
+int elem_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
+
+// Shape checks shared by every call.
+int check_cache(const pa_cache_desc* c) {
+    if (!c) return fail(PA_ERR_INVALID_ARG, "cache descriptor is NULL");
+    if (c->dtype != PA_F32 && c->dtype != PA_BF16)
+        return fail(PA_ERR_DTYPE, "dtype %d is neither PA_F32 (0) nor PA_BF16 (1)", c->dtype);
+    if (c->num_blocks <= 0 || c->num_kv_heads <= 0)
+        return fail(PA_ERR_INVALID_ARG, "num_blocks (%d) and num_kv_heads (%d) must be positive",
+                    c->num_blocks, c->num_kv_heads);
+    if (c->head_dim != 64 && c->head_dim != 128)
+        return fail(PA_ERR_UNSUPPORTED, "head_dim %d not compiled (64 or 128)", c->head_dim);
+    const int lg = ilog2_exact(c->block_size);
+    if (c->block_size < 16 || c->block_size > 256 || lg < 0)
+        return fail(PA_ERR_UNSUPPORTED, "block_size %d must be a power of two in [16, 256]",
+                    c->block_size);
+    return PA_OK;
+}
+
+pa::CopyParams copy_params(const pa_cache_desc* c) {
+    pa::CopyParams cp;
+    cp.num_blocks = c->num_blocks;
+    cp.num_kv_heads = c->num_kv_heads;
+    cp.block_size = c->block_size;
+    cp.log2_block_size = ilog2_exact(c->block_size);
+    cp.row_vecs = c->head_dim * elem_bytes(c->dtype) / 16;
+    return cp;
+}
+
+int sm_count() {
+    static int cache[128];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+constexpr int kMaxPartitions = 4096;
+constexpr int kAutoPartition = 512;
+
+struct Plan {
+    bool use_mma;
+    int partition_size;
+    int num_partitions;
+    size_t ws_bytes;
+    size_t ws_ml_offset;
+};
+
+int round_up16(int x) { return (x + 15) / 16 * 16; }
+
+// Partition policy: split the context only when the (sequence, head) work
+// units alone cannot fill the GPU, then into 512-token partitions.
+int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_cache_desc* c,
+                int32_t partition_size, Plan* plan) {
+    int rc = check_cache(c);
+    if (rc != PA_OK) return rc;
+    if (num_seqs < 0 || num_seqs > 65535)
+        return fail(PA_ERR_INVALID_ARG, "num_seqs %d outside [0, 65535]", num_seqs);
+    if (num_heads <= 0 || num_heads > 65535 || num_heads % c->num_kv_heads != 0)
+        return fail(PA_ERR_INVALID_ARG, "num_heads %d must be positive and a multiple of "
+                    "num_kv_heads %d", num_heads, c->num_kv_heads);
+    if (max_ctx < 0) return fail(PA_ERR_INVALID_ARG, "max_context_len %d is negative", max_ctx);
+    const int group = num_heads / c->num_kv_heads;
+    plan->use_mma = pa::mma_supported(c->dtype, c->head_dim, group);
+    if (!plan->use_mma && !pa::simt_supported(c->dtype, c->head_dim))
+        return fail(PA_ERR_UNSUPPORTED, "no kernel for dtype %d head_dim %d", c->dtype, c->head_dim);
+    const int whole = round_up16(max_ctx > 16 ? max_ctx : 16);
+    int ps = whole, np = 1;
+    if (partition_size > 0) {
+        if (partition_size % 16 != 0)
+            return fail(PA_ERR_INVALID_ARG, "partition_size %d is not a multiple of 16",
+                        partition_size);
+        ps = partition_size;
+        np = (max_ctx + ps - 1) / ps;
+        if (np < 1) np = 1;
+        if (np > kMaxPartitions)
+            return fail(PA_ERR_INVALID_ARG, "partition_size %d gives %d partitions (max %d)",
+                        partition_size, np, kMaxPartitions);
+    } else if (partition_size == 0) {
+        const long units = (long)num_seqs * (plan->use_mma ? c->num_kv_heads : num_heads);
+        if (units < 4L * sm_count() && max_ctx > kAutoPartition) {
+            ps = kAutoPartition;
+            np = (max_ctx + ps - 1) / ps;
+            while (np > kMaxPartitions) {
+                ps *= 2;
+                np = (max_ctx + ps - 1) / ps;
+            }
+        }
+    } else if (partition_size != -1) {
+        return fail(PA_ERR_INVALID_ARG, "partition_size %d: use 0 (policy), -1 (no split) or a "
+                    "positive multiple of 16", partition_size);
+    }
+    plan->partition_size = np == 1 ? whole : ps;
+    plan->num_partitions = np;
+    if (np == 1) {
+        plan->ws_bytes = 0;
+        plan->ws_ml_offset = 0;
+    } else {
+        const size_t rows = (size_t)num_seqs * num_heads * np;
+        const size_t o_bytes = rows * c->head_dim * sizeof(float);
+        plan->ws_ml_offset = (o_bytes + 255) / 256 * 256;
+        plan->ws_bytes = plan->ws_ml_offset + rows * 2 * sizeof(float);
+    }
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                 void* k_cache, void* v_cache, const pa_cache_desc* cache, void* stream) {
+    int rc = check_cache(cache);
+    if (rc != PA_OK) return rc;
+    if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens %d is negative", num_tokens);
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache)
+        return fail(PA_ERR_INVALID_ARG, "pa_kv_append: NULL pointer argument");
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_ALIGN, "pa_kv_append: k, v and the caches must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(slot_mapping) & 7u) != 0)
+        return fail(PA_ERR_ALIGN, "pa_kv_append: slot_mapping must be 8-byte aligned");
+    cudaError_t e = pa::launch_kv_append(k, v, slot_mapping, num_tokens, k_cache, v_cache,
+                                         copy_params(cache), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : fail_cuda(e, "pa_kv_append launch");
+}
+
+int pa_block_copy(const int64_t* src_dst_pairs, int32_t num_pairs, void* k_cache, void* v_cache,
+                  const pa_cache_desc* cache, void* stream) {
+    int rc = check_cache(cache);
+    if (rc != PA_OK) return rc;
+    if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "num_pairs %d is negative", num_pairs);
+    if (num_pairs == 0) return PA_OK;
+    if (!src_dst_pairs || !k_cache || !v_cache)
+        return fail(PA_ERR_INVALID_ARG, "pa_block_copy: NULL pointer argument");
+    if (!aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_ALIGN, "pa_block_copy: caches must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(src_dst_pairs) & 7u) != 0)
+        return fail(PA_ERR_ALIGN, "pa_block_copy: src_dst_pairs must be 8-byte aligned");
+    cudaError_t e = pa::launch_block_copy(src_dst_pairs, num_pairs, k_cache, v_cache,
+                                          copy_params(cache), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : fail_cuda(e, "pa_block_copy launch");
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t max_context_len,
+                                const pa_cache_desc* cache, int32_t partition_size) {
+    Plan plan;
+    if (plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan) != PA_OK)
+        return 0;
+    return plan.ws_bytes;
+}
+
+int pa_decode_num_partitions(int32_t num_seqs, int32_t num_heads, int32_t max_context_len,
+                             const pa_cache_desc* cache, int32_t partition_size) {
+    Plan plan;
+    int rc = plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan);
+    return rc != PA_OK ? rc : plan.num_partitions;
+}
+
+int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+              const int32_t* block_tables, int32_t block_table_stride,
+              const int32_t* context_lens, int32_t max_context_len, int32_t num_seqs,
+              int32_t num_heads, float scale, const pa_cache_desc* cache,
+              int32_t partition_size, void* workspace, size_t workspace_bytes, void* stream) {
+    Plan plan;
+    int rc = plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan);
+    if (rc != PA_OK) return rc;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode: NULL pointer argument");
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_ALIGN, "pa_decode: out, q and the caches must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(block_tables) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(context_lens) & 3u) != 0)
+        return fail(PA_ERR_ALIGN, "pa_decode: block_tables / context_lens must be 4-byte aligned");
+    if (block_table_stride < 0 ||
+        (int64_t)block_table_stride * cache->block_size < (int64_t)max_context_len)
+        return fail(PA_ERR_INVALID_ARG, "max_context_len %d exceeds block_table_stride %d * "
+                    "block_size %d", max_context_len, block_table_stride, cache->block_size);
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    if (plan.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < plan.ws_bytes)
+            return fail(PA_ERR_WORKSPACE, "pa_decode needs %zu workspace bytes, got %zu at %p",
+                        plan.ws_bytes, workspace_bytes, workspace);
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+            return fail(PA_ERR_ALIGN, "pa_decode: workspace must be 256-byte aligned");
+    }
+    pa::DecodeParams p;
+    p.out = out;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.ws_o = plan.ws_bytes ? static_cast<float*>(workspace) : nullptr;
+    p.ws_ml = plan.ws_bytes
+                  ? reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.ws_ml_offset)
+                  : nullptr;
+    p.table_stride = block_table_stride;
+    p.max_context_len = max_context_len;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = cache->num_kv_heads;
+    p.num_blocks = cache->num_blocks;
+    p.block_size = cache->block_size;
+    p.log2_block_size = ilog2_exact(cache->block_size);
+    p.partition_size = plan.partition_size;
+    p.num_partitions = plan.num_partitions;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = plan.use_mma ? pa::launch_decode_mma(p, cache->head_dim, st)
+                                 : pa::launch_decode_simt(p, cache->dtype, cache->head_dim, st);
+    if (e != cudaSuccess) return fail_cuda(e, "pa_decode launch");
+    if (plan.num_partitions > 1) {
+        e = pa::launch_partition_reduce(p, cache->dtype, cache->head_dim, st);
+        if (e != cudaSuccess) return fail_cuda(e, "pa_decode reduce launch");
+    }
+    return PA_OK;
+}
+
+int pa_sync_check(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail_cuda(e, "pa_sync_check: stream");
+    unsigned a = 0, b = 0, c = 0;
+    if ((e = pa::read_status_copy(&a, true)) != cudaSuccess ||
+        (e = pa::read_status_simt(&b, true)) != cudaSuccess ||
+        (e = pa::read_status_mma(&c, true)) != cudaSuccess)
+        return fail_cuda(e, "pa_sync_check: status word");
+    if ((a | b | c) & pa::kStatusBadIndex)
+        return fail(PA_ERR_BAD_INDEX, "a kernel met a block id, slot or context length outside "
+                    "its bounds (bits copy=%u simt=%u mma=%u)", a, b, c);
+    return PA_OK;
+}
+
+const char* pa_get_last_error(void) { return t_last_error.c_str(); }
+
+const char* pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+        case PA_ERR_DTYPE: return "PA_ERR_DTYPE";
+        case PA_ERR_ALIGN: return "PA_ERR_ALIGN";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA";
+        case PA_ERR_BAD_INDEX: return "PA_ERR_BAD_INDEX";
+        case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+        default: return "PA_ERR_UNKNOWN";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+// pa_internal.h — host-side interface between the C ABI (pa_api.cpp) and the
+// kernel translation units. Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pa {
+
+// Bit of the per-translation-unit status word a kernel sets when it meets an
+// out-of-range block id, slot or context length (and skips the access).
+constexpr unsigned kStatusBadIndex = 1u;
+
+// Everything one decode launch needs. Offsets are in elements unless noted.
+struct DecodeParams {
+    void* out;                  // [S][H][D], cache dtype
+    const void* q;              // [S][H][D]
+    const void* k_cache;        // [NB][Hkv][BS][D]
+    const void* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    float* ws_o;                // [S][H][P][D] normalised partial outputs (P > 1)
+    float* ws_ml;               // [S][H][P][2]  (running max in log2 units, running sum)
+    int64_t table_stride;
+    int32_t max_context_len;
+    int32_t num_seqs;
+    int32_t num_heads;
+    int32_t num_kv_heads;
+    int32_t num_blocks;
+    int32_t block_size;
+    int32_t log2_block_size;
+    int32_t partition_size;     // tokens per partition (whole context when P == 1)
+    int32_t num_partitions;     // P
+    float scale_log2;           // softmax scale * log2(e)
+};
+
+struct CopyParams {
+    int32_t num_blocks;
+    int32_t num_kv_heads;
+    int32_t block_size;
+    int32_t log2_block_size;
+    int32_t row_vecs;           // 16-byte chunks per K/V vector = head_dim * elem / 16
+};
+
+// Launchers: return cudaSuccess or the launch error. dtype: 0 = f32, 1 = bf16.
+cudaError_t launch_kv_append(const void* k, const void* v, const int64_t* slot_mapping,
+                             int32_t num_tokens, void* k_cache, void* v_cache,
+                             const CopyParams& cp, cudaStream_t stream);
+cudaError_t launch_block_copy(const int64_t* pairs, int32_t num_pairs, void* k_cache,
+                              void* v_cache, const CopyParams& cp, cudaStream_t stream);
+
+// CUDA-core decode: one CTA per (partition, query head, sequence).
+bool simt_supported(int dtype, int head_dim);
+cudaError_t launch_decode_simt(const DecodeParams& p, int dtype, int head_dim,
+                               cudaStream_t stream);
+// Tensor-core decode for grouped-query attention (bf16, 2 <= group <= 8): one
+// CTA per (partition, kv head, sequence) covering the whole query group.
+bool mma_supported(int dtype, int head_dim, int group);
+cudaError_t launch_decode_mma(const DecodeParams& p, int head_dim, cudaStream_t stream);
+// Log-sum-exp merge of the P partial results into out.
+cudaError_t launch_partition_reduce(const DecodeParams& p, int dtype, int head_dim,
+                                    cudaStream_t stream);
+
+// Status words of the kernel translation units: OR of kStatus* bits since the
+// last clear. Return cudaSuccess or the copy error.
+cudaError_t read_status_copy(unsigned* bits, bool clear);
+cudaError_t read_status_simt(unsigned* bits, bool clear);
+cudaError_t read_status_mma(unsigned* bits, bool clear);
+
+}  // namespace pa

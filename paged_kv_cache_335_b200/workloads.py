@@ -248,6 +248,20 @@ def cow_beam4(seed: int = 4, num_prompts: int = 32, beam_width: int = 4,
                "beam_width": beam_width, "refcount": bm.refcount.copy()})
 
 
+def decode_case(num_seqs, num_heads, num_kv_heads, head_dim, block_size, dtype, context_lens,
+                seed=0, pool_factor=1.3, partition_size=0, name=None) -> Workload:
+    """A decode workload with the given final context lengths, built like the
+    named configurations (shuffled pool, one appended token per sequence)."""
+    rng = np.random.default_rng(seed)
+    ctx = np.asarray(context_lens, dtype=np.int64)
+    assert ctx.shape == (num_seqs,)
+    demand = int(sum(-(-int(n) // block_size) for n in ctx))
+    nb = int(math.ceil(pool_factor * max(demand, 1))) + 2
+    name = name or f"case_{num_seqs}x{num_heads}/{num_kv_heads}_d{head_dim}_bs{block_size}_{dtype}"
+    return _decode_structure(name, dtype, ctx, num_heads, num_kv_heads, head_dim, block_size, nb,
+                             1.0 / math.sqrt(head_dim), seed, rng, partition_size=partition_size)
+
+
 CONFIGS = {
     "tiny": tiny,
     "llama7b": llama7b,
@@ -256,6 +270,49 @@ CONFIGS = {
     "llama70b_gqa": llama70b_gqa,
     "cow_beam4": cow_beam4,
 }
+
+
+def restrict(wl: Workload, seq_ids) -> Workload:
+    """The same step for a subset of sequences on a compact pool: their blocks
+    (and the sources of their copy pairs) renumbered 0..n-1 in first-use order,
+    plus one fresh poison block. Used to size bounded CPU samples."""
+    seq_ids = sorted({int(s) for s in seq_ids})
+    B = wl.block_size
+    remap = {}
+
+    def new_id(b):
+        b = int(b)
+        if b not in remap:
+            remap[b] = len(remap)
+        return remap[b]
+
+    nbs = [-(-int(wl.context_lens[s]) // B) for s in seq_ids]
+    for s, nb in zip(seq_ids, nbs):
+        for j in range(nb):
+            new_id(wl.block_tables[s, j])
+    dsts = set(remap)
+    pairs = [(new_id(a), remap[int(b)]) for a, b in wl.copy_pairs.tolist() if int(b) in dsts]
+    poison = len(remap)
+    width = max([1] + nbs)
+    tables = np.full((len(seq_ids), width), poison, dtype=np.int32)
+    for i, (s, nb) in enumerate(zip(seq_ids, nbs)):
+        tables[i, :nb] = [remap[int(b)] for b in wl.block_tables[s, :nb]]
+    pos = {s: i for i, s in enumerate(seq_ids)}
+    keep = [t for t, s in enumerate(wl.token_seq.tolist()) if s in pos]
+    slots = [remap[int(wl.slot_mapping[t]) // B] * B + int(wl.slot_mapping[t]) % B for t in keep]
+    sub = Workload(**{**wl.__dict__})
+    sub.name = f"{wl.name}[{len(seq_ids)} of {wl.num_seqs} seqs]"
+    sub.num_seqs = len(seq_ids)
+    sub.num_blocks = poison + 1
+    sub.context_lens = wl.context_lens[seq_ids].copy()
+    sub.history_lens = wl.history_lens[seq_ids].copy()
+    sub.block_tables = tables
+    sub.slot_mapping = np.asarray(slots, dtype=np.int64)
+    sub.token_seq = np.asarray([pos[int(wl.token_seq[t])] for t in keep], dtype=np.int32)
+    sub.copy_pairs = np.asarray(pairs, dtype=np.int64).reshape(-1, 2)
+    sub.poison_block = poison
+    sub.extra = dict(wl.extra)
+    return sub
 
 
 def make(name: str, **kw) -> Workload:

@@ -1,0 +1,106 @@
+"""The C-ABI library loads and exports what include/pa.h declares, and its
+host-side argument checks answer without touching a GPU."""
+import ctypes
+
+import pytest
+
+import paged_kv_cache_335_b200 as pa
+from paged_kv_cache_335_b200 import build as pbuild
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pbuild.build()
+    return pa.load_library()
+
+
+def test_header_declares_the_hot_path():
+    names = pa.header_functions()
+    for f in ("pa_kv_append", "pa_decode", "pa_block_copy", "pa_decode_workspace_size",
+              "pa_sync_check", "pa_get_last_error"):
+        assert f in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in pa.header_functions() if not hasattr(lib, n)]
+    assert not missing, f"libpa.so lacks {missing}"
+
+
+def _desc(**kw):
+    d = dict(num_blocks=64, num_kv_heads=4, block_size=16, head_dim=128, dtype=pa.PA_BF16)
+    d.update(kw)
+    return pa.pa_cache_desc(**d)
+
+
+def _decode_rc(lib, desc, num_seqs=4, num_heads=4, max_ctx=100, stride=8, ptr=16, ps=0,
+               scale=0.125):
+    p = ctypes.c_void_p(ptr)
+    return lib.pa_decode(p, p, p, p, p, stride, p, max_ctx, num_seqs, num_heads, scale,
+                         ctypes.byref(desc), ps, None, 0, None)
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("head_dim", 96, pa.PA_ERR_UNSUPPORTED),
+    ("block_size", 24, pa.PA_ERR_UNSUPPORTED),
+    ("block_size", 8, pa.PA_ERR_UNSUPPORTED),
+    ("dtype", 7, pa.PA_ERR_DTYPE),
+    ("num_blocks", 0, pa.PA_ERR_INVALID_ARG),
+])
+def test_decode_rejects_bad_cache(lib, field, value, code):
+    assert _decode_rc(lib, _desc(**{field: value})) == code
+    assert lib.pa_get_last_error()
+
+
+def test_decode_rejects_bad_arguments(lib):
+    assert _decode_rc(lib, _desc(), num_heads=6) == pa.PA_ERR_INVALID_ARG   # 6 % 4 != 0
+    assert _decode_rc(lib, _desc(), ptr=8) == pa.PA_ERR_ALIGN
+    assert _decode_rc(lib, _desc(), max_ctx=200, stride=8) == pa.PA_ERR_INVALID_ARG
+    assert _decode_rc(lib, _desc(), ps=24) == pa.PA_ERR_INVALID_ARG
+    assert _decode_rc(lib, _desc(), scale=float("inf")) == pa.PA_ERR_INVALID_ARG
+    assert _decode_rc(lib, _desc(), num_seqs=0) == pa.PA_OK                 # nothing to do
+
+
+def test_decode_needs_workspace_when_split(lib):
+    desc = _desc(num_kv_heads=1)
+    n = lib.pa_decode_num_partitions(1, 8, 4096, ctypes.byref(desc), 512)
+    assert n == 8
+    need = lib.pa_decode_workspace_size(1, 8, 4096, ctypes.byref(desc), 512)
+    assert need >= 8 * 8 * (128 + 2) * 4
+    rc = _decode_rc(lib, desc, num_seqs=1, num_heads=8, max_ctx=4096, stride=256, ps=512)
+    assert rc == pa.PA_ERR_WORKSPACE
+    assert lib.pa_decode_workspace_size(1, 8, 4096, ctypes.byref(desc), -1) == 0
+
+
+def test_partition_policy(lib):
+    # few (sequence, kv head) units and a long context: split into 512-token partitions
+    d70 = _desc(num_kv_heads=8)
+    assert lib.pa_decode_num_partitions(8, 64, 32768, ctypes.byref(d70), 0) == 64
+    # many units: no split
+    d13 = _desc(num_kv_heads=40)
+    assert lib.pa_decode_num_partitions(256, 40, 4096, ctypes.byref(d13), 0) == 1
+    assert lib.pa_decode_num_partitions(8, 64, 32768, ctypes.byref(d70), -1) == 1
+
+
+def test_append_and_copy_reject_bad_arguments(lib):
+    p = ctypes.c_void_p(16)
+    assert lib.pa_kv_append(p, p, p, -1, p, p, ctypes.byref(_desc()), None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_kv_append(p, p, p, 0, p, p, ctypes.byref(_desc()), None) == pa.PA_OK
+    assert lib.pa_kv_append(p, ctypes.c_void_p(4), p, 3, p, p, ctypes.byref(_desc()), None) \
+        == pa.PA_ERR_ALIGN
+    assert lib.pa_kv_append(None, p, p, 3, p, p, ctypes.byref(_desc()), None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_block_copy(p, 0, p, p, ctypes.byref(_desc()), None) == pa.PA_OK
+    assert lib.pa_block_copy(None, 2, p, p, ctypes.byref(_desc()), None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_block_copy(ctypes.c_void_p(12), 2, p, p, ctypes.byref(_desc()), None) \
+        == pa.PA_ERR_ALIGN
+
+
+def test_status_strings(lib):
+    assert lib.pa_status_string(pa.PA_ERR_BAD_INDEX) == b"PA_ERR_BAD_INDEX"
+    assert lib.pa_status_string(0) == b"PA_OK"
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    kc = torch.zeros((4, 1, 16, 64))
+    with pytest.raises(ValueError, match="CUDA"):
+        pa.pa_block_copy(torch.zeros((1, 2), dtype=torch.int64), kc, kc.clone())
