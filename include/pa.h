@@ -27,7 +27,8 @@
  * ---------------------------------------------------------------------------
  * Memory.  Every tensor pointer is a DEVICE pointer owned by the caller. The
  *   library never allocates, frees or retains caller memory; it keeps only a
- *   per-device 4-byte status word (see pa_sync_check).
+ *   per-device 4-byte status word (see pa_sync_check) and the fixed scratch
+ *   buffer of pa_decode_noalloc.
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *   default stream). Every call only enqueues work on that stream and returns;
  *   results are ready when the stream reaches that point.
@@ -197,6 +198,39 @@ int pa_decode_num_partitions(int32_t num_seqs, int32_t num_heads,
 int pa_block_copy(const int64_t* src_dst_pairs, int32_t num_pairs,
                   void* k_cache, void* v_cache, const pa_cache_desc* cache,
                   void* stream);
+
+/*
+ * PA_NOALLOC_SCRATCH_BYTES — size of the device buffer inside the library that
+ * pa_decode_noalloc uses as its workspace (32 MiB per GPU that loads the
+ * library, held until the process exits).
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * pa_decode_noalloc — pa_decode for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart: this is an interface convenience. Some callers
+ * cannot call cudaMalloc where they decode (code inside a memory arena sized up
+ * front, plug-ins of an engine that owns all device allocations, loops that
+ * must never enter an allocator). This entry point computes exactly what
+ * pa_decode computes, with the same arguments minus the workspace: when the
+ * context is split, the partial results go to a buffer of
+ * PA_NOALLOC_SCRATCH_BYTES inside the library. It allocates nothing.
+ *
+ * The first call on a device looks up that buffer's device address
+ * (cudaGetSymbolAddress) with the device current; make that first call before
+ * any stream capture. A call whose workspace need (pa_decode_workspace_size
+ * with the same arguments) exceeds PA_NOALLOC_SCRATCH_BYTES returns
+ * PA_ERR_WORKSPACE and enqueues nothing. All calls on one device share the
+ * buffer, which keeps the last call's contents: calls whose kernels may overlap
+ * on the GPU (different streams without ordering) race on it and must not be
+ * issued. The buffer needs no clearing between calls.
+ */
+int pa_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, int32_t block_table_stride,
+                      const int32_t* context_lens, int32_t max_context_len,
+                      int32_t num_seqs, int32_t num_heads, float scale,
+                      const pa_cache_desc* cache, int32_t partition_size, void* stream);
 
 /*
  * pa_sync_check — wait for `stream`, then read and clear the current device's

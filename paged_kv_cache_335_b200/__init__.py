@@ -35,6 +35,7 @@ PA_ERR_BAD_INDEX = -6
 PA_ERR_WORKSPACE = -7
 PA_F32 = 0
 PA_BF16 = 1
+PA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _lock = threading.Lock()
 _lib = None
@@ -77,6 +78,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_kv_append.argtypes = [vp, vp, vp, i32, vp, vp, desc, vp]
         lib.pa_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, desc, i32,
                                   vp, sz, vp]
+        lib.pa_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, desc,
+                                          i32, vp]
+        lib.pa_decode_noalloc.restype = ctypes.c_int
         lib.pa_decode_workspace_size.argtypes = [i32, i32, i32, desc, i32]
         lib.pa_decode_workspace_size.restype = sz
         lib.pa_decode_num_partitions.argtypes = [i32, i32, i32, desc, i32]
@@ -245,11 +249,35 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float
         _stream(stream)))
 
 
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                      max_context_len: int | None = None, partition_size: int = 0,
+                      stream=None) -> None:
+    """pa_decode without a workspace argument, for callers that cannot allocate
+    device memory: a split context uses the library's fixed scratch buffer of
+    PA_NOALLOC_SCRATCH_BYTES per device. Calls that overlap on the GPU race on
+    that buffer; make the first call on a device before any stream capture."""
+    torch = _torch()
+    _same_pool(k_cache, v_cache)
+    desc = cache_desc(k_cache)
+    s, h, d = (int(x) for x in q.shape)
+    if tuple(out.shape) != (s, h, d) or d != desc.head_dim:
+        raise ValueError("q and out must be [num_seqs][num_heads][head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or context_lens.shape != (s,):
+        raise ValueError("block_tables must be [num_seqs][stride], context_lens [num_seqs]")
+    if max_context_len is None:
+        max_context_len = int(context_lens.max().item()) if s else 0
+    _check(load_library().pa_decode_noalloc(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), int(block_tables.shape[1]),
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len), s, h,
+        float(scale), ctypes.byref(desc), int(partition_size), _stream(stream)))
+
+
 def pa_sync_check(stream=None) -> None:
     """Wait for the stream; raise PAError if a kernel met an out-of-range index."""
     _check(load_library().pa_sync_check(_stream(stream)))
 
 
-__all__ = ["pa_kv_append", "pa_decode", "pa_block_copy", "pa_decode_workspace_size",
+__all__ = ["pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_block_copy", "pa_decode_workspace_size",
            "pa_decode_num_partitions", "pa_sync_check", "pa_cache_desc", "cache_desc",
            "load_library", "header_functions", "PAError"]

@@ -150,6 +150,16 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
 
 }  // namespace
 
+int pa::report_error(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return code;
+}
+
 extern "C" {
 
 int pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,

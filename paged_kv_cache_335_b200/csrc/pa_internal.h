@@ -62,6 +62,10 @@ cudaError_t launch_decode_mma(const DecodeParams& p, int head_dim, cudaStream_t 
 cudaError_t launch_partition_reduce(const DecodeParams& p, int dtype, int head_dim,
                                     cudaStream_t stream);
 
+// Record `fmt` as this host thread's last error (read by pa_get_last_error)
+// and return `code`.
+int report_error(int code, const char* fmt, ...);
+
 // Status words of the kernel translation units: OR of kStatus* bits since the
 // last clear. Return cudaSuccess or the copy error.
 cudaError_t read_status_copy(unsigned* bits, bool clear);

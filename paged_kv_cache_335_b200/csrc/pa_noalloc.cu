@@ -1,0 +1,82 @@
+// pa_noalloc.cu — pa_decode_noalloc: pa_decode for callers that cannot
+// allocate device memory.
+//
+// Some callers cannot call cudaMalloc (or any allocating routine) where they
+// decode: code that runs inside a memory arena sized up front, plug-ins of a
+// host engine that owns every device allocation, or loops that must never
+// enter an allocator. When a long context is split into partitions, pa_decode
+// needs a workspace for the partial results; this entry point takes that
+// workspace from a buffer inside the library instead: a file-scope device
+// array of PA_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library
+// holds until the process exits. Nothing here allocates.
+//
+// On the host, `s_scratch` names a host-side stand-in, not device memory, so
+// its device address is looked up once per device with cudaGetSymbolAddress,
+// with that device current, and cached. Every call shares the one buffer per
+// device: calls whose kernels overlap on the GPU (different streams, no
+// ordering between them) race on it. The buffer needs no clearing: each call
+// writes every partial result before its merge reads it.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+static __device__ __align__(256) unsigned char s_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices];
+std::mutex g_scratch_mutex;
+
+// Device address of s_scratch on the current device; the first call on a
+// device looks it up.
+cudaError_t scratch_address(void** addr) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, s_scratch);
+        if (e != cudaSuccess) return e;
+        if (!p) return cudaErrorInvalidSymbol;
+        g_scratch_addr[dev] = p;
+    }
+    *addr = g_scratch_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" int pa_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* block_tables,
+                                 int32_t block_table_stride, const int32_t* context_lens,
+                                 int32_t max_context_len, int32_t num_seqs, int32_t num_heads,
+                                 float scale, const pa_cache_desc* cache,
+                                 int32_t partition_size, void* stream) {
+    // 0 means "no split" or invalid arguments; pa_decode reports the latter.
+    const size_t need = pa_decode_workspace_size(num_seqs, num_heads, max_context_len, cache,
+                                                 partition_size);
+    if (need > (size_t)PA_NOALLOC_SCRATCH_BYTES)
+        return pa::report_error(
+            PA_ERR_WORKSPACE,
+            "pa_decode_noalloc: this call needs %zu bytes of scratch, more than the library's "
+            "fixed %zu (PA_NOALLOC_SCRATCH_BYTES); use pa_decode with a workspace of your own, "
+            "or a larger partition_size",
+            need, (size_t)PA_NOALLOC_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    if (need > 0) {
+        const cudaError_t e = scratch_address(&scratch);
+        if (e != cudaSuccess)
+            return pa::report_error(PA_ERR_CUDA,
+                                    "pa_decode_noalloc: cudaGetSymbolAddress of the scratch "
+                                    "buffer failed: %s", cudaGetErrorString(e));
+    }
+    return pa_decode(out, q, k_cache, v_cache, block_tables, block_table_stride, context_lens,
+                     max_context_len, num_seqs, num_heads, scale, cache, partition_size, scratch,
+                     need > 0 ? (size_t)PA_NOALLOC_SCRATCH_BYTES : 0, stream);
+}
