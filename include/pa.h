@@ -82,6 +82,7 @@ extern "C" {
 #define PA_ERR_CUDA        (-5) /* a CUDA runtime call or launch failed       */
 #define PA_ERR_BAD_INDEX   (-6) /* a kernel met an out-of-range index         */
 #define PA_ERR_WORKSPACE   (-7) /* workspace missing or smaller than needed   */
+#define PA_ERR_TIMEOUT     (-8) /* a bounded in-kernel pipeline wait gave up  */
 
 /* ---- element types ------------------------------------------------------ */
 #define PA_F32  0
@@ -235,8 +236,9 @@ int pa_decode_noalloc(void* out, const void* q, const void* k_cache, const void*
 /*
  * pa_sync_check — wait for `stream`, then read and clear the current device's
  * status word. Returns PA_OK, PA_ERR_BAD_INDEX if any kernel since the last
- * check met an out-of-range index, or PA_ERR_CUDA if the stream reported an
- * error.
+ * check met an out-of-range index, PA_ERR_TIMEOUT if a kernel's bounded wait
+ * on its shared-memory pipeline gave up (its results are then invalid; the
+ * kernel still terminated), or PA_ERR_CUDA if the stream reported an error.
  */
 int pa_sync_check(void* stream);
 

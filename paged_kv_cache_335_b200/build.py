@@ -44,35 +44,40 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def _compile(src: str) -> tuple:
-    obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-    cmd = [_nvcc()] + NVCC_FLAGS + ["-Xptxas", "-v", "-c", src, "-o", obj]
+def _compile(src: str, bdir: str = BUILD_DIR, extra=()) -> tuple:
+    obj = os.path.join(bdir, os.path.basename(src) + ".o")
+    cmd = [_nvcc()] + NVCC_FLAGS + list(extra) + ["-Xptxas", "-v", "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
     return obj, r.stderr
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every source under csrc/ and link ``libpa.so``; returns its path."""
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, out: str | None = None,
+          defines=(), build_dir: str | None = None) -> str:
+    """Compile every source under csrc/ and link ``libpa.so`` (or ``out``);
+    ``defines`` ("NAME=VALUE" strings) override the kernels' compile-time tunables."""
+    lib_path = out or LIB_PATH
+    if not force and out is None and not defines and up_to_date():
         return LIB_PATH
-    os.makedirs(BUILD_DIR, exist_ok=True)
+    bdir = build_dir or BUILD_DIR
+    os.makedirs(bdir, exist_ok=True)
     srcs = sources()
+    flags = [f"-D{d}" for d in defines]
     with cf.ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 4)) as ex:
-        results = list(ex.map(_compile, srcs))
-    with open(os.path.join(BUILD_DIR, "ptxas.txt"), "w") as f:
+        results = list(ex.map(lambda src: _compile(src, bdir, flags), srcs))
+    with open(os.path.join(bdir, "ptxas.txt"), "w") as f:
         for (obj, log), src in zip(results, srcs):
             f.write(f"== {os.path.basename(src)}\n{log}\n")
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
+    tmp = lib_path + f".tmp{os.getpid()}"
     cmd = [_nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + [o for o, _ in results]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB_PATH)
+    os.replace(tmp, lib_path)
     if verbose:
-        print(open(os.path.join(BUILD_DIR, "ptxas.txt")).read(), file=sys.stderr)
-    return LIB_PATH
+        print(open(os.path.join(bdir, "ptxas.txt")).read(), file=sys.stderr)
+    return lib_path
 
 
 if __name__ == "__main__":

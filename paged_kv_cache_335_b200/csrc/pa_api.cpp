@@ -1,11 +1,15 @@
 // pa_api.cpp — the C ABI declared in include/pa.h: argument validation,
 // partition policy, workspace carving and dispatch to the kernels.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "pa.h"
@@ -53,6 +57,9 @@ int check_cache(const pa_cache_desc* c) {
     if (c->block_size < 16 || c->block_size > 256 || lg < 0)
         return fail(PA_ERR_UNSUPPORTED, "block_size %d must be a power of two in [16, 256]",
                     c->block_size);
+    if ((int64_t)c->num_blocks * c->num_kv_heads * c->block_size > (int64_t)INT32_MAX)
+        return fail(PA_ERR_UNSUPPORTED, "pool of %d blocks x %d kv heads x %d slots exceeds 2^31 "
+                    "rows", c->num_blocks, c->num_kv_heads, c->block_size);
     return PA_OK;
 }
 
@@ -77,6 +84,52 @@ int sm_count() {
         cache[dev] = n;
     }
     return cache[dev];
+}
+
+// ---- TMA tensor maps -------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// The pool as a 2-D tensor [num_blocks * num_kv_heads * block_size rows][head_dim],
+// loaded in boxes of 16 rows x 128 bytes with the 128-byte swizzle.
+int make_cache_map(CUtensorMap* map, const void* base, const pa_cache_desc* c) {
+    auto fn = encode_fn();
+    if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const int e = elem_bytes(c->dtype);
+    cuuint64_t dims[2] = {(cuuint64_t)c->head_dim,
+                          (cuuint64_t)c->num_blocks * c->num_kv_heads * c->block_size};
+    cuuint64_t strides[1] = {(cuuint64_t)c->head_dim * e};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / e), 16u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, c->dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                    2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PA_OK;
+}
+
+// Decode kernel family: TMA-staged (default) or direct register loads
+// (PA_DECODE_IMPL=regs), kept for A/B measurement.
+bool use_tma_kernels() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = std::getenv("PA_DECODE_IMPL");
+        v = (e && std::strcmp(e, "regs") == 0) ? 0 : 1;
+    }
+    return v == 1;
 }
 
 constexpr int kMaxPartitions = 4096;
@@ -121,8 +174,11 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
             return fail(PA_ERR_INVALID_ARG, "partition_size %d gives %d partitions (max %d)",
                         partition_size, np, kMaxPartitions);
     } else if (partition_size == 0) {
+        // The persistent tensor-core kernel balances its items statically, so it
+        // wants many equal items; the CUDA-core kernel only needs to fill the GPU.
         const long units = (long)num_seqs * (plan->use_mma ? c->num_kv_heads : num_heads);
-        if (units < 4L * sm_count() && max_ctx > kAutoPartition) {
+        const long want = (plan->use_mma ? 8L : 4L) * sm_count();
+        if (units < want && max_ctx > kAutoPartition) {
             ps = kAutoPartition;
             np = (max_ctx + ps - 1) / ps;
             while (np > kMaxPartitions) {
@@ -262,8 +318,16 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
     p.num_partitions = plan.num_partitions;
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = plan.use_mma ? pa::launch_decode_mma(p, cache->head_dim, st)
-                                 : pa::launch_decode_simt(p, cache->dtype, cache->head_dim, st);
+    cudaError_t e;
+    if (use_tma_kernels()) {
+        CUtensorMap kmap, vmap;
+        if ((rc = make_cache_map(&kmap, k_cache, cache)) != PA_OK) return rc;
+        if ((rc = make_cache_map(&vmap, v_cache, cache)) != PA_OK) return rc;
+        e = pa::launch_decode_tma(p, cache->dtype, cache->head_dim, plan.use_mma, kmap, vmap, st);
+    } else {
+        e = plan.use_mma ? pa::launch_decode_mma(p, cache->head_dim, st)
+                         : pa::launch_decode_simt(p, cache->dtype, cache->head_dim, st);
+    }
     if (e != cudaSuccess) return fail_cuda(e, "pa_decode launch");
     if (plan.num_partitions > 1) {
         e = pa::launch_partition_reduce(p, cache->dtype, cache->head_dim, st);
@@ -275,14 +339,18 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
 int pa_sync_check(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda(e, "pa_sync_check: stream");
-    unsigned a = 0, b = 0, c = 0;
+    unsigned a = 0, b = 0, c = 0, d = 0;
     if ((e = pa::read_status_copy(&a, true)) != cudaSuccess ||
         (e = pa::read_status_simt(&b, true)) != cudaSuccess ||
-        (e = pa::read_status_mma(&c, true)) != cudaSuccess)
+        (e = pa::read_status_mma(&c, true)) != cudaSuccess ||
+        (e = pa::read_status_tma(&d, true)) != cudaSuccess)
         return fail_cuda(e, "pa_sync_check: status word");
-    if ((a | b | c) & pa::kStatusBadIndex)
+    if ((a | b | c | d) & pa::kStatusTimeout)
+        return fail(PA_ERR_TIMEOUT, "a bounded pipeline wait gave up (bits copy=%u simt=%u mma=%u "
+                    "tma=%u)", a, b, c, d);
+    if ((a | b | c | d) & pa::kStatusBadIndex)
         return fail(PA_ERR_BAD_INDEX, "a kernel met a block id, slot or context length outside "
-                    "its bounds (bits copy=%u simt=%u mma=%u)", a, b, c);
+                    "its bounds (bits copy=%u simt=%u mma=%u tma=%u)", a, b, c, d);
     return PA_OK;
 }
 
@@ -298,6 +366,7 @@ const char* pa_status_string(int status) {
         case PA_ERR_CUDA: return "PA_ERR_CUDA";
         case PA_ERR_BAD_INDEX: return "PA_ERR_BAD_INDEX";
         case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+        case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT";
         default: return "PA_ERR_UNKNOWN";
     }
 }

@@ -206,34 +206,44 @@ decode_simt_kernel(const DecodeParams p) {
 // Merge of partitions j = 0 .. ceil(n / partition_size) - 1 of one (s, h):
 //   M = max_j m_j,  w_j = l_j * 2^(m_j - M),  out = sum_j w_j o_j / sum_j w_j,
 // where o_j is partition j's normalised output. This is the exact softmax over
-// the union of the partitions. grid = (num_heads, num_seqs).
+// the union of the partitions. grid = (num_heads, num_seqs). Launched as a
+// programmatic dependent of the decode kernel: it may start while the decode
+// drains and waits (griddepcontrol.wait) for all of its results.
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 partition_reduce_kernel(const DecodeParams p) {
     extern __shared__ float sm_w[];  // [num_partitions] weights
     __shared__ float sm_L;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int h = blockIdx.x;
     const int s = blockIdx.y;
     const int ctx = clamp_context(__ldg(p.context_lens + s), p.max_context_len, &s_status_simt, false);
     const int n = (ctx + p.partition_size - 1) / p.partition_size;
     const int64_t out_row = (int64_t)s * p.num_heads + h;
     const float* ml = p.ws_ml + out_row * p.num_partitions * 2;
-    if (threadIdx.x == 0) {
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
         float M = -INFINITY;
-        for (int j = 0; j < n; ++j) M = fmaxf(M, ml[2 * j]);
+        for (int j = lane; j < n; j += 32) M = fmaxf(M, ml[2 * j]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
         float L = 0.f;
-        for (int j = 0; j < n; ++j) {
-            const float w = ml[2 * j] == -INFINITY ? 0.f : ml[2 * j + 1] * exp2f(ml[2 * j] - M);
+        for (int j = lane; j < n; j += 32) {
+            const float mj = ml[2 * j];
+            const float w = mj == -INFINITY ? 0.f : ml[2 * j + 1] * exp2f(mj - M);
             sm_w[j] = w;
             L += w;
         }
-        sm_L = L;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+        if (lane == 0) sm_L = L;
     }
     __syncthreads();
     const float L = sm_L;
     const float* o = p.ws_o + out_row * p.num_partitions * D;
     for (int d = threadIdx.x; d < D; d += kThreads) {
         float acc = 0.f;
+#pragma unroll 8
         for (int j = 0; j < n; ++j) acc = fmaf(sm_w[j], o[(int64_t)j * D + d], acc);
         Elem<T>::store(p.out, out_row * D + d, L > 0.f ? acc / L : 0.f);
     }
@@ -248,10 +258,17 @@ cudaError_t launch_simt_t(const DecodeParams& p, cudaStream_t stream) {
 
 template <typename T, int D>
 cudaError_t launch_reduce_t(const DecodeParams& p, cudaStream_t stream) {
-    dim3 grid((unsigned)p.num_heads, (unsigned)p.num_seqs);
-    partition_reduce_kernel<T, D>
-        <<<grid, kThreads, (size_t)p.num_partitions * sizeof(float), stream>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.num_heads, (unsigned)p.num_seqs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)p.num_partitions * sizeof(float);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, partition_reduce_kernel<T, D>, p);
 }
 
 }  // namespace

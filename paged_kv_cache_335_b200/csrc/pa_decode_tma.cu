@@ -1,0 +1,817 @@
+// pa_decode_tma.cu — paged decode attention with K/V staged through shared
+// memory by the Tensor Memory Accelerator (sm_100a).
+//
+// What it computes is unchanged: for sequence s and query head h,
+// softmax(scale q . K_t) V_t over the n = context_lens[s] cached tokens, K_t and
+// V_t taken from physical block block_tables[s][t / block_size], slot
+// t % block_size ("AI 推理系列（十六）：PagedAttention——…", § PagedAttention 如何
+// 把连续序列映射到离散显存块 and § 非连续 KV 为什么需要专门的 Attention Kernel).
+//
+// How. One CTA = (partition, head or kv head, sequence), the three grid
+// dimensions of "vLLM的Paged Attention技术：高效注意力机制解析", § 3.2. Inside it:
+// * a producer warp reads the block-table entries of the partition 32 at a
+//   time and, for every 16-token sub-tile, issues tiled TMA loads of the K and
+//   V rows (boxes of 16 rows x 128 bytes, 128-byte swizzle, no multicast) into
+//   a ring of shared-memory stages guarded by mbarriers (full: data landed;
+//   empty: stage released);
+// * consumer warps take sub-tiles round robin (warp w: w, w+4, ...; § 4.2 of
+//   the same page), copy their fragments out of the stage, release it, and
+//   update a running max / sum / accumulator (online softmax in exp2).
+// Two consumers share this pipeline: the CUDA-core one (one query head per
+// CTA; any dtype) and the tensor-core one for grouped-query attention (bf16,
+// group 2..8: S^T = K Q^T and O^T += V^T P^T as m16n8k16 MMAs, tokens as M,
+// the query group as N). The swizzle makes every consumer fragment load
+// bank-conflict free. Every wait is bounded: after kWaitLimitNs the waiter
+// records PA_ERR_TIMEOUT and carries on, so the kernel always terminates.
+// The arithmetic order depends only on logical token positions.
+#include <math.h>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+#include "pa_tma.cuh"
+
+namespace pa {
+
+static __device__ unsigned int s_status_tma;
+
+namespace {
+
+// Tunables (compile-time; the defaults are the measured choice).
+#ifndef PA_TMA_CONSUMER_WARPS
+#define PA_TMA_CONSUMER_WARPS 4
+#endif
+#ifndef PA_TMA_RING_BYTES
+#define PA_TMA_RING_BYTES 65536
+#endif
+#ifndef PA_MMA_MIN_BLOCKS
+#define PA_MMA_MIN_BLOCKS 2
+#endif
+#ifndef PA_MMA_SPLIT_QK
+#define PA_MMA_SPLIT_QK 0
+#endif
+
+constexpr int kConsumerWarps = PA_TMA_CONSUMER_WARPS;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kBoxBytes = 16 * 128;                  // 16 rows x 128 bytes
+constexpr int kGroupMax = 8;
+
+template <typename T, int D>
+struct Geom {
+    static constexpr int kBoxes = D * (int)sizeof(T) / 128;     // boxes per K (or V) row set
+    static constexpr int kBoxElems = 128 / (int)sizeof(T);      // elements per box row
+    static constexpr int kStageBytes = 2 * kBoxes * kBoxBytes;  // K + V of one sub-tile
+    // Stages: as many as fit in PA_TMA_RING_BYTES, rounded DOWN to a multiple
+    // of the consumer warps. Consumers take sub-tiles round robin, so with a
+    // multiple every stage always belongs to the same warp and no warp can wait
+    // on a stage more than one phase ahead of its data; otherwise a warp can
+    // test a phase parity two phases early, see it as already complete, read a
+    // stage before its load lands and release it twice.
+    static constexpr int kFit = PA_TMA_RING_BYTES / kStageBytes;
+    static constexpr int kStages =
+        kFit < kConsumerWarps ? kConsumerWarps : (kFit / kConsumerWarps) * kConsumerWarps;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static_assert(kStages % kConsumerWarps == 0, "stage count must be a multiple of the consumer warps");
+};
+
+struct Ring {
+    uint32_t stages;  // shared address of stage 0 (1024-byte aligned)
+    uint32_t full;    // shared address of full[0]; full[i] at + 8 i
+    uint32_t empty;
+    int* valid;       // per stage: 1 = data loaded, 0 = skipped (bad block id)
+};
+
+// Issue of one sub-tile by one producer lane: wait until its stage is free,
+// then load K and V rows [row, row + 16) of kv head `kh` into it (or, for a
+// block id outside the pool, mark the stage empty-handed and complete it).
+// Returns false if the wait timed out (nothing was issued).
+template <typename T, int D>
+__device__ __forceinline__ bool issue_subtile(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                              const DecodeParams& p, const Ring& ring, int gi,
+                                              int phys, int kh, int tok0) {
+    using G = Geom<T, D>;
+    const int st = gi % G::kStages;
+    const uint32_t round = (uint32_t)(gi / G::kStages);
+    if (!mbar_wait_bounded(ring.empty + 8 * st, (round & 1u) ^ 1u)) {
+        atomicOr(&s_status_tma, kStatusTimeout);
+        return false;
+    }
+    if ((unsigned)phys < (unsigned)p.num_blocks) {
+        ring.valid[st] = 1;
+        const uint32_t full = ring.full + 8 * st;
+        mbar_arrive_expect_tx(full, G::kStageBytes);
+        const int32_t row = (phys * p.num_kv_heads + kh) * p.block_size + (tok0 & (p.block_size - 1));
+        const uint32_t sb = ring.stages + st * G::kStageBytes;
+#pragma unroll
+        for (int b = 0; b < G::kBoxes; ++b)
+            tma_load_2d(sb + b * kBoxBytes, kmap, b * G::kBoxElems, row, full);
+#pragma unroll
+        for (int b = 0; b < G::kBoxes; ++b)
+            tma_load_2d(sb + (G::kBoxes + b) * kBoxBytes, vmap, b * G::kBoxElems, row, full);
+    } else {
+        atomicOr(&s_status_tma, kStatusBadIndex);
+        ring.valid[st] = 0;
+        mbar_arrive(ring.full + 8 * st);
+    }
+    return true;
+}
+
+// Issue a batch of `cnt` <= 32 consecutive sub-tiles (ring positions g .. g+cnt-1)
+// of one item; lane l owns sub-tile l (`phys` = its block id). Lanes issue in
+// sub-rounds of kStages, so each sub-round touches every stage at most once and
+// a stage's rounds are issued in order. `issued` tracks 1 + the last position
+// issued; `dead` becomes warp-wide once any wait timed out.
+template <typename T, int D>
+__device__ __forceinline__ void issue_batch(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                            const DecodeParams& p, const Ring& ring, int g, int cnt,
+                                            int phys, int kh, int tok0_lane, int lane, int& issued,
+                                            bool& dead) {
+    using G = Geom<T, D>;
+    for (int k0 = 0; k0 < cnt && !dead; k0 += G::kStages) {
+        bool ok = true;
+        if (lane >= k0 && lane < k0 + G::kStages && lane < cnt) {
+            ok = issue_subtile<T, D>(kmap, vmap, p, ring, g + lane, phys, kh, tok0_lane);
+            if (ok) issued = g + lane + 1;
+        }
+        dead = __any_sync(0xffffffffu, !ok);
+    }
+    issued = __reduce_max_sync(0xffffffffu, issued);
+}
+
+// Producer of one item: all lanes fetch block-table entries, 32 sub-tiles at a
+// time, and issue them. Returns the ring position after the item.
+template <typename T, int D>
+__device__ __forceinline__ int produce_item(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                            const DecodeParams& p, const Ring& ring, int s, int kh,
+                                            int t0, int n_sub, int lane, int g, int& issued,
+                                            bool& dead) {
+    const int32_t* table = p.block_tables + (int64_t)s * p.table_stride;
+    for (int base = 0; base < n_sub && !dead; base += 32) {
+        const int i = base + lane;
+        const int tok0 = t0 + (i << 4);
+        int phys = -1;
+        if (i < n_sub) phys = __ldg(table + (tok0 >> p.log2_block_size));
+        issue_batch<T, D>(kmap, vmap, p, ring, g + base, min(32, n_sub - base), phys, kh, tok0,
+                          lane, issued, dead);
+    }
+    return g + n_sub;
+}
+
+// Drain: the last load of every stage has landed before the CTA reuses or
+// releases shared memory (immediate unless a consumer gave up waiting).
+template <typename T, int D>
+__device__ __forceinline__ void drain_ring(const Ring& ring, int issued, int lane) {
+    using G = Geom<T, D>;
+    if (lane != 0 || issued <= 0) return;
+    const int last = min(issued, G::kStages);
+    for (int st = 0; st < last; ++st) {
+        const int it = issued - 1 - ((issued - 1 - st) % G::kStages);
+        const uint32_t round = (uint32_t)(it / G::kStages);
+        if (!mbar_wait_bounded(ring.full + 8 * st, round & 1u)) atomicOr(&s_status_tma, kStatusTimeout);
+    }
+}
+
+// Shared memory: [pad to 1024] [ring] [extra_bytes] [full bars] [empty bars] [valid]
+template <typename T, int D>
+__device__ __forceinline__ uint8_t* setup_ring(uint8_t* smem_raw, Ring& ring, int extra_bytes = 0) {
+    using G = Geom<T, D>;
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+    uint8_t* base = smem_raw + pad;
+    ring.stages = raw + pad;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + G::kRingBytes + ((extra_bytes + 7) & ~7));
+    ring.full = smem_u32(bars);
+    ring.empty = smem_u32(bars + G::kStages);
+    ring.valid = reinterpret_cast<int*>(bars + 2 * G::kStages);
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < G::kStages; ++st) {
+            mbar_init(ring.full + 8 * st, 1);
+            mbar_init(ring.empty + 8 * st, 1);
+        }
+        fence_barrier_init();
+    }
+    return base;
+}
+
+template <typename T, int D>
+constexpr size_t smem_bytes(int extra_bytes = 0) {
+    using G = Geom<T, D>;
+    return 1024 + G::kRingBytes + ((extra_bytes + 7) & ~7) + 2 * G::kStages * 8 + G::kStages * 4 + 64;
+}
+
+__device__ __forceinline__ int clamp_ctx(int ctx, int max_ctx, bool report) {
+    if (ctx < 0 || ctx > max_ctx) {
+        if (report) atomicOr(&s_status_tma, kStatusBadIndex);
+        ctx = ctx < 0 ? 0 : max_ctx;
+    }
+    return ctx;
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core consumer: one query head per CTA.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
+                       const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
+    using G = Geom<T, D>;
+    constexpr int VEC = Elem<T>::kVec;          // elements per 16-byte chunk
+    constexpr int CPR = D / VEC;                // chunks per row
+    constexpr int RPL = 32 / CPR;               // rows per warp-wide pass
+    constexpr int ITER = 16 / RPL;              // passes per 16-row sub-tile
+    constexpr int IPP = ITER < 8 ? ITER : 8;    // passes held in registers at once
+    extern __shared__ uint8_t smem_raw[];
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    const int part = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ctx = clamp_ctx(__ldg(p.context_lens + s), p.max_context_len,
+                              threadIdx.x == 0 && part == 0);
+    const int t0 = part * p.partition_size;
+    const int t1 = min(ctx, t0 + p.partition_size);
+    const int64_t out_row = (int64_t)s * p.num_heads + h;
+    if (t0 >= t1) {
+        if (p.num_partitions == 1)
+            for (int d = threadIdx.x; d < D; d += kThreads) Elem<T>::store(p.out, out_row * D + d, 0.f);
+        return;
+    }
+    const int kh = h / (p.num_heads / p.num_kv_heads);
+    const int n_sub = (t1 - t0 + 15) >> 4;
+    Ring ring;
+    uint8_t* base = setup_ring<T, D>(smem_raw, ring);
+    __syncthreads();
+
+    float m = -INFINITY, l = 0.f;
+    float acc[VEC];
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
+
+    if (warp == kConsumerWarps) {
+        if (lane == 0) {
+            prefetch_tensormap(&kmap);
+            prefetch_tensormap(&vmap);
+        }
+        bool dead = false;
+        int issued = 0;
+        produce_item<T, D>(&kmap, &vmap, p, ring, s, kh, t0, n_sub, lane, 0, issued, dead);
+        drain_ring<T, D>(ring, issued, lane);
+    } else {
+        const int c = lane % CPR, rs = lane / CPR;
+        const uint32_t coff = (uint32_t)(c / 8) * kBoxBytes;  // box of this lane's chunk
+        const uint32_t cx = (uint32_t)(c % 8);
+        float qf[VEC];
+        {
+            const uint4 raw = ld_v4(static_cast<const T*>(p.q) + out_row * D + c * VEC);
+            Elem<T>::widen(raw, qf);
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) qf[j] *= p.scale_log2;
+        }
+        bool dead = false;
+        for (int i = warp; i < n_sub && !dead; i += kConsumerWarps) {
+            const int st = i % G::kStages;
+            const uint32_t round = (uint32_t)(i / G::kStages);
+            if (!mbar_wait_bounded(ring.full + 8 * st, round & 1u)) {
+                if (lane == 0) atomicOr(&s_status_tma, kStatusTimeout);
+                dead = true;
+                break;
+            }
+            const bool valid = ring.valid[st] != 0;
+            const uint32_t kb = ring.stages + st * G::kStageBytes + coff;
+            const uint32_t vb = kb + G::kBoxes * kBoxBytes;
+            const int tok0 = t0 + (i << 4);
+#pragma unroll
+            for (int pass = 0; pass < ITER; pass += IPP) {
+                uint4 kr[IPP], vr[IPP];
+#pragma unroll
+                for (int it = 0; it < IPP; ++it) {
+                    const uint32_t row = (uint32_t)((pass + it) * RPL + rs);
+                    kr[it] = lds128(kb + swz(row, cx));
+                    vr[it] = lds128(vb + swz(row, cx));
+                }
+                if (pass + IPP >= ITER) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(ring.empty + 8 * st);
+                }
+                if (!valid) continue;
+                float sc[IPP];
+#pragma unroll
+                for (int it = 0; it < IPP; ++it) {
+                    float kf[VEC];
+                    Elem<T>::widen(kr[it], kf);
+                    float dot = 0.f;
+#pragma unroll
+                    for (int j = 0; j < VEC; ++j) dot = fmaf(qf[j], kf[j], dot);
+#pragma unroll
+                    for (int off = 1; off < CPR; off <<= 1)
+                        dot += __shfl_xor_sync(0xffffffffu, dot, off);
+                    const int tok = tok0 + (pass + it) * RPL + rs;
+                    sc[it] = tok < t1 ? dot : -INFINITY;
+                }
+                float mt = sc[0];
+#pragma unroll
+                for (int it = 1; it < IPP; ++it) mt = fmaxf(mt, sc[it]);
+#pragma unroll
+                for (int off = CPR; off < 32; off <<= 1)
+                    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+                if (mt == -INFINITY) continue;  // only masked rows in this pass
+                const float m_new = fmaxf(m, mt);
+                const float alpha = exp2f(m - m_new);
+                l *= alpha;
+#pragma unroll
+                for (int j = 0; j < VEC; ++j) acc[j] *= alpha;
+#pragma unroll
+                for (int it = 0; it < IPP; ++it) {
+                    const float pr = exp2f(sc[it] - m_new);
+                    l += pr;
+                    const int tok = tok0 + (pass + it) * RPL + rs;
+                    if (tok < t1) {  // slots past the context may hold anything, even NaN
+                        float vf[VEC];
+                        Elem<T>::widen(vr[it], vf);
+#pragma unroll
+                        for (int j = 0; j < VEC; ++j) acc[j] = fmaf(pr, vf[j], acc[j]);
+                    }
+                }
+                m = m_new;
+            }
+        }
+#pragma unroll
+        for (int off = CPR; off < 32; off <<= 1) {
+            l += __shfl_xor_sync(0xffffffffu, l, off);
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+        }
+    }
+    __syncthreads();  // all loads landed and consumed: the ring is free
+
+    float* sm_o = reinterpret_cast<float*>(base);            // [warps][D]
+    float* sm_m = sm_o + kConsumerWarps * D;                 // [warps]
+    float* sm_l = sm_m + kConsumerWarps;
+    if (warp < kConsumerWarps) {
+        const int c = lane % CPR, rs = lane / CPR;
+        if (rs == 0) {
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) sm_o[warp * D + c * VEC + j] = acc[j];
+        }
+        if (lane == 0) {
+            sm_m[warp] = m;
+            sm_l[warp] = l;
+        }
+    }
+    __syncthreads();
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w]);
+    float wgt[kConsumerWarps];
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+        wgt[w] = sm_m[w] == -INFINITY ? 0.f : exp2f(sm_m[w] - M);
+        L = fmaf(sm_l[w], wgt[w], L);
+    }
+    for (int d = threadIdx.x; d < D; d += kThreads) {
+        float o = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) o = fmaf(sm_o[w * D + d], wgt[w], o);
+        const float val = L > 0.f ? o / L : 0.f;
+        if (p.num_partitions == 1)
+            Elem<T>::store(p.out, out_row * D + d, val);
+        else
+            p.ws_o[(out_row * p.num_partitions + part) * D + d] = val;
+    }
+    if (p.num_partitions > 1 && threadIdx.x == 0) {
+        float* ml = p.ws_ml + (out_row * p.num_partitions + part) * 2;
+        ml[0] = L > 0.f ? M : -INFINITY;
+        ml[1] = L;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core consumer: the whole query group of one kv head per CTA.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// Merge buffer of the tensor-core consumer: per warp and query row, the
+// running max, sum and head_dim accumulators (rows padded to D + 1 floats so
+// the fragment stores hit at most two banks per word).
+template <int D>
+constexpr int merge_bytes() {
+    return (kConsumerWarps * kGroupMax * (D + 1) + 2 * kConsumerWarps * kGroupMax) * 4;
+}
+
+// The work items of one persistent CTA, in order: u = blockIdx.x + k * gridDim.x,
+// item u = (partition u % P, kv head, sequence). Every warp walks them itself;
+// the context lengths of 32 upcoming items are held one per lane, so a warp
+// pays one load latency per 32 items, not per item.
+struct ItemWalk {
+    int k;        // ordinal of the current item within this CTA
+    int kbase;    // ordinal of the item whose context length lane 0 holds
+    int ctx_lane; // context length of item kbase + lane (clamped), -1 past the end
+};
+
+struct Item {
+    bool valid;   // false: no items left
+    int s, kh, part, t0, t1;
+};
+
+__device__ __forceinline__ int item_ctx_load(const DecodeParams& p, int num_items, int kbase,
+                                             int lane, bool report) {
+    const int u = blockIdx.x + (kbase + lane) * gridDim.x;
+    if (u >= num_items) return -1;
+    const int s = (u / p.num_partitions) / p.num_kv_heads;
+    const int part = u % p.num_partitions;
+    return clamp_ctx(__ldg(p.context_lens + s), p.max_context_len, report && part == 0);
+}
+
+// Next non-empty item (t0 < t1) or !valid. Items that are empty are returned
+// too when `want_empty` (consumers write zeros for them when P == 1).
+__device__ __forceinline__ Item item_next(ItemWalk& w, const DecodeParams& p, int num_items,
+                                          int lane, bool report, bool want_empty) {
+    for (;;) {
+        const int u = blockIdx.x + w.k * gridDim.x;
+        Item it;
+        it.valid = u < num_items;
+        if (!it.valid) return it;
+        if (w.k - w.kbase >= 32) {
+            w.kbase = w.k;
+            w.ctx_lane = item_ctx_load(p, num_items, w.kbase, lane, report);
+        }
+        const int ctx = __shfl_sync(0xffffffffu, w.ctx_lane, w.k - w.kbase);
+        it.part = u % p.num_partitions;
+        const int rest = u / p.num_partitions;
+        it.kh = rest % p.num_kv_heads;
+        it.s = rest / p.num_kv_heads;
+        it.t0 = it.part * p.partition_size;
+        it.t1 = min(ctx, it.t0 + p.partition_size);
+        ++w.k;
+        if (it.t0 < it.t1 || want_empty) return it;
+    }
+}
+
+// Persistent: each CTA walks its work items. The producer streams the items'
+// sub-tiles through the ring without a break between items (block-table
+// entries fetched one 32-sub-tile batch ahead), while the consumers finish one
+// item (cross-warp merge, store) and start the next (q fragments fetched one
+// item ahead).
+template <int D>
+__global__ void __launch_bounds__(kThreads, PA_MMA_MIN_BLOCKS)
+decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
+                      const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
+                      int num_items) {
+    using T = __nv_bfloat16;
+    using G = Geom<T, D>;
+    constexpr int KCH = D / 32;  // 16-byte K chunks per row per thread (2 k-steps each)
+    constexpr int VCH = D / 64;  // V boxes
+    constexpr int MT = D / 16;   // PV m-tiles
+    constexpr int OS = D + 1;    // merge-buffer row stride (floats)
+    extern __shared__ uint8_t smem_raw[];
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int P = p.num_partitions;
+    const int group = p.num_heads / p.num_kv_heads;
+    Ring ring;
+    uint8_t* base = setup_ring<T, D>(smem_raw, ring, merge_bytes<D>());
+    float* sm_o = reinterpret_cast<float*>(base + G::kRingBytes);  // [warps][8][OS]
+    float* sm_m = sm_o + kConsumerWarps * kGroupMax * OS;           // [warps][8]
+    float* sm_l = sm_m + kConsumerWarps * kGroupMax;
+    ItemWalk walk;
+    walk.k = 0;
+    walk.kbase = 0;
+    walk.ctx_lane = item_ctx_load(p, num_items, 0, lane, warp == 0);
+    __syncthreads();
+
+    if (warp == kConsumerWarps) {  // producer
+        if (lane == 0) {
+            prefetch_tensormap(&kmap);
+            prefetch_tensormap(&vmap);
+        }
+        bool dead = false;
+        int g = 0, issued = 0;
+        // batches of up to 32 sub-tiles, the next batch's table entries in flight
+        Item cur = item_next(walk, p, num_items, lane, false, false);
+        int cur_base = 0;
+        int phys_cur = -1;
+        if (cur.valid && lane < ((cur.t1 - cur.t0 + 15) >> 4))
+            phys_cur = __ldg(p.block_tables + (int64_t)cur.s * p.table_stride +
+                             ((cur.t0 + (lane << 4)) >> p.log2_block_size));
+        while (cur.valid && !dead) {
+            const int n_sub = (cur.t1 - cur.t0 + 15) >> 4;
+            Item nxt = cur;
+            int nxt_base = cur_base + 32;
+            if (nxt_base >= n_sub) {
+                nxt = item_next(walk, p, num_items, lane, false, false);
+                nxt_base = 0;
+            }
+            int phys_nxt = -1;
+            if (nxt.valid && nxt_base + lane < ((nxt.t1 - nxt.t0 + 15) >> 4))
+                phys_nxt = __ldg(p.block_tables + (int64_t)nxt.s * p.table_stride +
+                                 ((nxt.t0 + ((nxt_base + lane) << 4)) >> p.log2_block_size));
+            const int cnt = min(32, n_sub - cur_base);
+            issue_batch<T, D>(&kmap, &vmap, p, ring, g, cnt, phys_cur, cur.kh,
+                              cur.t0 + ((cur_base + lane) << 4), lane, issued, dead);
+            g += cnt;
+            cur = nxt;
+            cur_base = nxt_base;
+            phys_cur = phys_nxt;
+        }
+        drain_ring<T, D>(ring, issued, lane);
+        return;
+    }
+
+    // consumers (threads 0 .. 127)
+    const int r = lane >> 2, c = lane & 3;
+    const int tv0 = 2 * c, tv1 = 2 * c + 1, tv2 = 2 * c + 8, tv3 = 2 * c + 9;
+    bool dead = false;
+    int g = 0;
+    // Q^T (B operand of QK): thread (r, c) holds query row r. For chunk step jp
+    // (k-steps 2jp, 2jp+1) it reads 16-byte chunk x = 2c + (jp & 1) of box jp / 2,
+    // the same head_dim positions its K fragments come from.
+    auto load_q = [&](const Item& it, uint4 (&q)[KCH]) {
+        const int64_t head0 = (int64_t)it.s * p.num_heads + (int64_t)it.kh * group;
+        if (it.valid && it.t0 < it.t1 && r < group) {
+            const uint16_t* qrow = static_cast<const uint16_t*>(p.q) + (head0 + r) * D;
+#pragma unroll
+            for (int jp = 0; jp < KCH; ++jp)
+                q[jp] = ld_v4(qrow + (jp >> 1) * 64 + (2 * c + (jp & 1)) * 8);
+        } else {
+#pragma unroll
+            for (int jp = 0; jp < KCH; ++jp) q[jp] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    Item cur = item_next(walk, p, num_items, lane, warp == 0, true);
+    uint4 qcur[KCH];
+    load_q(cur, qcur);
+    while (cur.valid) {
+        Item nxt = item_next(walk, p, num_items, lane, warp == 0, true);
+        uint4 qnxt[KCH];
+        load_q(nxt, qnxt);  // in flight while this item is processed
+        const int64_t head0 = (int64_t)cur.s * p.num_heads + (int64_t)cur.kh * group;
+        if (cur.t0 >= cur.t1) {
+            if (P == 1)
+                for (int idx = threadIdx.x; idx < group * D; idx += kConsumerWarps * 32)
+                    Elem<T>::store(p.out, head0 * D + idx, 0.f);
+        } else {
+            const int t0 = cur.t0, t1 = cur.t1;
+            const int n_sub = (t1 - t0 + 15) >> 4;
+            float acc[MT][4];
+#pragma unroll
+            for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+            float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+            for (int i = warp; i < n_sub && !dead; i += kConsumerWarps) {
+                const int gi = g + i;
+                const int st = gi % G::kStages;
+                const uint32_t round = (uint32_t)(gi / G::kStages);
+                if (!mbar_wait_bounded(ring.full + 8 * st, round & 1u)) {
+                    if (lane == 0) atomicOr(&s_status_tma, kStatusTimeout);
+                    dead = true;
+                    break;
+                }
+                const bool valid = ring.valid[st] != 0;
+                const uint32_t kb = ring.stages + st * G::kStageBytes;
+                const uint32_t vb = kb + G::kBoxes * kBoxBytes;
+                float sc[4] = {0.f, 0.f, 0.f, 0.f};
+                {
+                    uint4 kr[2][KCH];
+#pragma unroll
+                    for (int jp = 0; jp < KCH; ++jp) {
+                        const uint32_t bx = kb + (jp >> 1) * kBoxBytes;
+                        const uint32_t x = (uint32_t)(2 * c + (jp & 1));
+                        kr[0][jp] = lds128(bx + swz(r, x));
+                        kr[1][jp] = lds128(bx + swz(r + 8, x));
+                    }
+                    // S^T = K . Q^T
+#if PA_MMA_SPLIT_QK
+                    float sd[4] = {0.f, 0.f, 0.f, 0.f};  // second chain: shorter MMA dependency
+#pragma unroll
+                    for (int jp = 0; jp < KCH; ++jp) {
+                        mma_16816(sc, kr[0][jp].x, kr[1][jp].x, kr[0][jp].y, kr[1][jp].y,
+                                  qcur[jp].x, qcur[jp].y);
+                        mma_16816(sd, kr[0][jp].z, kr[1][jp].z, kr[0][jp].w, kr[1][jp].w,
+                                  qcur[jp].z, qcur[jp].w);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sc[e] += sd[e];
+#else
+#pragma unroll
+                    for (int jp = 0; jp < KCH; ++jp) {
+                        mma_16816(sc, kr[0][jp].x, kr[1][jp].x, kr[0][jp].y, kr[1][jp].y,
+                                  qcur[jp].x, qcur[jp].y);
+                        mma_16816(sc, kr[0][jp].z, kr[1][jp].z, kr[0][jp].w, kr[1][jp].w,
+                                  qcur[jp].z, qcur[jp].w);
+                    }
+#endif
+                }
+                uint4 vr[4][VCH];
+#pragma unroll
+                for (int hh = 0; hh < VCH; ++hh) {
+                    const uint32_t bx = vb + hh * kBoxBytes;
+                    vr[0][hh] = lds128(bx + swz(tv0, r));
+                    vr[1][hh] = lds128(bx + swz(tv1, r));
+                    vr[2][hh] = lds128(bx + swz(tv2, r));
+                    vr[3][hh] = lds128(bx + swz(tv3, r));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
+                if (!valid) continue;
+
+                const int tok0 = t0 + (i << 4);
+                const int nvalid = t1 - tok0;
+                const bool lo_ok = r < nvalid, hi_ok = r + 8 < nvalid;
+                const float s0 = lo_ok ? sc[0] * p.scale_log2 : -INFINITY;  // token r,   head 2c
+                const float s1 = lo_ok ? sc[1] * p.scale_log2 : -INFINITY;  // token r,   head 2c+1
+                const float s2 = hi_ok ? sc[2] * p.scale_log2 : -INFINITY;  // token r+8, head 2c
+                const float s3 = hi_ok ? sc[3] * p.scale_log2 : -INFINITY;  // token r+8, head 2c+1
+                float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                }
+                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+                const uint32_t x0 = pack_bf16x2(exp2f(s0 - mn0), exp2f(s1 - mn1));
+                const uint32_t x1 = pack_bf16x2(exp2f(s2 - mn0), exp2f(s3 - mn1));
+                // the sums use the same rounded weights the PV product sees
+                l0 = fmaf(l0, al0, bf16_lo(x0) + bf16_lo(x1));
+                l1 = fmaf(l1, al1, bf16_hi(x0) + bf16_hi(x1));
+                m0 = mn0;
+                m1 = mn1;
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    acc[t][0] *= al0;
+                    acc[t][1] *= al1;
+                    acc[t][2] *= al0;
+                    acc[t][3] *= al1;
+                }
+                const uint32_t pb0 = movmatrix_trans(x0);  // P^T rows (tokens) 2c, 2c+1; col head r
+                const uint32_t pb1 = movmatrix_trans(x1);  // tokens 2c+8, 2c+9
+                if (nvalid < 16) {  // slots past the context may hold anything, even NaN
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int hh = 0; hh < VCH; ++hh) {
+                        if (tv0 >= nvalid) vr[0][hh] = z;
+                        if (tv1 >= nvalid) vr[1][hh] = z;
+                        if (tv2 >= nvalid) vr[2][hh] = z;
+                        if (tv3 >= nvalid) vr[3][hh] = z;
+                    }
+                }
+                // O^T += V^T . P^T ; m-tile t covers head_dim 64*(t/4) + 8r + 2*(t%4) (+1 for row r+8)
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    const int hh = t >> 2, w = t & 3;
+                    const uint32_t xa = word(vr[0][hh], w), xb = word(vr[1][hh], w);
+                    const uint32_t ya = word(vr[2][hh], w), yb = word(vr[3][hh], w);
+                    mma_16816(acc[t], __byte_perm(xa, xb, 0x5410), __byte_perm(xa, xb, 0x7632),
+                              __byte_perm(ya, yb, 0x5410), __byte_perm(ya, yb, 0x7632), pb0, pb1);
+                }
+            }
+            g += n_sub;
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+            }
+            // cross-warp merge of this item, in fixed warp order
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
+                float* o = sm_o + (warp * kGroupMax + 2 * c) * OS;
+                o[d0] = acc[t][0];
+                o[OS + d0] = acc[t][1];
+                o[d0 + 1] = acc[t][2];
+                o[OS + d0 + 1] = acc[t][3];
+            }
+            if (r == 0) {
+                sm_m[warp * kGroupMax + 2 * c] = m0;
+                sm_m[warp * kGroupMax + 2 * c + 1] = m1;
+                sm_l[warp * kGroupMax + 2 * c] = l0;
+                sm_l[warp * kGroupMax + 2 * c + 1] = l1;
+            }
+            named_barrier(1, kConsumerWarps * 32);
+            for (int idx = threadIdx.x; idx < group * D; idx += kConsumerWarps * 32) {
+                const int n = idx / D;
+                const int d = idx - n * D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * kGroupMax + n]);
+                float L = 0.f, o = 0.f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float mw = sm_m[w * kGroupMax + n];
+                    const float wg = mw == -INFINITY ? 0.f : exp2f(mw - M);
+                    L = fmaf(sm_l[w * kGroupMax + n], wg, L);
+                    o = fmaf(sm_o[(w * kGroupMax + n) * OS + d], wg, o);
+                }
+                const float val = L > 0.f ? o / L : 0.f;
+                const int64_t row = head0 + n;
+                if (P == 1) {
+                    Elem<T>::store(p.out, row * D + d, val);
+                } else {
+                    p.ws_o[(row * P + cur.part) * D + d] = val;
+                    if (d == 0) {
+                        float* ml = p.ws_ml + (row * P + cur.part) * 2;
+                        ml[0] = L > 0.f ? M : -INFINITY;
+                        ml[1] = L;
+                    }
+                }
+            }
+            named_barrier(1, kConsumerWarps * 32);  // merge buffer free for the next item
+        }
+        cur = nxt;
+#pragma unroll
+        for (int jp = 0; jp < KCH; ++jp) qcur[jp] = qnxt[jp];
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_simt_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
+                          cudaStream_t stream) {
+    constexpr size_t smem = smem_bytes<T, D>();
+    cudaError_t e = cudaFuncSetAttribute(decode_tma_simt_kernel<T, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_tma_simt_kernel<T, D>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)p.num_partitions, (unsigned)p.num_heads, (unsigned)p.num_seqs);
+    decode_tma_simt_kernel<T, D><<<grid, kThreads, smem, stream>>>(km, vm, p);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
+                         cudaStream_t stream) {
+    constexpr size_t smem = smem_bytes<__nv_bfloat16, D>(merge_bytes<D>());
+    auto kernel = decode_tma_mma_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    // persistent grid: every CTA slot of the GPU, or fewer if there are fewer items
+    static int per_sm[128] = {0};
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+    if (per_sm[dev] == 0) {
+        int n = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, smem)) != cudaSuccess)
+            return e;
+        per_sm[dev] = n > 0 ? n : 1;
+    }
+    int sms = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const long items = (long)p.num_partitions * p.num_kv_heads * p.num_seqs;
+    const long slots = (long)per_sm[dev] * sms;
+    const unsigned grid = (unsigned)(items < slots ? items : slots);
+    kernel<<<grid, kThreads, smem, stream>>>(km, vm, p, (int)items);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bool mma,
+                              const CUtensorMap& kmap, const CUtensorMap& vmap,
+                              cudaStream_t stream) {
+    if (mma) {
+        return head_dim == 64 ? launch_mma_t<64>(p, kmap, vmap, stream)
+                              : launch_mma_t<128>(p, kmap, vmap, stream);
+    }
+    if (dtype == 0) {
+        return head_dim == 64 ? launch_simt_t<float, 64>(p, kmap, vmap, stream)
+                              : launch_simt_t<float, 128>(p, kmap, vmap, stream);
+    }
+    return head_dim == 64 ? launch_simt_t<__nv_bfloat16, 64>(p, kmap, vmap, stream)
+                          : launch_simt_t<__nv_bfloat16, 128>(p, kmap, vmap, stream);
+}
+
+cudaError_t read_status_tma(unsigned* bits, bool clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(bits, s_status_tma, sizeof(unsigned));
+    if (e != cudaSuccess || !clear) return e;
+    const unsigned zero = 0;
+    return cudaMemcpyToSymbol(s_status_tma, &zero, sizeof(unsigned));
+}
+
+}  // namespace pa

@@ -2,6 +2,7 @@
 // kernel translation units. Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -11,6 +12,8 @@ namespace pa {
 // Bit of the per-translation-unit status word a kernel sets when it meets an
 // out-of-range block id, slot or context length (and skips the access).
 constexpr unsigned kStatusBadIndex = 1u;
+// Bit set when a bounded wait on a shared-memory pipeline barrier gave up.
+constexpr unsigned kStatusTimeout = 2u;
 
 // Everything one decode launch needs. Offsets are in elements unless noted.
 struct DecodeParams {
@@ -58,6 +61,13 @@ cudaError_t launch_decode_simt(const DecodeParams& p, int dtype, int head_dim,
 // CTA per (partition, kv head, sequence) covering the whole query group.
 bool mma_supported(int dtype, int head_dim, int group);
 cudaError_t launch_decode_mma(const DecodeParams& p, int head_dim, cudaStream_t stream);
+// Decode with K/V staged through shared memory by TMA (producer warp +
+// consumer warps); `mma` selects the tensor-core GQA consumer. The tensor maps
+// describe k_cache / v_cache as [num_blocks * num_kv_heads * block_size rows]
+// x [head_dim], boxes of 16 rows x 128 bytes, 128-byte swizzle.
+cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bool mma,
+                              const CUtensorMap& kmap, const CUtensorMap& vmap,
+                              cudaStream_t stream);
 // Log-sum-exp merge of the P partial results into out.
 cudaError_t launch_partition_reduce(const DecodeParams& p, int dtype, int head_dim,
                                     cudaStream_t stream);
@@ -71,5 +81,6 @@ int report_error(int code, const char* fmt, ...);
 cudaError_t read_status_copy(unsigned* bits, bool clear);
 cudaError_t read_status_simt(unsigned* bits, bool clear);
 cudaError_t read_status_mma(unsigned* bits, bool clear);
+cudaError_t read_status_tma(unsigned* bits, bool clear);
 
 }  // namespace pa
