@@ -10,8 +10,12 @@ Prints ONE JSON line (rank 0). ``value`` is algorithmic HBM bytes of the whole
 step (decode K/V + q + out, append read+write, block copy read+write) per second
 of device time, summed over ranks (weak scaling: each rank owns its own batch;
 sequences are independent, so no data-path collective exists). Inputs are
-resident in HBM; L2 is flushed between timed steps and every step is timed with
-its own CUDA events on the launching stream.
+resident in HBM and every step is timed with its own CUDA events on the
+launching stream. Between timed steps L2 is not flushed when the step's unique
+input bytes exceed twice the 126 MB L2 (every benched configuration: 0.3 to 6.8
+GB); a smaller workload is flushed by writing a 512 MiB buffer. A write flush
+leaves ~126 MB of dirty lines that the next step must write back, which is why
+it is not used where the inputs alone already evict L2.
 """
 from __future__ import annotations
 
@@ -34,9 +38,14 @@ sys.path.insert(0, ROOT)
 METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); seq-steps/s"
 UNIT = "GB/s"
 DEFAULT_CONFIG = "llama13b_bs16"
-EXTRA_CONFIGS = ["llama7b", "llama13b_bs16", "llama13b_bs32", "llama70b_gqa", "cow_beam4"]
+# (label, workload name, partition_size override or None = the workload's own)
+EXTRA_CONFIGS = [("llama7b", "llama7b", None), ("llama13b_bs16", "llama13b_bs16", None),
+                 ("llama13b_bs32", "llama13b_bs32", None), ("llama70b_gqa", "llama70b_gqa", None),
+                 ("llama70b_gqa_policy", "llama70b_gqa", 0), ("cow_beam4", "cow_beam4", None)]
 FALLBACK_HBM_GBS = 6650.0
+DATASHEET_HBM_GBS = 8000.0
 L2_FLUSH_BYTES = 512 << 20          # > 2x the 126 MB L2
+STREAM_BYTES = 4 << 30
 
 
 def parse_args():
@@ -46,6 +55,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--partition-size", type=int, default=None,
+                    help="override the workload's partition size (0 = library policy)")
     ap.add_argument("--no-extra-configs", action="store_true",
                     help="skip the per-configuration table")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -60,6 +71,50 @@ def parse_args():
 def dist_env():
     return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
             int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def dist_max(x: float, device) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(step_bytes: int, steps: int, world: int, max_total_ms: float) -> float:
+    """Whole-job GB/s: every rank moved step_bytes per step; the job took the
+    slowest rank's time."""
+    return world * step_bytes * steps / (max_total_ms / 1e3) / 1e9
+
+
+def stream_read_gbs(device, reps=10):
+    """Read bandwidth of the library's read-only streaming kernel over 4 GiB."""
+    import torch
+
+    import paged_kv_cache_335_b200 as pa
+    lib = pa.load_library()
+    buf = torch.empty(STREAM_BYTES, dtype=torch.uint8, device=device)
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    ctas = sms * 4
+    part = torch.empty(ctas, dtype=torch.int32, device=device)
+    st = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    args = (ctypes.c_void_p(buf.data_ptr()), ctypes.c_size_t(STREAM_BYTES),
+            ctypes.c_void_p(part.data_ptr()), ctas, st)
+    times = []
+    for i in range(reps + 3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        if lib.pa_stream_read(*args) != 0:
+            raise RuntimeError("pa_stream_read failed")
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            times.append(e0.elapsed_time(e1))
+    del buf
+    return STREAM_BYTES / (statistics.median(times) / 1e3) / 1e9
 
 
 def peaks():
@@ -173,7 +228,7 @@ def profile_traffic(kernel_file, workload):
 class Step:
     """Device-resident inputs of one workload and pre-marshalled C-ABI calls."""
 
-    def __init__(self, wl, device, seed_offset=0):
+    def __init__(self, wl, device, seed_offset=0, partition_size=None):
         import torch
 
         import paged_kv_cache_335_b200 as pa
@@ -189,7 +244,7 @@ class Step:
         self.pairs = torch.as_tensor(wl.copy_pairs, device=device)
         self.out = torch.empty_like(v["q"])
         self.desc = pa.cache_desc(v["k_cache"])
-        self.ps = wl.partition_size
+        self.ps = wl.partition_size if partition_size is None else partition_size
         self.num_partitions = pa.pa_decode_num_partitions(wl.num_seqs, wl.num_heads,
                                                           wl.max_context_len, v["k_cache"], self.ps)
         need = pa.pa_decode_workspace_size(wl.num_seqs, wl.num_heads, wl.max_context_len,
@@ -242,11 +297,22 @@ class Step:
         del self.vals, self.out, self.ws
 
 
+L2_BYTES = 126 * 10**6
+
+
+def needs_flush(wl) -> bool:
+    """Flush L2 between steps only when the step's inputs could stay in it."""
+    unique = wl.unique_kv_bytes() if wl.copy_pairs.shape[0] else wl.kv_bytes()
+    return unique < 2 * L2_BYTES
+
+
 def time_steps(step, steps, warmup, flush, barrier=None):
-    """Device time of `steps` steps (L2 flushed before each), per-step events."""
+    """Device time of `steps` steps with per-step events; `flush` (a tensor or
+    None) is overwritten before each step to evict L2."""
     torch = step.torch
     for _ in range(warmup):
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         step.run()
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
@@ -255,7 +321,8 @@ def time_steps(step, steps, warmup, flush, barrier=None):
     torch.cuda.synchronize()
     t_wall0 = time.time()
     for i in range(steps):
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         step.run(evs[i])
     torch.cuda.synchronize()
     t_wall1 = time.time()
@@ -372,7 +439,7 @@ def reference_arm(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.mean(secs),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_dict(wl),
+        "data": "synthetic", "config": config_dict(wl, needs_flush(wl)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -381,14 +448,15 @@ def reference_arm(args):
     return 0
 
 
-def config_dict(wl, flush=True):
+def config_dict(wl, flush=False):
     return {"workload": wl.name, "num_seqs": wl.num_seqs, "num_heads": wl.num_heads,
             "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
             "block_size": wl.block_size, "dtype": wl.dtype,
             "context_tokens": int(wl.context_lens.sum()),
             "max_context_len": wl.max_context_len, "copy_pairs": int(wl.copy_pairs.shape[0]),
             "appended_tokens": wl.num_tokens, "pool_blocks": wl.num_blocks,
-            "l2": ("flushed between timed steps (512 MiB write)" if flush else "not flushed"),
+            "l2": ("flushed between timed steps (512 MiB write)" if flush else
+                   f"not flushed: inputs larger than L2 ({(wl.unique_kv_bytes() if wl.copy_pairs.shape[0] else wl.kv_bytes()) / 1e9:.2f} GB unique K/V per step vs 126 MB L2)"),
             "description": wl.description}
 
 
@@ -425,8 +493,10 @@ def main():
         if world > 1:
             dist.barrier()
 
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     wl = W.make(args.config)
+    if args.partition_size is not None:
+        wl.partition_size = args.partition_size
     step = Step(wl, device, seed_offset=rank)
 
     uuid = None
@@ -436,6 +506,7 @@ def main():
         uuid = str(local_rank)
     clocks = ClockSampler(uuid)
     clocks.start()
+    flush = flush_buf if needs_flush(wl) else None
     res = time_steps(step, args.steps, args.warmup, flush, barrier)
     t0, t1 = res["wall"]
     # the timed region is short: continue the same (untimed) loop for >= 1.5 s so
@@ -445,7 +516,8 @@ def main():
         t_end = time.time() + 1.5
         while time.time() < t_end:
             for _ in range(20):
-                flush.zero_()
+                if flush is not None:
+                    flush.zero_()
                 step.run()
             torch.cuda.synchronize()
         probe_t1 = time.time()
@@ -462,48 +534,46 @@ def main():
     if remeasured:
         clk["remeasured"] = True
 
-    total_ms = sum(res["step_ms"])
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = dist_max(sum(res["step_ms"]), device)
     ms_per_step = total_ms / args.steps
-    value = world * step.step_bytes * args.steps / (total_ms / 1e3) / 1e9
+    value = weak_scaling_value(step.step_bytes, args.steps, world, total_ms)
     dec_ms = statistics.mean(res["decode_ms"])
     dec_gbs = wl.decode_bytes() / (dec_ms / 1e3) / 1e9
-    kernel_file = os.path.join(ROOT, "paged_kv_cache_335_b200", "csrc",
-                               "pa_decode_mma.cu" if wl.num_heads // wl.num_kv_heads in range(2, 9)
-                               else "pa_decode_simt.cu")
+    kernel_file = os.path.join(ROOT, "paged_kv_cache_335_b200", "csrc", "pa_decode_tma.cu")
+    gqa = wl.dtype == "bf16" and 2 <= wl.num_heads // wl.num_kv_heads <= 8
     traffic, sha = profile_traffic(kernel_file, wl.name)
 
     # end to end through the public binding with host buffers
     e2e_ms, h2d, d2h = e2e_steps(step, args.steps, max(3, args.warmup))
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * step.step_bytes * args.steps / (e2e_ms / 1e3) / 1e9
+    e2e_ms = dist_max(e2e_ms, device)
+    e2e_value = weak_scaling_value(step.step_bytes, args.steps, world, e2e_ms)
     launches = step.launches_per_step * args.steps
     step.release()
     del step
     torch.cuda.empty_cache()
 
+    read_gbs = stream_read_gbs(device) if world == 1 else None
     per_config = {}
     if world == 1 and not args.no_extra_configs:
-        for name in EXTRA_CONFIGS:
+        for label, name, ps in EXTRA_CONFIGS:
             w2 = W.make(name)
-            st = Step(w2, device)
-            r2 = time_steps(st, min(args.steps, 50), 3, flush)
+            st = Step(w2, device, partition_size=ps)
+            r2 = time_steps(st, min(args.steps, 50), 3, flush_buf if needs_flush(w2) else None)
             sm = statistics.median(r2["step_ms"])
             dm = statistics.median(r2["decode_ms"])
-            per_config[name] = {
+            per_config[label] = {
                 "decode_gbs": round(w2.decode_bytes() / (dm / 1e3) / 1e9, 1),
                 "decode_frac_of_peak": round(w2.decode_bytes() / (dm / 1e3) / 1e9 / hbm_peak, 4),
+                "decode_frac_of_datasheet": round(
+                    w2.decode_bytes() / (dm / 1e3) / 1e9 / DATASHEET_HBM_GBS, 4),
+                "decode_frac_of_stream_read": round(
+                    w2.decode_bytes() / (dm / 1e3) / 1e9 / read_gbs, 4) if read_gbs else None,
                 "decode_us": round(dm * 1e3, 2),
                 "step_us": round(sm * 1e3, 2),
                 "moves_us": round(statistics.median(r2["moves_ms"]) * 1e3, 2),
                 "seq_steps_per_s": round(w2.num_seqs / (sm / 1e3), 1),
                 "partitions": st.num_partitions,
+                "partition_size": "library policy" if st.ps == 0 else st.ps,
                 "decode_bytes": w2.decode_bytes(),
                 "unique_kv_bytes": w2.unique_kv_bytes() if name.startswith("cow") else None,
             }
@@ -524,15 +594,20 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic (seeded N(0,1) values, seeded shapes)",
-            "config": config_dict(wl),
+            "config": config_dict(wl, flush is not None),
             "seq_steps_per_s": round(world * wl.num_seqs / (ms_per_step / 1e3), 1),
             "frac_of_hbm_peak": round(value / world / hbm_peak, 4),
+            "reference_bandwidths_gbs": {
+                "measured_copy_hbm_gbs": hbm_peak, "datasheet": DATASHEET_HBM_GBS,
+                "stream_read_this_run": round(read_gbs, 1) if read_gbs else None},
+            "decode_frac_of_stream_read": round(dec_gbs / read_gbs, 4) if read_gbs else None,
             "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm_peak,
                          "unit": "GB/s", "frac": round(dec_gbs / hbm_peak, 4),
                          "traffic": traffic,
-                         "kernel": "pa_decode (" + ("tensor-core GQA" if "mma" in kernel_file
-                                                    else "CUDA-core") + " kernel"
-                                   + (" + partition reduce)" if step_partitions(wl) > 1 else ")"),
+                         "kernel": ("decode_tma_mma_kernel (persistent, tensor-core GQA)" if gqa
+                                    else "decode_tma_simt_kernel (CUDA-core)")
+                                   + (" + partition_reduce_kernel" if step_partitions(wl) > 1
+                                      else ""),
                          "algorithmic_bytes_per_launch": wl.decode_bytes(),
                          "avg_launch_us": round(dec_ms * 1e3, 2),
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"

@@ -1,0 +1,28 @@
+/*
+ * pa_test.h — test hook of the paged-attention library; not for production use.
+ *
+ * pa_test_skip_load — while `position` >= 0, every following pa_decode call
+ * (from any thread) leaves ring position `position` of each CTA's K/V pipeline
+ * unloaded. The consumer waiting for that position gives up after its bounded
+ * wait (about one second), the producer and the other waiters then give up in
+ * turn, the kernel still terminates, its outputs are invalid, and pa_sync_check
+ * returns PA_ERR_TIMEOUT; the CUDA context stays usable. -1 restores normal
+ * operation. It exists only so that the timeout path can be tested without a
+ * fault or a hang.
+ */
+#ifndef PA_TEST_H
+#define PA_TEST_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+void pa_test_skip_load(int32_t position);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_TEST_H */

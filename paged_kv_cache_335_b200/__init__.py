@@ -23,7 +23,8 @@ import threading
 
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG_DIR, "libpa.so")
-HEADER = os.path.join(os.path.dirname(PKG_DIR), "include", "pa.h")
+INCLUDE_DIR = os.path.join(os.path.dirname(PKG_DIR), "include")
+HEADER = os.path.join(INCLUDE_DIR, "pa.h")
 
 PA_OK = 0
 PA_ERR_INVALID_ARG = -1
@@ -33,6 +34,7 @@ PA_ERR_UNSUPPORTED = -4
 PA_ERR_CUDA = -5
 PA_ERR_BAD_INDEX = -6
 PA_ERR_WORKSPACE = -7
+PA_ERR_TIMEOUT = -8
 PA_F32 = 0
 PA_BF16 = 1
 PA_NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -86,6 +88,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_decode_num_partitions.argtypes = [i32, i32, i32, desc, i32]
         lib.pa_block_copy.argtypes = [vp, i32, vp, vp, desc, vp]
         lib.pa_sync_check.argtypes = [vp]
+        lib.pa_stream_read.argtypes = [vp, sz, vp, i32, vp]
+        lib.pa_test_skip_load.argtypes = [i32]
+        lib.pa_test_skip_load.restype = None
+        lib.pa_stream_read.restype = ctypes.c_int
         lib.pa_get_last_error.argtypes = []
         lib.pa_get_last_error.restype = ctypes.c_char_p
         lib.pa_status_string.argtypes = [ctypes.c_int]
@@ -98,12 +104,17 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         return lib
 
 
-def header_functions(header: str = HEADER) -> list:
-    """Names of the functions ``include/pa.h`` declares."""
-    text = open(header, encoding="utf-8").read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w]*\s*\*?\s*(pa_\w+)\s*\(",
-                                 text, flags=re.M)))
+def header_functions(header: str | None = None) -> list:
+    """Names of the functions the headers under ``include/`` declare (or one header)."""
+    paths = [header] if header else sorted(
+        os.path.join(INCLUDE_DIR, f) for f in os.listdir(INCLUDE_DIR) if f.endswith(".h"))
+    names = set()
+    for path in paths:
+        text = open(path, encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names.update(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w]*\s*\*?\s*(pa_\w+)\s*\(",
+                                text, flags=re.M))
+    return sorted(names)
 
 
 def _check(rc: int) -> None:

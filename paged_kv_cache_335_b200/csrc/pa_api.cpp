@@ -14,10 +14,12 @@
 
 #include "pa.h"
 #include "pa_internal.h"
+#include "pa_test.h"
 
 namespace {
 
 thread_local std::string t_last_error;
+int g_test_skip_position = -1;  // set only by pa_test_skip_load
 
 int fail(int code, const char* fmt, ...) {
     char buf[512];
@@ -121,19 +123,10 @@ int make_cache_map(CUtensorMap* map, const void* base, const pa_cache_desc* c) {
     return PA_OK;
 }
 
-// Decode kernel family: TMA-staged (default) or direct register loads
-// (PA_DECODE_IMPL=regs), kept for A/B measurement.
-bool use_tma_kernels() {
-    static int v = -1;
-    if (v < 0) {
-        const char* e = std::getenv("PA_DECODE_IMPL");
-        v = (e && std::strcmp(e, "regs") == 0) ? 0 : 1;
-    }
-    return v == 1;
-}
-
 constexpr int kMaxPartitions = 4096;
-constexpr int kAutoPartition = 512;
+constexpr int kAutoPartition = 512;    // CUDA-core kernel: partition when splitting
+constexpr int kMmaItemTokens = 2048;   // tensor-core kernel: target tokens per item
+constexpr int kMinPartition = 256;     // tensor-core kernel: smallest partition
 
 struct Plan {
     bool use_mma;
@@ -159,8 +152,6 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
     if (max_ctx < 0) return fail(PA_ERR_INVALID_ARG, "max_context_len %d is negative", max_ctx);
     const int group = num_heads / c->num_kv_heads;
     plan->use_mma = pa::mma_supported(c->dtype, c->head_dim, group);
-    if (!plan->use_mma && !pa::simt_supported(c->dtype, c->head_dim))
-        return fail(PA_ERR_UNSUPPORTED, "no kernel for dtype %d head_dim %d", c->dtype, c->head_dim);
     const int whole = round_up16(max_ctx > 16 ? max_ctx : 16);
     int ps = whole, np = 1;
     if (partition_size > 0) {
@@ -174,16 +165,34 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
             return fail(PA_ERR_INVALID_ARG, "partition_size %d gives %d partitions (max %d)",
                         partition_size, np, kMaxPartitions);
     } else if (partition_size == 0) {
-        // The persistent tensor-core kernel balances its items statically, so it
-        // wants many equal items; the CUDA-core kernel only needs to fill the GPU.
-        const long units = (long)num_seqs * (plan->use_mma ? c->num_kv_heads : num_heads);
-        const long want = (plan->use_mma ? 8L : 4L) * sm_count();
-        if (units < want && max_ctx > kAutoPartition) {
-            ps = kAutoPartition;
-            np = (max_ctx + ps - 1) / ps;
-            while (np > kMaxPartitions) {
-                ps *= 2;
+        if (plan->use_mma) {
+            // The persistent tensor-core kernel hands equal-sized items to its CTAs
+            // statically and pays a merge + partial write per item, so it wants few
+            // large items (about kMmaItemTokens tokens) of EQUAL size, and at least
+            // one per CTA slot. The context is cut into `np` equal partitions.
+            const long units = (long)num_seqs * c->num_kv_heads;
+            const long slots = (long)sm_count() * pa::mma_ctas_per_sm();
+            long want = (max_ctx + kMmaItemTokens - 1) / kMmaItemTokens;
+            const long fill = (slots + units - 1) / (units > 0 ? units : 1);
+            if (fill > want) want = fill;
+            const long most = (max_ctx + kMinPartition - 1) / kMinPartition;  // >= 256 tokens each
+            if (want > most) want = most;
+            if (want > kMaxPartitions) want = kMaxPartitions;
+            if (want > 1) {
+                ps = round_up16((int)((max_ctx + want - 1) / want));
                 np = (max_ctx + ps - 1) / ps;
+            }
+        } else {
+            // The CUDA-core kernel is not persistent: split only when the
+            // (sequence, head) units alone cannot fill the GPU.
+            const long units = (long)num_seqs * num_heads;
+            if (units < 4L * sm_count() && max_ctx > kAutoPartition) {
+                ps = kAutoPartition;
+                np = (max_ctx + ps - 1) / ps;
+                while (np > kMaxPartitions) {
+                    ps *= 2;
+                    np = (max_ctx + ps - 1) / ps;
+                }
             }
         }
     } else if (partition_size != -1) {
@@ -317,17 +326,13 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
     p.partition_size = plan.partition_size;
     p.num_partitions = plan.num_partitions;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.test_skip_position = g_test_skip_position;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    if (use_tma_kernels()) {
-        CUtensorMap kmap, vmap;
-        if ((rc = make_cache_map(&kmap, k_cache, cache)) != PA_OK) return rc;
-        if ((rc = make_cache_map(&vmap, v_cache, cache)) != PA_OK) return rc;
-        e = pa::launch_decode_tma(p, cache->dtype, cache->head_dim, plan.use_mma, kmap, vmap, st);
-    } else {
-        e = plan.use_mma ? pa::launch_decode_mma(p, cache->head_dim, st)
-                         : pa::launch_decode_simt(p, cache->dtype, cache->head_dim, st);
-    }
+    CUtensorMap kmap, vmap;
+    if ((rc = make_cache_map(&kmap, k_cache, cache)) != PA_OK) return rc;
+    if ((rc = make_cache_map(&vmap, v_cache, cache)) != PA_OK) return rc;
+    cudaError_t e =
+        pa::launch_decode_tma(p, cache->dtype, cache->head_dim, plan.use_mma, kmap, vmap, st);
     if (e != cudaSuccess) return fail_cuda(e, "pa_decode launch");
     if (plan.num_partitions > 1) {
         e = pa::launch_partition_reduce(p, cache->dtype, cache->head_dim, st);
@@ -339,22 +344,21 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
 int pa_sync_check(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail_cuda(e, "pa_sync_check: stream");
-    unsigned a = 0, b = 0, c = 0, d = 0;
+    unsigned a = 0, b = 0;
     if ((e = pa::read_status_copy(&a, true)) != cudaSuccess ||
-        (e = pa::read_status_simt(&b, true)) != cudaSuccess ||
-        (e = pa::read_status_mma(&c, true)) != cudaSuccess ||
-        (e = pa::read_status_tma(&d, true)) != cudaSuccess)
+        (e = pa::read_status_tma(&b, true)) != cudaSuccess)
         return fail_cuda(e, "pa_sync_check: status word");
-    if ((a | b | c | d) & pa::kStatusTimeout)
-        return fail(PA_ERR_TIMEOUT, "a bounded pipeline wait gave up (bits copy=%u simt=%u mma=%u "
-                    "tma=%u)", a, b, c, d);
-    if ((a | b | c | d) & pa::kStatusBadIndex)
+    if ((a | b) & pa::kStatusTimeout)
+        return fail(PA_ERR_TIMEOUT, "a bounded pipeline wait gave up (bits copy=%u decode=%u)", a, b);
+    if ((a | b) & pa::kStatusBadIndex)
         return fail(PA_ERR_BAD_INDEX, "a kernel met a block id, slot or context length outside "
-                    "its bounds (bits copy=%u simt=%u mma=%u tma=%u)", a, b, c, d);
+                    "its bounds (bits copy=%u decode=%u)", a, b);
     return PA_OK;
 }
 
 const char* pa_get_last_error(void) { return t_last_error.c_str(); }
+
+void pa_test_skip_load(int32_t position) { g_test_skip_position = position < 0 ? -1 : position; }
 
 const char* pa_status_string(int status) {
     switch (status) {

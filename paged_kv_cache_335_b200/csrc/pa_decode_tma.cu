@@ -36,41 +36,52 @@ static __device__ unsigned int s_status_tma;
 
 namespace {
 
-// Tunables (compile-time; the defaults are the measured choice).
-#ifndef PA_TMA_CONSUMER_WARPS
-#define PA_TMA_CONSUMER_WARPS 4
+// Tunables (compile-time; the defaults are the measured choice, see the
+// variant sweeps recorded with the profiles). Consumer warps per CTA, ring
+// bytes, and for the persistent tensor-core kernel the CTAs per SM it is
+// compiled (and its grid sized) for.
+#ifndef PA_SIMT_CONSUMER_WARPS
+#define PA_SIMT_CONSUMER_WARPS 4
 #endif
-#ifndef PA_TMA_RING_BYTES
-#define PA_TMA_RING_BYTES 65536
+#ifndef PA_SIMT_RING_BYTES
+#define PA_SIMT_RING_BYTES 65536
+#endif
+#ifndef PA_MMA_CONSUMER_WARPS
+#define PA_MMA_CONSUMER_WARPS 2
+#endif
+#ifndef PA_MMA_RING_BYTES
+#define PA_MMA_RING_BYTES 32768
 #endif
 #ifndef PA_MMA_MIN_BLOCKS
-#define PA_MMA_MIN_BLOCKS 2
+#define PA_MMA_MIN_BLOCKS 4
 #endif
 #ifndef PA_MMA_SPLIT_QK
 #define PA_MMA_SPLIT_QK 0
 #endif
 
-constexpr int kConsumerWarps = PA_TMA_CONSUMER_WARPS;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
-constexpr int kBoxBytes = 16 * 128;                  // 16 rows x 128 bytes
+constexpr int kBoxBytes = 16 * 128;  // 16 rows x 128 bytes
 constexpr int kGroupMax = 8;
 
-template <typename T, int D>
+// Geometry of one pipeline: element type, head_dim, consumer warps, ring bytes.
+template <typename T_, int D_, int CW_, int RING_>
 struct Geom {
-    static constexpr int kBoxes = D * (int)sizeof(T) / 128;     // boxes per K (or V) row set
-    static constexpr int kBoxElems = 128 / (int)sizeof(T);      // elements per box row
-    static constexpr int kStageBytes = 2 * kBoxes * kBoxBytes;  // K + V of one sub-tile
-    // Stages: as many as fit in PA_TMA_RING_BYTES, rounded DOWN to a multiple
-    // of the consumer warps. Consumers take sub-tiles round robin, so with a
-    // multiple every stage always belongs to the same warp and no warp can wait
-    // on a stage more than one phase ahead of its data; otherwise a warp can
-    // test a phase parity two phases early, see it as already complete, read a
+    using T = T_;
+    static constexpr int D = D_;
+    static constexpr int kCW = CW_;                              // consumer warps
+    static constexpr int kThreads = (CW_ + 1) * 32;              // + one producer warp
+    static constexpr int kBoxes = D_ * (int)sizeof(T_) / 128;    // boxes per K (or V) row set
+    static constexpr int kBoxElems = 128 / (int)sizeof(T_);      // elements per box row
+    static constexpr int kStageBytes = 2 * kBoxes * kBoxBytes;   // K + V of one sub-tile
+    // Stages: as many as fit in RING_ bytes, rounded DOWN to a multiple of the
+    // consumer warps. Consumers take sub-tiles round robin, so with a multiple
+    // every stage always belongs to the same warp and no warp can wait on a
+    // stage more than one phase ahead of its data; otherwise a warp can test
+    // a phase parity two phases early, see it as already complete, read a
     // stage before its load lands and release it twice.
-    static constexpr int kFit = PA_TMA_RING_BYTES / kStageBytes;
-    static constexpr int kStages =
-        kFit < kConsumerWarps ? kConsumerWarps : (kFit / kConsumerWarps) * kConsumerWarps;
+    static constexpr int kFit = RING_ / kStageBytes;
+    static constexpr int kStages = kFit < CW_ ? CW_ : (kFit / CW_) * CW_;
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static_assert(kStages % kConsumerWarps == 0, "stage count must be a multiple of the consumer warps");
+    static_assert(kStages % CW_ == 0, "stage count must be a multiple of the consumer warps");
 };
 
 struct Ring {
@@ -84,17 +95,17 @@ struct Ring {
 // then load K and V rows [row, row + 16) of kv head `kh` into it (or, for a
 // block id outside the pool, mark the stage empty-handed and complete it).
 // Returns false if the wait timed out (nothing was issued).
-template <typename T, int D>
+template <class G>
 __device__ __forceinline__ bool issue_subtile(const CUtensorMap* kmap, const CUtensorMap* vmap,
                                               const DecodeParams& p, const Ring& ring, int gi,
                                               int phys, int kh, int tok0) {
-    using G = Geom<T, D>;
     const int st = gi % G::kStages;
     const uint32_t round = (uint32_t)(gi / G::kStages);
     if (!mbar_wait_bounded(ring.empty + 8 * st, (round & 1u) ^ 1u)) {
         atomicOr(&s_status_tma, kStatusTimeout);
         return false;
     }
+    if (gi == p.test_skip_position) return true;  // test hook: leave this stage unloaded
     if ((unsigned)phys < (unsigned)p.num_blocks) {
         ring.valid[st] = 1;
         const uint32_t full = ring.full + 8 * st;
@@ -120,16 +131,15 @@ __device__ __forceinline__ bool issue_subtile(const CUtensorMap* kmap, const CUt
 // sub-rounds of kStages, so each sub-round touches every stage at most once and
 // a stage's rounds are issued in order. `issued` tracks 1 + the last position
 // issued; `dead` becomes warp-wide once any wait timed out.
-template <typename T, int D>
+template <class G>
 __device__ __forceinline__ void issue_batch(const CUtensorMap* kmap, const CUtensorMap* vmap,
                                             const DecodeParams& p, const Ring& ring, int g, int cnt,
                                             int phys, int kh, int tok0_lane, int lane, int& issued,
                                             bool& dead) {
-    using G = Geom<T, D>;
     for (int k0 = 0; k0 < cnt && !dead; k0 += G::kStages) {
         bool ok = true;
         if (lane >= k0 && lane < k0 + G::kStages && lane < cnt) {
-            ok = issue_subtile<T, D>(kmap, vmap, p, ring, g + lane, phys, kh, tok0_lane);
+            ok = issue_subtile<G>(kmap, vmap, p, ring, g + lane, phys, kh, tok0_lane);
             if (ok) issued = g + lane + 1;
         }
         dead = __any_sync(0xffffffffu, !ok);
@@ -139,7 +149,7 @@ __device__ __forceinline__ void issue_batch(const CUtensorMap* kmap, const CUten
 
 // Producer of one item: all lanes fetch block-table entries, 32 sub-tiles at a
 // time, and issue them. Returns the ring position after the item.
-template <typename T, int D>
+template <class G>
 __device__ __forceinline__ int produce_item(const CUtensorMap* kmap, const CUtensorMap* vmap,
                                             const DecodeParams& p, const Ring& ring, int s, int kh,
                                             int t0, int n_sub, int lane, int g, int& issued,
@@ -150,7 +160,7 @@ __device__ __forceinline__ int produce_item(const CUtensorMap* kmap, const CUten
         const int tok0 = t0 + (i << 4);
         int phys = -1;
         if (i < n_sub) phys = __ldg(table + (tok0 >> p.log2_block_size));
-        issue_batch<T, D>(kmap, vmap, p, ring, g + base, min(32, n_sub - base), phys, kh, tok0,
+        issue_batch<G>(kmap, vmap, p, ring, g + base, min(32, n_sub - base), phys, kh, tok0,
                           lane, issued, dead);
     }
     return g + n_sub;
@@ -158,9 +168,8 @@ __device__ __forceinline__ int produce_item(const CUtensorMap* kmap, const CUten
 
 // Drain: the last load of every stage has landed before the CTA reuses or
 // releases shared memory (immediate unless a consumer gave up waiting).
-template <typename T, int D>
+template <class G>
 __device__ __forceinline__ void drain_ring(const Ring& ring, int issued, int lane) {
-    using G = Geom<T, D>;
     if (lane != 0 || issued <= 0) return;
     const int last = min(issued, G::kStages);
     for (int st = 0; st < last; ++st) {
@@ -171,9 +180,8 @@ __device__ __forceinline__ void drain_ring(const Ring& ring, int issued, int lan
 }
 
 // Shared memory: [pad to 1024] [ring] [extra_bytes] [full bars] [empty bars] [valid]
-template <typename T, int D>
+template <class G>
 __device__ __forceinline__ uint8_t* setup_ring(uint8_t* smem_raw, Ring& ring, int extra_bytes = 0) {
-    using G = Geom<T, D>;
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     uint8_t* base = smem_raw + pad;
@@ -192,9 +200,8 @@ __device__ __forceinline__ uint8_t* setup_ring(uint8_t* smem_raw, Ring& ring, in
     return base;
 }
 
-template <typename T, int D>
+template <class G>
 constexpr size_t smem_bytes(int extra_bytes = 0) {
-    using G = Geom<T, D>;
     return 1024 + G::kRingBytes + ((extra_bytes + 7) & ~7) + 2 * G::kStages * 8 + G::kStages * 4 + 64;
 }
 
@@ -210,10 +217,15 @@ __device__ __forceinline__ int clamp_ctx(int ctx, int max_ctx, bool report) {
 // CUDA-core consumer: one query head per CTA.
 // ---------------------------------------------------------------------------
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
+using SimtGeom = Geom<T, D, PA_SIMT_CONSUMER_WARPS, PA_SIMT_RING_BYTES>;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(SimtGeom<T, D>::kThreads)
 decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
-    using G = Geom<T, D>;
+    using G = SimtGeom<T, D>;
+    constexpr int kConsumerWarps = G::kCW;
+    constexpr int kThreads = G::kThreads;
     constexpr int VEC = Elem<T>::kVec;          // elements per 16-byte chunk
     constexpr int CPR = D / VEC;                // chunks per row
     constexpr int RPL = 32 / CPR;               // rows per warp-wide pass
@@ -237,7 +249,7 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
     const int kh = h / (p.num_heads / p.num_kv_heads);
     const int n_sub = (t1 - t0 + 15) >> 4;
     Ring ring;
-    uint8_t* base = setup_ring<T, D>(smem_raw, ring);
+    uint8_t* base = setup_ring<G>(smem_raw, ring);
     __syncthreads();
 
     float m = -INFINITY, l = 0.f;
@@ -252,8 +264,8 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         bool dead = false;
         int issued = 0;
-        produce_item<T, D>(&kmap, &vmap, p, ring, s, kh, t0, n_sub, lane, 0, issued, dead);
-        drain_ring<T, D>(ring, issued, lane);
+        produce_item<G>(&kmap, &vmap, p, ring, s, kh, t0, n_sub, lane, 0, issued, dead);
+        drain_ring<G>(ring, issued, lane);
     } else {
         const int c = lane % CPR, rs = lane / CPR;
         const uint32_t coff = (uint32_t)(c / 8) * kBoxBytes;  // box of this lane's chunk
@@ -269,7 +281,8 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
         for (int i = warp; i < n_sub && !dead; i += kConsumerWarps) {
             const int st = i % G::kStages;
             const uint32_t round = (uint32_t)(i / G::kStages);
-            if (!mbar_wait_bounded(ring.full + 8 * st, round & 1u)) {
+            // warp-uniform outcome: lanes must not split on a wait that ran out
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(ring.full + 8 * st, round & 1u))) {
                 if (lane == 0) atomicOr(&s_status_tma, kStatusTimeout);
                 dead = true;
                 break;
@@ -314,10 +327,12 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                     mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
                 if (mt == -INFINITY) continue;  // only masked rows in this pass
                 const float m_new = fmaxf(m, mt);
-                const float alpha = exp2f(m - m_new);
-                l *= alpha;
+                if (m_new != m) {  // warp-uniform; a factor of exactly 1 changes no bit
+                    const float alpha = exp2f(m - m_new);
+                    l *= alpha;
 #pragma unroll
-                for (int j = 0; j < VEC; ++j) acc[j] *= alpha;
+                    for (int j = 0; j < VEC; ++j) acc[j] *= alpha;
+                }
 #pragma unroll
                 for (int it = 0; it < IPP; ++it) {
                     const float pr = exp2f(sc[it] - m_new);
@@ -414,8 +429,16 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
 // running max, sum and head_dim accumulators (rows padded to D + 1 floats so
 // the fragment stores hit at most two banks per word).
 template <int D>
+using MmaGeom = Geom<__nv_bfloat16, D, PA_MMA_CONSUMER_WARPS, PA_MMA_RING_BYTES>;
+
+template <int D>
+constexpr int merge_floats() {
+    // o[warps][8][D + 1], m[warps][8], l[warps][8], w[warps][8] (normalised weights)
+    return PA_MMA_CONSUMER_WARPS * kGroupMax * (D + 1) + 3 * PA_MMA_CONSUMER_WARPS * kGroupMax;
+}
+template <int D>
 constexpr int merge_bytes() {
-    return (kConsumerWarps * kGroupMax * (D + 1) + 2 * kConsumerWarps * kGroupMax) * 4;
+    return 2 * merge_floats<D>() * 4;  // double-buffered: item k uses buffer k % 2
 }
 
 // The work items of one persistent CTA, in order: u = blockIdx.x + k * gridDim.x,
@@ -473,12 +496,13 @@ __device__ __forceinline__ Item item_next(ItemWalk& w, const DecodeParams& p, in
 // item (cross-warp merge, store) and start the next (q fragments fetched one
 // item ahead).
 template <int D>
-__global__ void __launch_bounds__(kThreads, PA_MMA_MIN_BLOCKS)
+__global__ void __launch_bounds__(MmaGeom<D>::kThreads, PA_MMA_MIN_BLOCKS)
 decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
                       int num_items) {
     using T = __nv_bfloat16;
-    using G = Geom<T, D>;
+    using G = MmaGeom<D>;
+    constexpr int kConsumerWarps = G::kCW;
     constexpr int KCH = D / 32;  // 16-byte K chunks per row per thread (2 k-steps each)
     constexpr int VCH = D / 64;  // V boxes
     constexpr int MT = D / 16;   // PV m-tiles
@@ -490,10 +514,9 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
     const int P = p.num_partitions;
     const int group = p.num_heads / p.num_kv_heads;
     Ring ring;
-    uint8_t* base = setup_ring<T, D>(smem_raw, ring, merge_bytes<D>());
-    float* sm_o = reinterpret_cast<float*>(base + G::kRingBytes);  // [warps][8][OS]
-    float* sm_m = sm_o + kConsumerWarps * kGroupMax * OS;           // [warps][8]
-    float* sm_l = sm_m + kConsumerWarps * kGroupMax;
+    uint8_t* base = setup_ring<G>(smem_raw, ring, merge_bytes<D>());
+    float* merge_buf = reinterpret_cast<float*>(base + G::kRingBytes);
+    int merge_sel = 0;  // which half of the double-buffered merge area this item uses
     ItemWalk walk;
     walk.k = 0;
     walk.kbase = 0;
@@ -527,14 +550,14 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 phys_nxt = __ldg(p.block_tables + (int64_t)nxt.s * p.table_stride +
                                  ((nxt.t0 + ((nxt_base + lane) << 4)) >> p.log2_block_size));
             const int cnt = min(32, n_sub - cur_base);
-            issue_batch<T, D>(&kmap, &vmap, p, ring, g, cnt, phys_cur, cur.kh,
+            issue_batch<G>(&kmap, &vmap, p, ring, g, cnt, phys_cur, cur.kh,
                               cur.t0 + ((cur_base + lane) << 4), lane, issued, dead);
             g += cnt;
             cur = nxt;
             cur_base = nxt_base;
             phys_cur = phys_nxt;
         }
-        drain_ring<T, D>(ring, issued, lane);
+        drain_ring<G>(ring, issued, lane);
         return;
     }
 
@@ -582,7 +605,8 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 const int gi = g + i;
                 const int st = gi % G::kStages;
                 const uint32_t round = (uint32_t)(gi / G::kStages);
-                if (!mbar_wait_bounded(ring.full + 8 * st, round & 1u)) {
+                // warp-uniform outcome: lanes must not split on a wait that ran out
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(ring.full + 8 * st, round & 1u))) {
                     if (lane == 0) atomicOr(&s_status_tma, kStatusTimeout);
                     dead = true;
                     break;
@@ -649,7 +673,11 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
                 }
                 const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-                const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+                // The accumulator is rescaled only when some running max moved; a
+                // factor of exactly 1 would leave every bit unchanged anyway.
+                const bool moved = __any_sync(0xffffffffu, mn0 != m0 || mn1 != m1);
+                const float al0 = moved ? exp2f(m0 - mn0) : 1.f;
+                const float al1 = moved ? exp2f(m1 - mn1) : 1.f;
                 const uint32_t x0 = pack_bf16x2(exp2f(s0 - mn0), exp2f(s1 - mn1));
                 const uint32_t x1 = pack_bf16x2(exp2f(s2 - mn0), exp2f(s3 - mn1));
                 // the sums use the same rounded weights the PV product sees
@@ -657,12 +685,14 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 l1 = fmaf(l1, al1, bf16_hi(x0) + bf16_hi(x1));
                 m0 = mn0;
                 m1 = mn1;
+                if (moved) {
 #pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                    acc[t][0] *= al0;
-                    acc[t][1] *= al1;
-                    acc[t][2] *= al0;
-                    acc[t][3] *= al1;
+                    for (int t = 0; t < MT; ++t) {
+                        acc[t][0] *= al0;
+                        acc[t][1] *= al1;
+                        acc[t][2] *= al0;
+                        acc[t][3] *= al1;
+                    }
                 }
                 const uint32_t pb0 = movmatrix_trans(x0);  // P^T rows (tokens) 2c, 2c+1; col head r
                 const uint32_t pb1 = movmatrix_trans(x1);  // tokens 2c+8, 2c+9
@@ -692,7 +722,14 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 l0 += __shfl_xor_sync(0xffffffffu, l0, off);
                 l1 += __shfl_xor_sync(0xffffffffu, l1, off);
             }
-            // cross-warp merge of this item, in fixed warp order
+            // Cross-warp merge of this item, in fixed warp order. Buffers alternate
+            // between items, so a warp that races ahead to the next item's merge
+            // cannot overwrite what a slower warp still reads here.
+            float* sm_o = merge_buf + merge_sel * merge_floats<D>();  // [warps][8][OS]
+            float* sm_m = sm_o + kConsumerWarps * kGroupMax * OS;     // [warps][8]
+            float* sm_l = sm_m + kConsumerWarps * kGroupMax;
+            float* sm_w = sm_l + kConsumerWarps * kGroupMax;          // weight / L
+            merge_sel ^= 1;
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
                 const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
@@ -709,34 +746,42 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 sm_l[warp * kGroupMax + 2 * c + 1] = l1;
             }
             named_barrier(1, kConsumerWarps * 32);
-            for (int idx = threadIdx.x; idx < group * D; idx += kConsumerWarps * 32) {
-                const int n = idx / D;
-                const int d = idx - n * D;
+            if (threadIdx.x < group) {  // one thread per query row: the warps' weights
+                const int n = threadIdx.x;
                 float M = -INFINITY;
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * kGroupMax + n]);
-                float L = 0.f, o = 0.f;
+                float wg[kConsumerWarps];
+                float L = 0.f;
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) {
                     const float mw = sm_m[w * kGroupMax + n];
-                    const float wg = mw == -INFINITY ? 0.f : exp2f(mw - M);
-                    L = fmaf(sm_l[w * kGroupMax + n], wg, L);
-                    o = fmaf(sm_o[(w * kGroupMax + n) * OS + d], wg, o);
+                    wg[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
+                    L = fmaf(sm_l[w * kGroupMax + n], wg[w], L);
                 }
-                const float val = L > 0.f ? o / L : 0.f;
-                const int64_t row = head0 + n;
-                if (P == 1) {
-                    Elem<T>::store(p.out, row * D + d, val);
-                } else {
-                    p.ws_o[(row * P + cur.part) * D + d] = val;
-                    if (d == 0) {
-                        float* ml = p.ws_ml + (row * P + cur.part) * 2;
-                        ml[0] = L > 0.f ? M : -INFINITY;
-                        ml[1] = L;
-                    }
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w)
+                    sm_w[w * kGroupMax + n] = L > 0.f ? wg[w] / L : 0.f;
+                if (P > 1) {
+                    float* ml = p.ws_ml + ((head0 + n) * P + cur.part) * 2;
+                    ml[0] = L > 0.f ? M : -INFINITY;
+                    ml[1] = L;
                 }
             }
-            named_barrier(1, kConsumerWarps * 32);  // merge buffer free for the next item
+            named_barrier(1, kConsumerWarps * 32);
+            for (int idx = threadIdx.x; idx < group * D; idx += kConsumerWarps * 32) {
+                const int n = idx / D;
+                const int d = idx - n * D;
+                float val = 0.f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w)
+                    val = fmaf(sm_o[(w * kGroupMax + n) * OS + d], sm_w[w * kGroupMax + n], val);
+                const int64_t row = head0 + n;
+                if (P == 1)
+                    Elem<T>::store(p.out, row * D + d, val);
+                else
+                    p.ws_o[(row * P + cur.part) * D + d] = val;
+            }
         }
         cur = nxt;
 #pragma unroll
@@ -747,7 +792,8 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
 template <typename T, int D>
 cudaError_t launch_simt_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
                           cudaStream_t stream) {
-    constexpr size_t smem = smem_bytes<T, D>();
+    using G = SimtGeom<T, D>;
+    constexpr size_t smem = smem_bytes<G>();
     cudaError_t e = cudaFuncSetAttribute(decode_tma_simt_kernel<T, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -756,14 +802,15 @@ cudaError_t launch_simt_t(const DecodeParams& p, const CUtensorMap& km, const CU
                              (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)p.num_partitions, (unsigned)p.num_heads, (unsigned)p.num_seqs);
-    decode_tma_simt_kernel<T, D><<<grid, kThreads, smem, stream>>>(km, vm, p);
+    decode_tma_simt_kernel<T, D><<<grid, G::kThreads, smem, stream>>>(km, vm, p);
     return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
                          cudaStream_t stream) {
-    constexpr size_t smem = smem_bytes<__nv_bfloat16, D>(merge_bytes<D>());
+    using G = MmaGeom<D>;
+    constexpr size_t smem = smem_bytes<G>(merge_bytes<D>());
     auto kernel = decode_tma_mma_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -777,7 +824,7 @@ cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUt
     if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
     if (per_sm[dev] == 0) {
         int n = 0;
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, smem)) != cudaSuccess)
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, G::kThreads, smem)) != cudaSuccess)
             return e;
         per_sm[dev] = n > 0 ? n : 1;
     }
@@ -786,7 +833,7 @@ cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUt
     const long items = (long)p.num_partitions * p.num_kv_heads * p.num_seqs;
     const long slots = (long)per_sm[dev] * sms;
     const unsigned grid = (unsigned)(items < slots ? items : slots);
-    kernel<<<grid, kThreads, smem, stream>>>(km, vm, p, (int)items);
+    kernel<<<grid, G::kThreads, smem, stream>>>(km, vm, p, (int)items);
     return cudaGetLastError();
 }
 
@@ -805,6 +852,12 @@ cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bo
     }
     return head_dim == 64 ? launch_simt_t<__nv_bfloat16, 64>(p, kmap, vmap, stream)
                           : launch_simt_t<__nv_bfloat16, 128>(p, kmap, vmap, stream);
+}
+
+int mma_ctas_per_sm() { return PA_MMA_MIN_BLOCKS; }
+
+bool mma_supported(int dtype, int head_dim, int group) {
+    return dtype == 1 && (head_dim == 64 || head_dim == 128) && group >= 2 && group <= kGroupMax;
 }
 
 cudaError_t read_status_tma(unsigned* bits, bool clear) {

@@ -36,6 +36,7 @@ struct DecodeParams {
     int32_t partition_size;     // tokens per partition (whole context when P == 1)
     int32_t num_partitions;     // P
     float scale_log2;           // softmax scale * log2(e)
+    int32_t test_skip_position; // -1; >= 0 only under pa_test_skip_load (timeout test)
 };
 
 struct CopyParams {
@@ -53,14 +54,13 @@ cudaError_t launch_kv_append(const void* k, const void* v, const int64_t* slot_m
 cudaError_t launch_block_copy(const int64_t* pairs, int32_t num_pairs, void* k_cache,
                               void* v_cache, const CopyParams& cp, cudaStream_t stream);
 
-// CUDA-core decode: one CTA per (partition, query head, sequence).
-bool simt_supported(int dtype, int head_dim);
-cudaError_t launch_decode_simt(const DecodeParams& p, int dtype, int head_dim,
-                               cudaStream_t stream);
-// Tensor-core decode for grouped-query attention (bf16, 2 <= group <= 8): one
-// CTA per (partition, kv head, sequence) covering the whole query group.
+// Which decode kernel a call uses: the tensor-core GQA consumer for bf16 with
+// a query group of 2..8, the CUDA-core consumer otherwise.
 bool mma_supported(int dtype, int head_dim, int group);
-cudaError_t launch_decode_mma(const DecodeParams& p, int head_dim, cudaStream_t stream);
+// CTA slots per SM the persistent tensor-core kernel is built for (its grid is
+// at most this many CTAs per SM; the partition policy sizes items for it).
+int mma_ctas_per_sm();
+
 // Decode with K/V staged through shared memory by TMA (producer warp +
 // consumer warps); `mma` selects the tensor-core GQA consumer. The tensor maps
 // describe k_cache / v_cache as [num_blocks * num_kv_heads * block_size rows]
@@ -79,8 +79,6 @@ int report_error(int code, const char* fmt, ...);
 // Status words of the kernel translation units: OR of kStatus* bits since the
 // last clear. Return cudaSuccess or the copy error.
 cudaError_t read_status_copy(unsigned* bits, bool clear);
-cudaError_t read_status_simt(unsigned* bits, bool clear);
-cudaError_t read_status_mma(unsigned* bits, bool clear);
 cudaError_t read_status_tma(unsigned* bits, bool clear);
 
 }  // namespace pa
