@@ -125,8 +125,8 @@ int make_cache_map(CUtensorMap* map, const void* base, const pa_cache_desc* c) {
 
 constexpr int kMaxPartitions = 4096;
 constexpr int kAutoPartition = 512;    // CUDA-core kernel: partition when splitting
-constexpr int kMmaItemTokens = 2048;   // tensor-core kernel: target tokens per item
-constexpr int kMinPartition = 256;     // tensor-core kernel: smallest partition
+constexpr double kMmaItemOverhead = 8.0; // tensor-core kernel: per-item cost, in 16-token sub-tiles
+constexpr int kMinPartition = 256;       // tensor-core kernel: smallest partition
 
 struct Plan {
     bool use_mma;
@@ -166,22 +166,36 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
                         partition_size, np, kMaxPartitions);
     } else if (partition_size == 0) {
         if (plan->use_mma) {
-            // The persistent tensor-core kernel hands equal-sized items to its CTAs
-            // statically and pays a merge + partial write per item, so it wants few
-            // large items (about kMmaItemTokens tokens) of EQUAL size, and at least
-            // one per CTA slot. The context is cut into `np` equal partitions.
+            // The persistent tensor-core kernel hands items to its CTA slots statically
+            // (item u to CTA u mod slots), so its time is about
+            //   waves * (sub-tiles per item + per-item overhead),  waves = ceil(items / slots),
+            // the overhead being the item's merge, partial write and share of the reduce.
+            // Pick the partition count with the smallest such cost (ties: fewer partitions),
+            // partitions cut equal and at least kMinPartition tokens long.
             const long units = (long)num_seqs * c->num_kv_heads;
             const long slots = (long)sm_count() * pa::mma_ctas_per_sm();
-            long want = (max_ctx + kMmaItemTokens - 1) / kMmaItemTokens;
-            const long fill = (slots + units - 1) / (units > 0 ? units : 1);
-            if (fill > want) want = fill;
-            const long most = (max_ctx + kMinPartition - 1) / kMinPartition;  // >= 256 tokens each
-            if (want > most) want = most;
-            if (want > kMaxPartitions) want = kMaxPartitions;
-            if (want > 1) {
-                ps = round_up16((int)((max_ctx + want - 1) / want));
-                np = (max_ctx + ps - 1) / ps;
+            long most = (max_ctx + kMinPartition - 1) / kMinPartition;
+            if (most > kMaxPartitions) most = kMaxPartitions;
+            if (most < 1) most = 1;
+            long best_np = 1, best_ps = whole;
+            double best_cost = -1.0;
+            for (long n = 1; n <= most; ++n) {
+                const int cand_ps = round_up16((int)((max_ctx + n - 1) / n));
+                const long cand_np = (max_ctx + cand_ps - 1) / cand_ps;
+                if (cand_np != n) continue;  // rounding merged two cuts: seen already
+                const long items = units * cand_np;
+                const long waves = (items + slots - 1) / slots;
+                const double cost =
+                    (double)waves * ((double)(cand_np == 1 ? whole : cand_ps) / 16.0 +
+                                     (cand_np == 1 ? 0.0 : kMmaItemOverhead));
+                if (best_cost < 0.0 || cost < best_cost) {
+                    best_cost = cost;
+                    best_np = cand_np;
+                    best_ps = cand_ps;
+                }
             }
+            np = (int)best_np;
+            ps = np == 1 ? whole : (int)best_ps;
         } else {
             // The CUDA-core kernel is not persistent: split only when the
             // (sequence, head) units alone cannot fill the GPU.
@@ -348,6 +362,8 @@ int pa_sync_check(void* stream) {
     if ((e = pa::read_status_copy(&a, true)) != cudaSuccess ||
         (e = pa::read_status_tma(&b, true)) != cudaSuccess)
         return fail_cuda(e, "pa_sync_check: status word");
+    if ((a | b) & pa::kStatusSmemAlign)
+        return fail(PA_ERR_CUDA, "a decode kernel found its shared memory misaligned and did not run");
     if ((a | b) & pa::kStatusTimeout)
         return fail(PA_ERR_TIMEOUT, "a bounded pipeline wait gave up (bits copy=%u decode=%u)", a, b);
     if ((a | b) & pa::kStatusBadIndex)

@@ -50,13 +50,16 @@ namespace {
 #define PA_MMA_CONSUMER_WARPS 2
 #endif
 #ifndef PA_MMA_RING_BYTES
-#define PA_MMA_RING_BYTES 32768
+#define PA_MMA_RING_BYTES 49152
 #endif
 #ifndef PA_MMA_MIN_BLOCKS
 #define PA_MMA_MIN_BLOCKS 4
 #endif
 #ifndef PA_MMA_SPLIT_QK
 #define PA_MMA_SPLIT_QK 0
+#endif
+#ifndef PA_MMA_PREFETCH_Q
+#define PA_MMA_PREFETCH_Q 1
 #endif
 
 constexpr int kBoxBytes = 16 * 128;  // 16 rows x 128 bytes
@@ -179,13 +182,17 @@ __device__ __forceinline__ void drain_ring(const Ring& ring, int issued, int lan
     }
 }
 
-// Shared memory: [pad to 1024] [ring] [extra_bytes] [full bars] [empty bars] [valid]
+// Shared memory: [ring] [extra_bytes] [full bars] [empty bars] [valid]. The
+// dynamic shared memory is declared 1024-byte aligned (the 128-byte swizzle
+// repeats every 1024 bytes and the fragment addressing assumes box bases on
+// that boundary); setup_ring returns nullptr if it is not, and the kernel then
+// records kStatusSmemAlign and returns before touching shared memory.
 template <class G>
 __device__ __forceinline__ uint8_t* setup_ring(uint8_t* smem_raw, Ring& ring, int extra_bytes = 0) {
     const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
-    uint8_t* base = smem_raw + pad;
-    ring.stages = raw + pad;
+    if (raw & 1023u) return nullptr;
+    uint8_t* base = smem_raw;
+    ring.stages = raw;
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + G::kRingBytes + ((extra_bytes + 7) & ~7));
     ring.full = smem_u32(bars);
     ring.empty = smem_u32(bars + G::kStages);
@@ -202,7 +209,7 @@ __device__ __forceinline__ uint8_t* setup_ring(uint8_t* smem_raw, Ring& ring, in
 
 template <class G>
 constexpr size_t smem_bytes(int extra_bytes = 0) {
-    return 1024 + G::kRingBytes + ((extra_bytes + 7) & ~7) + 2 * G::kStages * 8 + G::kStages * 4 + 64;
+    return G::kRingBytes + ((extra_bytes + 7) & ~7) + 2 * G::kStages * 8 + G::kStages * 4 + 64;
 }
 
 __device__ __forceinline__ int clamp_ctx(int ctx, int max_ctx, bool report) {
@@ -231,7 +238,7 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
     constexpr int RPL = 32 / CPR;               // rows per warp-wide pass
     constexpr int ITER = 16 / RPL;              // passes per 16-row sub-tile
     constexpr int IPP = ITER < 8 ? ITER : 8;    // passes held in registers at once
-    extern __shared__ uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
 
     const int part = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
@@ -250,6 +257,10 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
     const int n_sub = (t1 - t0 + 15) >> 4;
     Ring ring;
     uint8_t* base = setup_ring<G>(smem_raw, ring);
+    if (base == nullptr) {
+        if (threadIdx.x == 0) atomicOr(&s_status_tma, kStatusSmemAlign);
+        return;
+    }
     __syncthreads();
 
     float m = -INFINITY, l = 0.f;
@@ -438,7 +449,12 @@ constexpr int merge_floats() {
 }
 template <int D>
 constexpr int merge_bytes() {
-    return 2 * merge_floats<D>() * 4;  // double-buffered: item k uses buffer k % 2
+    // one warp: none; two warps: warp 1's registers, in register order, for warp 0
+    // ((D/16 * 4 accumulators + m0, m1, l0, l1) x 32 lanes); more warps: a
+    // double-buffered [warps][8][D + 1] buffer (item k uses buffer k % 2)
+    return PA_MMA_CONSUMER_WARPS == 1   ? 0
+           : PA_MMA_CONSUMER_WARPS == 2 ? (D / 16 * 4 + 4) * 32 * 4
+                                        : 2 * merge_floats<D>() * 4;
 }
 
 // The work items of one persistent CTA, in order: u = blockIdx.x + k * gridDim.x,
@@ -507,7 +523,7 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
     constexpr int VCH = D / 64;  // V boxes
     constexpr int MT = D / 16;   // PV m-tiles
     constexpr int OS = D + 1;    // merge-buffer row stride (floats)
-    extern __shared__ uint8_t smem_raw[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -515,6 +531,10 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
     const int group = p.num_heads / p.num_kv_heads;
     Ring ring;
     uint8_t* base = setup_ring<G>(smem_raw, ring, merge_bytes<D>());
+    if (base == nullptr) {
+        if (threadIdx.x == 0) atomicOr(&s_status_tma, kStatusSmemAlign);
+        return;
+    }
     float* merge_buf = reinterpret_cast<float*>(base + G::kRingBytes);
     int merge_sel = 0;  // which half of the double-buffered merge area this item uses
     ItemWalk walk;
@@ -586,8 +606,10 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
     load_q(cur, qcur);
     while (cur.valid) {
         Item nxt = item_next(walk, p, num_items, lane, warp == 0, true);
+#if PA_MMA_PREFETCH_Q
         uint4 qnxt[KCH];
         load_q(nxt, qnxt);  // in flight while this item is processed
+#endif
         const int64_t head0 = (int64_t)cur.s * p.num_heads + (int64_t)cur.kh * group;
         if (cur.t0 >= cur.t1) {
             if (P == 1)
@@ -722,70 +744,156 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 l0 += __shfl_xor_sync(0xffffffffu, l0, off);
                 l1 += __shfl_xor_sync(0xffffffffu, l1, off);
             }
-            // Cross-warp merge of this item, in fixed warp order. Buffers alternate
-            // between items, so a warp that races ahead to the next item's merge
-            // cannot overwrite what a slower warp still reads here.
-            float* sm_o = merge_buf + merge_sel * merge_floats<D>();  // [warps][8][OS]
-            float* sm_m = sm_o + kConsumerWarps * kGroupMax * OS;     // [warps][8]
-            float* sm_l = sm_m + kConsumerWarps * kGroupMax;
-            float* sm_w = sm_l + kConsumerWarps * kGroupMax;          // weight / L
-            merge_sel ^= 1;
+            if constexpr (kConsumerWarps == 2) {
+                // Warp 1 hands its state to warp 0 in register order (conflict-free);
+                // warp 0 merges it into its own registers, in fixed order.
+                float* xb = merge_buf;
+                if (warp == 1) {
 #pragma unroll
-            for (int t = 0; t < MT; ++t) {
-                const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
-                float* o = sm_o + (warp * kGroupMax + 2 * c) * OS;
-                o[d0] = acc[t][0];
-                o[OS + d0] = acc[t][1];
-                o[d0 + 1] = acc[t][2];
-                o[OS + d0 + 1] = acc[t][3];
-            }
-            if (r == 0) {
-                sm_m[warp * kGroupMax + 2 * c] = m0;
-                sm_m[warp * kGroupMax + 2 * c + 1] = m1;
-                sm_l[warp * kGroupMax + 2 * c] = l0;
-                sm_l[warp * kGroupMax + 2 * c + 1] = l1;
-            }
-            named_barrier(1, kConsumerWarps * 32);
-            if (threadIdx.x < group) {  // one thread per query row: the warps' weights
-                const int n = threadIdx.x;
-                float M = -INFINITY;
+                    for (int t = 0; t < MT; ++t)
 #pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * kGroupMax + n]);
-                float wg[kConsumerWarps];
-                float L = 0.f;
-#pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float mw = sm_m[w * kGroupMax + n];
-                    wg[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
-                    L = fmaf(sm_l[w * kGroupMax + n], wg[w], L);
+                        for (int e = 0; e < 4; ++e) xb[(t * 4 + e) * 32 + lane] = acc[t][e];
+                    xb[(MT * 4 + 0) * 32 + lane] = m0;
+                    xb[(MT * 4 + 1) * 32 + lane] = m1;
+                    xb[(MT * 4 + 2) * 32 + lane] = l0;
+                    xb[(MT * 4 + 3) * 32 + lane] = l1;
                 }
+                named_barrier(1, 64);
+                if (warp == 0) {
+                    const float mb0 = xb[(MT * 4 + 0) * 32 + lane], mb1 = xb[(MT * 4 + 1) * 32 + lane];
+                    const float lb0 = xb[(MT * 4 + 2) * 32 + lane], lb1 = xb[(MT * 4 + 3) * 32 + lane];
+                    const float M0 = fmaxf(m0, mb0), M1 = fmaxf(m1, mb1);
+                    const float wa0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M0);
+                    const float wb0 = mb0 == -INFINITY ? 0.f : exp2f(mb0 - M0);
+                    const float wa1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M1);
+                    const float wb1 = mb1 == -INFINITY ? 0.f : exp2f(mb1 - M1);
 #pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w)
-                    sm_w[w * kGroupMax + n] = L > 0.f ? wg[w] / L : 0.f;
-                if (P > 1) {
-                    float* ml = p.ws_ml + ((head0 + n) * P + cur.part) * 2;
-                    ml[0] = L > 0.f ? M : -INFINITY;
-                    ml[1] = L;
+                    for (int t = 0; t < MT; ++t) {
+                        acc[t][0] = fmaf(xb[(t * 4 + 0) * 32 + lane], wb0, acc[t][0] * wa0);
+                        acc[t][1] = fmaf(xb[(t * 4 + 1) * 32 + lane], wb1, acc[t][1] * wa1);
+                        acc[t][2] = fmaf(xb[(t * 4 + 2) * 32 + lane], wb0, acc[t][2] * wa0);
+                        acc[t][3] = fmaf(xb[(t * 4 + 3) * 32 + lane], wb1, acc[t][3] * wa1);
+                    }
+                    l0 = fmaf(lb0, wb0, l0 * wa0);
+                    l1 = fmaf(lb1, wb1, l1 * wa1);
+                    m0 = M0;
+                    m1 = M1;
                 }
             }
-            named_barrier(1, kConsumerWarps * 32);
-            for (int idx = threadIdx.x; idx < group * D; idx += kConsumerWarps * 32) {
-                const int n = idx / D;
-                const int d = idx - n * D;
-                float val = 0.f;
+            if constexpr (kConsumerWarps <= 2) {
+                // One warp holds the whole item: normalise and store from registers.
+                // Thread (r, c) holds heads 2c, 2c+1 at head_dim 64*(t/4) + 8r + 2*(t%4) (+1).
+                if (warp == 0) {
+                    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f;
+                    const float inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+                    const int n0 = 2 * c, n1 = 2 * c + 1;
 #pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w)
-                    val = fmaf(sm_o[(w * kGroupMax + n) * OS + d], sm_w[w * kGroupMax + n], val);
-                const int64_t row = head0 + n;
-                if (P == 1)
-                    Elem<T>::store(p.out, row * D + d, val);
-                else
-                    p.ws_o[(row * P + cur.part) * D + d] = val;
+                    for (int t = 0; t < MT; ++t) {
+                        const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
+                        if (P == 1) {
+                            if (n0 < group)
+                                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) +
+                                                             (head0 + n0) * D + d0) =
+                                    pack_bf16x2(acc[t][0] * inv0, acc[t][2] * inv0);
+                            if (n1 < group)
+                                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) +
+                                                             (head0 + n1) * D + d0) =
+                                    pack_bf16x2(acc[t][1] * inv1, acc[t][3] * inv1);
+                        } else {
+                            if (n0 < group)
+                                *reinterpret_cast<float2*>(
+                                    p.ws_o + ((head0 + n0) * P + cur.part) * D + d0) =
+                                    make_float2(acc[t][0] * inv0, acc[t][2] * inv0);
+                            if (n1 < group)
+                                *reinterpret_cast<float2*>(
+                                    p.ws_o + ((head0 + n1) * P + cur.part) * D + d0) =
+                                    make_float2(acc[t][1] * inv1, acc[t][3] * inv1);
+                        }
+                    }
+                    if (P > 1 && r == 0) {
+                        if (n0 < group) {
+                            float* ml = p.ws_ml + ((head0 + n0) * P + cur.part) * 2;
+                            ml[0] = l0 > 0.f ? m0 : -INFINITY;
+                            ml[1] = l0;
+                        }
+                        if (n1 < group) {
+                            float* ml = p.ws_ml + ((head0 + n1) * P + cur.part) * 2;
+                            ml[0] = l1 > 0.f ? m1 : -INFINITY;
+                            ml[1] = l1;
+                        }
+                    }
+                }
+                if constexpr (kConsumerWarps == 2) named_barrier(1, 64);  // buffer free again
+            } else {
+                // Cross-warp merge of this item, in fixed warp order. Buffers alternate
+                // between items, so a warp that races ahead to the next item's merge
+                // cannot overwrite what a slower warp still reads here.
+                float* sm_o = merge_buf + merge_sel * merge_floats<D>();  // [warps][8][OS]
+                float* sm_m = sm_o + kConsumerWarps * kGroupMax * OS;     // [warps][8]
+                float* sm_l = sm_m + kConsumerWarps * kGroupMax;
+                float* sm_w = sm_l + kConsumerWarps * kGroupMax;          // weight / L
+                merge_sel ^= 1;
+    #pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
+                    float* o = sm_o + (warp * kGroupMax + 2 * c) * OS;
+                    o[d0] = acc[t][0];
+                    o[OS + d0] = acc[t][1];
+                    o[d0 + 1] = acc[t][2];
+                    o[OS + d0 + 1] = acc[t][3];
+                }
+                if (r == 0) {
+                    sm_m[warp * kGroupMax + 2 * c] = m0;
+                    sm_m[warp * kGroupMax + 2 * c + 1] = m1;
+                    sm_l[warp * kGroupMax + 2 * c] = l0;
+                    sm_l[warp * kGroupMax + 2 * c + 1] = l1;
+                }
+                named_barrier(1, kConsumerWarps * 32);
+                if (threadIdx.x < group) {  // one thread per query row: the warps' weights
+                    const int n = threadIdx.x;
+                    float M = -INFINITY;
+    #pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * kGroupMax + n]);
+                    float wg[kConsumerWarps];
+                    float L = 0.f;
+    #pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) {
+                        const float mw = sm_m[w * kGroupMax + n];
+                        wg[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
+                        L = fmaf(sm_l[w * kGroupMax + n], wg[w], L);
+                    }
+    #pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w)
+                        sm_w[w * kGroupMax + n] = L > 0.f ? wg[w] / L : 0.f;
+                    if (P > 1) {
+                        float* ml = p.ws_ml + ((head0 + n) * P + cur.part) * 2;
+                        ml[0] = L > 0.f ? M : -INFINITY;
+                        ml[1] = L;
+                    }
+                }
+                named_barrier(1, kConsumerWarps * 32);
+                for (int idx = threadIdx.x; idx < group * D; idx += kConsumerWarps * 32) {
+                    const int n = idx / D;
+                    const int d = idx - n * D;
+                    float val = 0.f;
+    #pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w)
+                        val = fmaf(sm_o[(w * kGroupMax + n) * OS + d], sm_w[w * kGroupMax + n], val);
+                    const int64_t row = head0 + n;
+                    if (P == 1)
+                        Elem<T>::store(p.out, row * D + d, val);
+                    else
+                        p.ws_o[(row * P + cur.part) * D + d] = val;
+                }
             }
         }
         cur = nxt;
+#if PA_MMA_PREFETCH_Q
 #pragma unroll
         for (int jp = 0; jp < KCH; ++jp) qcur[jp] = qnxt[jp];
+#else
+        load_q(cur, qcur);
+#endif
     }
 }
 

@@ -14,6 +14,9 @@ namespace pa {
 constexpr unsigned kStatusBadIndex = 1u;
 // Bit set when a bounded wait on a shared-memory pipeline barrier gave up.
 constexpr unsigned kStatusTimeout = 2u;
+// Bit set when a kernel found its dynamic shared memory not 1024-byte aligned
+// (it then returns without running; the outputs are not written).
+constexpr unsigned kStatusSmemAlign = 4u;
 
 // Everything one decode launch needs. Offsets are in elements unless noted.
 struct DecodeParams {

@@ -72,13 +72,13 @@ def test_decode_needs_workspace_when_split(lib):
 
 
 def test_partition_policy(lib):
-    # tensor-core GQA kernel: equal partitions of about 2048 tokens, at least one
-    # item per CTA slot (148 SMs x 4 when no GPU is visible), none under 256 tokens
+    # tensor-core GQA kernel (148 SMs x 4 CTA slots when no GPU is visible): equal
+    # partitions, the count minimising waves x (sub-tiles per item + per-item overhead)
     d70 = _desc(num_kv_heads=8)
-    assert lib.pa_decode_num_partitions(8, 64, 32768, ctypes.byref(d70), 0) == 16
-    assert lib.pa_decode_num_partitions(128, 64, 2303, ctypes.byref(d70), 0) == 2
-    assert lib.pa_decode_num_partitions(1, 64, 4096, ctypes.byref(d70), 0) == 16   # fill the GPU
-    assert lib.pa_decode_num_partitions(1, 64, 300, ctypes.byref(d70), 0) == 2     # >= 256 tokens
+    assert lib.pa_decode_num_partitions(8, 64, 32768, ctypes.byref(d70), 0) == 9     # 576 items: 1 wave
+    assert lib.pa_decode_num_partitions(128, 64, 2303, ctypes.byref(d70), 0) == 1    # 1024 items already
+    assert lib.pa_decode_num_partitions(1, 64, 4096, ctypes.byref(d70), 0) == 16     # >= 256 tokens each
+    assert lib.pa_decode_num_partitions(1, 64, 300, ctypes.byref(d70), 0) == 2
     # CUDA-core kernel: split into 512-token partitions only when units cannot fill the GPU
     d13 = _desc(num_kv_heads=40)
     assert lib.pa_decode_num_partitions(256, 40, 4096, ctypes.byref(d13), 0) == 1
