@@ -39,9 +39,16 @@ METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); seq-steps/s"
 UNIT = "GB/s"
 DEFAULT_CONFIG = "llama13b_bs16"
 # (label, workload name, partition_size override or None = the workload's own)
-EXTRA_CONFIGS = [("llama7b", "llama7b", None), ("llama13b_bs16", "llama13b_bs16", None),
-                 ("llama13b_bs32", "llama13b_bs32", None), ("llama70b_gqa", "llama70b_gqa", None),
-                 ("llama70b_gqa_policy", "llama70b_gqa", 0), ("cow_beam4", "cow_beam4", None)]
+# (label, workload, partition size (None: the workload's), sequences decoded together)
+EXTRA_CONFIGS = [("llama7b", "llama7b", None, 1), ("llama13b_bs16", "llama13b_bs16", None, 1),
+                 ("llama13b_bs32", "llama13b_bs32", None, 1),
+                 ("llama70b_gqa", "llama70b_gqa", None, 1),
+                 ("llama70b_gqa_policy", "llama70b_gqa", 0, 1), ("cow_beam4", "cow_beam4", None, 1),
+                 ("cow_beam4_grouped", "cow_beam4", 0, 4)]
+# pa_test_last_decode_kernel() -> the decode kernel a call enqueued
+KERNEL_NAMES = {0: "decode_tma_simt_kernel (CUDA-core)",
+                1: "decode_tma_mma_kernel (persistent, tensor-core GQA)",
+                2: "decode_tma_grouped_kernel (persistent, grouped sequences)"}
 FALLBACK_HBM_GBS = 6650.0
 DATASHEET_HBM_GBS = 8000.0
 L2_FLUSH_BYTES = 512 << 20          # > 2x the 126 MB L2
@@ -57,6 +64,8 @@ def parse_args():
     ap.add_argument("--config", default=DEFAULT_CONFIG)
     ap.add_argument("--partition-size", type=int, default=None,
                     help="override the workload's partition size (0 = library policy)")
+    ap.add_argument("--group-size", type=int, default=1,
+                    help="decode sequences [k g, (k+1) g) together (pa_decode_grouped) when > 1")
     ap.add_argument("--no-extra-configs", action="store_true",
                     help="skip the per-configuration table")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -228,7 +237,7 @@ def profile_traffic(kernel_file, workload):
 class Step:
     """Device-resident inputs of one workload and pre-marshalled C-ABI calls."""
 
-    def __init__(self, wl, device, seed_offset=0, partition_size=None):
+    def __init__(self, wl, device, seed_offset=0, partition_size=None, group_size=1):
         import torch
 
         import paged_kv_cache_335_b200 as pa
@@ -245,10 +254,11 @@ class Step:
         self.out = torch.empty_like(v["q"])
         self.desc = pa.cache_desc(v["k_cache"])
         self.ps = wl.partition_size if partition_size is None else partition_size
-        self.num_partitions = pa.pa_decode_num_partitions(wl.num_seqs, wl.num_heads,
-                                                          wl.max_context_len, v["k_cache"], self.ps)
-        need = pa.pa_decode_workspace_size(wl.num_seqs, wl.num_heads, wl.max_context_len,
-                                           v["k_cache"], self.ps)
+        self.group_size = group_size
+        self.num_partitions = pa.pa_decode_grouped_num_partitions(
+            wl.num_seqs, wl.num_heads, wl.max_context_len, v["k_cache"], group_size, self.ps)
+        need = pa.pa_decode_grouped_workspace_size(wl.num_seqs, wl.num_heads, wl.max_context_len,
+                                                   v["k_cache"], group_size, self.ps)
         self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
         self.ws_bytes = need
         self.stream = torch.cuda.current_stream(device)
@@ -264,8 +274,10 @@ class Step:
                             P(v["k_cache"].data_ptr()), P(v["v_cache"].data_ptr()),
                             P(self.tables.data_ptr()), int(self.tables.shape[1]),
                             P(self.ctx.data_ptr()), wl.max_context_len, wl.num_seqs,
-                            wl.num_heads, ctypes.c_float(wl.scale), ctypes.byref(self.desc),
-                            self.ps, P(self.ws.data_ptr()), ctypes.c_size_t(self.ws_bytes), self.sp)
+                            wl.num_heads, ctypes.c_float(wl.scale), ctypes.byref(self.desc)) + \
+            ((group_size,) if group_size > 1 else ()) + \
+            (self.ps, P(self.ws.data_ptr()), ctypes.c_size_t(self.ws_bytes), self.sp)
+        self.decode_fn = self.lib.pa_decode_grouped if group_size > 1 else self.lib.pa_decode
         self.has_copy = wl.copy_pairs.shape[0] > 0
         self.has_append = wl.num_tokens > 0
         self.launches_per_step = (self.num_partitions > 1) + 1 + int(self.has_append) + \
@@ -287,7 +299,7 @@ class Step:
                 raise RuntimeError(lib.pa_get_last_error().decode())
         if ev:
             ev[1].record(self.stream)
-        rc = lib.pa_decode(*self.args_decode)
+        rc = self.decode_fn(*self.args_decode)
         if rc:
             raise RuntimeError(lib.pa_get_last_error().decode())
         if ev:
@@ -497,7 +509,7 @@ def main():
     wl = W.make(args.config)
     if args.partition_size is not None:
         wl.partition_size = args.partition_size
-    step = Step(wl, device, seed_offset=rank)
+    step = Step(wl, device, seed_offset=rank, group_size=args.group_size)
 
     uuid = None
     try:
@@ -540,8 +552,11 @@ def main():
     dec_ms = statistics.mean(res["decode_ms"])
     dec_gbs = wl.decode_bytes() / (dec_ms / 1e3) / 1e9
     kernel_file = os.path.join(ROOT, "paged_kv_cache_335_b200", "csrc", "pa_decode_tma.cu")
-    gqa = wl.dtype == "bf16" and 2 <= wl.num_heads // wl.num_kv_heads <= 8
-    traffic, sha = profile_traffic(kernel_file, wl.name)
+    kernel_name = KERNEL_NAMES.get(step.lib.pa_test_last_decode_kernel(), "unknown")
+    if step.num_partitions > 1:
+        kernel_name += " + partition_reduce_kernel"
+    traffic, sha = profile_traffic(
+        kernel_file, wl.name if args.group_size == 1 else f"{wl.name}_grouped{args.group_size}")
 
     # end to end through the public binding with host buffers
     e2e_ms, h2d, d2h = e2e_steps(step, args.steps, max(3, args.warmup))
@@ -555,9 +570,9 @@ def main():
     read_gbs = stream_read_gbs(device) if world == 1 else None
     per_config = {}
     if world == 1 and not args.no_extra_configs:
-        for label, name, ps in EXTRA_CONFIGS:
+        for label, name, ps, gs in EXTRA_CONFIGS:
             w2 = W.make(name)
-            st = Step(w2, device, partition_size=ps)
+            st = Step(w2, device, partition_size=ps, group_size=gs)
             r2 = time_steps(st, min(args.steps, 50), 3, flush_buf if needs_flush(w2) else None)
             sm = statistics.median(r2["step_ms"])
             dm = statistics.median(r2["decode_ms"])
@@ -574,6 +589,7 @@ def main():
                 "seq_steps_per_s": round(w2.num_seqs / (sm / 1e3), 1),
                 "partitions": st.num_partitions,
                 "partition_size": "library policy" if st.ps == 0 else st.ps,
+                "group_size": gs,
                 "decode_bytes": w2.decode_bytes(),
                 "unique_kv_bytes": w2.unique_kv_bytes() if name.startswith("cow") else None,
             }
@@ -594,7 +610,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic (seeded N(0,1) values, seeded shapes)",
-            "config": config_dict(wl, flush is not None),
+            "config": {**config_dict(wl, flush is not None), "group_size": args.group_size},
             "seq_steps_per_s": round(world * wl.num_seqs / (ms_per_step / 1e3), 1),
             "frac_of_hbm_peak": round(value / world / hbm_peak, 4),
             "reference_bandwidths_gbs": {
@@ -604,10 +620,7 @@ def main():
             "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm_peak,
                          "unit": "GB/s", "frac": round(dec_gbs / hbm_peak, 4),
                          "traffic": traffic,
-                         "kernel": ("decode_tma_mma_kernel (persistent, tensor-core GQA)" if gqa
-                                    else "decode_tma_simt_kernel (CUDA-core)")
-                                   + (" + partition_reduce_kernel" if step_partitions(wl) > 1
-                                      else ""),
+                         "kernel": kernel_name,
                          "algorithmic_bytes_per_launch": wl.decode_bytes(),
                          "avg_launch_us": round(dec_ms * 1e3, 2),
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"
@@ -625,15 +638,6 @@ def main():
         dist.barrier()
         dist.destroy_process_group()
     return 0
-
-
-def step_partitions(wl):
-    import paged_kv_cache_335_b200 as pa
-    lib = pa.load_library()
-    desc = pa.pa_cache_desc(wl.num_blocks, wl.num_kv_heads, wl.block_size, wl.head_dim,
-                            pa.PA_F32 if wl.dtype == "f32" else pa.PA_BF16)
-    return lib.pa_decode_num_partitions(wl.num_seqs, wl.num_heads, wl.max_context_len,
-                                        ctypes.byref(desc), wl.partition_size)
 
 
 if __name__ == "__main__":

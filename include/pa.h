@@ -8,6 +8,9 @@
  *                  table gathers from fixed-size physical blocks
  *   pa_block_copy  copy whole physical blocks (copy-on-write at a fork)
  *
+ * and pa_decode_grouped, pa_decode for groups of sequences that share blocks
+ * (beams, parallel samples), which reads each shared block once per group.
+ *
  * Sources for what each call computes (page title, section):
  *   [P1] "PagedAttention：大模型推理性能优化的核心技术解析" (bmjup.com),
  *        § "PagedAttention 的核心工作机制与创新" (1 页表式管理, 2 写入时拷贝).
@@ -179,6 +182,52 @@ int pa_decode_num_partitions(int32_t num_seqs, int32_t num_heads,
                              int32_t max_context_len,
                              const pa_cache_desc* cache,
                              int32_t partition_size);
+
+/*
+ * pa_decode_grouped — pa_decode for batches whose sequences come in groups
+ * that share blocks: the beams of a beam search or the parallel samples of
+ * one prompt, which after a fork hold the prompt's blocks through reference
+ * counts ([P2 § Copy-on-Write、并行采样与 Prefix Caching 不是同一件事]: several
+ * logical sequences point at one physical block; [P3 § PagedAttention的三大
+ * 核心优势], point 2 and the beam-search paragraph).
+ *
+ * Computes exactly what pa_decode computes, for every sequence and head, with
+ * the same arguments and conventions. Sequences k*group_size ..
+ * (k+1)*group_size - 1 form group k (the last group may be shorter); the
+ * sequences of a group are decoded together, so a block that several of them
+ * reference, at the same logical position, is read from memory once for all
+ * of them. Grouping never changes a result: any sequences may be grouped,
+ * sharing or not, and each sequence's output is bit-identical to the one it
+ * gets when its blocks are private copies (for the same group_size and
+ * partitioning). The result can differ from pa_decode's in the last bits
+ * (another summation order), within the same tolerance of the exact value.
+ *
+ *   group_size    1 .. 8. The grouped kernel runs for bf16, head_dim 64/128
+ *                 and group_size * (num_heads / num_kv_heads) <= 64; other
+ *                 calls, and group_size 1, run pa_decode's kernels.
+ *   workspace     at least pa_decode_grouped_workspace_size(...) bytes with
+ *                 the same arguments.
+ * Returns PA_ERR_INVALID_ARG for group_size outside [1, 8] or a
+ * max_context_len above 2^27 on the grouped kernel.
+ */
+int pa_decode_grouped(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, int32_t block_table_stride,
+                      const int32_t* context_lens, int32_t max_context_len,
+                      int32_t num_seqs, int32_t num_heads, float scale,
+                      const pa_cache_desc* cache, int32_t group_size,
+                      int32_t partition_size, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* Workspace bytes and partition count of pa_decode_grouped (see
+ * pa_decode_workspace_size / pa_decode_num_partitions). */
+size_t pa_decode_grouped_workspace_size(int32_t num_seqs, int32_t num_heads,
+                                        int32_t max_context_len,
+                                        const pa_cache_desc* cache, int32_t group_size,
+                                        int32_t partition_size);
+int pa_decode_grouped_num_partitions(int32_t num_seqs, int32_t num_heads,
+                                     int32_t max_context_len,
+                                     const pa_cache_desc* cache, int32_t group_size,
+                                     int32_t partition_size);
 
 /*
  * pa_block_copy — copy whole physical blocks, the copy-on-write step that

@@ -9,7 +9,16 @@
  * returns PA_ERR_TIMEOUT; the CUDA context stays usable. -1 restores normal
  * operation. It exists only so that the timeout path can be tested without a
  * fault or a hang.
+ *
+ * pa_test_last_decode_kernel — which decode kernel the calling thread's last
+ * successful pa_decode / pa_decode_grouped / pa_decode_noalloc enqueued:
+ * PA_KERNEL_SIMT (CUDA-core consumer), PA_KERNEL_MMA (tensor-core GQA
+ * consumer), PA_KERNEL_GROUPED (grouped sequences), or -1 if none yet. Lets
+ * tests confirm which path a shape takes.
  */
+#define PA_KERNEL_SIMT 0
+#define PA_KERNEL_MMA 1
+#define PA_KERNEL_GROUPED 2
 #ifndef PA_TEST_H
 #define PA_TEST_H
 
@@ -20,6 +29,7 @@ extern "C" {
 #endif
 
 void pa_test_skip_load(int32_t position);
+int pa_test_last_decode_kernel(void);
 
 #ifdef __cplusplus
 }

@@ -38,6 +38,9 @@ PA_ERR_TIMEOUT = -8
 PA_F32 = 0
 PA_BF16 = 1
 PA_NOALLOC_SCRATCH_BYTES = 32 << 20
+PA_KERNEL_SIMT = 0          # pa_test_last_decode_kernel() values
+PA_KERNEL_MMA = 1
+PA_KERNEL_GROUPED = 2
 
 _lock = threading.Lock()
 _lib = None
@@ -86,11 +89,17 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_decode_workspace_size.argtypes = [i32, i32, i32, desc, i32]
         lib.pa_decode_workspace_size.restype = sz
         lib.pa_decode_num_partitions.argtypes = [i32, i32, i32, desc, i32]
+        lib.pa_decode_grouped.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, desc,
+                                          i32, i32, vp, sz, vp]
+        lib.pa_decode_grouped_workspace_size.argtypes = [i32, i32, i32, desc, i32, i32]
+        lib.pa_decode_grouped_workspace_size.restype = sz
+        lib.pa_decode_grouped_num_partitions.argtypes = [i32, i32, i32, desc, i32, i32]
         lib.pa_block_copy.argtypes = [vp, i32, vp, vp, desc, vp]
         lib.pa_sync_check.argtypes = [vp]
         lib.pa_stream_read.argtypes = [vp, sz, vp, i32, vp]
         lib.pa_test_skip_load.argtypes = [i32]
         lib.pa_test_skip_load.restype = None
+        lib.pa_test_last_decode_kernel.argtypes = []
         lib.pa_stream_read.restype = ctypes.c_int
         lib.pa_get_last_error.argtypes = []
         lib.pa_get_last_error.restype = ctypes.c_char_p
@@ -202,37 +211,55 @@ def pa_block_copy(src_dst_pairs, k_cache, v_cache, stream=None) -> None:
 
 def pa_decode_workspace_size(num_seqs: int, num_heads: int, max_context_len: int, k_cache,
                              partition_size: int = 0) -> int:
+    return pa_decode_grouped_workspace_size(num_seqs, num_heads, max_context_len, k_cache, 1,
+                                            partition_size)
+
+
+def pa_decode_num_partitions(num_seqs: int, num_heads: int, max_context_len: int, k_cache,
+                             partition_size: int = 0) -> int:
+    return pa_decode_grouped_num_partitions(num_seqs, num_heads, max_context_len, k_cache, 1,
+                                            partition_size)
+
+
+def pa_decode_grouped_workspace_size(num_seqs: int, num_heads: int, max_context_len: int,
+                                     k_cache, group_size: int, partition_size: int = 0) -> int:
+    lib = load_library()
     desc = cache_desc(k_cache)
-    n = load_library().pa_decode_workspace_size(num_seqs, num_heads, max_context_len,
-                                                ctypes.byref(desc), partition_size)
+    if group_size == 1:
+        n = lib.pa_decode_workspace_size(num_seqs, num_heads, max_context_len,
+                                         ctypes.byref(desc), partition_size)
+    else:
+        n = lib.pa_decode_grouped_workspace_size(num_seqs, num_heads, max_context_len,
+                                                 ctypes.byref(desc), group_size, partition_size)
     if n == 0:
-        msg = load_library().pa_get_last_error().decode()
-        rc = load_library().pa_decode_num_partitions(num_seqs, num_heads, max_context_len,
-                                                     ctypes.byref(desc), partition_size)
+        msg = lib.pa_get_last_error().decode()
+        rc = _num_partitions(num_seqs, num_heads, max_context_len, desc, group_size,
+                             partition_size)
         if rc < 0:
             raise PAError(rc, msg)
     return int(n)
 
 
-def pa_decode_num_partitions(num_seqs: int, num_heads: int, max_context_len: int, k_cache,
-                             partition_size: int = 0) -> int:
-    desc = cache_desc(k_cache)
-    rc = load_library().pa_decode_num_partitions(num_seqs, num_heads, max_context_len,
-                                                 ctypes.byref(desc), partition_size)
+def _num_partitions(num_seqs, num_heads, max_context_len, desc, group_size, partition_size):
+    lib = load_library()
+    if group_size == 1:
+        return lib.pa_decode_num_partitions(num_seqs, num_heads, max_context_len,
+                                            ctypes.byref(desc), partition_size)
+    return lib.pa_decode_grouped_num_partitions(num_seqs, num_heads, max_context_len,
+                                                ctypes.byref(desc), group_size, partition_size)
+
+
+def pa_decode_grouped_num_partitions(num_seqs: int, num_heads: int, max_context_len: int,
+                                     k_cache, group_size: int, partition_size: int = 0) -> int:
+    rc = _num_partitions(num_seqs, num_heads, max_context_len, cache_desc(k_cache), group_size,
+                         partition_size)
     if rc < 0:
         _check(rc)
     return rc
 
 
-def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
-              max_context_len: int | None = None, partition_size: int = 0, workspace=None,
-              stream=None) -> None:
-    """out[s][h] = softmax(scale q[s][h] . K) V over the context_lens[s] paged tokens.
-
-    ``max_context_len`` is a host bound on context_lens (computed with a device
-    sync if omitted). ``workspace``: a CUDA uint8 tensor of at least
-    ``pa_decode_workspace_size`` bytes (allocated here if omitted and needed).
-    """
+def _decode_call(entry, extra, out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                 max_context_len, group_size, partition_size, workspace, stream):
     torch = _torch()
     _same_pool(k_cache, v_cache)
     desc = cache_desc(k_cache)
@@ -245,19 +272,46 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float
         raise ValueError("block_tables must be [num_seqs][stride], context_lens [num_seqs]")
     if max_context_len is None:
         max_context_len = int(context_lens.max().item()) if s else 0
-    lib = load_library()
-    need = pa_decode_workspace_size(s, h, max_context_len, k_cache, partition_size)
+    need = pa_decode_grouped_workspace_size(s, h, max_context_len, k_cache, group_size,
+                                            partition_size)
     ws_ptr, ws_bytes = ctypes.c_void_p(0), 0
     if need:
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
-    _check(lib.pa_decode(
+    _check(entry(
         _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
         _dev(block_tables, "block_tables", torch.int32), int(block_tables.shape[1]),
         _dev(context_lens, "context_lens", torch.int32), int(max_context_len), s, h,
-        float(scale), ctypes.byref(desc), int(partition_size), ws_ptr, ws_bytes,
+        float(scale), ctypes.byref(desc), *extra, int(partition_size), ws_ptr, ws_bytes,
         _stream(stream)))
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+              max_context_len: int | None = None, partition_size: int = 0, workspace=None,
+              stream=None) -> None:
+    """out[s][h] = softmax(scale q[s][h] . K) V over the context_lens[s] paged tokens.
+
+    ``max_context_len`` is a host bound on context_lens (computed with a device
+    sync if omitted). ``workspace``: a CUDA uint8 tensor of at least
+    ``pa_decode_workspace_size`` bytes (allocated here if omitted and needed).
+    """
+    _decode_call(load_library().pa_decode, (), out, q, k_cache, v_cache, block_tables,
+                 context_lens, scale, max_context_len, 1, partition_size, workspace, stream)
+
+
+def pa_decode_grouped(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                      group_size: int, max_context_len: int | None = None,
+                      partition_size: int = 0, workspace=None, stream=None) -> None:
+    """pa_decode with sequences [k group_size, (k + 1) group_size) decoded together,
+    so blocks they share (beams, parallel samples of one prompt) are read once.
+
+    Same result contract as ``pa_decode``; ``workspace`` is sized by
+    ``pa_decode_grouped_workspace_size``.
+    """
+    _decode_call(load_library().pa_decode_grouped, (int(group_size),), out, q, k_cache, v_cache,
+                 block_tables, context_lens, scale, max_context_len, int(group_size),
+                 partition_size, workspace, stream)
 
 
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
@@ -290,5 +344,6 @@ def pa_sync_check(stream=None) -> None:
 
 
 __all__ = ["pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_block_copy", "pa_decode_workspace_size",
-           "pa_decode_num_partitions", "pa_sync_check", "pa_cache_desc", "cache_desc",
+           "pa_decode_num_partitions", "pa_decode_grouped", "pa_decode_grouped_workspace_size",
+           "pa_decode_grouped_num_partitions", "pa_sync_check", "pa_cache_desc", "cache_desc",
            "load_library", "header_functions", "PAError"]

@@ -19,6 +19,7 @@
 namespace {
 
 thread_local std::string t_last_error;
+thread_local int t_last_kernel = -1;  // PA_KERNEL_* of the last decode enqueued here
 int g_test_skip_position = -1;  // set only by pa_test_skip_load
 
 int fail(int code, const char* fmt, ...) {
@@ -130,6 +131,7 @@ constexpr int kMinPartition = 256;       // tensor-core kernel: smallest partiti
 
 struct Plan {
     bool use_mma;
+    bool grouped;       // the grouped kernel (group_size > 1 and supported)
     int partition_size;
     int num_partitions;
     size_t ws_bytes;
@@ -141,7 +143,7 @@ int round_up16(int x) { return (x + 15) / 16 * 16; }
 // Partition policy: split the context only when the (sequence, head) work
 // units alone cannot fill the GPU, then into 512-token partitions.
 int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_cache_desc* c,
-                int32_t partition_size, Plan* plan) {
+                int32_t partition_size, Plan* plan, int32_t group_size = 1) {
     int rc = check_cache(c);
     if (rc != PA_OK) return rc;
     if (num_seqs < 0 || num_seqs > 65535)
@@ -151,6 +153,11 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
                     "num_kv_heads %d", num_heads, c->num_kv_heads);
     if (max_ctx < 0) return fail(PA_ERR_INVALID_ARG, "max_context_len %d is negative", max_ctx);
     const int group = num_heads / c->num_kv_heads;
+    if (group_size < 1 || group_size > 8)
+        return fail(PA_ERR_INVALID_ARG, "group_size %d outside [1, 8]", group_size);
+    plan->grouped = group_size > 1 && pa::grouped_supported(c->dtype, c->head_dim, group, group_size);
+    if (plan->grouped && max_ctx > (1 << 27))
+        return fail(PA_ERR_INVALID_ARG, "max_context_len %d above 2^27 on the grouped kernel", max_ctx);
     plan->use_mma = pa::mma_supported(c->dtype, c->head_dim, group);
     const int whole = round_up16(max_ctx > 16 ? max_ctx : 16);
     int ps = whole, np = 1;
@@ -165,15 +172,20 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
             return fail(PA_ERR_INVALID_ARG, "partition_size %d gives %d partitions (max %d)",
                         partition_size, np, kMaxPartitions);
     } else if (partition_size == 0) {
-        if (plan->use_mma) {
+        if (plan->use_mma || plan->grouped) {
             // The persistent tensor-core kernel hands items to its CTA slots statically
             // (item u to CTA u mod slots), so its time is about
             //   waves * (sub-tiles per item + per-item overhead),  waves = ceil(items / slots),
             // the overhead being the item's merge, partial write and share of the reduce.
             // Pick the partition count with the smallest such cost (ties: fewer partitions),
             // partitions cut equal and at least kMinPartition tokens long.
-            const long units = (long)num_seqs * c->num_kv_heads;
-            const long slots = (long)sm_count() * pa::mma_ctas_per_sm();
+            // The grouped kernel is persistent the same way; its unit is a group.
+            const long units = plan->grouped
+                                   ? (long)((num_seqs + group_size - 1) / group_size) * c->num_kv_heads
+                                   : (long)num_seqs * c->num_kv_heads;
+            const long slots =
+                (long)sm_count() * (plan->grouped ? pa::grouped_ctas_per_sm(c->head_dim, group_size, group)
+                                                  : pa::mma_ctas_per_sm());
             long most = (max_ctx + kMinPartition - 1) / kMinPartition;
             if (most > kMaxPartitions) most = kMaxPartitions;
             if (most < 1) most = 1;
@@ -239,6 +251,76 @@ int pa::report_error(int code, const char* fmt, ...) {
     return code;
 }
 
+static int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* block_tables, int32_t block_table_stride,
+                       const int32_t* context_lens, int32_t max_context_len, int32_t num_seqs,
+                       int32_t num_heads, float scale, const pa_cache_desc* cache,
+                       int32_t group_size, int32_t partition_size, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    Plan plan;
+    int rc = plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan,
+                         group_size);
+    if (rc != PA_OK) return rc;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode: NULL pointer argument");
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_ALIGN, "pa_decode: out, q and the caches must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(block_tables) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(context_lens) & 3u) != 0)
+        return fail(PA_ERR_ALIGN, "pa_decode: block_tables / context_lens must be 4-byte aligned");
+    if (block_table_stride < 0 ||
+        (int64_t)block_table_stride * cache->block_size < (int64_t)max_context_len)
+        return fail(PA_ERR_INVALID_ARG, "max_context_len %d exceeds block_table_stride %d * "
+                    "block_size %d", max_context_len, block_table_stride, cache->block_size);
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    if (plan.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < plan.ws_bytes)
+            return fail(PA_ERR_WORKSPACE, "pa_decode needs %zu workspace bytes, got %zu at %p",
+                        plan.ws_bytes, workspace_bytes, workspace);
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+            return fail(PA_ERR_ALIGN, "pa_decode: workspace must be 256-byte aligned");
+    }
+    pa::DecodeParams p;
+    p.out = out;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.ws_o = plan.ws_bytes ? static_cast<float*>(workspace) : nullptr;
+    p.ws_ml = plan.ws_bytes
+                  ? reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.ws_ml_offset)
+                  : nullptr;
+    p.table_stride = block_table_stride;
+    p.max_context_len = max_context_len;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = cache->num_kv_heads;
+    p.num_blocks = cache->num_blocks;
+    p.block_size = cache->block_size;
+    p.log2_block_size = ilog2_exact(cache->block_size);
+    p.partition_size = plan.partition_size;
+    p.num_partitions = plan.num_partitions;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.test_skip_position = g_test_skip_position;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CUtensorMap kmap, vmap;
+    if ((rc = make_cache_map(&kmap, k_cache, cache)) != PA_OK) return rc;
+    if ((rc = make_cache_map(&vmap, v_cache, cache)) != PA_OK) return rc;
+    cudaError_t e =
+        plan.grouped
+            ? pa::launch_decode_grouped(p, cache->head_dim, group_size, kmap, vmap, st)
+            : pa::launch_decode_tma(p, cache->dtype, cache->head_dim, plan.use_mma, kmap, vmap, st);
+    if (e != cudaSuccess) return fail_cuda(e, "pa_decode launch");
+    t_last_kernel = plan.grouped ? PA_KERNEL_GROUPED : plan.use_mma ? PA_KERNEL_MMA : PA_KERNEL_SIMT;
+    if (plan.num_partitions > 1) {
+        e = pa::launch_partition_reduce(p, cache->dtype, cache->head_dim, st);
+        if (e != cudaSuccess) return fail_cuda(e, "pa_decode reduce launch");
+    }
+    return PA_OK;
+}
+
 extern "C" {
 
 int pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
@@ -295,64 +377,39 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
               const int32_t* context_lens, int32_t max_context_len, int32_t num_seqs,
               int32_t num_heads, float scale, const pa_cache_desc* cache,
               int32_t partition_size, void* workspace, size_t workspace_bytes, void* stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_tables, block_table_stride, context_lens,
+                       max_context_len, num_seqs, num_heads, scale, cache, 1, partition_size,
+                       workspace, workspace_bytes, stream);
+}
+
+int pa_decode_grouped(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, int32_t block_table_stride,
+                      const int32_t* context_lens, int32_t max_context_len, int32_t num_seqs,
+                      int32_t num_heads, float scale, const pa_cache_desc* cache,
+                      int32_t group_size, int32_t partition_size, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_tables, block_table_stride, context_lens,
+                       max_context_len, num_seqs, num_heads, scale, cache, group_size,
+                       partition_size, workspace, workspace_bytes, stream);
+}
+
+size_t pa_decode_grouped_workspace_size(int32_t num_seqs, int32_t num_heads,
+                                        int32_t max_context_len, const pa_cache_desc* cache,
+                                        int32_t group_size, int32_t partition_size) {
     Plan plan;
-    int rc = plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan);
-    if (rc != PA_OK) return rc;
-    if (num_seqs == 0) return PA_OK;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
-        return fail(PA_ERR_INVALID_ARG, "pa_decode: NULL pointer argument");
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-        return fail(PA_ERR_ALIGN, "pa_decode: out, q and the caches must be 16-byte aligned");
-    if ((reinterpret_cast<uintptr_t>(block_tables) & 3u) != 0 ||
-        (reinterpret_cast<uintptr_t>(context_lens) & 3u) != 0)
-        return fail(PA_ERR_ALIGN, "pa_decode: block_tables / context_lens must be 4-byte aligned");
-    if (block_table_stride < 0 ||
-        (int64_t)block_table_stride * cache->block_size < (int64_t)max_context_len)
-        return fail(PA_ERR_INVALID_ARG, "max_context_len %d exceeds block_table_stride %d * "
-                    "block_size %d", max_context_len, block_table_stride, cache->block_size);
-    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
-    if (plan.ws_bytes > 0) {
-        if (!workspace || workspace_bytes < plan.ws_bytes)
-            return fail(PA_ERR_WORKSPACE, "pa_decode needs %zu workspace bytes, got %zu at %p",
-                        plan.ws_bytes, workspace_bytes, workspace);
-        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-            return fail(PA_ERR_ALIGN, "pa_decode: workspace must be 256-byte aligned");
-    }
-    pa::DecodeParams p;
-    p.out = out;
-    p.q = q;
-    p.k_cache = k_cache;
-    p.v_cache = v_cache;
-    p.block_tables = block_tables;
-    p.context_lens = context_lens;
-    p.ws_o = plan.ws_bytes ? static_cast<float*>(workspace) : nullptr;
-    p.ws_ml = plan.ws_bytes
-                  ? reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.ws_ml_offset)
-                  : nullptr;
-    p.table_stride = block_table_stride;
-    p.max_context_len = max_context_len;
-    p.num_seqs = num_seqs;
-    p.num_heads = num_heads;
-    p.num_kv_heads = cache->num_kv_heads;
-    p.num_blocks = cache->num_blocks;
-    p.block_size = cache->block_size;
-    p.log2_block_size = ilog2_exact(cache->block_size);
-    p.partition_size = plan.partition_size;
-    p.num_partitions = plan.num_partitions;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.test_skip_position = g_test_skip_position;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    CUtensorMap kmap, vmap;
-    if ((rc = make_cache_map(&kmap, k_cache, cache)) != PA_OK) return rc;
-    if ((rc = make_cache_map(&vmap, v_cache, cache)) != PA_OK) return rc;
-    cudaError_t e =
-        pa::launch_decode_tma(p, cache->dtype, cache->head_dim, plan.use_mma, kmap, vmap, st);
-    if (e != cudaSuccess) return fail_cuda(e, "pa_decode launch");
-    if (plan.num_partitions > 1) {
-        e = pa::launch_partition_reduce(p, cache->dtype, cache->head_dim, st);
-        if (e != cudaSuccess) return fail_cuda(e, "pa_decode reduce launch");
-    }
-    return PA_OK;
+    if (plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan,
+                    group_size) != PA_OK)
+        return 0;
+    return plan.ws_bytes;
+}
+
+int pa_decode_grouped_num_partitions(int32_t num_seqs, int32_t num_heads,
+                                     int32_t max_context_len, const pa_cache_desc* cache,
+                                     int32_t group_size, int32_t partition_size) {
+    Plan plan;
+    int rc = plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan,
+                         group_size);
+    return rc != PA_OK ? rc : plan.num_partitions;
 }
 
 int pa_sync_check(void* stream) {
@@ -375,6 +432,8 @@ int pa_sync_check(void* stream) {
 const char* pa_get_last_error(void) { return t_last_error.c_str(); }
 
 void pa_test_skip_load(int32_t position) { g_test_skip_position = position < 0 ? -1 : position; }
+
+int pa_test_last_decode_kernel(void) { return t_last_kernel; }
 
 const char* pa_status_string(int status) {
     switch (status) {

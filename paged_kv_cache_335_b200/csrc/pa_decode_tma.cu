@@ -97,11 +97,13 @@ struct Ring {
 // Issue of one sub-tile by one producer lane: wait until its stage is free,
 // then load K and V rows [row, row + 16) of kv head `kh` into it (or, for a
 // block id outside the pool, mark the stage empty-handed and complete it).
-// Returns false if the wait timed out (nothing was issued).
+// A stage may carry a header word (`hdr`, one per stage), written before the
+// stage is completed. Returns false if the wait timed out (nothing was issued).
 template <class G>
 __device__ __forceinline__ bool issue_subtile(const CUtensorMap* kmap, const CUtensorMap* vmap,
                                               const DecodeParams& p, const Ring& ring, int gi,
-                                              int phys, int kh, int tok0) {
+                                              int phys, int kh, int tok0,
+                                              uint32_t* hdr = nullptr, uint32_t hval = 0) {
     const int st = gi % G::kStages;
     const uint32_t round = (uint32_t)(gi / G::kStages);
     if (!mbar_wait_bounded(ring.empty + 8 * st, (round & 1u) ^ 1u)) {
@@ -109,6 +111,7 @@ __device__ __forceinline__ bool issue_subtile(const CUtensorMap* kmap, const CUt
         return false;
     }
     if (gi == p.test_skip_position) return true;  // test hook: leave this stage unloaded
+    if (hdr != nullptr) hdr[st] = hval;
     if ((unsigned)phys < (unsigned)p.num_blocks) {
         ring.valid[st] = 1;
         const uint32_t full = ring.full + 8 * st;
@@ -187,8 +190,11 @@ __device__ __forceinline__ void drain_ring(const Ring& ring, int issued, int lan
 // repeats every 1024 bytes and the fragment addressing assumes box bases on
 // that boundary); setup_ring returns nullptr if it is not, and the kernel then
 // records kStatusSmemAlign and returns before touching shared memory.
+// `releases`: arrivals that free a stage (the consumer warps that read every
+// stage; 1 when each stage has a single reader).
 template <class G>
-__device__ __forceinline__ uint8_t* setup_ring(uint8_t* smem_raw, Ring& ring, int extra_bytes = 0) {
+__device__ __forceinline__ uint8_t* setup_ring(uint8_t* smem_raw, Ring& ring, int extra_bytes = 0,
+                                               int releases = 1) {
     const uint32_t raw = smem_u32(smem_raw);
     if (raw & 1023u) return nullptr;
     uint8_t* base = smem_raw;
@@ -200,7 +206,7 @@ __device__ __forceinline__ uint8_t* setup_ring(uint8_t* smem_raw, Ring& ring, in
     if (threadIdx.x == 0) {
         for (int st = 0; st < G::kStages; ++st) {
             mbar_init(ring.full + 8 * st, 1);
-            mbar_init(ring.empty + 8 * st, 1);
+            mbar_init(ring.empty + 8 * st, releases);
         }
         fence_barrier_init();
     }
@@ -439,6 +445,170 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
 // Merge buffer of the tensor-core consumer: per warp and query row, the
 // running max, sum and head_dim accumulators (rows padded to D + 1 floats so
 // the fragment stores hit at most two banks per word).
+// ---------------------------------------------------------------------------
+// The tensor-core step on one 16-token sub-tile in shared memory (shared by the
+// grouped and ungrouped GQA kernels). Thread (r, c) = (lane / 4, lane % 4).
+// ---------------------------------------------------------------------------
+
+// S^T[16 tokens][8 heads] = K . Q^T. For chunk step jp (k-steps 2jp, 2jp+1) the
+// thread reads 16-byte chunk x = 2c + (jp & 1) of box jp / 2 of rows r and r+8;
+// q holds the same head_dim positions of query row r.
+template <int D>
+__device__ __forceinline__ void mma_qk(uint32_t kb, const uint4 (&q)[D / 32], int r, int c,
+                                       float (&sc)[4]) {
+    constexpr int KCH = D / 32;
+    sc[0] = sc[1] = sc[2] = sc[3] = 0.f;
+    uint4 kr[2][KCH];
+#pragma unroll
+    for (int jp = 0; jp < KCH; ++jp) {
+        const uint32_t bx = kb + (jp >> 1) * kBoxBytes;
+        const uint32_t x = (uint32_t)(2 * c + (jp & 1));
+        kr[0][jp] = lds128(bx + swz(r, x));
+        kr[1][jp] = lds128(bx + swz(r + 8, x));
+    }
+#if PA_MMA_SPLIT_QK
+    float sd[4] = {0.f, 0.f, 0.f, 0.f};  // second chain: shorter MMA dependency
+#pragma unroll
+    for (int jp = 0; jp < KCH; ++jp) {
+        mma_16816(sc, kr[0][jp].x, kr[1][jp].x, kr[0][jp].y, kr[1][jp].y, q[jp].x, q[jp].y);
+        mma_16816(sd, kr[0][jp].z, kr[1][jp].z, kr[0][jp].w, kr[1][jp].w, q[jp].z, q[jp].w);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sc[e] += sd[e];
+#else
+#pragma unroll
+    for (int jp = 0; jp < KCH; ++jp) {
+        mma_16816(sc, kr[0][jp].x, kr[1][jp].x, kr[0][jp].y, kr[1][jp].y, q[jp].x, q[jp].y);
+        mma_16816(sc, kr[0][jp].z, kr[1][jp].z, kr[0][jp].w, kr[1][jp].w, q[jp].z, q[jp].w);
+    }
+#endif
+}
+
+// V fragments: tokens 2c, 2c+1, 2c+8, 2c+9; 16-byte chunk r of each box.
+template <int D>
+__device__ __forceinline__ void mma_load_v(uint32_t vb, int r, int c, uint4 (&vr)[4][D / 64]) {
+#pragma unroll
+    for (int hh = 0; hh < D / 64; ++hh) {
+        const uint32_t bx = vb + hh * kBoxBytes;
+        vr[0][hh] = lds128(bx + swz(2 * c, r));
+        vr[1][hh] = lds128(bx + swz(2 * c + 1, r));
+        vr[2][hh] = lds128(bx + swz(2 * c + 8, r));
+        vr[3][hh] = lds128(bx + swz(2 * c + 9, r));
+    }
+}
+
+// Online-softmax update with the sub-tile's scores and O^T += V^T . P^T.
+// nvalid = tokens of the sub-tile inside the context (>= 1). State: acc = O^T
+// fragments (rows head_dim 64*(t/4) + 8r + 2*(t%4) (+1), cols heads 2c, 2c+1),
+// m0/m1 running max (log2 units), l0/l1 this thread's share of the sums.
+template <int D>
+__device__ __forceinline__ void mma_softmax_pv(const float (&sc)[4], uint4 (&vr)[4][D / 64],
+                                               int nvalid, float scale_log2, int r, int c,
+                                               float (&acc)[D / 16][4], float& m0, float& m1,
+                                               float& l0, float& l1) {
+    constexpr int VCH = D / 64;
+    constexpr int MT = D / 16;
+    const bool lo_ok = r < nvalid, hi_ok = r + 8 < nvalid;
+    const float s0 = lo_ok ? sc[0] * scale_log2 : -INFINITY;  // token r,   head 2c
+    const float s1 = lo_ok ? sc[1] * scale_log2 : -INFINITY;  // token r,   head 2c+1
+    const float s2 = hi_ok ? sc[2] * scale_log2 : -INFINITY;  // token r+8, head 2c
+    const float s3 = hi_ok ? sc[3] * scale_log2 : -INFINITY;  // token r+8, head 2c+1
+    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    // The accumulator is rescaled only when some running max moved; a factor of
+    // exactly 1 would leave every bit unchanged anyway.
+    const bool moved = __any_sync(0xffffffffu, mn0 != m0 || mn1 != m1);
+    const float al0 = moved ? exp2f(m0 - mn0) : 1.f;
+    const float al1 = moved ? exp2f(m1 - mn1) : 1.f;
+    const uint32_t x0 = pack_bf16x2(exp2f(s0 - mn0), exp2f(s1 - mn1));
+    const uint32_t x1 = pack_bf16x2(exp2f(s2 - mn0), exp2f(s3 - mn1));
+    // the sums use the same rounded weights the PV product sees
+    l0 = fmaf(l0, al0, bf16_lo(x0) + bf16_lo(x1));
+    l1 = fmaf(l1, al1, bf16_hi(x0) + bf16_hi(x1));
+    m0 = mn0;
+    m1 = mn1;
+    if (moved) {
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+            acc[t][0] *= al0;
+            acc[t][1] *= al1;
+            acc[t][2] *= al0;
+            acc[t][3] *= al1;
+        }
+    }
+    const uint32_t pb0 = movmatrix_trans(x0);  // P^T rows (tokens) 2c, 2c+1; col head r
+    const uint32_t pb1 = movmatrix_trans(x1);  // tokens 2c+8, 2c+9
+    if (nvalid < 16) {  // slots past the context may hold anything, even NaN
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        const int tv0 = 2 * c, tv1 = 2 * c + 1, tv2 = 2 * c + 8, tv3 = 2 * c + 9;
+#pragma unroll
+        for (int hh = 0; hh < VCH; ++hh) {
+            if (tv0 >= nvalid) vr[0][hh] = z;
+            if (tv1 >= nvalid) vr[1][hh] = z;
+            if (tv2 >= nvalid) vr[2][hh] = z;
+            if (tv3 >= nvalid) vr[3][hh] = z;
+        }
+    }
+    // O^T += V^T . P^T ; m-tile t covers head_dim 64*(t/4) + 8r + 2*(t%4) (+1 for row r+8)
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+        const int hh = t >> 2, w = t & 3;
+        const uint32_t xa = word(vr[0][hh], w), xb = word(vr[1][hh], w);
+        const uint32_t ya = word(vr[2][hh], w), yb = word(vr[3][hh], w);
+        mma_16816(acc[t], __byte_perm(xa, xb, 0x5410), __byte_perm(xa, xb, 0x7632),
+                  __byte_perm(ya, yb, 0x5410), __byte_perm(ya, yb, 0x7632), pb0, pb1);
+    }
+}
+
+// Store one warp's item result (heads 2c, 2c+1 of query rows head0 + n) from its
+// registers: bf16 output when P == 1, else the normalised partial and (m, l).
+template <int D>
+__device__ __forceinline__ void mma_store_item(const DecodeParams& p, int64_t head0, int group,
+                                               int part, int r, int c, const float (&acc)[D / 16][4],
+                                               float m0, float m1, float l0, float l1) {
+    constexpr int MT = D / 16;
+    const int P = p.num_partitions;
+    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f;
+    const float inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    const int n0 = 2 * c, n1 = 2 * c + 1;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+        const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
+        if (P == 1) {
+            if (n0 < group)
+                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + (head0 + n0) * D + d0) =
+                    pack_bf16x2(acc[t][0] * inv0, acc[t][2] * inv0);
+            if (n1 < group)
+                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + (head0 + n1) * D + d0) =
+                    pack_bf16x2(acc[t][1] * inv1, acc[t][3] * inv1);
+        } else {
+            if (n0 < group)
+                *reinterpret_cast<float2*>(p.ws_o + ((head0 + n0) * P + part) * D + d0) =
+                    make_float2(acc[t][0] * inv0, acc[t][2] * inv0);
+            if (n1 < group)
+                *reinterpret_cast<float2*>(p.ws_o + ((head0 + n1) * P + part) * D + d0) =
+                    make_float2(acc[t][1] * inv1, acc[t][3] * inv1);
+        }
+    }
+    if (P > 1 && r == 0) {
+        if (n0 < group) {
+            float* ml = p.ws_ml + ((head0 + n0) * P + part) * 2;
+            ml[0] = l0 > 0.f ? m0 : -INFINITY;
+            ml[1] = l0;
+        }
+        if (n1 < group) {
+            float* ml = p.ws_ml + ((head0 + n1) * P + part) * 2;
+            ml[0] = l1 > 0.f ? m1 : -INFINITY;
+            ml[1] = l1;
+        }
+    }
+}
+
 template <int D>
 using MmaGeom = Geom<__nv_bfloat16, D, PA_MMA_CONSUMER_WARPS, PA_MMA_RING_BYTES>;
 
@@ -583,7 +753,6 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
 
     // consumers (threads 0 .. 127)
     const int r = lane >> 2, c = lane & 3;
-    const int tv0 = 2 * c, tv1 = 2 * c + 1, tv2 = 2 * c + 8, tv3 = 2 * c + 9;
     bool dead = false;
     int g = 0;
     // Q^T (B operand of QK): thread (r, c) holds query row r. For chunk step jp
@@ -636,107 +805,14 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 const bool valid = ring.valid[st] != 0;
                 const uint32_t kb = ring.stages + st * G::kStageBytes;
                 const uint32_t vb = kb + G::kBoxes * kBoxBytes;
-                float sc[4] = {0.f, 0.f, 0.f, 0.f};
-                {
-                    uint4 kr[2][KCH];
-#pragma unroll
-                    for (int jp = 0; jp < KCH; ++jp) {
-                        const uint32_t bx = kb + (jp >> 1) * kBoxBytes;
-                        const uint32_t x = (uint32_t)(2 * c + (jp & 1));
-                        kr[0][jp] = lds128(bx + swz(r, x));
-                        kr[1][jp] = lds128(bx + swz(r + 8, x));
-                    }
-                    // S^T = K . Q^T
-#if PA_MMA_SPLIT_QK
-                    float sd[4] = {0.f, 0.f, 0.f, 0.f};  // second chain: shorter MMA dependency
-#pragma unroll
-                    for (int jp = 0; jp < KCH; ++jp) {
-                        mma_16816(sc, kr[0][jp].x, kr[1][jp].x, kr[0][jp].y, kr[1][jp].y,
-                                  qcur[jp].x, qcur[jp].y);
-                        mma_16816(sd, kr[0][jp].z, kr[1][jp].z, kr[0][jp].w, kr[1][jp].w,
-                                  qcur[jp].z, qcur[jp].w);
-                    }
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) sc[e] += sd[e];
-#else
-#pragma unroll
-                    for (int jp = 0; jp < KCH; ++jp) {
-                        mma_16816(sc, kr[0][jp].x, kr[1][jp].x, kr[0][jp].y, kr[1][jp].y,
-                                  qcur[jp].x, qcur[jp].y);
-                        mma_16816(sc, kr[0][jp].z, kr[1][jp].z, kr[0][jp].w, kr[1][jp].w,
-                                  qcur[jp].z, qcur[jp].w);
-                    }
-#endif
-                }
+                float sc[4];
+                mma_qk<D>(kb, qcur, r, c, sc);
                 uint4 vr[4][VCH];
-#pragma unroll
-                for (int hh = 0; hh < VCH; ++hh) {
-                    const uint32_t bx = vb + hh * kBoxBytes;
-                    vr[0][hh] = lds128(bx + swz(tv0, r));
-                    vr[1][hh] = lds128(bx + swz(tv1, r));
-                    vr[2][hh] = lds128(bx + swz(tv2, r));
-                    vr[3][hh] = lds128(bx + swz(tv3, r));
-                }
+                mma_load_v<D>(vb, r, c, vr);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
                 if (!valid) continue;
-
-                const int tok0 = t0 + (i << 4);
-                const int nvalid = t1 - tok0;
-                const bool lo_ok = r < nvalid, hi_ok = r + 8 < nvalid;
-                const float s0 = lo_ok ? sc[0] * p.scale_log2 : -INFINITY;  // token r,   head 2c
-                const float s1 = lo_ok ? sc[1] * p.scale_log2 : -INFINITY;  // token r,   head 2c+1
-                const float s2 = hi_ok ? sc[2] * p.scale_log2 : -INFINITY;  // token r+8, head 2c
-                const float s3 = hi_ok ? sc[3] * p.scale_log2 : -INFINITY;  // token r+8, head 2c+1
-                float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-                }
-                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-                // The accumulator is rescaled only when some running max moved; a
-                // factor of exactly 1 would leave every bit unchanged anyway.
-                const bool moved = __any_sync(0xffffffffu, mn0 != m0 || mn1 != m1);
-                const float al0 = moved ? exp2f(m0 - mn0) : 1.f;
-                const float al1 = moved ? exp2f(m1 - mn1) : 1.f;
-                const uint32_t x0 = pack_bf16x2(exp2f(s0 - mn0), exp2f(s1 - mn1));
-                const uint32_t x1 = pack_bf16x2(exp2f(s2 - mn0), exp2f(s3 - mn1));
-                // the sums use the same rounded weights the PV product sees
-                l0 = fmaf(l0, al0, bf16_lo(x0) + bf16_lo(x1));
-                l1 = fmaf(l1, al1, bf16_hi(x0) + bf16_hi(x1));
-                m0 = mn0;
-                m1 = mn1;
-                if (moved) {
-#pragma unroll
-                    for (int t = 0; t < MT; ++t) {
-                        acc[t][0] *= al0;
-                        acc[t][1] *= al1;
-                        acc[t][2] *= al0;
-                        acc[t][3] *= al1;
-                    }
-                }
-                const uint32_t pb0 = movmatrix_trans(x0);  // P^T rows (tokens) 2c, 2c+1; col head r
-                const uint32_t pb1 = movmatrix_trans(x1);  // tokens 2c+8, 2c+9
-                if (nvalid < 16) {  // slots past the context may hold anything, even NaN
-                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                    for (int hh = 0; hh < VCH; ++hh) {
-                        if (tv0 >= nvalid) vr[0][hh] = z;
-                        if (tv1 >= nvalid) vr[1][hh] = z;
-                        if (tv2 >= nvalid) vr[2][hh] = z;
-                        if (tv3 >= nvalid) vr[3][hh] = z;
-                    }
-                }
-                // O^T += V^T . P^T ; m-tile t covers head_dim 64*(t/4) + 8r + 2*(t%4) (+1 for row r+8)
-#pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                    const int hh = t >> 2, w = t & 3;
-                    const uint32_t xa = word(vr[0][hh], w), xb = word(vr[1][hh], w);
-                    const uint32_t ya = word(vr[2][hh], w), yb = word(vr[3][hh], w);
-                    mma_16816(acc[t], __byte_perm(xa, xb, 0x5410), __byte_perm(xa, xb, 0x7632),
-                              __byte_perm(ya, yb, 0x5410), __byte_perm(ya, yb, 0x7632), pb0, pb1);
-                }
+                mma_softmax_pv<D>(sc, vr, t1 - (t0 + (i << 4)), p.scale_log2, r, c, acc, m0, m1, l0, l1);
             }
             g += n_sub;
 #pragma unroll
@@ -782,47 +858,7 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
             }
             if constexpr (kConsumerWarps <= 2) {
                 // One warp holds the whole item: normalise and store from registers.
-                // Thread (r, c) holds heads 2c, 2c+1 at head_dim 64*(t/4) + 8r + 2*(t%4) (+1).
-                if (warp == 0) {
-                    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f;
-                    const float inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
-                    const int n0 = 2 * c, n1 = 2 * c + 1;
-#pragma unroll
-                    for (int t = 0; t < MT; ++t) {
-                        const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
-                        if (P == 1) {
-                            if (n0 < group)
-                                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) +
-                                                             (head0 + n0) * D + d0) =
-                                    pack_bf16x2(acc[t][0] * inv0, acc[t][2] * inv0);
-                            if (n1 < group)
-                                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) +
-                                                             (head0 + n1) * D + d0) =
-                                    pack_bf16x2(acc[t][1] * inv1, acc[t][3] * inv1);
-                        } else {
-                            if (n0 < group)
-                                *reinterpret_cast<float2*>(
-                                    p.ws_o + ((head0 + n0) * P + cur.part) * D + d0) =
-                                    make_float2(acc[t][0] * inv0, acc[t][2] * inv0);
-                            if (n1 < group)
-                                *reinterpret_cast<float2*>(
-                                    p.ws_o + ((head0 + n1) * P + cur.part) * D + d0) =
-                                    make_float2(acc[t][1] * inv1, acc[t][3] * inv1);
-                        }
-                    }
-                    if (P > 1 && r == 0) {
-                        if (n0 < group) {
-                            float* ml = p.ws_ml + ((head0 + n0) * P + cur.part) * 2;
-                            ml[0] = l0 > 0.f ? m0 : -INFINITY;
-                            ml[1] = l0;
-                        }
-                        if (n1 < group) {
-                            float* ml = p.ws_ml + ((head0 + n1) * P + cur.part) * 2;
-                            ml[0] = l1 > 0.f ? m1 : -INFINITY;
-                            ml[1] = l1;
-                        }
-                    }
-                }
+                if (warp == 0) mma_store_item<D>(p, head0, group, cur.part, r, c, acc, m0, m1, l0, l1);
                 if constexpr (kConsumerWarps == 2) named_barrier(1, 64);  // buffer free again
             } else {
                 // Cross-warp merge of this item, in fixed warp order. Buffers alternate
@@ -897,6 +933,505 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
     }
 }
 
+// ---------------------------------------------------------------------------
+// Grouped decode: the sequences of one group (beams or parallel samples of
+// one prompt, which hold its blocks through reference counts) run in one CTA,
+// so a block they share crosses HBM once and feeds all of them.
+//
+// The CTA's query columns are (member, head) pairs, column = member * g + head
+// for g = H / Hkv; consumer warp w owns n-tiles NT w .. NT w + NT - 1 of 8
+// columns. Work item = (partition, kv head, group). For every logical 16-token
+// sub-tile of the item the producer reads each active member's block id and
+// issues one ring position ("unit") per distinct block, tagged in a per-stage
+// header with the mask of members that use it, the sub-tile index and an
+// end-of-item flag. Every consumer warp walks every position (the empty
+// barrier counts all consumer warps), computes only when one of its members
+// is in the mask, and keeps its members' running state in registers to the
+// end of the item, so each member's arithmetic is the same whichever blocks
+// it shares. Sharing of prefix blocks among parallel samples and beams:
+// "AI 推理系列（十六）：PagedAttention——…", § Copy-on-Write、并行采样与
+// Prefix Caching 不是同一件事; "PagedAttention原理详解：GPU显存优化与模型路由
+// 技术", § PagedAttention的三大核心优势 (point 2 and the beam-search paragraph).
+// ---------------------------------------------------------------------------
+#ifndef PA_GROUPED_RING_BYTES
+#define PA_GROUPED_RING_BYTES 49152
+#endif
+
+constexpr int kMaxGroupSeqs = 8;            // members per group (header mask bits 0..7)
+constexpr int kGroupedMaxCols = 64;         // query columns (member, head) per CTA
+constexpr uint32_t kUnitLast = 1u << 31;    // header: last unit of the item
+constexpr int kUnitSubShift = 8;            // header bits 8..30: sub-tile index in the item
+constexpr uint32_t kUnitSubMask = 0x7fffffu;
+
+template <int D>
+using GroupedGeom = Geom<__nv_bfloat16, D, 1, PA_GROUPED_RING_BYTES>;
+
+// CTAs per SM each grouped variant is compiled for: as many as fit without
+// spilling (two n-tiles per warp at head_dim 128 need about 200 registers).
+// Up to PA_GROUPED_ONE_TILE_WARPS n-tiles, each consumer warp takes one (more
+// warps in flight); beyond that, two per warp (at most 4 consumer warps).
+#ifndef PA_GROUPED_ONE_TILE_WARPS
+#define PA_GROUPED_ONE_TILE_WARPS 4
+#endif
+__host__ __device__ constexpr int grouped_min_blocks(int d, int cw, int nt) {
+    return nt == 1 ? (cw <= 2 ? 4 : 2)
+                   : d == 64 ? (cw <= 1 ? 4 : cw == 2 ? 3 : 2) : (cw <= 1 ? 4 : cw <= 3 ? 2 : 1);
+}
+
+// Walk over a grouped CTA's items, u = blockIdx.x + k * gridDim.x, item u =
+// (partition u % P, kv head, group u / (P Hkv)). Lane l holds the context
+// length of member l % gs of item kbase + l / gs (32 / gs items per load).
+struct GWalk {
+    int k, kbase, ctx_lane;
+};
+
+struct GItem {
+    bool valid;
+    int grp, kh, part, t0;
+    int tmax;     // end of the item's tokens over its members (== t0: nothing to read)
+    int t1_lane;  // end of member (lane & 7)'s tokens in the item (t0 if none)
+};
+
+__device__ __forceinline__ int gwalk_load(const DecodeParams& p, int num_items, int kbase, int lane,
+                                          int gs, int ipb, bool report) {
+    if (lane >= ipb * gs) return 0;
+    const int u = blockIdx.x + (kbase + lane / gs) * gridDim.x;
+    if (u >= num_items) return 0;
+    const int part = u % p.num_partitions;
+    const int s = (u / p.num_partitions / p.num_kv_heads) * gs + lane % gs;
+    if (s >= p.num_seqs) return 0;
+    return clamp_ctx(__ldg(p.context_lens + s), p.max_context_len, report && part == 0);
+}
+
+__device__ __forceinline__ GItem gitem_next(GWalk& w, const DecodeParams& p, int num_items, int gs,
+                                            int ipb, int lane, bool report, bool want_empty) {
+    for (;;) {
+        const int u = blockIdx.x + w.k * gridDim.x;
+        GItem it;
+        it.valid = u < num_items;
+        it.grp = it.kh = it.part = it.t0 = it.tmax = it.t1_lane = 0;
+        if (!it.valid) return it;
+        if (w.k - w.kbase >= ipb) {
+            w.kbase = w.k;
+            w.ctx_lane = gwalk_load(p, num_items, w.kbase, lane, gs, ipb, report);
+        }
+        const int m = lane & (kMaxGroupSeqs - 1);
+        const int ctx = __shfl_sync(0xffffffffu, w.ctx_lane, (w.k - w.kbase) * gs + (m < gs ? m : 0));
+        it.part = u % p.num_partitions;
+        const int rest = u / p.num_partitions;
+        it.kh = rest % p.num_kv_heads;
+        it.grp = rest / p.num_kv_heads;
+        it.t0 = it.part * p.partition_size;
+        it.t1_lane = m < gs ? max(it.t0, min(ctx, it.t0 + p.partition_size)) : it.t0;
+        it.tmax = __reduce_max_sync(0xffffffffu, it.t1_lane);
+        ++w.k;
+        if (it.tmax > it.t0 || want_empty) return it;
+    }
+}
+
+// Block ids of sub-tile base + lane for every member whose tokens reach it
+// (bit m of `act`).
+__device__ __forceinline__ void gload_phys(const DecodeParams& p, const GItem& it, int base, int gs,
+                                           int lane, uint32_t& act, int (&phys)[kMaxGroupSeqs]) {
+    act = 0;
+    const int tok0 = it.t0 + ((base + lane) << 4);
+#pragma unroll
+    for (int m = 0; m < kMaxGroupSeqs; ++m) {
+        const int t1 = __shfl_sync(0xffffffffu, it.t1_lane, m);
+        phys[m] = -1;
+        if (it.valid && m < gs && tok0 < t1) {
+            act |= 1u << m;
+            phys[m] = __ldg(p.block_tables + (int64_t)(it.grp * gs + m) * p.table_stride +
+                            (tok0 >> p.log2_block_size));
+        }
+    }
+}
+
+// Issue the units of a batch of up to 32 sub-tiles (lane l: sub-tile base + l).
+// Each lane finds the distinct block ids among its active members (the first
+// member holding an id leads its unit); units take ring positions g + exclusive
+// prefix sum, in sub-tile order and, within a sub-tile, in leader order. Lanes
+// issue in sub-rounds of kStages positions, so a sub-round touches each stage
+// at most once and a stage's rounds are issued in order.
+template <class G>
+__device__ __forceinline__ void issue_units(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                            const DecodeParams& p, const Ring& ring, uint32_t* hdr,
+                                            const GItem& it, int base, int n_sub, uint32_t act,
+                                            const int (&phys)[kMaxGroupSeqs], int lane, int& g,
+                                            int& issued, bool& dead) {
+    uint32_t lead = 0;
+    int nu = 0;
+#pragma unroll
+    for (int m = 0; m < kMaxGroupSeqs; ++m) {
+        bool first = ((act >> m) & 1u) != 0;
+#pragma unroll
+        for (int m2 = 0; m2 < m; ++m2)
+            if (((act >> m2) & 1u) && phys[m2] == phys[m]) first = false;
+        if (first) {
+            lead |= 1u << m;
+            ++nu;
+        }
+    }
+    int incl = nu;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    const int first_pos = incl - nu;
+    const bool last_batch = base + 32 >= n_sub;
+    const int i = base + lane;
+    const int tok0 = it.t0 + (i << 4);
+    for (int k0 = 0; k0 < total && !dead; k0 += G::kStages) {
+        bool ok = true;
+        int pos = first_pos;
+#pragma unroll
+        for (int m = 0; m < kMaxGroupSeqs; ++m) {
+            if ((lead >> m) & 1u) {
+                if (ok && pos >= k0 && pos < k0 + G::kStages) {
+                    uint32_t mask = 0;
+#pragma unroll
+                    for (int m2 = m; m2 < kMaxGroupSeqs; ++m2)
+                        if (((act >> m2) & 1u) && phys[m2] == phys[m]) mask |= 1u << m2;
+                    const uint32_t h = mask | ((uint32_t)i << kUnitSubShift) |
+                                       (last_batch && pos == total - 1 ? kUnitLast : 0u);
+                    ok = issue_subtile<G>(kmap, vmap, p, ring, g + pos, phys[m], it.kh, tok0, hdr, h);
+                    if (ok) issued = g + pos + 1;
+                }
+                ++pos;
+            }
+        }
+        dead = __any_sync(0xffffffffu, !ok);
+    }
+    issued = __reduce_max_sync(0xffffffffu, issued);
+    g += total;
+}
+
+// S^T for NT n-tiles from one set of K fragments (see mma_qk).
+template <int D, int NT>
+__device__ __forceinline__ void mma_qk_n(uint32_t kb, const uint4 (&q)[NT][D / 32], int r, int c,
+                                         float (&sc)[NT][4]) {
+    constexpr int KCH = D / 32;
+    uint4 kr[2][KCH];
+#pragma unroll
+    for (int jp = 0; jp < KCH; ++jp) {
+        const uint32_t bx = kb + (jp >> 1) * kBoxBytes;
+        const uint32_t x = (uint32_t)(2 * c + (jp & 1));
+        kr[0][jp] = lds128(bx + swz(r, x));
+        kr[1][jp] = lds128(bx + swz(r + 8, x));
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+#pragma unroll
+        for (int jp = 0; jp < KCH; ++jp) {
+            mma_16816(sc[j], kr[0][jp].x, kr[1][jp].x, kr[0][jp].y, kr[1][jp].y, q[j][jp].x, q[j][jp].y);
+            mma_16816(sc[j], kr[0][jp].z, kr[1][jp].z, kr[0][jp].w, kr[1][jp].w, q[j][jp].z, q[j][jp].w);
+        }
+    }
+}
+
+// Online-softmax update for NT n-tiles whose columns may each see a different
+// number of valid tokens: nva / nvb = valid tokens of this thread's columns 2c
+// and 2c + 1 of n-tile j (0 for a column whose member does not use the unit).
+// A column that has seen no valid token keeps max -inf and weight 0.
+template <int D, int NT>
+__device__ __forceinline__ void mma_softmax_pv_n(const float (&sc)[NT][4], uint4 (&vr)[4][D / 64],
+                                                 const int (&nva)[NT], const int (&nvb)[NT],
+                                                 float scale_log2, int r, int c,
+                                                 float (&acc)[NT][D / 16][4], float (&ma)[NT],
+                                                 float (&mb)[NT], float (&la)[NT], float (&lb)[NT]) {
+    constexpr int VCH = D / 64;
+    constexpr int MT = D / 16;
+    float s[NT][4], mxa[NT], mxb[NT];
+    int nvmax = 0;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        s[j][0] = r < nva[j] ? sc[j][0] * scale_log2 : -INFINITY;      // token r,   column 2c
+        s[j][1] = r < nvb[j] ? sc[j][1] * scale_log2 : -INFINITY;      // token r,   column 2c+1
+        s[j][2] = r + 8 < nva[j] ? sc[j][2] * scale_log2 : -INFINITY;  // token r+8, column 2c
+        s[j][3] = r + 8 < nvb[j] ? sc[j][3] * scale_log2 : -INFINITY;  // token r+8, column 2c+1
+        mxa[j] = fmaxf(s[j][0], s[j][2]);
+        mxb[j] = fmaxf(s[j][1], s[j][3]);
+        nvmax = max(nvmax, max(nva[j], nvb[j]));
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            mxa[j] = fmaxf(mxa[j], __shfl_xor_sync(0xffffffffu, mxa[j], off));
+            mxb[j] = fmaxf(mxb[j], __shfl_xor_sync(0xffffffffu, mxb[j], off));
+        }
+    }
+    bool mv = false;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        mxa[j] = fmaxf(ma[j], mxa[j]);  // new running max
+        mxb[j] = fmaxf(mb[j], mxb[j]);
+        mv = mv || mxa[j] != ma[j] || mxb[j] != mb[j];
+    }
+    const bool moved = __any_sync(0xffffffffu, mv);
+    uint32_t pb0[NT], pb1[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        const float ba = mxa[j] == -INFINITY ? 0.f : mxa[j];
+        const float bb = mxb[j] == -INFINITY ? 0.f : mxb[j];
+        const float ala = moved ? exp2f(ma[j] - ba) : 1.f;
+        const float alb = moved ? exp2f(mb[j] - bb) : 1.f;
+        const uint32_t x0 = pack_bf16x2(exp2f(s[j][0] - ba), exp2f(s[j][1] - bb));
+        const uint32_t x1 = pack_bf16x2(exp2f(s[j][2] - ba), exp2f(s[j][3] - bb));
+        la[j] = fmaf(la[j], ala, bf16_lo(x0) + bf16_lo(x1));
+        lb[j] = fmaf(lb[j], alb, bf16_hi(x0) + bf16_hi(x1));
+        ma[j] = mxa[j];
+        mb[j] = mxb[j];
+        if (moved) {
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                acc[j][t][0] *= ala;
+                acc[j][t][1] *= alb;
+                acc[j][t][2] *= ala;
+                acc[j][t][3] *= alb;
+            }
+        }
+        pb0[j] = movmatrix_trans(x0);
+        pb1[j] = movmatrix_trans(x1);
+    }
+    // Rows past every column's tokens are zeroed (those slots may hold
+    // anything); rows before it belong to some member's context.
+    nvmax = __reduce_max_sync(0xffffffffu, nvmax);
+    if (nvmax < 16) {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int hh = 0; hh < VCH; ++hh) {
+            if (2 * c >= nvmax) vr[0][hh] = z;
+            if (2 * c + 1 >= nvmax) vr[1][hh] = z;
+            if (2 * c + 8 >= nvmax) vr[2][hh] = z;
+            if (2 * c + 9 >= nvmax) vr[3][hh] = z;
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+        const int hh = t >> 2, w = t & 3;
+        const uint32_t xa = word(vr[0][hh], w), xb = word(vr[1][hh], w);
+        const uint32_t ya = word(vr[2][hh], w), yb = word(vr[3][hh], w);
+        const uint32_t a0 = __byte_perm(xa, xb, 0x5410), a1 = __byte_perm(xa, xb, 0x7632);
+        const uint32_t a2 = __byte_perm(ya, yb, 0x5410), a3 = __byte_perm(ya, yb, 0x7632);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma_16816(acc[j][t], a0, a1, a2, a3, pb0[j], pb1[j]);
+    }
+}
+
+// Store one column's result (m, l = its running max and summed weights): bf16
+// output when P == 1, else the normalised partial and (m, l).
+template <int D>
+__device__ __forceinline__ void grouped_store_col(const DecodeParams& p, int64_t row, int part, int r,
+                                                  int c, int e, const float (&acc)[D / 16][4],
+                                                  float m, float l) {
+    constexpr int MT = D / 16;
+    const int P = p.num_partitions;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+        const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
+        if (P == 1)
+            *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + row * D + d0) =
+                pack_bf16x2(acc[t][e] * inv, acc[t][e + 2] * inv);
+        else
+            *reinterpret_cast<float2*>(p.ws_o + (row * P + part) * D + d0) =
+                make_float2(acc[t][e] * inv, acc[t][e + 2] * inv);
+    }
+    if (P > 1 && r == 0) {
+        float* ml = p.ws_ml + (row * P + part) * 2;
+        ml[0] = l > 0.f ? m : -INFINITY;
+        ml[1] = l;
+    }
+}
+
+template <int D, int CW, int NT>
+__global__ void __launch_bounds__((CW + 1) * 32, grouped_min_blocks(D, CW, NT))
+decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
+                          const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
+                          int num_items, int gs) {
+    using G = GroupedGeom<D>;
+    constexpr int KCH = D / 32;
+    constexpr int VCH = D / 64;
+    constexpr int MT = D / 16;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int P = p.num_partitions;
+    const int group = p.num_heads / p.num_kv_heads;
+    const int ipb = 32 / gs;
+    Ring ring;
+    uint8_t* base = setup_ring<G>(smem_raw, ring, G::kStages * 4, CW);
+    if (base == nullptr) {
+        if (threadIdx.x == 0) atomicOr(&s_status_tma, kStatusSmemAlign);
+        return;
+    }
+    uint32_t* hdr = reinterpret_cast<uint32_t*>(base + G::kRingBytes);
+    GWalk walk;
+    walk.k = 0;
+    walk.kbase = 0;
+    walk.ctx_lane = gwalk_load(p, num_items, 0, lane, gs, ipb, warp == 0);
+    __syncthreads();
+
+    if (warp == CW) {  // producer
+        if (lane == 0) {
+            prefetch_tensormap(&kmap);
+            prefetch_tensormap(&vmap);
+        }
+        bool dead = false;
+        int g = 0, issued = 0;
+        GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
+        int cur_base = 0;
+        uint32_t act_cur;
+        int phys_cur[kMaxGroupSeqs];
+        gload_phys(p, cur, cur_base, gs, lane, act_cur, phys_cur);
+        while (cur.valid && !dead) {
+            const int n_sub = (cur.tmax - cur.t0 + 15) >> 4;
+            GItem nxt = cur;
+            int nxt_base = cur_base + 32;
+            if (nxt_base >= n_sub) {
+                nxt = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
+                nxt_base = 0;
+            }
+            uint32_t act_nxt;
+            int phys_nxt[kMaxGroupSeqs];
+            gload_phys(p, nxt, nxt_base, gs, lane, act_nxt, phys_nxt);  // in flight meanwhile
+            issue_units<G>(&kmap, &vmap, p, ring, hdr, cur, cur_base, n_sub, act_cur, phys_cur, lane,
+                           g, issued, dead);
+            cur = nxt;
+            cur_base = nxt_base;
+            act_cur = act_nxt;
+#pragma unroll
+            for (int m = 0; m < kMaxGroupSeqs; ++m) phys_cur[m] = phys_nxt[m];
+        }
+        drain_ring<G>(ring, issued, lane);
+        return;
+    }
+
+    // consumers: thread (r, c) holds q column 8 (NT warp + j) + r of n-tile j as
+    // the B operand, and C-fragment columns 8 (NT warp + j) + 2c, + 2c + 1
+    const int r = lane >> 2, c = lane & 3;
+    const int col0 = 8 * NT * warp;
+    uint32_t bita[NT], bitb[NT];  // mask bit of this thread's columns' members (0: none)
+    uint32_t wbits = 0;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        const int ma = (col0 + 8 * j + 2 * c) / group, mb = (col0 + 8 * j + 2 * c + 1) / group;
+        bita[j] = ma < gs ? 1u << ma : 0u;
+        bitb[j] = mb < gs ? 1u << mb : 0u;
+        wbits |= bita[j] | bitb[j];
+    }
+    wbits = __reduce_or_sync(0xffffffffu, wbits);
+    // q of the item's columns (zero for columns without a member, sequence or tokens)
+    auto load_q = [&](const GItem& it, uint4 (&q)[NT][KCH]) {
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            const int col = col0 + 8 * j + r;
+            const int m = col / group, hd = col - m * group;
+            const int t1 = __shfl_sync(0xffffffffu, it.t1_lane, m & (kMaxGroupSeqs - 1));
+            const int s = it.grp * gs + m;
+            if (it.valid && m < gs && s < p.num_seqs && t1 > it.t0) {
+                const uint16_t* qrow = static_cast<const uint16_t*>(p.q) +
+                                       ((int64_t)s * p.num_heads + (int64_t)it.kh * group + hd) * D;
+#pragma unroll
+                for (int jp = 0; jp < KCH; ++jp)
+                    q[j][jp] = ld_v4(qrow + (jp >> 1) * 64 + (2 * c + (jp & 1)) * 8);
+            } else {
+#pragma unroll
+                for (int jp = 0; jp < KCH; ++jp) q[j][jp] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    };
+    bool dead = false;
+    int g = 0;
+    GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, warp == 0, P == 1);
+    uint4 q[NT][KCH];
+    load_q(cur, q);
+    while (cur.valid && !dead) {
+        GItem nxt = gitem_next(walk, p, num_items, gs, ipb, lane, warp == 0, P == 1);
+        int t1a[NT], t1b[NT];
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            const int ma = (col0 + 8 * j + 2 * c) / group, mb = (col0 + 8 * j + 2 * c + 1) / group;
+            t1a[j] = __shfl_sync(0xffffffffu, cur.t1_lane, ma & (kMaxGroupSeqs - 1));
+            t1b[j] = __shfl_sync(0xffffffffu, cur.t1_lane, mb & (kMaxGroupSeqs - 1));
+        }
+        float acc[NT][MT][4];
+        float ma[NT], mb[NT], la[NT], lb[NT];
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+#pragma unroll
+            for (int t = 0; t < MT; ++t) acc[j][t][0] = acc[j][t][1] = acc[j][t][2] = acc[j][t][3] = 0.f;
+            ma[j] = mb[j] = -INFINITY;
+            la[j] = lb[j] = 0.f;
+        }
+        if (cur.tmax > cur.t0) {
+            for (;;) {
+                const int st = g % G::kStages;
+                const uint32_t round = (uint32_t)(g / G::kStages);
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(ring.full + 8 * st, round & 1u))) {
+                    if (lane == 0) atomicOr(&s_status_tma, kStatusTimeout);
+                    dead = true;
+                    break;
+                }
+                const uint32_t h = hdr[st];
+                const bool mine = ring.valid[st] != 0 && (h & wbits) != 0;
+                const int tok0 = cur.t0 + (int)((h >> kUnitSubShift) & kUnitSubMask) * 16;
+                const uint32_t kb = ring.stages + st * G::kStageBytes;
+                float sc[NT][4];
+                uint4 vr[4][VCH];
+                if (mine) {
+                    mma_qk_n<D, NT>(kb, q, r, c, sc);
+                    mma_load_v<D>(kb + G::kBoxes * kBoxBytes, r, c, vr);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
+                ++g;
+                if (mine) {
+                    int nva[NT], nvb[NT];
+#pragma unroll
+                    for (int j = 0; j < NT; ++j) {
+                        nva[j] = (h & bita[j]) ? min(16, t1a[j] - tok0) : 0;
+                        nvb[j] = (h & bitb[j]) ? min(16, t1b[j] - tok0) : 0;
+                    }
+                    mma_softmax_pv_n<D, NT>(sc, vr, nva, nvb, p.scale_log2, r, c, acc, ma, mb, la, lb);
+                }
+                if (h & kUnitLast) break;
+            }
+        }
+        if (dead) break;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                la[j] += __shfl_xor_sync(0xffffffffu, la[j], off);
+                lb[j] += __shfl_xor_sync(0xffffffffu, lb[j], off);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int col = col0 + 8 * j + 2 * c + e;
+                const int m = col / group, hd = col - m * group;
+                const int s = cur.grp * gs + m;
+                const int t1 = e == 0 ? t1a[j] : t1b[j];
+                if (m < gs && s < p.num_seqs && (P == 1 || t1 > cur.t0)) {
+                    const int64_t row = (int64_t)s * p.num_heads + (int64_t)cur.kh * group + hd;
+                    grouped_store_col<D>(p, row, cur.part, r, c, e, acc[j],
+                                         e == 0 ? ma[j] : mb[j], e == 0 ? la[j] : lb[j]);
+                }
+            }
+        }
+        cur = nxt;
+        load_q(cur, q);
+    }
+}
+
 template <typename T, int D>
 cudaError_t launch_simt_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
                           cudaStream_t stream) {
@@ -945,6 +1480,38 @@ cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUt
     return cudaGetLastError();
 }
 
+template <int D, int CW, int NT>
+cudaError_t launch_grouped_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
+                             int gs, cudaStream_t stream) {
+    using G = GroupedGeom<D>;
+    constexpr size_t smem = smem_bytes<G>(G::kStages * 4);
+    constexpr int kThreads = (CW + 1) * 32;
+    auto kernel = decode_tma_grouped_kernel<D, CW, NT>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    static int per_sm[128] = {0};
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+    if (per_sm[dev] == 0) {
+        int n = 0;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kThreads, smem)) != cudaSuccess)
+            return e;
+        per_sm[dev] = n > 0 ? n : 1;
+    }
+    int sms = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const long groups = (p.num_seqs + gs - 1) / gs;
+    const long items = (long)p.num_partitions * p.num_kv_heads * groups;
+    const long slots = (long)per_sm[dev] * sms;
+    const unsigned grid = (unsigned)(items < slots ? items : slots);
+    kernel<<<grid, kThreads, smem, stream>>>(km, vm, p, (int)items, gs);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bool mma,
@@ -966,6 +1533,64 @@ int mma_ctas_per_sm() { return PA_MMA_MIN_BLOCKS; }
 
 bool mma_supported(int dtype, int head_dim, int group) {
     return dtype == 1 && (head_dim == 64 || head_dim == 128) && group >= 2 && group <= kGroupMax;
+}
+
+// Query columns (member, head) -> n-tiles of 8 -> consumer warps: one n-tile
+// per warp when a single tile holds them all, else two per warp.
+static void grouped_shape(int gs, int group, int* cw, int* nt) {
+    const int tiles = (gs * group + 7) / 8;
+    *nt = tiles <= PA_GROUPED_ONE_TILE_WARPS ? 1 : 2;
+    *cw = (tiles + *nt - 1) / *nt;
+}
+
+bool grouped_supported(int dtype, int head_dim, int group, int gs) {
+    return dtype == 1 && (head_dim == 64 || head_dim == 128) && gs >= 2 && gs <= kMaxGroupSeqs &&
+           group >= 1 && gs * group <= kGroupedMaxCols;
+}
+
+int grouped_ctas_per_sm(int head_dim, int gs, int group) {
+    int cw = 1, nt = 1;
+    grouped_shape(gs, group, &cw, &nt);
+    return grouped_min_blocks(head_dim, cw, nt);
+}
+
+template <int D>
+static cudaError_t launch_grouped_d(const DecodeParams& p, int cw, int nt, int gs,
+                                   const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                   cudaStream_t stream) {
+    static_assert(PA_GROUPED_ONE_TILE_WARPS >= 1 && PA_GROUPED_ONE_TILE_WARPS <= 4,
+                  "one-tile warps: 1 .. 4");
+    if (nt == 1) {
+        switch (cw) {
+            case 1: return launch_grouped_t<D, 1, 1>(p, kmap, vmap, gs, stream);
+#if PA_GROUPED_ONE_TILE_WARPS >= 2
+            case 2: return launch_grouped_t<D, 2, 1>(p, kmap, vmap, gs, stream);
+#endif
+#if PA_GROUPED_ONE_TILE_WARPS >= 3
+            case 3: return launch_grouped_t<D, 3, 1>(p, kmap, vmap, gs, stream);
+#endif
+#if PA_GROUPED_ONE_TILE_WARPS >= 4
+            case 4: return launch_grouped_t<D, 4, 1>(p, kmap, vmap, gs, stream);
+#endif
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    switch (cw) {
+        case 1: return launch_grouped_t<D, 1, 2>(p, kmap, vmap, gs, stream);
+        case 2: return launch_grouped_t<D, 2, 2>(p, kmap, vmap, gs, stream);
+        case 3: return launch_grouped_t<D, 3, 2>(p, kmap, vmap, gs, stream);
+        case 4: return launch_grouped_t<D, 4, 2>(p, kmap, vmap, gs, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_decode_grouped(const DecodeParams& p, int head_dim, int gs,
+                                  const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                  cudaStream_t stream) {
+    int cw = 1, nt = 1;
+    grouped_shape(gs, p.num_heads / p.num_kv_heads, &cw, &nt);
+    return head_dim == 64 ? launch_grouped_d<64>(p, cw, nt, gs, kmap, vmap, stream)
+                          : launch_grouped_d<128>(p, cw, nt, gs, kmap, vmap, stream);
 }
 
 cudaError_t read_status_tma(unsigned* bits, bool clear) {

@@ -71,6 +71,15 @@ int mma_ctas_per_sm();
 cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bool mma,
                               const CUtensorMap& kmap, const CUtensorMap& vmap,
                               cudaStream_t stream);
+// Grouped decode: sequences [k gs, (k + 1) gs) form group k and run in one CTA,
+// so blocks they share are read once. bf16, head_dim 64 / 128, 2 <= gs <= 8,
+// gs * (H / Hkv) <= 64 query columns.
+bool grouped_supported(int dtype, int head_dim, int group, int gs);
+// CTA slots per SM of the grouped kernel chosen for (head_dim, gs, H / Hkv).
+int grouped_ctas_per_sm(int head_dim, int gs, int group);
+cudaError_t launch_decode_grouped(const DecodeParams& p, int head_dim, int gs,
+                                  const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                  cudaStream_t stream);
 // Log-sum-exp merge of the P partial results into out.
 cudaError_t launch_partition_reduce(const DecodeParams& p, int dtype, int head_dim,
                                     cudaStream_t stream);

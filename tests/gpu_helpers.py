@@ -29,9 +29,10 @@ def device_tensors(wl, vals):
     }
 
 
-def gpu_step(wl, vals, partition_size=None, out=None, workspace=None):
+def gpu_step(wl, vals, partition_size=None, out=None, workspace=None, group_size=1):
     """One pass of the hot path on the GPU, in place on vals' caches:
-    copy-on-write block copies, append of this step's tokens, decode."""
+    copy-on-write block copies, append of this step's tokens, decode (grouped
+    by ``group_size`` sequences when > 1)."""
     d = device_tensors(wl, vals)
     kc, vc = vals["k_cache"], vals["v_cache"]
     if wl.copy_pairs.shape[0]:
@@ -41,9 +42,18 @@ def gpu_step(wl, vals, partition_size=None, out=None, workspace=None):
     if out is None:
         out = torch.empty_like(vals["q"])
     ps = wl.partition_size if partition_size is None else partition_size
-    pa.pa_decode(out, vals["q"], kc, vc, d["tables"], d["ctx"], wl.scale,
-                 max_context_len=wl.max_context_len, partition_size=ps, workspace=workspace)
+    if group_size > 1:
+        pa.pa_decode_grouped(out, vals["q"], kc, vc, d["tables"], d["ctx"], wl.scale, group_size,
+                             max_context_len=wl.max_context_len, partition_size=ps,
+                             workspace=workspace)
+    else:
+        pa.pa_decode(out, vals["q"], kc, vc, d["tables"], d["ctx"], wl.scale,
+                     max_context_len=wl.max_context_len, partition_size=ps, workspace=workspace)
     return out
+
+
+def last_kernel():
+    return pa.load_library().pa_test_last_decode_kernel()
 
 
 def oracle_step(wl, host):

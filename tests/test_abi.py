@@ -88,6 +88,37 @@ def test_partition_policy(lib):
     assert lib.pa_decode_num_partitions(8, 64, 32768, ctypes.byref(d70), -1) == 1
 
 
+def test_grouped_partition_policy(lib):
+    d70 = _desc(num_kv_heads=8)
+    f = lib.pa_decode_grouped_num_partitions
+    # a group is the unit: 4-beam groups x 8 kv heads = 256 items fill 296 slots
+    # (2 CTAs per SM for 32 query columns at head_dim 128) in one wave
+    assert f(128, 64, 2303, ctypes.byref(d70), 4, 0) == 1
+    # one group of 8 (64 columns, 1 CTA per SM): 8 items, so split into 18 partitions
+    assert f(8, 64, 32768, ctypes.byref(d70), 8, 0) == 18
+    assert f(8, 64, 32768, ctypes.byref(d70), 4, 512) == 64           # explicit size
+    # group_size 1 and shapes without the grouped kernel follow pa_decode's policy
+    assert f(8, 64, 32768, ctypes.byref(d70), 1, 0) == \
+        lib.pa_decode_num_partitions(8, 64, 32768, ctypes.byref(d70), 0)
+    f32 = _desc(num_kv_heads=8, dtype=pa.PA_F32)
+    assert f(2, 64, 4096, ctypes.byref(f32), 4, 0) == \
+        lib.pa_decode_num_partitions(2, 64, 4096, ctypes.byref(f32), 0)
+    for bad in (0, 9, -1):
+        assert f(128, 64, 2303, ctypes.byref(d70), bad, 0) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_decode_grouped_workspace_size(8, 64, 32768, ctypes.byref(d70), 4, 512) == \
+        lib.pa_decode_workspace_size(8, 64, 32768, ctypes.byref(d70), 512)
+
+
+def test_grouped_decode_rejects_bad_group_size(lib):
+    p = ctypes.c_void_p(256)
+    desc = _desc()
+    for bad in (0, 9):
+        rc = lib.pa_decode_grouped(p, p, p, p, p, 8, p, 100, 4, 8, ctypes.c_float(0.1),
+                                   ctypes.byref(desc), bad, 0, None, 0, None)
+        assert rc == pa.PA_ERR_INVALID_ARG
+        assert b"group_size" in lib.pa_get_last_error()
+
+
 def test_append_and_copy_reject_bad_arguments(lib):
     p = ctypes.c_void_p(16)
     assert lib.pa_kv_append(p, p, p, -1, p, p, ctypes.byref(_desc()), None) == pa.PA_ERR_INVALID_ARG

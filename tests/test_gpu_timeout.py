@@ -16,15 +16,28 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-@pytest.mark.parametrize("name,kw", [
-    ("llama70b_gqa", dict(num_seqs=1, context_len=1024)),   # persistent tensor-core kernel
-    ("tiny", {}),                                             # CUDA-core kernel
+def _decode(wl, vals, d, out, gs):
+    kc, vc = vals["k_cache"], vals["v_cache"]
+    if gs > 1:
+        pa.pa_decode_grouped(out, vals["q"], kc, vc, d["tables"], d["ctx"], wl.scale, gs,
+                             max_context_len=wl.max_context_len, partition_size=0)
+    else:
+        pa.pa_decode(out, vals["q"], kc, vc, d["tables"], d["ctx"], wl.scale,
+                     max_context_len=wl.max_context_len, partition_size=0)
+
+
+@pytest.mark.parametrize("name,kw,gs", [
+    ("llama70b_gqa", dict(num_seqs=1, context_len=1024), 1),   # persistent tensor-core kernel
+    ("tiny", {}, 1),                                             # CUDA-core kernel
+    ("cow_beam4", dict(num_prompts=2, prompt_len=300, max_suffix=30), 4),   # grouped kernel
 ])
-def test_skipped_load_times_out_then_recovers(name, kw):
+def test_skipped_load_times_out_then_recovers(name, kw, gs):
     wl = W.make(name, **kw)
     vals = W.make_values(wl, DEV)
     d = G.device_tensors(wl, vals)
     kc, vc = vals["k_cache"], vals["v_cache"]
+    if wl.copy_pairs.shape[0]:
+        pa.pa_block_copy(d["pairs"], kc, vc)
     pa.pa_kv_append(vals["k_new"], vals["v_new"], d["slots"], kc, vc)
     pa.pa_sync_check()
     lib = pa.load_library()
@@ -32,8 +45,7 @@ def test_skipped_load_times_out_then_recovers(name, kw):
     lib.pa_test_skip_load(1)
     try:
         t0 = time.time()
-        pa.pa_decode(out, vals["q"], kc, vc, d["tables"], d["ctx"], wl.scale,
-                     max_context_len=wl.max_context_len, partition_size=0)
+        _decode(wl, vals, d, out, gs)
         with pytest.raises(pa.PAError) as e:
             pa.pa_sync_check()
         assert e.value.code == pa.PA_ERR_TIMEOUT
@@ -42,9 +54,10 @@ def test_skipped_load_times_out_then_recovers(name, kw):
         lib.pa_test_skip_load(-1)
     pa.pa_sync_check()                                  # status was cleared
     out2 = torch.empty_like(vals["q"])
-    pa.pa_decode(out2, vals["q"], kc, vc, d["tables"], d["ctx"], wl.scale,
-                 max_context_len=wl.max_context_len, partition_size=0)
+    _decode(wl, vals, d, out2, gs)
     pa.pa_sync_check()
+    if gs > 1:
+        assert G.last_kernel() == pa.PA_KERNEL_GROUPED
     seqs = list(range(wl.num_seqs))
     ref = G.oracle_sampled(wl, vals, seqs)
     G.check_tolerance(G.to_f64(out2), ref, wl.dtype, f"{name} after a timed-out call")

@@ -171,3 +171,101 @@ def test_rounding_rule():
     assert kernel_stages(8192, 65536) == 8
     assert kernel_stages(16384, 65536) == 4
     assert kernel_stages(16384, 32768) == 4         # never fewer than the warps
+
+
+# ---------------------------------------------------------------------------
+# The grouped kernel's ring: every consumer warp reads EVERY position (each
+# position is a unit some of the group's sequences use), the EMPTY barrier
+# counts all consumer warps, and there is no barrier between work items. A
+# warp can then never be more than one phase ahead of a slot, whatever the
+# stage count, because the producer cannot refill a slot that this warp has
+# not released.
+# ---------------------------------------------------------------------------
+def simulate_broadcast(stages, warps, batches, seed, max_steps=2_000_000):
+    rnd = random.Random(seed)
+    full = [Barrier(1) for _ in range(stages)]
+    empty = [Barrier(warps) for _ in range(stages)]
+    slot = [None] * stages
+    reads = [0] * stages              # warps that read the slot's current position
+    inflight = []
+    producer = []
+    g = 0
+    for units in batches:             # units issued by one batch, sub-rounds of `stages`
+        for k0 in range(0, units, stages):
+            producer.append([g + u for u in range(k0, min(k0 + stages, units))])
+        g += units
+    total = g
+    pc = [0] * warps
+    pi, pending = 0, None
+    for _ in range(max_steps):
+        progress = False
+        if inflight and rnd.random() < 0.5:
+            st, pos = inflight.pop(rnd.randrange(len(inflight)))
+            slot[st] = pos
+            reads[st] = 0
+            full[st].complete_tx(1)
+            progress = True
+        if pi < len(producer) and rnd.random() < 0.5:
+            if pending is None:
+                pending = list(producer[pi])
+            for pos in list(pending):
+                st, rd = pos % stages, pos // stages
+                if empty[st].test_parity((rd & 1) ^ 1):
+                    if slot[st] is not None and reads[st] != warps:
+                        return f"slot {st} overwritten before all warps read position {slot[st]}"
+                    full[st].arrive(tx=1)
+                    inflight.append((st, pos))
+                    pending.remove(pos)
+                    progress = True
+            if not pending:
+                pending = None
+                pi += 1
+        w = rnd.randrange(warps)
+        if pc[w] < total:
+            pos = pc[w]
+            st, rd = pos % stages, pos // stages
+            if full[st].test_parity(rd & 1):
+                if slot[st] != pos:
+                    return f"warp {w}: position {pos} read from slot {st} holding {slot[st]}"
+                reads[st] += 1
+                empty[st].arrive()
+                pc[w] += 1
+                progress = True
+        if pi >= len(producer) and all(x >= total for x in pc) and not inflight:
+            return "ok"
+        if not progress and not inflight:
+            lanes = (pending if pending is not None else producer[pi]) if pi < len(producer) else []
+            can = any(empty[p % stages].test_parity(((p // stages) & 1) ^ 1) for p in lanes)
+            can |= any(pc[x] < total and full[pc[x] % stages].test_parity((pc[x] // stages) & 1)
+                       for x in range(warps))
+            if not can:
+                return "deadlock"
+    return "did not finish"
+
+
+def _batches(seed):
+    r = random.Random(seed)
+    return [r.choice([1, 3, 32, 40, 64, 7, 128]) for _ in range(r.randint(1, 6))]
+
+
+@pytest.mark.parametrize("stages,warps", [(6, 2), (6, 4), (5, 3), (12, 1), (3, 4), (7, 8)])
+def test_broadcast_ring_is_safe_for_any_stage_count(stages, warps):
+    for seed in range(40):
+        assert simulate_broadcast(stages, warps, _batches(seed), seed) == "ok"
+
+
+def test_broadcast_ring_needs_every_warp_to_release():
+    """With an EMPTY count below the number of readers the producer refills a
+    slot that a warp has not read: the model must catch it."""
+    def broken(stages, warps, batches, seed):
+        orig = Barrier.__init__
+
+        def init(self, count):
+            orig(self, 1 if count == warps else count)
+        Barrier.__init__ = init
+        try:
+            return simulate_broadcast(stages, warps, batches, seed)
+        finally:
+            Barrier.__init__ = orig
+    results = [broken(6, 2, _batches(seed), seed) for seed in range(40)]
+    assert any(r != "ok" for r in results)
