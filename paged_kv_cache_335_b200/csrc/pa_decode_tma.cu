@@ -953,8 +953,15 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
 // Prefix Caching 不是同一件事; "PagedAttention原理详解：GPU显存优化与模型路由
 // 技术", § PagedAttention的三大核心优势 (point 2 and the beam-search paragraph).
 // ---------------------------------------------------------------------------
-#ifndef PA_GROUPED_RING_BYTES
-#define PA_GROUPED_RING_BYTES 49152
+
+// V fragments by ldmatrix.trans (head_dim in natural order in the accumulator)
+// rather than 16-byte loads plus byte permutes; independent accumulation
+// chains per QK product (the 8-long MMA chain is the kernel's critical path).
+#ifndef PA_GROUPED_LDSM_V
+#define PA_GROUPED_LDSM_V 1
+#endif
+#ifndef PA_GROUPED_QK_CHAINS
+#define PA_GROUPED_QK_CHAINS 2
 #endif
 
 constexpr int kMaxGroupSeqs = 8;            // members per group (header mask bits 0..7)
@@ -963,20 +970,50 @@ constexpr uint32_t kUnitLast = 1u << 31;    // header: last unit of the item
 constexpr int kUnitSubShift = 8;            // header bits 8..30: sub-tile index in the item
 constexpr uint32_t kUnitSubMask = 0x7fffffu;
 
-template <int D>
-using GroupedGeom = Geom<__nv_bfloat16, D, 1, PA_GROUPED_RING_BYTES>;
 
-// CTAs per SM each grouped variant is compiled for: as many as fit without
-// spilling (two n-tiles per warp at head_dim 128 need about 200 registers).
-// Up to PA_GROUPED_ONE_TILE_WARPS n-tiles, each consumer warp takes one (more
-// warps in flight); beyond that, two per warp (at most 4 consumer warps).
+// Ring bytes and CTAs per SM of each grouped variant (consumer warps CW,
+// n-tiles per warp NT), the measured best of ring / occupancy sweeps on the
+// beam workloads: the kernel is latency-bound per warp, so each variant runs
+// as many warps per SM as its ~168 registers allow (12), and four consumer
+// warps take a deeper ring. Two n-tiles per warp need about 240 registers at
+// head_dim 128. Overridable for sweeps.
 #ifndef PA_GROUPED_ONE_TILE_WARPS
 #define PA_GROUPED_ONE_TILE_WARPS 4
 #endif
+#ifndef PA_G_RING1
+#define PA_G_RING1 49152
+#endif
+#ifndef PA_G_BLK1
+#define PA_G_BLK1 4
+#endif
+#ifndef PA_G_RING2
+#define PA_G_RING2 49152
+#endif
+#ifndef PA_G_BLK2
+#define PA_G_BLK2 4
+#endif
+#ifndef PA_G_RING3
+#define PA_G_RING3 49152
+#endif
+#ifndef PA_G_BLK3
+#define PA_G_BLK3 3
+#endif
+#ifndef PA_G_RING4
+#define PA_G_RING4 65536
+#endif
+#ifndef PA_G_BLK4
+#define PA_G_BLK4 2
+#endif
+__host__ __device__ constexpr int grouped_ring_bytes(int cw, int nt) {
+    return nt != 1 ? 49152 : cw == 1 ? PA_G_RING1 : cw == 2 ? PA_G_RING2 : cw == 3 ? PA_G_RING3 : PA_G_RING4;
+}
 __host__ __device__ constexpr int grouped_min_blocks(int d, int cw, int nt) {
-    return nt == 1 ? (cw <= 2 ? 4 : 2)
+    return nt == 1 ? (cw == 1 ? PA_G_BLK1 : cw == 2 ? PA_G_BLK2 : cw == 3 ? PA_G_BLK3 : PA_G_BLK4)
                    : d == 64 ? (cw <= 1 ? 4 : cw == 2 ? 3 : 2) : (cw <= 1 ? 4 : cw <= 3 ? 2 : 1);
 }
+
+template <int D, int CW, int NT>
+using GroupedGeom = Geom<__nv_bfloat16, D, 1, grouped_ring_bytes(CW, NT)>;
 
 // Walk over a grouped CTA's items, u = blockIdx.x + k * gridDim.x, item u =
 // (partition u % P, kv head, group u / (P Hkv)). Lane l holds the context
@@ -1124,25 +1161,57 @@ __device__ __forceinline__ void mma_qk_n(uint32_t kb, const uint4 (&q)[NT][D / 3
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
         sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+#if PA_GROUPED_QK_CHAINS == 2
+        float sd[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int jp = 0; jp < KCH; ++jp) {
+            mma_16816(sc[j], kr[0][jp].x, kr[1][jp].x, kr[0][jp].y, kr[1][jp].y, q[j][jp].x, q[j][jp].y);
+            mma_16816(sd, kr[0][jp].z, kr[1][jp].z, kr[0][jp].w, kr[1][jp].w, q[j][jp].z, q[j][jp].w);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[j][e] += sd[e];
+#else
 #pragma unroll
         for (int jp = 0; jp < KCH; ++jp) {
             mma_16816(sc[j], kr[0][jp].x, kr[1][jp].x, kr[0][jp].y, kr[1][jp].y, q[j][jp].x, q[j][jp].y);
             mma_16816(sc[j], kr[0][jp].z, kr[1][jp].z, kr[0][jp].w, kr[1][jp].w, q[j][jp].z, q[j][jp].w);
         }
+#endif
+    }
+}
+
+// V^T A-fragments of m-tile t (head_dim 16t .. 16t+15, natural order) by
+// ldmatrix.trans: lane l addresses row l % 8 of matrix l / 8, i.e. token
+// 8 (i / 2) + l % 8, head_dim 16t + 8 (i % 2) .. + 7. Thread (r, c) then holds
+// A[r (+8)][tokens 2c, 2c+1 (+8)] as the m16n8k16 A operand wants.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&a)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(addr));
+}
+
+template <int D>
+__device__ __forceinline__ void ldsm_load_v(uint32_t vb, int lane, uint32_t (&va)[D / 16][4]) {
+    const int i = lane >> 3, row = 8 * (i >> 1) + (lane & 7);
+#pragma unroll
+    for (int t = 0; t < D / 16; ++t) {
+        const int d0 = 16 * t + 8 * (i & 1);
+        ldsm_x4_trans(vb + (d0 >> 6) * kBoxBytes + swz(row, (d0 & 63) >> 3), va[t]);
     }
 }
 
 // Online-softmax update for NT n-tiles whose columns may each see a different
 // number of valid tokens: nva / nvb = valid tokens of this thread's columns 2c
 // and 2c + 1 of n-tile j (0 for a column whose member does not use the unit).
-// A column that has seen no valid token keeps max -inf and weight 0.
+// A column that has seen no valid token keeps max -inf and weight 0. Leaves
+// the P^T B-fragments in pb0 / pb1 and returns the largest valid count of the
+// warp's columns (V rows from there on must be zeroed).
 template <int D, int NT>
-__device__ __forceinline__ void mma_softmax_pv_n(const float (&sc)[NT][4], uint4 (&vr)[4][D / 64],
-                                                 const int (&nva)[NT], const int (&nvb)[NT],
-                                                 float scale_log2, int r, int c,
-                                                 float (&acc)[NT][D / 16][4], float (&ma)[NT],
-                                                 float (&mb)[NT], float (&la)[NT], float (&lb)[NT]) {
-    constexpr int VCH = D / 64;
+__device__ __forceinline__ int softmax_update_n(const float (&sc)[NT][4], const int (&nva)[NT],
+                                                const int (&nvb)[NT], float scale_log2, int r,
+                                                float (&acc)[NT][D / 16][4], float (&ma)[NT],
+                                                float (&mb)[NT], float (&la)[NT], float (&lb)[NT],
+                                                uint32_t (&pb0)[NT], uint32_t (&pb1)[NT]) {
     constexpr int MT = D / 16;
     float s[NT][4], mxa[NT], mxb[NT];
     int nvmax = 0;
@@ -1172,7 +1241,6 @@ __device__ __forceinline__ void mma_softmax_pv_n(const float (&sc)[NT][4], uint4
         mv = mv || mxa[j] != ma[j] || mxb[j] != mb[j];
     }
     const bool moved = __any_sync(0xffffffffu, mv);
-    uint32_t pb0[NT], pb1[NT];
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
         const float ba = mxa[j] == -INFINITY ? 0.f : mxa[j];
@@ -1194,16 +1262,23 @@ __device__ __forceinline__ void mma_softmax_pv_n(const float (&sc)[NT][4], uint4
                 acc[j][t][3] *= alb;
             }
         }
-        pb0[j] = movmatrix_trans(x0);
-        pb1[j] = movmatrix_trans(x1);
+        pb0[j] = movmatrix_trans(x0);  // P^T rows (tokens) 2c, 2c+1; column r
+        pb1[j] = movmatrix_trans(x1);  // tokens 2c+8, 2c+9
     }
-    // Rows past every column's tokens are zeroed (those slots may hold
-    // anything); rows before it belong to some member's context.
-    nvmax = __reduce_max_sync(0xffffffffu, nvmax);
+    return __reduce_max_sync(0xffffffffu, nvmax);
+}
+
+// O^T += V^T . P^T from 16-byte V loads (head_dim order of mma_load_v). Rows
+// past every column's tokens are zeroed first (those slots may hold anything);
+// rows before that belong to some member's context.
+template <int D, int NT>
+__device__ __forceinline__ void pv_lds(uint4 (&vr)[4][D / 64], int nvmax, int c,
+                                       const uint32_t (&pb0)[NT], const uint32_t (&pb1)[NT],
+                                       float (&acc)[NT][D / 16][4]) {
     if (nvmax < 16) {
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int hh = 0; hh < VCH; ++hh) {
+        for (int hh = 0; hh < D / 64; ++hh) {
             if (2 * c >= nvmax) vr[0][hh] = z;
             if (2 * c + 1 >= nvmax) vr[1][hh] = z;
             if (2 * c + 8 >= nvmax) vr[2][hh] = z;
@@ -1211,7 +1286,7 @@ __device__ __forceinline__ void mma_softmax_pv_n(const float (&sc)[NT][4], uint4
         }
     }
 #pragma unroll
-    for (int t = 0; t < MT; ++t) {
+    for (int t = 0; t < D / 16; ++t) {
         const int hh = t >> 2, w = t & 3;
         const uint32_t xa = word(vr[0][hh], w), xb = word(vr[1][hh], w);
         const uint32_t ya = word(vr[2][hh], w), yb = word(vr[3][hh], w);
@@ -1220,6 +1295,29 @@ __device__ __forceinline__ void mma_softmax_pv_n(const float (&sc)[NT][4], uint4
 #pragma unroll
         for (int j = 0; j < NT; ++j) mma_16816(acc[j][t], a0, a1, a2, a3, pb0[j], pb1[j]);
     }
+}
+
+// O^T += V^T . P^T from ldmatrix.trans fragments (natural head_dim order):
+// a0 / a1 hold tokens 2c, 2c+1, a2 / a3 tokens 2c+8, 2c+9, low half first.
+template <int D, int NT>
+__device__ __forceinline__ void pv_ldsm(uint32_t (&va)[D / 16][4], int nvmax, int c,
+                                        const uint32_t (&pb0)[NT], const uint32_t (&pb1)[NT],
+                                        float (&acc)[NT][D / 16][4]) {
+    if (nvmax < 16) {
+        const uint32_t m01 = (2 * c < nvmax ? 0x0000ffffu : 0u) | (2 * c + 1 < nvmax ? 0xffff0000u : 0u);
+        const uint32_t m89 = (2 * c + 8 < nvmax ? 0x0000ffffu : 0u) | (2 * c + 9 < nvmax ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int t = 0; t < D / 16; ++t) {
+            va[t][0] &= m01;
+            va[t][1] &= m01;
+            va[t][2] &= m89;
+            va[t][3] &= m89;
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < D / 16; ++t)
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma_16816(acc[j][t], va[t][0], va[t][1], va[t][2], va[t][3], pb0[j], pb1[j]);
 }
 
 // Store one column's result (m, l = its running max and summed weights): bf16
@@ -1233,6 +1331,20 @@ __device__ __forceinline__ void grouped_store_col(const DecodeParams& p, int64_t
     const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
+#if PA_GROUPED_LDSM_V
+        // rows r and r + 8 of m-tile t: head_dim 16t + r and 16t + 8 + r
+        const int d0 = 16 * t + r, d1 = d0 + 8;
+        if (P == 1) {
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + row * D;
+            o[d0] = __float2bfloat16_rn(acc[t][e] * inv);
+            o[d1] = __float2bfloat16_rn(acc[t][e + 2] * inv);
+        } else {
+            float* o = p.ws_o + (row * P + part) * D;
+            o[d0] = acc[t][e] * inv;
+            o[d1] = acc[t][e + 2] * inv;
+        }
+#else
+        // rows r and r + 8 of m-tile t: head_dim d0 and d0 + 1
         const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
         if (P == 1)
             *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + row * D + d0) =
@@ -1240,6 +1352,7 @@ __device__ __forceinline__ void grouped_store_col(const DecodeParams& p, int64_t
         else
             *reinterpret_cast<float2*>(p.ws_o + (row * P + part) * D + d0) =
                 make_float2(acc[t][e] * inv, acc[t][e + 2] * inv);
+#endif
     }
     if (P > 1 && r == 0) {
         float* ml = p.ws_ml + (row * P + part) * 2;
@@ -1253,7 +1366,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, grouped_min_blocks(D, CW, NT))
 decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                           const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
                           int num_items, int gs) {
-    using G = GroupedGeom<D>;
+    using G = GroupedGeom<D, CW, NT>;
     constexpr int KCH = D / 32;
     constexpr int VCH = D / 64;
     constexpr int MT = D / 16;
@@ -1383,10 +1496,18 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                 const int tok0 = cur.t0 + (int)((h >> kUnitSubShift) & kUnitSubMask) * 16;
                 const uint32_t kb = ring.stages + st * G::kStageBytes;
                 float sc[NT][4];
+#if PA_GROUPED_LDSM_V
+                uint32_t va[MT][4];
+#else
                 uint4 vr[4][VCH];
+#endif
                 if (mine) {
                     mma_qk_n<D, NT>(kb, q, r, c, sc);
+#if PA_GROUPED_LDSM_V
+                    ldsm_load_v<D>(kb + G::kBoxes * kBoxBytes, lane, va);
+#else
                     mma_load_v<D>(kb + G::kBoxes * kBoxBytes, r, c, vr);
+#endif
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
@@ -1398,7 +1519,14 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                         nva[j] = (h & bita[j]) ? min(16, t1a[j] - tok0) : 0;
                         nvb[j] = (h & bitb[j]) ? min(16, t1b[j] - tok0) : 0;
                     }
-                    mma_softmax_pv_n<D, NT>(sc, vr, nva, nvb, p.scale_log2, r, c, acc, ma, mb, la, lb);
+                    uint32_t pb0[NT], pb1[NT];
+                    const int nvmax = softmax_update_n<D, NT>(sc, nva, nvb, p.scale_log2, r, acc, ma,
+                                                              mb, la, lb, pb0, pb1);
+#if PA_GROUPED_LDSM_V
+                    pv_ldsm<D, NT>(va, nvmax, c, pb0, pb1, acc);
+#else
+                    pv_lds<D, NT>(vr, nvmax, c, pb0, pb1, acc);
+#endif
                 }
                 if (h & kUnitLast) break;
             }
@@ -1483,7 +1611,7 @@ cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUt
 template <int D, int CW, int NT>
 cudaError_t launch_grouped_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
                              int gs, cudaStream_t stream) {
-    using G = GroupedGeom<D>;
+    using G = GroupedGeom<D, CW, NT>;
     constexpr size_t smem = smem_bytes<G>(G::kStages * 4);
     constexpr int kThreads = (CW + 1) * 32;
     auto kernel = decode_tma_grouped_kernel<D, CW, NT>;
