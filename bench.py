@@ -351,6 +351,53 @@ def time_steps(step, steps, warmup, flush, barrier=None):
             "wall": (t_wall0, t_wall1)}
 
 
+def swap_bandwidth(device, blocks=1024, reps=5):
+    """pa_block_swap of `blocks` scattered blocks of the 13B pool shape (40 kv heads
+    x 16 slots x 128 dims, bf16: 160 KiB per block per cache) to a pinned host pool
+    and back, next to the copy engine moving one contiguous buffer of the same size."""
+    import torch
+
+    import paged_kv_cache_335_b200 as pa
+    shape = (40, 16, 128)
+    dev_blocks, host_blocks = 2 * blocks + 64, blocks + 16
+    kd = torch.randn((dev_blocks,) + shape, device=device).to(torch.bfloat16)
+    vd = torch.randn((dev_blocks,) + shape, device=device).to(torch.bfloat16)
+    kh = torch.empty((host_blocks,) + shape, dtype=torch.bfloat16).pin_memory()
+    vh = torch.empty((host_blocks,) + shape, dtype=torch.bfloat16).pin_memory()
+    g = torch.Generator().manual_seed(5)
+    src = torch.randperm(dev_blocks, generator=g)[:blocks]
+    dst = torch.randperm(host_blocks, generator=g)[:blocks]
+    out_pairs = torch.stack([src, dst], 1).to(device)
+    in_pairs = torch.stack([dst, torch.randperm(dev_blocks, generator=g)[:blocks]], 1).to(device)
+    nbytes = 2 * blocks * kd[0].numel() * kd.element_size()
+    flat_d = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=device)
+    flat_h = torch.empty(nbytes // 2, dtype=torch.bfloat16).pin_memory()
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 1):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if i:
+                ts.append(e0.elapsed_time(e1) / 1e3)
+        return nbytes / statistics.median(ts) / 1e9
+
+    res = {
+        "blocks": blocks, "bytes_per_direction": nbytes,
+        "out_gbs": round(timed(lambda: pa.pa_block_swap(out_pairs, kd, vd, kh, vh)), 1),
+        "in_gbs": round(timed(lambda: pa.pa_block_swap(in_pairs, kh, vh, kd, vd)), 1),
+        "copy_engine_d2h_gbs": round(timed(lambda: flat_h.copy_(flat_d, non_blocking=True)), 1),
+        "copy_engine_h2d_gbs": round(timed(lambda: flat_d.copy_(flat_h, non_blocking=True)), 1),
+    }
+    pa.pa_sync_check()
+    del kd, vd, kh, vh, flat_d, flat_h
+    torch.cuda.empty_cache()
+    return res
+
+
 def e2e_steps(step, steps, warmup):
     """The same step through the Python binding of the C ABI with inputs in
     pinned HOST memory: H2D of the step's inputs and D2H of the output are
@@ -596,6 +643,7 @@ def main():
             st.release()
             del st
             torch.cuda.empty_cache()
+        per_config["swap_llama13b_blocks"] = swap_bandwidth(device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

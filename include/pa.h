@@ -8,6 +8,7 @@
  *                  table gathers from fixed-size physical blocks
  *   pa_block_copy  copy whole physical blocks (copy-on-write at a fork)
  *
+ * plus pa_block_swap (blocks between a device pool and a pinned host pool),
  * and pa_decode_grouped, pa_decode for groups of sequences that share blocks
  * (beams, parallel samples), which reads each shared block once per group.
  *
@@ -248,6 +249,35 @@ int pa_decode_grouped_num_partitions(int32_t num_seqs, int32_t num_heads,
 int pa_block_copy(const int64_t* src_dst_pairs, int32_t num_pairs,
                   void* k_cache, void* v_cache, const pa_cache_desc* cache,
                   void* stream);
+
+/*
+ * pa_block_swap — copy whole blocks from one pool into another pool of the
+ * same block shape, where either pool may live in pinned host memory: the
+ * swap-out of a preempted request's blocks to host memory and their swap-in
+ * when it resumes ([P2 § 生产环境 monitoring list]: the frequency and latency
+ * of CPU offload or swap are among the signals a deployment watches; the
+ * pages give no more).
+ *
+ * For every pair p: block dst = src_dst_pairs[2p+1] of the destination pool
+ * receives all slots of all kv heads of block src = src_dst_pairs[2p] of the
+ * source pool, in both caches, bit for bit.
+ *   src_dst_pairs  device (or mapped pinned host) int64 [num_pairs][2].
+ *   src_k, src_v   the source pool, `src` its shape; dst_k, dst_v and `dst`
+ *                  the destination. num_kv_heads, block_size, head_dim and
+ *                  dtype must agree; num_blocks may differ. Each pointer is
+ *                  device memory or pinned host memory (cudaHostAlloc, or
+ *                  cudaHostRegister'ed) that the device can address; pageable
+ *                  host memory returns PA_ERR_INVALID_ARG.
+ * The two pools must not overlap (within one pool use pa_block_copy), and dst
+ * ids must be distinct within a call. Ids outside their pool are skipped and
+ * recorded as PA_ERR_BAD_INDEX. The copy runs on the SMs (one launch for any
+ * number of scattered blocks), reading and writing host memory over the host
+ * link; the host pool must not be touched by the CPU until the stream passes
+ * the call.
+ */
+int pa_block_swap(const int64_t* src_dst_pairs, int32_t num_pairs,
+                  const void* src_k, const void* src_v, const pa_cache_desc* src,
+                  void* dst_k, void* dst_v, const pa_cache_desc* dst, void* stream);
 
 /*
  * PA_NOALLOC_SCRATCH_BYTES — size of the device buffer inside the library that

@@ -52,9 +52,10 @@ def _bind(path: str):
     p, i32 = ctypes.c_void_p, ctypes.c_int32
     lib.oracle_kv_append.argtypes = [p, p, p, i32, p, p, i32, i32, i32, i32, i32]
     lib.oracle_block_copy.argtypes = [p, i32, p, p, i32, i32, i32, i32, i32]
+    lib.oracle_block_swap.argtypes = [p, i32, p, p, i32, p, p, i32, i32, i32, i32, i32]
     lib.oracle_decode.argtypes = [p, p, p, p, p, i32, p, i32, i32, i32, i32, i32,
                                   i32, i32, ctypes.c_float, i32]
-    for f in (lib.oracle_kv_append, lib.oracle_block_copy, lib.oracle_decode,
+    for f in (lib.oracle_kv_append, lib.oracle_block_copy, lib.oracle_block_swap, lib.oracle_decode,
               lib.oracle_max_threads):
         f.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
@@ -151,6 +152,25 @@ def block_copy(pairs: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray) -> N
     rc = _load().oracle_block_copy(_ptr(pairs), pairs.shape[0], _ptr(k_cache), _ptr(v_cache),
                                    nb, hkv, bs, d, _dtype_code(k_cache))
     _check(rc, "block_copy")
+
+
+def block_swap(pairs: np.ndarray, src_k: np.ndarray, src_v: np.ndarray, dst_k: np.ndarray,
+               dst_v: np.ndarray) -> None:
+    """In place on dst: for every (src, dst) row of ``pairs`` copy block src of the
+    source pool to block dst of the destination pool (same block shape)."""
+    src_k = _contig(src_k)
+    src_v = _contig(src_v, src_k.dtype)
+    dst_k = _contig(dst_k, src_k.dtype)
+    dst_v = _contig(dst_v, src_k.dtype)
+    if src_k.shape[1:] != dst_k.shape[1:] or src_v.shape != src_k.shape or \
+            dst_v.shape != dst_k.shape:
+        raise ValueError("the pools differ in block shape")
+    pairs = _contig(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+    _, hkv, bs, d = src_k.shape
+    rc = _load().oracle_block_swap(_ptr(pairs), pairs.shape[0], _ptr(src_k), _ptr(src_v),
+                                   src_k.shape[0], _ptr(dst_k), _ptr(dst_v), dst_k.shape[0],
+                                   hkv, bs, d, _dtype_code(src_k))
+    _check(rc, "block_swap")
 
 
 def decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,

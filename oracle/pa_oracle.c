@@ -128,6 +128,36 @@ int oracle_block_copy(const int64_t* pairs, int32_t num_pairs, void* k_cache,
 }
 
 /*
+ * Swap of whole blocks between two pools of one block shape ([P2] § 生产环境
+ * monitoring list: CPU offload / swap of KV blocks): every pair (src, dst)
+ * gives block dst of the destination pool the full contents of block src of
+ * the source pool, K and V. The pools are distinct memory, so the pairs are
+ * independent copies.
+ */
+int oracle_block_swap(const int64_t* pairs, int32_t num_pairs, const void* src_k,
+                      const void* src_v, int32_t src_blocks, void* dst_k, void* dst_v,
+                      int32_t dst_blocks, int32_t num_kv_heads, int32_t block_size,
+                      int32_t head_dim, int32_t dtype) {
+    if (num_pairs < 0 || !shape_ok(src_blocks, num_kv_heads, block_size, head_dim, dtype) ||
+        !shape_ok(dst_blocks, num_kv_heads, block_size, head_dim, dtype))
+        return OR_ERR_ARG;
+    const size_t block_bytes =
+        (size_t)num_kv_heads * block_size * head_dim * elem_bytes(dtype);
+    for (int32_t p = 0; p < num_pairs; ++p) {
+        if (pairs[2 * p] < 0 || pairs[2 * p] >= src_blocks || pairs[2 * p + 1] < 0 ||
+            pairs[2 * p + 1] >= dst_blocks)
+            return OR_ERR_INDEX;
+    }
+    for (int32_t p = 0; p < num_pairs; ++p) {
+        const size_t from = (size_t)pairs[2 * p] * block_bytes;
+        const size_t to = (size_t)pairs[2 * p + 1] * block_bytes;
+        memcpy((char*)dst_k + to, (const char*)src_k + from, block_bytes);
+        memcpy((char*)dst_v + to, (const char*)src_v + from, block_bytes);
+    }
+    return OR_OK;
+}
+
+/*
  * Decode attention for one (sequence, query head), straight from the
  * definition: gather the n logical K and V vectors through the block table
  * ([P2] block-table example: logical block j -> physical table[j]), then

@@ -95,6 +95,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_decode_grouped_workspace_size.restype = sz
         lib.pa_decode_grouped_num_partitions.argtypes = [i32, i32, i32, desc, i32, i32]
         lib.pa_block_copy.argtypes = [vp, i32, vp, vp, desc, vp]
+        lib.pa_block_swap.argtypes = [vp, i32, vp, vp, desc, vp, vp, desc, vp]
         lib.pa_sync_check.argtypes = [vp]
         lib.pa_stream_read.argtypes = [vp, sz, vp, i32, vp]
         lib.pa_test_skip_load.argtypes = [i32]
@@ -159,6 +160,15 @@ def _dev(t, name: str, dtype=None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _addressable(t, name: str):
+    """A CUDA tensor or a pinned host tensor (which the device addresses directly)."""
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
 def _stream(stream):
     torch = _torch()
     if stream is None:
@@ -207,6 +217,24 @@ def pa_block_copy(src_dst_pairs, k_cache, v_cache, stream=None) -> None:
     _check(load_library().pa_block_copy(
         _dev(src_dst_pairs, "src_dst_pairs", torch.int64), int(src_dst_pairs.shape[0]),
         _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), ctypes.byref(desc), _stream(stream)))
+
+
+def pa_block_swap(src_dst_pairs, src_k, src_v, dst_k, dst_v, stream=None) -> None:
+    """Copy whole blocks between two pools of the same block shape (swap-out to /
+    swap-in from pinned host memory): for each (src, dst) row of ``src_dst_pairs``
+    (int64 [P][2], on the device), block dst of (dst_k, dst_v) gets block src of
+    (src_k, src_v). Either pool may be a CUDA tensor or a pinned host tensor."""
+    torch = _torch()
+    _same_pool(src_k, src_v)
+    _same_pool(dst_k, dst_v)
+    sd, dd = cache_desc(src_k), cache_desc(dst_k)
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [num_pairs][2]")
+    _check(load_library().pa_block_swap(
+        _dev(src_dst_pairs, "src_dst_pairs", torch.int64), int(src_dst_pairs.shape[0]),
+        _addressable(src_k, "src_k"), _addressable(src_v, "src_v"), ctypes.byref(sd),
+        _addressable(dst_k, "dst_k"), _addressable(dst_v, "dst_v"), ctypes.byref(dd),
+        _stream(stream)))
 
 
 def pa_decode_workspace_size(num_seqs: int, num_heads: int, max_context_len: int, k_cache,
@@ -345,5 +373,5 @@ def pa_sync_check(stream=None) -> None:
 
 __all__ = ["pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_block_copy", "pa_decode_workspace_size",
            "pa_decode_num_partitions", "pa_decode_grouped", "pa_decode_grouped_workspace_size",
-           "pa_decode_grouped_num_partitions", "pa_sync_check", "pa_cache_desc", "cache_desc",
+           "pa_decode_grouped_num_partitions", "pa_block_swap", "pa_sync_check", "pa_cache_desc", "cache_desc",
            "load_library", "header_functions", "PAError"]

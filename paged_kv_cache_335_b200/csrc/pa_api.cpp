@@ -357,6 +357,62 @@ int pa_block_copy(const int64_t* src_dst_pairs, int32_t num_pairs, void* k_cache
     return e == cudaSuccess ? PA_OK : fail_cuda(e, "pa_block_copy launch");
 }
 
+int pa_block_swap(const int64_t* src_dst_pairs, int32_t num_pairs, const void* src_k,
+                  const void* src_v, const pa_cache_desc* src, void* dst_k, void* dst_v,
+                  const pa_cache_desc* dst, void* stream) {
+    int rc = check_cache(src);
+    if (rc != PA_OK) return rc;
+    if ((rc = check_cache(dst)) != PA_OK) return rc;
+    if (src->num_kv_heads != dst->num_kv_heads || src->block_size != dst->block_size ||
+        src->head_dim != dst->head_dim || src->dtype != dst->dtype)
+        return fail(PA_ERR_INVALID_ARG, "pa_block_swap: the two pools differ in block shape or dtype");
+    if (num_pairs < 0) return fail(PA_ERR_INVALID_ARG, "num_pairs %d is negative", num_pairs);
+    if (num_pairs == 0) return PA_OK;
+    if (!src_dst_pairs || !src_k || !src_v || !dst_k || !dst_v)
+        return fail(PA_ERR_INVALID_ARG, "pa_block_swap: NULL pointer argument");
+    if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v))
+        return fail(PA_ERR_ALIGN, "pa_block_swap: the pools must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(src_dst_pairs) & 7u) != 0)
+        return fail(PA_ERR_ALIGN, "pa_block_swap: src_dst_pairs must be 8-byte aligned");
+    const size_t block_bytes =
+        (size_t)src->num_kv_heads * src->block_size * src->head_dim * elem_bytes(src->dtype);
+    const char* sk = static_cast<const char*>(src_k);
+    const char* dk = static_cast<const char*>(dst_k);
+    const size_t sbytes = block_bytes * (size_t)src->num_blocks;
+    const size_t dbytes = block_bytes * (size_t)dst->num_blocks;
+    const char* sv = static_cast<const char*>(src_v);
+    const char* dv = static_cast<const char*>(dst_v);
+    auto overlap = [](const char* a, size_t na, const char* b, size_t nb) {
+        return a < b + nb && b < a + na;
+    };
+    if (overlap(sk, sbytes, dk, dbytes) || overlap(sk, sbytes, dv, dbytes) ||
+        overlap(sv, sbytes, dk, dbytes) || overlap(sv, sbytes, dv, dbytes) ||
+        overlap(dk, dbytes, dv, dbytes))
+        return fail(PA_ERR_INVALID_ARG, "pa_block_swap: destination caches overlap each other "
+                    "or the source pool");
+    // every pointer must be addressable by the device: device, managed or pinned host memory
+    const void* ptrs[5] = {src_dst_pairs, src_k, src_v, dst_k, dst_v};
+    const void* dev[5];
+    const char* names[5] = {"src_dst_pairs", "src_k", "src_v", "dst_k", "dst_v"};
+    for (int i = 0; i < 5; ++i) {
+        cudaPointerAttributes a;
+        cudaError_t e = cudaPointerGetAttributes(&a, ptrs[i]);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return fail(PA_ERR_INVALID_ARG, "pa_block_swap: %s is not CUDA-visible memory", names[i]);
+        }
+        if (a.type == cudaMemoryTypeUnregistered || a.devicePointer == nullptr)
+            return fail(PA_ERR_INVALID_ARG, "pa_block_swap: %s is pageable host memory; pin it "
+                        "(cudaHostAlloc / cudaHostRegister)", names[i]);
+        dev[i] = a.devicePointer;
+    }
+    cudaError_t e = pa::launch_block_swap(static_cast<const int64_t*>(dev[0]), num_pairs, dev[1],
+                                          dev[2], src->num_blocks, const_cast<void*>(dev[3]),
+                                          const_cast<void*>(dev[4]), dst->num_blocks,
+                                          copy_params(src), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : fail_cuda(e, "pa_block_swap launch");
+}
+
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t max_context_len,
                                 const pa_cache_desc* cache, int32_t partition_size) {
     Plan plan;

@@ -79,7 +79,63 @@ block_copy_kernel(const int64_t* __restrict__ pairs, uint4* __restrict__ k_cache
     }
 }
 
+// Swap between two pools of the same block shape, either of which may be
+// pinned host memory mapped into the device address space (swap-out to host
+// when a request is preempted, swap-in when it resumes; "AI 推理系列（十六）：
+// PagedAttention——…", § 生产环境 signals: CPU offload / swap frequency and
+// latency). grid = (chunks of one block, pairs, 2 = {K, V}); the SMs move the
+// data over the host link with plain 16-byte loads and stores, many in flight
+// per thread, so one launch carries any number of scattered blocks.
+constexpr int kSwapUnroll = 8;
+
+__global__ void __launch_bounds__(kThreads)
+block_swap_kernel(const int64_t* __restrict__ pairs, const uint4* __restrict__ src_k,
+                  const uint4* __restrict__ src_v, uint4* __restrict__ dst_k,
+                  uint4* __restrict__ dst_v, int64_t vecs_per_block, int32_t src_blocks,
+                  int32_t dst_blocks) {
+    const int64_t src = __ldg(pairs + 2 * (int64_t)blockIdx.y);
+    const int64_t dst = __ldg(pairs + 2 * (int64_t)blockIdx.y + 1);
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+        if (threadIdx.x == 0) atomicOr(&s_status_copy, kStatusBadIndex);
+        return;
+    }
+    const uint4* s = (blockIdx.z ? src_v : src_k) + src * vecs_per_block;
+    uint4* d = (blockIdx.z ? dst_v : dst_k) + dst * vecs_per_block;
+    const int64_t start = (int64_t)blockIdx.x * (kThreads * kSwapUnroll) + threadIdx.x;
+    uint4 tmp[kSwapUnroll];
+#pragma unroll
+    for (int i = 0; i < kSwapUnroll; ++i) {
+        const int64_t idx = start + i * kThreads;
+        if (idx < vecs_per_block) tmp[i] = ld_v4(s + idx);
+    }
+#pragma unroll
+    for (int i = 0; i < kSwapUnroll; ++i) {
+        const int64_t idx = start + i * kThreads;
+        if (idx < vecs_per_block) d[idx] = tmp[i];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_block_swap(const int64_t* pairs, int32_t num_pairs, const void* src_k,
+                              const void* src_v, int32_t src_blocks, void* dst_k, void* dst_v,
+                              int32_t dst_blocks, const CopyParams& cp, cudaStream_t stream) {
+    if (num_pairs == 0) return cudaSuccess;
+    const int64_t vecs = (int64_t)cp.num_kv_heads * cp.block_size * cp.row_vecs;
+    const int64_t chunks = (vecs + kThreads * kSwapUnroll - 1) / (kThreads * kSwapUnroll);
+    constexpr int32_t kMaxGridY = 65535;
+    for (int32_t first = 0; first < num_pairs; first += kMaxGridY) {
+        const int32_t n = num_pairs - first < kMaxGridY ? num_pairs - first : kMaxGridY;
+        dim3 grid((unsigned)chunks, (unsigned)n, 2);
+        block_swap_kernel<<<grid, kThreads, 0, stream>>>(
+            pairs + 2 * (int64_t)first, static_cast<const uint4*>(src_k),
+            static_cast<const uint4*>(src_v), static_cast<uint4*>(dst_k),
+            static_cast<uint4*>(dst_v), vecs, src_blocks, dst_blocks);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
 
 cudaError_t launch_kv_append(const void* k, const void* v, const int64_t* slot_mapping,
                              int32_t num_tokens, void* k_cache, void* v_cache,

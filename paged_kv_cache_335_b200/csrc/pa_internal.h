@@ -56,6 +56,11 @@ cudaError_t launch_kv_append(const void* k, const void* v, const int64_t* slot_m
                              const CopyParams& cp, cudaStream_t stream);
 cudaError_t launch_block_copy(const int64_t* pairs, int32_t num_pairs, void* k_cache,
                               void* v_cache, const CopyParams& cp, cudaStream_t stream);
+// Blocks of one pool into another of the same block shape (either may be
+// mapped pinned host memory); block ids checked against each pool's size.
+cudaError_t launch_block_swap(const int64_t* pairs, int32_t num_pairs, const void* src_k,
+                              const void* src_v, int32_t src_blocks, void* dst_k, void* dst_v,
+                              int32_t dst_blocks, const CopyParams& cp, cudaStream_t stream);
 
 // Which decode kernel a call uses: the tensor-core GQA consumer for bf16 with
 // a query group of 2..8, the CUDA-core consumer otherwise.

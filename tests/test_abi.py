@@ -119,6 +119,26 @@ def test_grouped_decode_rejects_bad_group_size(lib):
         assert b"group_size" in lib.pa_get_last_error()
 
 
+def test_swap_rejects_bad_arguments(lib):
+    p = ctypes.c_void_p(256)
+    a, b = _desc(num_blocks=8), _desc(num_blocks=4)
+    assert lib.pa_block_swap(p, 0, p, p, ctypes.byref(a), p, p, ctypes.byref(b), None) == pa.PA_OK
+    assert lib.pa_block_swap(p, -1, p, p, ctypes.byref(a), p, p, ctypes.byref(b), None) \
+        == pa.PA_ERR_INVALID_ARG
+    c = _desc(num_blocks=4, head_dim=64)
+    assert lib.pa_block_swap(p, 1, p, p, ctypes.byref(a), p, p, ctypes.byref(c), None) \
+        == pa.PA_ERR_INVALID_ARG                                    # block shapes differ
+    assert lib.pa_block_swap(None, 1, p, p, ctypes.byref(a), p, p, ctypes.byref(b), None) \
+        == pa.PA_ERR_INVALID_ARG
+    q = ctypes.c_void_p(1 << 20)
+    assert lib.pa_block_swap(p, 1, p, p, ctypes.byref(a), q, q, ctypes.byref(b), None) \
+        == pa.PA_ERR_INVALID_ARG                                    # dst_k == dst_v overlaps
+    assert b"overlap" in lib.pa_get_last_error()
+    assert lib.pa_block_swap(p, 1, p, ctypes.c_void_p(8 << 20), ctypes.byref(a),
+                             ctypes.c_void_p(1 << 30), ctypes.c_void_p(3 << 20),
+                             ctypes.byref(b), None) == pa.PA_ERR_INVALID_ARG   # src_k overlaps dst_v
+
+
 def test_append_and_copy_reject_bad_arguments(lib):
     p = ctypes.c_void_p(16)
     assert lib.pa_kv_append(p, p, p, -1, p, p, ctypes.byref(_desc()), None) == pa.PA_ERR_INVALID_ARG

@@ -367,3 +367,38 @@ def test_tiny_workload_step_matches_sdpa():
     ref = _sdpa_reference(W.to_numpy(vals["q"]).astype(np.float64), K, V, wl.context_lens,
                           wl.scale, wl.num_kv_heads)
     np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# swap between pools
+# ---------------------------------------------------------------------------
+def test_block_swap_equals_indexed_assignment():
+    """Swap out / in against numpy's own indexed assignment (a library routine)."""
+    rng = np.random.default_rng(7)
+    dev_k = rng.standard_normal((11, 3, 16, 8)).astype(np.float32)
+    dev_v = rng.standard_normal((11, 3, 16, 8)).astype(np.float32)
+    host_k = np.full((6, 3, 16, 8), np.nan, np.float32)
+    host_v = np.full((6, 3, 16, 8), np.nan, np.float32)
+    pairs = np.array([[9, 0], [2, 5], [4, 3]], np.int64)
+    want_k, want_v = host_k.copy(), host_v.copy()
+    want_k[pairs[:, 1]] = dev_k[pairs[:, 0]]
+    want_v[pairs[:, 1]] = dev_v[pairs[:, 0]]
+    oracle.block_swap(pairs, dev_k, dev_v, host_k, host_v)
+    assert want_k.view(np.uint32).tobytes() == host_k.view(np.uint32).tobytes()
+    assert want_v.view(np.uint32).tobytes() == host_v.view(np.uint32).tobytes()
+    # round trip into fresh device blocks restores every bit
+    back = np.array([[0, 1], [5, 6], [3, 10]], np.int64)
+    k2, v2 = dev_k.copy(), dev_v.copy()
+    oracle.block_swap(back, host_k, host_v, k2, v2)
+    for (s, _), (_, d) in zip(pairs, back):
+        assert k2[d].tobytes() == dev_k[s].tobytes() and v2[d].tobytes() == dev_v[s].tobytes()
+
+
+def test_block_swap_rejects_bad_ids_and_shapes():
+    a = np.zeros((4, 2, 16, 8), np.float32)
+    b = np.zeros((2, 2, 16, 8), np.float32)
+    with pytest.raises(oracle.OracleError):
+        oracle.block_swap(np.array([[3, 2]]), a, a.copy(), b, b.copy())     # dst 2 of 2
+    with pytest.raises(ValueError):
+        oracle.block_swap(np.array([[0, 0]]), a, a.copy(), np.zeros((2, 2, 16, 4), np.float32),
+                          np.zeros((2, 2, 16, 4), np.float32))
