@@ -44,7 +44,8 @@ EXTRA_CONFIGS = [("llama7b", "llama7b", None, 1), ("llama13b_bs16", "llama13b_bs
                  ("llama13b_bs32", "llama13b_bs32", None, 1),
                  ("llama70b_gqa", "llama70b_gqa", None, 1),
                  ("llama70b_gqa_policy", "llama70b_gqa", 0, 1), ("cow_beam4", "cow_beam4", None, 1),
-                 ("cow_beam4_grouped", "cow_beam4", 0, 4)]
+                 ("cow_beam4_grouped", "cow_beam4", 0, 4),
+                 ("llama70b_verify4", "llama70b_verify4", 0, 1)]
 # pa_test_last_decode_kernel() -> the decode kernel a call enqueued
 KERNEL_NAMES = {0: "decode_tma_simt_kernel (CUDA-core)",
                 1: "decode_tma_mma_kernel (persistent, tensor-core GQA)",
@@ -255,10 +256,20 @@ class Step:
         self.desc = pa.cache_desc(v["k_cache"])
         self.ps = wl.partition_size if partition_size is None else partition_size
         self.group_size = group_size
-        self.num_partitions = pa.pa_decode_grouped_num_partitions(
-            wl.num_seqs, wl.num_heads, wl.max_context_len, v["k_cache"], group_size, self.ps)
-        need = pa.pa_decode_grouped_workspace_size(wl.num_seqs, wl.num_heads, wl.max_context_len,
-                                                   v["k_cache"], group_size, self.ps)
+        self.multi = wl.query_start is not None
+        if self.multi:
+            self.query_start = torch.as_tensor(wl.query_start, device=device)
+            self.num_partitions = pa.pa_decode_multi_num_partitions(
+                wl.num_seqs, wl.num_query_rows, wl.max_query_len, wl.num_heads,
+                wl.max_context_len, v["k_cache"], self.ps)
+            need = pa.pa_decode_multi_workspace_size(
+                wl.num_seqs, wl.num_query_rows, wl.max_query_len, wl.num_heads,
+                wl.max_context_len, v["k_cache"], self.ps)
+        else:
+            self.num_partitions = pa.pa_decode_grouped_num_partitions(
+                wl.num_seqs, wl.num_heads, wl.max_context_len, v["k_cache"], group_size, self.ps)
+            need = pa.pa_decode_grouped_workspace_size(
+                wl.num_seqs, wl.num_heads, wl.max_context_len, v["k_cache"], group_size, self.ps)
         self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
         self.ws_bytes = need
         self.stream = torch.cuda.current_stream(device)
@@ -278,6 +289,16 @@ class Step:
             ((group_size,) if group_size > 1 else ()) + \
             (self.ps, P(self.ws.data_ptr()), ctypes.c_size_t(self.ws_bytes), self.sp)
         self.decode_fn = self.lib.pa_decode_grouped if group_size > 1 else self.lib.pa_decode
+        if self.multi:
+            self.args_decode = (P(self.out.data_ptr()), P(v["q"].data_ptr()),
+                                P(v["k_cache"].data_ptr()), P(v["v_cache"].data_ptr()),
+                                P(self.tables.data_ptr()), int(self.tables.shape[1]),
+                                P(self.ctx.data_ptr()), P(self.query_start.data_ptr()),
+                                wl.max_context_len, wl.num_seqs, wl.num_query_rows,
+                                wl.max_query_len, wl.num_heads, ctypes.c_float(wl.scale),
+                                ctypes.byref(self.desc), self.ps, P(self.ws.data_ptr()),
+                                ctypes.c_size_t(self.ws_bytes), self.sp)
+            self.decode_fn = self.lib.pa_decode_multi
         self.has_copy = wl.copy_pairs.shape[0] > 0
         self.has_append = wl.num_tokens > 0
         self.launches_per_step = (self.num_partitions > 1) + 1 + int(self.has_append) + \
@@ -409,6 +430,8 @@ def e2e_steps(step, steps, warmup):
             "v_new": v["v_new"].cpu().pin_memory(),
             "tables": step.tables.cpu().pin_memory(), "ctx": step.ctx.cpu().pin_memory(),
             "slots": step.slots.cpu().pin_memory(), "pairs": step.pairs.cpu().pin_memory()}
+    if step.multi:
+        host["query_start"] = step.query_start.cpu().pin_memory()
     dev = {k: torch.empty_like(t, device=v["q"].device) for k, t in host.items()}
     out_host = torch.empty_like(step.out, device="cpu").pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -421,9 +444,21 @@ def e2e_steps(step, steps, warmup):
             pa.pa_block_copy(dev["pairs"], v["k_cache"], v["v_cache"])
         if wl.num_tokens:
             pa.pa_kv_append(dev["k_new"], dev["v_new"], dev["slots"], v["k_cache"], v["v_cache"])
-        pa.pa_decode(step.out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"], dev["ctx"],
-                     wl.scale, max_context_len=wl.max_context_len, partition_size=step.ps,
-                     workspace=step.ws)
+        if step.multi:
+            pa.pa_decode_multi(step.out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"],
+                               dev["ctx"], dev["query_start"], wl.scale,
+                               max_context_len=wl.max_context_len,
+                               max_query_len=wl.max_query_len, partition_size=step.ps,
+                               workspace=step.ws)
+        elif step.group_size > 1:
+            pa.pa_decode_grouped(step.out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"],
+                                 dev["ctx"], wl.scale, step.group_size,
+                                 max_context_len=wl.max_context_len, partition_size=step.ps,
+                                 workspace=step.ws)
+        else:
+            pa.pa_decode(step.out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"],
+                         dev["ctx"], wl.scale, max_context_len=wl.max_context_len,
+                         partition_size=step.ps, workspace=step.ws)
         out_host.copy_(step.out, non_blocking=True)
 
     for _ in range(warmup):
@@ -460,8 +495,13 @@ def oracle_sample(wl, target_s, threads):
         if sub.num_tokens:
             oracle.kv_append(host["k_new"], host["v_new"], sub.slot_mapping, host["k_cache"],
                              host["v_cache"])
-        oracle.decode(host["q"], host["k_cache"], host["v_cache"], sub.block_tables,
-                      sub.context_lens, sub.scale, num_threads=threads)
+        if sub.query_start is not None:
+            oracle.decode_multi(host["q"], host["k_cache"], host["v_cache"], sub.block_tables,
+                                sub.context_lens, sub.query_start, sub.scale,
+                                num_threads=threads)
+        else:
+            oracle.decode(host["q"], host["k_cache"], host["v_cache"], sub.block_tables,
+                          sub.context_lens, sub.scale, num_threads=threads)
         dt = time.perf_counter() - t0
         return dt, sub.decode_bytes() + sub.append_bytes() + sub.copy_bytes(), sub
 

@@ -9,7 +9,8 @@
  *   pa_block_copy  copy whole physical blocks (copy-on-write at a fork)
  *
  * plus pa_block_swap (blocks between a device pool and a pinned host pool),
- * and pa_decode_grouped, pa_decode for groups of sequences that share blocks
+ * pa_decode_multi (several query tokens per sequence: chunked prefill,
+ * speculative verification), and pa_decode_grouped, pa_decode for groups of sequences that share blocks
  * (beams, parallel samples), which reads each shared block once per group.
  *
  * Sources for what each call computes (page title, section):
@@ -229,6 +230,52 @@ int pa_decode_grouped_num_partitions(int32_t num_seqs, int32_t num_heads,
                                      int32_t max_context_len,
                                      const pa_cache_desc* cache, int32_t group_size,
                                      int32_t partition_size);
+
+/*
+ * pa_decode_multi — attention of several new query tokens per sequence over
+ * the paged cache: a chunk of a prompt processed against the cache (chunked
+ * prefill, which [P2 § 如何判断服务瓶颈是否真的来自 PagedAttention] names
+ * among the things to check when prefill dominates), or the draft tokens of a
+ * speculative step being verified. Same block tables, same cache.
+ *
+ * Sequence s has n_s = query_start[s+1] - query_start[s] new tokens, whose K/V
+ * have already been appended: they are the last n_s of its context_lens[s]
+ * positions. Query token j (0 <= j < n_s, row query_start[s] + j of q and out)
+ * sits at position p = context_lens[s] - n_s + j and attends causally to
+ * positions 0 .. p:
+ *     out[row][h] = softmax_{t <= p}(scale q[row][h] . K_t) . V
+ * with K_t, V_t read through block_tables[s] exactly as in pa_decode.
+ *
+ *   q, out        device, [num_query_tokens][num_heads][head_dim], bf16.
+ *   query_start   device int32 [num_seqs + 1], non-decreasing, query_start[0]
+ *                 = 0, query_start[num_seqs] = num_query_tokens (<= 65535).
+ *   max_query_len host bound on n_s (>= 1). Tokens of one sequence are
+ *                 decoded together in groups of up to 8 (at most 64 query
+ *                 columns per group), so each block is read once per group.
+ *   workspace     at least pa_decode_multi_workspace_size(...) bytes.
+ * Needs a bf16 cache with head_dim 64 or 128 (PA_ERR_UNSUPPORTED otherwise).
+ * n_s > context_lens[s] is recorded as PA_ERR_BAD_INDEX (those rows get 0).
+ * A query token's result does not depend on the other tokens in the call (it
+ * is bit-identical to a call holding only that token with the context cut at
+ * its position, for the same partition size).
+ */
+int pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int32_t block_table_stride,
+                    const int32_t* context_lens, const int32_t* query_start,
+                    int32_t max_context_len, int32_t num_seqs, int32_t num_query_tokens,
+                    int32_t max_query_len, int32_t num_heads, float scale,
+                    const pa_cache_desc* cache, int32_t partition_size, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* Workspace bytes and partition count of pa_decode_multi. */
+size_t pa_decode_multi_workspace_size(int32_t num_seqs, int32_t num_query_tokens,
+                                      int32_t max_query_len, int32_t num_heads,
+                                      int32_t max_context_len, const pa_cache_desc* cache,
+                                      int32_t partition_size);
+int pa_decode_multi_num_partitions(int32_t num_seqs, int32_t num_query_tokens,
+                                   int32_t max_query_len, int32_t num_heads,
+                                   int32_t max_context_len, const pa_cache_desc* cache,
+                                   int32_t partition_size);
 
 /*
  * pa_block_copy — copy whole physical blocks, the copy-on-write step that

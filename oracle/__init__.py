@@ -53,9 +53,12 @@ def _bind(path: str):
     lib.oracle_kv_append.argtypes = [p, p, p, i32, p, p, i32, i32, i32, i32, i32]
     lib.oracle_block_copy.argtypes = [p, i32, p, p, i32, i32, i32, i32, i32]
     lib.oracle_block_swap.argtypes = [p, i32, p, p, i32, p, p, i32, i32, i32, i32, i32]
+    lib.oracle_decode_multi.argtypes = [p, p, p, p, p, i32, p, p, i32, i32, i32, i32, i32,
+                                        i32, i32, ctypes.c_float, i32]
     lib.oracle_decode.argtypes = [p, p, p, p, p, i32, p, i32, i32, i32, i32, i32,
                                   i32, i32, ctypes.c_float, i32]
-    for f in (lib.oracle_kv_append, lib.oracle_block_copy, lib.oracle_block_swap, lib.oracle_decode,
+    for f in (lib.oracle_kv_append, lib.oracle_block_copy, lib.oracle_block_swap,
+              lib.oracle_decode, lib.oracle_decode_multi,
               lib.oracle_max_threads):
         f.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
@@ -193,6 +196,34 @@ def decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
                                _ptr(tables), tables.shape[1], _ptr(ctx), s, h, hkv, nb, bs, d,
                                _dtype_code(k_cache), float(np.float32(scale)), int(num_threads))
     _check(rc, "decode")
+    return out
+
+
+def decode_multi(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+                 block_tables: np.ndarray, context_lens: np.ndarray, query_start: np.ndarray,
+                 scale: float, num_threads: int = 1) -> np.ndarray:
+    """Several query tokens per sequence: q [T][H][d], rows query_start[s] ..
+    query_start[s+1]-1 of sequence s are its last n_s context positions, each
+    attending causally. Returns out (float64 [T][H][d])."""
+    k_cache = _contig(k_cache)
+    v_cache = _contig(v_cache, k_cache.dtype)
+    nb, hkv, bs, d = k_cache.shape
+    q = _contig(q, k_cache.dtype)
+    t, h, dq = q.shape
+    if dq != d:
+        raise ValueError("q head_dim differs from the cache's")
+    tables = _contig(block_tables, np.int32)
+    ctx = _contig(context_lens, np.int32)
+    qs = _contig(query_start, np.int32)
+    s = ctx.shape[0]
+    if tables.ndim != 2 or tables.shape[0] != s or qs.shape != (s + 1,) or qs[-1] != t:
+        raise ValueError("block_tables [S][stride], context_lens [S], query_start [S+1] ending at T")
+    out = np.zeros((t, h, d), dtype=np.float64)
+    rc = _load().oracle_decode_multi(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                     _ptr(tables), tables.shape[1], _ptr(ctx), _ptr(qs), s, h,
+                                     hkv, nb, bs, d, _dtype_code(k_cache),
+                                     float(np.float32(scale)), int(num_threads))
+    _check(rc, "decode_multi")
     return out
 
 

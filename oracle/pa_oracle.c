@@ -173,6 +173,7 @@ static int decode_one(double* out, const void* q, const void* k_cache,
                       int32_t s, int32_t h, int32_t num_heads, int32_t num_kv_heads,
                       int32_t num_blocks, int32_t block_size, int32_t head_dim,
                       int32_t dtype, double scale) {
+    /* s: the row of q and out (the sequence, or the query token) */
     double* o = out + ((size_t)s * num_heads + h) * head_dim;
     for (int32_t i = 0; i < head_dim; ++i) o[i] = 0.0;
     if (n == 0) return OR_OK;
@@ -252,6 +253,59 @@ int oracle_decode(double* out, const void* q, const void* k_cache, const void* v
         int32_t h = (int32_t)(idx % num_heads);
         int r = decode_one(out, q, k_cache, v_cache,
                            block_tables + (size_t)s * block_table_stride, context_lens[s], s, h,
+                           num_heads, num_kv_heads, num_blocks, block_size, head_dim, dtype,
+                           (double)scale);
+        if (r != OR_OK) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+            rc = r;
+        }
+    }
+    return rc;
+}
+
+/*
+ * Several new query tokens per sequence (chunked prefill / verification of
+ * draft tokens, [P2] § 如何判断服务瓶颈是否真的来自 PagedAttention names chunked
+ * prefill): sequence s owns q / out rows query_start[s] .. query_start[s+1]-1;
+ * those n tokens are the last n of its context_lens[s] positions, so row
+ * query_start[s] + j is the query at position p = ctx - n + j and sees keys
+ * 0 .. p (causal), i.e. exactly the single-query decode above with the
+ * context cut at p + 1. p < 0 (more query tokens than context) is an error.
+ */
+int oracle_decode_multi(double* out, const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, int32_t block_table_stride,
+                        const int32_t* context_lens, const int32_t* query_start,
+                        int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                        int32_t num_blocks, int32_t block_size, int32_t head_dim, int32_t dtype,
+                        float scale, int32_t num_threads) {
+    if (num_seqs < 0 || num_heads <= 0 ||
+        !shape_ok(num_blocks, num_kv_heads, block_size, head_dim, dtype) ||
+        num_heads % num_kv_heads != 0 || block_table_stride < 0 || query_start[0] != 0)
+        return OR_ERR_ARG;
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        int32_t n = query_start[s + 1] - query_start[s];
+        if (n < 0 || n > context_lens[s] ||
+            (int64_t)context_lens[s] > (int64_t)block_table_stride * block_size)
+            return OR_ERR_ARG;
+    }
+    const int64_t rows = query_start[num_seqs];
+    const int64_t pairs = rows * num_heads;
+    int rc = OR_OK;
+    if (num_threads < 1) num_threads = 1;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads)
+#endif
+    for (int64_t idx = 0; idx < pairs; ++idx) {
+        int32_t row = (int32_t)(idx / num_heads);
+        int32_t h = (int32_t)(idx % num_heads);
+        int32_t s = 0;
+        while (query_start[s + 1] <= row) ++s;          /* the sequence holding this row */
+        int32_t n = query_start[s + 1] - query_start[s];
+        int32_t pos = context_lens[s] - n + (row - query_start[s]);
+        int r = decode_one(out, q, k_cache, v_cache,
+                           block_tables + (size_t)s * block_table_stride, pos + 1, row, h,
                            num_heads, num_kv_heads, num_blocks, block_size, head_dim, dtype,
                            (double)scale);
         if (r != OR_OK) {

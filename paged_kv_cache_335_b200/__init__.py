@@ -91,6 +91,11 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_decode_num_partitions.argtypes = [i32, i32, i32, desc, i32]
         lib.pa_decode_grouped.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, desc,
                                           i32, i32, vp, sz, vp]
+        lib.pa_decode_multi.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, i32,
+                                        f32, desc, i32, vp, sz, vp]
+        lib.pa_decode_multi_workspace_size.argtypes = [i32, i32, i32, i32, i32, desc, i32]
+        lib.pa_decode_multi_workspace_size.restype = sz
+        lib.pa_decode_multi_num_partitions.argtypes = [i32, i32, i32, i32, i32, desc, i32]
         lib.pa_decode_grouped_workspace_size.argtypes = [i32, i32, i32, desc, i32, i32]
         lib.pa_decode_grouped_workspace_size.restype = sz
         lib.pa_decode_grouped_num_partitions.argtypes = [i32, i32, i32, desc, i32, i32]
@@ -342,6 +347,72 @@ def pa_decode_grouped(out, q, k_cache, v_cache, block_tables, context_lens, scal
                  partition_size, workspace, stream)
 
 
+def pa_decode_multi_workspace_size(num_seqs: int, num_query_tokens: int, max_query_len: int,
+                                   num_heads: int, max_context_len: int, k_cache,
+                                   partition_size: int = 0) -> int:
+    lib = load_library()
+    desc = cache_desc(k_cache)
+    n = lib.pa_decode_multi_workspace_size(num_seqs, num_query_tokens, max_query_len, num_heads,
+                                           max_context_len, ctypes.byref(desc), partition_size)
+    if n == 0:
+        msg = lib.pa_get_last_error().decode()
+        rc = lib.pa_decode_multi_num_partitions(num_seqs, num_query_tokens, max_query_len,
+                                                num_heads, max_context_len, ctypes.byref(desc),
+                                                partition_size)
+        if rc < 0:
+            raise PAError(rc, msg)
+    return int(n)
+
+
+def pa_decode_multi_num_partitions(num_seqs: int, num_query_tokens: int, max_query_len: int,
+                                   num_heads: int, max_context_len: int, k_cache,
+                                   partition_size: int = 0) -> int:
+    rc = load_library().pa_decode_multi_num_partitions(
+        num_seqs, num_query_tokens, max_query_len, num_heads, max_context_len,
+        ctypes.byref(cache_desc(k_cache)), partition_size)
+    if rc < 0:
+        _check(rc)
+    return rc
+
+
+def pa_decode_multi(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                    scale: float, max_context_len: int | None = None,
+                    max_query_len: int | None = None, partition_size: int = 0, workspace=None,
+                    stream=None) -> None:
+    """Several query tokens per sequence (chunked prefill, draft verification):
+    q / out [T][H][D] with rows query_start[s] .. query_start[s+1]-1 for sequence
+    s, its last n_s context positions, each attending causally over the cache."""
+    torch = _torch()
+    _same_pool(k_cache, v_cache)
+    desc = cache_desc(k_cache)
+    t, h, d = (int(x) for x in q.shape)
+    s = int(context_lens.shape[0])
+    if tuple(out.shape) != (t, h, d) or d != desc.head_dim:
+        raise ValueError("q and out must be [num_query_tokens][num_heads][head_dim]")
+    if q.dtype != k_cache.dtype or out.dtype != k_cache.dtype:
+        raise TypeError("q, out and the caches must share one dtype")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or query_start.shape != (s + 1,):
+        raise ValueError("block_tables [S][stride], context_lens [S], query_start [S + 1]")
+    if max_context_len is None:
+        max_context_len = int(context_lens.max().item()) if s else 0
+    if max_query_len is None:
+        max_query_len = max(1, int((query_start[1:] - query_start[:-1]).max().item())) if s else 1
+    need = pa_decode_multi_workspace_size(s, t, max_query_len, h, max_context_len, k_cache,
+                                          partition_size)
+    ws_ptr, ws_bytes = ctypes.c_void_p(0), 0
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    _check(load_library().pa_decode_multi(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), int(block_tables.shape[1]),
+        _dev(context_lens, "context_lens", torch.int32),
+        _dev(query_start, "query_start", torch.int32), int(max_context_len), s, t,
+        int(max_query_len), h, float(scale), ctypes.byref(desc), int(partition_size), ws_ptr,
+        ws_bytes, _stream(stream)))
+
+
 def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
                       max_context_len: int | None = None, partition_size: int = 0,
                       stream=None) -> None:
@@ -373,5 +444,6 @@ def pa_sync_check(stream=None) -> None:
 
 __all__ = ["pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_block_copy", "pa_decode_workspace_size",
            "pa_decode_num_partitions", "pa_decode_grouped", "pa_decode_grouped_workspace_size",
-           "pa_decode_grouped_num_partitions", "pa_block_swap", "pa_sync_check", "pa_cache_desc", "cache_desc",
+           "pa_decode_grouped_num_partitions", "pa_decode_multi", "pa_decode_multi_workspace_size",
+           "pa_decode_multi_num_partitions", "pa_block_swap", "pa_sync_check", "pa_cache_desc", "cache_desc",
            "load_library", "header_functions", "PAError"]

@@ -131,7 +131,10 @@ constexpr int kMinPartition = 256;       // tensor-core kernel: smallest partiti
 
 struct Plan {
     bool use_mma;
-    bool grouped;       // the grouped kernel (group_size > 1 and supported)
+    bool grouped;       // the grouped kernel (group_size > 1 and supported, or multi-token)
+    bool multi;         // several query tokens per sequence (pa_decode_multi)
+    int group_size;     // members per grouped item: sequences, or query tokens of one sequence
+    int q_chunks;       // multi: items per (sequence, kv head, partition) = ceil(max_query_len / gs)
     int partition_size;
     int num_partitions;
     size_t ws_bytes;
@@ -142,8 +145,11 @@ int round_up16(int x) { return (x + 15) / 16 * 16; }
 
 // Partition policy: split the context only when the (sequence, head) work
 // units alone cannot fill the GPU, then into 512-token partitions.
+// num_query_tokens >= 0 selects the multi-token mode (pa_decode_multi): query
+// tokens of one sequence are grouped (at most 8, at most 64 query columns).
 int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_cache_desc* c,
-                int32_t partition_size, Plan* plan, int32_t group_size = 1) {
+                int32_t partition_size, Plan* plan, int32_t group_size = 1,
+                int32_t num_query_tokens = -1, int32_t max_query_len = 0) {
     int rc = check_cache(c);
     if (rc != PA_OK) return rc;
     if (num_seqs < 0 || num_seqs > 65535)
@@ -155,7 +161,25 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
     const int group = num_heads / c->num_kv_heads;
     if (group_size < 1 || group_size > 8)
         return fail(PA_ERR_INVALID_ARG, "group_size %d outside [1, 8]", group_size);
-    plan->grouped = group_size > 1 && pa::grouped_supported(c->dtype, c->head_dim, group, group_size);
+    plan->multi = num_query_tokens >= 0;
+    plan->q_chunks = 1;
+    if (plan->multi) {
+        if (max_query_len < 1 || max_query_len > num_query_tokens + (num_query_tokens == 0))
+            return fail(PA_ERR_INVALID_ARG, "max_query_len %d must be in [1, num_query_tokens %d]",
+                        max_query_len, num_query_tokens);
+        int gs = max_query_len < 8 ? max_query_len : 8;
+        while (gs > 1 && gs * group > 64) --gs;
+        if (!pa::grouped_supported(c->dtype, c->head_dim, group, gs))
+            return fail(PA_ERR_UNSUPPORTED, "multi-token decode needs a bf16 cache, head_dim 64 "
+                        "or 128 and num_heads / num_kv_heads <= 64");
+        group_size = gs;
+        plan->q_chunks = (max_query_len + gs - 1) / gs;
+        plan->grouped = true;
+    } else {
+        plan->grouped =
+            group_size > 1 && pa::grouped_supported(c->dtype, c->head_dim, group, group_size);
+    }
+    plan->group_size = group_size;
     if (plan->grouped && max_ctx > (1 << 27))
         return fail(PA_ERR_INVALID_ARG, "max_context_len %d above 2^27 on the grouped kernel", max_ctx);
     plan->use_mma = pa::mma_supported(c->dtype, c->head_dim, group);
@@ -180,9 +204,10 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
             // Pick the partition count with the smallest such cost (ties: fewer partitions),
             // partitions cut equal and at least kMinPartition tokens long.
             // The grouped kernel is persistent the same way; its unit is a group.
-            const long units = plan->grouped
-                                   ? (long)((num_seqs + group_size - 1) / group_size) * c->num_kv_heads
-                                   : (long)num_seqs * c->num_kv_heads;
+            const long units =
+                plan->multi     ? (long)num_seqs * plan->q_chunks * c->num_kv_heads
+                : plan->grouped ? (long)((num_seqs + group_size - 1) / group_size) * c->num_kv_heads
+                                : (long)num_seqs * c->num_kv_heads;
             const long slots =
                 (long)sm_count() * (plan->grouped ? pa::grouped_ctas_per_sm(c->head_dim, group_size, group)
                                                   : pa::mma_ctas_per_sm());
@@ -231,7 +256,8 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
         plan->ws_bytes = 0;
         plan->ws_ml_offset = 0;
     } else {
-        const size_t rows = (size_t)num_seqs * num_heads * np;
+        const size_t rows =
+            (size_t)(plan->multi ? num_query_tokens : num_seqs) * num_heads * np;
         const size_t o_bytes = rows * c->head_dim * sizeof(float);
         plan->ws_ml_offset = (o_bytes + 255) / 256 * 256;
         plan->ws_bytes = plan->ws_ml_offset + rows * 2 * sizeof(float);
@@ -251,17 +277,24 @@ int pa::report_error(int code, const char* fmt, ...) {
     return code;
 }
 
+// num_query_tokens >= 0: multi-token queries (query_start [num_seqs + 1]).
 static int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
                        const int32_t* block_tables, int32_t block_table_stride,
                        const int32_t* context_lens, int32_t max_context_len, int32_t num_seqs,
                        int32_t num_heads, float scale, const pa_cache_desc* cache,
                        int32_t group_size, int32_t partition_size, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+                       size_t workspace_bytes, void* stream, const int32_t* query_start = nullptr,
+                       int32_t num_query_tokens = -1, int32_t max_query_len = 0) {
     Plan plan;
+    if (num_query_tokens > 65535)
+        return fail(PA_ERR_INVALID_ARG, "num_query_tokens %d above 65535", num_query_tokens);
     int rc = plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan,
-                         group_size);
+                         group_size, num_query_tokens, max_query_len);
     if (rc != PA_OK) return rc;
-    if (num_seqs == 0) return PA_OK;
+    if (num_seqs == 0 || num_query_tokens == 0) return PA_OK;
+    if (plan.multi && (!query_start || (reinterpret_cast<uintptr_t>(query_start) & 3u) != 0))
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_multi: query_start must be a 4-byte aligned "
+                    "device array of num_seqs + 1 entries");
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
         return fail(PA_ERR_INVALID_ARG, "pa_decode: NULL pointer argument");
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
@@ -304,13 +337,16 @@ static int decode_impl(void* out, const void* q, const void* k_cache, const void
     p.num_partitions = plan.num_partitions;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.test_skip_position = g_test_skip_position;
+    p.query_start = plan.multi ? query_start : nullptr;
+    p.q_chunks = plan.q_chunks;
+    p.num_rows = plan.multi ? num_query_tokens : num_seqs;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     CUtensorMap kmap, vmap;
     if ((rc = make_cache_map(&kmap, k_cache, cache)) != PA_OK) return rc;
     if ((rc = make_cache_map(&vmap, v_cache, cache)) != PA_OK) return rc;
     cudaError_t e =
         plan.grouped
-            ? pa::launch_decode_grouped(p, cache->head_dim, group_size, kmap, vmap, st)
+            ? pa::launch_decode_grouped(p, cache->head_dim, plan.group_size, kmap, vmap, st)
             : pa::launch_decode_tma(p, cache->dtype, cache->head_dim, plan.use_mma, kmap, vmap, st);
     if (e != cudaSuccess) return fail_cuda(e, "pa_decode launch");
     t_last_kernel = plan.grouped ? PA_KERNEL_GROUPED : plan.use_mma ? PA_KERNEL_MMA : PA_KERNEL_SIMT;
@@ -447,6 +483,45 @@ int pa_decode_grouped(void* out, const void* q, const void* k_cache, const void*
     return decode_impl(out, q, k_cache, v_cache, block_tables, block_table_stride, context_lens,
                        max_context_len, num_seqs, num_heads, scale, cache, group_size,
                        partition_size, workspace, workspace_bytes, stream);
+}
+
+int pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int32_t block_table_stride,
+                    const int32_t* context_lens, const int32_t* query_start,
+                    int32_t max_context_len, int32_t num_seqs, int32_t num_query_tokens,
+                    int32_t max_query_len, int32_t num_heads, float scale,
+                    const pa_cache_desc* cache, int32_t partition_size, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+    if (num_query_tokens < 0)
+        return fail(PA_ERR_INVALID_ARG, "num_query_tokens %d is negative", num_query_tokens);
+    return decode_impl(out, q, k_cache, v_cache, block_tables, block_table_stride, context_lens,
+                       max_context_len, num_seqs, num_heads, scale, cache, 1, partition_size,
+                       workspace, workspace_bytes, stream, query_start, num_query_tokens,
+                       max_query_len);
+}
+
+size_t pa_decode_multi_workspace_size(int32_t num_seqs, int32_t num_query_tokens,
+                                      int32_t max_query_len, int32_t num_heads,
+                                      int32_t max_context_len, const pa_cache_desc* cache,
+                                      int32_t partition_size) {
+    Plan plan;
+    if (num_query_tokens < 0 ||
+        plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan, 1,
+                    num_query_tokens, max_query_len) != PA_OK)
+        return 0;
+    return plan.ws_bytes;
+}
+
+int pa_decode_multi_num_partitions(int32_t num_seqs, int32_t num_query_tokens,
+                                   int32_t max_query_len, int32_t num_heads,
+                                   int32_t max_context_len, const pa_cache_desc* cache,
+                                   int32_t partition_size) {
+    if (num_query_tokens < 0)
+        return fail(PA_ERR_INVALID_ARG, "num_query_tokens %d is negative", num_query_tokens);
+    Plan plan;
+    int rc = plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan, 1,
+                         num_query_tokens, max_query_len);
+    return rc != PA_OK ? rc : plan.num_partitions;
 }
 
 size_t pa_decode_grouped_workspace_size(int32_t num_seqs, int32_t num_heads,

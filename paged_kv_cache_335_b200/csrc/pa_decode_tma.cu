@@ -1022,22 +1022,46 @@ struct GWalk {
     int k, kbase, ctx_lane;
 };
 
+// Members of an item: sequences grp * gs + m (beams, samples), or, with
+// multi-token queries, query tokens c * gs + m of sequence grp / q_chunks
+// (c = grp % q_chunks), which all read that sequence's blocks.
 struct GItem {
     bool valid;
     int grp, kh, part, t0;
     int tmax;     // end of the item's tokens over its members (== t0: nothing to read)
     int t1_lane;  // end of member (lane & 7)'s tokens in the item (t0 if none)
+    int row0;     // q / out row of member 0 (member m: row0 + m)
+    int nmem;     // members that exist (rows to write); <= 0: none
+    int tab0;     // block-table row of member 0 (member m: tab0 + m * tab_step)
+    int tab_step;
 };
 
+// Member m's token limit: its context length, or for query token j of a
+// sequence with n new tokens (the last n of its context_len positions), the
+// causal end ctx - n + j + 1. 0 for members that do not exist.
 __device__ __forceinline__ int gwalk_load(const DecodeParams& p, int num_items, int kbase, int lane,
                                           int gs, int ipb, bool report) {
     if (lane >= ipb * gs) return 0;
     const int u = blockIdx.x + (kbase + lane / gs) * gridDim.x;
     if (u >= num_items) return 0;
     const int part = u % p.num_partitions;
-    const int s = (u / p.num_partitions / p.num_kv_heads) * gs + lane % gs;
-    if (s >= p.num_seqs) return 0;
-    return clamp_ctx(__ldg(p.context_lens + s), p.max_context_len, report && part == 0);
+    const int grp = u / p.num_partitions / p.num_kv_heads;
+    const int m = lane % gs;
+    if (p.query_start == nullptr) {
+        const int s = grp * gs + m;
+        if (s >= p.num_seqs) return 0;
+        return clamp_ctx(__ldg(p.context_lens + s), p.max_context_len, report && part == 0);
+    }
+    const int s = grp / p.q_chunks, j = (grp % p.q_chunks) * gs + m;
+    const int q0 = __ldg(p.query_start + s), n = __ldg(p.query_start + s + 1) - q0;
+    if (j >= n) return 0;
+    const int ctx = clamp_ctx(__ldg(p.context_lens + s), p.max_context_len, report && part == 0);
+    const int lim = ctx - n + j + 1;
+    if (lim < 1) {  // more new query tokens than context: not a valid step
+        if (report && part == 0) atomicOr(&s_status_tma, kStatusBadIndex);
+        return 0;
+    }
+    return lim;
 }
 
 __device__ __forceinline__ GItem gitem_next(GWalk& w, const DecodeParams& p, int num_items, int gs,
@@ -1047,6 +1071,7 @@ __device__ __forceinline__ GItem gitem_next(GWalk& w, const DecodeParams& p, int
         GItem it;
         it.valid = u < num_items;
         it.grp = it.kh = it.part = it.t0 = it.tmax = it.t1_lane = 0;
+        it.row0 = it.nmem = it.tab0 = it.tab_step = 0;
         if (!it.valid) return it;
         if (w.k - w.kbase >= ipb) {
             w.kbase = w.k;
@@ -1062,7 +1087,21 @@ __device__ __forceinline__ GItem gitem_next(GWalk& w, const DecodeParams& p, int
         it.t1_lane = m < gs ? max(it.t0, min(ctx, it.t0 + p.partition_size)) : it.t0;
         it.tmax = __reduce_max_sync(0xffffffffu, it.t1_lane);
         ++w.k;
-        if (it.tmax > it.t0 || want_empty) return it;
+        if (it.tmax > it.t0 || want_empty) {
+            if (p.query_start == nullptr) {
+                it.row0 = it.tab0 = it.grp * gs;
+                it.tab_step = 1;
+                it.nmem = min(gs, p.num_seqs - it.row0);
+            } else {
+                const int sq = it.grp / p.q_chunks, c = it.grp % p.q_chunks;
+                const int q0 = __ldg(p.query_start + sq);
+                it.row0 = q0 + c * gs;
+                it.nmem = min(gs, __ldg(p.query_start + sq + 1) - it.row0);
+                it.tab0 = sq;
+                it.tab_step = 0;
+            }
+            return it;
+        }
     }
 }
 
@@ -1078,7 +1117,7 @@ __device__ __forceinline__ void gload_phys(const DecodeParams& p, const GItem& i
         phys[m] = -1;
         if (it.valid && m < gs && tok0 < t1) {
             act |= 1u << m;
-            phys[m] = __ldg(p.block_tables + (int64_t)(it.grp * gs + m) * p.table_stride +
+            phys[m] = __ldg(p.block_tables + (int64_t)(it.tab0 + m * it.tab_step) * p.table_stride +
                             (tok0 >> p.log2_block_size));
         }
     }
@@ -1446,10 +1485,10 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             const int col = col0 + 8 * j + r;
             const int m = col / group, hd = col - m * group;
             const int t1 = __shfl_sync(0xffffffffu, it.t1_lane, m & (kMaxGroupSeqs - 1));
-            const int s = it.grp * gs + m;
-            if (it.valid && m < gs && s < p.num_seqs && t1 > it.t0) {
-                const uint16_t* qrow = static_cast<const uint16_t*>(p.q) +
-                                       ((int64_t)s * p.num_heads + (int64_t)it.kh * group + hd) * D;
+            if (it.valid && m < gs && m < it.nmem && t1 > it.t0) {
+                const uint16_t* qrow =
+                    static_cast<const uint16_t*>(p.q) +
+                    ((int64_t)(it.row0 + m) * p.num_heads + (int64_t)it.kh * group + hd) * D;
 #pragma unroll
                 for (int jp = 0; jp < KCH; ++jp)
                     q[j][jp] = ld_v4(qrow + (jp >> 1) * 64 + (2 * c + (jp & 1)) * 8);
@@ -1546,10 +1585,10 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             for (int e = 0; e < 2; ++e) {
                 const int col = col0 + 8 * j + 2 * c + e;
                 const int m = col / group, hd = col - m * group;
-                const int s = cur.grp * gs + m;
                 const int t1 = e == 0 ? t1a[j] : t1b[j];
-                if (m < gs && s < p.num_seqs && (P == 1 || t1 > cur.t0)) {
-                    const int64_t row = (int64_t)s * p.num_heads + (int64_t)cur.kh * group + hd;
+                if (m < gs && m < cur.nmem && (P == 1 || t1 > cur.t0)) {
+                    const int64_t row =
+                        (int64_t)(cur.row0 + m) * p.num_heads + (int64_t)cur.kh * group + hd;
                     grouped_store_col<D>(p, row, cur.part, r, c, e, acc[j],
                                          e == 0 ? ma[j] : mb[j], e == 0 ? la[j] : lb[j]);
                 }
@@ -1632,7 +1671,8 @@ cudaError_t launch_grouped_t(const DecodeParams& p, const CUtensorMap& km, const
     }
     int sms = 0;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const long groups = (p.num_seqs + gs - 1) / gs;
+    const long groups = p.query_start != nullptr ? (long)p.num_seqs * p.q_chunks
+                                                 : (long)(p.num_seqs + gs - 1) / gs;
     const long items = (long)p.num_partitions * p.num_kv_heads * groups;
     const long slots = (long)per_sm[dev] * sms;
     const unsigned grid = (unsigned)(items < slots ? items : slots);
@@ -1672,7 +1712,7 @@ static void grouped_shape(int gs, int group, int* cw, int* nt) {
 }
 
 bool grouped_supported(int dtype, int head_dim, int group, int gs) {
-    return dtype == 1 && (head_dim == 64 || head_dim == 128) && gs >= 2 && gs <= kMaxGroupSeqs &&
+    return dtype == 1 && (head_dim == 64 || head_dim == 128) && gs >= 1 && gs <= kMaxGroupSeqs &&
            group >= 1 && gs * group <= kGroupedMaxCols;
 }
 

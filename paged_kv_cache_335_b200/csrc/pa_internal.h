@@ -40,6 +40,12 @@ struct DecodeParams {
     int32_t num_partitions;     // P
     float scale_log2;           // softmax scale * log2(e)
     int32_t test_skip_position; // -1; >= 0 only under pa_test_skip_load (timeout test)
+    // Multi-token queries (pa_decode_multi), else query_start == nullptr: q / out
+    // rows of sequence s are query_start[s] .. query_start[s+1]-1 of num_rows;
+    // grouped items take q_chunks chunks of <= gs query tokens per sequence.
+    const int32_t* query_start;
+    int32_t q_chunks;
+    int32_t num_rows;           // rows of q / out: num_seqs, or the query tokens
 };
 
 struct CopyParams {
@@ -77,8 +83,9 @@ cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bo
                               const CUtensorMap& kmap, const CUtensorMap& vmap,
                               cudaStream_t stream);
 // Grouped decode: sequences [k gs, (k + 1) gs) form group k and run in one CTA,
-// so blocks they share are read once. bf16, head_dim 64 / 128, 2 <= gs <= 8,
-// gs * (H / Hkv) <= 64 query columns.
+// so blocks they share are read once; with p.query_start set, the members of an
+// item are up to gs query tokens of one sequence instead. bf16, head_dim
+// 64 / 128, 1 <= gs <= 8, gs * (H / Hkv) <= 64 query columns.
 bool grouped_supported(int dtype, int head_dim, int group, int gs);
 // CTA slots per SM of the grouped kernel chosen for (head_dim, gs, H / Hkv).
 int grouped_ctas_per_sm(int head_dim, int gs, int group);

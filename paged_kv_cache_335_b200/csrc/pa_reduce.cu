@@ -24,7 +24,7 @@ __device__ __forceinline__ int clamp_context(int ctx, int max_ctx) {
 // Merge of partitions j = 0 .. ceil(n / partition_size) - 1 of one (s, h):
 //   M = max_j m_j,  w_j = l_j * 2^(m_j - M),  out = sum_j w_j o_j / sum_j w_j,
 // where o_j is partition j's normalised output. This is the exact softmax over
-// the union of the partitions. grid = (num_heads, num_seqs). Launched as a
+// the union of the partitions. grid = (num_heads, rows of out). Launched as a
 // programmatic dependent of the decode kernel: it may start while the decode
 // drains and waits (griddepcontrol.wait) for all of its results.
 template <typename T, int D>
@@ -34,10 +34,24 @@ partition_reduce_kernel(const DecodeParams p) {
     __shared__ float sm_L;
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int h = blockIdx.x;
-    const int s = blockIdx.y;
-    const int ctx = clamp_context(__ldg(p.context_lens + s), p.max_context_len);
+    const int row = blockIdx.y;  // sequence, or query token with multi-token queries
+    int ctx;
+    if (p.query_start == nullptr) {
+        ctx = clamp_context(__ldg(p.context_lens + row), p.max_context_len);
+    } else {
+        // the sequence holding query token `row`: query_start[s] <= row < query_start[s+1]
+        int lo = 0, hi = p.num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(p.query_start + mid) <= row) lo = mid; else hi = mid - 1;
+        }
+        const int q0 = __ldg(p.query_start + lo), n_new = __ldg(p.query_start + lo + 1) - q0;
+        const int lim = clamp_context(__ldg(p.context_lens + lo), p.max_context_len) - n_new +
+                        (row - q0) + 1;  // causal end of this query token
+        ctx = lim < 0 ? 0 : lim;
+    }
     const int n = (ctx + p.partition_size - 1) / p.partition_size;
-    const int64_t out_row = (int64_t)s * p.num_heads + h;
+    const int64_t out_row = (int64_t)row * p.num_heads + h;
     const float* ml = p.ws_ml + out_row * p.num_partitions * 2;
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
@@ -70,7 +84,7 @@ partition_reduce_kernel(const DecodeParams p) {
 template <typename T, int D>
 cudaError_t launch_reduce_t(const DecodeParams& p, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.num_heads, (unsigned)p.num_seqs);
+    cfg.gridDim = dim3((unsigned)p.num_heads, (unsigned)p.num_rows);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = (size_t)p.num_partitions * sizeof(float);
     cfg.stream = stream;

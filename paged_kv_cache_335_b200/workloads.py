@@ -52,6 +52,9 @@ class Workload:
     partition_size: int = 0           # 0 = library policy
     description: str = ""
     extra: dict = field(default_factory=dict)
+    # multi-token queries: int32 [S + 1]; sequence s owns q rows query_start[s] ..
+    # query_start[s+1]-1, its last n_s context positions (None: one query per sequence)
+    query_start: np.ndarray | None = None
 
     @property
     def torch_dtype(self):
@@ -74,9 +77,19 @@ class Workload:
         return int(self.context_lens.astype(np.int64).sum()) * self.num_kv_heads * \
             self.head_dim * 2 * self.elem_bytes
 
+    @property
+    def num_query_rows(self) -> int:
+        """Rows of q / out: one per sequence, or every query token."""
+        return self.num_seqs if self.query_start is None else int(self.query_start[-1])
+
+    @property
+    def max_query_len(self) -> int:
+        return 1 if self.query_start is None else int(np.diff(self.query_start).max(initial=1))
+
     def decode_bytes(self) -> int:
-        """Algorithmic bytes of one decode call: K/V of every context token + q + out."""
-        qo = 2 * self.num_seqs * self.num_heads * self.head_dim * self.elem_bytes
+        """Algorithmic bytes of one decode call: K/V of every context token (once
+        per sequence, whatever its query count) + q + out."""
+        qo = 2 * self.num_query_rows * self.num_heads * self.head_dim * self.elem_bytes
         return self.kv_bytes() + qo
 
     def append_bytes(self) -> int:
@@ -106,19 +119,23 @@ class Workload:
 # structure
 # ---------------------------------------------------------------------------
 def _decode_structure(name, dtype, ctx, num_heads, num_kv_heads, head_dim, block_size,
-                      num_blocks, scale, seed, rng, partition_size=0, description=""):
-    """Sequences of the given final context lengths, each holding ctx-1 tokens
-    before the step and appending one token (position ctx-1) in it."""
+                      num_blocks, scale, seed, rng, partition_size=0, description="",
+                      new_tokens=None):
+    """Sequences of the given final context lengths, each holding ctx - n tokens
+    before the step and appending n in it (positions ctx-n .. ctx-1); n = 1
+    unless ``new_tokens`` gives one count per sequence (multi-token queries)."""
     ctx = np.asarray(ctx, dtype=np.int64)
     s_count = ctx.shape[0]
+    news = np.ones(s_count, np.int64) if new_tokens is None else np.asarray(new_tokens, np.int64)
+    news = np.minimum(news, ctx)
     order = rng.permutation(num_blocks)
     poison = int(order[-1])                      # a valid id that no sequence owns
     bm = BlockManager(num_blocks, block_size, order=order, reserved=(poison,))
     seqs, slots, token_seq = [], [], []
     for s in range(s_count):
         n = int(ctx[s])
-        seq = bm.new_sequence(max(n - 1, 0))
-        if n >= 1:
+        seq = bm.new_sequence(n - int(news[s]))
+        for _ in range(int(news[s])):
             slots.append(bm.append_slot(seq))
             token_seq.append(s)
         seqs.append(seq)
@@ -128,11 +145,13 @@ def _decode_structure(name, dtype, ctx, num_heads, num_kv_heads, head_dim, block
         name=name, dtype=dtype, num_seqs=s_count, num_heads=num_heads,
         num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=block_size,
         num_blocks=num_blocks, scale=float(np.float32(scale)), seed=seed,
-        context_lens=ctx.astype(np.int32), history_lens=np.maximum(ctx - 1, 0).astype(np.int32),
+        context_lens=ctx.astype(np.int32), history_lens=(ctx - news).astype(np.int32),
         block_tables=tables, slot_mapping=np.asarray(slots, dtype=np.int64),
         token_seq=np.asarray(token_seq, dtype=np.int32),
         copy_pairs=np.zeros((0, 2), dtype=np.int64), poison_block=poison,
-        partition_size=partition_size, description=description)
+        partition_size=partition_size, description=description,
+        query_start=None if new_tokens is None else
+        np.concatenate([[0], np.cumsum(news)]).astype(np.int32))
 
 
 def _pool_size(ctx, block_size, factor=1.2):
@@ -262,6 +281,35 @@ def decode_case(num_seqs, num_heads, num_kv_heads, head_dim, block_size, dtype, 
                              1.0 / math.sqrt(head_dim), seed, rng, partition_size=partition_size)
 
 
+def multi_query_case(num_seqs, num_heads, num_kv_heads, head_dim, block_size, dtype,
+                     context_lens, query_lens, seed=0, pool_factor=1.3, partition_size=0,
+                     name=None) -> Workload:
+    """Multi-token queries: sequence s appends query_lens[s] tokens this step
+    (its last positions) and each of them attends causally over the cache, as
+    in chunked prefill or the verification of draft tokens."""
+    rng = np.random.default_rng(seed)
+    ctx = np.asarray(context_lens, dtype=np.int64)
+    demand = int(sum(-(-int(n) // block_size) for n in ctx))
+    nb = int(math.ceil(pool_factor * max(demand, 1))) + 2
+    name = name or (f"multi_{num_seqs}x{num_heads}/{num_kv_heads}_d{head_dim}_bs{block_size}_"
+                    f"{dtype}")
+    return _decode_structure(name, dtype, ctx, num_heads, num_kv_heads, head_dim, block_size, nb,
+                             1.0 / math.sqrt(head_dim), seed, rng, partition_size=partition_size,
+                             new_tokens=query_lens)
+
+
+def llama70b_verify(seed: int = 6, num_seqs: int = 8, context_len: int = 32768,
+                    draft: int = 4) -> Workload:
+    """Speculative verification on the 70B-shaped layer: 8 sequences of 32K
+    context each check ``draft`` new tokens in one pass (64/8 heads, d128, bf16)."""
+    wl = multi_query_case(num_seqs, 64, 8, 128, 16, "bf16", [context_len] * num_seqs,
+                          [draft] * num_seqs, seed=seed, pool_factor=1.05,
+                          name=f"llama70b_verify{draft}")
+    wl.description = (f"{num_seqs} seqs x {context_len} ctx, {draft} query tokens each "
+                      "(verification), 64/8 heads, d128, bs16, bf16")
+    return wl
+
+
 CONFIGS = {
     "tiny": tiny,
     "llama7b": llama7b,
@@ -269,6 +317,7 @@ CONFIGS = {
     "llama13b_bs32": lambda seed=2: llama13b(seed, 32),
     "llama70b_gqa": llama70b_gqa,
     "cow_beam4": cow_beam4,
+    "llama70b_verify4": llama70b_verify,
 }
 
 
@@ -312,6 +361,9 @@ def restrict(wl: Workload, seq_ids) -> Workload:
     sub.copy_pairs = np.asarray(pairs, dtype=np.int64).reshape(-1, 2)
     sub.poison_block = poison
     sub.extra = dict(wl.extra)
+    if wl.query_start is not None:
+        counts = np.diff(wl.query_start)[seq_ids]
+        sub.query_start = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
     return sub
 
 
@@ -337,7 +389,7 @@ def make_values(wl: Workload, device="cpu", poison: bool = False, seed_offset: i
     g = torch.Generator(device=device).manual_seed(wl.seed * 1000003 + seed_offset)
     dt = wl.torch_dtype
     S, H, Hkv, d = wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim
-    q = torch.randn((S, H, d), generator=g, device=device, dtype=dt)
+    q = torch.randn((wl.num_query_rows, H, d), generator=g, device=device, dtype=dt)
     k_new = torch.randn((wl.num_tokens, Hkv, d), generator=g, device=device, dtype=dt)
     v_new = torch.randn((wl.num_tokens, Hkv, d), generator=g, device=device, dtype=dt)
     shape = (wl.num_blocks, Hkv, wl.block_size, d)

@@ -119,6 +119,27 @@ def test_grouped_decode_rejects_bad_group_size(lib):
         assert b"group_size" in lib.pa_get_last_error()
 
 
+def test_multi_query_policy_and_arguments(lib):
+    d70 = _desc(num_kv_heads=8)
+    f = lib.pa_decode_multi_num_partitions
+    # 8 sequences x 4 query tokens (one group of 4 per sequence and kv head):
+    # 64 items for 296 slots, so the 32K context is split
+    n = f(8, 32, 4, 64, 32768, ctypes.byref(d70), 0)
+    assert 1 < n <= 32768 // 256
+    assert f(8, 32, 4, 64, 32768, ctypes.byref(d70), 512) == 64
+    assert lib.pa_decode_multi_workspace_size(8, 32, 4, 64, 32768, ctypes.byref(d70), 512) >= \
+        32 * 64 * 64 * (128 + 2) * 4                                 # rows are query tokens
+    assert f(8, 32, 0, 64, 32768, ctypes.byref(d70), 0) == pa.PA_ERR_INVALID_ARG   # max_query_len
+    assert f(8, 32, 33, 64, 32768, ctypes.byref(d70), 0) == pa.PA_ERR_INVALID_ARG
+    assert f(8, -1, 1, 64, 32768, ctypes.byref(d70), 0) == pa.PA_ERR_INVALID_ARG
+    f32 = _desc(num_kv_heads=8, dtype=pa.PA_F32)
+    assert f(8, 32, 4, 64, 32768, ctypes.byref(f32), 0) == pa.PA_ERR_UNSUPPORTED
+    p = ctypes.c_void_p(256)
+    rc = lib.pa_decode_multi(p, p, p, p, p, 8, p, None, 100, 2, 4, 2, 64, ctypes.c_float(0.1),
+                             ctypes.byref(d70), -1, None, 0, None)
+    assert rc == pa.PA_ERR_INVALID_ARG and b"query_start" in lib.pa_get_last_error()
+
+
 def test_swap_rejects_bad_arguments(lib):
     p = ctypes.c_void_p(256)
     a, b = _desc(num_blocks=8), _desc(num_blocks=4)

@@ -1,0 +1,132 @@
+"""Multi-token paged queries (pa_decode_multi) against the fp64 oracle.
+
+Each sequence appends n_s tokens this step and every one of them attends
+causally over the paged cache (chunked prefill, verification of draft tokens).
+Bars: appended slots bit-exact; outputs within the bf16 tolerance of the
+unrounded oracle; a query token's result bit-identical whether or not other
+tokens share the call; bad inputs reported, unsupported dtypes refused.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_335_b200 as pa
+from paged_kv_cache_335_b200 import workloads as W
+from tests import gpu_helpers as G
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _multi(wl, vals, ps=0, out=None):
+    d = G.device_tensors(wl, vals)
+    if out is None:
+        out = torch.empty_like(vals["q"])
+    pa.pa_decode_multi(out, vals["q"], vals["k_cache"], vals["v_cache"], d["tables"], d["ctx"],
+                       torch.as_tensor(wl.query_start, device=DEV), wl.scale,
+                       max_context_len=wl.max_context_len, max_query_len=wl.max_query_len,
+                       partition_size=ps)
+    return out
+
+
+def _step_check(wl, ps):
+    vals = W.make_values(wl, DEV, poison=True)
+    host = G.host_copy(vals)
+    d = G.device_tensors(wl, vals)
+    pa.pa_kv_append(vals["k_new"], vals["v_new"], d["slots"], vals["k_cache"], vals["v_cache"])
+    out = _multi(wl, vals, ps)
+    pa.pa_sync_check()
+    assert G.last_kernel() == pa.PA_KERNEL_GROUPED
+    oracle.kv_append(host["k_new"], host["v_new"], wl.slot_mapping, host["k_cache"], host["v_cache"])
+    assert G.bits_equal(vals["k_cache"], host["k_cache"])
+    assert G.bits_equal(vals["v_cache"], host["v_cache"])
+    ref = oracle.decode_multi(host["q"], host["k_cache"], host["v_cache"], wl.block_tables,
+                              wl.context_lens, wl.query_start, wl.scale, num_threads=G.THREADS)
+    return G.check_tolerance(G.to_f64(out), ref, wl.dtype, f"{wl.name} ps={ps}"), out, vals
+
+
+CTX = [1, 2, 15, 16, 17, 40, 64, 65, 129, 300, 511, 513]
+NQ = [1, 2, 15, 3, 9, 8, 1, 17, 4, 300, 0, 33]
+
+
+@pytest.mark.parametrize("d,bs", [(64, 16), (128, 16), (128, 64)])
+@pytest.mark.parametrize("H,Hkv", [(8, 8), (8, 4), (16, 2), (12, 3), (64, 8)])
+def test_parity_shape_sweep(d, bs, H, Hkv):
+    """Query counts from 0 to a whole 300-token prompt (38 groups of 8), contexts
+    at block and partition edges, every n-tile layout."""
+    wl = W.multi_query_case(len(CTX), H, Hkv, d, bs, "bf16", CTX, NQ, seed=d + bs + H)
+    for ps in (-1, 0, 64):
+        _step_check(wl, ps)
+
+
+def test_token_result_independent_of_the_other_tokens():
+    """Row j of a 6-token verification equals, bit for bit, a call holding only
+    that token with the context cut at its position (same partition size)."""
+    wl = W.multi_query_case(2, 32, 4, 128, 16, "bf16", [900, 333], [6, 5], seed=3)
+    vals = W.make_values(wl, DEV, poison=False)
+    d = G.device_tensors(wl, vals)
+    pa.pa_kv_append(vals["k_new"], vals["v_new"], d["slots"], vals["k_cache"], vals["v_cache"])
+    for ps in (128, -1):
+        full = _multi(wl, vals, ps if ps > 0 else -1)
+        for s, j in ((0, 0), (0, 5), (1, 2), (1, 4)):
+            row = int(wl.query_start[s]) + j
+            n = int(wl.query_start[s + 1] - wl.query_start[s])
+            cut = int(wl.context_lens[s]) - n + j + 1
+            one = torch.empty_like(vals["q"][row:row + 1])
+            ps_one = ps if ps > 0 else (-(-int(wl.max_context_len) // 16) * 16)
+            pa.pa_decode_multi(one, vals["q"][row:row + 1].contiguous(), vals["k_cache"],
+                               vals["v_cache"], d["tables"][s:s + 1].contiguous(),
+                               torch.tensor([cut], dtype=torch.int32, device=DEV),
+                               torch.tensor([0, 1], dtype=torch.int32, device=DEV), wl.scale,
+                               max_context_len=wl.max_context_len, max_query_len=1,
+                               partition_size=ps_one)
+            torch.cuda.synchronize()
+            assert G.bits_equal(full[row:row + 1], one), (ps, s, j)
+
+
+def test_verification_full_size_sampled():
+    """8 x 32K-context sequences verifying 4 draft tokens (64/8 heads), library
+    partition policy: every row of two sequences against the oracle."""
+    wl = W.make("llama70b_verify4")
+    vals = W.make_values(wl, DEV, poison=True)
+    d = G.device_tensors(wl, vals)
+    pa.pa_kv_append(vals["k_new"], vals["v_new"], d["slots"], vals["k_cache"], vals["v_cache"])
+    out = _multi(wl, vals, 0)
+    pa.pa_sync_check()
+    assert torch.isfinite(out.float()).all()
+    for s in (0, 7):
+        sub = W.subproblem(wl, vals["k_cache"], vals["v_cache"], [s])
+        r0, r1 = int(wl.query_start[s]), int(wl.query_start[s + 1])
+        q_rows = W.to_numpy(vals["q"][r0:r1]).copy()
+        ref = oracle.decode_multi(q_rows, sub["k_cache"], sub["v_cache"], sub["block_tables"],
+                                  sub["context_lens"], np.array([0, r1 - r0], np.int32), wl.scale,
+                                  num_threads=G.THREADS)
+        G.check_tolerance(G.to_f64(out[r0:r1]), ref, "bf16", f"verify seq {s}")
+
+
+def test_more_queries_than_context_reported():
+    wl = W.multi_query_case(2, 16, 2, 128, 16, "bf16", [40, 30], [3, 2], seed=1)
+    vals = W.make_values(wl, DEV)
+    d = G.device_tensors(wl, vals)
+    out = torch.empty_like(vals["q"])
+    pa.pa_sync_check()
+    qs = torch.tensor([0, 3, 5], dtype=torch.int32, device=DEV)
+    d["ctx"][1] = 1                                          # 2 queries, 1 context position
+    pa.pa_decode_multi(out, vals["q"], vals["k_cache"], vals["v_cache"], d["tables"], d["ctx"], qs,
+                       wl.scale, max_context_len=40, max_query_len=3)
+    with pytest.raises(pa.PAError) as e:
+        pa.pa_sync_check()
+    assert e.value.code == pa.PA_ERR_BAD_INDEX
+
+
+def test_f32_cache_is_refused():
+    wl = W.tiny()
+    vals = W.make_values(wl, DEV)
+    d = G.device_tensors(wl, vals)
+    qs = torch.arange(wl.num_seqs + 1, dtype=torch.int32, device=DEV)
+    with pytest.raises(pa.PAError) as e:
+        pa.pa_decode_multi(torch.empty_like(vals["q"]), vals["q"], vals["k_cache"], vals["v_cache"],
+                           d["tables"], d["ctx"], qs, wl.scale, max_context_len=wl.max_context_len,
+                           max_query_len=1)
+    assert e.value.code == pa.PA_ERR_UNSUPPORTED

@@ -32,6 +32,8 @@ MUTANTS = [
     ("copy direction", "size_t src = (size_t)pairs[2 * p] * block_bytes;",
      "size_t src = (size_t)pairs[2 * p + 1] * block_bytes;"),
     ("padding test", "if (slot < 0) continue;", "if (slot <= 0) continue;"),
+    ("causal end", "int32_t pos = context_lens[s] - n + (row - query_start[s]);",
+     "int32_t pos = context_lens[s] - n + (row - query_start[s]) - (n > 1);"),
     ("swap K from V", "memcpy((char*)dst_k + to, (const char*)src_k + from, block_bytes);",
      "memcpy((char*)dst_k + to, (const char*)src_v + from, block_bytes);"),
     ("query row", "qd[i] = load_elem(q, ((int64_t)s * num_heads + h) * head_dim + i, dtype);",
@@ -51,6 +53,7 @@ PINS = [
     pins.test_prefix_sharing_bitwise,
     pins.test_tiny_workload_step_matches_sdpa,
     pins.test_block_swap_equals_indexed_assignment,
+    lambda: pins.test_decode_multi_equals_masked_sdpa("bf16", 16, 8, 2),
 ]
 
 

@@ -402,3 +402,57 @@ def test_block_swap_rejects_bad_ids_and_shapes():
     with pytest.raises(ValueError):
         oracle.block_swap(np.array([[0, 0]]), a, a.copy(), np.zeros((2, 2, 16, 4), np.float32),
                           np.zeros((2, 2, 16, 4), np.float32))
+
+
+# ---------------------------------------------------------------------------
+# multi-token queries (chunked prefill / draft verification)
+# ---------------------------------------------------------------------------
+def _sdpa_multi_reference(q_rows, K, V, ctx, nq, scale, num_kv_heads):
+    """torch float64 SDPA per sequence with an explicit bottom-right causal mask:
+    query j of n sees keys 0 .. ctx - n + j (a library routine on the contiguous
+    context, independent of the oracle's own code)."""
+    out = np.zeros_like(q_rows)
+    row = 0
+    H, d = q_rows.shape[1], q_rows.shape[2]
+    for s in range(len(ctx)):
+        n, c = int(nq[s]), int(ctx[s])
+        if n == 0:
+            continue
+        qs = torch.from_numpy(np.ascontiguousarray(q_rows[row:row + n].transpose(1, 0, 2))).view(1, H, n, d)
+        ks = torch.from_numpy(np.ascontiguousarray(K[s, :c].transpose(1, 0, 2))).view(1, num_kv_heads, c, d)
+        vs = torch.from_numpy(np.ascontiguousarray(V[s, :c].transpose(1, 0, 2))).view(1, num_kv_heads, c, d)
+        mask = torch.arange(c).view(1, c) <= (c - n + torch.arange(n)).view(n, 1)
+        o = torch.nn.functional.scaled_dot_product_attention(
+            qs, ks, vs, attn_mask=mask, scale=scale, enable_gqa=(H != num_kv_heads))
+        out[row:row + n] = o.view(H, n, d).permute(1, 0, 2).numpy()
+        row += n
+    return out
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("B,H,Hkv", [(1, 4, 4), (16, 8, 2), (2, 4, 1)])
+def test_decode_multi_equals_masked_sdpa(dtype, B, H, Hkv):
+    c = _random_case(seed=300 + B + H, S=4, H=H, Hkv=Hkv, d=16, B=B, max_ctx=40, dtype=dtype)
+    nq = np.minimum(np.array([1, 5, 0, 12]), c["ctx"])
+    nq[3] = c["ctx"][3]                       # a whole prompt as one chunk (full causal prefill)
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    g = torch.Generator().manual_seed(9)
+    qf = torch.randn((int(qs[-1]), H, 16), generator=g, dtype=torch.float64)
+    if dtype == "f32":
+        q_store = qf.to(torch.float32).numpy()
+        q_val = q_store.astype(np.float64)
+    else:
+        q_store = _bits_bf16(qf)
+        q_val = qf.to(torch.bfloat16).double().numpy()
+    scale = float(np.float32(1 / 4))
+    out = oracle.decode_multi(q_store, c["kc"], c["vc"], c["tables"], c["ctx"], qs, scale)
+    ref = _sdpa_multi_reference(q_val, c["K"], c["V"], c["ctx"], nq, scale, Hkv)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_decode_multi_rejects_more_queries_than_context():
+    kc = np.zeros((2, 1, 4, 4), np.float32)
+    with pytest.raises(oracle.OracleError):
+        oracle.decode_multi(np.zeros((3, 1, 4), np.float32), kc, kc.copy(),
+                            np.zeros((1, 1), np.int32), np.array([2], np.int32),
+                            np.array([0, 3], np.int32), 1.0)
