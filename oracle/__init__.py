@@ -31,6 +31,9 @@ _lib = None
 
 F32 = 0
 BF16 = 1
+FP8_E4M3 = 2     # quantised cache codes (uint8 arrays)
+INT8 = 3
+QUANT_FORMATS = {"fp8": FP8_E4M3, "int8": INT8}
 
 
 def build(force: bool = False) -> str:
@@ -55,10 +58,16 @@ def _bind(path: str):
     lib.oracle_block_swap.argtypes = [p, i32, p, p, i32, p, p, i32, i32, i32, i32, i32]
     lib.oracle_decode_multi.argtypes = [p, p, p, p, p, i32, p, p, i32, i32, i32, i32, i32,
                                         i32, i32, ctypes.c_float, i32]
+    lib.oracle_kv_append_quant.argtypes = [p, p, p, i32, p, p, p, p, i32, i32, i32, i32, i32]
+    lib.oracle_quantize.argtypes = [p, ctypes.c_int64, ctypes.c_float, i32, p]
+    lib.oracle_code_values.argtypes = [p, ctypes.c_int64, i32, p]
+    lib.oracle_decode_quant.argtypes = [p, p, p, p, p, p, p, i32, p, i32, i32, i32, i32, i32,
+                                        i32, i32, ctypes.c_float, i32]
     lib.oracle_decode.argtypes = [p, p, p, p, p, i32, p, i32, i32, i32, i32, i32,
                                   i32, i32, ctypes.c_float, i32]
     for f in (lib.oracle_kv_append, lib.oracle_block_copy, lib.oracle_block_swap,
-              lib.oracle_decode, lib.oracle_decode_multi,
+              lib.oracle_decode, lib.oracle_decode_multi, lib.oracle_kv_append_quant,
+              lib.oracle_quantize, lib.oracle_code_values, lib.oracle_decode_quant,
               lib.oracle_max_threads):
         f.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
@@ -224,6 +233,71 @@ def decode_multi(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
                                      hkv, nb, bs, d, _dtype_code(k_cache),
                                      float(np.float32(scale)), int(num_threads))
     _check(rc, "decode_multi")
+    return out
+
+
+def quantize(x: np.ndarray, scale: float, fmt: str) -> np.ndarray:
+    """Codes (uint8) of binary32 values x under ``scale``: the code of x / scale
+    (binary32 division) in FP8 E4M3 ("fp8", nearest-even, saturating to +-448,
+    NaN -> 0x7F) or int8 ("int8", clamp to +-127 then nearest-even)."""
+    x = _contig(np.asarray(x, dtype=np.float32))
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    _check(_load().oracle_quantize(_ptr(x), x.size, float(np.float32(scale)),
+                                   QUANT_FORMATS[fmt], _ptr(codes)), "quantize")
+    return codes
+
+
+def code_values(codes: np.ndarray, fmt: str) -> np.ndarray:
+    """float64 values of stored codes (unscaled)."""
+    codes = _contig(np.asarray(codes, dtype=np.uint8))
+    out = np.zeros(codes.shape, dtype=np.float64)
+    _check(_load().oracle_code_values(_ptr(codes), codes.size, QUANT_FORMATS[fmt], _ptr(out)),
+           "code_values")
+    return out
+
+
+def kv_append_quant(k: np.ndarray, v: np.ndarray, slot_mapping: np.ndarray,
+                    k_cache: np.ndarray, v_cache: np.ndarray, k_scale: np.ndarray,
+                    v_scale: np.ndarray, fmt: str) -> None:
+    """In place: bf16 (uint16 bits) k, v [T][Hkv][d] quantised into uint8 caches
+    [NB][Hkv][B][d] with per-kv-head binary32 scales."""
+    k = _contig(k, np.uint16)
+    v = _contig(v, np.uint16)
+    k_cache = _contig(k_cache, np.uint8)
+    v_cache = _contig(v_cache, np.uint8)
+    nb, hkv, bs, d = k_cache.shape
+    ks = _contig(np.asarray(k_scale, np.float32))
+    vs = _contig(np.asarray(v_scale, np.float32))
+    slots = _contig(np.asarray(slot_mapping, np.int64))
+    if ks.shape != (hkv,) or vs.shape != (hkv,) or k.shape != (slots.shape[0], hkv, d):
+        raise ValueError("k, v [T][Hkv][d]; scales [Hkv]")
+    _check(_load().oracle_kv_append_quant(_ptr(k), _ptr(v), _ptr(slots), slots.shape[0],
+                                          _ptr(k_cache), _ptr(v_cache), _ptr(ks), _ptr(vs),
+                                          nb, hkv, bs, d, QUANT_FORMATS[fmt]), "kv_append_quant")
+
+
+def decode_quant(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+                 k_scale: np.ndarray, v_scale: np.ndarray, block_tables: np.ndarray,
+                 context_lens: np.ndarray, scale: float, fmt: str,
+                 num_threads: int = 1) -> np.ndarray:
+    """Decode over quantised caches (uint8 codes, per-kv-head scales); q bf16 bits."""
+    k_cache = _contig(k_cache, np.uint8)
+    v_cache = _contig(v_cache, np.uint8)
+    nb, hkv, bs, d = k_cache.shape
+    q = _contig(q, np.uint16)
+    s, h, dq = q.shape
+    ks = _contig(np.asarray(k_scale, np.float32))
+    vs = _contig(np.asarray(v_scale, np.float32))
+    tables = _contig(block_tables, np.int32)
+    ctx = _contig(context_lens, np.int32)
+    if dq != d or ks.shape != (hkv,) or vs.shape != (hkv,) or tables.shape[0] != s:
+        raise ValueError("shapes: q [S][H][d], scales [Hkv], tables [S][stride]")
+    out = np.zeros((s, h, d), dtype=np.float64)
+    _check(_load().oracle_decode_quant(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(ks), _ptr(vs), _ptr(tables), tables.shape[1],
+                                       _ptr(ctx), s, h, hkv, nb, bs, d, QUANT_FORMATS[fmt],
+                                       float(np.float32(scale)), int(num_threads)),
+           "decode_quant")
     return out
 
 

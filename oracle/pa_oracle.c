@@ -18,8 +18,10 @@
  * CUDA sources): cache[num_blocks][num_kv_heads][block_size][head_dim]; token
  * position t of a sequence lives in block table[t / block_size], slot
  * t % block_size. Element types: 0 = binary32, 1 = bfloat16 (the upper half
- * of a binary32). All arithmetic is double precision, in one pass, with no
- * partitioning, blocking or reordering.
+ * of a binary32), 2 = FP8 E4M3 code, 3 = int8 code (quantised caches, one
+ * scale per kv head). All attention arithmetic is double precision, in one
+ * pass, with no partitioning, blocking or reordering; a quantiser takes its
+ * decision in binary32, the precision the stored code is defined in.
  *
  * Pins (what checks this file against something other than itself) live in
  * tests/test_oracle_pins.py: contiguous attention through a library routine,
@@ -38,12 +40,75 @@
 #define OR_ERR_INDEX (-2)
 #define OR_ERR_NOMEM (-3)
 
-static size_t elem_bytes(int32_t dtype) { return dtype == 0 ? 4u : 2u; }
+/* Element types: 0 binary32, 1 bfloat16, 2 FP8 E4M3 code, 3 int8 code. */
+static size_t elem_bytes(int32_t dtype) { return dtype == 0 ? 4u : dtype == 1 ? 2u : 1u; }
+
+/*
+ * KV-cache quantisation ([P2] mechanisms table: KV cache quantisation lowers
+ * the bits per cached element at the cost of quantisation error and
+ * conversion; [P3] § 量化技术: INT8 KV halves KV memory, orthogonal to paging).
+ * The pages give no format details; the reading used: one binary32 scale per
+ * kv head for K and one for V, supplied by the caller; a stored code c stands
+ * for value(c) * scale; a value x is stored as the code of y = x / scale (the
+ * division in binary32, as a GPU does it).
+ *
+ * FP8 E4M3 (the OCP 8-bit format with 4 exponent bits, bias 7, 3 mantissa
+ * bits, no infinities; S.1111.111 is NaN): value = (-1)^S 2^(E-7) (1 + M/8)
+ * for E > 0, (-1)^S 2^-6 (M/8) for E = 0.
+ */
+static double e4m3_value(uint8_t c) {
+    const int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* y -> E4M3 code: round to nearest, ties to the even code; magnitudes of 448
+ * (the largest finite value) and above, infinities included, saturate to
+ * +-448; NaN gives the NaN code 0x7F. Plain search over the 127 finite
+ * magnitudes. */
+static uint8_t e4m3_code(float y) {
+    if (isnan(y)) return 0x7F;
+    const uint8_t sgn = signbit(y) ? 0x80 : 0x00;
+    const double a = fabs((double)y);
+    if (a >= 448.0) return sgn | 0x7E;
+    uint8_t best = 0;
+    double best_err = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        const double err = fabs(a - e4m3_value((uint8_t)c));
+        if (err < best_err || (err == best_err && (c & 1) == 0)) {
+            best = (uint8_t)c;
+            best_err = err;
+        }
+    }
+    return sgn | best;
+}
+
+/* y -> int8 code: clamp to [-127, 127] (fmaxf / fminf: a NaN operand yields
+ * the other one), then round to nearest, ties to even. */
+static int8_t int8_code(float y) {
+    const float c = fminf(fmaxf(y, -127.0f), 127.0f);
+    return (int8_t)lrintf(c);
+}
+
+/* The stored code of element x (a binary32 value) under `scale`. */
+static uint8_t quantize(float x, float scale, int32_t fmt) {
+    const float y = x / scale;
+    if (fmt == 2) return e4m3_code(y);
+    const int8_t q = int8_code(y);
+    uint8_t u;
+    memcpy(&u, &q, 1);
+    return u;
+}
 
 /* Widen one stored element to double. bfloat16 -> binary32 is exact: the 16
  * stored bits become the high half of the binary32 pattern. */
 static double load_elem(const void* base, int64_t idx, int32_t dtype) {
     float f;
+    if (dtype == 2) return e4m3_value(((const uint8_t*)base)[idx]);
+    if (dtype == 3) return (double)((const int8_t*)base)[idx];
     if (dtype == 0) {
         memcpy(&f, (const char*)base + 4 * idx, 4);
     } else {
@@ -59,7 +124,7 @@ static double load_elem(const void* base, int64_t idx, int32_t dtype) {
 static int shape_ok(int32_t num_blocks, int32_t num_kv_heads, int32_t block_size,
                     int32_t head_dim, int32_t dtype) {
     return num_blocks > 0 && num_kv_heads > 0 && block_size > 0 && head_dim > 0 &&
-           (dtype == 0 || dtype == 1);
+           dtype >= 0 && dtype <= 3;
 }
 
 /*
@@ -168,12 +233,14 @@ int oracle_block_swap(const int64_t* pairs, int32_t num_pairs, const void* src_k
  * access scheme, not a new attention formula). Query head h reads kv head
  * h / (num_heads / num_kv_heads) (contiguous groups). n == 0 gives zeros.
  */
-static int decode_one(double* out, const void* q, const void* k_cache,
-                      const void* v_cache, const int32_t* table_row, int32_t n,
-                      int32_t s, int32_t h, int32_t num_heads, int32_t num_kv_heads,
-                      int32_t num_blocks, int32_t block_size, int32_t head_dim,
-                      int32_t dtype, double scale) {
-    /* s: the row of q and out (the sequence, or the query token) */
+static int decode_one_q(double* out, const void* q, int32_t q_dtype, const void* k_cache,
+                        const void* v_cache, const float* k_scale, const float* v_scale,
+                        const int32_t* table_row, int32_t n,
+                        int32_t s, int32_t h, int32_t num_heads, int32_t num_kv_heads,
+                        int32_t num_blocks, int32_t block_size, int32_t head_dim,
+                        int32_t dtype, double scale) {
+    /* s: the row of q and out (the sequence, or the query token); k_scale /
+     * v_scale (per kv head) multiply the stored codes of a quantised cache */
     double* o = out + ((size_t)s * num_heads + h) * head_dim;
     for (int32_t i = 0; i < head_dim; ++i) o[i] = 0.0;
     if (n == 0) return OR_OK;
@@ -196,14 +263,16 @@ static int decode_one(double* out, const void* q, const void* k_cache,
         }
         int64_t base = (((int64_t)phys * num_kv_heads + kh) * block_size + t % block_size) *
                        (int64_t)head_dim;
+        const double ks = k_scale ? (double)k_scale[kh] : 1.0;
+        const double vs = v_scale ? (double)v_scale[kh] : 1.0;
         for (int32_t i = 0; i < head_dim; ++i) {
-            K[(size_t)t * head_dim + i] = load_elem(k_cache, base + i, dtype);
-            V[(size_t)t * head_dim + i] = load_elem(v_cache, base + i, dtype);
+            K[(size_t)t * head_dim + i] = load_elem(k_cache, base + i, dtype) * ks;
+            V[(size_t)t * head_dim + i] = load_elem(v_cache, base + i, dtype) * vs;
         }
     }
     if (rc == OR_OK) {
         for (int32_t i = 0; i < head_dim; ++i)
-            qd[i] = load_elem(q, ((int64_t)s * num_heads + h) * head_dim + i, dtype);
+            qd[i] = load_elem(q, ((int64_t)s * num_heads + h) * head_dim + i, q_dtype);
         double m = -INFINITY;
         for (int32_t t = 0; t < n; ++t) {
             double dot = 0.0;
@@ -222,6 +291,15 @@ static int decode_one(double* out, const void* q, const void* k_cache,
     }
     free(K); free(V); free(w); free(qd);
     return rc;
+}
+
+static int decode_one(double* out, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* table_row, int32_t n,
+                      int32_t s, int32_t h, int32_t num_heads, int32_t num_kv_heads,
+                      int32_t num_blocks, int32_t block_size, int32_t head_dim,
+                      int32_t dtype, double scale) {
+    return decode_one_q(out, q, dtype, k_cache, v_cache, NULL, NULL, table_row, n, s, h,
+                        num_heads, num_kv_heads, num_blocks, block_size, head_dim, dtype, scale);
 }
 
 /*
@@ -308,6 +386,93 @@ int oracle_decode_multi(double* out, const void* q, const void* k_cache, const v
                            block_tables + (size_t)s * block_table_stride, pos + 1, row, h,
                            num_heads, num_kv_heads, num_blocks, block_size, head_dim, dtype,
                            (double)scale);
+        if (r != OR_OK) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+            rc = r;
+        }
+    }
+    return rc;
+}
+
+/*
+ * Quantising append: as oracle_kv_append, but k and v are bfloat16 vectors
+ * and each element is stored as its code under the kv head's scale (fmt 2 =
+ * FP8 E4M3, 3 = int8).
+ */
+int oracle_kv_append_quant(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping,
+                           int32_t num_tokens, uint8_t* k_cache, uint8_t* v_cache,
+                           const float* k_scale, const float* v_scale, int32_t num_blocks,
+                           int32_t num_kv_heads, int32_t block_size, int32_t head_dim,
+                           int32_t fmt) {
+    if (num_tokens < 0 || (fmt != 2 && fmt != 3) ||
+        !shape_ok(num_blocks, num_kv_heads, block_size, head_dim, fmt))
+        return OR_ERR_ARG;
+    for (int32_t i = 0; i < num_tokens; ++i) {
+        const int64_t slot = slot_mapping[i];
+        if (slot <= -1) continue; /* padding token */
+        if (slot >= (int64_t)num_blocks * block_size) return OR_ERR_INDEX;
+        const int64_t blk = slot / block_size, off = slot % block_size;
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            const int64_t src = ((int64_t)i * num_kv_heads + h) * head_dim;
+            const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;
+            for (int32_t d = 0; d < head_dim; ++d) {
+                k_cache[dst + d] = quantize((float)load_elem(k, src + d, 1), k_scale[h], fmt);
+                v_cache[dst + d] = quantize((float)load_elem(v, src + d, 1), v_scale[h], fmt);
+            }
+        }
+    }
+    return OR_OK;
+}
+
+/* Codes of an array of binary32 values (for the quantiser's own pins). */
+int oracle_quantize(const float* x, int64_t n, float scale, int32_t fmt, uint8_t* codes) {
+    if (fmt != 2 && fmt != 3) return OR_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i) codes[i] = quantize(x[i], scale, fmt);
+    return OR_OK;
+}
+
+/* Values of an array of codes (fmt 2 or 3), unscaled. */
+int oracle_code_values(const uint8_t* codes, int64_t n, int32_t fmt, double* out) {
+    if (fmt != 2 && fmt != 3) return OR_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i) out[i] = load_elem(codes, i, fmt);
+    return OR_OK;
+}
+
+/*
+ * Decode over a quantised cache: the plain attention of oracle_decode with
+ * K_t = value(code) * k_scale[kh], V_t = value(code) * v_scale[kh]; q is
+ * bfloat16.
+ */
+int oracle_decode_quant(double* out, const uint16_t* q, const uint8_t* k_cache,
+                        const uint8_t* v_cache, const float* k_scale, const float* v_scale,
+                        const int32_t* block_tables, int32_t block_table_stride,
+                        const int32_t* context_lens, int32_t num_seqs, int32_t num_heads,
+                        int32_t num_kv_heads, int32_t num_blocks, int32_t block_size,
+                        int32_t head_dim, int32_t fmt, float scale, int32_t num_threads) {
+    if (num_seqs < 0 || num_heads <= 0 || (fmt != 2 && fmt != 3) ||
+        !shape_ok(num_blocks, num_kv_heads, block_size, head_dim, fmt) ||
+        num_heads % num_kv_heads != 0 || block_table_stride < 0)
+        return OR_ERR_ARG;
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        int32_t n = context_lens[s];
+        if (n < 0 || (int64_t)n > (int64_t)block_table_stride * block_size) return OR_ERR_ARG;
+    }
+    const int64_t pairs = (int64_t)num_seqs * num_heads;
+    int rc = OR_OK;
+    if (num_threads < 1) num_threads = 1;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads)
+#endif
+    for (int64_t idx = 0; idx < pairs; ++idx) {
+        int32_t s = (int32_t)(idx / num_heads);
+        int32_t h = (int32_t)(idx % num_heads);
+        const int32_t n_ctx = context_lens[s];
+        int r = decode_one_q(out, q, 1, k_cache, v_cache, k_scale, v_scale,
+                             block_tables + (size_t)s * block_table_stride, n_ctx, s, h,
+                             num_heads, num_kv_heads, num_blocks, block_size, head_dim, fmt,
+                             (double)scale);
         if (r != OR_OK) {
 #ifdef _OPENMP
 #pragma omp critical

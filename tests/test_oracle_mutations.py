@@ -34,10 +34,15 @@ MUTANTS = [
     ("padding test", "if (slot < 0) continue;", "if (slot <= 0) continue;"),
     ("causal end", "int32_t pos = context_lens[s] - n + (row - query_start[s]);",
      "int32_t pos = context_lens[s] - n + (row - query_start[s]) - (n > 1);"),
+    ("e4m3 exponent bias", "else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+     "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    ("int8 rounding", "return (int8_t)lrintf(c);", "return (int8_t)c;"),
+    ("quant tie break", "(err == best_err && (c & 1) == 0)", "(err == best_err && (c & 1) == 1)"),
+    ("k scale dropped", "load_elem(k_cache, base + i, dtype) * ks;", "load_elem(k_cache, base + i, dtype);"),
     ("swap K from V", "memcpy((char*)dst_k + to, (const char*)src_k + from, block_bytes);",
      "memcpy((char*)dst_k + to, (const char*)src_v + from, block_bytes);"),
-    ("query row", "qd[i] = load_elem(q, ((int64_t)s * num_heads + h) * head_dim + i, dtype);",
-     "qd[i] = load_elem(q, ((int64_t)s * num_heads + (h / group) * group) * head_dim + i, dtype);"),
+    ("query row", "qd[i] = load_elem(q, ((int64_t)s * num_heads + h) * head_dim + i, q_dtype);",
+     "qd[i] = load_elem(q, ((int64_t)s * num_heads + (h / group) * group) * head_dim + i, q_dtype);"),
 ]
 
 PINS = [
@@ -54,6 +59,10 @@ PINS = [
     pins.test_tiny_workload_step_matches_sdpa,
     pins.test_block_swap_equals_indexed_assignment,
     lambda: pins.test_decode_multi_equals_masked_sdpa("bf16", 16, 8, 2),
+    pins.test_e4m3_values_match_torch_for_every_code,
+    pins.test_e4m3_encoding_matches_torch_round_to_nearest_even,
+    pins.test_int8_codes,
+    lambda: pins.test_decode_quant_equals_sdpa_on_dequantised_values("fp8", 16, 8, 2),
 ]
 
 

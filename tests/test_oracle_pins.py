@@ -456,3 +456,137 @@ def test_decode_multi_rejects_more_queries_than_context():
         oracle.decode_multi(np.zeros((3, 1, 4), np.float32), kc, kc.copy(),
                             np.zeros((1, 1), np.int32), np.array([2], np.int32),
                             np.array([0, 3], np.int32), 1.0)
+
+
+# ---------------------------------------------------------------------------
+# quantised KV cache: FP8 E4M3 / int8 codes with per-kv-head scales
+# ---------------------------------------------------------------------------
+def test_e4m3_values_match_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle.code_values(codes, "fp8")
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(lib))
+    assert np.array_equal(mine[~np.isnan(mine)], lib[~np.isnan(lib)])
+    assert mine[0x7E] == 448.0 and mine[0x01] == 2.0 ** -9 and mine[0x38] == 1.0 and mine[0xB8] == -1.0
+
+
+def test_e4m3_encoding_matches_torch_round_to_nearest_even():
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([
+        rng.standard_normal(20000) * 40, rng.standard_normal(5000) * 0.01,
+        oracle.code_values(np.arange(0x7F, dtype=np.uint8), "fp8"),            # exact codes
+        (oracle.code_values(np.arange(0x7E, dtype=np.uint8), "fp8") +
+         oracle.code_values(np.arange(1, 0x7F, dtype=np.uint8), "fp8")) / 2,   # exact ties
+    ]).astype(np.float32)
+    vals = np.concatenate([vals, -vals])
+    vals = vals[np.abs(vals) < 448]
+    mine = oracle.quantize(vals, 1.0, "fp8")
+    lib = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(mine, lib)
+
+
+def test_e4m3_saturation_nan_and_scale():
+    x = np.array([448, 449, 1e30, np.inf, -np.inf, np.nan, -0.0, 2.0 ** -10, 3 * 2.0 ** -10],
+                 np.float32)
+    assert [int(c) for c in oracle.quantize(x, 1.0, "fp8")] == \
+        [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0x7F, 0x80, 0x00, 0x02]
+    # the code is that of x / scale, divided in binary32
+    assert int(oracle.quantize(np.array([3.0], np.float32), 2.0, "fp8")[0]) == 0x3C   # 1.5
+
+
+def test_int8_codes():
+    x = np.array([2.5, 3.5, -2.5, -3.5, 126.6, 127.4, 200, -1e9, np.inf, -np.inf, np.nan, -0.4],
+                 np.float32)
+    assert oracle.quantize(x, 1.0, "int8").view(np.int8).tolist() == \
+        [2, 4, -2, -4, 127, 127, 127, -127, 127, -127, -127, 0]
+    rng = np.random.default_rng(2)
+    y = (rng.standard_normal(50000) * 60).astype(np.float32)
+    s = np.float32(0.37)
+    lib = np.clip(np.rint(y / s), -127, 127).astype(np.int8)         # numpy: IEEE binary32 divide
+    assert np.array_equal(oracle.quantize(y, float(s), "int8").view(np.int8), lib)
+
+
+def test_quantisation_error_bounds():
+    rng = np.random.default_rng(3)
+    s = 0.05
+    x = (rng.uniform(-1, 1, 40000) * 127 * s).astype(np.float32)
+    deq = oracle.code_values(oracle.quantize(x, s, "int8"), "int8") * np.float32(s)
+    assert np.max(np.abs(deq - x)) <= s / 2 * (1 + 1e-6)
+    xf = (rng.uniform(2.0 ** -6, 440, 40000) * rng.choice([-1, 1], 40000)).astype(np.float32)
+    deqf = oracle.code_values(oracle.quantize(xf, 1.0, "fp8"), "fp8")
+    assert np.max(np.abs(deqf - xf) / np.abs(xf)) <= 2.0 ** -4
+
+
+def test_quant_append_places_codes():
+    """Codes land in (slot / B, head, slot % B): numpy placement of torch / numpy
+    quantised values."""
+    rng = np.random.default_rng(4)
+    T, Hkv, B, d, NB = 6, 3, 4, 8, 5
+    k = torch.randn((T, Hkv, d), generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    v = torch.randn((T, Hkv, d), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    ks = np.array([0.01, 0.02, 0.5], np.float32)
+    vs = np.array([0.03, 0.04, 0.25], np.float32)
+    slots = np.array([19, 0, -1, 7, 12, 3], np.int64)
+    for fmt in ("fp8", "int8"):
+        kc = np.zeros((NB, Hkv, B, d), np.uint8)
+        vc = np.zeros_like(kc)
+        oracle.kv_append_quant(_bits_bf16(k), _bits_bf16(v), slots, kc, vc, ks, vs, fmt)
+        want_k, want_v = np.zeros_like(kc), np.zeros_like(vc)
+        for t, sl in enumerate(slots):
+            if sl < 0:
+                continue
+            for h in range(Hkv):
+                for src, sc, dst in ((k, ks, want_k), (v, vs, want_v)):
+                    y = src[t, h].float().numpy() / sc[h]
+                    if fmt == "int8":
+                        code = np.clip(np.rint(y), -127, 127).astype(np.int8).view(np.uint8)
+                    else:
+                        code = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+                    dst[sl // B, h, sl % B] = code
+        assert np.array_equal(kc, want_k) and np.array_equal(vc, want_v), fmt
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("B,H,Hkv", [(16, 8, 2), (2, 4, 4)])
+def test_decode_quant_equals_sdpa_on_dequantised_values(fmt, B, H, Hkv):
+    """Decode over codes = contiguous SDPA over value(code) * scale, the values
+    taken through torch's float8 type (fp8) or plain integers (int8)."""
+    rng = np.random.default_rng(5 + B + H)
+    S, d, NB = 3, 16, 40
+    ctx = np.array([1, 37, 20], np.int32)
+    ks = rng.uniform(0.005, 0.05, Hkv).astype(np.float32)
+    vs = rng.uniform(0.005, 0.05, Hkv).astype(np.float32)
+    kc = rng.integers(0, 256, (NB, Hkv, B, d), dtype=np.uint8)
+    vc = rng.integers(0, 256, (NB, Hkv, B, d), dtype=np.uint8)
+    if fmt == "fp8":                                # no NaN codes
+        kc[(kc & 0x7F) == 0x7F] = 0x7E
+        vc[(vc & 0x7F) == 0x7F] = 0x7E
+    perm = rng.permutation(NB)
+    tables = np.zeros((S, -(-int(ctx.max()) // B)), np.int32)
+    used = 0
+    for s in range(S):
+        nb = -(-int(ctx[s]) // B)
+        tables[s, :nb] = perm[used:used + nb]
+        used += nb
+    qf = torch.randn((S, H, d), generator=torch.Generator().manual_seed(7))
+    q_bits = _bits_bf16(qf)
+    q_val = qf.to(torch.bfloat16).double().numpy()
+    if fmt == "fp8":
+        kval = torch.from_numpy(kc).view(torch.float8_e4m3fn).double().numpy()
+        vval = torch.from_numpy(vc).view(torch.float8_e4m3fn).double().numpy()
+    else:
+        kval = kc.view(np.int8).astype(np.float64)
+        vval = vc.view(np.int8).astype(np.float64)
+    kval = kval * ks.astype(np.float64)[None, :, None, None]
+    vval = vval * vs.astype(np.float64)[None, :, None, None]
+    Tm = int(ctx.max())
+    K = np.zeros((S, Tm, Hkv, d))
+    V = np.zeros((S, Tm, Hkv, d))
+    for s in range(S):
+        for t in range(int(ctx[s])):
+            K[s, t] = kval[tables[s, t // B], :, t % B]
+            V[s, t] = vval[tables[s, t // B], :, t % B]
+    scale = float(np.float32(0.25))
+    out = oracle.decode_quant(q_bits, kc, vc, ks, vs, tables, ctx, scale, fmt)
+    ref = _sdpa_reference(q_val, K, V, ctx, scale, Hkv)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
