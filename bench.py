@@ -45,7 +45,10 @@ EXTRA_CONFIGS = [("llama7b", "llama7b", None, 1), ("llama13b_bs16", "llama13b_bs
                  ("llama70b_gqa", "llama70b_gqa", None, 1),
                  ("llama70b_gqa_policy", "llama70b_gqa", 0, 1), ("cow_beam4", "cow_beam4", None, 1),
                  ("cow_beam4_grouped", "cow_beam4", 0, 4),
-                 ("llama70b_verify4", "llama70b_verify4", 0, 1)]
+                 ("llama70b_verify4", "llama70b_verify4", 0, 1),
+                 ("llama13b_bs16_fp8", "llama13b_bs16_fp8", None, 1),
+                 ("llama13b_bs16_int8", "llama13b_bs16_int8", None, 1),
+                 ("llama70b_gqa_policy_fp8", "llama70b_gqa_fp8", 0, 1)]
 # pa_test_last_decode_kernel() -> the decode kernel a call enqueued
 KERNEL_NAMES = {0: "decode_tma_simt_kernel (CUDA-core)",
                 1: "decode_tma_mma_kernel (persistent, tensor-core GQA)",
@@ -281,6 +284,12 @@ class Step:
         self.args_append = (P(v["k_new"].data_ptr()), P(v["v_new"].data_ptr()),
                             P(self.slots.data_ptr()), wl.num_tokens, P(v["k_cache"].data_ptr()),
                             P(v["v_cache"].data_ptr()), ctypes.byref(self.desc), self.sp)
+        self.append_fn = self.lib.pa_kv_append
+        if wl.kv_quant:                                  # quantised cache: codes + scales
+            self.args_append = self.args_append[:6] + (P(v["k_scale"].data_ptr()),
+                                                       P(v["v_scale"].data_ptr())) + \
+                self.args_append[6:]
+            self.append_fn = self.lib.pa_kv_append_quant
         self.args_decode = (P(self.out.data_ptr()), P(v["q"].data_ptr()),
                             P(v["k_cache"].data_ptr()), P(v["v_cache"].data_ptr()),
                             P(self.tables.data_ptr()), int(self.tables.shape[1]),
@@ -289,6 +298,11 @@ class Step:
             ((group_size,) if group_size > 1 else ()) + \
             (self.ps, P(self.ws.data_ptr()), ctypes.c_size_t(self.ws_bytes), self.sp)
         self.decode_fn = self.lib.pa_decode_grouped if group_size > 1 else self.lib.pa_decode
+        if wl.kv_quant:
+            self.args_decode = self.args_decode[:4] + (P(v["k_scale"].data_ptr()),
+                                                       P(v["v_scale"].data_ptr())) + \
+                self.args_decode[4:]
+            self.decode_fn = self.lib.pa_decode_quant
         if self.multi:
             self.args_decode = (P(self.out.data_ptr()), P(v["q"].data_ptr()),
                                 P(v["k_cache"].data_ptr()), P(v["v_cache"].data_ptr()),
@@ -315,7 +329,7 @@ class Step:
             if rc:
                 raise RuntimeError(lib.pa_get_last_error().decode())
         if self.has_append:
-            rc = lib.pa_kv_append(*self.args_append)
+            rc = self.append_fn(*self.args_append)
             if rc:
                 raise RuntimeError(lib.pa_get_last_error().decode())
         if ev:
@@ -442,9 +456,17 @@ def e2e_steps(step, steps, warmup):
             dev[k].copy_(host[k], non_blocking=True)
         if wl.copy_pairs.shape[0]:
             pa.pa_block_copy(dev["pairs"], v["k_cache"], v["v_cache"])
-        if wl.num_tokens:
+        if wl.num_tokens and wl.kv_quant:
+            pa.pa_kv_append_quant(dev["k_new"], dev["v_new"], dev["slots"], v["k_cache"],
+                                  v["v_cache"], v["k_scale"], v["v_scale"])
+        elif wl.num_tokens:
             pa.pa_kv_append(dev["k_new"], dev["v_new"], dev["slots"], v["k_cache"], v["v_cache"])
-        if step.multi:
+        if wl.kv_quant:
+            pa.pa_decode_quant(step.out, dev["q"], v["k_cache"], v["v_cache"], v["k_scale"],
+                               v["v_scale"], dev["tables"], dev["ctx"], wl.scale,
+                               max_context_len=wl.max_context_len, partition_size=step.ps,
+                               workspace=step.ws)
+        elif step.multi:
             pa.pa_decode_multi(step.out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"],
                                dev["ctx"], dev["query_start"], wl.scale,
                                max_context_len=wl.max_context_len,
@@ -481,6 +503,7 @@ def oracle_sample(wl, target_s, threads):
     """Time the oracle's step (copies, append, decode) on a bounded sample of the
     workload's sequences; returns (GB/s, seconds, sample description, bytes)."""
     import numpy as np
+    import torch
 
     import oracle
     from paged_kv_cache_335_b200 import workloads as W
@@ -488,14 +511,23 @@ def oracle_sample(wl, target_s, threads):
     def run(ids):
         sub = W.restrict(wl, ids)
         vals = W.make_values(sub, "cpu", poison=False)
-        host = {k: W.to_numpy(t).copy() for k, t in vals.items()}
+        host = {k: (t.numpy().copy() if t.dtype == torch.float32 and t.dim() == 1
+                    else W.to_numpy(t).copy()) for k, t in vals.items()}
         t0 = time.perf_counter()
         if sub.copy_pairs.shape[0]:
             oracle.block_copy(sub.copy_pairs, host["k_cache"], host["v_cache"])
-        if sub.num_tokens:
+        if sub.num_tokens and sub.kv_quant:
+            oracle.kv_append_quant(host["k_new"], host["v_new"], sub.slot_mapping,
+                                   host["k_cache"], host["v_cache"], host["k_scale"],
+                                   host["v_scale"], sub.kv_quant)
+        elif sub.num_tokens:
             oracle.kv_append(host["k_new"], host["v_new"], sub.slot_mapping, host["k_cache"],
                              host["v_cache"])
-        if sub.query_start is not None:
+        if sub.kv_quant:
+            oracle.decode_quant(host["q"], host["k_cache"], host["v_cache"], host["k_scale"],
+                                host["v_scale"], sub.block_tables, sub.context_lens, sub.scale,
+                                sub.kv_quant, num_threads=threads)
+        elif sub.query_start is not None:
             oracle.decode_multi(host["q"], host["k_cache"], host["v_cache"], sub.block_tables,
                                 sub.context_lens, sub.query_start, sub.scale,
                                 num_threads=threads)

@@ -9,6 +9,8 @@
  *   pa_block_copy  copy whole physical blocks (copy-on-write at a fork)
  *
  * plus pa_block_swap (blocks between a device pool and a pinned host pool),
+ * pa_kv_append_quant / pa_decode_quant (FP8 E4M3 or int8 caches with per-head
+ * scales),
  * pa_decode_multi (several query tokens per sequence: chunked prefill,
  * speculative verification), and pa_decode_grouped, pa_decode for groups of sequences that share blocks
  * (beams, parallel samples), which reads each shared block once per group.
@@ -45,7 +47,8 @@
  *   which skip the offending access, never fault, and record PA_ERR_BAD_INDEX
  *   in the device status word that pa_sync_check reads.
  * Element type.  PA_F32 (IEEE binary32) or PA_BF16 (bfloat16). q, out, k, v
- *   and both caches of one call share that type. Attention arithmetic is
+ *   and both caches of one call share that type (quantised caches: see
+ *   pa_decode_quant). Attention arithmetic is
  *   fp32 internally; outputs are rounded to nearest-even into the type.
  *
  * Cache layout (identical for k_cache and v_cache):
@@ -81,7 +84,7 @@ extern "C" {
 /* ---- status codes ------------------------------------------------------- */
 #define PA_OK               0
 #define PA_ERR_INVALID_ARG (-1) /* null pointer, negative size, bad shape     */
-#define PA_ERR_DTYPE       (-2) /* dtype not PA_F32 / PA_BF16                 */
+#define PA_ERR_DTYPE       (-2) /* dtype unknown, or wrong for this call        */
 #define PA_ERR_ALIGN       (-3) /* a pointer is not 16-byte aligned           */
 #define PA_ERR_UNSUPPORTED (-4) /* head_dim / block_size not compiled         */
 #define PA_ERR_CUDA        (-5) /* a CUDA runtime call or launch failed       */
@@ -92,6 +95,8 @@ extern "C" {
 /* ---- element types ------------------------------------------------------ */
 #define PA_F32  0
 #define PA_BF16 1
+#define PA_FP8_E4M3 2  /* quantised cache: one-byte OCP FP8 E4M3 codes (pa_*_quant calls) */
+#define PA_INT8 3      /* quantised cache: one-byte signed int8 codes (pa_*_quant calls)  */
 
 /* Shape of one physical KV pool (both k_cache and v_cache). */
 typedef struct pa_cache_desc {
@@ -99,7 +104,7 @@ typedef struct pa_cache_desc {
     int32_t num_kv_heads; /* KV heads stored per block                      */
     int32_t block_size;   /* token slots per block                          */
     int32_t head_dim;     /* elements per K or V vector                     */
-    int32_t dtype;        /* PA_F32 or PA_BF16                              */
+    int32_t dtype;        /* PA_F32, PA_BF16, PA_FP8_E4M3 or PA_INT8        */
 } pa_cache_desc;
 
 /*
@@ -276,6 +281,48 @@ int pa_decode_multi_num_partitions(int32_t num_seqs, int32_t num_query_tokens,
                                    int32_t max_query_len, int32_t num_heads,
                                    int32_t max_context_len, const pa_cache_desc* cache,
                                    int32_t partition_size);
+
+/*
+ * Quantised KV cache ([P2] mechanisms table: KV cache quantisation lowers
+ * the bits stored per cached element, at the price of quantisation error and
+ * conversion work; [P3] § 量化技术: INT8 KV cache quantisation halves KV
+ * memory without touching the weights and composes with paging). The pages
+ * fix no format; this library stores one byte per element, a PA_FP8_E4M3 or
+ * PA_INT8 code, with one binary32 scale per kv head for K and one for V:
+ *     stored code  c = Q(x / scale[kv head])      (division in binary32)
+ *     cached value   = value(c) * scale[kv head]
+ * Q for PA_FP8_E4M3: round to nearest even, magnitudes >= 448 (infinities
+ * too) saturate to +-448, NaN gives the NaN code 0x7F. Q for PA_INT8: clamp
+ * to [-127, 127] (a NaN becomes -127), then round to nearest even. Scales are
+ * the caller's (calibrated, or from the data); they must be positive and
+ * finite for the codes to mean anything. The cache layout is unchanged with
+ * one-byte elements; pa_block_copy and pa_block_swap move quantised pools as
+ * they are. q and out stay bf16.
+ *
+ * pa_kv_append_quant — pa_kv_append for a quantised cache: k, v are bf16
+ * [num_tokens][num_kv_heads][head_dim] (device); each element is stored as
+ * its code. k_scale, v_scale: device float [num_kv_heads]. head_dim 64 or 128.
+ *
+ * pa_decode_quant — pa_decode over a quantised cache: the same attention with
+ * K_t and V_t the cached values above (the K scale folds into the scores, the
+ * V scale into the output). Arguments as pa_decode plus the two scale arrays;
+ * head_dim 128 (PA_ERR_UNSUPPORTED otherwise); workspace sized by
+ * pa_decode_workspace_size with the quantised descriptor. pa_decode,
+ * pa_kv_append and the other decode calls refuse a quantised descriptor
+ * (PA_ERR_DTYPE), and these two refuse an unquantised one.
+ */
+int pa_kv_append_quant(const void* k, const void* v, const int64_t* slot_mapping,
+                       int32_t num_tokens, void* k_cache, void* v_cache,
+                       const float* k_scale, const float* v_scale,
+                       const pa_cache_desc* cache, void* stream);
+
+int pa_decode_quant(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const float* k_scale, const float* v_scale,
+                    const int32_t* block_tables, int32_t block_table_stride,
+                    const int32_t* context_lens, int32_t max_context_len,
+                    int32_t num_seqs, int32_t num_heads, float scale,
+                    const pa_cache_desc* cache, int32_t partition_size,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * pa_block_copy — copy whole physical blocks, the copy-on-write step that

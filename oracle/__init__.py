@@ -7,7 +7,8 @@ product package ``paged_kv_cache_335_b200`` never imports it, and the C source
 
 What each function computes is documented in ``pa_oracle.c`` with the page and
 section it follows. Arrays are numpy: element type ``float32`` for binary32
-caches and ``uint16`` (raw bit patterns) for bfloat16 caches.
+caches, ``uint16`` (raw bit patterns) for bfloat16 caches and ``uint8`` for
+quantised caches (FP8 E4M3 or int8 codes, with per-kv-head binary32 scales).
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against
 something other than itself (a library attention routine, hand-written golden
@@ -115,7 +116,10 @@ def _dtype_code(a: np.ndarray) -> int:
         return F32
     if a.dtype == np.uint16:
         return BF16
-    raise TypeError(f"cache element type must be float32 or uint16 (bf16 bits), got {a.dtype}")
+    if a.dtype == np.uint8:
+        return FP8_E4M3      # one-byte codes: moves do not look at their meaning
+    raise TypeError(f"cache element type must be float32, uint16 (bf16 bits) or uint8 (codes), "
+                    f"got {a.dtype}")
 
 
 def _ptr(a: np.ndarray) -> int:

@@ -37,6 +37,8 @@ PA_ERR_WORKSPACE = -7
 PA_ERR_TIMEOUT = -8
 PA_F32 = 0
 PA_BF16 = 1
+PA_FP8_E4M3 = 2             # quantised caches: torch.float8_e4m3fn / torch.int8 code tensors
+PA_INT8 = 3
 PA_NOALLOC_SCRATCH_BYTES = 32 << 20
 PA_KERNEL_SIMT = 0          # pa_test_last_decode_kernel() values
 PA_KERNEL_MMA = 1
@@ -100,6 +102,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_decode_grouped_workspace_size.restype = sz
         lib.pa_decode_grouped_num_partitions.argtypes = [i32, i32, i32, desc, i32, i32]
         lib.pa_block_copy.argtypes = [vp, i32, vp, vp, desc, vp]
+        lib.pa_kv_append_quant.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, desc, vp]
+        lib.pa_decode_quant.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, f32,
+                                        desc, i32, vp, sz, vp]
         lib.pa_block_swap.argtypes = [vp, i32, vp, vp, desc, vp, vp, desc, vp]
         lib.pa_sync_check.argtypes = [vp]
         lib.pa_stream_read.argtypes = [vp, sz, vp, i32, vp]
@@ -152,7 +157,12 @@ def _dtype_code(t) -> int:
         return PA_F32
     if t.dtype == torch.bfloat16:
         return PA_BF16
-    raise TypeError(f"unsupported element type {t.dtype}: float32 or bfloat16")
+    if t.dtype == torch.float8_e4m3fn:
+        return PA_FP8_E4M3
+    if t.dtype == torch.int8:
+        return PA_INT8
+    raise TypeError(f"unsupported element type {t.dtype}: float32, bfloat16, float8_e4m3fn "
+                    "(FP8 E4M3 codes) or int8 (int8 codes)")
 
 
 def _dev(t, name: str, dtype=None):
@@ -222,6 +232,55 @@ def pa_block_copy(src_dst_pairs, k_cache, v_cache, stream=None) -> None:
     _check(load_library().pa_block_copy(
         _dev(src_dst_pairs, "src_dst_pairs", torch.int64), int(src_dst_pairs.shape[0]),
         _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), ctypes.byref(desc), _stream(stream)))
+
+
+def pa_kv_append_quant(k, v, slot_mapping, k_cache, v_cache, k_scale, v_scale,
+                       stream=None) -> None:
+    """Quantising append: bf16 k, v [T][Hkv][D] into a float8_e4m3fn or int8 code
+    pool, each element stored as the code of x / scale[kv head] (k_scale, v_scale:
+    float32 [Hkv] on the device)."""
+    torch = _torch()
+    _same_pool(k_cache, v_cache)
+    desc = cache_desc(k_cache)
+    if k.shape != v.shape or k.dim() != 3 or k.shape[1:] != (desc.num_kv_heads, desc.head_dim):
+        raise ValueError("k and v must be [num_tokens][num_kv_heads][head_dim]")
+    if k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("k and v must be bfloat16")
+    _check(load_library().pa_kv_append_quant(
+        _dev(k, "k"), _dev(v, "v"), _dev(slot_mapping, "slot_mapping", torch.int64),
+        int(k.shape[0]), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+        ctypes.byref(desc), _stream(stream)))
+
+
+def pa_decode_quant(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                    scale: float, max_context_len: int | None = None, partition_size: int = 0,
+                    workspace=None, stream=None) -> None:
+    """pa_decode over a quantised (float8_e4m3fn / int8 code) pool with per-kv-head
+    float32 scales; q and out bfloat16."""
+    torch = _torch()
+    _same_pool(k_cache, v_cache)
+    desc = cache_desc(k_cache)
+    s, h, d = (int(x) for x in q.shape)
+    if tuple(out.shape) != (s, h, d) or d != desc.head_dim:
+        raise ValueError("q and out must be [num_seqs][num_heads][head_dim]")
+    if q.dtype != torch.bfloat16 or out.dtype != torch.bfloat16:
+        raise TypeError("q and out must be bfloat16")
+    if max_context_len is None:
+        max_context_len = int(context_lens.max().item()) if s else 0
+    need = pa_decode_workspace_size(s, h, max_context_len, k_cache, partition_size)
+    ws_ptr, ws_bytes = ctypes.c_void_p(0), 0
+    if need:
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    _check(load_library().pa_decode_quant(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+        _dev(block_tables, "block_tables", torch.int32), int(block_tables.shape[1]),
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len), s, h,
+        float(scale), ctypes.byref(desc), int(partition_size), ws_ptr, ws_bytes,
+        _stream(stream)))
 
 
 def pa_block_swap(src_dst_pairs, src_k, src_v, dst_k, dst_v, stream=None) -> None:
@@ -445,5 +504,6 @@ def pa_sync_check(stream=None) -> None:
 __all__ = ["pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_block_copy", "pa_decode_workspace_size",
            "pa_decode_num_partitions", "pa_decode_grouped", "pa_decode_grouped_workspace_size",
            "pa_decode_grouped_num_partitions", "pa_decode_multi", "pa_decode_multi_workspace_size",
-           "pa_decode_multi_num_partitions", "pa_block_swap", "pa_sync_check", "pa_cache_desc", "cache_desc",
+           "pa_decode_multi_num_partitions", "pa_kv_append_quant", "pa_decode_quant", "pa_block_swap",
+           "pa_sync_check", "pa_cache_desc", "cache_desc",
            "load_library", "header_functions", "PAError"]

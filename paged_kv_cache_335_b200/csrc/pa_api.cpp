@@ -44,13 +44,16 @@ int ilog2_exact(int x) {
     return (1 << l) == x ? l : -1;
 }
 
-int elem_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
+int elem_bytes(int dtype) { return dtype == PA_F32 ? 4 : dtype == PA_BF16 ? 2 : 1; }
+
+bool quantised(int dtype) { return dtype == PA_FP8_E4M3 || dtype == PA_INT8; }
 
 // Shape checks shared by every call.
 int check_cache(const pa_cache_desc* c) {
     if (!c) return fail(PA_ERR_INVALID_ARG, "cache descriptor is NULL");
-    if (c->dtype != PA_F32 && c->dtype != PA_BF16)
-        return fail(PA_ERR_DTYPE, "dtype %d is neither PA_F32 (0) nor PA_BF16 (1)", c->dtype);
+    if (c->dtype != PA_F32 && c->dtype != PA_BF16 && !quantised(c->dtype))
+        return fail(PA_ERR_DTYPE, "dtype %d is not PA_F32, PA_BF16, PA_FP8_E4M3 or PA_INT8",
+                    c->dtype);
     if (c->num_blocks <= 0 || c->num_kv_heads <= 0)
         return fail(PA_ERR_INVALID_ARG, "num_blocks (%d) and num_kv_heads (%d) must be positive",
                     c->num_blocks, c->num_kv_heads);
@@ -115,8 +118,9 @@ int make_cache_map(CUtensorMap* map, const void* base, const pa_cache_desc* c) {
     cuuint64_t strides[1] = {(cuuint64_t)c->head_dim * e};
     cuuint32_t box[2] = {(cuuint32_t)(128 / e), 16u};
     cuuint32_t estr[2] = {1u, 1u};
-    CUresult r = fn(map, c->dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+    CUresult r = fn(map, c->dtype == PA_BF16  ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                         : c->dtype == PA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                              : CU_TENSOR_MAP_DATA_TYPE_UINT8,
                     2, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -284,8 +288,22 @@ static int decode_impl(void* out, const void* q, const void* k_cache, const void
                        int32_t num_heads, float scale, const pa_cache_desc* cache,
                        int32_t group_size, int32_t partition_size, void* workspace,
                        size_t workspace_bytes, void* stream, const int32_t* query_start = nullptr,
-                       int32_t num_query_tokens = -1, int32_t max_query_len = 0) {
+                       int32_t num_query_tokens = -1, int32_t max_query_len = 0,
+                       const float* k_scale = nullptr, const float* v_scale = nullptr) {
     Plan plan;
+    if (cache && quantised(cache->dtype) != (k_scale != nullptr || v_scale != nullptr))
+        return fail(PA_ERR_DTYPE, quantised(cache->dtype)
+                                      ? "a quantised cache decodes through pa_decode_quant"
+                                      : "pa_decode_quant needs a PA_FP8_E4M3 or PA_INT8 cache");
+    if (cache && quantised(cache->dtype)) {
+        if (!k_scale || !v_scale ||
+            (reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+            return fail(PA_ERR_INVALID_ARG, "pa_decode_quant: k_scale and v_scale must be 4-byte "
+                        "aligned device arrays of num_kv_heads floats");
+        if (cache->head_dim != 128)
+            return fail(PA_ERR_UNSUPPORTED, "quantised caches decode at head_dim 128 (got %d)",
+                        cache->head_dim);
+    }
     if (num_query_tokens > 65535)
         return fail(PA_ERR_INVALID_ARG, "num_query_tokens %d above 65535", num_query_tokens);
     int rc = plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan,
@@ -337,6 +355,8 @@ static int decode_impl(void* out, const void* q, const void* k_cache, const void
     p.num_partitions = plan.num_partitions;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.test_skip_position = g_test_skip_position;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
     p.query_start = plan.multi ? query_start : nullptr;
     p.q_chunks = plan.q_chunks;
     p.num_rows = plan.multi ? num_query_tokens : num_seqs;
@@ -363,6 +383,8 @@ int pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int3
                  void* k_cache, void* v_cache, const pa_cache_desc* cache, void* stream) {
     int rc = check_cache(cache);
     if (rc != PA_OK) return rc;
+    if (quantised(cache->dtype))
+        return fail(PA_ERR_DTYPE, "a quantised cache is written through pa_kv_append_quant");
     if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens %d is negative", num_tokens);
     if (num_tokens == 0) return PA_OK;
     if (!k || !v || !slot_mapping || !k_cache || !v_cache)
@@ -374,6 +396,42 @@ int pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping, int3
     cudaError_t e = pa::launch_kv_append(k, v, slot_mapping, num_tokens, k_cache, v_cache,
                                          copy_params(cache), static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : fail_cuda(e, "pa_kv_append launch");
+}
+
+int pa_kv_append_quant(const void* k, const void* v, const int64_t* slot_mapping,
+                       int32_t num_tokens, void* k_cache, void* v_cache, const float* k_scale,
+                       const float* v_scale, const pa_cache_desc* cache, void* stream) {
+    int rc = check_cache(cache);
+    if (rc != PA_OK) return rc;
+    if (!quantised(cache->dtype))
+        return fail(PA_ERR_DTYPE, "pa_kv_append_quant needs a PA_FP8_E4M3 or PA_INT8 cache");
+    if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "num_tokens %d is negative", num_tokens);
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale)
+        return fail(PA_ERR_INVALID_ARG, "pa_kv_append_quant: NULL pointer argument");
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_ALIGN, "pa_kv_append_quant: k, v and the caches must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(slot_mapping) & 7u) != 0 ||
+        (reinterpret_cast<uintptr_t>(k_scale) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(v_scale) & 3u) != 0)
+        return fail(PA_ERR_ALIGN, "pa_kv_append_quant: slot_mapping 8-byte, scales 4-byte aligned");
+    cudaError_t e = pa::launch_kv_append_quant(k, v, slot_mapping, num_tokens, k_cache, v_cache,
+                                               k_scale, v_scale, cache->dtype, copy_params(cache),
+                                               static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : fail_cuda(e, "pa_kv_append_quant launch");
+}
+
+int pa_decode_quant(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                    int32_t block_table_stride, const int32_t* context_lens,
+                    int32_t max_context_len, int32_t num_seqs, int32_t num_heads, float scale,
+                    const pa_cache_desc* cache, int32_t partition_size, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+    if (!k_scale || !v_scale)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_quant: k_scale and v_scale are required");
+    return decode_impl(out, q, k_cache, v_cache, block_tables, block_table_stride, context_lens,
+                       max_context_len, num_seqs, num_heads, scale, cache, 1, partition_size,
+                       workspace, workspace_bytes, stream, nullptr, -1, 0, k_scale, v_scale);
 }
 
 int pa_block_copy(const int64_t* src_dst_pairs, int32_t num_pairs, void* k_cache, void* v_cache,

@@ -79,6 +79,69 @@ block_copy_kernel(const int64_t* __restrict__ pairs, uint4* __restrict__ k_cache
     }
 }
 
+// Quantising append (KV cache quantisation, "AI 推理系列（十六）：PagedAttention——…",
+// mechanisms table; "PagedAttention原理详解…", § 量化技术): each thread turns
+// 16 bf16 elements of one (token, kv head) row into 16 one-byte codes of
+// y = x / scale[head] (binary32 division): FP8 E4M3 rounded to nearest even
+// and saturated to +-448, or int8 clamped to +-127 then rounded to nearest
+// even. The slot is checked as in kv_append_kernel.
+__device__ __forceinline__ uint32_t e4m3x2_code(float lo, float hi) {
+    uint32_t d;
+    asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tcvt.u32.u16 %0, t;\n\t}"
+        : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t int8_code(float y) {
+    return (uint32_t)(__float2int_rn(fminf(fmaxf(y, -127.f), 127.f)) & 0xff);
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads)
+kv_append_quant_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                       const int64_t* __restrict__ slot_mapping, int64_t total_chunks,
+                       uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                       const float* __restrict__ k_scale, const float* __restrict__ v_scale,
+                       CopyParams cp, int64_t num_slots) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total_chunks;
+         idx += stride) {
+        const int64_t row = idx / cp.row_vecs;          // token * num_kv_heads + head
+        const int32_t c = (int32_t)(idx - row * cp.row_vecs);
+        const int64_t token = row / cp.num_kv_heads;
+        const int32_t h = (int32_t)(row - token * cp.num_kv_heads);
+        const int64_t slot = __ldg(slot_mapping + token);
+        if (slot < 0) continue;                         // padding token
+        if (slot >= num_slots) {
+            atomicOr(&s_status_copy, kStatusBadIndex);
+            continue;
+        }
+        const int64_t blk = slot >> cp.log2_block_size;
+        const int64_t off = slot & (cp.block_size - 1);
+        const int64_t dst = ((blk * cp.num_kv_heads + h) * cp.block_size + off) * cp.row_vecs + c;
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+            const uint4* src = (kv ? v : k) + 2 * idx;  // 16 bf16 = two 16-byte chunks
+            const float sc = __ldg((kv ? v_scale : k_scale) + h);
+            const uint4 a = ld_stream(src), b = ld_stream(src + 1);
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            uint32_t out[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float y[4] = {__fdiv_rn(bf16_lo(w[2 * i]), sc), __fdiv_rn(bf16_hi(w[2 * i]), sc),
+                              __fdiv_rn(bf16_lo(w[2 * i + 1]), sc),
+                              __fdiv_rn(bf16_hi(w[2 * i + 1]), sc)};
+                if (FMT == 2)
+                    out[i] = e4m3x2_code(y[0], y[1]) | (e4m3x2_code(y[2], y[3]) << 16);
+                else
+                    out[i] = int8_code(y[0]) | (int8_code(y[1]) << 8) | (int8_code(y[2]) << 16) |
+                             (int8_code(y[3]) << 24);
+            }
+            (kv ? v_cache : k_cache)[dst] = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+    }
+}
+
 // Swap between two pools of the same block shape, either of which may be
 // pinned host memory mapped into the device address space (swap-out to host
 // when a request is preempted, swap-in when it resumes; "AI 推理系列（十六）：
@@ -148,6 +211,23 @@ cudaError_t launch_kv_append(const void* k, const void* v, const int64_t* slot_m
     kv_append_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(
         static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, total,
         static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), cp, num_slots);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kv_append_quant(const void* k, const void* v, const int64_t* slot_mapping,
+                                   int32_t num_tokens, void* k_cache, void* v_cache,
+                                   const float* k_scale, const float* v_scale, int fmt,
+                                   const CopyParams& cp, cudaStream_t stream) {
+    const int64_t total = (int64_t)num_tokens * cp.num_kv_heads * cp.row_vecs;
+    if (total == 0) return cudaSuccess;
+    int64_t blocks = (total + kThreads - 1) / kThreads;
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    const int64_t num_slots = (int64_t)cp.num_blocks * cp.block_size;
+    auto kern = fmt == 2 ? kv_append_quant_kernel<2> : kv_append_quant_kernel<3>;
+    kern<<<(unsigned)blocks, kThreads, 0, stream>>>(
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, total,
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), k_scale, v_scale, cp,
+        num_slots);
     return cudaGetLastError();
 }
 

@@ -237,9 +237,11 @@ __global__ void __launch_bounds__(SimtGeom<T, D>::kThreads)
 decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, const DecodeParams p) {
     using G = SimtGeom<T, D>;
+    using TQ = typename QType<T>::type;         // q / out element type
     constexpr int kConsumerWarps = G::kCW;
     constexpr int kThreads = G::kThreads;
-    constexpr int VEC = Elem<T>::kVec;          // elements per 16-byte chunk
+    constexpr int VEC = Elem<T>::kVec;          // cache elements per 16-byte chunk
+    constexpr int QV = Elem<TQ>::kVec;          // q elements per 16-byte chunk
     constexpr int CPR = D / VEC;                // chunks per row
     constexpr int RPL = 32 / CPR;               // rows per warp-wide pass
     constexpr int ITER = 16 / RPL;              // passes per 16-row sub-tile
@@ -256,7 +258,7 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
     const int64_t out_row = (int64_t)s * p.num_heads + h;
     if (t0 >= t1) {
         if (p.num_partitions == 1)
-            for (int d = threadIdx.x; d < D; d += kThreads) Elem<T>::store(p.out, out_row * D + d, 0.f);
+            for (int d = threadIdx.x; d < D; d += kThreads) Elem<TQ>::store(p.out, out_row * D + d, 0.f);
         return;
     }
     const int kh = h / (p.num_heads / p.num_kv_heads);
@@ -289,10 +291,15 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
         const uint32_t cx = (uint32_t)(c % 8);
         float qf[VEC];
         {
-            const uint4 raw = ld_v4(static_cast<const T*>(p.q) + out_row * D + c * VEC);
-            Elem<T>::widen(raw, qf);
+            // the K scale of a quantised cache folds into q (exactly 1 otherwise)
+            const float qs = p.scale_log2 * (p.k_scale != nullptr ? __ldg(p.k_scale + kh) : 1.f);
 #pragma unroll
-            for (int j = 0; j < VEC; ++j) qf[j] *= p.scale_log2;
+            for (int u = 0; u < VEC / QV; ++u) {
+                float f[QV];
+                Elem<TQ>::widen(ld_v4(static_cast<const TQ*>(p.q) + out_row * D + c * VEC + u * QV), f);
+#pragma unroll
+                for (int j = 0; j < QV; ++j) qf[u * QV + j] = f[j] * qs;
+            }
         }
         bool dead = false;
         for (int i = warp; i < n_sub && !dead; i += kConsumerWarps) {
@@ -399,13 +406,15 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
         wgt[w] = sm_m[w] == -INFINITY ? 0.f : exp2f(sm_m[w] - M);
         L = fmaf(sm_l[w], wgt[w], L);
     }
+    const float vs = p.v_scale != nullptr ? __ldg(p.v_scale + kh) : 1.f;
     for (int d = threadIdx.x; d < D; d += kThreads) {
         float o = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) o = fmaf(sm_o[w * D + d], wgt[w], o);
-        const float val = L > 0.f ? o / L : 0.f;
+        float val = L > 0.f ? o / L : 0.f;
+        if (p.v_scale != nullptr) val *= vs;  // V scale of a quantised cache
         if (p.num_partitions == 1)
-            Elem<T>::store(p.out, out_row * D + d, val);
+            Elem<TQ>::store(p.out, out_row * D + d, val);
         else
             p.ws_o[(out_row * p.num_partitions + part) * D + d] = val;
     }
@@ -1693,6 +1702,8 @@ cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bo
         return head_dim == 64 ? launch_simt_t<float, 64>(p, kmap, vmap, stream)
                               : launch_simt_t<float, 128>(p, kmap, vmap, stream);
     }
+    if (dtype == 2) return launch_simt_t<E4M3Code, 128>(p, kmap, vmap, stream);
+    if (dtype == 3) return launch_simt_t<Int8Code, 128>(p, kmap, vmap, stream);
     return head_dim == 64 ? launch_simt_t<__nv_bfloat16, 64>(p, kmap, vmap, stream)
                           : launch_simt_t<__nv_bfloat16, 128>(p, kmap, vmap, stream);
 }

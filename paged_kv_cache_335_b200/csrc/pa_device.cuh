@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -68,5 +69,52 @@ struct Elem<__nv_bfloat16> {
         reinterpret_cast<uint16_t*>(base)[idx] = float_to_bf16_bits(v);
     }
 };
+
+// Quantised cache codes (one byte per element; the value is code value x the
+// kv head's scale, applied by the caller of widen): tag types for Elem.
+struct E4M3Code {};
+struct Int8Code {};
+
+// Two FP8 E4M3 codes (low byte first) -> two floats, by the hardware
+// conversion to f16x2 (exact: every E4M3 value, NaN included, is an f16).
+__device__ __forceinline__ void e4m3x2_to_float2(uint32_t two, float& lo, float& hi) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(h2) : "h"((unsigned short)two));
+    const __half2 v = *reinterpret_cast<const __half2*>(&h2);
+    lo = __low2float(v);
+    hi = __high2float(v);
+}
+
+template <>
+struct Elem<E4M3Code> {
+    static constexpr int kVec = 16;
+    __device__ __forceinline__ static void widen(const uint4& c, float (&f)[16]) {
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            e4m3x2_to_float2(w[i] & 0xffffu, f[4 * i], f[4 * i + 1]);
+            e4m3x2_to_float2(w[i] >> 16, f[4 * i + 2], f[4 * i + 3]);
+        }
+    }
+};
+
+template <>
+struct Elem<Int8Code> {
+    static constexpr int kVec = 16;
+    __device__ __forceinline__ static void widen(const uint4& c, float (&f)[16]) {
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                f[4 * i + b] = (float)(int8_t)(uint8_t)(w[i] >> (8 * b));
+    }
+};
+
+// q / out element type for a cache element type (quantised caches: bf16).
+template <typename TC> struct QType { using type = TC; };
+template <> struct QType<E4M3Code> { using type = __nv_bfloat16; };
+template <> struct QType<Int8Code> { using type = __nv_bfloat16; };
 
 }  // namespace pa

@@ -46,6 +46,10 @@ struct DecodeParams {
     const int32_t* query_start;
     int32_t q_chunks;
     int32_t num_rows;           // rows of q / out: num_seqs, or the query tokens
+    // Quantised caches (codes): per-kv-head scales, K_t = value(code) * k_scale[kh];
+    // nullptr for bf16 / f32 caches.
+    const float* k_scale;
+    const float* v_scale;
 };
 
 struct CopyParams {
@@ -60,6 +64,12 @@ struct CopyParams {
 cudaError_t launch_kv_append(const void* k, const void* v, const int64_t* slot_mapping,
                              int32_t num_tokens, void* k_cache, void* v_cache,
                              const CopyParams& cp, cudaStream_t stream);
+// Quantising append: bf16 k, v [T][Hkv][D] -> codes (fmt 2 = FP8 E4M3, 3 = int8)
+// of x / scale[kv head].
+cudaError_t launch_kv_append_quant(const void* k, const void* v, const int64_t* slot_mapping,
+                                   int32_t num_tokens, void* k_cache, void* v_cache,
+                                   const float* k_scale, const float* v_scale, int fmt,
+                                   const CopyParams& cp, cudaStream_t stream);
 cudaError_t launch_block_copy(const int64_t* pairs, int32_t num_pairs, void* k_cache,
                               void* v_cache, const CopyParams& cp, cudaStream_t stream);
 // Blocks of one pool into another of the same block shape (either may be

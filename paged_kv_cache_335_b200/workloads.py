@@ -55,6 +55,9 @@ class Workload:
     # multi-token queries: int32 [S + 1]; sequence s owns q rows query_start[s] ..
     # query_start[s+1]-1, its last n_s context positions (None: one query per sequence)
     query_start: np.ndarray | None = None
+    # quantised caches: "fp8" (E4M3 codes) or "int8" codes with per-kv-head scales;
+    # q, new k / v and out stay in `dtype` (bf16)
+    kv_quant: str | None = None
 
     @property
     def torch_dtype(self):
@@ -63,6 +66,11 @@ class Workload:
     @property
     def elem_bytes(self) -> int:
         return 4 if self.dtype == "f32" else 2
+
+    @property
+    def kv_elem_bytes(self) -> int:
+        """Bytes per cached element: 1 for a quantised cache."""
+        return 1 if self.kv_quant else self.elem_bytes
 
     @property
     def num_tokens(self) -> int:
@@ -75,7 +83,7 @@ class Workload:
     def kv_bytes(self) -> int:
         """Logical K+V bytes one decode call reads: every context token, K and V."""
         return int(self.context_lens.astype(np.int64).sum()) * self.num_kv_heads * \
-            self.head_dim * 2 * self.elem_bytes
+            self.head_dim * 2 * self.kv_elem_bytes
 
     @property
     def num_query_rows(self) -> int:
@@ -94,11 +102,12 @@ class Workload:
 
     def append_bytes(self) -> int:
         """Bytes one append call moves: new k, v read and written once each."""
-        return 2 * 2 * self.num_tokens * self.num_kv_heads * self.head_dim * self.elem_bytes
+        return 2 * self.num_tokens * self.num_kv_heads * self.head_dim * \
+            (self.elem_bytes + self.kv_elem_bytes)
 
     def copy_bytes(self) -> int:
         """Bytes one block-copy call moves: K and V block read + written per pair."""
-        blk = self.num_kv_heads * self.block_size * self.head_dim * self.elem_bytes
+        blk = self.num_kv_heads * self.block_size * self.head_dim * self.kv_elem_bytes
         return 2 * 2 * int(self.copy_pairs.shape[0]) * blk
 
     def unique_kv_bytes(self) -> int:
@@ -112,7 +121,7 @@ class Workload:
                 fill = min(self.block_size, n - j * self.block_size)
                 seen[b] = max(seen.get(b, 0), fill)
         toks = sum(seen.values())
-        return toks * self.num_kv_heads * self.head_dim * 2 * self.elem_bytes
+        return toks * self.num_kv_heads * self.head_dim * 2 * self.kv_elem_bytes
 
 
 # ---------------------------------------------------------------------------
@@ -367,7 +376,22 @@ def restrict(wl: Workload, seq_ids) -> Workload:
     return sub
 
 
+def quantized(wl: Workload, fmt: str) -> Workload:
+    """The same step over a quantised cache ("fp8" E4M3 or "int8" codes); q, the
+    new k / v and the output stay bf16."""
+    if fmt not in ("fp8", "int8") or wl.dtype != "bf16":
+        raise ValueError("quantised caches: fmt fp8 / int8 over a bf16 workload")
+    sub = Workload(**{**wl.__dict__})
+    sub.name = f"{wl.name}_{fmt}"
+    sub.kv_quant = fmt
+    sub.description = f"{wl.description}; {fmt} KV codes with per-kv-head scales"
+    return sub
+
+
 def make(name: str, **kw) -> Workload:
+    for fmt in ("fp8", "int8"):
+        if name.endswith("_" + fmt) and name[:-len(fmt) - 1] in CONFIGS:
+            return quantized(CONFIGS[name[:-len(fmt) - 1]](**kw), fmt)
     if name not in CONFIGS:
         raise KeyError(f"unknown workload {name!r}; known: {sorted(CONFIGS)}")
     return CONFIGS[name](**kw)
@@ -393,6 +417,8 @@ def make_values(wl: Workload, device="cpu", poison: bool = False, seed_offset: i
     k_new = torch.randn((wl.num_tokens, Hkv, d), generator=g, device=device, dtype=dt)
     v_new = torch.randn((wl.num_tokens, Hkv, d), generator=g, device=device, dtype=dt)
     shape = (wl.num_blocks, Hkv, wl.block_size, d)
+    if wl.kv_quant:
+        return _quant_values(wl, device, g, q, k_new, v_new, shape, poison)
     k_cache = torch.randn(shape, generator=g, device=device, dtype=dt)
     v_cache = torch.randn(shape, generator=g, device=device, dtype=dt)
     if poison:
@@ -407,6 +433,43 @@ def make_values(wl: Workload, device="cpu", poison: bool = False, seed_offset: i
             k_cache[wi] = float("nan")
             v_cache[wi] = float("nan")
     return {"q": q, "k_new": k_new, "v_new": v_new, "k_cache": k_cache, "v_cache": v_cache}
+
+
+def _quant_values(wl, device, g, q, k_new, v_new, shape, poison):
+    """Quantised pools drawn as codes (no quantiser runs here): FP8 E4M3 codes
+    with a random sign, exponent field 4..10 and mantissa (values 2^-3 .. 15),
+    or int8 codes uniform in [-127, 127]; per-kv-head scales U(0.2, 0.3) (fp8)
+    or U(0.02, 0.03) (int8). Poisoned slots hold the NaN code (fp8) or -128."""
+    Hkv = wl.num_kv_heads
+
+    def codes():
+        if wl.kv_quant == "fp8":
+            sign = torch.randint(0, 2, shape, generator=g, device=device, dtype=torch.int32) << 7
+            exp = torch.randint(4, 11, shape, generator=g, device=device, dtype=torch.int32) << 3
+            man = torch.randint(0, 8, shape, generator=g, device=device, dtype=torch.int32)
+            return (sign | exp | man).to(torch.uint8)
+        return (torch.randint(-127, 128, shape, generator=g, device=device,
+                              dtype=torch.int32) & 0xFF).to(torch.uint8)
+
+    k_cache, v_cache = codes(), codes()
+    lo, hi = (0.2, 0.3) if wl.kv_quant == "fp8" else (0.02, 0.03)
+    k_scale = lo + (hi - lo) * torch.rand((Hkv,), generator=g, device=device, dtype=torch.float32)
+    v_scale = lo + (hi - lo) * torch.rand((Hkv,), generator=g, device=device, dtype=torch.float32)
+    if poison:
+        bad = 0x7F if wl.kv_quant == "fp8" else 0x80
+        blocks, offs, whole = poison_slots(wl)
+        if blocks.size:
+            bi = torch.as_tensor(blocks, device=device)
+            oi = torch.as_tensor(offs, device=device)
+            k_cache[bi, :, oi, :] = bad
+            v_cache[bi, :, oi, :] = bad
+        if whole.size:
+            wi = torch.as_tensor(whole, device=device)
+            k_cache[wi] = bad
+            v_cache[wi] = bad
+    view = torch.float8_e4m3fn if wl.kv_quant == "fp8" else torch.int8
+    return {"q": q, "k_new": k_new, "v_new": v_new, "k_cache": k_cache.view(view),
+            "v_cache": v_cache.view(view), "k_scale": k_scale, "v_scale": v_scale}
 
 
 def poison_slots(wl: Workload):
@@ -438,6 +501,8 @@ def to_numpy(t: torch.Tensor) -> np.ndarray:
         return t.view(torch.int16).numpy().view(np.uint16)
     if t.dtype == torch.float32:
         return t.numpy()
+    if t.dtype in (torch.float8_e4m3fn, torch.int8, torch.uint8):
+        return t.view(torch.uint8).numpy()           # quantised codes, raw bytes
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -470,6 +535,8 @@ def subproblem(wl: Workload, k_cache: torch.Tensor, v_cache: torch.Tensor,
     for i, r in enumerate(rows):
         tables[i, :len(r)] = r
     ids = torch.as_tensor(used if used else [0], dtype=torch.long, device=k_cache.device)
+    if k_cache.dtype in (torch.float8_e4m3fn, torch.int8):     # code pools: gather raw bytes
+        k_cache, v_cache = k_cache.view(torch.uint8), v_cache.view(torch.uint8)
     out = {
         "k_cache": to_numpy(k_cache.index_select(0, ids)),
         "v_cache": to_numpy(v_cache.index_select(0, ids)),

@@ -1,0 +1,168 @@
+"""Quantised KV caches (FP8 E4M3 / int8 codes, per-kv-head scales) on the GPU.
+
+The quantising append must match the oracle's codes bit for bit over the whole
+pool (edge values included: ties, saturation, infinities, NaN, signed zero,
+subnormals); decode over codes must meet the bf16 bars against the oracle's
+fp64 decode of value(code) * scale; block copy / swap move code pools exactly;
+the calls refuse descriptors of the wrong kind.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_335_b200 as pa
+from paged_kv_cache_335_b200 import workloads as W
+from tests import gpu_helpers as G
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _codes(t):
+    return W.to_numpy(t)
+
+
+def _quant_step(wl, vals, ps=0):
+    d = G.device_tensors(wl, vals)
+    kc, vc = vals["k_cache"], vals["v_cache"]
+    if wl.copy_pairs.shape[0]:
+        pa.pa_block_copy(d["pairs"], kc, vc)
+    if wl.num_tokens:
+        pa.pa_kv_append_quant(vals["k_new"], vals["v_new"], d["slots"], kc, vc, vals["k_scale"],
+                              vals["v_scale"])
+    out = torch.empty_like(vals["q"])
+    pa.pa_decode_quant(out, vals["q"], kc, vc, vals["k_scale"], vals["v_scale"], d["tables"],
+                       d["ctx"], wl.scale, max_context_len=wl.max_context_len, partition_size=ps)
+    return out
+
+
+def _oracle_step(wl, host):
+    kc, vc = host["k_cache"], host["v_cache"]
+    if wl.copy_pairs.shape[0]:
+        oracle.block_copy(wl.copy_pairs, kc, vc)
+    if wl.num_tokens:
+        oracle.kv_append_quant(host["k_new"], host["v_new"], wl.slot_mapping, kc, vc,
+                               host["k_scale"], host["v_scale"], wl.kv_quant)
+    return oracle.decode_quant(host["q"], kc, vc, host["k_scale"], host["v_scale"],
+                               wl.block_tables, wl.context_lens, wl.scale, wl.kv_quant,
+                               num_threads=G.THREADS)
+
+
+def _host(vals):
+    return {k: (W.to_numpy(t).copy() if t.dtype != torch.float32 else t.cpu().numpy().copy())
+            for k, t in vals.items()}
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("H,Hkv", [(8, 8), (16, 2), (12, 3), (32, 2)])
+@pytest.mark.parametrize("bs", [16, 64])
+def test_step_parity_edges(fmt, H, Hkv, bs):
+    ctx = [0, 1, 2, 15, 16, 17, 33, 64, 129, 511, 513, 1000]
+    wl = W.quantized(G.custom(len(ctx), H, Hkv, 128, bs, "bf16", ctx, seed=bs + H), fmt)
+    for ps in (-1, 64, 0):
+        vals = W.make_values(wl, DEV, poison=True)
+        host = _host(vals)
+        out = _quant_step(wl, vals, ps)
+        pa.pa_sync_check()
+        ref = _oracle_step(wl, host)
+        assert np.array_equal(_codes(vals["k_cache"]), host["k_cache"]), "k codes differ"
+        assert np.array_equal(_codes(vals["v_cache"]), host["v_cache"]), "v codes differ"
+        G.check_tolerance(G.to_f64(out), ref, "bf16", f"{wl.name} ps={ps}")
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_append_codes_bit_exact_on_edge_values(fmt, d):
+    """Ties, saturation, infinities, NaN, signed zero and subnormal quotients,
+    through binary32 division by per-head scales."""
+    wl = W.quantized(G.custom(4, 8, 4, d, 16, "bf16", [30, 1, 17, 64], seed=d), fmt)
+    vals = W.make_values(wl, DEV, poison=False)
+    special = torch.tensor([0.0, -0.0, float("inf"), -float("inf"), float("nan"), 1e30, -1e30,
+                            2.5, 3.5, -2.5, 448.0, 449.0, 1e-30, -3e-38, 0.375, 7.0],
+                           dtype=torch.float32)
+    k_new = vals["k_new"].float()
+    k_new.view(-1)[:special.numel()] = special.to(DEV)
+    vals["k_new"] = k_new.to(torch.bfloat16)
+    vals["k_scale"][0] = 0.5
+    vals["k_scale"][1] = 1.0 / 3.0
+    host = _host(vals)
+    d_ = G.device_tensors(wl, vals)
+    pa.pa_kv_append_quant(vals["k_new"], vals["v_new"], d_["slots"], vals["k_cache"],
+                          vals["v_cache"], vals["k_scale"], vals["v_scale"])
+    pa.pa_sync_check()
+    oracle.kv_append_quant(host["k_new"], host["v_new"], wl.slot_mapping, host["k_cache"],
+                           host["v_cache"], host["k_scale"], host["v_scale"], fmt)
+    assert np.array_equal(_codes(vals["k_cache"]), host["k_cache"])
+    assert np.array_equal(_codes(vals["v_cache"]), host["v_cache"])
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+def test_llama13b_full_size_sampled(fmt):
+    """The headline 13B step over a quantised pool, in the bench's launch
+    configuration: sampled sequences against the oracle, codes of the appended
+    slots bit-exact."""
+    wl = W.make(f"llama13b_bs16_{fmt}")
+    vals = W.make_values(wl, DEV, poison=(fmt == "fp8"))
+    out = _quant_step(wl, vals)
+    pa.pa_sync_check()
+    assert torch.isfinite(out.float()).all()
+    # appended codes against the oracle's quantiser on the same inputs
+    slots = torch.as_tensor(wl.slot_mapping, device=DEV)
+    b, o = slots // wl.block_size, slots % wl.block_size
+    for cache, new, sc in ((vals["k_cache"], vals["k_new"], vals["k_scale"]),
+                           (vals["v_cache"], vals["v_new"], vals["v_scale"])):
+        got = _codes(cache.view(torch.uint8)[b, :, o, :])
+        x = new.float().cpu().numpy()
+        want = np.stack([np.stack([oracle.quantize(x[t, h], float(sc[h]), fmt)
+                                   for h in range(wl.num_kv_heads)]) for t in range(x.shape[0])])
+        assert np.array_equal(got, want)
+    seqs = G.sample_seqs(wl, 6)
+    sub = W.subproblem(wl, vals["k_cache"], vals["v_cache"], seqs, vals["q"])
+    ref = oracle.decode_quant(sub["q"], sub["k_cache"], sub["v_cache"],
+                              vals["k_scale"].cpu().numpy(), vals["v_scale"].cpu().numpy(),
+                              sub["block_tables"], sub["context_lens"], wl.scale, fmt,
+                              num_threads=G.THREADS)
+    G.check_tolerance(G.to_f64(out[torch.as_tensor(seqs, device=DEV)]), ref, "bf16", wl.name)
+
+
+def test_copy_and_swap_move_code_pools():
+    wl = W.quantized(W.cow_beam4(num_prompts=2, prompt_len=100, max_suffix=20, num_heads=16,
+                                 num_kv_heads=2, head_dim=128), "fp8")
+    vals = W.make_values(wl, DEV, poison=True)
+    host = _host(vals)
+    out = _quant_step(wl, vals)
+    pa.pa_sync_check()
+    ref = _oracle_step(wl, host)
+    assert np.array_equal(_codes(vals["k_cache"]), host["k_cache"])
+    G.check_tolerance(G.to_f64(out), ref, "bf16", "cow fp8")
+    hk = torch.zeros((8,) + tuple(vals["k_cache"].shape[1:]), dtype=torch.uint8).pin_memory()
+    hv = torch.zeros_like(hk).pin_memory()
+    pairs = np.array([[3, 0], [7, 5]], np.int64)
+    pa.pa_block_swap(torch.as_tensor(pairs, device=DEV), vals["k_cache"], vals["v_cache"],
+                     hk.view(torch.float8_e4m3fn), hv.view(torch.float8_e4m3fn))
+    torch.cuda.synchronize()
+    assert np.array_equal(hk.numpy()[0], host["k_cache"][3])
+    assert np.array_equal(hv.numpy()[5], host["v_cache"][7])
+
+
+def test_wrong_descriptor_kind_refused():
+    wl = W.quantized(G.custom(2, 8, 8, 128, 16, "bf16", [20, 30], seed=2), "int8")
+    vals = W.make_values(wl, DEV)
+    d = G.device_tensors(wl, vals)
+    out = torch.empty_like(vals["q"])
+    with pytest.raises(pa.PAError) as e:
+        pa.pa_decode(out, vals["q"], vals["k_cache"], vals["v_cache"], d["tables"], d["ctx"],
+                     wl.scale, max_context_len=30)
+    assert e.value.code == pa.PA_ERR_DTYPE
+    with pytest.raises(pa.PAError) as e:
+        pa.pa_kv_append(vals["k_new"], vals["v_new"], d["slots"], vals["k_cache"], vals["v_cache"])
+    assert e.value.code == pa.PA_ERR_DTYPE
+    wl64 = W.quantized(G.custom(2, 8, 8, 64, 16, "bf16", [20, 30], seed=2), "fp8")
+    v64 = W.make_values(wl64, DEV)
+    d64 = G.device_tensors(wl64, v64)
+    with pytest.raises(pa.PAError) as e:
+        pa.pa_decode_quant(torch.empty_like(v64["q"]), v64["q"], v64["k_cache"], v64["v_cache"],
+                           v64["k_scale"], v64["v_scale"], d64["tables"], d64["ctx"], wl64.scale,
+                           max_context_len=30)
+    assert e.value.code == pa.PA_ERR_UNSUPPORTED
