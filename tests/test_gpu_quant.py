@@ -6,6 +6,8 @@ subnormals); decode over codes must meet the bf16 bars against the oracle's
 fp64 decode of value(code) * scale; block copy / swap move code pools exactly;
 the calls refuse descriptors of the wrong kind.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -151,13 +153,18 @@ def test_wrong_descriptor_kind_refused():
     vals = W.make_values(wl, DEV)
     d = G.device_tensors(wl, vals)
     out = torch.empty_like(vals["q"])
-    with pytest.raises(pa.PAError) as e:
-        pa.pa_decode(out, vals["q"], vals["k_cache"], vals["v_cache"], d["tables"], d["ctx"],
-                     wl.scale, max_context_len=30)
-    assert e.value.code == pa.PA_ERR_DTYPE
-    with pytest.raises(pa.PAError) as e:
-        pa.pa_kv_append(vals["k_new"], vals["v_new"], d["slots"], vals["k_cache"], vals["v_cache"])
-    assert e.value.code == pa.PA_ERR_DTYPE
+    lib = pa.load_library()
+    desc = pa.cache_desc(vals["k_cache"])
+    P = ctypes.c_void_p
+    rc = lib.pa_decode(P(out.data_ptr()), P(vals["q"].data_ptr()), P(vals["k_cache"].data_ptr()),
+                       P(vals["v_cache"].data_ptr()), P(d["tables"].data_ptr()), 2,
+                       P(d["ctx"].data_ptr()), 30, 2, 8, ctypes.c_float(wl.scale),
+                       ctypes.byref(desc), 0, None, 0, None)
+    assert rc == pa.PA_ERR_DTYPE                       # codes need pa_decode_quant
+    rc = lib.pa_kv_append(P(vals["k_new"].data_ptr()), P(vals["v_new"].data_ptr()),
+                          P(d["slots"].data_ptr()), 2, P(vals["k_cache"].data_ptr()),
+                          P(vals["v_cache"].data_ptr()), ctypes.byref(desc), None)
+    assert rc == pa.PA_ERR_DTYPE                       # codes need pa_kv_append_quant
     wl64 = W.quantized(G.custom(2, 8, 8, 64, 16, "bf16", [20, 30], seed=2), "fp8")
     v64 = W.make_values(wl64, DEV)
     d64 = G.device_tensors(wl64, v64)
