@@ -26,6 +26,8 @@
 // The arithmetic order depends only on logical token positions.
 #include <math.h>
 
+#include <type_traits>
+
 #include "pa_device.cuh"
 #include "pa_internal.h"
 #include "pa_tma.cuh"
@@ -574,20 +576,188 @@ __device__ __forceinline__ void mma_softmax_pv(const float (&sc)[4], uint4 (&vr)
     }
 }
 
+// ---------------------------------------------------------------------------
+// The tensor-core step over quantised codes (FP8 E4M3 / int8, head_dim 128):
+// codes become f16 exactly (every E4M3 value and every integer up to 2048 is
+// an f16), q becomes f16 exactly within f16 range, and the MMAs run in f16
+// with fp32 accumulation. K fragments: thread (r, c) reads 16-byte chunks
+// 2c, 2c+1 of rows r, r+8; k-step ks takes word ks & 3 of chunk 2c + ks / 4,
+// so its head_dim positions are 32c + 4 ks + {0,1} (A cols 2c, 2c+1) and
+// + {2,3} (cols 2c+8, 2c+9); q uses the same positions. V fragments: chunk r
+// of tokens 2c, 2c+1, 2c+8, 2c+9; m-tile t rows r / r+8 are head_dim
+// 16 r + 2t / + 1.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ float f16_lo(uint32_t w) {
+    return __low2float(*reinterpret_cast<const __half2*>(&w));
+}
+__device__ __forceinline__ float f16_hi(uint32_t w) {
+    return __high2float(*reinterpret_cast<const __half2*>(&w));
+}
+
+// Word t = [x0, y0, x1, y1] (bytes, low first) of codes -> f16x2 (x0, y0) and
+// (x1, y1). Int8 words arrive with their sign bits flipped (byte = code + 128):
+// 0x64uu as an f16 is 1024 + u, and subtracting 1152 leaves the code.
+template <typename TC>
+__device__ __forceinline__ void code_pairs_f16(uint32_t t, uint32_t& p0, uint32_t& p1) {
+    if constexpr (std::is_same<TC, E4M3Code>::value) {
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+            "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+            : "=r"(p0), "=r"(p1) : "r"(t));
+    } else {
+        const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+        uint32_t u0 = __byte_perm(t, 0x64646464u, 0x5140), u1 = __byte_perm(t, 0x64646464u, 0x7362);
+        const __half2 h0 = __hsub2(*reinterpret_cast<__half2*>(&u0), bias);
+        const __half2 h1 = __hsub2(*reinterpret_cast<__half2*>(&u1), bias);
+        p0 = *reinterpret_cast<const uint32_t*>(&h0);
+        p1 = *reinterpret_cast<const uint32_t*>(&h1);
+    }
+}
+
+template <typename TC>
+__device__ __forceinline__ uint32_t code_word(uint32_t w) {
+    return std::is_same<TC, Int8Code>::value ? w ^ 0x80808080u : w;
+}
+
+// q row of the B operand for codes: head_dim 32c .. 32c+31 as 16 f16x2 words.
+__device__ __forceinline__ void load_q_codes(const uint16_t* qrow, int c, uint4 (&q)[4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const uint4 raw = ld_v4(qrow + 32 * c + 8 * u);
+        q[u] = make_uint4(pack_f16x2(bf16_lo(raw.x), bf16_hi(raw.x)),
+                          pack_f16x2(bf16_lo(raw.y), bf16_hi(raw.y)),
+                          pack_f16x2(bf16_lo(raw.z), bf16_hi(raw.z)),
+                          pack_f16x2(bf16_lo(raw.w), bf16_hi(raw.w)));
+    }
+}
+
+template <typename TC>
+__device__ __forceinline__ void codes_qk(uint32_t kb, const uint4 (&q)[4], int r, int c,
+                                         float (&sc)[4]) {
+    uint4 kr[2][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        kr[0][h] = lds128(kb + swz(r, 2 * c + h));
+        kr[1][h] = lds128(kb + swz(r + 8, 2 * c + h));
+    }
+    float sd[4] = {0.f, 0.f, 0.f, 0.f};
+    sc[0] = sc[1] = sc[2] = sc[3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t wa = code_word<TC>(word(kr[0][ks >> 2], ks & 3));
+        const uint32_t wb = code_word<TC>(word(kr[1][ks >> 2], ks & 3));
+        uint32_t a0, a1, a2, a3;
+        code_pairs_f16<TC>(wa, a0, a2);
+        code_pairs_f16<TC>(wb, a1, a3);
+        const uint32_t b0 = word(q[ks >> 1], 2 * (ks & 1)), b1 = word(q[ks >> 1], 2 * (ks & 1) + 1);
+        if (ks & 1)
+            mma_16816_f16(sd, a0, a1, a2, a3, b0, b1);
+        else
+            mma_16816_f16(sc, a0, a1, a2, a3, b0, b1);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sc[e] += sd[e];
+}
+
+__device__ __forceinline__ void codes_load_v(uint32_t vb, int r, int c, uint4 (&vr)[4]) {
+    vr[0] = lds128(vb + swz(2 * c, r));
+    vr[1] = lds128(vb + swz(2 * c + 1, r));
+    vr[2] = lds128(vb + swz(2 * c + 8, r));
+    vr[3] = lds128(vb + swz(2 * c + 9, r));
+}
+
+// As mma_softmax_pv, over codes: scores scaled by scale_log2 x k_scale (sl),
+// weights packed as f16, V^T fragments built from the code chunks.
+template <typename TC>
+__device__ __forceinline__ void codes_softmax_pv(const float (&sc)[4], uint4 (&vr)[4], int nvalid,
+                                                 float sl, int r, int c, float (&acc)[8][4],
+                                                 float& m0, float& m1, float& l0, float& l1) {
+    const bool lo_ok = r < nvalid, hi_ok = r + 8 < nvalid;
+    const float s0 = lo_ok ? sc[0] * sl : -INFINITY;
+    const float s1 = lo_ok ? sc[1] * sl : -INFINITY;
+    const float s2 = hi_ok ? sc[2] * sl : -INFINITY;
+    const float s3 = hi_ok ? sc[3] * sl : -INFINITY;
+    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const bool moved = __any_sync(0xffffffffu, mn0 != m0 || mn1 != m1);
+    const float al0 = moved ? exp2f(m0 - mn0) : 1.f;
+    const float al1 = moved ? exp2f(m1 - mn1) : 1.f;
+    const uint32_t x0 = pack_f16x2(exp2f(s0 - mn0), exp2f(s1 - mn1));
+    const uint32_t x1 = pack_f16x2(exp2f(s2 - mn0), exp2f(s3 - mn1));
+    l0 = fmaf(l0, al0, f16_lo(x0) + f16_lo(x1));
+    l1 = fmaf(l1, al1, f16_hi(x0) + f16_hi(x1));
+    m0 = mn0;
+    m1 = mn1;
+    if (moved) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            acc[t][0] *= al0;
+            acc[t][1] *= al1;
+            acc[t][2] *= al0;
+            acc[t][3] *= al1;
+        }
+    }
+    const uint32_t pb0 = movmatrix_trans(x0);
+    const uint32_t pb1 = movmatrix_trans(x1);
+    if (nvalid < 16) {  // a zero code is the value 0 in both formats
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        if (2 * c >= nvalid) vr[0] = z;
+        if (2 * c + 1 >= nvalid) vr[1] = z;
+        if (2 * c + 8 >= nvalid) vr[2] = z;
+        if (2 * c + 9 >= nvalid) vr[3] = z;
+    }
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t va = code_word<TC>(word(vr[0], w)), vb = code_word<TC>(word(vr[1], w));
+        const uint32_t vc = code_word<TC>(word(vr[2], w)), vd = code_word<TC>(word(vr[3], w));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // m-tile t = 2w + h: bytes 2h, 2h+1 of word w
+            const uint32_t sel = h ? 0x7362u : 0x5140u;
+            uint32_t a0, a1, a2, a3;
+            code_pairs_f16<TC>(__byte_perm(va, vb, sel), a0, a1);
+            code_pairs_f16<TC>(__byte_perm(vc, vd, sel), a2, a3);
+            mma_16816_f16(acc[2 * w + h], a0, a1, a2, a3, pb0, pb1);
+        }
+    }
+}
+
 // Store one warp's item result (heads 2c, 2c+1 of query rows head0 + n) from its
 // registers: bf16 output when P == 1, else the normalised partial and (m, l).
-template <int D>
+// kCodes: the m-tile rows of the code consumer (head_dim 16 r + 2t, + 1) and
+// the V scale `vs` of a quantised cache.
+template <int D, bool kCodes = false>
 __device__ __forceinline__ void mma_store_item(const DecodeParams& p, int64_t head0, int group,
                                                int part, int r, int c, const float (&acc)[D / 16][4],
-                                               float m0, float m1, float l0, float l1) {
+                                               float m0, float m1, float l0, float l1,
+                                               float vs = 1.f) {
     constexpr int MT = D / 16;
     const int P = p.num_partitions;
-    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f;
-    const float inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    float inv0 = l0 > 0.f ? 1.f / l0 : 0.f;
+    float inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    if constexpr (kCodes) {
+        inv0 *= vs;
+        inv1 *= vs;
+    }
     const int n0 = 2 * c, n1 = 2 * c + 1;
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
-        const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
+        const int d0 = kCodes ? 16 * r + 2 * t : (t >> 2) * 64 + r * 8 + 2 * (t & 3);
         if (P == 1) {
             if (n0 < group)
                 *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + (head0 + n0) * D + d0) =
@@ -618,8 +788,8 @@ __device__ __forceinline__ void mma_store_item(const DecodeParams& p, int64_t he
     }
 }
 
-template <int D>
-using MmaGeom = Geom<__nv_bfloat16, D, PA_MMA_CONSUMER_WARPS, PA_MMA_RING_BYTES>;
+template <int D, typename TC = __nv_bfloat16>
+using MmaGeom = Geom<TC, D, PA_MMA_CONSUMER_WARPS, PA_MMA_RING_BYTES>;
 
 template <int D>
 constexpr int merge_floats() {
@@ -690,13 +860,16 @@ __device__ __forceinline__ Item item_next(ItemWalk& w, const DecodeParams& p, in
 // entries fetched one 32-sub-tile batch ahead), while the consumers finish one
 // item (cross-warp merge, store) and start the next (q fragments fetched one
 // item ahead).
-template <int D>
-__global__ void __launch_bounds__(MmaGeom<D>::kThreads, PA_MMA_MIN_BLOCKS)
+template <int D, typename TC = __nv_bfloat16>
+__global__ void __launch_bounds__(MmaGeom<D, TC>::kThreads, PA_MMA_MIN_BLOCKS)
 decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
                       int num_items) {
     using T = __nv_bfloat16;
-    using G = MmaGeom<D>;
+    using G = MmaGeom<D, TC>;
+    constexpr bool kCodes = !std::is_same<TC, __nv_bfloat16>::value;
+    static_assert(!kCodes || D == 128, "quantised codes: head_dim 128");
+    static_assert(!kCodes || G::kCW <= 2, "the code consumer's head_dim order needs the register merge");
     constexpr int kConsumerWarps = G::kCW;
     constexpr int KCH = D / 32;  // 16-byte K chunks per row per thread (2 k-steps each)
     constexpr int VCH = D / 64;  // V boxes
@@ -771,9 +944,13 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
         const int64_t head0 = (int64_t)it.s * p.num_heads + (int64_t)it.kh * group;
         if (it.valid && it.t0 < it.t1 && r < group) {
             const uint16_t* qrow = static_cast<const uint16_t*>(p.q) + (head0 + r) * D;
+            if constexpr (kCodes) {
+                load_q_codes(qrow, c, q);
+            } else {
 #pragma unroll
-            for (int jp = 0; jp < KCH; ++jp)
-                q[jp] = ld_v4(qrow + (jp >> 1) * 64 + (2 * c + (jp & 1)) * 8);
+                for (int jp = 0; jp < KCH; ++jp)
+                    q[jp] = ld_v4(qrow + (jp >> 1) * 64 + (2 * c + (jp & 1)) * 8);
+            }
         } else {
 #pragma unroll
             for (int jp = 0; jp < KCH; ++jp) q[jp] = make_uint4(0u, 0u, 0u, 0u);
@@ -796,6 +973,8 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
         } else {
             const int t0 = cur.t0, t1 = cur.t1;
             const int n_sub = (t1 - t0 + 15) >> 4;
+            // score scale (the K scale of a quantised cache folds in)
+            const float sl = kCodes ? p.scale_log2 * __ldg(p.k_scale + cur.kh) : p.scale_log2;
             float acc[MT][4];
 #pragma unroll
             for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
@@ -815,13 +994,23 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 const uint32_t kb = ring.stages + st * G::kStageBytes;
                 const uint32_t vb = kb + G::kBoxes * kBoxBytes;
                 float sc[4];
-                mma_qk<D>(kb, qcur, r, c, sc);
-                uint4 vr[4][VCH];
-                mma_load_v<D>(vb, r, c, vr);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
-                if (!valid) continue;
-                mma_softmax_pv<D>(sc, vr, t1 - (t0 + (i << 4)), p.scale_log2, r, c, acc, m0, m1, l0, l1);
+                if constexpr (kCodes) {
+                    codes_qk<TC>(kb, qcur, r, c, sc);
+                    uint4 vr[4];
+                    codes_load_v(vb, r, c, vr);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
+                    if (!valid) continue;
+                    codes_softmax_pv<TC>(sc, vr, t1 - (t0 + (i << 4)), sl, r, c, acc, m0, m1, l0, l1);
+                } else {
+                    mma_qk<D>(kb, qcur, r, c, sc);
+                    uint4 vr[4][VCH];
+                    mma_load_v<D>(vb, r, c, vr);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
+                    if (!valid) continue;
+                    mma_softmax_pv<D>(sc, vr, t1 - (t0 + (i << 4)), sl, r, c, acc, m0, m1, l0, l1);
+                }
             }
             g += n_sub;
 #pragma unroll
@@ -867,7 +1056,9 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
             }
             if constexpr (kConsumerWarps <= 2) {
                 // One warp holds the whole item: normalise and store from registers.
-                if (warp == 0) mma_store_item<D>(p, head0, group, cur.part, r, c, acc, m0, m1, l0, l1);
+                if (warp == 0)
+                    mma_store_item<D, kCodes>(p, head0, group, cur.part, r, c, acc, m0, m1, l0, l1,
+                                              kCodes ? __ldg(p.v_scale + cur.kh) : 1.f);
                 if constexpr (kConsumerWarps == 2) named_barrier(1, 64);  // buffer free again
             } else {
                 // Cross-warp merge of this item, in fixed warp order. Buffers alternate
@@ -1625,12 +1816,12 @@ cudaError_t launch_simt_t(const DecodeParams& p, const CUtensorMap& km, const CU
     return cudaGetLastError();
 }
 
-template <int D>
+template <int D, typename TC = __nv_bfloat16>
 cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
                          cudaStream_t stream) {
-    using G = MmaGeom<D>;
+    using G = MmaGeom<D, TC>;
     constexpr size_t smem = smem_bytes<G>(merge_bytes<D>());
-    auto kernel = decode_tma_mma_kernel<D>;
+    auto kernel = decode_tma_mma_kernel<D, TC>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -1695,6 +1886,8 @@ cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bo
                               const CUtensorMap& kmap, const CUtensorMap& vmap,
                               cudaStream_t stream) {
     if (mma) {
+        if (dtype == 2) return launch_mma_t<128, E4M3Code>(p, kmap, vmap, stream);
+        if (dtype == 3) return launch_mma_t<128, Int8Code>(p, kmap, vmap, stream);
         return head_dim == 64 ? launch_mma_t<64>(p, kmap, vmap, stream)
                               : launch_mma_t<128>(p, kmap, vmap, stream);
     }
@@ -1711,7 +1904,9 @@ cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bo
 int mma_ctas_per_sm() { return PA_MMA_MIN_BLOCKS; }
 
 bool mma_supported(int dtype, int head_dim, int group) {
-    return dtype == 1 && (head_dim == 64 || head_dim == 128) && group >= 2 && group <= kGroupMax;
+    const bool codes = (dtype == 2 || dtype == 3) && head_dim == 128;
+    return (codes || (dtype == 1 && (head_dim == 64 || head_dim == 128))) && group >= 2 &&
+           group <= kGroupMax;
 }
 
 // Query columns (member, head) -> n-tiles of 8 -> consumer warps: one n-tile

@@ -99,16 +99,24 @@ struct Elem<E4M3Code> {
     }
 };
 
+// Int8 codes -> floats without an integer conversion: with the sign bit
+// flipped, byte b is u = code + 128 in [0, 255]; one byte permute places it
+// as the low mantissa byte of 2^23 (bits 0x4B0000uu = 2^23 + u exactly) and
+// one subtraction of 2^23 + 128 leaves the code, exactly.
 template <>
 struct Elem<Int8Code> {
     static constexpr int kVec = 16;
     __device__ __forceinline__ static void widen(const uint4& c, float (&f)[16]) {
-        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        const uint32_t w[4] = {c.x ^ 0x80808080u, c.y ^ 0x80808080u, c.z ^ 0x80808080u,
+                               c.w ^ 0x80808080u};
+        constexpr float kBias = 8388736.0f;  // 2^23 + 128
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-                f[4 * i + b] = (float)(int8_t)(uint8_t)(w[i] >> (8 * b));
+        for (int i = 0; i < 4; ++i) {
+            f[4 * i + 0] = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540)) - kBias;
+            f[4 * i + 1] = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7541)) - kBias;
+            f[4 * i + 2] = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7542)) - kBias;
+            f[4 * i + 3] = __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7543)) - kBias;
+        }
     }
 };
 

@@ -173,3 +173,22 @@ def test_wrong_descriptor_kind_refused():
                            v64["k_scale"], v64["v_scale"], d64["tables"], d64["ctx"], wl64.scale,
                            max_context_len=30)
     assert e.value.code == pa.PA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+def test_llama70b_gqa_tensor_core_path_sampled(fmt):
+    """The 70B GQA step (8 x 32K contexts, group 8) over codes runs the
+    tensor-core consumer (f16 MMAs on exactly converted codes) with the library
+    partition policy; one sequence against the oracle."""
+    wl = W.make(f"llama70b_gqa_{fmt}")
+    vals = W.make_values(wl, DEV, poison=(fmt == "fp8"))
+    out = _quant_step(wl, vals, 0)
+    pa.pa_sync_check()
+    assert G.last_kernel() == pa.PA_KERNEL_MMA
+    assert torch.isfinite(out.float()).all()
+    sub = W.subproblem(wl, vals["k_cache"], vals["v_cache"], [5], vals["q"])
+    ref = oracle.decode_quant(sub["q"], sub["k_cache"], sub["v_cache"],
+                              vals["k_scale"].cpu().numpy(), vals["v_scale"].cpu().numpy(),
+                              sub["block_tables"], sub["context_lens"], wl.scale, fmt,
+                              num_threads=G.THREADS)
+    G.check_tolerance(G.to_f64(out[5:6]), ref, "bf16", wl.name)
