@@ -227,7 +227,8 @@ def profile_traffic(kernel_file, workload):
         if not name.endswith((".md", ".txt")):
             continue
         text = open(os.path.join(pdir, name), encoding="utf-8").read()
-        if f"source_sha256: {sha}" not in text or f"workload: {workload}" not in text:
+        lines = text.splitlines()
+        if f"source_sha256: {sha}" not in lines or f"workload: {workload}" not in lines:
             continue
         m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
         if m:
