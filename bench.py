@@ -52,7 +52,8 @@ EXTRA_CONFIGS = [("llama7b", "llama7b", None, 1), ("llama13b_bs16", "llama13b_bs
 # pa_test_last_decode_kernel() -> the decode kernel a call enqueued
 KERNEL_NAMES = {0: "decode_tma_simt_kernel (CUDA-core)",
                 1: "decode_tma_mma_kernel (persistent, tensor-core GQA)",
-                2: "decode_tma_grouped_kernel (persistent, grouped sequences)"}
+                2: "decode_tma_grouped_kernel (persistent, grouped sequences)",
+                3: "decode_umma_grouped_kernel (tcgen05, grouped sequences)"}
 FALLBACK_HBM_GBS = 6650.0
 DATASHEET_HBM_GBS = 8000.0
 L2_FLUSH_BYTES = 512 << 20          # > 2x the 126 MB L2

@@ -325,6 +325,26 @@ int pa_decode_quant(void* out, const void* q, const void* k_cache, const void* v
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * pa_set_grouped_consumer — which consumer pa_decode_grouped and pa_decode_multi
+ * use for bf16 head_dim 128 with 16..64 query columns (sequences or query
+ * tokens x query heads per kv head):
+ *   PA_GROUPED_MMA_SYNC (default): one warp per 8 query columns, m16n8k16 MMAs
+ *     from registers;
+ *   PA_GROUPED_TCGEN05: one thread issues tcgen05.mma from shared memory with
+ *     S, P and O in tensor memory, softmax warps read and write TMEM.
+ * Both compute the same attention within the same tolerance of the exact
+ * value, and both keep a sequence's result independent of which blocks it
+ * shares; they round differently from each other. On the measured beam and
+ * verification workloads the default is faster (decode-sized contractions
+ * leave the single-issuer pipeline latency-bound). Process-wide, not
+ * synchronised with calls in flight on other threads: set it before decoding.
+ * Returns the previous consumer, or PA_ERR_INVALID_ARG for an unknown value.
+ */
+#define PA_GROUPED_MMA_SYNC 0
+#define PA_GROUPED_TCGEN05 1
+int pa_set_grouped_consumer(int consumer);
+
+/*
  * pa_block_copy — copy whole physical blocks, the copy-on-write step that
  * [P1 § 2 写入时拷贝], [P2 § Copy-on-Write、并行采样与 Prefix Caching] and
  * [P3 § PagedAttention的三大核心优势] describe: when a sequence is about to

@@ -13,12 +13,15 @@
  * pa_test_last_decode_kernel — which decode kernel the calling thread's last
  * successful pa_decode / pa_decode_grouped / pa_decode_noalloc enqueued:
  * PA_KERNEL_SIMT (CUDA-core consumer), PA_KERNEL_MMA (tensor-core GQA
- * consumer), PA_KERNEL_GROUPED (grouped sequences), or -1 if none yet. Lets
+ * consumer), PA_KERNEL_GROUPED (grouped sequences / multi-token queries),
+ * PA_KERNEL_GROUPED_TCGEN05 (the same on the tcgen05 consumer, see
+ * pa_set_grouped_consumer), or -1 if none yet. Lets
  * tests confirm which path a shape takes.
  */
 #define PA_KERNEL_SIMT 0
 #define PA_KERNEL_MMA 1
 #define PA_KERNEL_GROUPED 2
+#define PA_KERNEL_GROUPED_TCGEN05 3
 #ifndef PA_TEST_H
 #define PA_TEST_H
 

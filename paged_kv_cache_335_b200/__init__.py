@@ -40,9 +40,12 @@ PA_BF16 = 1
 PA_FP8_E4M3 = 2             # quantised caches: torch.float8_e4m3fn / torch.int8 code tensors
 PA_INT8 = 3
 PA_NOALLOC_SCRATCH_BYTES = 32 << 20
+PA_GROUPED_MMA_SYNC = 0     # pa_set_grouped_consumer() values
+PA_GROUPED_TCGEN05 = 1
 PA_KERNEL_SIMT = 0          # pa_test_last_decode_kernel() values
 PA_KERNEL_MMA = 1
 PA_KERNEL_GROUPED = 2
+PA_KERNEL_GROUPED_TCGEN05 = 3
 
 _lock = threading.Lock()
 _lib = None
@@ -111,6 +114,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_test_skip_load.argtypes = [i32]
         lib.pa_test_skip_load.restype = None
         lib.pa_test_last_decode_kernel.argtypes = []
+        lib.pa_set_grouped_consumer.argtypes = [ctypes.c_int]
         lib.pa_stream_read.restype = ctypes.c_int
         lib.pa_get_last_error.argtypes = []
         lib.pa_get_last_error.restype = ctypes.c_char_p
@@ -496,6 +500,14 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scal
         float(scale), ctypes.byref(desc), int(partition_size), _stream(stream)))
 
 
+def pa_set_grouped_consumer(consumer: int) -> int:
+    """Select the grouped / multi-token consumer (PA_GROUPED_MMA_SYNC or
+    PA_GROUPED_TCGEN05); returns the previous one. Process-wide."""
+    rc = load_library().pa_set_grouped_consumer(int(consumer))
+    _check(min(rc, 0))
+    return rc
+
+
 def pa_sync_check(stream=None) -> None:
     """Wait for the stream; raise PAError if a kernel met an out-of-range index."""
     _check(load_library().pa_sync_check(_stream(stream)))
@@ -505,5 +517,6 @@ __all__ = ["pa_kv_append", "pa_decode", "pa_decode_noalloc", "pa_block_copy", "p
            "pa_decode_num_partitions", "pa_decode_grouped", "pa_decode_grouped_workspace_size",
            "pa_decode_grouped_num_partitions", "pa_decode_multi", "pa_decode_multi_workspace_size",
            "pa_decode_multi_num_partitions", "pa_kv_append_quant", "pa_decode_quant", "pa_block_swap",
+           "pa_set_grouped_consumer",
            "pa_sync_check", "pa_cache_desc", "cache_desc",
            "load_library", "header_functions", "PAError"]

@@ -369,7 +369,11 @@ static int decode_impl(void* out, const void* q, const void* k_cache, const void
             ? pa::launch_decode_grouped(p, cache->head_dim, plan.group_size, kmap, vmap, st)
             : pa::launch_decode_tma(p, cache->dtype, cache->head_dim, plan.use_mma, kmap, vmap, st);
     if (e != cudaSuccess) return fail_cuda(e, "pa_decode launch");
-    t_last_kernel = plan.grouped ? PA_KERNEL_GROUPED : plan.use_mma ? PA_KERNEL_MMA : PA_KERNEL_SIMT;
+    t_last_kernel = !plan.grouped ? (plan.use_mma ? PA_KERNEL_MMA : PA_KERNEL_SIMT)
+                    : pa::grouped_is_tcgen05(cache->head_dim, plan.group_size,
+                                             num_heads / cache->num_kv_heads)
+                        ? PA_KERNEL_GROUPED_TCGEN05
+                        : PA_KERNEL_GROUPED;
     if (plan.num_partitions > 1) {
         e = pa::launch_partition_reduce(p, cache->dtype, cache->head_dim, st);
         if (e != cudaSuccess) return fail_cuda(e, "pa_decode reduce launch");
@@ -599,6 +603,12 @@ int pa_decode_grouped_num_partitions(int32_t num_seqs, int32_t num_heads,
     int rc = plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan,
                          group_size);
     return rc != PA_OK ? rc : plan.num_partitions;
+}
+
+int pa_set_grouped_consumer(int consumer) {
+    if (consumer != PA_GROUPED_MMA_SYNC && consumer != PA_GROUPED_TCGEN05)
+        return fail(PA_ERR_INVALID_ARG, "unknown grouped consumer %d", consumer);
+    return pa::set_grouped_consumer(consumer);
 }
 
 int pa_sync_check(void* stream) {

@@ -28,6 +28,7 @@
 
 #include <type_traits>
 
+#include "pa.h"
 #include "pa_device.cuh"
 #include "pa_internal.h"
 #include "pa_tma.cuh"
@@ -105,7 +106,8 @@ template <class G>
 __device__ __forceinline__ bool issue_subtile(const CUtensorMap* kmap, const CUtensorMap* vmap,
                                               const DecodeParams& p, const Ring& ring, int gi,
                                               int phys, int kh, int tok0,
-                                              uint32_t* hdr = nullptr, uint32_t hval = 0) {
+                                              uint32_t* hdr = nullptr, uint32_t hval = 0,
+                                              uint32_t* hdr2 = nullptr, uint32_t hval2 = 0) {
     const int st = gi % G::kStages;
     const uint32_t round = (uint32_t)(gi / G::kStages);
     if (!mbar_wait_bounded(ring.empty + 8 * st, (round & 1u) ^ 1u)) {
@@ -114,6 +116,7 @@ __device__ __forceinline__ bool issue_subtile(const CUtensorMap* kmap, const CUt
     }
     if (gi == p.test_skip_position) return true;  // test hook: leave this stage unloaded
     if (hdr != nullptr) hdr[st] = hval;
+    if (hdr2 != nullptr) hdr2[st] = hval2;
     if ((unsigned)phys < (unsigned)p.num_blocks) {
         ring.valid[st] = 1;
         const uint32_t full = ring.full + 8 * st;
@@ -1330,11 +1333,16 @@ __device__ __forceinline__ void gload_phys(const DecodeParams& p, const GItem& i
 // issue in sub-rounds of kStages positions, so a sub-round touches each stage
 // at most once and a stage's rounds are issued in order.
 template <class G>
+// hdr2 (optional): per stage, the unit's largest valid token count over the
+// members that use it (1..16).
 __device__ __forceinline__ void issue_units(const CUtensorMap* kmap, const CUtensorMap* vmap,
                                             const DecodeParams& p, const Ring& ring, uint32_t* hdr,
                                             const GItem& it, int base, int n_sub, uint32_t act,
                                             const int (&phys)[kMaxGroupSeqs], int lane, int& g,
-                                            int& issued, bool& dead) {
+                                            int& issued, bool& dead, uint32_t* hdr2 = nullptr) {
+    int t1m[kMaxGroupSeqs];
+#pragma unroll
+    for (int m = 0; m < kMaxGroupSeqs; ++m) t1m[m] = __shfl_sync(0xffffffffu, it.t1_lane, m);
     uint32_t lead = 0;
     int nu = 0;
 #pragma unroll
@@ -1372,7 +1380,12 @@ __device__ __forceinline__ void issue_units(const CUtensorMap* kmap, const CUten
                         if (((act >> m2) & 1u) && phys[m2] == phys[m]) mask |= 1u << m2;
                     const uint32_t h = mask | ((uint32_t)i << kUnitSubShift) |
                                        (last_batch && pos == total - 1 ? kUnitLast : 0u);
-                    ok = issue_subtile<G>(kmap, vmap, p, ring, g + pos, phys[m], it.kh, tok0, hdr, h);
+                    int nv = 0;
+#pragma unroll
+                    for (int m2 = 0; m2 < kMaxGroupSeqs; ++m2)
+                        if ((mask >> m2) & 1u) nv = max(nv, min(16, t1m[m2] - tok0));
+                    ok = issue_subtile<G>(kmap, vmap, p, ring, g + pos, phys[m], it.kh, tok0, hdr, h,
+                                          hdr2, (uint32_t)nv);
                     if (ok) issued = g + pos + 1;
                 }
                 ++pos;
@@ -1799,6 +1812,503 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
     }
 }
 
+// ---------------------------------------------------------------------------
+// 5th-generation tensor-core (tcgen05) helpers.
+// ---------------------------------------------------------------------------
+// Shared-memory matrix descriptor: start address, leading / stride byte
+// offsets (16-byte units), descriptor version 1, layout 2 = 128-byte swizzle.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor for kind::f16: fp32 accumulator, bf16 A and B, A
+// K-major, B K-major or MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t umma_idesc(int m, int n, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+// D (TMEM) (+)= A (shared) . B (shared)^T, issued by one thread.
+__device__ __forceinline__ void umma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                        bool acc) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)acc) : "memory");
+}
+// D (TMEM) (+)= A (TMEM) . B (shared)^T.
+__device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                        bool acc) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                 :: "r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"((uint32_t)acc) : "memory");
+}
+// The mbarrier at `bar` gets one arrival once every tcgen05 operation this
+// thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// generic-proxy shared-memory writes made visible to the tensor core's reads
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(slot), "r"(ncols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                 :: "r"(taddr), "r"(ncols) : "memory");
+}
+// Loads / stores of this warp's 32 TMEM lanes (32x32b): thread t reads or
+// writes lane (lane of taddr) + t, consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]) : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+                 :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]) : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Grouped and multi-token decode on the 5th-generation tensor cores
+// (head_dim 128, bf16, 16..64 query columns; opt-in, see grouped_consumer).
+// Same work items, producer and ring as decode_tma_grouped_kernel (one unit
+// per distinct block of a 16-token sub-tile, mask + sub-tile index in a
+// per-stage header, plus the unit's largest valid token count); the consumer
+// is split by role:
+//   warp 3, lane 0, issues per unit S = Q . K^T (M = 128 query rows, N = 16
+//     tokens, K = 128; Q and the K tile from shared memory, S in TMEM) and
+//     O += P . V (A = P in TMEM, B = the V tile read MN-major from shared
+//     memory, O in TMEM) with tcgen05.mma, completions signalled by
+//     tcgen05.commit;
+//   warps 0 and 1 (TMEM lane quarters 0 and 1): softmax, thread = query row:
+//     the row's 16 scores come from TMEM, the running max and sum stay in
+//     registers, P goes back to TMEM; they also stage each item's q in shared
+//     memory and write the item's output from O;
+//   warp 2: the producer (TMA).
+// S and P are double-buffered, so the next unit's QK overlaps this unit's
+// softmax. Rescaling is lazy: a row's O is rescaled (in TMEM) only when its max
+// grows by more than kRescaleLog2 (log2 units); until then the weights use the
+// older max, which numerator and denominator share, so the result is the same
+// exact softmax (weights stay below 2^kRescaleLog2). The running max moves per
+// logical 16-token sub-tile of a member, so a member's result does not depend on
+// which blocks it shares. V rows past every member's context are zeroed in
+// shared memory before the PV product reads them.
+// Measured against the mma.sync consumer (4-beam GQA CoW, 4-token verification
+// over 32K contexts): slower, 172 vs 106 and 444 vs 291 us. Per CTA one softmax
+// warp walks the units one after the other, and with at most 2 CTAs per SM (TMEM,
+// shared memory) too few warps hide the TMEM / barrier round trips of a 16 x 32
+// contraction; batching 4 units per softmax pass made it slower still.
+// ---------------------------------------------------------------------------
+constexpr int kUmmaRing = 49152;
+constexpr int kUmmaQBuf = 16384;           // one item's q: 64 rows x 256 B, two 128-B-swizzled atoms
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColO = 0, kColS = 128, kColP = 160;  // S at 128 / 144, P at 160 / 168
+constexpr float kRescaleLog2 = 8.f;
+constexpr uint32_t kIdescQK = umma_idesc(128, 16, false);
+constexpr uint32_t kIdescPV = umma_idesc(128, 128, true);
+using UmmaGeom = Geom<__nv_bfloat16, 128, 1, kUmmaRing>;
+
+struct UmmaBars {
+    uint32_t full, empty, s, pv, pfull, q, ofree, done, fin;  // shared addresses
+    volatile int* dead;
+};
+
+// Bounded wait by a whole warp, warp-uniform outcome; gives up at once when
+// another role already gave up (so timeouts do not chain).
+__device__ __forceinline__ bool umma_wait(const UmmaBars& b, uint32_t bar, uint32_t parity) {
+    const bool ok = __all_sync(0xffffffffu, *b.dead == 0 && mbar_wait_bounded(bar, parity));
+    if (!ok && (threadIdx.x & 31) == 0) {
+        if (*b.dead == 0) atomicOr(&s_status_tma, kStatusTimeout);
+        *b.dead = 1;
+    }
+    return ok;
+}
+
+template <int D>
+__global__ void __launch_bounds__(128, 2)
+decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
+                           const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
+                           int num_items, int gs) {
+    static_assert(D == 128, "head_dim 128");
+    using G = UmmaGeom;
+    constexpr int S_ = G::kStages;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    asm volatile("griddepcontrol.launch_dependents;");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int P = p.num_partitions;
+    const int group = p.num_heads / p.num_kv_heads;
+    const int ncols = gs * group;
+    const int sw = (ncols + 31) >> 5;  // softmax warps
+    const int ipb = 32 / gs;
+    const uint32_t raw = smem_u32(smem_raw);
+    if (raw & 1023u) {
+        if (threadIdx.x == 0) atomicOr(&s_status_tma, kStatusSmemAlign);
+        return;
+    }
+    // [q buffers 2 x 16 KB][ring][hdr][hdr2][barriers][valid][tmem slot][dead]
+    const uint32_t qbuf = raw;
+    Ring ring;
+    ring.stages = raw + 2 * kUmmaQBuf;
+    uint32_t* hdr = reinterpret_cast<uint32_t*>(smem_raw + 2 * kUmmaQBuf + G::kRingBytes);
+    uint32_t* hdr2 = hdr + S_;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + 2 * kUmmaQBuf + G::kRingBytes +
+                                                 ((2 * S_ * 4 + 7) & ~7));
+    UmmaBars B;
+    B.full = smem_u32(bars);
+    B.empty = B.full + 8 * S_;
+    B.s = B.empty + 8 * S_;       // [2]
+    B.pv = B.s + 16;              // [2]
+    B.pfull = B.pv + 16;          // [2]
+    B.q = B.pfull + 16;           // [2]
+    B.ofree = B.q + 16;
+    B.done = B.ofree + 8;
+    B.fin = B.done + 8;
+    ring.full = B.full;
+    ring.empty = B.empty;
+    ring.valid = reinterpret_cast<int*>(bars + 2 * S_ + 13);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(ring.valid + S_);
+    B.dead = reinterpret_cast<volatile int*>(tslot + 1);
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < S_; ++st) {
+            mbar_init(B.full + 8 * st, 1);
+            mbar_init(B.empty + 8 * st, 1);  // released by the MMA thread's commit
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(B.s + 8 * i, 1);
+            mbar_init(B.pv + 8 * i, 1);
+            mbar_init(B.pfull + 8 * i, sw);
+            mbar_init(B.q + 8 * i, sw);
+        }
+        mbar_init(B.ofree, sw);
+        mbar_init(B.done, sw);
+        mbar_init(B.fin, 1);
+        *B.dead = 0;
+        fence_barrier_init();
+    }
+    if (warp == 3) tmem_alloc(smem_u32(tslot), kTmemCols);
+    GWalk walk;
+    walk.k = 0;
+    walk.kbase = 0;
+    walk.ctx_lane = gwalk_load(p, num_items, 0, lane, gs, ipb, warp == 0);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tslot;
+
+    if (warp == 2) {  // producer
+        if (lane == 0) {
+            prefetch_tensormap(&kmap);
+            prefetch_tensormap(&vmap);
+        }
+        bool dead = false;
+        int g = 0, issued = 0;
+        GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
+        int cur_base = 0;
+        uint32_t act_cur;
+        int phys_cur[kMaxGroupSeqs];
+        gload_phys(p, cur, cur_base, gs, lane, act_cur, phys_cur);
+        while (cur.valid && !dead) {
+            const int n_sub = (cur.tmax - cur.t0 + 15) >> 4;
+            GItem nxt = cur;
+            int nxt_base = cur_base + 32;
+            if (nxt_base >= n_sub) {
+                nxt = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
+                nxt_base = 0;
+            }
+            uint32_t act_nxt;
+            int phys_nxt[kMaxGroupSeqs];
+            gload_phys(p, nxt, nxt_base, gs, lane, act_nxt, phys_nxt);
+            issue_units<G>(&kmap, &vmap, p, ring, hdr, cur, cur_base, n_sub, act_cur, phys_cur,
+                           lane, g, issued, dead, hdr2);
+            if (*B.dead) dead = true;
+            cur = nxt;
+            cur_base = nxt_base;
+            act_cur = act_nxt;
+#pragma unroll
+            for (int m = 0; m < kMaxGroupSeqs; ++m) phys_cur[m] = phys_nxt[m];
+        }
+        if (dead) *B.dead = 1;
+        drain_ring<G>(ring, issued, lane);
+        return;
+    }
+
+    if (warp == 3) {  // MMA issuer: lane 0 issues, the warp walks the items with it
+        int g = 0, n = 0;
+        bool have_prev = false, prev_valid = false, prev_first = false, o_started = false;
+        int prev_st = 0, prev_g = 0, prev_item = 0;
+        // PV of a unit: after its P is in TMEM (and, for an item's first unit,
+        // after the previous item's output left O); then release its stage.
+        auto issue_pv = [&]() -> bool {
+            if (!umma_wait(B, B.pfull + 8 * (prev_g & 1), (prev_g >> 1) & 1)) return false;
+            if (prev_first) {
+                o_started = false;
+                if (prev_item >= 1 && !umma_wait(B, B.ofree, (prev_item - 1) & 1)) return false;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+                if (prev_valid) {
+                    const uint32_t vb = ring.stages + prev_st * G::kStageBytes + 2 * kBoxBytes;
+                    // V read MN-major: head_dim atoms of 64 (one box each) kBoxBytes
+                    // apart, 8-token groups 1024 B apart
+                    umma_ts(tm + kColO, tm + kColP + 8 * (prev_g & 1), umma_desc(vb, kBoxBytes, 1024),
+                            kIdescPV, o_started);
+                }
+                umma_commit(B.pv + 8 * (prev_g & 1));
+                umma_commit(B.empty + 8 * prev_st);
+            }
+            if (prev_valid) o_started = true;
+            __syncwarp();
+            return true;
+        };
+        bool ok = true;
+        GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
+        while (cur.valid && ok) {
+            if (!umma_wait(B, B.q + 8 * (n & 1), (n >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            bool first = true;
+            for (;;) {
+                const int st = g % S_;
+                if (!umma_wait(B, B.full + 8 * st, (uint32_t)(g / S_) & 1u)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t h = hdr[st];
+                const bool valid = ring.valid[st] != 0;
+                if (lane == 0) {
+                    const uint32_t kb = ring.stages + st * G::kStageBytes;
+                    const uint32_t qa = qbuf + (n & 1) * kUmmaQBuf;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        umma_ss(tm + kColS + 16 * (g & 1),
+                                umma_desc(qa + (k >> 2) * (kUmmaQBuf / 2) + (k & 3) * 32, 16, 1024),
+                                umma_desc(kb + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024),
+                                kIdescQK, k > 0);
+                    umma_commit(B.s + 8 * (g & 1));
+                }
+                __syncwarp();
+                if (have_prev && !issue_pv()) { ok = false; break; }
+                have_prev = true;
+                prev_st = st;
+                prev_g = g;
+                prev_valid = valid;
+                prev_first = first;
+                prev_item = n;
+                first = false;
+                ++g;
+                if (h & kUnitLast) break;
+            }
+            ++n;
+            if (ok) cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
+        }
+        if (ok && have_prev) ok = issue_pv();
+        // wait for the softmax warps (even after a timeout: they stop touching
+        // TMEM before they arrive), then for every issued MMA, then free TMEM
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(B.done, 0)) && lane == 0)
+            atomicOr(&s_status_tma, kStatusTimeout);
+        if (lane == 0) umma_commit(B.fin);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(B.fin, 0)) && lane == 0)
+            atomicOr(&s_status_tma, kStatusTimeout);
+        tc_fence_after();
+        tmem_dealloc(tm, kTmemCols);
+        return;
+    }
+
+    if (warp >= sw) {  // no query rows for this warp
+        return;
+    }
+
+    // softmax warps: thread = query column (member, head) = row of S, P and O
+    const int col = 32 * warp + lane;
+    const int mem = col / group, hd = col - mem * group;
+    const uint32_t mybit = (col < ncols && mem < gs) ? 1u << mem : 0u;
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const uint8_t* qsrc_base = static_cast<const uint8_t*>(p.q);
+    int g = 0, n = 0;
+    bool ok = true;
+    // Next item with tokens; with one partition, members of items without any
+    // tokens get a zero output here.
+    auto next_item = [&]() -> GItem {
+        for (;;) {
+            GItem it = gitem_next(walk, p, num_items, gs, ipb, lane, warp == 0, P == 1);
+            if (!it.valid || it.tmax > it.t0) return it;
+            if (col < ncols && mem < it.nmem) {
+                uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
+                    ((int64_t)(it.row0 + mem) * p.num_heads + (int64_t)it.kh * group + hd) * D);
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) o[c] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    };
+    // this row's q into buffer `buf`, 128-byte swizzled (two atoms of 64 rows)
+    auto stage_q = [&](const GItem& it, int buf) {
+        const int t1 = __shfl_sync(0xffffffffu, it.t1_lane, mem & (kMaxGroupSeqs - 1));
+        const bool has = col < ncols && mem < it.nmem && t1 > it.t0;
+        const uint4* src = reinterpret_cast<const uint4*>(qsrc_base +
+            ((int64_t)(it.row0 + mem) * p.num_heads + (int64_t)it.kh * group + hd) * D * 2);
+        uint8_t* dst = smem_raw + buf * kUmmaQBuf;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const uint4 v = has ? ld_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            const int atom = c >> 3, x = c & 7;
+            *reinterpret_cast<uint4*>(dst + atom * (kUmmaQBuf / 2) + col * 128 + ((x ^ (col & 7)) << 4)) = v;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(B.q + 8 * buf);
+    };
+    GItem cur = next_item();
+    if (cur.valid) stage_q(cur, 0);
+    while (cur.valid && ok) {
+        const int t1 = __shfl_sync(0xffffffffu, cur.t1_lane, mem & (kMaxGroupSeqs - 1));
+        const float sl = p.scale_log2;
+        float m_ref = -INFINITY, l = 0.f;
+        for (;;) {
+            if (!umma_wait(B, B.s + 8 * (g & 1), (g >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const int st = g % S_;
+            const uint32_t h = hdr[st];
+            const bool valid = ring.valid[st] != 0;
+            const int nvmax = (int)hdr2[st];
+            const int tok0 = cur.t0 + (int)((h >> kUnitSubShift) & kUnitSubMask) * 16;
+            uint32_t sr[16];
+            tmem_ld16(tm + lane_off + kColS + 16 * (g & 1), sr);
+            const int nv = (valid && (h & mybit)) ? min(16, t1 - tok0) : 0;
+            float sv[16];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                sv[j] = j < nv ? __uint_as_float(sr[j]) * sl : -INFINITY;
+                mx = fmaxf(mx, sv[j]);
+            }
+            // O must not be rescaled, nor P(g & 1) rewritten, before the PV that
+            // reads them is done (the PV of unit g - 1, resp. g - 2)
+            const bool resc = m_ref != -INFINITY && mx > m_ref + kRescaleLog2;
+            const bool any_resc = __any_sync(0xffffffffu, resc);
+            if (any_resc) {
+                if (!umma_wait(B, B.pv + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1)) { ok = false; break; }
+            } else if (g >= 2) {
+                if (!umma_wait(B, B.pv + 8 * (g & 1), ((g - 2) >> 1) & 1)) { ok = false; break; }
+            }
+            tc_fence_after();
+            if (any_resc) {
+                const float alpha = resc ? exp2f(m_ref - mx) : 1.f;
+#pragma unroll
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tm + lane_off + kColO + c0, o);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                    tmem_st32(tm + lane_off + kColO + c0, o);
+                }
+                if (resc) {
+                    l *= alpha;
+                    m_ref = mx;
+                }
+            } else if (m_ref == -INFINITY && mx != -INFINITY) {
+                m_ref = mx;
+            }
+            // a row that has seen no valid token keeps max -inf: weights 0
+            const float base = m_ref == -INFINITY ? 0.f : m_ref;
+            uint32_t pk[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                pk[j] = pack_bf16x2(exp2f(sv[2 * j] - base), exp2f(sv[2 * j + 1] - base));
+                l += bf16_lo(pk[j]) + bf16_hi(pk[j]);
+            }
+            tmem_st8(tm + lane_off + kColP + 8 * (g & 1), pk);
+            if (warp == 0 && valid && nvmax < 16) {
+                // V rows nvmax..15 (both boxes) belong to no member's context
+                const uint32_t vb = ring.stages + st * G::kStageBytes + 2 * kBoxBytes;
+                for (int i = lane; i < (16 - nvmax) * 16; i += 32) {
+                    const int row = nvmax + (i >> 4), c16 = i & 15;
+                    const uint32_t a = vb + (c16 >> 3) * kBoxBytes + row * 128 + (c16 & 7) * 16;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" :: "r"(a), "r"(0u) : "memory");
+                }
+                fence_async_smem();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(B.pfull + 8 * (g & 1));
+            ++g;
+            if (h & kUnitLast) break;
+        }
+        if (!ok) break;
+        // next item's q first: the MMA thread needs it before the PV of this
+        // item's last unit, which the output below waits for
+        const GItem nxt = next_item();
+        if (nxt.valid) stage_q(nxt, (n + 1) & 1);
+        if (!umma_wait(B, B.pv + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const bool has = col < ncols && mem < cur.nmem && t1 > cur.t0;
+        const int64_t row = ((int64_t)(cur.row0 + mem) * p.num_heads + (int64_t)cur.kh * group + hd);
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tm + lane_off + kColO + c0, o);
+            if (col < ncols && mem < cur.nmem) {
+                if (P == 1) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        w[j] = l > 0.f ? pack_bf16x2(__uint_as_float(o[2 * j]) * inv,
+                                                     __uint_as_float(o[2 * j + 1]) * inv)
+                                       : 0u;
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * D + c0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                } else if (has) {
+                    float* dst = p.ws_o + (row * P + cur.part) * D + c0;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) dst[j] = l > 0.f ? __uint_as_float(o[j]) * inv : 0.f;
+                }
+            }
+        }
+        if (P > 1 && has) {
+            float* ml = p.ws_ml + (row * P + cur.part) * 2;
+            ml[0] = l > 0.f ? m_ref : -INFINITY;
+            ml[1] = l;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(B.ofree);
+        cur = nxt;
+        ++n;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(B.done);
+}
+
+template <int D>
+constexpr size_t umma_smem_bytes() {
+    using G = UmmaGeom;
+    return 2 * kUmmaQBuf + G::kRingBytes + ((2 * G::kStages * 4 + 7) & ~7) +
+           (2 * G::kStages + 13) * 8 + G::kStages * 4 + 16 + 64;
+}
+
 template <typename T, int D>
 cudaError_t launch_simt_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
                           cudaStream_t stream) {
@@ -1844,6 +2354,27 @@ cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUt
     const long slots = (long)per_sm[dev] * sms;
     const unsigned grid = (unsigned)(items < slots ? items : slots);
     kernel<<<grid, G::kThreads, smem, stream>>>(km, vm, p, (int)items);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_umma_grouped(const DecodeParams& p, const CUtensorMap& km,
+                                const CUtensorMap& vm, int gs, cudaStream_t stream) {
+    constexpr size_t smem = umma_smem_bytes<128>();
+    auto kernel = decode_umma_grouped_kernel<128>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const long groups = p.query_start != nullptr ? (long)p.num_seqs * p.q_chunks
+                                                 : (long)(p.num_seqs + gs - 1) / gs;
+    const long items = (long)p.num_partitions * p.num_kv_heads * groups;
+    const long slots = 2L * sms;  // two CTAs per SM: 256 TMEM columns and ~81 KB each
+    const unsigned grid = (unsigned)(items < slots ? items : slots);
+    kernel<<<grid, 128, smem, stream>>>(km, vm, p, (int)items, gs);
     return cudaGetLastError();
 }
 
@@ -1909,6 +2440,16 @@ bool mma_supported(int dtype, int head_dim, int group) {
            group <= kGroupMax;
 }
 
+// Grouped consumer selected by pa_set_grouped_consumer (process-wide). The
+// tcgen05 consumer takes head_dim 128 with 16..64 query columns (its 128-row
+// MMAs would mostly idle below that); other shapes stay on mma.sync.
+static int g_grouped_consumer = PA_GROUPED_MMA_SYNC;
+
+static bool use_umma(int head_dim, int gs, int group) {
+    return g_grouped_consumer == PA_GROUPED_TCGEN05 && head_dim == 128 && gs * group >= 16 &&
+           gs * group <= 64;
+}
+
 // Query columns (member, head) -> n-tiles of 8 -> consumer warps: one n-tile
 // per warp when a single tile holds them all, else two per warp.
 static void grouped_shape(int gs, int group, int* cw, int* nt) {
@@ -1923,6 +2464,7 @@ bool grouped_supported(int dtype, int head_dim, int group, int gs) {
 }
 
 int grouped_ctas_per_sm(int head_dim, int gs, int group) {
+    if (use_umma(head_dim, gs, group)) return 2;
     int cw = 1, nt = 1;
     grouped_shape(gs, group, &cw, &nt);
     return grouped_min_blocks(head_dim, cw, nt);
@@ -1961,10 +2503,20 @@ static cudaError_t launch_grouped_d(const DecodeParams& p, int cw, int nt, int g
 cudaError_t launch_decode_grouped(const DecodeParams& p, int head_dim, int gs,
                                   const CUtensorMap& kmap, const CUtensorMap& vmap,
                                   cudaStream_t stream) {
+    if (use_umma(head_dim, gs, p.num_heads / p.num_kv_heads))
+        return launch_umma_grouped(p, kmap, vmap, gs, stream);
     int cw = 1, nt = 1;
     grouped_shape(gs, p.num_heads / p.num_kv_heads, &cw, &nt);
     return head_dim == 64 ? launch_grouped_d<64>(p, cw, nt, gs, kmap, vmap, stream)
                           : launch_grouped_d<128>(p, cw, nt, gs, kmap, vmap, stream);
+}
+
+bool grouped_is_tcgen05(int head_dim, int gs, int group) { return use_umma(head_dim, gs, group); }
+
+int set_grouped_consumer(int consumer) {
+    const int prev = g_grouped_consumer;
+    g_grouped_consumer = consumer;
+    return prev;
 }
 
 cudaError_t read_status_tma(unsigned* bits, bool clear) {

@@ -97,6 +97,11 @@ cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bo
 // item are up to gs query tokens of one sequence instead. bf16, head_dim
 // 64 / 128, 1 <= gs <= 8, gs * (H / Hkv) <= 64 query columns.
 bool grouped_supported(int dtype, int head_dim, int group, int gs);
+// Select the grouped consumer (PA_GROUPED_MMA_SYNC / PA_GROUPED_TCGEN05);
+// returns the previous one.
+int set_grouped_consumer(int consumer);
+// Whether the grouped kernel for (head_dim, gs, H / Hkv) is the tcgen05 consumer.
+bool grouped_is_tcgen05(int head_dim, int gs, int group);
 // CTA slots per SM of the grouped kernel chosen for (head_dim, gs, H / Hkv).
 int grouped_ctas_per_sm(int head_dim, int gs, int group);
 cudaError_t launch_decode_grouped(const DecodeParams& p, int head_dim, int gs,

@@ -56,6 +56,14 @@ def last_kernel():
     return pa.load_library().pa_test_last_decode_kernel()
 
 
+def kernel_set(kernel):
+    """The decode kernels that count as `kernel`: the grouped kernel runs on either
+    grouped consumer (pa_set_grouped_consumer)."""
+    if kernel == pa.PA_KERNEL_GROUPED:
+        return (pa.PA_KERNEL_GROUPED, pa.PA_KERNEL_GROUPED_TCGEN05)
+    return (kernel,)
+
+
 def oracle_step(wl, host):
     """The same step on the oracle. ``host``: numpy copies of the inputs taken
     before the GPU step (caches are modified in place)."""

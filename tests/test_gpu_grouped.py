@@ -26,7 +26,7 @@ def _check(wl, gs, ps, kernel=pa.PA_KERNEL_GROUPED):
     host = G.host_copy(vals)
     out = G.gpu_step(wl, vals, partition_size=ps, group_size=gs)
     pa.pa_sync_check()
-    assert G.last_kernel() == kernel
+    assert G.last_kernel() in G.kernel_set(kernel)
     ref = G.oracle_step(wl, host)
     assert G.bits_equal(vals["k_cache"], host["k_cache"])
     assert G.bits_equal(vals["v_cache"], host["v_cache"])
@@ -41,7 +41,7 @@ def test_cow_beam4_full_size_sampled():
     vals = W.make_values(wl, DEV, poison=True)
     out = G.gpu_step(wl, vals, partition_size=0, group_size=4)
     pa.pa_sync_check()
-    assert G.last_kernel() == pa.PA_KERNEL_GROUPED
+    assert G.last_kernel() in G.kernel_set(pa.PA_KERNEL_GROUPED)
     assert torch.isfinite(out.float()).all()
     seqs = sorted(set(G.sample_seqs(wl, 6)) | {0, 1, 2, 3, 124, 125, 126, 127})
     ref = G.oracle_sampled(wl, vals, seqs)
@@ -180,5 +180,5 @@ def test_bad_block_id_is_reported():
     with pytest.raises(pa.PAError) as e:
         pa.pa_sync_check()
     assert e.value.code == pa.PA_ERR_BAD_INDEX
-    assert G.last_kernel() == pa.PA_KERNEL_GROUPED
+    assert G.last_kernel() in G.kernel_set(pa.PA_KERNEL_GROUPED)
     pa.pa_sync_check()

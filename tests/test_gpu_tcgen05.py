@@ -1,0 +1,42 @@
+"""The grouped / multi-token decode on the tcgen05 consumer (pa_set_grouped_consumer):
+one thread issues 5th-generation tensor-core MMAs from shared memory with S, P
+and O in tensor memory. The same oracle parity, bitwise invariants and
+bounded-wait behaviour as the default consumer, re-run with this one selected
+(the test functions are those of the default consumer's modules)."""
+import pytest
+import torch
+
+import paged_kv_cache_335_b200 as pa
+from paged_kv_cache_335_b200 import workloads as W
+from tests import gpu_helpers as G
+from tests.test_gpu_grouped import (test_cow_small_full_pool,  # noqa: F401
+                                    test_deterministic_repeat,
+                                    test_long_shared_context_many_partitions,
+                                    test_members_with_empty_contexts,
+                                    test_placement_invariance_bitwise,
+                                    test_shared_equals_private_bitwise)
+from tests.test_gpu_multi import (test_parity_shape_sweep,  # noqa: F401
+                                  test_token_result_independent_of_the_other_tokens,
+                                  test_verification_full_size_sampled)
+from tests.test_gpu_timeout import test_skipped_load_times_out_then_recovers  # noqa: F401
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(autouse=True)
+def tcgen05_consumer():
+    prev = pa.pa_set_grouped_consumer(pa.PA_GROUPED_TCGEN05)
+    yield
+    pa.pa_set_grouped_consumer(prev)
+
+
+def test_selector_takes_the_tcgen05_path():
+    wl = W.cow_beam4(num_prompts=2, prompt_len=100, max_suffix=20, num_heads=16, num_kv_heads=2,
+                     head_dim=128)
+    vals = W.make_values(wl, DEV)
+    G.gpu_step(wl, vals, partition_size=0, group_size=4)
+    pa.pa_sync_check()
+    assert G.last_kernel() == pa.PA_KERNEL_GROUPED_TCGEN05
+    with pytest.raises(pa.PAError):
+        pa.pa_set_grouped_consumer(7)

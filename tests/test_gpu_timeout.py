@@ -57,7 +57,7 @@ def test_skipped_load_times_out_then_recovers(name, kw, gs):
     _decode(wl, vals, d, out2, gs)
     pa.pa_sync_check()
     if gs > 1:
-        assert G.last_kernel() == pa.PA_KERNEL_GROUPED
+        assert G.last_kernel() in G.kernel_set(pa.PA_KERNEL_GROUPED)
     seqs = list(range(wl.num_seqs))
     ref = G.oracle_sampled(wl, vals, seqs)
     G.check_tolerance(G.to_f64(out2), ref, wl.dtype, f"{name} after a timed-out call")
