@@ -140,6 +140,20 @@ def test_multi_query_policy_and_arguments(lib):
     assert rc == pa.PA_ERR_INVALID_ARG and b"query_start" in lib.pa_get_last_error()
 
 
+def test_grouped_consumer_selector(lib):
+    assert lib.pa_set_grouped_consumer(pa.PA_GROUPED_TCGEN05) == pa.PA_GROUPED_MMA_SYNC
+    assert lib.pa_set_grouped_consumer(pa.PA_GROUPED_MMA_SYNC) == pa.PA_GROUPED_TCGEN05
+    assert lib.pa_set_grouped_consumer(5) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_set_grouped_consumer(-1) == pa.PA_ERR_INVALID_ARG
+    # the tcgen05 consumer's plan: 2 CTAs per SM, so the 4-beam CoW items (256) fit one wave
+    d70 = _desc(num_kv_heads=8)
+    lib.pa_set_grouped_consumer(pa.PA_GROUPED_TCGEN05)
+    try:
+        assert lib.pa_decode_grouped_num_partitions(128, 64, 2303, ctypes.byref(d70), 4, 0) == 1
+    finally:
+        lib.pa_set_grouped_consumer(pa.PA_GROUPED_MMA_SYNC)
+
+
 def test_swap_rejects_bad_arguments(lib):
     p = ctypes.c_void_p(256)
     a, b = _desc(num_blocks=8), _desc(num_blocks=4)
