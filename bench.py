@@ -39,16 +39,21 @@ METRIC = "paged decode attention KV-read GB/s (% of B200 HBM peak); seq-steps/s"
 UNIT = "GB/s"
 DEFAULT_CONFIG = "llama13b_bs16"
 # (label, workload name, partition_size override or None = the workload's own)
-# (label, workload, partition size (None: the workload's), sequences decoded together)
-EXTRA_CONFIGS = [("llama7b", "llama7b", None, 1), ("llama13b_bs16", "llama13b_bs16", None, 1),
-                 ("llama13b_bs32", "llama13b_bs32", None, 1),
-                 ("llama70b_gqa", "llama70b_gqa", None, 1),
-                 ("llama70b_gqa_policy", "llama70b_gqa", 0, 1), ("cow_beam4", "cow_beam4", None, 1),
-                 ("cow_beam4_grouped", "cow_beam4", 0, 4),
-                 ("llama70b_verify4", "llama70b_verify4", 0, 1),
-                 ("llama13b_bs16_fp8", "llama13b_bs16_fp8", None, 1),
-                 ("llama13b_bs16_int8", "llama13b_bs16_int8", None, 1),
-                 ("llama70b_gqa_policy_fp8", "llama70b_gqa_fp8", 0, 1)]
+# (label, workload, partition size (None: the workload's), sequences decoded together,
+#  grouped consumer (None: the run's))
+EXTRA_CONFIGS = [("llama7b", "llama7b", None, 1, None),
+                 ("llama13b_bs16", "llama13b_bs16", None, 1, None),
+                 ("llama13b_bs32", "llama13b_bs32", None, 1, None),
+                 ("llama70b_gqa", "llama70b_gqa", None, 1, None),
+                 ("llama70b_gqa_policy", "llama70b_gqa", 0, 1, None),
+                 ("cow_beam4", "cow_beam4", None, 1, None),
+                 ("cow_beam4_grouped", "cow_beam4", 0, 4, None),
+                 ("cow_beam4_grouped_tcgen05", "cow_beam4", 0, 4, "tcgen05"),
+                 ("llama70b_verify4", "llama70b_verify4", 0, 1, None),
+                 ("llama70b_verify4_tcgen05", "llama70b_verify4", 0, 1, "tcgen05"),
+                 ("llama13b_bs16_fp8", "llama13b_bs16_fp8", None, 1, None),
+                 ("llama13b_bs16_int8", "llama13b_bs16_int8", None, 1, None),
+                 ("llama70b_gqa_policy_fp8", "llama70b_gqa_fp8", 0, 1, None)]
 # pa_test_last_decode_kernel() -> the decode kernel a call enqueued
 KERNEL_NAMES = {0: "decode_tma_simt_kernel (CUDA-core)",
                 1: "decode_tma_mma_kernel (persistent, tensor-core GQA)",
@@ -71,6 +76,8 @@ def parse_args():
                     help="override the workload's partition size (0 = library policy)")
     ap.add_argument("--group-size", type=int, default=1,
                     help="decode sequences [k g, (k+1) g) together (pa_decode_grouped) when > 1")
+    ap.add_argument("--grouped-consumer", choices=["mma_sync", "tcgen05"], default="mma_sync",
+                    help="consumer of the grouped / multi-token decode (pa_set_grouped_consumer)")
     ap.add_argument("--no-extra-configs", action="store_true",
                     help="skip the per-configuration table")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -630,6 +637,9 @@ def main():
     wl = W.make(args.config)
     if args.partition_size is not None:
         wl.partition_size = args.partition_size
+    import paged_kv_cache_335_b200 as pa
+    pa.pa_set_grouped_consumer(pa.PA_GROUPED_TCGEN05 if args.grouped_consumer == "tcgen05"
+                               else pa.PA_GROUPED_MMA_SYNC)
     step = Step(wl, device, seed_offset=rank, group_size=args.group_size)
 
     uuid = None
@@ -676,8 +686,10 @@ def main():
     kernel_name = KERNEL_NAMES.get(step.lib.pa_test_last_decode_kernel(), "unknown")
     if step.num_partitions > 1:
         kernel_name += " + partition_reduce_kernel"
-    traffic, sha = profile_traffic(
-        kernel_file, wl.name if args.group_size == 1 else f"{wl.name}_grouped{args.group_size}")
+    tag = wl.name if args.group_size == 1 else f"{wl.name}_grouped{args.group_size}"
+    if step.lib.pa_test_last_decode_kernel() == pa.PA_KERNEL_GROUPED_TCGEN05:
+        tag += "_tcgen05"
+    traffic, sha = profile_traffic(kernel_file, tag)
 
     # end to end through the public binding with host buffers
     e2e_ms, h2d, d2h = e2e_steps(step, args.steps, max(3, args.warmup))
@@ -691,8 +703,11 @@ def main():
     read_gbs = stream_read_gbs(device) if world == 1 else None
     per_config = {}
     if world == 1 and not args.no_extra_configs:
-        for label, name, ps, gs in EXTRA_CONFIGS:
+        for label, name, ps, gs, consumer in EXTRA_CONFIGS:
             w2 = W.make(name)
+            prev = None
+            if consumer == "tcgen05":
+                prev = pa.pa_set_grouped_consumer(pa.PA_GROUPED_TCGEN05)
             st = Step(w2, device, partition_size=ps, group_size=gs)
             r2 = time_steps(st, min(args.steps, 50), 3, flush_buf if needs_flush(w2) else None)
             sm = statistics.median(r2["step_ms"])
@@ -711,11 +726,14 @@ def main():
                 "partitions": st.num_partitions,
                 "partition_size": "library policy" if st.ps == 0 else st.ps,
                 "group_size": gs,
+                "grouped_consumer": consumer or args.grouped_consumer,
                 "decode_bytes": w2.decode_bytes(),
                 "unique_kv_bytes": w2.unique_kv_bytes() if name.startswith("cow") else None,
             }
             st.release()
             del st
+            if prev is not None:
+                pa.pa_set_grouped_consumer(prev)
             torch.cuda.empty_cache()
         per_config["swap_llama13b_blocks"] = swap_bandwidth(device)
 
@@ -732,7 +750,8 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic (seeded N(0,1) values, seeded shapes)",
-            "config": {**config_dict(wl, flush is not None), "group_size": args.group_size},
+            "config": {**config_dict(wl, flush is not None), "group_size": args.group_size,
+                       "grouped_consumer": args.grouped_consumer},
             "seq_steps_per_s": round(world * wl.num_seqs / (ms_per_step / 1e3), 1),
             "frac_of_hbm_peak": round(value / world / hbm_peak, 4),
             "reference_bandwidths_gbs": {
