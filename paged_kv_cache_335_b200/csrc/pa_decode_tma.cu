@@ -1143,26 +1143,23 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
 //
 // The CTA's query columns are (member, head) pairs, column = member * g + head
 // for g = H / Hkv; consumer warp w owns n-tiles NT w .. NT w + NT - 1 of 8
-// columns. Work item = (partition, kv head, group). For every logical 16-token
-// sub-tile of the item the producer reads each active member's block id and
-// issues one ring position ("unit") per distinct block, tagged in a per-stage
-// header with the mask of members that use it, the sub-tile index and an
-// end-of-item flag. Every consumer warp walks every position (the empty
-// barrier counts all consumer warps), computes only when one of its members
-// is in the mask, and keeps its members' running state in registers to the
-// end of the item, so each member's arithmetic is the same whichever blocks
-// it shares. Sharing of prefix blocks among parallel samples and beams:
+// columns. Work item = (partition, kv head, group). The item's logical tokens
+// are cut into units of SUB 16-token sub-tiles; for every unit the producer
+// reads each active member's block ids and issues one ring position per
+// distinct block sequence, tagged in a per-stage header with the mask of
+// members that use it, the unit index and an end-of-item flag. Every consumer
+// warp walks every position (the empty barrier counts all consumer warps),
+// computes only when one of its members is in the mask (one online-softmax
+// step per unit), and keeps its members' running state in registers to the
+// end of the item; unit boundaries are logical positions, so each member's
+// arithmetic is the same whichever blocks it shares. Sharing of prefix blocks among parallel samples and beams:
 // "AI 推理系列（十六）：PagedAttention——…", § Copy-on-Write、并行采样与
 // Prefix Caching 不是同一件事; "PagedAttention原理详解：GPU显存优化与模型路由
 // 技术", § PagedAttention的三大核心优势 (point 2 and the beam-search paragraph).
 // ---------------------------------------------------------------------------
 
-// V fragments by ldmatrix.trans (head_dim in natural order in the accumulator)
-// rather than 16-byte loads plus byte permutes; independent accumulation
-// chains per QK product (the 8-long MMA chain is the kernel's critical path).
-#ifndef PA_GROUPED_LDSM_V
-#define PA_GROUPED_LDSM_V 1
-#endif
+// V fragments by ldmatrix.trans (head_dim in natural order in the
+// accumulator); independent accumulation chains per QK product.
 #ifndef PA_GROUPED_QK_CHAINS
 #define PA_GROUPED_QK_CHAINS 2
 #endif
@@ -1170,16 +1167,16 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
 constexpr int kMaxGroupSeqs = 8;            // members per group (header mask bits 0..7)
 constexpr int kGroupedMaxCols = 64;         // query columns (member, head) per CTA
 constexpr uint32_t kUnitLast = 1u << 31;    // header: last unit of the item
-constexpr int kUnitSubShift = 8;            // header bits 8..30: sub-tile index in the item
+constexpr int kUnitSubShift = 8;            // header bits 8..30: unit index in the item
 constexpr uint32_t kUnitSubMask = 0x7fffffu;
 
 
 // Ring bytes and CTAs per SM of each grouped variant (consumer warps CW,
 // n-tiles per warp NT), the measured best of ring / occupancy sweeps on the
-// beam workloads: the kernel is latency-bound per warp, so each variant runs
-// as many warps per SM as its ~168 registers allow (12), and four consumer
-// warps take a deeper ring. Two n-tiles per warp need about 240 registers at
-// head_dim 128. Overridable for sweeps.
+// beam and verification workloads: the kernel is latency-bound per warp, so
+// each variant runs as many warps per SM as its ~168 registers allow, and
+// four consumer warps take a deeper ring. Two n-tiles per warp need about 240
+// registers at head_dim 128. Overridable for sweeps.
 #ifndef PA_GROUPED_ONE_TILE_WARPS
 #define PA_GROUPED_ONE_TILE_WARPS 4
 #endif
@@ -1207,16 +1204,60 @@ constexpr uint32_t kUnitSubMask = 0x7fffffu;
 #ifndef PA_G_BLK4
 #define PA_G_BLK4 2
 #endif
+// Sub-tiles per unit: a unit is SUB consecutive 16-token sub-tiles of one
+// distinct block sequence, consumed in one online-softmax step, so the
+// per-step work (barrier waits, the cross-lane max, rescaling) is paid once
+// per 16 SUB tokens. SUB and the ring bytes of each variant (a stage holds
+// 2 SUB sub-tiles of K and V) are the measured best; at least two stages.
+#ifndef PA_G_SUB1
+#define PA_G_SUB1 2
+#endif
+#ifndef PA_G_SUB2
+#define PA_G_SUB2 2
+#endif
+#ifndef PA_G_SUB3
+#define PA_G_SUB3 2
+#endif
+#ifndef PA_G_SUB4
+#define PA_G_SUB4 4
+#endif
+#ifndef PA_G_SUB_NT2
+#define PA_G_SUB_NT2 2
+#endif
+#ifndef PA_G_SRING4
+#define PA_G_SRING4 98304
+#endif
+__host__ __device__ constexpr int grouped_sub(int cw, int nt) {
+    return nt != 1 ? PA_G_SUB_NT2 : cw == 1 ? PA_G_SUB1 : cw == 2 ? PA_G_SUB2 : cw == 3 ? PA_G_SUB3 : PA_G_SUB4;
+}
 __host__ __device__ constexpr int grouped_ring_bytes(int cw, int nt) {
-    return nt != 1 ? 49152 : cw == 1 ? PA_G_RING1 : cw == 2 ? PA_G_RING2 : cw == 3 ? PA_G_RING3 : PA_G_RING4;
+    return nt != 1 ? 49152
+                   : cw == 1 ? PA_G_RING1
+                   : cw == 2 ? PA_G_RING2
+                   : cw == 3 ? PA_G_RING3
+                   : grouped_sub(cw, nt) > 2 ? PA_G_SRING4 : PA_G_RING4;
 }
 __host__ __device__ constexpr int grouped_min_blocks(int d, int cw, int nt) {
     return nt == 1 ? (cw == 1 ? PA_G_BLK1 : cw == 2 ? PA_G_BLK2 : cw == 3 ? PA_G_BLK3 : PA_G_BLK4)
                    : d == 64 ? (cw <= 1 ? 4 : cw == 2 ? 3 : 2) : (cw <= 1 ? 4 : cw <= 3 ? 2 : 1);
 }
 
+// Ring of the grouped kernel: stage = K of the unit's SUB sub-tiles, then
+// their V (kSubBytes each). Every consumer warp reads every stage.
+template <int D, int SUB, int RING>
+struct GroupedRing {
+    using T = __nv_bfloat16;
+    static constexpr int kSub = SUB;
+    static constexpr int kBoxes = D * 2 / 128;
+    static constexpr int kBoxElems = 64;
+    static constexpr int kSubBytes = kBoxes * kBoxBytes;
+    static constexpr int kStageBytes = 2 * SUB * kSubBytes;
+    static constexpr int kStages = RING / kStageBytes;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static_assert(kStages >= 2, "grouped ring: at least two stages");
+};
 template <int D, int CW, int NT>
-using GroupedGeom = Geom<__nv_bfloat16, D, 1, grouped_ring_bytes(CW, NT)>;
+using GroupedGeom = GroupedRing<D, grouped_sub(CW, NT), grouped_ring_bytes(CW, NT)>;
 
 // Walk over a grouped CTA's items, u = blockIdx.x + k * gridDim.x, item u =
 // (partition u % P, kv head, group u / (P Hkv)). Lane l holds the context
@@ -1397,6 +1438,150 @@ __device__ __forceinline__ void issue_units(const CUtensorMap* kmap, const CUten
     g += total;
 }
 
+// Units of SUB sub-tiles. Lane l of a batch holds unit ubase + l, logical
+// tokens tok0 .. tok0 + 16 SUB - 1 (tok0 = t0 + 16 SUB (ubase + l)), and for
+// every member whose tokens reach the unit (bit m of `act`) the block ids of
+// the sub-tiles it uses (-1 past its last token).
+template <int SUB>
+__device__ __forceinline__ void gload_units(const DecodeParams& p, const GItem& it, int ubase, int gs,
+                                            int lane, uint32_t& act, int (&phys)[kMaxGroupSeqs][SUB]) {
+    act = 0;
+    const int tok0 = it.t0 + (ubase + lane) * (16 * SUB);
+#pragma unroll
+    for (int m = 0; m < kMaxGroupSeqs; ++m) {
+        const int t1 = __shfl_sync(0xffffffffu, it.t1_lane, m);
+        const bool on = it.valid && m < gs && tok0 < t1;
+        if (on) act |= 1u << m;
+        const int32_t* row = p.block_tables + (int64_t)(it.tab0 + m * it.tab_step) * p.table_stride;
+#pragma unroll
+        for (int s = 0; s < SUB; ++s) {
+            const int tk = tok0 + 16 * s;
+            phys[m][s] = on && tk < t1 ? __ldg(row + (tk >> p.log2_block_size)) : -1;
+        }
+    }
+}
+
+// Issue of one unit by one producer lane: wait until its stage is free, write
+// the header, then load K and V of its first `nsub` sub-tiles (block ids ph)
+// of kv head kh; the full barrier expects exactly those bytes. A block id
+// outside the pool marks the stage empty-handed (nothing loaded) and records
+// PA_ERR_BAD_INDEX. Returns false if the wait timed out.
+template <class G>
+__device__ __forceinline__ bool issue_unit(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                           const DecodeParams& p, const Ring& ring, int gi,
+                                           const int (&ph)[G::kSub], int nsub, int kh, int tok0,
+                                           uint32_t* hdr, uint32_t hval) {
+    const int st = gi % G::kStages;
+    const uint32_t round = (uint32_t)(gi / G::kStages);
+    if (!mbar_wait_bounded(ring.empty + 8 * st, (round & 1u) ^ 1u)) {
+        atomicOr(&s_status_tma, kStatusTimeout);
+        return false;
+    }
+    if (gi == p.test_skip_position) return true;  // test hook: leave this stage unloaded
+    hdr[st] = hval;
+    bool ok = true;
+#pragma unroll
+    for (int s = 0; s < G::kSub; ++s)
+        if (s < nsub && (unsigned)ph[s] >= (unsigned)p.num_blocks) ok = false;
+    if (ok) {
+        ring.valid[st] = 1;
+        const uint32_t full = ring.full + 8 * st;
+        mbar_arrive_expect_tx(full, (uint32_t)(nsub * 2 * G::kSubBytes));
+        const uint32_t sb = ring.stages + st * G::kStageBytes;
+#pragma unroll
+        for (int s = 0; s < G::kSub; ++s) {
+            if (s < nsub) {
+                const int32_t row = (ph[s] * p.num_kv_heads + kh) * p.block_size +
+                                    ((tok0 + 16 * s) & (p.block_size - 1));
+#pragma unroll
+                for (int b = 0; b < G::kBoxes; ++b)
+                    tma_load_2d(sb + s * G::kSubBytes + b * kBoxBytes, kmap, b * G::kBoxElems, row, full);
+#pragma unroll
+                for (int b = 0; b < G::kBoxes; ++b)
+                    tma_load_2d(sb + (G::kSub + s) * G::kSubBytes + b * kBoxBytes, vmap, b * G::kBoxElems,
+                                row, full);
+            }
+        }
+    } else {
+        atomicOr(&s_status_tma, kStatusBadIndex);
+        ring.valid[st] = 0;
+        mbar_arrive(ring.full + 8 * st);
+    }
+    return true;
+}
+
+// Issue the units of a batch of up to 32 (lane l: unit ubase + l). Members
+// whose block ids and sub-tile counts agree share one ring position, led by
+// the first of them; positions follow the same prefix-sum and sub-round order
+// as issue_units.
+template <class G>
+__device__ __forceinline__ void issue_units_sub(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                                const DecodeParams& p, const Ring& ring, uint32_t* hdr,
+                                                const GItem& it, int ubase, int n_units, uint32_t act,
+                                                const int (&phys)[kMaxGroupSeqs][G::kSub], int lane,
+                                                int& g, int& issued, bool& dead) {
+    constexpr int SUB = G::kSub;
+    const int i = ubase + lane;
+    const int tok0 = it.t0 + i * (16 * SUB);
+    int nsub[kMaxGroupSeqs];
+#pragma unroll
+    for (int m = 0; m < kMaxGroupSeqs; ++m) {
+        const int t1 = __shfl_sync(0xffffffffu, it.t1_lane, m);
+        nsub[m] = ((act >> m) & 1u) ? min(SUB, (t1 - tok0 + 15) >> 4) : 0;
+    }
+    auto same = [&](int a, int b) {
+        bool eq = nsub[a] == nsub[b];
+#pragma unroll
+        for (int s = 0; s < SUB; ++s) eq = eq && phys[a][s] == phys[b][s];
+        return eq;
+    };
+    uint32_t lead = 0;
+    int nu = 0;
+#pragma unroll
+    for (int m = 0; m < kMaxGroupSeqs; ++m) {
+        bool first = ((act >> m) & 1u) != 0;
+#pragma unroll
+        for (int m2 = 0; m2 < m; ++m2)
+            if (((act >> m2) & 1u) && same(m2, m)) first = false;
+        if (first) {
+            lead |= 1u << m;
+            ++nu;
+        }
+    }
+    int incl = nu;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    const int first_pos = incl - nu;
+    const bool last_batch = ubase + 32 >= n_units;
+    for (int k0 = 0; k0 < total && !dead; k0 += G::kStages) {
+        bool ok = true;
+        int pos = first_pos;
+#pragma unroll
+        for (int m = 0; m < kMaxGroupSeqs; ++m) {
+            if ((lead >> m) & 1u) {
+                if (ok && pos >= k0 && pos < k0 + G::kStages) {
+                    uint32_t mask = 0;
+#pragma unroll
+                    for (int m2 = m; m2 < kMaxGroupSeqs; ++m2)
+                        if (((act >> m2) & 1u) && same(m, m2)) mask |= 1u << m2;
+                    const uint32_t h = mask | ((uint32_t)i << kUnitSubShift) |
+                                       (last_batch && pos == total - 1 ? kUnitLast : 0u);
+                    ok = issue_unit<G>(kmap, vmap, p, ring, g + pos, phys[m], nsub[m], it.kh, tok0, hdr, h);
+                    if (ok) issued = g + pos + 1;
+                }
+                ++pos;
+            }
+        }
+        dead = __any_sync(0xffffffffu, !ok);
+    }
+    issued = __reduce_max_sync(0xffffffffu, issued);
+    g += total;
+}
+
 // S^T for NT n-tiles from one set of K fragments (see mma_qk).
 template <int D, int NT>
 __device__ __forceinline__ void mma_qk_n(uint32_t kb, const uint4 (&q)[NT][D / 32], int r, int c,
@@ -1442,39 +1627,36 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&a)[4]) {
                  : "r"(addr));
 }
 
-template <int D>
-__device__ __forceinline__ void ldsm_load_v(uint32_t vb, int lane, uint32_t (&va)[D / 16][4]) {
-    const int i = lane >> 3, row = 8 * (i >> 1) + (lane & 7);
-#pragma unroll
-    for (int t = 0; t < D / 16; ++t) {
-        const int d0 = 16 * t + 8 * (i & 1);
-        ldsm_x4_trans(vb + (d0 >> 6) * kBoxBytes + swz(row, (d0 & 63) >> 3), va[t]);
-    }
-}
-
-// Online-softmax update for NT n-tiles whose columns may each see a different
-// number of valid tokens: nva / nvb = valid tokens of this thread's columns 2c
-// and 2c + 1 of n-tile j (0 for a column whose member does not use the unit).
-// A column that has seen no valid token keeps max -inf and weight 0. Leaves
-// the P^T B-fragments in pb0 / pb1 and returns the largest valid count of the
-// warp's columns (V rows from there on must be zeroed).
-template <int D, int NT>
-__device__ __forceinline__ int softmax_update_n(const float (&sc)[NT][4], const int (&nva)[NT],
+// Online-softmax update over a unit of SUB sub-tiles for NT n-tiles whose
+// columns may each see a different number of valid tokens: nva / nvb = valid
+// tokens (from the unit's first) of this thread's columns 2c and 2c + 1 of
+// n-tile j, 0 for a column whose member does not use the unit. sc[s][j]: the
+// S^T fragment of sub-tile s (tokens 16 s + r, 16 s + r + 8). A column that
+// has seen no valid token keeps max -inf and weight 0. Leaves the P^T
+// B-fragments of sub-tile s in pb0[s] / pb1[s] and returns the largest valid
+// count of the warp's columns (V rows from there on must be zeroed).
+template <int D, int NT, int SUB>
+__device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], const int (&nva)[NT],
                                                 const int (&nvb)[NT], float scale_log2, int r,
                                                 float (&acc)[NT][D / 16][4], float (&ma)[NT],
                                                 float (&mb)[NT], float (&la)[NT], float (&lb)[NT],
-                                                uint32_t (&pb0)[NT], uint32_t (&pb1)[NT]) {
+                                                uint32_t (&pb0)[SUB][NT], uint32_t (&pb1)[SUB][NT]) {
     constexpr int MT = D / 16;
-    float s[NT][4], mxa[NT], mxb[NT];
+    float sv[SUB][NT][4], mxa[NT], mxb[NT];
     int nvmax = 0;
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
-        s[j][0] = r < nva[j] ? sc[j][0] * scale_log2 : -INFINITY;      // token r,   column 2c
-        s[j][1] = r < nvb[j] ? sc[j][1] * scale_log2 : -INFINITY;      // token r,   column 2c+1
-        s[j][2] = r + 8 < nva[j] ? sc[j][2] * scale_log2 : -INFINITY;  // token r+8, column 2c
-        s[j][3] = r + 8 < nvb[j] ? sc[j][3] * scale_log2 : -INFINITY;  // token r+8, column 2c+1
-        mxa[j] = fmaxf(s[j][0], s[j][2]);
-        mxb[j] = fmaxf(s[j][1], s[j][3]);
+        mxa[j] = mxb[j] = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < SUB; ++s) {
+            const int t0 = 16 * s + r, t1 = t0 + 8;
+            sv[s][j][0] = t0 < nva[j] ? sc[s][j][0] * scale_log2 : -INFINITY;  // token t0, column 2c
+            sv[s][j][1] = t0 < nvb[j] ? sc[s][j][1] * scale_log2 : -INFINITY;  // token t0, column 2c+1
+            sv[s][j][2] = t1 < nva[j] ? sc[s][j][2] * scale_log2 : -INFINITY;  // token t1, column 2c
+            sv[s][j][3] = t1 < nvb[j] ? sc[s][j][3] * scale_log2 : -INFINITY;  // token t1, column 2c+1
+            mxa[j] = fmaxf(mxa[j], fmaxf(sv[s][j][0], sv[s][j][2]));
+            mxb[j] = fmaxf(mxb[j], fmaxf(sv[s][j][1], sv[s][j][3]));
+        }
         nvmax = max(nvmax, max(nva[j], nvb[j]));
     }
 #pragma unroll
@@ -1499,10 +1681,18 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[NT][4], const 
         const float bb = mxb[j] == -INFINITY ? 0.f : mxb[j];
         const float ala = moved ? exp2f(ma[j] - ba) : 1.f;
         const float alb = moved ? exp2f(mb[j] - bb) : 1.f;
-        const uint32_t x0 = pack_bf16x2(exp2f(s[j][0] - ba), exp2f(s[j][1] - bb));
-        const uint32_t x1 = pack_bf16x2(exp2f(s[j][2] - ba), exp2f(s[j][3] - bb));
-        la[j] = fmaf(la[j], ala, bf16_lo(x0) + bf16_lo(x1));
-        lb[j] = fmaf(lb[j], alb, bf16_hi(x0) + bf16_hi(x1));
+        float suma = 0.f, sumb = 0.f;
+#pragma unroll
+        for (int s = 0; s < SUB; ++s) {
+            const uint32_t x0 = pack_bf16x2(exp2f(sv[s][j][0] - ba), exp2f(sv[s][j][1] - bb));
+            const uint32_t x1 = pack_bf16x2(exp2f(sv[s][j][2] - ba), exp2f(sv[s][j][3] - bb));
+            suma += bf16_lo(x0) + bf16_lo(x1);
+            sumb += bf16_hi(x0) + bf16_hi(x1);
+            pb0[s][j] = movmatrix_trans(x0);  // P^T rows (tokens) 16s + 2c, 2c+1; column r
+            pb1[s][j] = movmatrix_trans(x1);  // tokens 16s + 2c+8, 2c+9
+        }
+        la[j] = fmaf(la[j], ala, suma);
+        lb[j] = fmaf(lb[j], alb, sumb);
         ma[j] = mxa[j];
         mb[j] = mxb[j];
         if (moved) {
@@ -1514,62 +1704,58 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[NT][4], const 
                 acc[j][t][3] *= alb;
             }
         }
-        pb0[j] = movmatrix_trans(x0);  // P^T rows (tokens) 2c, 2c+1; column r
-        pb1[j] = movmatrix_trans(x1);  // tokens 2c+8, 2c+9
     }
     return __reduce_max_sync(0xffffffffu, nvmax);
 }
 
-// O^T += V^T . P^T from 16-byte V loads (head_dim order of mma_load_v). Rows
-// past every column's tokens are zeroed first (those slots may hold anything);
-// rows before that belong to some member's context.
-template <int D, int NT>
-__device__ __forceinline__ void pv_lds(uint4 (&vr)[4][D / 64], int nvmax, int c,
-                                       const uint32_t (&pb0)[NT], const uint32_t (&pb1)[NT],
-                                       float (&acc)[NT][D / 16][4]) {
-    if (nvmax < 16) {
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+// O^T += V^T . P^T over the unit's SUB sub-tiles, V^T fragments by
+// ldmatrix.trans from the stage (vb: V of sub-tile 0, sub-tile s at
+// vb + s * sub_bytes; natural head_dim order): a0 / a1 hold tokens 2c, 2c+1,
+// a2 / a3 tokens 2c+8, 2c+9 of the sub-tile. Rows at or past nvmax (past every
+// column's tokens: they may hold anything) are zeroed first; rows before that
+// belong to some member's context. The stage is released (`release`: its
+// empty barrier) as soon as the last fragments are in registers.
+template <int D, int NT, int SUB>
+__device__ __forceinline__ void pv_ldsm(uint32_t vb, int sub_bytes, int lane, int nvmax, int c,
+                                        const uint32_t (&pb0)[SUB][NT], const uint32_t (&pb1)[SUB][NT],
+                                        float (&acc)[NT][D / 16][4], uint32_t release) {
+    constexpr int MT = D / 16;
+    const int i = lane >> 3, row = 8 * (i >> 1) + (lane & 7);
+    // sub-tiles that hold a token of some column (nvmax >= 1 for a unit in use)
+    const int nsub = max(1, min(SUB, (nvmax + 15) >> 4));
 #pragma unroll
-        for (int hh = 0; hh < D / 64; ++hh) {
-            if (2 * c >= nvmax) vr[0][hh] = z;
-            if (2 * c + 1 >= nvmax) vr[1][hh] = z;
-            if (2 * c + 8 >= nvmax) vr[2][hh] = z;
-            if (2 * c + 9 >= nvmax) vr[3][hh] = z;
+    for (int s = 0; s < SUB; ++s) {
+        if (s >= nsub) break;
+        uint32_t va[MT][4];
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+            const int d0 = 16 * t + 8 * (i & 1);
+            ldsm_x4_trans(vb + s * sub_bytes + (d0 >> 6) * kBoxBytes + swz(row, (d0 & 63) >> 3), va[t]);
         }
-    }
-#pragma unroll
-    for (int t = 0; t < D / 16; ++t) {
-        const int hh = t >> 2, w = t & 3;
-        const uint32_t xa = word(vr[0][hh], w), xb = word(vr[1][hh], w);
-        const uint32_t ya = word(vr[2][hh], w), yb = word(vr[3][hh], w);
-        const uint32_t a0 = __byte_perm(xa, xb, 0x5410), a1 = __byte_perm(xa, xb, 0x7632);
-        const uint32_t a2 = __byte_perm(ya, yb, 0x5410), a3 = __byte_perm(ya, yb, 0x7632);
-#pragma unroll
-        for (int j = 0; j < NT; ++j) mma_16816(acc[j][t], a0, a1, a2, a3, pb0[j], pb1[j]);
-    }
-}
-
-// O^T += V^T . P^T from ldmatrix.trans fragments (natural head_dim order):
-// a0 / a1 hold tokens 2c, 2c+1, a2 / a3 tokens 2c+8, 2c+9, low half first.
-template <int D, int NT>
-__device__ __forceinline__ void pv_ldsm(uint32_t (&va)[D / 16][4], int nvmax, int c,
-                                        const uint32_t (&pb0)[NT], const uint32_t (&pb1)[NT],
-                                        float (&acc)[NT][D / 16][4]) {
-    if (nvmax < 16) {
-        const uint32_t m01 = (2 * c < nvmax ? 0x0000ffffu : 0u) | (2 * c + 1 < nvmax ? 0xffff0000u : 0u);
-        const uint32_t m89 = (2 * c + 8 < nvmax ? 0x0000ffffu : 0u) | (2 * c + 9 < nvmax ? 0xffff0000u : 0u);
-#pragma unroll
-        for (int t = 0; t < D / 16; ++t) {
-            va[t][0] &= m01;
-            va[t][1] &= m01;
-            va[t][2] &= m89;
-            va[t][3] &= m89;
+        if (s == nsub - 1) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(release);
         }
+        const int k0 = 16 * s;
+        if (k0 + 16 > nvmax) {
+            const uint32_t m01 = (k0 + 2 * c < nvmax ? 0x0000ffffu : 0u) |
+                                 (k0 + 2 * c + 1 < nvmax ? 0xffff0000u : 0u);
+            const uint32_t m89 = (k0 + 2 * c + 8 < nvmax ? 0x0000ffffu : 0u) |
+                                 (k0 + 2 * c + 9 < nvmax ? 0xffff0000u : 0u);
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+                va[t][0] &= m01;
+                va[t][1] &= m01;
+                va[t][2] &= m89;
+                va[t][3] &= m89;
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < MT; ++t)
+#pragma unroll
+            for (int j = 0; j < NT; ++j)
+                mma_16816(acc[j][t], va[t][0], va[t][1], va[t][2], va[t][3], pb0[s][j], pb1[s][j]);
     }
-#pragma unroll
-    for (int t = 0; t < D / 16; ++t)
-#pragma unroll
-        for (int j = 0; j < NT; ++j) mma_16816(acc[j][t], va[t][0], va[t][1], va[t][2], va[t][3], pb0[j], pb1[j]);
 }
 
 // Store one column's result (m, l = its running max and summed weights): bf16
@@ -1583,7 +1769,6 @@ __device__ __forceinline__ void grouped_store_col(const DecodeParams& p, int64_t
     const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
-#if PA_GROUPED_LDSM_V
         // rows r and r + 8 of m-tile t: head_dim 16t + r and 16t + 8 + r
         const int d0 = 16 * t + r, d1 = d0 + 8;
         if (P == 1) {
@@ -1595,16 +1780,6 @@ __device__ __forceinline__ void grouped_store_col(const DecodeParams& p, int64_t
             o[d0] = acc[t][e] * inv;
             o[d1] = acc[t][e + 2] * inv;
         }
-#else
-        // rows r and r + 8 of m-tile t: head_dim d0 and d0 + 1
-        const int d0 = (t >> 2) * 64 + r * 8 + 2 * (t & 3);
-        if (P == 1)
-            *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + row * D + d0) =
-                pack_bf16x2(acc[t][e] * inv, acc[t][e + 2] * inv);
-        else
-            *reinterpret_cast<float2*>(p.ws_o + (row * P + part) * D + d0) =
-                make_float2(acc[t][e] * inv, acc[t][e + 2] * inv);
-#endif
     }
     if (P > 1 && r == 0) {
         float* ml = p.ws_ml + (row * P + part) * 2;
@@ -1619,9 +1794,10 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                           const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
                           int num_items, int gs) {
     using G = GroupedGeom<D, CW, NT>;
+    constexpr int SUB = G::kSub;
     constexpr int KCH = D / 32;
-    constexpr int VCH = D / 64;
     constexpr int MT = D / 16;
+    constexpr int kUnitTokens = 16 * SUB;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
 
@@ -1652,26 +1828,28 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
         int cur_base = 0;
         uint32_t act_cur;
-        int phys_cur[kMaxGroupSeqs];
-        gload_phys(p, cur, cur_base, gs, lane, act_cur, phys_cur);
+        int phys_cur[kMaxGroupSeqs][SUB];
+        gload_units<SUB>(p, cur, cur_base, gs, lane, act_cur, phys_cur);
         while (cur.valid && !dead) {
-            const int n_sub = (cur.tmax - cur.t0 + 15) >> 4;
+            const int n_units = (cur.tmax - cur.t0 + kUnitTokens - 1) / kUnitTokens;
             GItem nxt = cur;
             int nxt_base = cur_base + 32;
-            if (nxt_base >= n_sub) {
+            if (nxt_base >= n_units) {
                 nxt = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
                 nxt_base = 0;
             }
             uint32_t act_nxt;
-            int phys_nxt[kMaxGroupSeqs];
-            gload_phys(p, nxt, nxt_base, gs, lane, act_nxt, phys_nxt);  // in flight meanwhile
-            issue_units<G>(&kmap, &vmap, p, ring, hdr, cur, cur_base, n_sub, act_cur, phys_cur, lane,
-                           g, issued, dead);
+            int phys_nxt[kMaxGroupSeqs][SUB];
+            gload_units<SUB>(p, nxt, nxt_base, gs, lane, act_nxt, phys_nxt);  // in flight meanwhile
+            issue_units_sub<G>(&kmap, &vmap, p, ring, hdr, cur, cur_base, n_units, act_cur, phys_cur,
+                               lane, g, issued, dead);
             cur = nxt;
             cur_base = nxt_base;
             act_cur = act_nxt;
 #pragma unroll
-            for (int m = 0; m < kMaxGroupSeqs; ++m) phys_cur[m] = phys_nxt[m];
+            for (int m = 0; m < kMaxGroupSeqs; ++m)
+#pragma unroll
+                for (int u = 0; u < SUB; ++u) phys_cur[m][u] = phys_nxt[m][u];
         }
         drain_ring<G>(ring, issued, lane);
         return;
@@ -1745,41 +1923,28 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                 }
                 const uint32_t h = hdr[st];
                 const bool mine = ring.valid[st] != 0 && (h & wbits) != 0;
-                const int tok0 = cur.t0 + (int)((h >> kUnitSubShift) & kUnitSubMask) * 16;
-                const uint32_t kb = ring.stages + st * G::kStageBytes;
-                float sc[NT][4];
-#if PA_GROUPED_LDSM_V
-                uint32_t va[MT][4];
-#else
-                uint4 vr[4][VCH];
-#endif
                 if (mine) {
-                    mma_qk_n<D, NT>(kb, q, r, c, sc);
-#if PA_GROUPED_LDSM_V
-                    ldsm_load_v<D>(kb + G::kBoxes * kBoxBytes, lane, va);
-#else
-                    mma_load_v<D>(kb + G::kBoxes * kBoxBytes, r, c, vr);
-#endif
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
-                ++g;
-                if (mine) {
+                    const int tok0 = cur.t0 + (int)((h >> kUnitSubShift) & kUnitSubMask) * kUnitTokens;
+                    const uint32_t kb = ring.stages + st * G::kStageBytes;
+                    float sc[SUB][NT][4];
+#pragma unroll
+                    for (int u = 0; u < SUB; ++u) mma_qk_n<D, NT>(kb + u * G::kSubBytes, q, r, c, sc[u]);
                     int nva[NT], nvb[NT];
 #pragma unroll
                     for (int j = 0; j < NT; ++j) {
-                        nva[j] = (h & bita[j]) ? min(16, t1a[j] - tok0) : 0;
-                        nvb[j] = (h & bitb[j]) ? min(16, t1b[j] - tok0) : 0;
+                        nva[j] = (h & bita[j]) ? min(kUnitTokens, t1a[j] - tok0) : 0;
+                        nvb[j] = (h & bitb[j]) ? min(kUnitTokens, t1b[j] - tok0) : 0;
                     }
-                    uint32_t pb0[NT], pb1[NT];
-                    const int nvmax = softmax_update_n<D, NT>(sc, nva, nvb, p.scale_log2, r, acc, ma,
-                                                              mb, la, lb, pb0, pb1);
-#if PA_GROUPED_LDSM_V
-                    pv_ldsm<D, NT>(va, nvmax, c, pb0, pb1, acc);
-#else
-                    pv_lds<D, NT>(vr, nvmax, c, pb0, pb1, acc);
-#endif
+                    uint32_t pb0[SUB][NT], pb1[SUB][NT];
+                    const int nvmax = softmax_update_n<D, NT, SUB>(sc, nva, nvb, p.scale_log2, r, acc, ma,
+                                                                   mb, la, lb, pb0, pb1);
+                    pv_ldsm<D, NT, SUB>(kb + SUB * G::kSubBytes, G::kSubBytes, lane, nvmax, c, pb0, pb1,
+                                        acc, ring.empty + 8 * st);  // releases the stage
+                } else {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
                 }
+                ++g;
                 if (h & kUnitLast) break;
             }
         }
