@@ -64,6 +64,9 @@ namespace {
 #ifndef PA_MMA_PREFETCH_Q
 #define PA_MMA_PREFETCH_Q 1
 #endif
+#ifndef PA_MMA_CODES_MHA
+#define PA_MMA_CODES_MHA 0
+#endif
 
 constexpr int kBoxBytes = 16 * 128;  // 16 rows x 128 bytes
 constexpr int kGroupMax = 8;
@@ -1159,9 +1162,16 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
 // ---------------------------------------------------------------------------
 
 // V fragments by ldmatrix.trans (head_dim in natural order in the
-// accumulator); independent accumulation chains per QK product.
+// accumulator). QK accumulation chains per sub-tile (1: a unit of several
+// sub-tiles already gives independent chains).
 #ifndef PA_GROUPED_QK_CHAINS
-#define PA_GROUPED_QK_CHAINS 2
+#define PA_GROUPED_QK_CHAINS 1
+#endif
+// Softmax weights by the hardware 2^x approximation (ex2.approx.ftz: relative
+// error ~2^-22, far below the bf16 rounding the weights then take) on
+// fma(score, scale, -max) instead of exp2f on separately scaled scores.
+#ifndef PA_GROUPED_FAST_EXP
+#define PA_GROUPED_FAST_EXP 1
 #endif
 
 constexpr int kMaxGroupSeqs = 8;            // members per group (header mask bits 0..7)
@@ -1627,6 +1637,12 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&a)[4]) {
                  : "r"(addr));
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Online-softmax update over a unit of SUB sub-tiles for NT n-tiles whose
 // columns may each see a different number of valid tokens: nva / nvb = valid
 // tokens (from the unit's first) of this thread's columns 2c and 2c + 1 of
@@ -1642,6 +1658,9 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], c
                                                 float (&mb)[NT], float (&la)[NT], float (&lb)[NT],
                                                 uint32_t (&pb0)[SUB][NT], uint32_t (&pb1)[SUB][NT]) {
     constexpr int MT = D / 16;
+    // kFast: masked raw scores, max scaled once, weights 2^fma(s, scale, -max)
+    constexpr bool kFast = PA_GROUPED_FAST_EXP != 0;
+    const float mul = kFast ? 1.f : scale_log2;
     float sv[SUB][NT][4], mxa[NT], mxb[NT];
     int nvmax = 0;
 #pragma unroll
@@ -1650,10 +1669,10 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], c
 #pragma unroll
         for (int s = 0; s < SUB; ++s) {
             const int t0 = 16 * s + r, t1 = t0 + 8;
-            sv[s][j][0] = t0 < nva[j] ? sc[s][j][0] * scale_log2 : -INFINITY;  // token t0, column 2c
-            sv[s][j][1] = t0 < nvb[j] ? sc[s][j][1] * scale_log2 : -INFINITY;  // token t0, column 2c+1
-            sv[s][j][2] = t1 < nva[j] ? sc[s][j][2] * scale_log2 : -INFINITY;  // token t1, column 2c
-            sv[s][j][3] = t1 < nvb[j] ? sc[s][j][3] * scale_log2 : -INFINITY;  // token t1, column 2c+1
+            sv[s][j][0] = t0 < nva[j] ? sc[s][j][0] * mul : -INFINITY;  // token t0, column 2c
+            sv[s][j][1] = t0 < nvb[j] ? sc[s][j][1] * mul : -INFINITY;  // token t0, column 2c+1
+            sv[s][j][2] = t1 < nva[j] ? sc[s][j][2] * mul : -INFINITY;  // token t1, column 2c
+            sv[s][j][3] = t1 < nvb[j] ? sc[s][j][3] * mul : -INFINITY;  // token t1, column 2c+1
             mxa[j] = fmaxf(mxa[j], fmaxf(sv[s][j][0], sv[s][j][2]));
             mxb[j] = fmaxf(mxb[j], fmaxf(sv[s][j][1], sv[s][j][3]));
         }
@@ -1670,6 +1689,10 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], c
     bool mv = false;
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
+        if (kFast) {  // the scaled max: scaling by a positive factor keeps the order
+            mxa[j] *= scale_log2;
+            mxb[j] *= scale_log2;
+        }
         mxa[j] = fmaxf(ma[j], mxa[j]);  // new running max
         mxb[j] = fmaxf(mb[j], mxb[j]);
         mv = mv || mxa[j] != ma[j] || mxb[j] != mb[j];
@@ -1679,13 +1702,24 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], c
     for (int j = 0; j < NT; ++j) {
         const float ba = mxa[j] == -INFINITY ? 0.f : mxa[j];
         const float bb = mxb[j] == -INFINITY ? 0.f : mxb[j];
-        const float ala = moved ? exp2f(ma[j] - ba) : 1.f;
-        const float alb = moved ? exp2f(mb[j] - bb) : 1.f;
+        float ala = 1.f, alb = 1.f;
+        if (moved) {
+            if (kFast) {  // a max that did not move rescales by exactly 1
+                ala = ma[j] == mxa[j] ? 1.f : ex2_approx(ma[j] - ba);
+                alb = mb[j] == mxb[j] ? 1.f : ex2_approx(mb[j] - bb);
+            } else {
+                ala = exp2f(ma[j] - ba);
+                alb = exp2f(mb[j] - bb);
+            }
+        }
+        auto wt = [&](float x, float b) {
+            return kFast ? ex2_approx(fmaf(x, scale_log2, -b)) : exp2f(x - b);
+        };
         float suma = 0.f, sumb = 0.f;
 #pragma unroll
         for (int s = 0; s < SUB; ++s) {
-            const uint32_t x0 = pack_bf16x2(exp2f(sv[s][j][0] - ba), exp2f(sv[s][j][1] - bb));
-            const uint32_t x1 = pack_bf16x2(exp2f(sv[s][j][2] - ba), exp2f(sv[s][j][3] - bb));
+            const uint32_t x0 = pack_bf16x2(wt(sv[s][j][0], ba), wt(sv[s][j][1], bb));
+            const uint32_t x1 = pack_bf16x2(wt(sv[s][j][2], ba), wt(sv[s][j][3], bb));
             suma += bf16_lo(x0) + bf16_lo(x1);
             sumb += bf16_hi(x0) + bf16_hi(x1);
             pb0[s][j] = movmatrix_trans(x0);  // P^T rows (tokens) 16s + 2c, 2c+1; column r
@@ -2599,9 +2633,15 @@ cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bo
 
 int mma_ctas_per_sm() { return PA_MMA_MIN_BLOCKS; }
 
+// The tensor-core consumer takes grouped-query bf16 and codes. With
+// PA_MMA_CODES_MHA it also takes one query head per kv head over codes (one
+// MMA column of eight): fewer instructions per element than the CUDA-core
+// consumer, but measured slower on B200 (13B MHA: fp8 564 vs 536 us, int8 661
+// vs 622 us; 7B fp8 173 vs 125 us), so it is off by default.
 bool mma_supported(int dtype, int head_dim, int group) {
     const bool codes = (dtype == 2 || dtype == 3) && head_dim == 128;
-    return (codes || (dtype == 1 && (head_dim == 64 || head_dim == 128))) && group >= 2 &&
+    const int least = codes && PA_MMA_CODES_MHA ? 1 : 2;
+    return (codes || (dtype == 1 && (head_dim == 64 || head_dim == 128))) && group >= least &&
            group <= kGroupMax;
 }
 

@@ -27,14 +27,36 @@ __device__ __forceinline__ int clamp_context(int ctx, int max_ctx) {
 // the union of the partitions. grid = (num_heads, rows of out). Launched as a
 // programmatic dependent of the decode kernel: it may start while the decode
 // drains and waits (griddepcontrol.wait) for all of its results.
+//
+// Warp w takes partitions w, w + 4, ...; each lane holds D / 32 consecutive
+// elements of a partial output, and a warp issues the loads of up to kBatch
+// partitions before it uses any of them, so one round trip to memory covers
+// the typical partition count. The warps' sums meet in shared memory.
+constexpr int kWarps = kThreads / 32;
+constexpr int kBatch = 16;
+
+template <int V>
+struct VecF;
+template <>
+struct VecF<2> {
+    using type = float2;
+};
+template <>
+struct VecF<4> {
+    using type = float4;
+};
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 partition_reduce_kernel(const DecodeParams p) {
-    extern __shared__ float sm_w[];  // [num_partitions] weights
-    __shared__ float sm_L;
+    constexpr int V = D / 32;  // elements per lane
+    using Vec = typename VecF<V>::type;
+    __shared__ float sm_acc[kWarps][D];
+    __shared__ float sm_l[kWarps];
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int h = blockIdx.x;
     const int row = blockIdx.y;  // sequence, or query token with multi-token queries
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int ctx;
     if (p.query_start == nullptr) {
         ctx = clamp_context(__ldg(p.context_lens + row), p.max_context_len);
@@ -52,32 +74,52 @@ partition_reduce_kernel(const DecodeParams p) {
     }
     const int n = (ctx + p.partition_size - 1) / p.partition_size;
     const int64_t out_row = (int64_t)row * p.num_heads + h;
-    const float* ml = p.ws_ml + out_row * p.num_partitions * 2;
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        float M = -INFINITY;
-        for (int j = lane; j < n; j += 32) M = fmaxf(M, ml[2 * j]);
+    const float2* ml = reinterpret_cast<const float2*>(p.ws_ml + out_row * p.num_partitions * 2);
+    const float* o = p.ws_o + out_row * p.num_partitions * D;
+    // M over all partitions, by every warp (no block barrier needed for it)
+    float M = -INFINITY;
+    for (int j = lane; j < n; j += 32) M = fmaxf(M, ml[j].x);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        float L = 0.f;
-        for (int j = lane; j < n; j += 32) {
-            const float mj = ml[2 * j];
-            const float w = mj == -INFINITY ? 0.f : ml[2 * j + 1] * exp2f(mj - M);
-            sm_w[j] = w;
-            L += w;
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float acc[V];
+#pragma unroll
+    for (int k = 0; k < V; ++k) acc[k] = 0.f;
+    float L = 0.f;
+    for (int j0 = warp; j0 < n; j0 += kWarps * kBatch) {
+        Vec ov[kBatch];
+        float2 mlv[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int j = j0 + u * kWarps;
+            if (j < n) {
+                ov[u] = *reinterpret_cast<const Vec*>(o + (int64_t)j * D + lane * V);
+                mlv[u] = ml[j];
+            }
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-        if (lane == 0) sm_L = L;
+        for (int u = 0; u < kBatch; ++u) {
+            const int j = j0 + u * kWarps;
+            if (j < n) {
+                const float w = mlv[u].x == -INFINITY ? 0.f : mlv[u].y * exp2f(mlv[u].x - M);
+                const float* x = reinterpret_cast<const float*>(&ov[u]);
+#pragma unroll
+                for (int k = 0; k < V; ++k) acc[k] = fmaf(w, x[k], acc[k]);
+                L += w;
+            }
+        }
     }
+#pragma unroll
+    for (int k = 0; k < V; ++k) sm_acc[warp][lane * V + k] = acc[k];
+    if (lane == 0) sm_l[warp] = L;
     __syncthreads();
-    const float L = sm_L;
-    const float* o = p.ws_o + out_row * p.num_partitions * D;
+    float Lt = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) Lt += sm_l[w];
     for (int d = threadIdx.x; d < D; d += kThreads) {
-        float acc = 0.f;
-#pragma unroll 8
-        for (int j = 0; j < n; ++j) acc = fmaf(sm_w[j], o[(int64_t)j * D + d], acc);
-        Elem<T>::store(p.out, out_row * D + d, L > 0.f ? acc / L : 0.f);
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) a += sm_acc[w][d];
+        Elem<T>::store(p.out, out_row * D + d, Lt > 0.f ? a / Lt : 0.f);
     }
 }
 
@@ -86,7 +128,7 @@ cudaError_t launch_reduce_t(const DecodeParams& p, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.num_heads, (unsigned)p.num_rows);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = (size_t)p.num_partitions * sizeof(float);
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
