@@ -1173,6 +1173,19 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
 #ifndef PA_GROUPED_FAST_EXP
 #define PA_GROUPED_FAST_EXP 1
 #endif
+// Column sums of the softmax weights by the tensor core: one more MMA per
+// sub-tile with an all-ones A operand (each row of the result is the column's
+// sum over the sub-tile's tokens), kept and rescaled like the accumulator,
+// instead of unpacking and adding the weights on the CUDA cores.
+#ifndef PA_GROUPED_MMA_SUM
+#define PA_GROUPED_MMA_SUM 1
+#endif
+// The producer's unit issue written once (leader picked at run time) rather
+// than unrolled over the eight possible leaders: a smaller kernel, but slower
+// on 8-beam MHA (116 vs 107 us), so off.
+#ifndef PA_GROUPED_ROLLED_ISSUE
+#define PA_GROUPED_ROLLED_ISSUE 0
+#endif
 
 constexpr int kMaxGroupSeqs = 8;            // members per group (header mask bits 0..7)
 constexpr int kGroupedMaxCols = 64;         // query columns (member, head) per CTA
@@ -1570,6 +1583,38 @@ __device__ __forceinline__ void issue_units_sub(const CUtensorMap* kmap, const C
     for (int k0 = 0; k0 < total && !dead; k0 += G::kStages) {
         bool ok = true;
         int pos = first_pos;
+#if PA_GROUPED_ROLLED_ISSUE
+        // one copy of the issue code: the leader's ids picked by selects
+#pragma unroll 1
+        for (uint32_t rest = lead; rest != 0u && ok; rest &= rest - 1u, ++pos) {
+            const int m = __ffs(rest) - 1;
+            if (pos < k0 || pos >= k0 + G::kStages) continue;
+            int ph[SUB];
+            int ns = nsub[0];
+#pragma unroll
+            for (int u = 0; u < SUB; ++u) ph[u] = phys[0][u];
+#pragma unroll
+            for (int mm = 1; mm < kMaxGroupSeqs; ++mm) {
+                if (m == mm) {
+                    ns = nsub[mm];
+#pragma unroll
+                    for (int u = 0; u < SUB; ++u) ph[u] = phys[mm][u];
+                }
+            }
+            uint32_t mask = 0;
+#pragma unroll
+            for (int m2 = 0; m2 < kMaxGroupSeqs; ++m2) {
+                bool eq = m2 >= m && ((act >> m2) & 1u) && nsub[m2] == ns;
+#pragma unroll
+                for (int u = 0; u < SUB; ++u) eq = eq && phys[m2][u] == ph[u];
+                if (eq) mask |= 1u << m2;
+            }
+            const uint32_t h = mask | ((uint32_t)i << kUnitSubShift) |
+                               (last_batch && pos == total - 1 ? kUnitLast : 0u);
+            ok = issue_unit<G>(kmap, vmap, p, ring, g + pos, ph, ns, it.kh, tok0, hdr, h);
+            if (ok) issued = g + pos + 1;
+        }
+#else
 #pragma unroll
         for (int m = 0; m < kMaxGroupSeqs; ++m) {
             if ((lead >> m) & 1u) {
@@ -1586,6 +1631,7 @@ __device__ __forceinline__ void issue_units_sub(const CUtensorMap* kmap, const C
                 ++pos;
             }
         }
+#endif
         dead = __any_sync(0xffffffffu, !ok);
     }
     issued = __reduce_max_sync(0xffffffffu, issued);
@@ -1656,8 +1702,10 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], c
                                                 const int (&nvb)[NT], float scale_log2, int r,
                                                 float (&acc)[NT][D / 16][4], float (&ma)[NT],
                                                 float (&mb)[NT], float (&la)[NT], float (&lb)[NT],
-                                                uint32_t (&pb0)[SUB][NT], uint32_t (&pb1)[SUB][NT]) {
+                                                float (&ls)[NT][4], uint32_t (&pb0)[SUB][NT],
+                                                uint32_t (&pb1)[SUB][NT]) {
     constexpr int MT = D / 16;
+    constexpr bool kMmaSum = PA_GROUPED_MMA_SUM != 0;
     // kFast: masked raw scores, max scaled once, weights 2^fma(s, scale, -max)
     constexpr bool kFast = PA_GROUPED_FAST_EXP != 0;
     const float mul = kFast ? 1.f : scale_log2;
@@ -1720,13 +1768,17 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], c
         for (int s = 0; s < SUB; ++s) {
             const uint32_t x0 = pack_bf16x2(wt(sv[s][j][0], ba), wt(sv[s][j][1], bb));
             const uint32_t x1 = pack_bf16x2(wt(sv[s][j][2], ba), wt(sv[s][j][3], bb));
-            suma += bf16_lo(x0) + bf16_lo(x1);
-            sumb += bf16_hi(x0) + bf16_hi(x1);
+            if (!kMmaSum) {
+                suma += bf16_lo(x0) + bf16_lo(x1);
+                sumb += bf16_hi(x0) + bf16_hi(x1);
+            }
             pb0[s][j] = movmatrix_trans(x0);  // P^T rows (tokens) 16s + 2c, 2c+1; column r
             pb1[s][j] = movmatrix_trans(x1);  // tokens 16s + 2c+8, 2c+9
         }
-        la[j] = fmaf(la[j], ala, suma);
-        lb[j] = fmaf(lb[j], alb, sumb);
+        if (!kMmaSum) {
+            la[j] = fmaf(la[j], ala, suma);
+            lb[j] = fmaf(lb[j], alb, sumb);
+        }
         ma[j] = mxa[j];
         mb[j] = mxb[j];
         if (moved) {
@@ -1736,6 +1788,12 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], c
                 acc[j][t][1] *= alb;
                 acc[j][t][2] *= ala;
                 acc[j][t][3] *= alb;
+            }
+            if (kMmaSum) {
+                ls[j][0] *= ala;
+                ls[j][1] *= alb;
+                ls[j][2] *= ala;
+                ls[j][3] *= alb;
             }
         }
     }
@@ -1752,7 +1810,8 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], c
 template <int D, int NT, int SUB>
 __device__ __forceinline__ void pv_ldsm(uint32_t vb, int sub_bytes, int lane, int nvmax, int c,
                                         const uint32_t (&pb0)[SUB][NT], const uint32_t (&pb1)[SUB][NT],
-                                        float (&acc)[NT][D / 16][4], uint32_t release) {
+                                        float (&acc)[NT][D / 16][4], float (&ls)[NT][4],
+                                        uint32_t release) {
     constexpr int MT = D / 16;
     const int i = lane >> 3, row = 8 * (i >> 1) + (lane & 7);
     // sub-tiles that hold a token of some column (nvmax >= 1 for a unit in use)
@@ -1789,6 +1848,11 @@ __device__ __forceinline__ void pv_ldsm(uint32_t vb, int sub_bytes, int lane, in
 #pragma unroll
             for (int j = 0; j < NT; ++j)
                 mma_16816(acc[j][t], va[t][0], va[t][1], va[t][2], va[t][3], pb0[s][j], pb1[s][j]);
+        if (PA_GROUPED_MMA_SUM) {
+            constexpr uint32_t kOnes = 0x3F803F80u;  // bf16 1.0, 1.0
+#pragma unroll
+            for (int j = 0; j < NT; ++j) mma_16816(ls[j], kOnes, kOnes, kOnes, kOnes, pb0[s][j], pb1[s][j]);
+        }
     }
 }
 
@@ -1937,12 +2001,13 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             t1a[j] = __shfl_sync(0xffffffffu, cur.t1_lane, ma & (kMaxGroupSeqs - 1));
             t1b[j] = __shfl_sync(0xffffffffu, cur.t1_lane, mb & (kMaxGroupSeqs - 1));
         }
-        float acc[NT][MT][4];
+        float acc[NT][MT][4], ls[NT][4];
         float ma[NT], mb[NT], la[NT], lb[NT];
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
 #pragma unroll
             for (int t = 0; t < MT; ++t) acc[j][t][0] = acc[j][t][1] = acc[j][t][2] = acc[j][t][3] = 0.f;
+            ls[j][0] = ls[j][1] = ls[j][2] = ls[j][3] = 0.f;
             ma[j] = mb[j] = -INFINITY;
             la[j] = lb[j] = 0.f;
         }
@@ -1971,9 +2036,9 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                     }
                     uint32_t pb0[SUB][NT], pb1[SUB][NT];
                     const int nvmax = softmax_update_n<D, NT, SUB>(sc, nva, nvb, p.scale_log2, r, acc, ma,
-                                                                   mb, la, lb, pb0, pb1);
+                                                                   mb, la, lb, ls, pb0, pb1);
                     pv_ldsm<D, NT, SUB>(kb + SUB * G::kSubBytes, G::kSubBytes, lane, nvmax, c, pb0, pb1,
-                                        acc, ring.empty + 8 * st);  // releases the stage
+                                        acc, ls, ring.empty + 8 * st);  // releases the stage
                 } else {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
@@ -1985,10 +2050,15 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         if (dead) break;
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
+            if (PA_GROUPED_MMA_SUM) {  // every row of the sums tile holds the column sums
+                la[j] = ls[j][0];
+                lb[j] = ls[j][1];
+            } else {
 #pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
-                la[j] += __shfl_xor_sync(0xffffffffu, la[j], off);
-                lb[j] += __shfl_xor_sync(0xffffffffu, lb[j], off);
+                for (int off = 4; off < 32; off <<= 1) {
+                    la[j] += __shfl_xor_sync(0xffffffffu, la[j], off);
+                    lb[j] += __shfl_xor_sync(0xffffffffu, lb[j], off);
+                }
             }
         }
 #pragma unroll
