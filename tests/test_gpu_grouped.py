@@ -101,6 +101,34 @@ def test_shared_equals_private_bitwise(ps):
     assert G.bits_equal(shared, out2)
 
 
+@pytest.mark.parametrize("ps", [0, 48])
+def test_members_sharing_blocks_with_different_lengths(ps):
+    """Members that share every block but end at different tokens of one unit
+    of the grouped kernel (a sequence and prefixes of it): each member takes
+    its own units there, so results match the oracle and equal a private-copy
+    layout bit for bit."""
+    ctx = [150, 120, 97, 150, 64, 65, 0, 33]
+    wl = G.custom(len(ctx), 16, 2, 128, 16, "bf16", ctx, seed=21)
+    wl.block_tables[1:4, :] = wl.block_tables[0, :]   # 1..3 read 0's blocks
+    wl.block_tables[5, :] = wl.block_tables[4, :]
+    wl.slot_mapping[:] = -1                            # no appends into shared blocks
+    vals = W.make_values(wl, DEV, poison=False)
+    host = G.host_copy(vals)
+    shared = G.gpu_step(wl, vals, partition_size=ps, group_size=4)
+    pa.pa_sync_check()
+    assert G.last_kernel() in G.kernel_set(pa.PA_KERNEL_GROUPED)
+    ref = G.oracle_step(wl, host)
+    G.check_tolerance(G.to_f64(shared), ref, "bf16", f"prefix members ps={ps}")
+    kc2, vc2, tables2, was_shared = _private_copy(wl, vals)
+    out2 = torch.empty_like(vals["q"])
+    pa.pa_decode_grouped(out2, vals["q"], kc2, vc2, tables2,
+                         torch.as_tensor(wl.context_lens, device=DEV), wl.scale, 4,
+                         max_context_len=wl.max_context_len, partition_size=ps)
+    torch.cuda.synchronize()
+    assert was_shared
+    assert G.bits_equal(shared, out2)
+
+
 def test_placement_invariance_bitwise():
     wl = W.cow_beam4(num_prompts=2, prompt_len=250, max_suffix=40, num_heads=32, num_kv_heads=4,
                      head_dim=128)
