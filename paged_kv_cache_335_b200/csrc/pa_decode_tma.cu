@@ -234,6 +234,21 @@ __device__ __forceinline__ int clamp_ctx(int ctx, int max_ctx, bool report) {
     return ctx;
 }
 
+// 2^x by the hardware approximation (ex2.approx.ftz: relative error about
+// 2^-22; results below 2^-126 flush to 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Softmax weights of the CUDA-core consumer over quantised codes by
+// ex2_approx rather than exp2f: that consumer is bound by instruction issue
+// (one widening per code), bf16 and fp32 caches are bound by HBM.
+#ifndef PA_SIMT_CODES_FAST_EXP
+#define PA_SIMT_CODES_FAST_EXP 1
+#endif
+
 // ---------------------------------------------------------------------------
 // CUDA-core consumer: one query head per CTA.
 // ---------------------------------------------------------------------------
@@ -254,6 +269,8 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
     constexpr int RPL = 32 / CPR;               // rows per warp-wide pass
     constexpr int ITER = 16 / RPL;              // passes per 16-row sub-tile
     constexpr int IPP = ITER < 8 ? ITER : 8;    // passes held in registers at once
+    constexpr bool kFastExp = PA_SIMT_CODES_FAST_EXP && (std::is_same<T, E4M3Code>::value ||
+                                                         std::is_same<T, Int8Code>::value);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
 
@@ -360,14 +377,14 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                 if (mt == -INFINITY) continue;  // only masked rows in this pass
                 const float m_new = fmaxf(m, mt);
                 if (m_new != m) {  // warp-uniform; a factor of exactly 1 changes no bit
-                    const float alpha = exp2f(m - m_new);
+                    const float alpha = kFastExp ? ex2_approx(m - m_new) : exp2f(m - m_new);
                     l *= alpha;
 #pragma unroll
                     for (int j = 0; j < VEC; ++j) acc[j] *= alpha;
                 }
 #pragma unroll
                 for (int it = 0; it < IPP; ++it) {
-                    const float pr = exp2f(sc[it] - m_new);
+                    const float pr = kFastExp ? ex2_approx(sc[it] - m_new) : exp2f(sc[it] - m_new);
                     l += pr;
                     const int tok = tok0 + (pass + it) * RPL + rs;
                     if (tok < t1) {  // slots past the context may hold anything, even NaN
@@ -1681,12 +1698,6 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&a)[4]) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
                  : "r"(addr));
-}
-
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
 }
 
 // Online-softmax update over a unit of SUB sub-tiles for NT n-tiles whose
