@@ -248,6 +248,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
 #ifndef PA_SIMT_CODES_FAST_EXP
 #define PA_SIMT_CODES_FAST_EXP 1
 #endif
+// Int8 codes widened with a bias of 1152 (one byte permute per two codes, no
+// per-code subtraction); the bias leaves the scores as 1152 x the sum of the
+// lane's q elements and the output as 1152 x the sum of the weights.
+#ifndef PA_SIMT_INT8_BIASED
+#define PA_SIMT_INT8_BIASED 1
+#endif
 
 // ---------------------------------------------------------------------------
 // CUDA-core consumer: one query head per CTA.
@@ -271,6 +277,7 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
     constexpr int IPP = ITER < 8 ? ITER : 8;    // passes held in registers at once
     constexpr bool kFastExp = PA_SIMT_CODES_FAST_EXP && (std::is_same<T, E4M3Code>::value ||
                                                          std::is_same<T, Int8Code>::value);
+    constexpr bool kBiased = PA_SIMT_INT8_BIASED && std::is_same<T, Int8Code>::value;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
 
@@ -326,6 +333,11 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                 for (int j = 0; j < QV; ++j) qf[u * QV + j] = f[j] * qs;
             }
         }
+        float qsum = 0.f;  // biased int8 widening: what the bias adds to this lane's dot products
+        if constexpr (kBiased) {
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) qsum += qf[j];
+        }
         bool dead = false;
         for (int i = warp; i < n_sub && !dead; i += kConsumerWarps) {
             const int st = i % G::kStages;
@@ -358,10 +370,12 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
                 for (int it = 0; it < IPP; ++it) {
                     float kf[VEC];
-                    Elem<T>::widen(kr[it], kf);
+                    if constexpr (kBiased) int8_widen_biased(kr[it], kf);
+                    else Elem<T>::widen(kr[it], kf);
                     float dot = 0.f;
 #pragma unroll
                     for (int j = 0; j < VEC; ++j) dot = fmaf(qf[j], kf[j], dot);
+                    if constexpr (kBiased) dot = fmaf(-kInt8WidenBias, qsum, dot);
 #pragma unroll
                     for (int off = 1; off < CPR; off <<= 1)
                         dot += __shfl_xor_sync(0xffffffffu, dot, off);
@@ -389,13 +403,18 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                     const int tok = tok0 + (pass + it) * RPL + rs;
                     if (tok < t1) {  // slots past the context may hold anything, even NaN
                         float vf[VEC];
-                        Elem<T>::widen(vr[it], vf);
+                        if constexpr (kBiased) int8_widen_biased(vr[it], vf);
+                        else Elem<T>::widen(vr[it], vf);
 #pragma unroll
                         for (int j = 0; j < VEC; ++j) acc[j] = fmaf(pr, vf[j], acc[j]);
                     }
                 }
                 m = m_new;
             }
+        }
+        if constexpr (kBiased) {  // the bias's share of the weighted sum: 1152 x the weights
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) acc[j] = fmaf(-kInt8WidenBias, l, acc[j]);
         }
 #pragma unroll
         for (int off = CPR; off < 32; off <<= 1) {

@@ -120,6 +120,28 @@ struct Elem<Int8Code> {
     }
 };
 
+// Int8 codes -> floats biased by 1152: with the sign bit flipped, byte b is
+// u = code + 128; one byte permute per two codes places u under the f16
+// exponent of 1024 (f16 bits 0x64uu = 1024 + u exactly), and the f16 -> f32
+// widening gives 1152 + code, exactly. The caller removes the bias once per
+// sum (bias x the sum of the weights) instead of once per code.
+constexpr float kInt8WidenBias = 1152.0f;
+__device__ __forceinline__ void int8_widen_biased(const uint4& c, float (&f)[16]) {
+    const uint32_t w[4] = {c.x ^ 0x80808080u, c.y ^ 0x80808080u, c.z ^ 0x80808080u,
+                           c.w ^ 0x80808080u};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t h01 = __byte_perm(w[i], 0x64646464u, 0x5140);  // f16x2 (1024 + u0, 1024 + u1)
+        const uint32_t h23 = __byte_perm(w[i], 0x64646464u, 0x5342);
+        const __half2 a = *reinterpret_cast<const __half2*>(&h01);
+        const __half2 b = *reinterpret_cast<const __half2*>(&h23);
+        f[4 * i + 0] = __low2float(a);
+        f[4 * i + 1] = __high2float(a);
+        f[4 * i + 2] = __low2float(b);
+        f[4 * i + 3] = __high2float(b);
+    }
+}
+
 // q / out element type for a cache element type (quantised caches: bf16).
 template <typename TC> struct QType { using type = TC; };
 template <> struct QType<E4M3Code> { using type = __nv_bfloat16; };
