@@ -64,9 +64,7 @@ namespace {
 #ifndef PA_MMA_PREFETCH_Q
 #define PA_MMA_PREFETCH_Q 1
 #endif
-#ifndef PA_MMA_CODES_MHA
-#define PA_MMA_CODES_MHA 0
-#endif
+
 
 constexpr int kBoxBytes = 16 * 128;  // 16 rows x 128 bytes
 constexpr int kGroupMax = 8;
@@ -1216,12 +1214,6 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
 #ifndef PA_GROUPED_MMA_SUM
 #define PA_GROUPED_MMA_SUM 1
 #endif
-// The producer's unit issue written once (leader picked at run time) rather
-// than unrolled over the eight possible leaders: a smaller kernel, but slower
-// on 8-beam MHA (116 vs 107 us), so off.
-#ifndef PA_GROUPED_ROLLED_ISSUE
-#define PA_GROUPED_ROLLED_ISSUE 0
-#endif
 
 constexpr int kMaxGroupSeqs = 8;            // members per group (header mask bits 0..7)
 constexpr int kGroupedMaxCols = 64;         // query columns (member, head) per CTA
@@ -1619,38 +1611,6 @@ __device__ __forceinline__ void issue_units_sub(const CUtensorMap* kmap, const C
     for (int k0 = 0; k0 < total && !dead; k0 += G::kStages) {
         bool ok = true;
         int pos = first_pos;
-#if PA_GROUPED_ROLLED_ISSUE
-        // one copy of the issue code: the leader's ids picked by selects
-#pragma unroll 1
-        for (uint32_t rest = lead; rest != 0u && ok; rest &= rest - 1u, ++pos) {
-            const int m = __ffs(rest) - 1;
-            if (pos < k0 || pos >= k0 + G::kStages) continue;
-            int ph[SUB];
-            int ns = nsub[0];
-#pragma unroll
-            for (int u = 0; u < SUB; ++u) ph[u] = phys[0][u];
-#pragma unroll
-            for (int mm = 1; mm < kMaxGroupSeqs; ++mm) {
-                if (m == mm) {
-                    ns = nsub[mm];
-#pragma unroll
-                    for (int u = 0; u < SUB; ++u) ph[u] = phys[mm][u];
-                }
-            }
-            uint32_t mask = 0;
-#pragma unroll
-            for (int m2 = 0; m2 < kMaxGroupSeqs; ++m2) {
-                bool eq = m2 >= m && ((act >> m2) & 1u) && nsub[m2] == ns;
-#pragma unroll
-                for (int u = 0; u < SUB; ++u) eq = eq && phys[m2][u] == ph[u];
-                if (eq) mask |= 1u << m2;
-            }
-            const uint32_t h = mask | ((uint32_t)i << kUnitSubShift) |
-                               (last_batch && pos == total - 1 ? kUnitLast : 0u);
-            ok = issue_unit<G>(kmap, vmap, p, ring, g + pos, ph, ns, it.kh, tok0, hdr, h);
-            if (ok) issued = g + pos + 1;
-        }
-#else
 #pragma unroll
         for (int m = 0; m < kMaxGroupSeqs; ++m) {
             if ((lead >> m) & 1u) {
@@ -1667,7 +1627,6 @@ __device__ __forceinline__ void issue_units_sub(const CUtensorMap* kmap, const C
                 ++pos;
             }
         }
-#endif
         dead = __any_sync(0xffffffffu, !ok);
     }
     issued = __reduce_max_sync(0xffffffffu, issued);
@@ -2733,15 +2692,13 @@ cudaError_t launch_decode_tma(const DecodeParams& p, int dtype, int head_dim, bo
 
 int mma_ctas_per_sm() { return PA_MMA_MIN_BLOCKS; }
 
-// The tensor-core consumer takes grouped-query bf16 and codes. With
-// PA_MMA_CODES_MHA it also takes one query head per kv head over codes (one
-// MMA column of eight): fewer instructions per element than the CUDA-core
-// consumer, but measured slower on B200 (13B MHA: fp8 564 vs 536 us, int8 661
-// vs 622 us; 7B fp8 173 vs 125 us), so it is off by default.
+// The tensor-core consumer takes grouped-query heads (g = 2..8) over bf16 or
+// codes. One query head per kv head stays on the CUDA-core consumer: over
+// codes the tensor-core one with one MMA column of eight measured slower on
+// B200 (13B MHA: fp8 564 vs 536 us, int8 661 vs 622 us; 7B fp8 173 vs 125 us).
 bool mma_supported(int dtype, int head_dim, int group) {
     const bool codes = (dtype == 2 || dtype == 3) && head_dim == 128;
-    const int least = codes && PA_MMA_CODES_MHA ? 1 : 2;
-    return (codes || (dtype == 1 && (head_dim == 64 || head_dim == 128))) && group >= least &&
+    return (codes || (dtype == 1 && (head_dim == 64 || head_dim == 128))) && group >= 2 &&
            group <= kGroupMax;
 }
 
