@@ -252,6 +252,46 @@ __device__ __forceinline__ float ex2_approx(float x) {
 #ifndef PA_SIMT_INT8_BIASED
 #define PA_SIMT_INT8_BIASED 1
 #endif
+// Codes as f16 operands of the mixed-precision fma (f16 x f16 + f32 -> f32,
+// one instruction per code, no widening to f32): q is rounded to f16 (exact
+// for bf16 values of magnitude 2^-14 .. 65504, as on the tensor-core path
+// over codes) and scaled after the dot product; the weights are rounded to
+// f16 and their sum is kept over the rounded values.
+#ifndef PA_SIMT_CODES_MIXED_FMA
+#define PA_SIMT_CODES_MIXED_FMA 1
+#endif
+
+// d = a * b + c for the two f16 halves of a and b (low with c0, high with c1),
+// products exact, one rounding to f32 each.
+__device__ __forceinline__ void fma2_f16_f32(uint32_t a, uint32_t b, float& c0, float& c1) {
+    asm("{\n .reg .b16 al, ah, bl, bh;\n mov.b32 {al, ah}, %2;\n mov.b32 {bl, bh}, %3;\n"
+        " fma.rn.f32.f16 %0, al, bl, %0;\n fma.rn.f32.f16 %1, ah, bh, %1;\n}"
+        : "+f"(c0), "+f"(c1) : "r"(a), "r"(b));
+}
+// d = p * (both halves of b) + c, p one f16 value (the low half of pp).
+__device__ __forceinline__ void fma2_f16s_f32(uint32_t pp, uint32_t b, float& c0, float& c1) {
+    asm("{\n .reg .b16 pl, ph, bl, bh;\n mov.b32 {pl, ph}, %2;\n mov.b32 {bl, bh}, %3;\n"
+        " fma.rn.f32.f16 %0, pl, bl, %0;\n fma.rn.f32.f16 %1, pl, bh, %1;\n}"
+        : "+f"(c0), "+f"(c1) : "r"(pp), "r"(b));
+}
+
+// 16 codes -> 8 f16x2 words: E4M3 exactly; int8 as 1152 + code (exact).
+template <typename TC>
+__device__ __forceinline__ void codes_to_f16x2(const uint4& c, uint32_t (&h)[8]) {
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if constexpr (std::is_same<TC, E4M3Code>::value) {
+            asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n"
+                " cvt.rn.f16x2.e4m3x2 %0, lo;\n cvt.rn.f16x2.e4m3x2 %1, hi;\n}"
+                : "=r"(h[2 * i]), "=r"(h[2 * i + 1]) : "r"(w[i]));
+        } else {
+            const uint32_t u = w[i] ^ 0x80808080u;
+            h[2 * i] = __byte_perm(u, 0x64646464u, 0x5140);
+            h[2 * i + 1] = __byte_perm(u, 0x64646464u, 0x5342);
+        }
+    }
+}
 
 // ---------------------------------------------------------------------------
 // CUDA-core consumer: one query head per CTA.
@@ -275,7 +315,9 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
     constexpr int IPP = ITER < 8 ? ITER : 8;    // passes held in registers at once
     constexpr bool kFastExp = PA_SIMT_CODES_FAST_EXP && (std::is_same<T, E4M3Code>::value ||
                                                          std::is_same<T, Int8Code>::value);
-    constexpr bool kBiased = PA_SIMT_INT8_BIASED && std::is_same<T, Int8Code>::value;
+    constexpr bool kCodes = std::is_same<T, E4M3Code>::value || std::is_same<T, Int8Code>::value;
+    constexpr bool kMixed = PA_SIMT_CODES_MIXED_FMA && kCodes;
+    constexpr bool kBiased = (PA_SIMT_INT8_BIASED || kMixed) && std::is_same<T, Int8Code>::value;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
 
@@ -320,15 +362,24 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
         const uint32_t coff = (uint32_t)(c / 8) * kBoxBytes;  // box of this lane's chunk
         const uint32_t cx = (uint32_t)(c % 8);
         float qf[VEC];
-        {
-            // the K scale of a quantised cache folds into q (exactly 1 otherwise)
-            const float qs = p.scale_log2 * (p.k_scale != nullptr ? __ldg(p.k_scale + kh) : 1.f);
+        uint32_t qh[VEC / 2];  // mixed-precision path: q as unscaled f16 pairs
+        // the K scale of a quantised cache folds into q (exactly 1 otherwise); the
+        // mixed-precision path applies it to the dot product instead
+        const float qs = p.scale_log2 * (p.k_scale != nullptr ? __ldg(p.k_scale + kh) : 1.f);
 #pragma unroll
-            for (int u = 0; u < VEC / QV; ++u) {
-                float f[QV];
-                Elem<TQ>::widen(ld_v4(static_cast<const TQ*>(p.q) + out_row * D + c * VEC + u * QV), f);
+        for (int u = 0; u < VEC / QV; ++u) {
+            float f[QV];
+            Elem<TQ>::widen(ld_v4(static_cast<const TQ*>(p.q) + out_row * D + c * VEC + u * QV), f);
 #pragma unroll
-                for (int j = 0; j < QV; ++j) qf[u * QV + j] = f[j] * qs;
+            for (int j = 0; j < QV; ++j) qf[u * QV + j] = kMixed ? f[j] : f[j] * qs;
+        }
+        if constexpr (kMixed) {
+#pragma unroll
+            for (int j = 0; j < VEC / 2; ++j) {
+                const __half2 h2 = __floats2half2_rn(qf[2 * j], qf[2 * j + 1]);
+                qh[j] = *reinterpret_cast<const uint32_t*>(&h2);
+                qf[2 * j] = __low2float(h2);  // the values the products use
+                qf[2 * j + 1] = __high2float(h2);
             }
         }
         float qsum = 0.f;  // biased int8 widening: what the bias adds to this lane's dot products
@@ -367,13 +418,24 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                 float sc[IPP];
 #pragma unroll
                 for (int it = 0; it < IPP; ++it) {
-                    float kf[VEC];
-                    if constexpr (kBiased) int8_widen_biased(kr[it], kf);
-                    else Elem<T>::widen(kr[it], kf);
                     float dot = 0.f;
+                    if constexpr (kMixed) {
+                        uint32_t kh2[VEC / 2];
+                        codes_to_f16x2<T>(kr[it], kh2);
+                        float d1 = 0.f;
 #pragma unroll
-                    for (int j = 0; j < VEC; ++j) dot = fmaf(qf[j], kf[j], dot);
-                    if constexpr (kBiased) dot = fmaf(-kInt8WidenBias, qsum, dot);
+                        for (int j = 0; j < VEC / 2; ++j) fma2_f16_f32(qh[j], kh2[j], dot, d1);
+                        dot += d1;
+                        if constexpr (kBiased) dot = fmaf(-kInt8WidenBias, qsum, dot);
+                        dot *= qs;
+                    } else {
+                        float kf[VEC];
+                        if constexpr (kBiased) int8_widen_biased(kr[it], kf);
+                        else Elem<T>::widen(kr[it], kf);
+#pragma unroll
+                        for (int j = 0; j < VEC; ++j) dot = fmaf(qf[j], kf[j], dot);
+                        if constexpr (kBiased) dot = fmaf(-kInt8WidenBias, qsum, dot);
+                    }
 #pragma unroll
                     for (int off = 1; off < CPR; off <<= 1)
                         dot += __shfl_xor_sync(0xffffffffu, dot, off);
@@ -397,14 +459,27 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
                 for (int it = 0; it < IPP; ++it) {
                     const float pr = kFastExp ? ex2_approx(sc[it] - m_new) : exp2f(sc[it] - m_new);
-                    l += pr;
                     const int tok = tok0 + (pass + it) * RPL + rs;
-                    if (tok < t1) {  // slots past the context may hold anything, even NaN
-                        float vf[VEC];
-                        if constexpr (kBiased) int8_widen_biased(vr[it], vf);
-                        else Elem<T>::widen(vr[it], vf);
+                    if constexpr (kMixed) {
+                        const __half ph = __float2half_rn(pr);  // the weight the products use
+                        l += __half2float(ph);
+                        if (tok < t1) {  // slots past the context may hold anything, even NaN
+                            uint32_t vh2[VEC / 2];
+                            codes_to_f16x2<T>(vr[it], vh2);
+                            const uint32_t pp = (uint32_t)__half_as_ushort(ph);
 #pragma unroll
-                        for (int j = 0; j < VEC; ++j) acc[j] = fmaf(pr, vf[j], acc[j]);
+                            for (int j = 0; j < VEC / 2; ++j)
+                                fma2_f16s_f32(pp, vh2[j], acc[2 * j], acc[2 * j + 1]);
+                        }
+                    } else {
+                        l += pr;
+                        if (tok < t1) {  // slots past the context may hold anything, even NaN
+                            float vf[VEC];
+                            if constexpr (kBiased) int8_widen_biased(vr[it], vf);
+                            else Elem<T>::widen(vr[it], vf);
+#pragma unroll
+                            for (int j = 0; j < VEC; ++j) acc[j] = fmaf(pr, vf[j], acc[j]);
+                        }
                     }
                 }
                 m = m_new;
