@@ -1774,21 +1774,33 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], c
     constexpr bool kFast = PA_GROUPED_FAST_EXP != 0;
     const float mul = kFast ? 1.f : scale_log2;
     float sv[SUB][NT][4], mxa[NT], mxb[NT];
-    int nvmax = 0;
+    int nvmax = 0, nvmin = 16 * SUB;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        nvmax = max(nvmax, max(nva[j], nvb[j]));
+        nvmin = min(nvmin, min(nva[j], nvb[j]));
+    }
+    // every column of the warp uses every token of the unit (the common case):
+    // no masking
+    const bool full = __all_sync(0xffffffffu, nvmin >= 16 * SUB);
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
         mxa[j] = mxb[j] = -INFINITY;
 #pragma unroll
         for (int s = 0; s < SUB; ++s) {
             const int t0 = 16 * s + r, t1 = t0 + 8;
-            sv[s][j][0] = t0 < nva[j] ? sc[s][j][0] * mul : -INFINITY;  // token t0, column 2c
-            sv[s][j][1] = t0 < nvb[j] ? sc[s][j][1] * mul : -INFINITY;  // token t0, column 2c+1
-            sv[s][j][2] = t1 < nva[j] ? sc[s][j][2] * mul : -INFINITY;  // token t1, column 2c
-            sv[s][j][3] = t1 < nvb[j] ? sc[s][j][3] * mul : -INFINITY;  // token t1, column 2c+1
+            if (full) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sv[s][j][e] = sc[s][j][e] * mul;
+            } else {
+                sv[s][j][0] = t0 < nva[j] ? sc[s][j][0] * mul : -INFINITY;  // token t0, column 2c
+                sv[s][j][1] = t0 < nvb[j] ? sc[s][j][1] * mul : -INFINITY;  // token t0, column 2c+1
+                sv[s][j][2] = t1 < nva[j] ? sc[s][j][2] * mul : -INFINITY;  // token t1, column 2c
+                sv[s][j][3] = t1 < nvb[j] ? sc[s][j][3] * mul : -INFINITY;  // token t1, column 2c+1
+            }
             mxa[j] = fmaxf(mxa[j], fmaxf(sv[s][j][0], sv[s][j][2]));
             mxb[j] = fmaxf(mxb[j], fmaxf(sv[s][j][1], sv[s][j][3]));
         }
-        nvmax = max(nvmax, max(nva[j], nvb[j]));
     }
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
