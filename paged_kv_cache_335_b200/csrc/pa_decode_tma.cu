@@ -17,13 +17,17 @@
 // * consumer warps take sub-tiles round robin (warp w: w, w+4, ...; § 4.2 of
 //   the same page), copy their fragments out of the stage, release it, and
 //   update a running max / sum / accumulator (online softmax in exp2).
-// Two consumers share this pipeline: the CUDA-core one (one query head per
-// CTA; any dtype) and the tensor-core one for grouped-query attention (bf16,
-// group 2..8: S^T = K Q^T and O^T += V^T P^T as m16n8k16 MMAs, tokens as M,
-// the query group as N). The swizzle makes every consumer fragment load
-// bank-conflict free. Every wait is bounded: after kWaitLimitNs the waiter
-// records PA_ERR_TIMEOUT and carries on, so the kernel always terminates.
-// The arithmetic order depends only on logical token positions.
+// Four consumers share this pipeline: the CUDA-core one (one query head per
+// CTA; any dtype, quantised codes through a mixed-precision fma), the
+// tensor-core one for grouped-query attention (bf16 or codes, group 2..8:
+// S^T = K Q^T and O^T += V^T P^T as m16n8k16 MMAs, tokens as M, the query
+// group as N), the grouped one (several sequences or query tokens that share
+// blocks, one CTA per group, units of several sub-tiles per softmax step) and
+// an opt-in tcgen05 variant of the grouped one. The swizzle makes every
+// consumer fragment load bank-conflict free. Every wait is bounded: after
+// kWaitLimitNs the waiter records PA_ERR_TIMEOUT and carries on, so the kernel
+// always terminates. The arithmetic order depends only on logical token
+// positions.
 #include <math.h>
 
 #include <type_traits>
