@@ -300,8 +300,19 @@ __device__ __forceinline__ void codes_to_f16x2(const uint4& c, uint32_t (&h)[8])
 // ---------------------------------------------------------------------------
 // CUDA-core consumer: one query head per CTA.
 // ---------------------------------------------------------------------------
+// Ring bytes of the consumer over one-byte codes (a 16-token K+V sub-tile is
+// 4 KiB there, half the bf16 one): 48 KiB lets 4 CTAs share an SM (13B on a
+// B200: int8 508 -> 494 us, fp8 493 -> 484 us against 64 KiB; 32 KiB 498 / 488).
+#ifndef PA_SIMT_CODES_RING_BYTES
+#define PA_SIMT_CODES_RING_BYTES 49152
+#endif
+template <typename T>
+constexpr bool is_code_type() {
+    return std::is_same<T, E4M3Code>::value || std::is_same<T, Int8Code>::value;
+}
 template <typename T, int D>
-using SimtGeom = Geom<T, D, PA_SIMT_CONSUMER_WARPS, PA_SIMT_RING_BYTES>;
+using SimtGeom = Geom<T, D, PA_SIMT_CONSUMER_WARPS,
+                      is_code_type<T>() ? PA_SIMT_CODES_RING_BYTES : PA_SIMT_RING_BYTES>;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(SimtGeom<T, D>::kThreads)
