@@ -310,7 +310,7 @@ int pa_decode_multi_num_partitions(int32_t num_seqs, int32_t num_query_tokens,
  * pa_decode_workspace_size with the quantised descriptor. Precision: the
  * products run with q rounded to f16 (exact for bf16 magnitudes from 2^-14
  * to 65504; larger q is outside this call's range) and the softmax weights
- * rounded to f16 (grouped-query heads: bf16), accumulated in fp32; results
+ * rounded to f16, accumulated in fp32; results
  * meet the bf16 bars of pa_decode. pa_decode,
  * pa_kv_append and the other decode calls refuse a quantised descriptor
  * (PA_ERR_DTYPE), and these two refuse an unquantised one.
