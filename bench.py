@@ -53,7 +53,9 @@ EXTRA_CONFIGS = [("llama7b", "llama7b", None, 1, None),
                  ("llama70b_verify4_tcgen05", "llama70b_verify4", 0, 1, "tcgen05"),
                  ("llama13b_bs16_fp8", "llama13b_bs16_fp8", None, 1, None),
                  ("llama13b_bs16_int8", "llama13b_bs16_int8", None, 1, None),
-                 ("llama70b_gqa_policy_fp8", "llama70b_gqa_fp8", 0, 1, None)]
+                 ("llama70b_gqa_policy_fp8", "llama70b_gqa_fp8", 0, 1, None),
+                 ("cow_beam4_grouped_fp8", "cow_beam4_fp8", 0, 4, None),
+                 ("llama70b_verify4_fp8", "llama70b_verify4_fp8", 0, 1, None)]
 # pa_test_last_decode_kernel() -> the decode kernel a call enqueued
 KERNEL_NAMES = {0: "decode_tma_simt_kernel (CUDA-core)",
                 1: "decode_tma_mma_kernel (persistent, tensor-core GQA)",
@@ -307,21 +309,21 @@ class Step:
             ((group_size,) if group_size > 1 else ()) + \
             (self.ps, P(self.ws.data_ptr()), ctypes.c_size_t(self.ws_bytes), self.sp)
         self.decode_fn = self.lib.pa_decode_grouped if group_size > 1 else self.lib.pa_decode
+        scales = (P(v["k_scale"].data_ptr()), P(v["v_scale"].data_ptr())) if wl.kv_quant else ()
         if wl.kv_quant:
-            self.args_decode = self.args_decode[:4] + (P(v["k_scale"].data_ptr()),
-                                                       P(v["v_scale"].data_ptr())) + \
-                self.args_decode[4:]
-            self.decode_fn = self.lib.pa_decode_quant
+            self.args_decode = self.args_decode[:4] + scales + self.args_decode[4:]
+            self.decode_fn = (self.lib.pa_decode_grouped_quant if group_size > 1
+                              else self.lib.pa_decode_quant)
         if self.multi:
             self.args_decode = (P(self.out.data_ptr()), P(v["q"].data_ptr()),
-                                P(v["k_cache"].data_ptr()), P(v["v_cache"].data_ptr()),
-                                P(self.tables.data_ptr()), int(self.tables.shape[1]),
-                                P(self.ctx.data_ptr()), P(self.query_start.data_ptr()),
-                                wl.max_context_len, wl.num_seqs, wl.num_query_rows,
-                                wl.max_query_len, wl.num_heads, ctypes.c_float(wl.scale),
-                                ctypes.byref(self.desc), self.ps, P(self.ws.data_ptr()),
-                                ctypes.c_size_t(self.ws_bytes), self.sp)
-            self.decode_fn = self.lib.pa_decode_multi
+                                P(v["k_cache"].data_ptr()), P(v["v_cache"].data_ptr())) + \
+                scales + (P(self.tables.data_ptr()), int(self.tables.shape[1]),
+                          P(self.ctx.data_ptr()), P(self.query_start.data_ptr()),
+                          wl.max_context_len, wl.num_seqs, wl.num_query_rows,
+                          wl.max_query_len, wl.num_heads, ctypes.c_float(wl.scale),
+                          ctypes.byref(self.desc), self.ps, P(self.ws.data_ptr()),
+                          ctypes.c_size_t(self.ws_bytes), self.sp)
+            self.decode_fn = self.lib.pa_decode_multi_quant if wl.kv_quant else self.lib.pa_decode_multi
         self.has_copy = wl.copy_pairs.shape[0] > 0
         self.has_append = wl.num_tokens > 0
         self.launches_per_step = (self.num_partitions > 1) + 1 + int(self.has_append) + \
@@ -470,7 +472,19 @@ def e2e_steps(step, steps, warmup):
                                   v["v_cache"], v["k_scale"], v["v_scale"])
         elif wl.num_tokens:
             pa.pa_kv_append(dev["k_new"], dev["v_new"], dev["slots"], v["k_cache"], v["v_cache"])
-        if wl.kv_quant:
+        if wl.kv_quant and step.multi:
+            pa.pa_decode_multi_quant(step.out, dev["q"], v["k_cache"], v["v_cache"], v["k_scale"],
+                                     v["v_scale"], dev["tables"], dev["ctx"], dev["query_start"],
+                                     wl.scale, max_context_len=wl.max_context_len,
+                                     max_query_len=wl.max_query_len, partition_size=step.ps,
+                                     workspace=step.ws)
+        elif wl.kv_quant and step.group_size > 1:
+            pa.pa_decode_grouped_quant(step.out, dev["q"], v["k_cache"], v["v_cache"],
+                                       v["k_scale"], v["v_scale"], dev["tables"], dev["ctx"],
+                                       wl.scale, step.group_size,
+                                       max_context_len=wl.max_context_len,
+                                       partition_size=step.ps, workspace=step.ws)
+        elif wl.kv_quant:
             pa.pa_decode_quant(step.out, dev["q"], v["k_cache"], v["v_cache"], v["k_scale"],
                                v["v_scale"], dev["tables"], dev["ctx"], wl.scale,
                                max_context_len=wl.max_context_len, partition_size=step.ps,
@@ -532,7 +546,21 @@ def oracle_sample(wl, target_s, threads):
         elif sub.num_tokens:
             oracle.kv_append(host["k_new"], host["v_new"], sub.slot_mapping, host["k_cache"],
                              host["v_cache"])
-        if sub.kv_quant:
+        if sub.kv_quant and sub.query_start is not None:
+            # each query token as a row of its own, at its causal end
+            qs = np.asarray(sub.query_start)
+            rows_t, rows_c = [], []
+            for s in range(sub.num_seqs):
+                n = int(qs[s + 1] - qs[s])
+                for j in range(n):
+                    rows_t.append(sub.block_tables[s])
+                    rows_c.append(int(sub.context_lens[s]) - n + j + 1)
+            oracle.decode_quant(host["q"], host["k_cache"], host["v_cache"], host["k_scale"],
+                                host["v_scale"],
+                                np.asarray(rows_t, np.int32).reshape(len(rows_c), -1),
+                                np.asarray(rows_c, np.int32), sub.scale, sub.kv_quant,
+                                num_threads=threads)
+        elif sub.kv_quant:
             oracle.decode_quant(host["q"], host["k_cache"], host["v_cache"], host["k_scale"],
                                 host["v_scale"], sub.block_tables, sub.context_lens, sub.scale,
                                 sub.kv_quant, num_threads=threads)

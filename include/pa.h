@@ -329,6 +329,34 @@ int pa_decode_quant(void* out, const void* q, const void* k_cache, const void* v
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * pa_decode_grouped_quant / pa_decode_multi_quant — pa_decode_grouped and
+ * pa_decode_multi over a quantised cache (the two compositions of the calls
+ * above): arguments as those calls plus k_scale, v_scale after v_cache; the
+ * precision of pa_decode_quant; head_dim 128. Workspace and partitions as
+ * pa_decode_grouped_workspace_size / pa_decode_multi_workspace_size (and the
+ * _num_partitions queries) with the quantised descriptor. Grouped and
+ * multi-token decode are the same computation as pa_decode_quant: a group's
+ * members, and each query token, get exactly the result pa_decode_quant
+ * gives them alone up to rounding (grouping never changes a result beyond
+ * that; within one call it changes no bit).
+ */
+int pa_decode_grouped_quant(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const float* k_scale, const float* v_scale,
+                            const int32_t* block_tables, int32_t block_table_stride,
+                            const int32_t* context_lens, int32_t max_context_len,
+                            int32_t num_seqs, int32_t num_heads, float scale,
+                            const pa_cache_desc* cache, int32_t group_size,
+                            int32_t partition_size, void* workspace, size_t workspace_bytes,
+                            void* stream);
+int pa_decode_multi_quant(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                          int32_t block_table_stride, const int32_t* context_lens,
+                          const int32_t* query_start, int32_t max_context_len, int32_t num_seqs,
+                          int32_t num_query_tokens, int32_t max_query_len, int32_t num_heads,
+                          float scale, const pa_cache_desc* cache, int32_t partition_size,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * pa_set_grouped_consumer — which consumer pa_decode_grouped and pa_decode_multi
  * use for bf16 head_dim 128 with 16..64 query columns (sequences or query
  * tokens x query heads per kv head):

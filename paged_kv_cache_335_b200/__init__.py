@@ -108,6 +108,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         lib.pa_kv_append_quant.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, desc, vp]
         lib.pa_decode_quant.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, f32,
                                         desc, i32, vp, sz, vp]
+        lib.pa_decode_grouped_quant.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32,
+                                                i32, f32, desc, i32, i32, vp, sz, vp]
+        lib.pa_decode_multi_quant.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32,
+                                              i32, i32, i32, f32, desc, i32, vp, sz, vp]
         lib.pa_block_swap.argtypes = [vp, i32, vp, vp, desc, vp, vp, desc, vp]
         lib.pa_sync_check.argtypes = [vp]
         lib.pa_stream_read.argtypes = [vp, sz, vp, i32, vp]
@@ -285,6 +289,76 @@ def pa_decode_quant(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, co
         _dev(context_lens, "context_lens", torch.int32), int(max_context_len), s, h,
         float(scale), ctypes.byref(desc), int(partition_size), ws_ptr, ws_bytes,
         _stream(stream)))
+
+
+def _quant_ws(need, workspace, device):
+    torch = _torch()
+    if not need:
+        return ctypes.c_void_p(0), 0
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    return _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+
+
+def pa_decode_grouped_quant(out, q, k_cache, v_cache, k_scale, v_scale, block_tables,
+                            context_lens, scale: float, group_size: int,
+                            max_context_len: int | None = None, partition_size: int = 0,
+                            workspace=None, stream=None) -> None:
+    """pa_decode_grouped over a quantised pool (pa_decode_quant's arguments plus
+    group_size): sequences [k group_size, (k + 1) group_size) decoded together."""
+    torch = _torch()
+    _same_pool(k_cache, v_cache)
+    desc = cache_desc(k_cache)
+    s, h, d = (int(x) for x in q.shape)
+    if tuple(out.shape) != (s, h, d) or d != desc.head_dim:
+        raise ValueError("q and out must be [num_seqs][num_heads][head_dim]")
+    if q.dtype != torch.bfloat16 or out.dtype != torch.bfloat16:
+        raise TypeError("q and out must be bfloat16")
+    if max_context_len is None:
+        max_context_len = int(context_lens.max().item()) if s else 0
+    need = pa_decode_grouped_workspace_size(s, h, max_context_len, k_cache, int(group_size),
+                                            partition_size)
+    ws_ptr, ws_bytes = _quant_ws(need, workspace, q.device)
+    _check(load_library().pa_decode_grouped_quant(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+        _dev(block_tables, "block_tables", torch.int32), int(block_tables.shape[1]),
+        _dev(context_lens, "context_lens", torch.int32), int(max_context_len), s, h,
+        float(scale), ctypes.byref(desc), int(group_size), int(partition_size), ws_ptr,
+        ws_bytes, _stream(stream)))
+
+
+def pa_decode_multi_quant(out, q, k_cache, v_cache, k_scale, v_scale, block_tables,
+                          context_lens, query_start, scale: float,
+                          max_context_len: int | None = None, max_query_len: int | None = None,
+                          partition_size: int = 0, workspace=None, stream=None) -> None:
+    """pa_decode_multi over a quantised pool (q / out bfloat16 [T][H][D])."""
+    torch = _torch()
+    _same_pool(k_cache, v_cache)
+    desc = cache_desc(k_cache)
+    t, h, d = (int(x) for x in q.shape)
+    s = int(context_lens.shape[0])
+    if tuple(out.shape) != (t, h, d) or d != desc.head_dim:
+        raise ValueError("q and out must be [num_query_tokens][num_heads][head_dim]")
+    if q.dtype != torch.bfloat16 or out.dtype != torch.bfloat16:
+        raise TypeError("q and out must be bfloat16")
+    if block_tables.dim() != 2 or block_tables.shape[0] != s or query_start.shape != (s + 1,):
+        raise ValueError("block_tables [S][stride], context_lens [S], query_start [S + 1]")
+    if max_context_len is None:
+        max_context_len = int(context_lens.max().item()) if s else 0
+    if max_query_len is None:
+        max_query_len = max(1, int((query_start[1:] - query_start[:-1]).max().item())) if s else 1
+    need = pa_decode_multi_workspace_size(s, t, max_query_len, h, max_context_len, k_cache,
+                                          partition_size)
+    ws_ptr, ws_bytes = _quant_ws(need, workspace, q.device)
+    _check(load_library().pa_decode_multi_quant(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(k_scale, "k_scale", torch.float32), _dev(v_scale, "v_scale", torch.float32),
+        _dev(block_tables, "block_tables", torch.int32), int(block_tables.shape[1]),
+        _dev(context_lens, "context_lens", torch.int32),
+        _dev(query_start, "query_start", torch.int32), int(max_context_len), s, t,
+        int(max_query_len), h, float(scale), ctypes.byref(desc), int(partition_size), ws_ptr,
+        ws_bytes, _stream(stream)))
 
 
 def pa_block_swap(src_dst_pairs, src_k, src_v, dst_k, dst_v, stream=None) -> None:

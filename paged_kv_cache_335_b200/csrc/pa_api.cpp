@@ -174,8 +174,8 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
         int gs = max_query_len < 8 ? max_query_len : 8;
         while (gs > 1 && gs * group > 64) --gs;
         if (!pa::grouped_supported(c->dtype, c->head_dim, group, gs))
-            return fail(PA_ERR_UNSUPPORTED, "multi-token decode needs a bf16 cache, head_dim 64 "
-                        "or 128 and num_heads / num_kv_heads <= 64");
+            return fail(PA_ERR_UNSUPPORTED, "multi-token decode needs a bf16 cache at head_dim 64 "
+                        "or 128 or a quantised one at 128, and num_heads / num_kv_heads <= 64");
         group_size = gs;
         plan->q_chunks = (max_query_len + gs - 1) / gs;
         plan->grouped = true;
@@ -213,7 +213,7 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
                 : plan->grouped ? (long)((num_seqs + group_size - 1) / group_size) * c->num_kv_heads
                                 : (long)num_seqs * c->num_kv_heads;
             const long slots =
-                (long)sm_count() * (plan->grouped ? pa::grouped_ctas_per_sm(c->head_dim, group_size, group)
+                (long)sm_count() * (plan->grouped ? pa::grouped_ctas_per_sm(c->dtype, c->head_dim, group_size, group)
                                                   : pa::mma_ctas_per_sm());
             long most = (max_ctx + kMinPartition - 1) / kMinPartition;
             if (most > kMaxPartitions) most = kMaxPartitions;
@@ -366,11 +366,11 @@ static int decode_impl(void* out, const void* q, const void* k_cache, const void
     if ((rc = make_cache_map(&vmap, v_cache, cache)) != PA_OK) return rc;
     cudaError_t e =
         plan.grouped
-            ? pa::launch_decode_grouped(p, cache->head_dim, plan.group_size, kmap, vmap, st)
+            ? pa::launch_decode_grouped(p, cache->dtype, cache->head_dim, plan.group_size, kmap, vmap, st)
             : pa::launch_decode_tma(p, cache->dtype, cache->head_dim, plan.use_mma, kmap, vmap, st);
     if (e != cudaSuccess) return fail_cuda(e, "pa_decode launch");
     t_last_kernel = !plan.grouped ? (plan.use_mma ? PA_KERNEL_MMA : PA_KERNEL_SIMT)
-                    : pa::grouped_is_tcgen05(cache->head_dim, plan.group_size,
+                    : pa::grouped_is_tcgen05(cache->dtype, cache->head_dim, plan.group_size,
                                              num_heads / cache->num_kv_heads)
                         ? PA_KERNEL_GROUPED_TCGEN05
                         : PA_KERNEL_GROUPED;
@@ -560,6 +560,39 @@ int pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v
                        max_context_len, num_seqs, num_heads, scale, cache, 1, partition_size,
                        workspace, workspace_bytes, stream, query_start, num_query_tokens,
                        max_query_len);
+}
+
+int pa_decode_grouped_quant(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const float* k_scale, const float* v_scale,
+                            const int32_t* block_tables, int32_t block_table_stride,
+                            const int32_t* context_lens, int32_t max_context_len,
+                            int32_t num_seqs, int32_t num_heads, float scale,
+                            const pa_cache_desc* cache, int32_t group_size,
+                            int32_t partition_size, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+    if (!k_scale || !v_scale)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_grouped_quant: k_scale and v_scale are required");
+    return decode_impl(out, q, k_cache, v_cache, block_tables, block_table_stride, context_lens,
+                       max_context_len, num_seqs, num_heads, scale, cache, group_size,
+                       partition_size, workspace, workspace_bytes, stream, nullptr, -1, 0, k_scale,
+                       v_scale);
+}
+
+int pa_decode_multi_quant(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                          int32_t block_table_stride, const int32_t* context_lens,
+                          const int32_t* query_start, int32_t max_context_len, int32_t num_seqs,
+                          int32_t num_query_tokens, int32_t max_query_len, int32_t num_heads,
+                          float scale, const pa_cache_desc* cache, int32_t partition_size,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    if (!k_scale || !v_scale)
+        return fail(PA_ERR_INVALID_ARG, "pa_decode_multi_quant: k_scale and v_scale are required");
+    if (num_query_tokens < 0)
+        return fail(PA_ERR_INVALID_ARG, "num_query_tokens %d is negative", num_query_tokens);
+    return decode_impl(out, q, k_cache, v_cache, block_tables, block_table_stride, context_lens,
+                       max_context_len, num_seqs, num_heads, scale, cache, 1, partition_size,
+                       workspace, workspace_bytes, stream, query_start, num_query_tokens,
+                       max_query_len, k_scale, v_scale);
 }
 
 size_t pa_decode_multi_workspace_size(int32_t num_seqs, int32_t num_query_tokens,

@@ -1385,20 +1385,20 @@ __host__ __device__ constexpr int grouped_min_blocks(int d, int cw, int nt) {
 
 // Ring of the grouped kernel: stage = K of the unit's SUB sub-tiles, then
 // their V (kSubBytes each). Every consumer warp reads every stage.
-template <int D, int SUB, int RING>
+template <typename TC, int D, int SUB, int RING>
 struct GroupedRing {
-    using T = __nv_bfloat16;
+    using T = TC;
     static constexpr int kSub = SUB;
-    static constexpr int kBoxes = D * 2 / 128;
-    static constexpr int kBoxElems = 64;
+    static constexpr int kBoxes = D * (int)sizeof(TC) / 128;
+    static constexpr int kBoxElems = 128 / (int)sizeof(TC);
     static constexpr int kSubBytes = kBoxes * kBoxBytes;
     static constexpr int kStageBytes = 2 * SUB * kSubBytes;
     static constexpr int kStages = RING / kStageBytes;
     static constexpr int kRingBytes = kStages * kStageBytes;
     static_assert(kStages >= 2, "grouped ring: at least two stages");
 };
-template <int D, int CW, int NT>
-using GroupedGeom = GroupedRing<D, grouped_sub(CW, NT), grouped_ring_bytes(CW, NT)>;
+template <int D, int CW, int NT, typename TC = __nv_bfloat16>
+using GroupedGeom = GroupedRing<TC, D, grouped_sub(CW, NT), grouped_ring_bytes(CW, NT)>;
 
 // Walk over a grouped CTA's items, u = blockIdx.x + k * gridDim.x, item u =
 // (partition u % P, kv head, group u / (P Hkv)). Lane l holds the context
@@ -1776,7 +1776,7 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&a)[4]) {
 // has seen no valid token keeps max -inf and weight 0. Leaves the P^T
 // B-fragments of sub-tile s in pb0[s] / pb1[s] and returns the largest valid
 // count of the warp's columns (V rows from there on must be zeroed).
-template <int D, int NT, int SUB>
+template <int D, int NT, int SUB, bool kF16 = false>
 __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], const int (&nva)[NT],
                                                 const int (&nvb)[NT], float scale_log2, int r,
                                                 float (&acc)[NT][D / 16][4], float (&ma)[NT],
@@ -1857,11 +1857,14 @@ __device__ __forceinline__ int softmax_update_n(const float (&sc)[SUB][NT][4], c
         float suma = 0.f, sumb = 0.f;
 #pragma unroll
         for (int s = 0; s < SUB; ++s) {
-            const uint32_t x0 = pack_bf16x2(wt(sv[s][j][0], ba), wt(sv[s][j][1], bb));
-            const uint32_t x1 = pack_bf16x2(wt(sv[s][j][2], ba), wt(sv[s][j][3], bb));
+            // weights as the PV operand type: bf16, or f16 beside codes
+            const uint32_t x0 = kF16 ? pack_f16x2(wt(sv[s][j][0], ba), wt(sv[s][j][1], bb))
+                                     : pack_bf16x2(wt(sv[s][j][0], ba), wt(sv[s][j][1], bb));
+            const uint32_t x1 = kF16 ? pack_f16x2(wt(sv[s][j][2], ba), wt(sv[s][j][3], bb))
+                                     : pack_bf16x2(wt(sv[s][j][2], ba), wt(sv[s][j][3], bb));
             if (!kMmaSum) {
-                suma += bf16_lo(x0) + bf16_lo(x1);
-                sumb += bf16_hi(x0) + bf16_hi(x1);
+                suma += kF16 ? f16_lo(x0) + f16_lo(x1) : bf16_lo(x0) + bf16_lo(x1);
+                sumb += kF16 ? f16_hi(x0) + f16_hi(x1) : bf16_hi(x0) + bf16_hi(x1);
             }
             pb0[s][j] = movmatrix_trans(x0);  // P^T rows (tokens) 16s + 2c, 2c+1; column r
             pb1[s][j] = movmatrix_trans(x1);  // tokens 16s + 2c+8, 2c+9
@@ -1947,19 +1950,72 @@ __device__ __forceinline__ void pv_ldsm(uint32_t vb, int sub_bytes, int lane, in
     }
 }
 
+// O^T += V^T . P^T over the unit's SUB sub-tiles of codes (f16 MMAs; V^T
+// fragments built from 16-byte chunks as in codes_softmax_pv: m-tile t rows r
+// and r + 8 are head_dim 16 r + 2t and + 1). Tokens at or past nvmax are
+// zeroed (a zero code is the value 0); the stage is released once the last
+// chunks are in registers.
+template <typename TC, int NT, int SUB>
+__device__ __forceinline__ void pv_codes(uint32_t vb, int sub_bytes, int lane, int nvmax, int r,
+                                         int c, const uint32_t (&pb0)[SUB][NT],
+                                         const uint32_t (&pb1)[SUB][NT], float (&acc)[NT][8][4],
+                                         float (&ls)[NT][4], uint32_t release) {
+    const int nsub = max(1, min(SUB, (nvmax + 15) >> 4));
+#pragma unroll
+    for (int s = 0; s < SUB; ++s) {
+        if (s >= nsub) break;
+        uint4 vr[4];
+        codes_load_v(vb + s * sub_bytes, r, c, vr);
+        if (s == nsub - 1) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(release);
+        }
+        const int k0 = 16 * s;
+        if (k0 + 16 > nvmax) {
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            if (k0 + 2 * c >= nvmax) vr[0] = z;
+            if (k0 + 2 * c + 1 >= nvmax) vr[1] = z;
+            if (k0 + 2 * c + 8 >= nvmax) vr[2] = z;
+            if (k0 + 2 * c + 9 >= nvmax) vr[3] = z;
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const uint32_t va = code_word<TC>(word(vr[0], w)), vbw = code_word<TC>(word(vr[1], w));
+            const uint32_t vc = code_word<TC>(word(vr[2], w)), vd = code_word<TC>(word(vr[3], w));
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t sel = h ? 0x7362u : 0x5140u;
+                uint32_t a0, a1, a2, a3;
+                code_pairs_f16<TC>(__byte_perm(va, vbw, sel), a0, a1);
+                code_pairs_f16<TC>(__byte_perm(vc, vd, sel), a2, a3);
+#pragma unroll
+                for (int j = 0; j < NT; ++j)
+                    mma_16816_f16(acc[j][2 * w + h], a0, a1, a2, a3, pb0[s][j], pb1[s][j]);
+            }
+        }
+        if (PA_GROUPED_MMA_SUM) {
+            constexpr uint32_t kOnes = 0x3C003C00u;  // f16 1.0, 1.0
+#pragma unroll
+            for (int j = 0; j < NT; ++j)
+                mma_16816_f16(ls[j], kOnes, kOnes, kOnes, kOnes, pb0[s][j], pb1[s][j]);
+        }
+    }
+}
+
 // Store one column's result (m, l = its running max and summed weights): bf16
 // output when P == 1, else the normalised partial and (m, l).
-template <int D>
+template <int D, bool kCodes = false>
 __device__ __forceinline__ void grouped_store_col(const DecodeParams& p, int64_t row, int part, int r,
                                                   int c, int e, const float (&acc)[D / 16][4],
-                                                  float m, float l) {
+                                                  float m, float l, float vs = 1.f) {
     constexpr int MT = D / 16;
     const int P = p.num_partitions;
-    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const float inv = (l > 0.f ? 1.f / l : 0.f) * vs;  // vs: V scale of a quantised cache
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
-        // rows r and r + 8 of m-tile t: head_dim 16t + r and 16t + 8 + r
-        const int d0 = 16 * t + r, d1 = d0 + 8;
+        // rows r and r + 8 of m-tile t: head_dim 16t + r and 16t + 8 + r (codes:
+        // 16r + 2t and 16r + 2t + 1)
+        const int d0 = kCodes ? 16 * r + 2 * t : 16 * t + r, d1 = kCodes ? d0 + 1 : d0 + 8;
         if (P == 1) {
             __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + row * D;
             o[d0] = __float2bfloat16_rn(acc[t][e] * inv);
@@ -1977,12 +2033,17 @@ __device__ __forceinline__ void grouped_store_col(const DecodeParams& p, int64_t
     }
 }
 
-template <int D, int CW, int NT>
+template <int D, int CW, int NT, typename TC = __nv_bfloat16>
 __global__ void __launch_bounds__((CW + 1) * 32, grouped_min_blocks(D, CW, NT))
 decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                           const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
                           int num_items, int gs) {
-    using G = GroupedGeom<D, CW, NT>;
+    using G = GroupedGeom<D, CW, NT, TC>;
+    // quantised codes: f16 MMAs on exactly converted codes (as the tensor-core
+    // consumer over codes), q rounded to f16, the K scale in the score scale
+    // and the V scale in the output
+    constexpr bool kCodes = !std::is_same<TC, __nv_bfloat16>::value;
+    static_assert(!kCodes || D == 128, "quantised codes: head_dim 128");
     constexpr int SUB = G::kSub;
     constexpr int KCH = D / 32;
     constexpr int MT = D / 16;
@@ -2069,9 +2130,13 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                 const uint16_t* qrow =
                     static_cast<const uint16_t*>(p.q) +
                     ((int64_t)(it.row0 + m) * p.num_heads + (int64_t)it.kh * group + hd) * D;
+                if constexpr (kCodes) {
+                    load_q_codes(qrow, c, q[j]);
+                } else {
 #pragma unroll
-                for (int jp = 0; jp < KCH; ++jp)
-                    q[j][jp] = ld_v4(qrow + (jp >> 1) * 64 + (2 * c + (jp & 1)) * 8);
+                    for (int jp = 0; jp < KCH; ++jp)
+                        q[j][jp] = ld_v4(qrow + (jp >> 1) * 64 + (2 * c + (jp & 1)) * 8);
+                }
             } else {
 #pragma unroll
                 for (int jp = 0; jp < KCH; ++jp) q[j][jp] = make_uint4(0u, 0u, 0u, 0u);
@@ -2094,6 +2159,8 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         float acc[NT][MT][4], ls[NT][4];
         float ma[NT], mb[NT], la[NT], lb[NT];
+        // score scale in log2 units (a quantised cache's K scale folds in)
+        const float sl = kCodes ? p.scale_log2 * __ldg(p.k_scale + cur.kh) : p.scale_log2;
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
 #pragma unroll
@@ -2118,7 +2185,15 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                     const uint32_t kb = ring.stages + st * G::kStageBytes;
                     float sc[SUB][NT][4];
 #pragma unroll
-                    for (int u = 0; u < SUB; ++u) mma_qk_n<D, NT>(kb + u * G::kSubBytes, q, r, c, sc[u]);
+                    for (int u = 0; u < SUB; ++u) {
+                        if constexpr (kCodes) {
+#pragma unroll
+                            for (int j = 0; j < NT; ++j)
+                                codes_qk<TC>(kb + u * G::kSubBytes, q[j], r, c, sc[u][j]);
+                        } else {
+                            mma_qk_n<D, NT>(kb + u * G::kSubBytes, q, r, c, sc[u]);
+                        }
+                    }
                     int nva[NT], nvb[NT];
 #pragma unroll
                     for (int j = 0; j < NT; ++j) {
@@ -2126,10 +2201,14 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                         nvb[j] = (h & bitb[j]) ? min(kUnitTokens, t1b[j] - tok0) : 0;
                     }
                     uint32_t pb0[SUB][NT], pb1[SUB][NT];
-                    const int nvmax = softmax_update_n<D, NT, SUB>(sc, nva, nvb, p.scale_log2, r, acc, ma,
-                                                                   mb, la, lb, ls, pb0, pb1);
-                    pv_ldsm<D, NT, SUB>(kb + SUB * G::kSubBytes, G::kSubBytes, lane, nvmax, c, pb0, pb1,
-                                        acc, ls, ring.empty + 8 * st);  // releases the stage
+                    const int nvmax = softmax_update_n<D, NT, SUB, kCodes>(sc, nva, nvb, sl, r, acc, ma,
+                                                                           mb, la, lb, ls, pb0, pb1);
+                    if constexpr (kCodes)
+                        pv_codes<TC, NT, SUB>(kb + SUB * G::kSubBytes, G::kSubBytes, lane, nvmax, r, c,
+                                              pb0, pb1, acc, ls, ring.empty + 8 * st);
+                    else
+                        pv_ldsm<D, NT, SUB>(kb + SUB * G::kSubBytes, G::kSubBytes, lane, nvmax, c, pb0,
+                                            pb1, acc, ls, ring.empty + 8 * st);  // releases the stage
                 } else {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(ring.empty + 8 * st);  // stage released
@@ -2162,8 +2241,9 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                 if (m < gs && m < cur.nmem && (P == 1 || t1 > cur.t0)) {
                     const int64_t row =
                         (int64_t)(cur.row0 + m) * p.num_heads + (int64_t)cur.kh * group + hd;
-                    grouped_store_col<D>(p, row, cur.part, r, c, e, acc[j],
-                                         e == 0 ? ma[j] : mb[j], e == 0 ? la[j] : lb[j]);
+                    grouped_store_col<D, kCodes>(p, row, cur.part, r, c, e, acc[j],
+                                                 e == 0 ? ma[j] : mb[j], e == 0 ? la[j] : lb[j],
+                                                 kCodes ? __ldg(p.v_scale + cur.kh) : 1.f);
                 }
             }
         }
@@ -2738,13 +2818,13 @@ cudaError_t launch_umma_grouped(const DecodeParams& p, const CUtensorMap& km,
     return cudaGetLastError();
 }
 
-template <int D, int CW, int NT>
+template <int D, int CW, int NT, typename TC = __nv_bfloat16>
 cudaError_t launch_grouped_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
                              int gs, cudaStream_t stream) {
-    using G = GroupedGeom<D, CW, NT>;
+    using G = GroupedGeom<D, CW, NT, TC>;
     constexpr size_t smem = smem_bytes<G>(G::kStages * 4);
     constexpr int kThreads = (CW + 1) * 32;
-    auto kernel = decode_tma_grouped_kernel<D, CW, NT>;
+    auto kernel = decode_tma_grouped_kernel<D, CW, NT, TC>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -2822,19 +2902,26 @@ static void grouped_shape(int gs, int group, int* cw, int* nt) {
     *cw = (tiles + *nt - 1) / *nt;
 }
 
+// bf16 at head_dim 64 or 128; quantised codes (PA_FP8_E4M3, PA_INT8) at 128.
 bool grouped_supported(int dtype, int head_dim, int group, int gs) {
-    return dtype == 1 && (head_dim == 64 || head_dim == 128) && gs >= 1 && gs <= kMaxGroupSeqs &&
-           group >= 1 && gs * group <= kGroupedMaxCols;
+    const bool shape = (dtype == 1 && (head_dim == 64 || head_dim == 128)) ||
+                       ((dtype == 2 || dtype == 3) && head_dim == 128);
+    return shape && gs >= 1 && gs <= kMaxGroupSeqs && group >= 1 && gs * group <= kGroupedMaxCols;
 }
 
-int grouped_ctas_per_sm(int head_dim, int gs, int group) {
-    if (use_umma(head_dim, gs, group)) return 2;
+// The tcgen05 consumer takes bf16 only.
+bool grouped_is_tcgen05(int dtype, int head_dim, int gs, int group) {
+    return dtype == 1 && use_umma(head_dim, gs, group);
+}
+
+int grouped_ctas_per_sm(int dtype, int head_dim, int gs, int group) {
+    if (grouped_is_tcgen05(dtype, head_dim, gs, group)) return 2;
     int cw = 1, nt = 1;
     grouped_shape(gs, group, &cw, &nt);
     return grouped_min_blocks(head_dim, cw, nt);
 }
 
-template <int D>
+template <int D, typename TC = __nv_bfloat16>
 static cudaError_t launch_grouped_d(const DecodeParams& p, int cw, int nt, int gs,
                                    const CUtensorMap& kmap, const CUtensorMap& vmap,
                                    cudaStream_t stream) {
@@ -2842,40 +2929,42 @@ static cudaError_t launch_grouped_d(const DecodeParams& p, int cw, int nt, int g
                   "one-tile warps: 1 .. 4");
     if (nt == 1) {
         switch (cw) {
-            case 1: return launch_grouped_t<D, 1, 1>(p, kmap, vmap, gs, stream);
+            case 1: return launch_grouped_t<D, 1, 1, TC>(p, kmap, vmap, gs, stream);
 #if PA_GROUPED_ONE_TILE_WARPS >= 2
-            case 2: return launch_grouped_t<D, 2, 1>(p, kmap, vmap, gs, stream);
+            case 2: return launch_grouped_t<D, 2, 1, TC>(p, kmap, vmap, gs, stream);
 #endif
 #if PA_GROUPED_ONE_TILE_WARPS >= 3
-            case 3: return launch_grouped_t<D, 3, 1>(p, kmap, vmap, gs, stream);
+            case 3: return launch_grouped_t<D, 3, 1, TC>(p, kmap, vmap, gs, stream);
 #endif
 #if PA_GROUPED_ONE_TILE_WARPS >= 4
-            case 4: return launch_grouped_t<D, 4, 1>(p, kmap, vmap, gs, stream);
+            case 4: return launch_grouped_t<D, 4, 1, TC>(p, kmap, vmap, gs, stream);
 #endif
             default: return cudaErrorInvalidValue;
         }
     }
     switch (cw) {
-        case 1: return launch_grouped_t<D, 1, 2>(p, kmap, vmap, gs, stream);
-        case 2: return launch_grouped_t<D, 2, 2>(p, kmap, vmap, gs, stream);
-        case 3: return launch_grouped_t<D, 3, 2>(p, kmap, vmap, gs, stream);
-        case 4: return launch_grouped_t<D, 4, 2>(p, kmap, vmap, gs, stream);
+        case 1: return launch_grouped_t<D, 1, 2, TC>(p, kmap, vmap, gs, stream);
+        case 2: return launch_grouped_t<D, 2, 2, TC>(p, kmap, vmap, gs, stream);
+        case 3: return launch_grouped_t<D, 3, 2, TC>(p, kmap, vmap, gs, stream);
+        case 4: return launch_grouped_t<D, 4, 2, TC>(p, kmap, vmap, gs, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
-cudaError_t launch_decode_grouped(const DecodeParams& p, int head_dim, int gs,
+cudaError_t launch_decode_grouped(const DecodeParams& p, int dtype, int head_dim, int gs,
                                   const CUtensorMap& kmap, const CUtensorMap& vmap,
                                   cudaStream_t stream) {
-    if (use_umma(head_dim, gs, p.num_heads / p.num_kv_heads))
+    if (grouped_is_tcgen05(dtype, head_dim, gs, p.num_heads / p.num_kv_heads))
         return launch_umma_grouped(p, kmap, vmap, gs, stream);
     int cw = 1, nt = 1;
     grouped_shape(gs, p.num_heads / p.num_kv_heads, &cw, &nt);
+    if (dtype == 2) return launch_grouped_d<128, E4M3Code>(p, cw, nt, gs, kmap, vmap, stream);
+    if (dtype == 3) return launch_grouped_d<128, Int8Code>(p, cw, nt, gs, kmap, vmap, stream);
     return head_dim == 64 ? launch_grouped_d<64>(p, cw, nt, gs, kmap, vmap, stream)
                           : launch_grouped_d<128>(p, cw, nt, gs, kmap, vmap, stream);
 }
 
-bool grouped_is_tcgen05(int head_dim, int gs, int group) { return use_umma(head_dim, gs, group); }
+
 
 int set_grouped_consumer(int consumer) {
     const int prev = g_grouped_consumer;

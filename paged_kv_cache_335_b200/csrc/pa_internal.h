@@ -100,11 +100,11 @@ bool grouped_supported(int dtype, int head_dim, int group, int gs);
 // Select the grouped consumer (PA_GROUPED_MMA_SYNC / PA_GROUPED_TCGEN05);
 // returns the previous one.
 int set_grouped_consumer(int consumer);
-// Whether the grouped kernel for (head_dim, gs, H / Hkv) is the tcgen05 consumer.
-bool grouped_is_tcgen05(int head_dim, int gs, int group);
-// CTA slots per SM of the grouped kernel chosen for (head_dim, gs, H / Hkv).
-int grouped_ctas_per_sm(int head_dim, int gs, int group);
-cudaError_t launch_decode_grouped(const DecodeParams& p, int head_dim, int gs,
+// Whether the grouped kernel for (dtype, head_dim, gs, H / Hkv) is the tcgen05 consumer.
+bool grouped_is_tcgen05(int dtype, int head_dim, int gs, int group);
+// CTA slots per SM of the grouped kernel chosen for (dtype, head_dim, gs, H / Hkv).
+int grouped_ctas_per_sm(int dtype, int head_dim, int gs, int group);
+cudaError_t launch_decode_grouped(const DecodeParams& p, int dtype, int head_dim, int gs,
                                   const CUtensorMap& kmap, const CUtensorMap& vmap,
                                   cudaStream_t stream);
 // Log-sum-exp merge of the P partial results into out.
