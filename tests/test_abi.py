@@ -140,6 +140,35 @@ def test_multi_query_policy_and_arguments(lib):
     assert rc == pa.PA_ERR_INVALID_ARG and b"query_start" in lib.pa_get_last_error()
 
 
+def test_quantised_grouped_and_multi_arguments(lib):
+    """pa_decode_grouped_quant / pa_decode_multi_quant: the scales are required,
+    the pool must be quantised (and at head_dim 128), the group size and the
+    multi-token arguments are checked as on the bf16 calls."""
+    p = ctypes.c_void_p(256)
+    fp8 = _desc(num_kv_heads=2, dtype=pa.PA_FP8_E4M3)
+    bf16 = _desc(num_kv_heads=2)
+    g = lib.pa_decode_grouped_quant
+
+    def grouped(desc, ks=p, vs=p, gs=4):
+        return g(p, p, p, p, ks, vs, p, 8, p, 100, 4, 16, ctypes.c_float(0.1), ctypes.byref(desc),
+                 gs, -1, None, 0, None)
+    assert grouped(fp8, ks=None) == pa.PA_ERR_INVALID_ARG
+    assert grouped(bf16) == pa.PA_ERR_DTYPE
+    assert grouped(_desc(num_kv_heads=2, dtype=pa.PA_INT8, head_dim=64)) == pa.PA_ERR_UNSUPPORTED
+    assert grouped(fp8, gs=9) == pa.PA_ERR_INVALID_ARG
+    m = lib.pa_decode_multi_quant
+    rc = m(p, p, p, p, p, p, p, 8, p, None, 100, 2, 4, 2, 16, ctypes.c_float(0.1),
+           ctypes.byref(fp8), -1, None, 0, None)
+    assert rc == pa.PA_ERR_INVALID_ARG and b"query_start" in lib.pa_get_last_error()
+    rc = m(p, p, p, p, None, p, p, 8, p, p, 100, 2, 4, 2, 16, ctypes.c_float(0.1),
+           ctypes.byref(fp8), -1, None, 0, None)
+    assert rc == pa.PA_ERR_INVALID_ARG
+    # the grouped and multi-token plans accept a quantised pool at head_dim 128
+    d70 = _desc(num_kv_heads=8, dtype=pa.PA_FP8_E4M3)
+    assert lib.pa_decode_grouped_num_partitions(128, 64, 2303, ctypes.byref(d70), 4, 0) == 1
+    assert lib.pa_decode_multi_num_partitions(8, 32, 4, 64, 32768, ctypes.byref(d70), 512) == 64
+
+
 def test_grouped_consumer_selector(lib):
     assert lib.pa_set_grouped_consumer(pa.PA_GROUPED_TCGEN05) == pa.PA_GROUPED_MMA_SYNC
     assert lib.pa_set_grouped_consumer(pa.PA_GROUPED_MMA_SYNC) == pa.PA_GROUPED_TCGEN05
