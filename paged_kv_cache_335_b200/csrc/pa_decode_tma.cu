@@ -2334,10 +2334,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 // ---------------------------------------------------------------------------
 // Grouped and multi-token decode on the 5th-generation tensor cores
 // (head_dim 128, bf16, 16..64 query columns; opt-in, see grouped_consumer).
-// Same work items, producer and ring as decode_tma_grouped_kernel (one unit
-// per distinct block of a 16-token sub-tile, mask + sub-tile index in a
-// per-stage header, plus the unit's largest valid token count); the consumer
-// is split by role:
+// Same work items as decode_tma_grouped_kernel, with one-sub-tile units: one
+// ring position per distinct block of a 16-token sub-tile, mask + sub-tile
+// index in a per-stage header, plus the unit's largest valid token count
+// (issue_units); the consumer is split by role:
 //   warp 3, lane 0, issues per unit S = Q . K^T (M = 128 query rows, N = 16
 //     tokens, K = 128; Q and the K tile from shared memory, S in TMEM) and
 //     O += P . V (A = P in TMEM, B = the V tile read MN-major from shared
@@ -2357,7 +2357,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 // which blocks it shares. V rows past every member's context are zeroed in
 // shared memory before the PV product reads them.
 // Measured against the mma.sync consumer (4-beam GQA CoW, 4-token verification
-// over 32K contexts): slower, 172 vs 106 and 444 vs 291 us. Per CTA one softmax
+// over 32K contexts): slower, 172 vs 90 and 452 vs 212 us. Per CTA one softmax
 // warp walks the units one after the other, and with at most 2 CTAs per SM (TMEM,
 // shared memory) too few warps hide the TMEM / barrier round trips of a 16 x 32
 // contraction; batching 4 units per softmax pass made it slower still.
