@@ -226,3 +226,22 @@ def test_python_binding_refuses_cpu_tensors():
     kc = torch.zeros((4, 1, 16, 64))
     with pytest.raises(ValueError, match="CUDA"):
         pa.pa_block_copy(torch.zeros((1, 2), dtype=torch.int64), kc, kc.clone())
+
+
+def test_python_binding_quantised_calls_refuse_cpu_tensors():
+    """The quantised grouped / multi-token bindings marshal device pointers only:
+    host tensors are refused before anything reaches the library."""
+    import torch
+    kc = torch.zeros((8, 2, 16, 128), dtype=torch.float8_e4m3fn)
+    q = torch.zeros((4, 16, 128), dtype=torch.bfloat16)
+    scales = torch.ones(2)
+    tables = torch.zeros((4, 2), dtype=torch.int32)
+    ctx = torch.full((4,), 20, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        pa.pa_decode_grouped_quant(torch.empty_like(q), q, kc, kc.clone(), scales, scales, tables,
+                                   ctx, 0.1, 2, max_context_len=20, partition_size=-1)
+    qs = torch.tensor([0, 1, 2, 3, 4], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        pa.pa_decode_multi_quant(torch.empty_like(q), q, kc, kc.clone(), scales, scales, tables,
+                                 ctx, qs, 0.1, max_context_len=20, max_query_len=1,
+                                 partition_size=-1)
