@@ -444,6 +444,43 @@ def swap_bandwidth(device, blocks=1024, reps=5):
     return res
 
 
+def measure_config(w2, device, ps, gs, consumer, args, flush_buf, hbm_peak, read_gbs):
+    """Decode figures of one extra configuration (same step timing as the headline)."""
+    import paged_kv_cache_335_b200 as pa
+    prev = None
+    if consumer == "tcgen05":
+        prev = pa.pa_set_grouped_consumer(pa.PA_GROUPED_TCGEN05)
+    try:
+        st = Step(w2, device, partition_size=ps, group_size=gs)
+        try:
+            r2 = time_steps(st, min(args.steps, 50), 3, flush_buf if needs_flush(w2) else None)
+            sm = statistics.median(r2["step_ms"])
+            dm = statistics.median(r2["decode_ms"])
+            gbs = w2.decode_bytes() / (dm / 1e3) / 1e9
+            return {
+                "decode_gbs": round(gbs, 1),
+                "decode_frac_of_peak": round(gbs / hbm_peak, 4),
+                "decode_frac_of_datasheet": round(gbs / DATASHEET_HBM_GBS, 4),
+                "decode_frac_of_stream_read": round(gbs / read_gbs, 4) if read_gbs else None,
+                "decode_us": round(dm * 1e3, 2),
+                "step_us": round(sm * 1e3, 2),
+                "moves_us": round(statistics.median(r2["moves_ms"]) * 1e3, 2),
+                "seq_steps_per_s": round(w2.num_seqs / (sm / 1e3), 1),
+                "partitions": st.num_partitions,
+                "partition_size": "library policy" if st.ps == 0 else st.ps,
+                "group_size": gs,
+                "grouped_consumer": consumer or args.grouped_consumer,
+                "decode_bytes": w2.decode_bytes(),
+                "unique_kv_bytes": w2.unique_kv_bytes() if w2.name.startswith("cow") else None,
+            }
+        finally:
+            st.release()
+            del st
+    finally:
+        if prev is not None:
+            pa.pa_set_grouped_consumer(prev)
+
+
 def e2e_steps(step, steps, warmup):
     """The same step through the Python binding of the C ABI with inputs in
     pinned HOST memory: H2D of the step's inputs and D2H of the output are
@@ -732,36 +769,12 @@ def main():
     per_config = {}
     if world == 1 and not args.no_extra_configs:
         for label, name, ps, gs, consumer in EXTRA_CONFIGS:
-            w2 = W.make(name)
-            prev = None
-            if consumer == "tcgen05":
-                prev = pa.pa_set_grouped_consumer(pa.PA_GROUPED_TCGEN05)
-            st = Step(w2, device, partition_size=ps, group_size=gs)
-            r2 = time_steps(st, min(args.steps, 50), 3, flush_buf if needs_flush(w2) else None)
-            sm = statistics.median(r2["step_ms"])
-            dm = statistics.median(r2["decode_ms"])
-            per_config[label] = {
-                "decode_gbs": round(w2.decode_bytes() / (dm / 1e3) / 1e9, 1),
-                "decode_frac_of_peak": round(w2.decode_bytes() / (dm / 1e3) / 1e9 / hbm_peak, 4),
-                "decode_frac_of_datasheet": round(
-                    w2.decode_bytes() / (dm / 1e3) / 1e9 / DATASHEET_HBM_GBS, 4),
-                "decode_frac_of_stream_read": round(
-                    w2.decode_bytes() / (dm / 1e3) / 1e9 / read_gbs, 4) if read_gbs else None,
-                "decode_us": round(dm * 1e3, 2),
-                "step_us": round(sm * 1e3, 2),
-                "moves_us": round(statistics.median(r2["moves_ms"]) * 1e3, 2),
-                "seq_steps_per_s": round(w2.num_seqs / (sm / 1e3), 1),
-                "partitions": st.num_partitions,
-                "partition_size": "library policy" if st.ps == 0 else st.ps,
-                "group_size": gs,
-                "grouped_consumer": consumer or args.grouped_consumer,
-                "decode_bytes": w2.decode_bytes(),
-                "unique_kv_bytes": w2.unique_kv_bytes() if name.startswith("cow") else None,
-            }
-            st.release()
-            del st
-            if prev is not None:
-                pa.pa_set_grouped_consumer(prev)
+            try:
+                per_config[label] = measure_config(W.make(name), device, ps, gs, consumer, args,
+                                                   flush_buf, hbm_peak, read_gbs)
+            except Exception as e:  # one configuration failing must not lose the others
+                print(f"bench: configuration {label} failed: {e!r}", file=sys.stderr)
+                per_config[label] = {"error": repr(e)[:300]}
             torch.cuda.empty_cache()
         per_config["swap_llama13b_blocks"] = swap_bandwidth(device)
 
