@@ -123,3 +123,24 @@ def test_poison_covers_unfilled_and_unowned():
         slot = int(wl.slot_mapping[s])
         b, o = divmod(slot, wl.block_size)
         assert any((blocks == b) & (offs == o))
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+def test_quantised_values_stay_below_four(fmt):
+    """The quantised pools' values (code value x per-head scale) stay below 4 in
+    magnitude, the range in which bf16 rounding of an output stays inside the
+    1e-2 bar; poisoned slots are the NaN code (fp8) or -128 (int8)."""
+    import numpy as np
+    import oracle
+    wl = W.quantized(W.cow_beam4(num_prompts=2, prompt_len=120, max_suffix=20, num_heads=8,
+                                 num_kv_heads=2, head_dim=128), fmt)
+    vals = W.make_values(wl, "cpu", poison=False)
+    for cache, scale in (("k_cache", "k_scale"), ("v_cache", "v_scale")):
+        codes = W.to_numpy(vals[cache])
+        v = oracle.code_values(codes, fmt)
+        s = vals[scale].numpy().astype(np.float64)
+        assert np.all(np.isfinite(v))
+        assert float((np.abs(v) * s[None, :, None, None]).max()) < 4.0
+    poisoned = W.to_numpy(W.make_values(wl, "cpu", poison=True)["k_cache"])
+    bad = 0x7F if fmt == "fp8" else 0x80
+    assert (poisoned.view(np.uint8) == bad).any()
