@@ -444,8 +444,11 @@ int pa_block_swap(const int64_t* src_dst_pairs, int32_t num_pairs,
  * PA_NOALLOC_SCRATCH_BYTES inside the library. It allocates nothing.
  *
  * The first call on a device looks up that buffer's device address
- * (cudaGetSymbolAddress) with the device current; make that first call before
- * any stream capture. A call whose workspace need (pa_decode_workspace_size
+ * (cudaGetSymbolAddress) with the device current and keeps it with the CUDA
+ * context it belongs to; a later call that finds another context current (a
+ * cudaDeviceReset makes the runtime create a new one, and the buffer may then
+ * move) looks it up again. Make the first call on a device, and the first
+ * after a reset, before any stream capture. A call whose workspace need (pa_decode_workspace_size
  * with the same arguments) exceeds PA_NOALLOC_SCRATCH_BYTES returns
  * PA_ERR_WORKSPACE and enqueues nothing. All calls on one device share the
  * buffer, which keeps the last call's contents: calls whose kernels may overlap

@@ -173,9 +173,19 @@ def _dtype_code(t) -> int:
                     "(FP8 E4M3 codes) or int8 (int8 codes)")
 
 
+def _on_current_device(t, name: str):
+    """The library launches on the current device and stream: a tensor of another
+    GPU would hand its kernels a pointer they cannot use."""
+    cur = _torch().cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device}, but the current CUDA device is cuda:{cur}; "
+                         "call under torch.cuda.device(...) of the tensors' device")
+
+
 def _dev(t, name: str, dtype=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    _on_current_device(t, name)
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
@@ -187,6 +197,8 @@ def _addressable(t, name: str):
     """A CUDA tensor or a pinned host tensor (which the device addresses directly)."""
     if not (t.is_cuda or t.is_pinned()):
         raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    if t.is_cuda:
+        _on_current_device(t, name)
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return ctypes.c_void_p(t.data_ptr())

@@ -11,11 +11,17 @@
 // holds until the process exits. Nothing here allocates.
 //
 // On the host, `s_scratch` names a host-side stand-in, not device memory, so
-// its device address is looked up once per device with cudaGetSymbolAddress,
-// with that device current, and cached. Every call shares the one buffer per
-// device: calls whose kernels overlap on the GPU (different streams, no
-// ordering between them) race on it. The buffer needs no clearing: each call
-// writes every partial result before its merge reads it.
+// its device address is looked up with cudaGetSymbolAddress, with the device
+// current, and cached per device together with the CUDA context it was looked
+// up in. A call that finds another context current on the device (after a
+// cudaDeviceReset, the runtime creates a new primary context and loads the
+// library's device code again, so the buffer may move) looks it up again; that
+// call, like the first one on a device, should come before any stream capture.
+// Every call shares the one buffer per device: calls whose kernels overlap on
+// the GPU (different streams, no ordering between them) race on it. The buffer
+// needs no clearing: each call writes every partial result before its merge
+// reads it.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -28,25 +34,54 @@ static __device__ __align__(256) unsigned char s_scratch[PA_NOALLOC_SCRATCH_BYTE
 namespace {
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices];
+struct ScratchEntry {
+    CUcontext ctx;  // context current when the address was looked up
+    void* addr;
+};
+ScratchEntry g_scratch[kMaxDevices];
 std::mutex g_scratch_mutex;
 
-// Device address of s_scratch on the current device; the first call on a
-// device looks it up.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// cuCtxGetCurrent from the driver (the library links only the runtime).
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(f);
+    });
+    return fn;
+}
+
+// Device address of s_scratch on the current device: looked up on the first
+// call on a device and again whenever the current context is not the one the
+// cached address belongs to.
 cudaError_t scratch_address(void** addr) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (!get_ctx) return cudaErrorNotSupported;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[dev]) {
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    ScratchEntry& ent = g_scratch[dev];
+    if (!ent.addr || !ctx || ctx != ent.ctx) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, s_scratch);
+        e = cudaGetSymbolAddress(&p, s_scratch);  // binds the device's primary context
         if (e != cudaSuccess) return e;
         if (!p) return cudaErrorInvalidSymbol;
-        g_scratch_addr[dev] = p;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+        ent.ctx = ctx;
+        ent.addr = p;
     }
-    *addr = g_scratch_addr[dev];
+    *addr = ent.addr;
     return cudaSuccess;
 }
 

@@ -126,15 +126,9 @@ def dev_bits_equal(a: torch.Tensor, b: torch.Tensor) -> bool:
     return bool(torch.equal(a.contiguous().view(view), b.contiguous().view(view)))
 
 
-def sample_seqs(wl, n, seed=0):
-    """Sequences for sampled parity at full size: the longest, the shortest and
-    a seeded random choice of the rest."""
-    rng = np.random.default_rng(seed)
-    order = np.argsort(wl.context_lens)
-    pick = {int(order[0]), int(order[-1])}
-    rest = [i for i in range(wl.num_seqs) if i not in pick]
-    pick.update(int(x) for x in rng.choice(rest, size=min(n - 2, len(rest)), replace=False))
-    return sorted(pick)
+def oracle_all(wl, vals_after):
+    """Oracle decode of every sequence, read from the post-step device pool."""
+    return oracle_sampled(wl, vals_after, range(wl.num_seqs))
 
 
 def oracle_sampled(wl, vals_after, seq_ids):

@@ -245,3 +245,28 @@ def test_python_binding_quantised_calls_refuse_cpu_tensors():
         pa.pa_decode_multi_quant(torch.empty_like(q), q, kc, kc.clone(), scales, scales, tables,
                                  ctx, qs, 0.1, max_context_len=20, max_query_len=1,
                                  partition_size=-1)
+
+
+def test_python_binding_refuses_a_tensor_of_another_device(monkeypatch):
+    """The library launches on the current device: a tensor living on another
+    GPU is refused in the binding instead of reaching a kernel as a foreign
+    pointer (a stand-in tensor object plays the CUDA tensor; no GPU needed)."""
+    import types
+
+    import torch
+
+    class OtherGpuTensor:
+        is_cuda = True
+        device = types.SimpleNamespace(index=1, type="cuda")
+
+        def is_contiguous(self):
+            return True
+
+        def data_ptr(self):
+            return 256
+
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(ValueError, match="current CUDA device is cuda:0"):
+        pa._dev(OtherGpuTensor(), "q")
+    with pytest.raises(ValueError, match="current CUDA device"):
+        pa._addressable(OtherGpuTensor(), "dst_k")

@@ -17,7 +17,7 @@ from tests.test_gpu_grouped import (test_cow_small_full_pool,  # noqa: F401
                                     test_shared_equals_private_bitwise)
 from tests.test_gpu_multi import (test_parity_shape_sweep,  # noqa: F401
                                   test_token_result_independent_of_the_other_tokens,
-                                  test_verification_full_size_sampled)
+                                  test_verification_full_size)
 from tests.test_gpu_timeout import test_skipped_load_times_out_then_recovers  # noqa: F401
 
 pytestmark = pytest.mark.gpu
