@@ -113,6 +113,16 @@ def weak_scaling_value(step_bytes: int, steps: int, world: int, max_total_ms: fl
     return world * step_bytes * steps / (max_total_ms / 1e3) / 1e9
 
 
+def pct(xs, scale=1.0, nd=2):
+    """p10 / p50 / p90 of a list of timings (same unit as xs x scale)."""
+    ys = sorted(x * scale for x in xs)
+    def q(f):
+        k = (len(ys) - 1) * f
+        lo, hi = int(math.floor(k)), int(math.ceil(k))
+        return ys[lo] + (ys[hi] - ys[lo]) * (k - lo)
+    return {"p10": round(q(0.1), nd), "p50": round(q(0.5), nd), "p90": round(q(0.9), nd)}
+
+
 def stream_read_gbs(device, reps=10):
     """Read bandwidth of the library's read-only streaming kernel over 4 GiB."""
     import torch
@@ -121,7 +131,7 @@ def stream_read_gbs(device, reps=10):
     lib = pa.load_library()
     buf = torch.empty(STREAM_BYTES, dtype=torch.uint8, device=device)
     sms = torch.cuda.get_device_properties(device).multi_processor_count
-    ctas = sms * 4
+    ctas = sms * 2                      # two 96 KiB rings per SM
     part = torch.empty(ctas, dtype=torch.int32, device=device)
     st = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
     args = (ctypes.c_void_p(buf.data_ptr()), ctypes.c_size_t(STREAM_BYTES),
@@ -463,6 +473,7 @@ def measure_config(w2, device, ps, gs, consumer, args, flush_buf, hbm_peak, read
                 "decode_frac_of_datasheet": round(gbs / DATASHEET_HBM_GBS, 4),
                 "decode_frac_of_stream_read": round(gbs / read_gbs, 4) if read_gbs else None,
                 "decode_us": round(dm * 1e3, 2),
+                "decode_us_pct": pct(r2["decode_ms"], 1e3),
                 "step_us": round(sm * 1e3, 2),
                 "moves_us": round(statistics.median(r2["moves_ms"]) * 1e3, 2),
                 "seq_steps_per_s": round(w2.num_seqs / (sm / 1e3), 1),
@@ -761,6 +772,7 @@ def main():
     e2e_ms = dist_max(e2e_ms, device)
     e2e_value = weak_scaling_value(step.step_bytes, args.steps, world, e2e_ms)
     launches = step.launches_per_step * args.steps
+    step_ps, step_np = step.ps, step.num_partitions
     step.release()
     del step
     torch.cuda.empty_cache()
@@ -782,8 +794,11 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = host_cores()
         gbs, secs, desc, _ = oracle_sample(wl, args.cpu_seconds, threads)
+        gbs1, secs1, desc1, _ = oracle_sample(wl, args.cpu_seconds / 2, 1)
         cpu = {"value": gbs, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": desc, "seconds": round(secs, 2)}
+               "sample": desc, "seconds": round(secs, 2),
+               "single_thread": {"value": gbs1, "unit": UNIT, "cores": 1, "sample": desc1,
+                                 "seconds": round(secs1, 2)}}
 
     if rank == 0:
         line = {
@@ -791,8 +806,12 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": wl.dtype, "data": "synthetic (seeded N(0,1) values, seeded shapes)",
-            "config": {**config_dict(wl, flush is not None), "group_size": args.group_size,
-                       "grouped_consumer": args.grouped_consumer},
+            "config": config_dict(wl, flush is not None),
+            "launch": {"group_size": args.group_size, "grouped_consumer": args.grouped_consumer,
+                       "partition_size": "library policy" if step_ps == 0 else step_ps,
+                       "partitions": step_np},
+            "step_us_pct": pct(res["step_ms"], 1e3),
+            "decode_us_pct": pct(res["decode_ms"], 1e3),
             "seq_steps_per_s": round(world * wl.num_seqs / (ms_per_step / 1e3), 1),
             "frac_of_hbm_peak": round(value / world / hbm_peak, 4),
             "reference_bandwidths_gbs": {
@@ -801,6 +820,7 @@ def main():
             "decode_frac_of_stream_read": round(dec_gbs / read_gbs, 4) if read_gbs else None,
             "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": hbm_peak,
                          "unit": "GB/s", "frac": round(dec_gbs / hbm_peak, 4),
+                         "frac_of_datasheet": round(dec_gbs / DATASHEET_HBM_GBS, 4),
                          "traffic": traffic,
                          "kernel": kernel_name,
                          "algorithmic_bytes_per_launch": wl.decode_bytes(),

@@ -4,11 +4,14 @@
  * bandwidth this GPU sustains, the reference a read-dominated kernel is
  * compared with next to the copy (read + write) bandwidth.
  *
- * pa_stream_read — read every byte of `src` once (16-byte loads, `num_ctas`
- * CTAs of 512 threads, grid-stride) and write one 32-bit checksum per CTA to
- * `partial` (device, num_ctas entries). `bytes` must be a multiple of 16 and
- * `src` 16-byte aligned. Asynchronous on `stream` (a cudaStream_t, NULL = the
- * default stream). Returns 0, -1 on bad arguments, -5 if the launch failed.
+ * pa_stream_read — read every byte of `src` once and write one 32-bit checksum
+ * per CTA to `partial` (device, num_ctas entries). Each of the `num_ctas` CTAs
+ * (two fit on an SM) streams 16 KiB chunks c, c + num_ctas, ... through a
+ * 6-stage shared-memory ring with bulk asynchronous copies (cp.async.bulk, no
+ * multicast), the way the decode kernels read the cache. `bytes` must be a
+ * multiple of 16 and `src` 16-byte aligned. Asynchronous on `stream` (a
+ * cudaStream_t, NULL = the default stream). Returns 0, -1 on bad arguments,
+ * -5 if the launch failed.
  */
 #ifndef PA_STREAM_H
 #define PA_STREAM_H

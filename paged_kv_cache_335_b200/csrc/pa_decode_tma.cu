@@ -244,6 +244,24 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// q on the paths over codes is rounded to f16 (the MMA operand type beside the
+// codes). To keep that rounding exact whatever q's magnitude, q is scaled by
+// 2^-sh first, sh chosen so that the largest |q| a warp holds lands in
+// [2^14, 2^15), and the scores are scaled by 2^sh after the products. Both
+// scalings are by powers of two: every bf16 q within 2^29 of that largest one
+// becomes an f16 exactly (f16: 11 significant bits from 2^-14 up to 65504),
+// and the fp32 products and sums are the unshifted ones times 2^-sh exactly,
+// so the scores do not depend on sh. (Rounding q to f16 unshifted would turn
+// |q| > 65504 into infinity and drop bits below 2^-14.)
+__device__ __forceinline__ int q_shift_warp(float amax_lane) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(amax_lane));
+    if (m == 0u) return 0;
+    const int e = (int)((m >> 23) & 0xFFu) - 127;  // floor(log2 of the largest |q|)
+    return max(-112, min(113, e - 14));
+}
+// 2^e for -126 <= e <= 127
+__device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
+
 // Softmax weights of the CUDA-core consumer over quantised codes by
 // ex2_approx rather than exp2f: that consumer is bound by instruction issue
 // (one widening per code), bf16 and fp32 caches are bound by HBM.
@@ -388,7 +406,18 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
             for (int j = 0; j < QV; ++j) qf[u * QV + j] = kMixed ? f[j] : f[j] * qs;
         }
+        float qsc = qs;  // score scale applied to the dot product
         if constexpr (kMixed) {
+            // q to f16 with the power-of-two shift of q_shift_warp (every lane
+            // holds a part of this head's q row)
+            float am = 0.f;
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) am = fmaxf(am, fabsf(qf[j]));
+            const int sh = q_shift_warp(am);
+            const float mul = pow2i(-sh);
+            qsc = qs * pow2i(sh);
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) qf[j] *= mul;
 #pragma unroll
             for (int j = 0; j < VEC / 2; ++j) {
                 const __half2 h2 = __floats2half2_rn(qf[2 * j], qf[2 * j + 1]);
@@ -442,7 +471,7 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                         for (int j = 0; j < VEC / 2; ++j) fma2_f16_f32(qh[j], kh2[j], dot, d1);
                         dot += d1;
                         if constexpr (kBiased) dot = fmaf(-kInt8WidenBias, qsum, dot);
-                        dot *= qs;
+                        dot *= qsc;
                     } else {
                         float kf[VEC];
                         if constexpr (kBiased) int8_widen_biased(kr[it], kf);
@@ -760,16 +789,31 @@ __device__ __forceinline__ uint32_t code_word(uint32_t w) {
     return std::is_same<TC, Int8Code>::value ? w ^ 0x80808080u : w;
 }
 
-// q row of the B operand for codes: head_dim 32c .. 32c+31 as 16 f16x2 words.
-__device__ __forceinline__ void load_q_codes(const uint16_t* qrow, int c, uint4 (&q)[4]) {
+// q row of the B operand for codes: head_dim 32c .. 32c+31 as raw bf16 words
+// (zeros without a row), their largest magnitude, and their conversion to 16
+// f16x2 words of q * mul (mul a signed power of two: exact).
+__device__ __forceinline__ void load_q_raw(const uint16_t* qrow, int c, uint4 (&raw)[4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        raw[u] = qrow != nullptr ? ld_v4(qrow + 32 * c + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
+}
+__device__ __forceinline__ float q_raw_amax(const uint4 (&raw)[4]) {
+    uint32_t m = 0;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-        const uint4 raw = ld_v4(qrow + 32 * c + 8 * u);
-        q[u] = make_uint4(pack_f16x2(bf16_lo(raw.x), bf16_hi(raw.x)),
-                          pack_f16x2(bf16_lo(raw.y), bf16_hi(raw.y)),
-                          pack_f16x2(bf16_lo(raw.z), bf16_hi(raw.z)),
-                          pack_f16x2(bf16_lo(raw.w), bf16_hi(raw.w)));
+        const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = max(m, max((w[i] << 16) & 0x7fffffffu, w[i] & 0x7fff0000u));
     }
+    return __uint_as_float(m);
+}
+__device__ __forceinline__ void q_raw_to_f16(const uint4 (&raw)[4], float mul, uint4 (&q)[4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        q[u] = make_uint4(pack_f16x2(bf16_lo(raw[u].x) * mul, bf16_hi(raw[u].x) * mul),
+                          pack_f16x2(bf16_lo(raw[u].y) * mul, bf16_hi(raw[u].y) * mul),
+                          pack_f16x2(bf16_lo(raw[u].z) * mul, bf16_hi(raw[u].z) * mul),
+                          pack_f16x2(bf16_lo(raw[u].w) * mul, bf16_hi(raw[u].w) * mul));
 }
 
 template <typename TC>
@@ -1070,12 +1114,14 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
     // Q^T (B operand of QK): thread (r, c) holds query row r. For chunk step jp
     // (k-steps 2jp, 2jp+1) it reads 16-byte chunk x = 2c + (jp & 1) of box jp / 2,
     // the same head_dim positions its K fragments come from.
+    // Over codes q stays raw bf16 here; it becomes f16 with its power-of-two
+    // shift when the item starts (q_shift_warp).
     auto load_q = [&](const Item& it, uint4 (&q)[KCH]) {
         const int64_t head0 = (int64_t)it.s * p.num_heads + (int64_t)it.kh * group;
         if (it.valid && it.t0 < it.t1 && r < group) {
             const uint16_t* qrow = static_cast<const uint16_t*>(p.q) + (head0 + r) * D;
             if constexpr (kCodes) {
-                load_q_codes(qrow, c, q);
+                load_q_raw(qrow, c, q);
             } else {
 #pragma unroll
                 for (int jp = 0; jp < KCH; ++jp)
@@ -1095,6 +1141,11 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
         uint4 qnxt[KCH];
         load_q(nxt, qnxt);  // in flight while this item is processed
 #endif
+        int qsh = 0;  // over codes: this item's q to f16, scaled by 2^-qsh
+        if constexpr (kCodes) {
+            qsh = q_shift_warp(q_raw_amax(qcur));
+            q_raw_to_f16(qcur, pow2i(-qsh), qcur);
+        }
         const int64_t head0 = (int64_t)cur.s * p.num_heads + (int64_t)cur.kh * group;
         if (cur.t0 >= cur.t1) {
             if (P == 1)
@@ -1103,8 +1154,9 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
         } else {
             const int t0 = cur.t0, t1 = cur.t1;
             const int n_sub = (t1 - t0 + 15) >> 4;
-            // score scale (the K scale of a quantised cache folds in)
-            const float sl = kCodes ? p.scale_log2 * __ldg(p.k_scale + cur.kh) : p.scale_log2;
+            // score scale (the K scale of a quantised cache and q's shift fold in)
+            const float sl =
+                kCodes ? p.scale_log2 * __ldg(p.k_scale + cur.kh) * pow2i(qsh) : p.scale_log2;
             float acc[MT][4];
 #pragma unroll
             for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
@@ -1388,6 +1440,7 @@ __host__ __device__ constexpr int grouped_min_blocks(int d, int cw, int nt) {
 template <typename TC, int D, int SUB, int RING>
 struct GroupedRing {
     using T = TC;
+    static constexpr bool kU2 = false;  // stage layout: [K sub-tiles][V sub-tiles]
     static constexpr int kSub = SUB;
     static constexpr int kBoxes = D * (int)sizeof(TC) / 128;
     static constexpr int kBoxElems = 128 / (int)sizeof(TC);
@@ -1607,11 +1660,17 @@ __device__ __forceinline__ void gload_units(const DecodeParams& p, const GItem& 
 // of kv head kh; the full barrier expects exactly those bytes. A block id
 // outside the pool marks the stage empty-handed (nothing loaded) and records
 // PA_ERR_BAD_INDEX. Returns false if the wait timed out.
+// With G::kU2 (the tcgen05 consumer's ring) a stage holds K as two d-halves of
+// kSub * 16 rows x 128 bytes, then V the same way (one canonical operand tile
+// per half), K completing on ring.full[st] and V on the barrier kStages
+// entries after it; hdr2 (if given) receives the unit's largest valid token
+// count over the members that use it.
 template <class G>
 __device__ __forceinline__ bool issue_unit(const CUtensorMap* kmap, const CUtensorMap* vmap,
                                            const DecodeParams& p, const Ring& ring, int gi,
                                            const int (&ph)[G::kSub], int nsub, int kh, int tok0,
-                                           uint32_t* hdr, uint32_t hval) {
+                                           uint32_t* hdr, uint32_t hval, uint32_t* hdr2 = nullptr,
+                                           uint32_t hval2 = 0) {
     const int st = gi % G::kStages;
     const uint32_t round = (uint32_t)(gi / G::kStages);
     if (!mbar_wait_bounded(ring.empty + 8 * st, (round & 1u) ^ 1u)) {
@@ -1620,10 +1679,42 @@ __device__ __forceinline__ bool issue_unit(const CUtensorMap* kmap, const CUtens
     }
     if (gi == p.test_skip_position) return true;  // test hook: leave this stage unloaded
     hdr[st] = hval;
+    if (hdr2 != nullptr) hdr2[st] = hval2;
     bool ok = true;
 #pragma unroll
     for (int s = 0; s < G::kSub; ++s)
         if (s < nsub && (unsigned)ph[s] >= (unsigned)p.num_blocks) ok = false;
+    if constexpr (G::kU2) {
+        const uint32_t full_k = ring.full + 8 * st, full_v = ring.full + 8 * (G::kStages + st);
+        if (ok) {
+            ring.valid[st] = 1;
+            const uint32_t bytes = (uint32_t)(nsub * G::kBoxes * kBoxBytes);
+            mbar_arrive_expect_tx(full_k, bytes);
+            mbar_arrive_expect_tx(full_v, bytes);
+            const uint32_t sb = ring.stages + st * G::kStageBytes;
+#pragma unroll
+            for (int s = 0; s < G::kSub; ++s) {
+                if (s < nsub) {
+                    const int32_t row = (ph[s] * p.num_kv_heads + kh) * p.block_size +
+                                        ((tok0 + 16 * s) & (p.block_size - 1));
+#pragma unroll
+                    for (int b = 0; b < G::kBoxes; ++b)
+                        tma_load_2d(sb + b * G::kHalfBytes + s * kBoxBytes, kmap, b * G::kBoxElems, row,
+                                    full_k);
+#pragma unroll
+                    for (int b = 0; b < G::kBoxes; ++b)
+                        tma_load_2d(sb + (G::kBoxes + b) * G::kHalfBytes + s * kBoxBytes, vmap,
+                                    b * G::kBoxElems, row, full_v);
+                }
+            }
+        } else {
+            atomicOr(&s_status_tma, kStatusBadIndex);
+            ring.valid[st] = 0;
+            mbar_arrive(full_k);
+            mbar_arrive(full_v);
+        }
+        return true;
+    }
     if (ok) {
         ring.valid[st] = 1;
         const uint32_t full = ring.full + 8 * st;
@@ -1660,15 +1751,17 @@ __device__ __forceinline__ void issue_units_sub(const CUtensorMap* kmap, const C
                                                 const DecodeParams& p, const Ring& ring, uint32_t* hdr,
                                                 const GItem& it, int ubase, int n_units, uint32_t act,
                                                 const int (&phys)[kMaxGroupSeqs][G::kSub], int lane,
-                                                int& g, int& issued, bool& dead) {
+                                                int& g, int& issued, bool& dead,
+                                                uint32_t* hdr2 = nullptr) {
     constexpr int SUB = G::kSub;
     const int i = ubase + lane;
     const int tok0 = it.t0 + i * (16 * SUB);
-    int nsub[kMaxGroupSeqs];
+    int nsub[kMaxGroupSeqs], nvm[kMaxGroupSeqs];
 #pragma unroll
     for (int m = 0; m < kMaxGroupSeqs; ++m) {
         const int t1 = __shfl_sync(0xffffffffu, it.t1_lane, m);
         nsub[m] = ((act >> m) & 1u) ? min(SUB, (t1 - tok0 + 15) >> 4) : 0;
+        nvm[m] = ((act >> m) & 1u) ? min(16 * SUB, t1 - tok0) : 0;
     }
     auto same = [&](int a, int b) {
         bool eq = nsub[a] == nsub[b];
@@ -1711,7 +1804,12 @@ __device__ __forceinline__ void issue_units_sub(const CUtensorMap* kmap, const C
                         if (((act >> m2) & 1u) && same(m, m2)) mask |= 1u << m2;
                     const uint32_t h = mask | ((uint32_t)i << kUnitSubShift) |
                                        (last_batch && pos == total - 1 ? kUnitLast : 0u);
-                    ok = issue_unit<G>(kmap, vmap, p, ring, g + pos, phys[m], nsub[m], it.kh, tok0, hdr, h);
+                    int nv = 0;
+#pragma unroll
+                    for (int m2 = 0; m2 < kMaxGroupSeqs; ++m2)
+                        if ((mask >> m2) & 1u) nv = max(nv, nvm[m2]);
+                    ok = issue_unit<G>(kmap, vmap, p, ring, g + pos, phys[m], nsub[m], it.kh, tok0, hdr, h,
+                                       hdr2, (uint32_t)nv);
                     if (ok) issued = g + pos + 1;
                 }
                 ++pos;
@@ -2119,35 +2217,52 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         wbits |= bita[j] | bitb[j];
     }
     wbits = __reduce_or_sync(0xffffffffu, wbits);
-    // q of the item's columns (zero for columns without a member, sequence or tokens)
-    auto load_q = [&](const GItem& it, uint4 (&q)[NT][KCH]) {
+    // q of the item's columns (zero for columns without a member, sequence or
+    // tokens). The softmax below takes the max of unscaled scores, so the sign
+    // of the score scale goes into q (an exact negation) and the scale used is
+    // its magnitude; over codes q is rounded to f16 with a power-of-two shift
+    // (q_shift_warp) that the returned score scale undoes.
+    auto load_q = [&](const GItem& it, uint4 (&q)[NT][KCH]) -> float {
+        const float sl0 = kCodes && it.valid ? p.scale_log2 * __ldg(p.k_scale + it.kh) : p.scale_log2;
+        const bool neg = sl0 < 0.f;
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
             const int col = col0 + 8 * j + r;
             const int m = col / group, hd = col - m * group;
             const int t1 = __shfl_sync(0xffffffffu, it.t1_lane, m & (kMaxGroupSeqs - 1));
-            if (it.valid && m < gs && m < it.nmem && t1 > it.t0) {
-                const uint16_t* qrow =
-                    static_cast<const uint16_t*>(p.q) +
-                    ((int64_t)(it.row0 + m) * p.num_heads + (int64_t)it.kh * group + hd) * D;
-                if constexpr (kCodes) {
-                    load_q_codes(qrow, c, q[j]);
-                } else {
-#pragma unroll
-                    for (int jp = 0; jp < KCH; ++jp)
-                        q[j][jp] = ld_v4(qrow + (jp >> 1) * 64 + (2 * c + (jp & 1)) * 8);
-                }
+            const uint16_t* qrow = nullptr;
+            if (it.valid && m < gs && m < it.nmem && t1 > it.t0)
+                qrow = static_cast<const uint16_t*>(p.q) +
+                       ((int64_t)(it.row0 + m) * p.num_heads + (int64_t)it.kh * group + hd) * D;
+            if constexpr (kCodes) {
+                load_q_raw(qrow, c, q[j]);
             } else {
+                const uint32_t sg = neg ? 0x80008000u : 0u;
 #pragma unroll
-                for (int jp = 0; jp < KCH; ++jp) q[j][jp] = make_uint4(0u, 0u, 0u, 0u);
+                for (int jp = 0; jp < KCH; ++jp) {
+                    uint4 v = qrow != nullptr ? ld_v4(qrow + (jp >> 1) * 64 + (2 * c + (jp & 1)) * 8)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+                    q[j][jp] = make_uint4(v.x ^ sg, v.y ^ sg, v.z ^ sg, v.w ^ sg);
+                }
             }
         }
+        if constexpr (kCodes) {
+            float am = 0.f;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) am = fmaxf(am, q_raw_amax(q[j]));
+            const int sh = q_shift_warp(am);
+            const float mul = neg ? -pow2i(-sh) : pow2i(-sh);
+#pragma unroll
+            for (int j = 0; j < NT; ++j) q_raw_to_f16(q[j], mul, q[j]);
+            return fabsf(sl0) * pow2i(sh);
+        }
+        return fabsf(sl0);
     };
     bool dead = false;
     int g = 0;
     GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, warp == 0, P == 1);
     uint4 q[NT][KCH];
-    load_q(cur, q);
+    float sl = load_q(cur, q);  // the item's score scale (log2 units, positive)
     while (cur.valid && !dead) {
         GItem nxt = gitem_next(walk, p, num_items, gs, ipb, lane, warp == 0, P == 1);
         int t1a[NT], t1b[NT];
@@ -2159,8 +2274,6 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         float acc[NT][MT][4], ls[NT][4];
         float ma[NT], mb[NT], la[NT], lb[NT];
-        // score scale in log2 units (a quantised cache's K scale folds in)
-        const float sl = kCodes ? p.scale_log2 * __ldg(p.k_scale + cur.kh) : p.scale_log2;
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
 #pragma unroll
@@ -2248,7 +2361,7 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             }
         }
         cur = nxt;
-        load_q(cur, q);
+        sl = load_q(cur, q);
     }
 }
 
@@ -2332,53 +2445,94 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 }
 
 // ---------------------------------------------------------------------------
-// Grouped and multi-token decode on the 5th-generation tensor cores
-// (head_dim 128, bf16, 16..64 query columns; opt-in, see grouped_consumer).
-// Same work items as decode_tma_grouped_kernel, with one-sub-tile units: one
-// ring position per distinct block of a 16-token sub-tile, mask + sub-tile
-// index in a per-stage header, plus the unit's largest valid token count
-// (issue_units); the consumer is split by role:
-//   warp 3, lane 0, issues per unit S = Q . K^T (M = 128 query rows, N = 16
-//     tokens, K = 128; Q and the K tile from shared memory, S in TMEM) and
-//     O += P . V (A = P in TMEM, B = the V tile read MN-major from shared
-//     memory, O in TMEM) with tcgen05.mma, completions signalled by
-//     tcgen05.commit;
-//   warps 0 and 1 (TMEM lane quarters 0 and 1): softmax, thread = query row:
-//     the row's 16 scores come from TMEM, the running max and sum stay in
-//     registers, P goes back to TMEM; they also stage each item's q in shared
-//     memory and write the item's output from O;
-//   warp 2: the producer (TMA).
-// S and P are double-buffered, so the next unit's QK overlaps this unit's
-// softmax. Rescaling is lazy: a row's O is rescaled (in TMEM) only when its max
-// grows by more than kRescaleLog2 (log2 units); until then the weights use the
-// older max, which numerator and denominator share, so the result is the same
-// exact softmax (weights stay below 2^kRescaleLog2). The running max moves per
-// logical 16-token sub-tile of a member, so a member's result does not depend on
-// which blocks it shares. V rows past every member's context are zeroed in
-// shared memory before the PV product reads them.
-// Measured against the mma.sync consumer (4-beam GQA CoW, 4-token verification
-// over 32K contexts): slower, 172 vs 90 and 452 vs 212 us. Per CTA one softmax
-// warp walks the units one after the other, and with at most 2 CTAs per SM (TMEM,
-// shared memory) too few warps hide the TMEM / barrier round trips of a 16 x 32
-// contraction; batching 4 units per softmax pass made it slower still.
+// Grouped and multi-token decode on the 5th-generation tensor cores (bf16,
+// head_dim 128, at most 32 query columns (member, head) per item).
+// Same work items as decode_tma_grouped_kernel, with 64-token units: four
+// 16-token sub-tiles of one distinct block sequence, a header per stage
+// (member mask, unit index, last-unit flag) and the unit's largest valid
+// token count over its members. Roles:
+//   warp 4: the producer. A stage holds the unit's K as two d-halves of 64
+//     rows x 128 bytes (128-byte swizzle), then its V the same way, so each
+//     is one canonical operand tile; K and V complete on barriers of their
+//     own, so S = Q K^T can start while V is still landing;
+//   warp 5, lane 0: per unit S = Q . K^T (M = 128 rows, N = 64 tokens,
+//     K = 128: 8 tcgen05.mma kind::f16 steps, S in TMEM, double-buffered) and
+//     O += P . V (A = P from shared memory, B = V read MN-major; M = 128,
+//     N = 128, K = 64: 4 steps, O in TMEM); completions by tcgen05.commit;
+//   warps 0..3 (TMEM lane quarters 0..3): softmax. The item's (up to) 32 query
+//     columns are replicated into the four 32-row quarters of the 128-row Q
+//     tile, so warp w finds every column's scores in its own TMEM lanes; it
+//     takes tokens 16 w .. 16 w + 15 of each unit (thread = column x token
+//     slice). The four warps share one reference max per column.
+// A unit's weights are 2^(score - m) with m the column's reference max, moved
+// only when a score exceeds it by more than kU2RescaleLog2 (log2 units);
+// numerator and denominator share m, so the result is the exact softmax with
+// weights below 2^kU2RescaleLog2. Whether any column must move is one
+// bar.red.or over the softmax warps per unit; only then do they exchange their
+// slice maxima through shared memory, and warp 0 (whose TMEM lanes hold O's
+// rows) rescales O. A column's decisions depend only on its own scores in
+// logical order, so its result is the same whichever blocks it shares and
+// whichever members share its CTA. P (bf16, row = column, 64 tokens) goes to a
+// double-buffered shared tile that the PV MMA reads. V rows past every
+// member's tokens are zeroed before the PV MMA reads them. Every wait is
+// bounded; a give-up is agreed by the softmax warps at the next per-unit vote,
+// and TMEM is freed after a final commit on every path.
 // ---------------------------------------------------------------------------
-constexpr int kUmmaRing = 49152;
-constexpr int kUmmaQBuf = 16384;           // one item's q: 64 rows x 256 B, two 128-B-swizzled atoms
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColO = 0, kColS = 128, kColP = 160;  // S at 128 / 144, P at 160 / 168
-constexpr float kRescaleLog2 = 8.f;
-constexpr uint32_t kIdescQK = umma_idesc(128, 16, false);
-constexpr uint32_t kIdescPV = umma_idesc(128, 128, true);
-using UmmaGeom = Geom<__nv_bfloat16, 128, 1, kUmmaRing>;
+constexpr int kU2Tokens = 64;                   // tokens per unit
+constexpr int kU2Cols = 32;                     // query columns per item, at most
+constexpr int kU2Slice = kU2Tokens / 4;         // tokens per softmax warp per unit
+constexpr int kU2HalfBytes = kU2Tokens * 128;   // one d-half of a K or V tile: 8 KB
+#ifndef PA_U2_STAGES
+#define PA_U2_STAGES 2
+#endif
+constexpr int kU2PBytes = kU2Cols * 128;        // P tile: 32 rows x 64 bf16 tokens
+constexpr int kU2QBytes = 2 * 128 * 128;        // Q tile: 128 rows x 128 bf16, two d-halves
+constexpr int kU2QOff = 2 * kU2PBytes;          // shared memory: [P0][P1][Q][ring][...]
+constexpr int kU2RingOff = kU2QOff + kU2QBytes;
+constexpr uint32_t kU2TmemCols = 256;
+constexpr uint32_t kU2ColO = 0, kU2ColS = 128;  // S buffers at columns 128 and 192
+constexpr float kU2RescaleLog2 = 8.f;
+constexpr uint32_t kU2IdescQK = umma_idesc(128, 64, false);
+constexpr uint32_t kU2IdescPV = umma_idesc(128, 128, true);
 
-struct UmmaBars {
-    uint32_t full, empty, s, pv, pfull, q, ofree, done, fin;  // shared addresses
+struct U2Geom {
+    using T = __nv_bfloat16;
+    static constexpr bool kU2 = true;
+    static constexpr int kSub = kU2Tokens / 16;
+    static constexpr int kStages = PA_U2_STAGES;
+    static constexpr int kBoxes = 2;
+    static constexpr int kBoxElems = 64;
+    static constexpr int kHalfBytes = kU2HalfBytes;
+    static constexpr int kSubBytes = kBoxes * kBoxBytes;
+    static constexpr int kStageBytes = 4 * kU2HalfBytes;  // K halves, then V halves: 32 KB
+    static constexpr int kRingBytes = kStages * kStageBytes;
+};
+static_assert(kU2RingOff % 1024 == 0, "ring stages on 1024-byte boundaries");
+// the PV MMA reads 128 rows (16 KB) of a P buffer; rows 32..127 (results never
+// used) come from the shared memory after it
+static_assert(kU2PBytes + 16384 <= kU2RingOff + U2Geom::kRingBytes, "P windows inside the CTA");
+
+// [hdr S][hdr2 S][valid S] then barriers: full_k S, full_v S, empty S, s 2,
+// pv 2, p 2, q, ofree, done, fin; then the TMEM slot and the dead flag; then
+// the slice maxima [2][4][32], give-up flags [2][4] and slice sums [4][32].
+constexpr int kU2ExtHdr = 12 * U2Geom::kStages;
+constexpr int kU2ExtBars = (kU2ExtHdr + 7) & ~7;
+constexpr int kU2NumBars = 3 * U2Geom::kStages + 10;
+constexpr int kU2ExtSlot = kU2ExtBars + 8 * kU2NumBars;
+constexpr int kU2ExtXm = (kU2ExtSlot + 8 + 15) & ~15;
+constexpr int kU2ExtXf = kU2ExtXm + 2 * 4 * 32 * 4;
+constexpr int kU2ExtXl = kU2ExtXf + 2 * 4 * 4;
+constexpr int kU2ExtBytes = kU2ExtXl + 4 * 32 * 4;
+constexpr size_t kU2Smem = (size_t)kU2RingOff + U2Geom::kRingBytes + kU2ExtBytes;
+
+struct U2Bars {
+    uint32_t full_k, full_v, empty, s, pv, p, q, ofree, done, fin;  // shared addresses
     volatile int* dead;
 };
 
 // Bounded wait by a whole warp, warp-uniform outcome; gives up at once when
 // another role already gave up (so timeouts do not chain).
-__device__ __forceinline__ bool umma_wait(const UmmaBars& b, uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool u2_wait(const U2Bars& b, uint32_t bar, uint32_t parity) {
     const bool ok = __all_sync(0xffffffffu, *b.dead == 0 && mbar_wait_bounded(bar, parity));
     if (!ok && (threadIdx.x & 31) == 0) {
         if (*b.dead == 0) atomicOr(&s_status_tma, kStatusTimeout);
@@ -2387,68 +2541,79 @@ __device__ __forceinline__ bool umma_wait(const UmmaBars& b, uint32_t bar, uint3
     return ok;
 }
 
-template <int D>
-__global__ void __launch_bounds__(128, 2)
+// OR of `pred` over the 128 threads of the softmax warps (named barrier 1).
+__device__ __forceinline__ bool softmax_any(bool pred) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n"
+                 " bar.red.or.pred p, 1, 128, q;\n selp.u32 %0, 1, 0, p;\n}"
+                 : "=r"(r) : "r"((uint32_t)pred) : "memory");
+    return r != 0;
+}
+
+__global__ void __launch_bounds__(192, 2)
 decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                            const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
                            int num_items, int gs) {
-    static_assert(D == 128, "head_dim 128");
-    using G = UmmaGeom;
+    using G = U2Geom;
     constexpr int S_ = G::kStages;
+    constexpr int D = 128;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = p.num_partitions;
     const int group = p.num_heads / p.num_kv_heads;
     const int ncols = gs * group;
-    const int sw = (ncols + 31) >> 5;  // softmax warps
     const int ipb = 32 / gs;
     const uint32_t raw = smem_u32(smem_raw);
     if (raw & 1023u) {
         if (threadIdx.x == 0) atomicOr(&s_status_tma, kStatusSmemAlign);
         return;
     }
-    // [q buffers 2 x 16 KB][ring][hdr][hdr2][barriers][valid][tmem slot][dead]
-    const uint32_t qbuf = raw;
-    Ring ring;
-    ring.stages = raw + 2 * kUmmaQBuf;
-    uint32_t* hdr = reinterpret_cast<uint32_t*>(smem_raw + 2 * kUmmaQBuf + G::kRingBytes);
+    const uint32_t pbuf = raw, qbuf = raw + kU2QOff;
+    uint8_t* ext = smem_raw + kU2RingOff + G::kRingBytes;
+    uint32_t* hdr = reinterpret_cast<uint32_t*>(ext);
     uint32_t* hdr2 = hdr + S_;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + 2 * kUmmaQBuf + G::kRingBytes +
-                                                 ((2 * S_ * 4 + 7) & ~7));
-    UmmaBars B;
-    B.full = smem_u32(bars);
-    B.empty = B.full + 8 * S_;
-    B.s = B.empty + 8 * S_;       // [2]
-    B.pv = B.s + 16;              // [2]
-    B.pfull = B.pv + 16;          // [2]
-    B.q = B.pfull + 16;           // [2]
-    B.ofree = B.q + 16;
+    int* valid = reinterpret_cast<int*>(hdr2 + S_);
+    U2Bars B;
+    B.full_k = smem_u32(ext + kU2ExtBars);
+    B.full_v = B.full_k + 8 * S_;
+    B.empty = B.full_v + 8 * S_;
+    B.s = B.empty + 8 * S_;  // [2]
+    B.pv = B.s + 16;         // [2]
+    B.p = B.pv + 16;         // [2]
+    B.q = B.p + 16;
+    B.ofree = B.q + 8;
     B.done = B.ofree + 8;
     B.fin = B.done + 8;
-    ring.full = B.full;
-    ring.empty = B.empty;
-    ring.valid = reinterpret_cast<int*>(bars + 2 * S_ + 13);
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(ring.valid + S_);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(ext + kU2ExtSlot);
     B.dead = reinterpret_cast<volatile int*>(tslot + 1);
+    float* xm = reinterpret_cast<float*>(ext + kU2ExtXm);  // [2][4][32] slice maxima
+    volatile int* xf = reinterpret_cast<volatile int*>(ext + kU2ExtXf);  // [2][4] give-ups
+    float* xl = reinterpret_cast<float*>(ext + kU2ExtXl);  // [4][32] slice sums
+    Ring ring;
+    ring.stages = raw + kU2RingOff;
+    ring.full = B.full_k;
+    ring.empty = B.empty;
+    ring.valid = valid;
     if (threadIdx.x == 0) {
         for (int st = 0; st < S_; ++st) {
-            mbar_init(B.full + 8 * st, 1);
-            mbar_init(B.empty + 8 * st, 1);  // released by the MMA thread's commit
+            mbar_init(B.full_k + 8 * st, 1);
+            mbar_init(B.full_v + 8 * st, 1);
+            mbar_init(B.empty + 8 * st, 1);  // the MMA thread's commit after the unit's PV
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(B.s + 8 * i, 1);
             mbar_init(B.pv + 8 * i, 1);
-            mbar_init(B.pfull + 8 * i, sw);
-            mbar_init(B.q + 8 * i, sw);
+            mbar_init(B.p + 8 * i, 4);
         }
-        mbar_init(B.ofree, sw);
-        mbar_init(B.done, sw);
+        mbar_init(B.q, 4);
+        mbar_init(B.ofree, 4);
+        mbar_init(B.done, 4);
         mbar_init(B.fin, 1);
         *B.dead = 0;
         fence_barrier_init();
     }
-    if (warp == 3) tmem_alloc(smem_u32(tslot), kTmemCols);
+    if (warp == 5) tmem_alloc(smem_u32(tslot), kU2TmemCols);
     GWalk walk;
     walk.k = 0;
     walk.kbase = 0;
@@ -2458,63 +2623,80 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
     tc_fence_after();
     const uint32_t tm = *tslot;
 
-    if (warp == 2) {  // producer
+    if (warp == 4) {  // producer
         if (lane == 0) {
             prefetch_tensormap(&kmap);
             prefetch_tensormap(&vmap);
         }
+        constexpr int SUB = G::kSub;
         bool dead = false;
         int g = 0, issued = 0;
         GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
         int cur_base = 0;
         uint32_t act_cur;
-        int phys_cur[kMaxGroupSeqs];
-        gload_phys(p, cur, cur_base, gs, lane, act_cur, phys_cur);
+        int phys_cur[kMaxGroupSeqs][SUB];
+        gload_units<SUB>(p, cur, cur_base, gs, lane, act_cur, phys_cur);
         while (cur.valid && !dead) {
-            const int n_sub = (cur.tmax - cur.t0 + 15) >> 4;
+            const int n_units = (cur.tmax - cur.t0 + kU2Tokens - 1) / kU2Tokens;
             GItem nxt = cur;
             int nxt_base = cur_base + 32;
-            if (nxt_base >= n_sub) {
+            if (nxt_base >= n_units) {
                 nxt = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
                 nxt_base = 0;
             }
             uint32_t act_nxt;
-            int phys_nxt[kMaxGroupSeqs];
-            gload_phys(p, nxt, nxt_base, gs, lane, act_nxt, phys_nxt);
-            issue_units<G>(&kmap, &vmap, p, ring, hdr, cur, cur_base, n_sub, act_cur, phys_cur,
-                           lane, g, issued, dead, hdr2);
+            int phys_nxt[kMaxGroupSeqs][SUB];
+            gload_units<SUB>(p, nxt, nxt_base, gs, lane, act_nxt, phys_nxt);
+            issue_units_sub<G>(&kmap, &vmap, p, ring, hdr, cur, cur_base, n_units, act_cur, phys_cur,
+                               lane, g, issued, dead, hdr2);
             if (*B.dead) dead = true;
             cur = nxt;
             cur_base = nxt_base;
             act_cur = act_nxt;
 #pragma unroll
-            for (int m = 0; m < kMaxGroupSeqs; ++m) phys_cur[m] = phys_nxt[m];
+            for (int m = 0; m < kMaxGroupSeqs; ++m)
+#pragma unroll
+                for (int u = 0; u < SUB; ++u) phys_cur[m][u] = phys_nxt[m][u];
         }
         if (dead) *B.dead = 1;
-        drain_ring<G>(ring, issued, lane);
+        // drain: the last loads (K and V) of every stage have landed
+        if (lane == 0 && issued > 0) {
+            const int last = min(issued, S_);
+            for (int st = 0; st < last; ++st) {
+                const int it = issued - 1 - ((issued - 1 - st) % S_);
+                const uint32_t par = (uint32_t)(it / S_) & 1u;
+                if (!mbar_wait_bounded(B.full_k + 8 * st, par) ||
+                    !mbar_wait_bounded(B.full_v + 8 * st, par))
+                    atomicOr(&s_status_tma, kStatusTimeout);
+            }
+        }
         return;
     }
 
-    if (warp == 3) {  // MMA issuer: lane 0 issues, the warp walks the items with it
+    if (warp == 5) {  // MMA issuer: lane 0 issues, the warp walks the items with it
         int g = 0, n = 0;
-        bool have_prev = false, prev_valid = false, prev_first = false, o_started = false;
-        int prev_st = 0, prev_g = 0, prev_item = 0;
-        // PV of a unit: after its P is in TMEM (and, for an item's first unit,
-        // after the previous item's output left O); then release its stage.
+        int prev_g = -1, prev_st = 0, prev_item = 0;
+        bool prev_valid = false, prev_first = false, o_started = false;
+        // PV of unit prev_g: after its P is in shared memory and its V landed
+        // (and, for an item's first unit, after the previous item's output left
+        // O); then release its stage.
         auto issue_pv = [&]() -> bool {
-            if (!umma_wait(B, B.pfull + 8 * (prev_g & 1), (prev_g >> 1) & 1)) return false;
+            if (!u2_wait(B, B.p + 8 * (prev_g & 1), (prev_g >> 1) & 1)) return false;
             if (prev_first) {
                 o_started = false;
-                if (prev_item >= 1 && !umma_wait(B, B.ofree, (prev_item - 1) & 1)) return false;
+                if (prev_item >= 1 && !u2_wait(B, B.ofree, (prev_item - 1) & 1)) return false;
             }
+            if (!u2_wait(B, B.full_v + 8 * prev_st, (uint32_t)(prev_g / S_) & 1u)) return false;
             tc_fence_after();
             if (lane == 0) {
                 if (prev_valid) {
-                    const uint32_t vb = ring.stages + prev_st * G::kStageBytes + 2 * kBoxBytes;
-                    // V read MN-major: head_dim atoms of 64 (one box each) kBoxBytes
-                    // apart, 8-token groups 1024 B apart
-                    umma_ts(tm + kColO, tm + kColP + 8 * (prev_g & 1), umma_desc(vb, kBoxBytes, 1024),
-                            kIdescPV, o_started);
+                    const uint32_t pa = pbuf + (prev_g & 1) * kU2PBytes;
+                    const uint32_t vb = ring.stages + prev_st * G::kStageBytes + 2 * kU2HalfBytes;
+#pragma unroll
+                    for (int k = 0; k < kU2Tokens / 16; ++k)
+                        umma_ss(tm + kU2ColO, umma_desc(pa + 32 * k, 16, 1024),
+                                umma_desc(vb + 2048 * k, kU2HalfBytes, 1024), kU2IdescPV,
+                                o_started || k > 0);
                 }
                 umma_commit(B.pv + 8 * (prev_g & 1));
                 umma_commit(B.empty + 8 * prev_st);
@@ -2526,32 +2708,32 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         bool ok = true;
         GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
         while (cur.valid && ok) {
-            if (!umma_wait(B, B.q + 8 * (n & 1), (n >> 1) & 1)) { ok = false; break; }
+            if (!u2_wait(B, B.q, n & 1)) { ok = false; break; }
             tc_fence_after();
             bool first = true;
             for (;;) {
                 const int st = g % S_;
-                if (!umma_wait(B, B.full + 8 * st, (uint32_t)(g / S_) & 1u)) { ok = false; break; }
+                if (!u2_wait(B, B.full_k + 8 * st, (uint32_t)(g / S_) & 1u)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t h = hdr[st];
-                const bool valid = ring.valid[st] != 0;
+                const bool v = valid[st] != 0;
                 if (lane == 0) {
-                    const uint32_t kb = ring.stages + st * G::kStageBytes;
-                    const uint32_t qa = qbuf + (n & 1) * kUmmaQBuf;
+                    if (v) {
+                        const uint32_t kb = ring.stages + st * G::kStageBytes;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        umma_ss(tm + kColS + 16 * (g & 1),
-                                umma_desc(qa + (k >> 2) * (kUmmaQBuf / 2) + (k & 3) * 32, 16, 1024),
-                                umma_desc(kb + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024),
-                                kIdescQK, k > 0);
+                        for (int k = 0; k < 8; ++k)
+                            umma_ss(tm + kU2ColS + 64 * (g & 1),
+                                    umma_desc(qbuf + (k >> 2) * (kU2QBytes / 2) + (k & 3) * 32, 16, 1024),
+                                    umma_desc(kb + (k >> 2) * kU2HalfBytes + (k & 3) * 32, 16, 1024),
+                                    kU2IdescQK, k > 0);
+                    }
                     umma_commit(B.s + 8 * (g & 1));
                 }
                 __syncwarp();
-                if (have_prev && !issue_pv()) { ok = false; break; }
-                have_prev = true;
-                prev_st = st;
+                if (prev_g >= 0 && !issue_pv()) { ok = false; break; }
                 prev_g = g;
-                prev_valid = valid;
+                prev_st = st;
+                prev_valid = v;
                 prev_first = first;
                 prev_item = n;
                 first = false;
@@ -2561,8 +2743,8 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             ++n;
             if (ok) cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
         }
-        if (ok && have_prev) ok = issue_pv();
-        // wait for the softmax warps (even after a timeout: they stop touching
+        if (ok && prev_g >= 0) ok = issue_pv();
+        // wait for the softmax warps (even after a give-up: they stop touching
         // TMEM before they arrive), then for every issued MMA, then free TMEM
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(B.done, 0)) && lane == 0)
             atomicOr(&s_status_tma, kStatusTimeout);
@@ -2571,29 +2753,28 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(B.fin, 0)) && lane == 0)
             atomicOr(&s_status_tma, kStatusTimeout);
         tc_fence_after();
-        tmem_dealloc(tm, kTmemCols);
+        tmem_dealloc(tm, kU2TmemCols);
         return;
     }
 
-    if (warp >= sw) {  // no query rows for this warp
-        return;
-    }
-
-    // softmax warps: thread = query column (member, head) = row of S, P and O
-    const int col = 32 * warp + lane;
+    // softmax warps: thread = query column `lane` (member, head) of the item,
+    // tokens 16 warp .. 16 warp + 15 of every unit; Q row 32 warp + lane
+    const int col = lane;
     const int mem = col / group, hd = col - mem * group;
-    const uint32_t mybit = (col < ncols && mem < gs) ? 1u << mem : 0u;
+    const bool colv = col < ncols;
+    const uint32_t mybit = (colv && mem < gs) ? 1u << mem : 0u;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const int slice0 = kU2Slice * warp;
     const uint8_t* qsrc_base = static_cast<const uint8_t*>(p.q);
     int g = 0, n = 0;
-    bool ok = true;
-    // Next item with tokens; with one partition, members of items without any
-    // tokens get a zero output here.
+    bool ok = true, healthy = true;
+    // Next item with tokens; with one partition, the members of items without
+    // any tokens get a zero output here.
     auto next_item = [&]() -> GItem {
         for (;;) {
             GItem it = gitem_next(walk, p, num_items, gs, ipb, lane, warp == 0, P == 1);
             if (!it.valid || it.tmax > it.t0) return it;
-            if (col < ncols && mem < it.nmem) {
+            if (warp == 0 && colv && mem < it.nmem) {
                 uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
                     ((int64_t)(it.row0 + mem) * p.num_heads + (int64_t)it.kh * group + hd) * D);
 #pragma unroll
@@ -2601,136 +2782,199 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             }
         }
     };
-    // this row's q into buffer `buf`, 128-byte swizzled (two atoms of 64 rows)
-    auto stage_q = [&](const GItem& it, int buf) {
+    // this thread's Q row (32 warp + lane) := q of its column, 128-byte
+    // swizzled; the softmax takes maxima of unscaled scores, so the sign of the
+    // scale goes into q (an exact negation) and its magnitude is used below
+    const uint32_t qsign = p.scale_log2 < 0.f ? 0x80008000u : 0u;
+    auto stage_q = [&](const GItem& it) {
         const int t1 = __shfl_sync(0xffffffffu, it.t1_lane, mem & (kMaxGroupSeqs - 1));
-        const bool has = col < ncols && mem < it.nmem && t1 > it.t0;
+        const bool has = colv && mem < it.nmem && t1 > it.t0;
         const uint4* src = reinterpret_cast<const uint4*>(qsrc_base +
             ((int64_t)(it.row0 + mem) * p.num_heads + (int64_t)it.kh * group + hd) * D * 2);
-        uint8_t* dst = smem_raw + buf * kUmmaQBuf;
+        const uint32_t row = 32 * warp + lane;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-            const uint4 v = has ? ld_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
-            const int atom = c >> 3, x = c & 7;
-            *reinterpret_cast<uint4*>(dst + atom * (kUmmaQBuf / 2) + col * 128 + ((x ^ (col & 7)) << 4)) = v;
+            uint4 v = has ? ld_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            v = make_uint4(v.x ^ qsign, v.y ^ qsign, v.z ^ qsign, v.w ^ qsign);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                         :: "r"(qbuf + (c >> 3) * (kU2QBytes / 2) + swz(row, c & 7)),
+                            "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
         }
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(B.q + 8 * buf);
+        if (lane == 0) mbar_arrive(B.q);
     };
     GItem cur = next_item();
-    if (cur.valid) stage_q(cur, 0);
+    if (cur.valid) stage_q(cur);
     while (cur.valid && ok) {
         const int t1 = __shfl_sync(0xffffffffu, cur.t1_lane, mem & (kMaxGroupSeqs - 1));
-        const float sl = p.scale_log2;
+        const float sl = fabsf(p.scale_log2);
         float m_ref = -INFINITY, l = 0.f;
         for (;;) {
-            if (!umma_wait(B, B.s + 8 * (g & 1), (g >> 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-            const int st = g % S_;
-            const uint32_t h = hdr[st];
-            const bool valid = ring.valid[st] != 0;
-            const int nvmax = (int)hdr2[st];
-            const int tok0 = cur.t0 + (int)((h >> kUnitSubShift) & kUnitSubMask) * 16;
-            uint32_t sr[16];
-            tmem_ld16(tm + lane_off + kColS + 16 * (g & 1), sr);
-            const int nv = (valid && (h & mybit)) ? min(16, t1 - tok0) : 0;
-            float sv[16];
+            const int b = g & 1, st = g % S_;
+            // S of unit g (and with it every earlier MMA: the PV of unit g - 2
+            // no longer reads P buffer b); the K barrier orders the header reads
+            if (healthy) healthy = u2_wait(B, B.s + 8 * b, (g >> 1) & 1);
+            if (healthy) healthy = u2_wait(B, B.full_k + 8 * st, (uint32_t)(g / S_) & 1u);
+            uint32_t h = 0;
+            int nvmax = 0;
+            bool v = false;
+            float sv[kU2Slice];
             float mx = -INFINITY;
+            if (healthy) {
+                tc_fence_after();
+                h = hdr[st];
+                v = valid[st] != 0;
+                nvmax = (int)hdr2[st];
+                const int tok0 = cur.t0 + (int)((h >> kUnitSubShift) & kUnitSubMask) * kU2Tokens;
+                uint32_t sr[kU2Slice];
+                tmem_ld16(tm + lane_off + kU2ColS + 64 * b + slice0, sr);
+                const int nv = (v && (h & mybit)) ? min(kU2Slice, t1 - tok0 - slice0) : 0;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                sv[j] = j < nv ? __uint_as_float(sr[j]) * sl : -INFINITY;
-                mx = fmaxf(mx, sv[j]);
+                for (int j = 0; j < kU2Slice; ++j) sv[j] = j < nv ? __uint_as_float(sr[j]) : -INFINITY;
+                float m4[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    m4[j] = fmaxf(fmaxf(sv[4 * j], sv[4 * j + 1]), fmaxf(sv[4 * j + 2], sv[4 * j + 3]));
+                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            } else {
+#pragma unroll
+                for (int j = 0; j < kU2Slice; ++j) sv[j] = -INFINITY;
             }
-            // O must not be rescaled, nor P(g & 1) rewritten, before the PV that
-            // reads them is done (the PV of unit g - 1, resp. g - 2)
-            const bool resc = m_ref != -INFINITY && mx > m_ref + kRescaleLog2;
-            const bool any_resc = __any_sync(0xffffffffu, resc);
-            if (any_resc) {
-                if (!umma_wait(B, B.pv + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1)) { ok = false; break; }
-            } else if (g >= 2) {
-                if (!umma_wait(B, B.pv + 8 * (g & 1), ((g - 2) >> 1) & 1)) { ok = false; break; }
-            }
-            tc_fence_after();
-            if (any_resc) {
-                const float alpha = resc ? exp2f(m_ref - mx) : 1.f;
-#pragma unroll
-                for (int c0 = 0; c0 < 128; c0 += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(tm + lane_off + kColO + c0, o);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                    tmem_st32(tm + lane_off + kColO + c0, o);
+            // a column's reference max moves when a score exceeds it by more
+            // than the threshold (or on its first scores)
+            const bool exceed =
+                mx != -INFINITY && (m_ref == -INFINITY || mx * sl > m_ref + kU2RescaleLog2);
+            if (softmax_any(exceed || !healthy)) {
+                xm[(b * 4 + warp) * 32 + lane] = mx;
+                if (lane == 0) xf[b * 4 + warp] = healthy ? 0 : 1;
+                named_barrier(1, 128);
+                if (xf[b * 4] | xf[b * 4 + 1] | xf[b * 4 + 2] | xf[b * 4 + 3]) {
+                    ok = false;
+                    break;
                 }
-                if (resc) {
-                    l *= alpha;
-                    m_ref = mx;
+                float M = xm[(b * 4) * 32 + lane];
+#pragma unroll
+                for (int w = 1; w < 4; ++w) M = fmaxf(M, xm[(b * 4 + w) * 32 + lane]);
+                float alpha = 1.f;
+                bool resc = false;
+                if (M != -INFINITY && (m_ref == -INFINITY || M * sl > m_ref + kU2RescaleLog2)) {
+                    const float nm = M * sl;
+                    if (m_ref != -INFINITY) {
+                        alpha = exp2f(m_ref - nm);
+                        l *= alpha;
+                        resc = true;
+                    }
+                    m_ref = nm;
                 }
-            } else if (m_ref == -INFINITY && mx != -INFINITY) {
-                m_ref = mx;
+                // warp 0's TMEM lanes hold O's rows: rescale them once the PV of
+                // the previous unit is done
+                if (warp == 0 && __any_sync(0xffffffffu, resc)) {
+                    healthy = u2_wait(B, B.pv + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1);
+                    if (healthy) {
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int c0 = 0; c0 < 128; c0 += 32) {
+                            uint32_t o[32];
+                            tmem_ld32(tm + lane_off + kU2ColO + c0, o);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                            tmem_st32(tm + lane_off + kU2ColO + c0, o);
+                        }
+                    }
+                }
             }
-            // a row that has seen no valid token keeps max -inf: weights 0
+            // weights of the slice (masked scores give 2^-inf = 0), bf16, summed
+            // as rounded
             const float base = m_ref == -INFINITY ? 0.f : m_ref;
-            uint32_t pk[8];
+            uint32_t pk[kU2Slice / 2];
+            float ps = 0.f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                pk[j] = pack_bf16x2(exp2f(sv[2 * j] - base), exp2f(sv[2 * j + 1] - base));
-                l += bf16_lo(pk[j]) + bf16_hi(pk[j]);
+            for (int j = 0; j < kU2Slice / 2; ++j) {
+                pk[j] = pack_bf16x2(ex2_approx(fmaf(sv[2 * j], sl, -base)),
+                                    ex2_approx(fmaf(sv[2 * j + 1], sl, -base)));
+                ps += bf16_lo(pk[j]) + bf16_hi(pk[j]);
             }
-            tmem_st8(tm + lane_off + kColP + 8 * (g & 1), pk);
-            if (warp == 0 && valid && nvmax < 16) {
-                // V rows nvmax..15 (both boxes) belong to no member's context
-                const uint32_t vb = ring.stages + st * G::kStageBytes + 2 * kBoxBytes;
-                for (int i = lane; i < (16 - nvmax) * 16; i += 32) {
-                    const int row = nvmax + (i >> 4), c16 = i & 15;
-                    const uint32_t a = vb + (c16 >> 3) * kBoxBytes + row * 128 + (c16 & 7) * 16;
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" :: "r"(a), "r"(0u) : "memory");
+            l += ps;
+            // P row `col`, tokens 16 warp .. + 15: 16-byte chunks 2 warp, 2 warp + 1
+            const uint32_t prow = pbuf + b * kU2PBytes;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                         :: "r"(prow + swz(col, 2 * warp)), "r"(pk[0]), "r"(pk[1]), "r"(pk[2]),
+                            "r"(pk[3]) : "memory");
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                         :: "r"(prow + swz(col, 2 * warp + 1)), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
+                            "r"(pk[7]) : "memory");
+            // V rows of the slice at or past every member's tokens may hold
+            // anything (NaN included): zero them once V has landed
+            if (healthy && v && nvmax < slice0 + kU2Slice) {
+                healthy = u2_wait(B, B.full_v + 8 * st, (uint32_t)(g / S_) & 1u);
+                if (healthy) {
+                    const uint32_t vb = ring.stages + st * G::kStageBytes + 2 * kU2HalfBytes;
+                    const int r0 = max(nvmax, slice0);
+                    for (int i = lane; i < (slice0 + kU2Slice - r0) * 16; i += 32) {
+                        const int row = r0 + (i >> 4), c16 = i & 15;
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};"
+                                     :: "r"(vb + (c16 >> 3) * kU2HalfBytes + row * 128 + (c16 & 7) * 16),
+                                        "r"(0u) : "memory");
+                    }
                 }
-                fence_async_smem();
             }
+            fence_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(B.pfull + 8 * (g & 1));
+            if (lane == 0) mbar_arrive(B.p + 8 * b);
             ++g;
             if (h & kUnitLast) break;
         }
         if (!ok) break;
-        // next item's q first: the MMA thread needs it before the PV of this
-        // item's last unit, which the output below waits for
+        // the column's weight sum over the four slices (fixed order)
+        xl[warp * 32 + lane] = l;
+        named_barrier(1, 128);
+        const float lt = ((xl[lane] + xl[32 + lane]) + xl[64 + lane]) + xl[96 + lane];
+        // the next item's q: every QK of this item is complete (its last S was read)
         const GItem nxt = next_item();
-        if (nxt.valid) stage_q(nxt, (n + 1) & 1);
-        if (!umma_wait(B, B.pv + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        const bool has = col < ncols && mem < cur.nmem && t1 > cur.t0;
-        const int64_t row = ((int64_t)(cur.row0 + mem) * p.num_heads + (int64_t)cur.kh * group + hd);
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        if (nxt.valid) stage_q(nxt);
+        if (warp == 0) {
+            if (healthy) healthy = u2_wait(B, B.pv + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1);
+            const bool has = colv && mem < cur.nmem && t1 > cur.t0;
+            const int64_t row = (int64_t)(cur.row0 + mem) * p.num_heads + (int64_t)cur.kh * group + hd;
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            if (healthy) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tm + lane_off + kU2ColO + c0, o);
+                    if (colv && mem < cur.nmem) {
+                        if (P == 1) {
+                            uint32_t w[16];
 #pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tm + lane_off + kColO + c0, o);
-            if (col < ncols && mem < cur.nmem) {
-                if (P == 1) {
-                    uint32_t w[16];
+                            for (int j = 0; j < 16; ++j)
+                                w[j] = lt > 0.f ? pack_bf16x2(__uint_as_float(o[2 * j]) * inv,
+                                                              __uint_as_float(o[2 * j + 1]) * inv)
+                                                : 0u;
+                            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * D + c0);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        w[j] = l > 0.f ? pack_bf16x2(__uint_as_float(o[2 * j]) * inv,
-                                                     __uint_as_float(o[2 * j + 1]) * inv)
-                                       : 0u;
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * D + c0);
+                            for (int j = 0; j < 4; ++j)
+                                dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                        } else if (has) {
+                            float4* dst = reinterpret_cast<float4*>(p.ws_o + (row * P + cur.part) * D + c0);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                } else if (has) {
-                    float* dst = p.ws_o + (row * P + cur.part) * D + c0;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) dst[j] = l > 0.f ? __uint_as_float(o[j]) * inv : 0.f;
+                            for (int j = 0; j < 8; ++j)
+                                dst[j] = lt > 0.f ? make_float4(__uint_as_float(o[4 * j]) * inv,
+                                                                __uint_as_float(o[4 * j + 1]) * inv,
+                                                                __uint_as_float(o[4 * j + 2]) * inv,
+                                                                __uint_as_float(o[4 * j + 3]) * inv)
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                    }
+                }
+                if (P > 1 && has) {
+                    float* ml = p.ws_ml + (row * P + cur.part) * 2;
+                    ml[0] = lt > 0.f ? m_ref : -INFINITY;
+                    ml[1] = lt;
                 }
             }
-        }
-        if (P > 1 && has) {
-            float* ml = p.ws_ml + (row * P + cur.part) * 2;
-            ml[0] = l > 0.f ? m_ref : -INFINITY;
-            ml[1] = l;
         }
         tc_fence_before();
         __syncwarp();
@@ -2740,13 +2984,6 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(B.done);
-}
-
-template <int D>
-constexpr size_t umma_smem_bytes() {
-    using G = UmmaGeom;
-    return 2 * kUmmaQBuf + G::kRingBytes + ((2 * G::kStages * 4 + 7) & ~7) +
-           (2 * G::kStages + 13) * 8 + G::kStages * 4 + 16 + 64;
 }
 
 template <typename T, int D>
@@ -2799,8 +3036,8 @@ cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUt
 
 cudaError_t launch_umma_grouped(const DecodeParams& p, const CUtensorMap& km,
                                 const CUtensorMap& vm, int gs, cudaStream_t stream) {
-    constexpr size_t smem = umma_smem_bytes<128>();
-    auto kernel = decode_umma_grouped_kernel<128>;
+    constexpr size_t smem = kU2Smem;
+    auto kernel = decode_umma_grouped_kernel;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -2812,9 +3049,9 @@ cudaError_t launch_umma_grouped(const DecodeParams& p, const CUtensorMap& km,
     const long groups = p.query_start != nullptr ? (long)p.num_seqs * p.q_chunks
                                                  : (long)(p.num_seqs + gs - 1) / gs;
     const long items = (long)p.num_partitions * p.num_kv_heads * groups;
-    const long slots = 2L * sms;  // two CTAs per SM: 256 TMEM columns and ~81 KB each
+    const long slots = 2L * sms;  // two CTAs per SM: 256 TMEM columns and ~106 KB each
     const unsigned grid = (unsigned)(items < slots ? items : slots);
-    kernel<<<grid, 128, smem, stream>>>(km, vm, p, (int)items, gs);
+    kernel<<<grid, 192, smem, stream>>>(km, vm, p, (int)items, gs);
     return cudaGetLastError();
 }
 
@@ -2885,13 +3122,14 @@ bool mma_supported(int dtype, int head_dim, int group) {
 }
 
 // Grouped consumer selected by pa_set_grouped_consumer (process-wide). The
-// tcgen05 consumer takes head_dim 128 with 16..64 query columns (its 128-row
-// MMAs would mostly idle below that); other shapes stay on mma.sync.
+// tcgen05 consumer takes head_dim 128 with 8..32 query columns (its 128-row
+// MMAs hold four copies of up to 32 columns; with fewer than 8 they would mostly
+// idle); other shapes stay on mma.sync.
 static int g_grouped_consumer = PA_GROUPED_MMA_SYNC;
 
 static bool use_umma(int head_dim, int gs, int group) {
-    return g_grouped_consumer == PA_GROUPED_TCGEN05 && head_dim == 128 && gs * group >= 16 &&
-           gs * group <= 64;
+    return g_grouped_consumer == PA_GROUPED_TCGEN05 && head_dim == 128 && gs * group >= 8 &&
+           gs * group <= kU2Cols;
 }
 
 // Query columns (member, head) -> n-tiles of 8 -> consumer warps: one n-tile

@@ -191,3 +191,33 @@ def test_llama70b_gqa_tensor_core_path(fmt):
                               sub["block_tables"], sub["context_lens"], wl.scale, fmt,
                               num_threads=G.THREADS)
     G.check_tolerance(G.to_f64(out), ref, "bf16", wl.name)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "int8"])
+@pytest.mark.parametrize("mag", [1e6, 1e-6])
+def test_q_magnitudes_outside_f16_range(fmt, mag):
+    """Over codes q becomes an f16 MMA / fma operand. bf16 q far above f16's
+    range (|q| ~ 1e6 > 65504) or far below its normal range (~1e-6 < 2^-14)
+    still meets the bars against the oracle: q is shifted by a power of two
+    before the rounding and the scores after the products (exact). Covers the
+    CUDA-core consumer (MHA), the tensor-core consumer (GQA g = 8) and the
+    grouped / multi-token consumer."""
+    ctx = [1, 15, 16, 17, 130, 700]
+    for H, Hkv in ((8, 8), (16, 2)):
+        wl = W.quantized(G.custom(len(ctx), H, Hkv, 128, 16, "bf16", ctx, seed=31), fmt)
+        vals = W.make_values(wl, DEV, poison=False)
+        vals["q"] = (vals["q"].float() * mag).to(torch.bfloat16)
+        host = _host(vals)
+        out = _quant_step(wl, vals, ps=-1)
+        pa.pa_sync_check()
+        ref = _oracle_step(wl, host)
+        G.check_tolerance(G.to_f64(out), ref, "bf16", f"{fmt} |q|~{mag} H={H}/{Hkv}")
+        # the grouped consumer over the same (now appended) pool
+        d = G.device_tensors(wl, vals)
+        outg = torch.empty_like(vals["q"])
+        pa.pa_decode_grouped_quant(outg, vals["q"], vals["k_cache"], vals["v_cache"],
+                                   vals["k_scale"], vals["v_scale"], d["tables"], d["ctx"],
+                                   wl.scale, 2, max_context_len=wl.max_context_len,
+                                   partition_size=-1)
+        pa.pa_sync_check()
+        G.check_tolerance(G.to_f64(outg), ref, "bf16", f"{fmt} grouped |q|~{mag} H={H}/{Hkv}")

@@ -1,20 +1,26 @@
 """The grouped / multi-token decode on the tcgen05 consumer (pa_set_grouped_consumer):
-one thread issues 5th-generation tensor-core MMAs from shared memory with S, P
-and O in tensor memory. The same oracle parity, bitwise invariants and
-bounded-wait behaviour as the default consumer, re-run with this one selected
-(the test functions are those of the default consumer's modules)."""
+one thread issues 5th-generation tensor-core MMAs (S = Q K^T and O += P V, S and
+O in tensor memory, P in shared memory) for four softmax warps that split each
+64-token unit. The same oracle parity (full-size configurations included),
+bitwise invariants and bounded-wait behaviour as the default consumer, re-run
+with this one selected (the test functions are those of the default consumer's
+modules); shapes it does not take fall back to the default consumer."""
 import pytest
 import torch
 
 import paged_kv_cache_335_b200 as pa
 from paged_kv_cache_335_b200 import workloads as W
 from tests import gpu_helpers as G
-from tests.test_gpu_grouped import (test_cow_small_full_pool,  # noqa: F401
+from tests.test_gpu_grouped import (test_bad_block_id_is_reported,  # noqa: F401
+                                    test_cow_beam4_full_size,
+                                    test_cow_small_full_pool,
                                     test_deterministic_repeat,
                                     test_long_shared_context_many_partitions,
+                                    test_members_sharing_blocks_with_different_lengths,
                                     test_members_with_empty_contexts,
                                     test_placement_invariance_bitwise,
-                                    test_shared_equals_private_bitwise)
+                                    test_shared_equals_private_bitwise,
+                                    test_unshared_shape_sweep_edges)
 from tests.test_gpu_multi import (test_parity_shape_sweep,  # noqa: F401
                                   test_token_result_independent_of_the_other_tokens,
                                   test_verification_full_size)
