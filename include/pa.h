@@ -251,14 +251,19 @@ int pa_decode_grouped_num_partitions(int32_t num_seqs, int32_t num_heads,
  *     out[row][h] = softmax_{t <= p}(scale q[row][h] . K_t) . V
  * with K_t, V_t read through block_tables[s] exactly as in pa_decode.
  *
- *   q, out        device, [num_query_tokens][num_heads][head_dim], bf16.
+ *   q, out        device, [num_query_tokens][num_heads][head_dim], the cache's
+ *                 dtype (bf16 or fp32).
  *   query_start   device int32 [num_seqs + 1], non-decreasing, query_start[0]
  *                 = 0, query_start[num_seqs] = num_query_tokens (<= 65535).
- *   max_query_len host bound on n_s (>= 1). Tokens of one sequence are
- *                 decoded together in groups of up to 8 (at most 64 query
- *                 columns per group), so each block is read once per group.
+ *   max_query_len host bound on n_s (>= 1). Over bf16 caches the tokens of one
+ *                 sequence are decoded together in groups of up to 8 (at most
+ *                 64 query columns per group), so each block is read once per
+ *                 group; over fp32 caches (and for query groups above 64
+ *                 columns) each token is a row of its own on the CUDA-core
+ *                 consumer, which keeps the fp32 accuracy of pa_decode.
  *   workspace     at least pa_decode_multi_workspace_size(...) bytes.
- * Needs a bf16 cache with head_dim 64 or 128 (PA_ERR_UNSUPPORTED otherwise).
+ * Needs a bf16 or fp32 cache with head_dim 64 or 128 (PA_ERR_UNSUPPORTED
+ * otherwise).
  * n_s > context_lens[s] is recorded as PA_ERR_BAD_INDEX (those rows get 0).
  * A query token's result does not depend on the other tokens in the call (it
  * is bit-identical to a call holding only that token with the context cut at

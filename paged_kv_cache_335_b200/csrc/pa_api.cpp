@@ -173,12 +173,16 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
                         max_query_len, num_query_tokens);
         int gs = max_query_len < 8 ? max_query_len : 8;
         while (gs > 1 && gs * group > 64) --gs;
-        if (!pa::grouped_supported(c->dtype, c->head_dim, group, gs))
-            return fail(PA_ERR_UNSUPPORTED, "multi-token decode needs a bf16 cache at head_dim 64 "
-                        "or 128 or a quantised one at 128, and num_heads / num_kv_heads <= 64");
-        group_size = gs;
-        plan->q_chunks = (max_query_len + gs - 1) / gs;
-        plan->grouped = true;
+        if (pa::grouped_supported(c->dtype, c->head_dim, group, gs)) {
+            group_size = gs;
+            plan->q_chunks = (max_query_len + gs - 1) / gs;
+            plan->grouped = true;
+        } else {
+            // fp32 caches, or query groups above 64 columns: one query token per
+            // row of the CUDA-core consumer, which reads its sequence's blocks
+            group_size = 1;
+            plan->grouped = false;
+        }
     } else {
         plan->grouped =
             group_size > 1 && pa::grouped_supported(c->dtype, c->head_dim, group, group_size);
@@ -186,7 +190,8 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
     plan->group_size = group_size;
     if (plan->grouped && max_ctx > (1 << 27))
         return fail(PA_ERR_INVALID_ARG, "max_context_len %d above 2^27 on the grouped kernel", max_ctx);
-    plan->use_mma = pa::mma_supported(c->dtype, c->head_dim, group);
+    // the tensor-core GQA consumer takes one query row per sequence
+    plan->use_mma = !plan->multi && pa::mma_supported(c->dtype, c->head_dim, group);
     const int whole = round_up16(max_ctx > 16 ? max_ctx : 16);
     int ps = whole, np = 1;
     if (partition_size > 0) {
@@ -239,8 +244,8 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
             ps = np == 1 ? whole : (int)best_ps;
         } else {
             // The CUDA-core kernel is not persistent: split only when the
-            // (sequence, head) units alone cannot fill the GPU.
-            const long units = (long)num_seqs * num_heads;
+            // (row, head) units alone cannot fill the GPU.
+            const long units = (long)(plan->multi ? num_query_tokens : num_seqs) * num_heads;
             if (units < 4L * sm_count() && max_ctx > kAutoPartition) {
                 ps = kAutoPartition;
                 np = (max_ctx + ps - 1) / ps;

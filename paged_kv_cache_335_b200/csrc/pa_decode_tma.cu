@@ -354,13 +354,31 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
 
-    const int part = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    // grid z = rows of q / out: sequences, or with multi-token queries the query
+    // tokens, each of which reads its sequence's blocks up to its causal end
+    const int part = blockIdx.x, h = blockIdx.y, row = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ctx = clamp_ctx(__ldg(p.context_lens + s), p.max_context_len,
-                              threadIdx.x == 0 && part == 0);
+    int s = row, ctx;
+    if (p.query_start == nullptr) {
+        ctx = clamp_ctx(__ldg(p.context_lens + s), p.max_context_len, threadIdx.x == 0 && part == 0);
+    } else {
+        // the sequence holding query token `row`: query_start[s] <= row < query_start[s + 1]
+        int lo = 0, hi = p.num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldg(p.query_start + mid) <= row) lo = mid; else hi = mid - 1;
+        }
+        s = lo;
+        const int q0 = __ldg(p.query_start + s), n_new = __ldg(p.query_start + s + 1) - q0;
+        const bool report = threadIdx.x == 0 && part == 0 && h == 0;
+        const int lim = clamp_ctx(__ldg(p.context_lens + s), p.max_context_len, report && row == q0) -
+                        n_new + (row - q0) + 1;  // causal end of this query token
+        if (lim < 1 && report) atomicOr(&s_status_tma, kStatusBadIndex);  // more queries than context
+        ctx = lim < 1 ? 0 : lim;
+    }
     const int t0 = part * p.partition_size;
     const int t1 = min(ctx, t0 + p.partition_size);
-    const int64_t out_row = (int64_t)s * p.num_heads + h;
+    const int64_t out_row = (int64_t)row * p.num_heads + h;
     if (t0 >= t1) {
         if (p.num_partitions == 1)
             for (int d = threadIdx.x; d < D; d += kThreads) Elem<TQ>::store(p.out, out_row * D + d, 0.f);
@@ -2998,7 +3016,7 @@ cudaError_t launch_simt_t(const DecodeParams& p, const CUtensorMap& km, const CU
                              cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)p.num_partitions, (unsigned)p.num_heads, (unsigned)p.num_seqs);
+    dim3 grid((unsigned)p.num_partitions, (unsigned)p.num_heads, (unsigned)p.num_rows);
     decode_tma_simt_kernel<T, D><<<grid, G::kThreads, smem, stream>>>(km, vm, p);
     return cudaGetLastError();
 }

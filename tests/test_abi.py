@@ -132,8 +132,11 @@ def test_multi_query_policy_and_arguments(lib):
     assert f(8, 32, 0, 64, 32768, ctypes.byref(d70), 0) == pa.PA_ERR_INVALID_ARG   # max_query_len
     assert f(8, 32, 33, 64, 32768, ctypes.byref(d70), 0) == pa.PA_ERR_INVALID_ARG
     assert f(8, -1, 1, 64, 32768, ctypes.byref(d70), 0) == pa.PA_ERR_INVALID_ARG
+    # fp32: one CUDA-core row per query token; 32 rows x 64 heads fill the GPU unsplit
     f32 = _desc(num_kv_heads=8, dtype=pa.PA_F32)
-    assert f(8, 32, 4, 64, 32768, ctypes.byref(f32), 0) == pa.PA_ERR_UNSUPPORTED
+    assert f(8, 32, 4, 64, 32768, ctypes.byref(f32), 0) == 1
+    assert f(8, 32, 4, 64, 32768, ctypes.byref(f32), 512) == 64
+    assert f(8, 32, 4, 64, 32768, ctypes.byref(_desc(num_kv_heads=8, dtype=7)), 0) == pa.PA_ERR_DTYPE
     p = ctypes.c_void_p(256)
     rc = lib.pa_decode_multi(p, p, p, p, p, 8, p, None, 100, 2, 4, 2, 64, ctypes.c_float(0.1),
                              ctypes.byref(d70), -1, None, 0, None)

@@ -4,7 +4,7 @@ Each sequence appends n_s tokens this step and every one of them attends
 causally over the paged cache (chunked prefill, verification of draft tokens).
 Bars: appended slots bit-exact; outputs within the bf16 tolerance of the
 unrounded oracle; a query token's result bit-identical whether or not other
-tokens share the call; bad inputs reported, unsupported dtypes refused.
+tokens share the call; bad inputs reported. fp32 caches meet the fp32 bar.
 """
 import numpy as np
 import pytest
@@ -120,13 +120,64 @@ def test_more_queries_than_context_reported():
     assert e.value.code == pa.PA_ERR_BAD_INDEX
 
 
-def test_f32_cache_is_refused():
-    wl = W.tiny()
+@pytest.mark.parametrize("d,bs", [(64, 16), (128, 32)])
+@pytest.mark.parametrize("H,Hkv", [(4, 4), (16, 2), (12, 3)])
+def test_f32_cache_parity(d, bs, H, Hkv):
+    """fp32 caches: each query token is a row of its own on the CUDA-core consumer
+    (it reads its sequence's blocks up to its causal end); the fp32 bar of
+    pa_decode (row-normwise relative error <= 1e-5) holds, split or not."""
+    wl = W.multi_query_case(len(CTX), H, Hkv, d, bs, "f32", CTX, NQ, seed=d + bs + H + 1)
+    for ps in (-1, 0, 64):
+        vals = W.make_values(wl, DEV, poison=True)
+        host = G.host_copy(vals)
+        d_ = G.device_tensors(wl, vals)
+        pa.pa_kv_append(vals["k_new"], vals["v_new"], d_["slots"], vals["k_cache"],
+                        vals["v_cache"])
+        out = _multi(wl, vals, ps)
+        pa.pa_sync_check()
+        assert G.last_kernel() == pa.PA_KERNEL_SIMT
+        oracle.kv_append(host["k_new"], host["v_new"], wl.slot_mapping, host["k_cache"],
+                         host["v_cache"])
+        assert G.bits_equal(vals["k_cache"], host["k_cache"])
+        ref = oracle.decode_multi(host["q"], host["k_cache"], host["v_cache"], wl.block_tables,
+                                  wl.context_lens, wl.query_start, wl.scale,
+                                  num_threads=G.THREADS)
+        errs = G.check_tolerance(G.to_f64(out), ref, "f32", f"f32 multi ps={ps}")
+        assert errs["row_rel"] <= G.F32_ROW_REL
+
+
+def test_f32_more_queries_than_context_reported():
+    """A sequence with more new tokens than context positions (not a valid step)
+    on the fp32 path: reported, and the token without any position gets 0."""
+    wl = W.multi_query_case(2, 4, 4, 64, 16, "f32", [40, 30], [3, 2], seed=1)
     vals = W.make_values(wl, DEV)
     d = G.device_tensors(wl, vals)
-    qs = torch.arange(wl.num_seqs + 1, dtype=torch.int32, device=DEV)
+    out = torch.full_like(vals["q"], float("nan"))
+    pa.pa_sync_check()
+    qs = torch.tensor([0, 3, 5], dtype=torch.int32, device=DEV)
+    d["ctx"][1] = 1                                          # 2 queries, 1 context position
+    pa.pa_decode_multi(out, vals["q"], vals["k_cache"], vals["v_cache"], d["tables"], d["ctx"], qs,
+                       wl.scale, max_context_len=40, max_query_len=3, partition_size=-1)
     with pytest.raises(pa.PAError) as e:
-        pa.pa_decode_multi(torch.empty_like(vals["q"]), vals["q"], vals["k_cache"], vals["v_cache"],
-                           d["tables"], d["ctx"], qs, wl.scale, max_context_len=wl.max_context_len,
-                           max_query_len=1)
-    assert e.value.code == pa.PA_ERR_UNSUPPORTED
+        pa.pa_sync_check()
+    assert e.value.code == pa.PA_ERR_BAD_INDEX
+    assert G.last_kernel() == pa.PA_KERNEL_SIMT
+    assert torch.equal(out[3], torch.zeros_like(out[3]))      # causal end 0: nothing to attend
+    assert torch.isfinite(out).all()
+
+
+def test_bf16_query_groups_above_64_columns():
+    """A query group of 128 heads per kv head: too many columns for the grouped
+    kernel, so every query token takes a CUDA-core row of its own."""
+    wl = W.multi_query_case(3, 128, 1, 128, 16, "bf16", [70, 33, 300], [3, 1, 5], seed=5)
+    vals = W.make_values(wl, DEV, poison=True)
+    host = G.host_copy(vals)
+    d_ = G.device_tensors(wl, vals)
+    pa.pa_kv_append(vals["k_new"], vals["v_new"], d_["slots"], vals["k_cache"], vals["v_cache"])
+    out = _multi(wl, vals, 0)
+    pa.pa_sync_check()
+    assert G.last_kernel() == pa.PA_KERNEL_SIMT
+    oracle.kv_append(host["k_new"], host["v_new"], wl.slot_mapping, host["k_cache"], host["v_cache"])
+    ref = oracle.decode_multi(host["q"], host["k_cache"], host["v_cache"], wl.block_tables,
+                              wl.context_lens, wl.query_start, wl.scale, num_threads=G.THREADS)
+    G.check_tolerance(G.to_f64(out), ref, "bf16", "128 heads per kv head")
