@@ -311,12 +311,13 @@ int pa_decode_multi_num_partitions(int32_t num_seqs, int32_t num_query_tokens,
  * pa_decode_quant — pa_decode over a quantised cache: the same attention with
  * K_t and V_t the cached values above (the K scale folds into the scores, the
  * V scale into the output). Arguments as pa_decode plus the two scale arrays;
- * head_dim 128 (PA_ERR_UNSUPPORTED otherwise); workspace sized by
- * pa_decode_workspace_size with the quantised descriptor. Precision: the
- * products run with q rounded to f16 (exact for bf16 magnitudes from 2^-14
- * to 65504; larger q is outside this call's range) and the softmax weights
- * rounded to f16, accumulated in fp32; results
- * meet the bf16 bars of pa_decode. pa_decode,
+ * head_dim 64 or 128; workspace sized by pa_decode_workspace_size with the
+ * quantised descriptor. Precision: the products run with q rounded to f16
+ * after a power-of-two shift that puts the largest |q| of the q values a warp
+ * holds in [2^14, 2^15) (the scores are shifted back after the products; both
+ * exact, so any bf16 q within 2^29 of that largest one is rounded exactly,
+ * whatever its magnitude) and the softmax weights rounded to f16, accumulated
+ * in fp32; results meet the bf16 bars of pa_decode. pa_decode,
  * pa_kv_append and the other decode calls refuse a quantised descriptor
  * (PA_ERR_DTYPE), and these two refuse an unquantised one.
  */
@@ -337,7 +338,7 @@ int pa_decode_quant(void* out, const void* q, const void* k_cache, const void* v
  * pa_decode_grouped_quant / pa_decode_multi_quant — pa_decode_grouped and
  * pa_decode_multi over a quantised cache (the two compositions of the calls
  * above): arguments as those calls plus k_scale, v_scale after v_cache; the
- * precision of pa_decode_quant; head_dim 128. Workspace and partitions as
+ * precision of pa_decode_quant; head_dim 64 or 128. Workspace and partitions as
  * pa_decode_grouped_workspace_size / pa_decode_multi_workspace_size (and the
  * _num_partitions queries) with the quantised descriptor. Grouped and
  * multi-token decode are the same computation as pa_decode_quant: a group's
@@ -363,19 +364,19 @@ int pa_decode_multi_quant(void* out, const void* q, const void* k_cache, const v
 
 /*
  * pa_set_grouped_consumer — which consumer pa_decode_grouped and pa_decode_multi
- * use for bf16 head_dim 128 with 16..64 query columns (sequences or query
+ * use for bf16 head_dim 128 with 8..32 query columns (sequences or query
  * tokens x query heads per kv head):
- *   PA_GROUPED_MMA_SYNC (default): one warp per 8 query columns, m16n8k16 MMAs
- *     from registers;
- *   PA_GROUPED_TCGEN05: one thread issues tcgen05.mma from shared memory with
- *     S, P and O in tensor memory, softmax warps read and write TMEM.
+ *   PA_GROUPED_MMA_SYNC: one warp per 8 query columns, m16n8k16 MMAs from
+ *     registers;
+ *   PA_GROUPED_TCGEN05: one thread issues tcgen05.mma (S = Q K^T and O += P V,
+ *     S and O in tensor memory, P in shared memory) for four softmax warps
+ *     that split each 64-token unit.
  * Both compute the same attention within the same tolerance of the exact
  * value, and both keep a sequence's result independent of which blocks it
- * shares; they round differently from each other. On the measured beam and
- * verification workloads the default is faster (decode-sized contractions
- * leave the single-issuer pipeline latency-bound). Process-wide, not
- * synchronised with calls in flight on other threads: set it before decoding.
- * Returns the previous consumer, or PA_ERR_INVALID_ARG for an unknown value.
+ * shares; they round differently from each other. Other shapes always take
+ * the mma.sync consumer. The setting belongs to the calling host thread (each
+ * thread starts with the default). Returns the previous consumer, or
+ * PA_ERR_INVALID_ARG for an unknown value.
  */
 #define PA_GROUPED_MMA_SYNC 0
 #define PA_GROUPED_TCGEN05 1

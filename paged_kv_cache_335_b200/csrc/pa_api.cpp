@@ -108,7 +108,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // The pool as a 2-D tensor [num_blocks * num_kv_heads * block_size rows][head_dim],
-// loaded in boxes of 16 rows x 128 bytes with the 128-byte swizzle.
+// loaded in boxes of 16 rows x 128 bytes with the 128-byte swizzle. A head_dim 64
+// pool of one-byte codes has 64-byte rows: its box still spans 128 codes, the TMA
+// fills the 64 past the row's end with zero codes without reading memory, and
+// the consumers over codes (built for 128-code rows) take the padding as zeros.
 int make_cache_map(CUtensorMap* map, const void* base, const pa_cache_desc* c) {
     auto fn = encode_fn();
     if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
@@ -305,9 +308,6 @@ static int decode_impl(void* out, const void* q, const void* k_cache, const void
             (reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
             return fail(PA_ERR_INVALID_ARG, "pa_decode_quant: k_scale and v_scale must be 4-byte "
                         "aligned device arrays of num_kv_heads floats");
-        if (cache->head_dim != 128)
-            return fail(PA_ERR_UNSUPPORTED, "quantised caches decode at head_dim 128 (got %d)",
-                        cache->head_dim);
     }
     if (num_query_tokens > 65535)
         return fail(PA_ERR_INVALID_ARG, "num_query_tokens %d above 65535", num_query_tokens);
@@ -362,6 +362,7 @@ static int decode_impl(void* out, const void* q, const void* k_cache, const void
     p.test_skip_position = g_test_skip_position;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
+    p.head_dim = cache->head_dim;
     p.query_start = plan.multi ? query_start : nullptr;
     p.q_chunks = plan.q_chunks;
     p.num_rows = plan.multi ? num_query_tokens : num_seqs;

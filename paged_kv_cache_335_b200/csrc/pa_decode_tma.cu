@@ -379,9 +379,10 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
     const int t0 = part * p.partition_size;
     const int t1 = min(ctx, t0 + p.partition_size);
     const int64_t out_row = (int64_t)row * p.num_heads + h;
+    const int DQ = kCodes ? p.head_dim : D;  // q / out head_dim (codes: 64 or 128)
     if (t0 >= t1) {
         if (p.num_partitions == 1)
-            for (int d = threadIdx.x; d < D; d += kThreads) Elem<TQ>::store(p.out, out_row * D + d, 0.f);
+            for (int d = threadIdx.x; d < DQ; d += kThreads) Elem<TQ>::store(p.out, out_row * DQ + d, 0.f);
         return;
     }
     const int kh = h / (p.num_heads / p.num_kv_heads);
@@ -420,7 +421,9 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
         for (int u = 0; u < VEC / QV; ++u) {
             float f[QV];
-            Elem<TQ>::widen(ld_v4(static_cast<const TQ*>(p.q) + out_row * D + c * VEC + u * QV), f);
+            const int d0 = c * VEC + u * QV;
+            Elem<TQ>::widen(d0 < DQ ? ld_v4(static_cast<const TQ*>(p.q) + out_row * DQ + d0)
+                                    : make_uint4(0u, 0u, 0u, 0u), f);
 #pragma unroll
             for (int j = 0; j < QV; ++j) qf[u * QV + j] = kMixed ? f[j] : f[j] * qs;
         }
@@ -586,16 +589,16 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
         L = fmaf(sm_l[w], wgt[w], L);
     }
     const float vs = p.v_scale != nullptr ? __ldg(p.v_scale + kh) : 1.f;
-    for (int d = threadIdx.x; d < D; d += kThreads) {
+    for (int d = threadIdx.x; d < DQ; d += kThreads) {
         float o = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) o = fmaf(sm_o[w * D + d], wgt[w], o);
         float val = L > 0.f ? o / L : 0.f;
         if (p.v_scale != nullptr) val *= vs;  // V scale of a quantised cache
         if (p.num_partitions == 1)
-            Elem<TQ>::store(p.out, out_row * D + d, val);
+            Elem<TQ>::store(p.out, out_row * DQ + d, val);
         else
-            p.ws_o[(out_row * p.num_partitions + part) * D + d] = val;
+            p.ws_o[(out_row * p.num_partitions + part) * DQ + d] = val;
     }
     if (p.num_partitions > 1 && threadIdx.x == 0) {
         float* ml = p.ws_ml + (out_row * p.num_partitions + part) * 2;
@@ -810,10 +813,12 @@ __device__ __forceinline__ uint32_t code_word(uint32_t w) {
 // q row of the B operand for codes: head_dim 32c .. 32c+31 as raw bf16 words
 // (zeros without a row), their largest magnitude, and their conversion to 16
 // f16x2 words of q * mul (mul a signed power of two: exact).
-__device__ __forceinline__ void load_q_raw(const uint16_t* qrow, int c, uint4 (&raw)[4]) {
+// (head_dim positions at or past dq, the padding of a head_dim 64 pool, are zero).
+__device__ __forceinline__ void load_q_raw(const uint16_t* qrow, int c, uint4 (&raw)[4], int dq) {
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-        raw[u] = qrow != nullptr ? ld_v4(qrow + 32 * c + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
+        raw[u] = qrow != nullptr && 32 * c + 8 * u < dq ? ld_v4(qrow + 32 * c + 8 * u)
+                                                        : make_uint4(0u, 0u, 0u, 0u);
 }
 __device__ __forceinline__ float q_raw_amax(const uint4 (&raw)[4]) {
     uint32_t m = 0;
@@ -940,6 +945,7 @@ __device__ __forceinline__ void mma_store_item(const DecodeParams& p, int64_t he
                                                float vs = 1.f) {
     constexpr int MT = D / 16;
     const int P = p.num_partitions;
+    const int DQ = kCodes ? p.head_dim : D;  // out / workspace row length
     float inv0 = l0 > 0.f ? 1.f / l0 : 0.f;
     float inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
     if constexpr (kCodes) {
@@ -950,19 +956,20 @@ __device__ __forceinline__ void mma_store_item(const DecodeParams& p, int64_t he
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
         const int d0 = kCodes ? 16 * r + 2 * t : (t >> 2) * 64 + r * 8 + 2 * (t & 3);
+        if (d0 >= DQ) continue;  // padding of a head_dim 64 pool of codes
         if (P == 1) {
             if (n0 < group)
-                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + (head0 + n0) * D + d0) =
+                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + (head0 + n0) * DQ + d0) =
                     pack_bf16x2(acc[t][0] * inv0, acc[t][2] * inv0);
             if (n1 < group)
-                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + (head0 + n1) * D + d0) =
+                *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + (head0 + n1) * DQ + d0) =
                     pack_bf16x2(acc[t][1] * inv1, acc[t][3] * inv1);
         } else {
             if (n0 < group)
-                *reinterpret_cast<float2*>(p.ws_o + ((head0 + n0) * P + part) * D + d0) =
+                *reinterpret_cast<float2*>(p.ws_o + ((head0 + n0) * P + part) * DQ + d0) =
                     make_float2(acc[t][0] * inv0, acc[t][2] * inv0);
             if (n1 < group)
-                *reinterpret_cast<float2*>(p.ws_o + ((head0 + n1) * P + part) * D + d0) =
+                *reinterpret_cast<float2*>(p.ws_o + ((head0 + n1) * P + part) * DQ + d0) =
                     make_float2(acc[t][1] * inv1, acc[t][3] * inv1);
         }
     }
@@ -1137,10 +1144,11 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
     auto load_q = [&](const Item& it, uint4 (&q)[KCH]) {
         const int64_t head0 = (int64_t)it.s * p.num_heads + (int64_t)it.kh * group;
         if (it.valid && it.t0 < it.t1 && r < group) {
-            const uint16_t* qrow = static_cast<const uint16_t*>(p.q) + (head0 + r) * D;
             if constexpr (kCodes) {
-                load_q_raw(qrow, c, q);
+                load_q_raw(static_cast<const uint16_t*>(p.q) + (head0 + r) * p.head_dim, c, q,
+                           p.head_dim);
             } else {
+                const uint16_t* qrow = static_cast<const uint16_t*>(p.q) + (head0 + r) * D;
 #pragma unroll
                 for (int jp = 0; jp < KCH; ++jp)
                     q[jp] = ld_v4(qrow + (jp >> 1) * 64 + (2 * c + (jp & 1)) * 8);
@@ -1166,9 +1174,10 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         const int64_t head0 = (int64_t)cur.s * p.num_heads + (int64_t)cur.kh * group;
         if (cur.t0 >= cur.t1) {
+            const int DQ = kCodes ? p.head_dim : D;
             if (P == 1)
-                for (int idx = threadIdx.x; idx < group * D; idx += kConsumerWarps * 32)
-                    Elem<T>::store(p.out, head0 * D + idx, 0.f);
+                for (int idx = threadIdx.x; idx < group * DQ; idx += kConsumerWarps * 32)
+                    Elem<T>::store(p.out, head0 * DQ + idx, 0.f);
         } else {
             const int t0 = cur.t0, t1 = cur.t1;
             const int n_sub = (t1 - t0 + 15) >> 4;
@@ -2126,18 +2135,20 @@ __device__ __forceinline__ void grouped_store_col(const DecodeParams& p, int64_t
                                                   float m, float l, float vs = 1.f) {
     constexpr int MT = D / 16;
     const int P = p.num_partitions;
+    const int DQ = kCodes ? p.head_dim : D;  // out / workspace row length
     const float inv = (l > 0.f ? 1.f / l : 0.f) * vs;  // vs: V scale of a quantised cache
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
         // rows r and r + 8 of m-tile t: head_dim 16t + r and 16t + 8 + r (codes:
-        // 16r + 2t and 16r + 2t + 1)
+        // 16r + 2t and 16r + 2t + 1; at or past DQ: padding, not stored)
         const int d0 = kCodes ? 16 * r + 2 * t : 16 * t + r, d1 = kCodes ? d0 + 1 : d0 + 8;
+        if (kCodes && d0 >= DQ) continue;
         if (P == 1) {
-            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + row * D;
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + row * DQ;
             o[d0] = __float2bfloat16_rn(acc[t][e] * inv);
             o[d1] = __float2bfloat16_rn(acc[t][e + 2] * inv);
         } else {
-            float* o = p.ws_o + (row * P + part) * D;
+            float* o = p.ws_o + (row * P + part) * DQ;
             o[d0] = acc[t][e] * inv;
             o[d1] = acc[t][e + 2] * inv;
         }
@@ -2164,6 +2175,7 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
     constexpr int KCH = D / 32;
     constexpr int MT = D / 16;
     constexpr int kUnitTokens = 16 * SUB;
+    const int DQ = kCodes ? p.head_dim : D;  // q / out head_dim (codes: 64 or 128)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
 
@@ -2251,9 +2263,9 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             const uint16_t* qrow = nullptr;
             if (it.valid && m < gs && m < it.nmem && t1 > it.t0)
                 qrow = static_cast<const uint16_t*>(p.q) +
-                       ((int64_t)(it.row0 + m) * p.num_heads + (int64_t)it.kh * group + hd) * D;
+                       ((int64_t)(it.row0 + m) * p.num_heads + (int64_t)it.kh * group + hd) * DQ;
             if constexpr (kCodes) {
-                load_q_raw(qrow, c, q[j]);
+                load_q_raw(qrow, c, q[j], DQ);
             } else {
                 const uint32_t sg = neg ? 0x80008000u : 0u;
 #pragma unroll
@@ -3134,7 +3146,7 @@ int mma_ctas_per_sm() { return PA_MMA_MIN_BLOCKS; }
 // codes the tensor-core one with one MMA column of eight measured slower on
 // B200 (13B MHA: fp8 564 vs 536 us, int8 661 vs 622 us; 7B fp8 173 vs 125 us).
 bool mma_supported(int dtype, int head_dim, int group) {
-    const bool codes = (dtype == 2 || dtype == 3) && head_dim == 128;
+    const bool codes = (dtype == 2 || dtype == 3) && (head_dim == 64 || head_dim == 128);
     return (codes || (dtype == 1 && (head_dim == 64 || head_dim == 128))) && group >= 2 &&
            group <= kGroupMax;
 }
@@ -3143,7 +3155,7 @@ bool mma_supported(int dtype, int head_dim, int group) {
 // tcgen05 consumer takes head_dim 128 with 8..32 query columns (its 128-row
 // MMAs hold four copies of up to 32 columns; with fewer than 8 they would mostly
 // idle); other shapes stay on mma.sync.
-static int g_grouped_consumer = PA_GROUPED_MMA_SYNC;
+static thread_local int g_grouped_consumer = PA_GROUPED_MMA_SYNC;  // per host thread
 
 static bool use_umma(int head_dim, int gs, int group) {
     return g_grouped_consumer == PA_GROUPED_TCGEN05 && head_dim == 128 && gs * group >= 8 &&
@@ -3158,10 +3170,10 @@ static void grouped_shape(int gs, int group, int* cw, int* nt) {
     *cw = (tiles + *nt - 1) / *nt;
 }
 
-// bf16 at head_dim 64 or 128; quantised codes (PA_FP8_E4M3, PA_INT8) at 128.
+// bf16 or quantised codes (PA_FP8_E4M3, PA_INT8) at head_dim 64 or 128 (codes
+// at 64 on the 128-code consumer, rows zero-filled past 64).
 bool grouped_supported(int dtype, int head_dim, int group, int gs) {
-    const bool shape = (dtype == 1 && (head_dim == 64 || head_dim == 128)) ||
-                       ((dtype == 2 || dtype == 3) && head_dim == 128);
+    const bool shape = (dtype == 1 || dtype == 2 || dtype == 3) && (head_dim == 64 || head_dim == 128);
     return shape && gs >= 1 && gs <= kMaxGroupSeqs && group >= 1 && gs * group <= kGroupedMaxCols;
 }
 

@@ -50,6 +50,10 @@ struct DecodeParams {
     // nullptr for bf16 / f32 caches.
     const float* k_scale;
     const float* v_scale;
+    // head_dim of q / out / the workspace rows. The consumers over codes are
+    // built for 128-code rows and take head_dim 64 pools as rows whose upper
+    // half the TMA fills with zero codes (q zero there too, outputs not stored).
+    int32_t head_dim;
 };
 
 struct CopyParams {

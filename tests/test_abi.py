@@ -157,7 +157,10 @@ def test_quantised_grouped_and_multi_arguments(lib):
                  gs, -1, None, 0, None)
     assert grouped(fp8, ks=None) == pa.PA_ERR_INVALID_ARG
     assert grouped(bf16) == pa.PA_ERR_DTYPE
-    assert grouped(_desc(num_kv_heads=2, dtype=pa.PA_INT8, head_dim=64)) == pa.PA_ERR_UNSUPPORTED
+    assert grouped(_desc(num_kv_heads=2, dtype=pa.PA_INT8, head_dim=96)) == pa.PA_ERR_UNSUPPORTED
+    # head_dim 64 over codes is accepted: its partition query answers without a GPU
+    assert lib.pa_decode_grouped_num_partitions(8, 16, 100, ctypes.byref(
+        _desc(num_kv_heads=2, dtype=pa.PA_INT8, head_dim=64)), 4, -1) == 1
     assert grouped(fp8, gs=9) == pa.PA_ERR_INVALID_ARG
     m = lib.pa_decode_multi_quant
     rc = m(p, p, p, p, p, p, p, 8, p, None, 100, 2, 4, 2, 16, ctypes.c_float(0.1),

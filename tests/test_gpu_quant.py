@@ -59,9 +59,14 @@ def _host(vals):
 @pytest.mark.parametrize("fmt", ["fp8", "int8"])
 @pytest.mark.parametrize("H,Hkv", [(8, 8), (16, 2), (12, 3), (32, 2)])
 @pytest.mark.parametrize("bs", [16, 64])
-def test_step_parity_edges(fmt, H, Hkv, bs):
+@pytest.mark.parametrize("d", [64, 128])
+def test_step_parity_edges(fmt, H, Hkv, bs, d):
+    """Contexts at block and partition edges (0 included) on the CUDA-core (MHA,
+    group 16) and tensor-core (group 2..8) consumers over codes, head_dim 64
+    (64-code rows read as 128-code rows whose upper half the TMA zero-fills) and
+    128; appended codes bit-exact."""
     ctx = [0, 1, 2, 15, 16, 17, 33, 64, 129, 511, 513, 1000]
-    wl = W.quantized(G.custom(len(ctx), H, Hkv, 128, bs, "bf16", ctx, seed=bs + H), fmt)
+    wl = W.quantized(G.custom(len(ctx), H, Hkv, d, bs, "bf16", ctx, seed=bs + H + d), fmt)
     for ps in (-1, 64, 0):
         vals = W.make_values(wl, DEV, poison=True)
         host = _host(vals)
@@ -164,14 +169,13 @@ def test_wrong_descriptor_kind_refused():
                           P(d["slots"].data_ptr()), 2, P(vals["k_cache"].data_ptr()),
                           P(vals["v_cache"].data_ptr()), ctypes.byref(desc), None)
     assert rc == pa.PA_ERR_DTYPE                       # codes need pa_kv_append_quant
-    wl64 = W.quantized(G.custom(2, 8, 8, 64, 16, "bf16", [20, 30], seed=2), "fp8")
-    v64 = W.make_values(wl64, DEV)
-    d64 = G.device_tensors(wl64, v64)
-    with pytest.raises(pa.PAError) as e:
-        pa.pa_decode_quant(torch.empty_like(v64["q"]), v64["q"], v64["k_cache"], v64["v_cache"],
-                           v64["k_scale"], v64["v_scale"], d64["tables"], d64["ctx"], wl64.scale,
-                           max_context_len=30)
-    assert e.value.code == pa.PA_ERR_UNSUPPORTED
+    wl3 = W.quantized(G.custom(2, 8, 8, 128, 16, "bf16", [20, 30], seed=2), "fp8")
+    v3 = W.make_values(wl3, DEV)
+    d3 = G.device_tensors(wl3, v3)
+    with pytest.raises(TypeError):             # q must be bf16 over a quantised cache
+        pa.pa_decode_quant(torch.empty_like(v3["q"]).float(), v3["q"].float(), v3["k_cache"],
+                           v3["v_cache"], v3["k_scale"], v3["v_scale"], d3["tables"], d3["ctx"],
+                           wl3.scale, max_context_len=30)
 
 
 @pytest.mark.parametrize("fmt", ["fp8", "int8"])

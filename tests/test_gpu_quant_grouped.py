@@ -90,10 +90,12 @@ def test_grouped_cow_parity(fmt, gs, ps):
 
 @pytest.mark.parametrize("fmt", ["fp8", "int8"])
 @pytest.mark.parametrize("H,Hkv", [(8, 8), (16, 4), (12, 3)])
-def test_grouped_unshared_edges(fmt, H, Hkv):
-    """Unrelated sequences grouped, contexts at block and unit edges including 0."""
+@pytest.mark.parametrize("d", [64, 128])
+def test_grouped_unshared_edges(fmt, H, Hkv, d):
+    """Unrelated sequences grouped, contexts at block and unit edges including 0,
+    head_dim 64 (zero-filled halves of 128-code rows) and 128."""
     ctx = [0, 1, 15, 16, 17, 63, 64, 65, 129, 300, 511, 513]
-    wl = W.quantized(G.custom(len(ctx), H, Hkv, 128, 16, "bf16", ctx, seed=H + 7), fmt)
+    wl = W.quantized(G.custom(len(ctx), H, Hkv, d, 16, "bf16", ctx, seed=H + 7 + d), fmt)
     for ps in (-1, 64):
         vals = W.make_values(wl, DEV, poison=True)
         host = _host(vals)
@@ -139,11 +141,11 @@ def test_grouped_shared_equals_private_bitwise(fmt):
 
 
 @pytest.mark.parametrize("fmt", ["fp8", "int8"])
-@pytest.mark.parametrize("H,Hkv", [(8, 8), (16, 2), (64, 8)])
-def test_multi_parity(fmt, H, Hkv):
+@pytest.mark.parametrize("H,Hkv,d", [(8, 8, 128), (16, 2, 128), (64, 8, 128), (16, 2, 64)])
+def test_multi_parity(fmt, H, Hkv, d):
     """Query counts from 0 to a 300-token chunk, contexts at block and partition
     edges; each query token against the oracle at its causal end."""
-    wl = W.quantized(W.multi_query_case(len(CTX), H, Hkv, 128, 16, "bf16", CTX, NQ, seed=H + 3),
+    wl = W.quantized(W.multi_query_case(len(CTX), H, Hkv, d, 16, "bf16", CTX, NQ, seed=H + 3 + d),
                      fmt)
     tables_r, ctx_r = _multi_rows(wl)
     for ps in (-1, 0, 64):
