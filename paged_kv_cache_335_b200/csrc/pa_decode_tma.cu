@@ -2404,11 +2404,11 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
-// Instruction descriptor for kind::f16: fp32 accumulator, bf16 A and B, A
-// K-major, B K-major or MN-major, shape M x N.
-__host__ __device__ constexpr uint32_t umma_idesc(int m, int n, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+// Instruction descriptor for kind::f16: fp32 accumulator, bf16 (or, with
+// f16, f16) A and B, A K-major, B K-major or MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t umma_idesc(int m, int n, bool b_mn_major, bool f16 = false) {
+    return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) |
+           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 // D (TMEM) (+)= A (shared) . B (shared)^T, issued by one thread.
 __device__ __forceinline__ void umma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
@@ -2475,16 +2475,24 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 }
 
 // ---------------------------------------------------------------------------
-// Grouped and multi-token decode on the 5th-generation tensor cores (bf16,
-// head_dim 128, at most 32 query columns (member, head) per item).
+// Grouped and multi-token decode on the 5th-generation tensor cores (head_dim
+// 128, at most 32 query columns (member, head) per item; bf16 caches, or
+// FP8 E4M3 / int8 codes converted to f16 in shared memory).
 // Same work items as decode_tma_grouped_kernel, with 64-token units: four
 // 16-token sub-tiles of one distinct block sequence, a header per stage
 // (member mask, unit index, last-unit flag) and the unit's largest valid
 // token count over its members. Roles:
-//   warp 4: the producer. A stage holds the unit's K as two d-halves of 64
-//     rows x 128 bytes (128-byte swizzle), then its V the same way, so each
-//     is one canonical operand tile; K and V complete on barriers of their
-//     own, so S = Q K^T can start while V is still landing;
+//   warp 4: the producer. Over bf16 a stage holds the unit's K as two
+//     d-halves of 64 rows x 128 bytes (128-byte swizzle), then its V the same
+//     way, so each is one canonical operand tile; K and V complete on barriers
+//     of their own, so S = Q K^T can start while V is still landing. Over
+//     codes a stage holds the 64 rows of 128 codes of K, then of V;
+//   warps 6 and 7 (codes only): the converters. They turn a unit's codes into
+//     an f16 K tile and an f16 V tile laid out as the bf16 stage (exact: every
+//     E4M3 and int8 value is an f16), V rows past every member's tokens as
+//     zeros, copy the unit's header into one of four slots, and release the
+//     stage; the K tile is rewritten once the previous unit's QK is done, the
+//     V tile once its PV is;
 //   warp 5, lane 0: per unit S = Q . K^T (M = 128 rows, N = 64 tokens,
 //     K = 128: 8 tcgen05.mma kind::f16 steps, S in TMEM, double-buffered) and
 //     O += P . V (A = P from shared memory, B = V read MN-major; M = 128,
@@ -2502,11 +2510,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 // slice maxima through shared memory, and warp 0 (whose TMEM lanes hold O's
 // rows) rescales O. A column's decisions depend only on its own scores in
 // logical order, so its result is the same whichever blocks it shares and
-// whichever members share its CTA. P (bf16, row = column, 64 tokens) goes to a
-// double-buffered shared tile that the PV MMA reads. V rows past every
-// member's tokens are zeroed before the PV MMA reads them. Every wait is
-// bounded; a give-up is agreed by the softmax warps at the next per-unit vote,
-// and TMEM is freed after a final commit on every path.
+// whichever members share its CTA. P (bf16, or f16 beside codes; row =
+// column, 64 tokens) goes to a double-buffered shared tile that the PV MMA
+// reads. Over codes q is rounded to f16 after a power-of-two shift of its own
+// column (q_shift_warp's rule per row), undone in the column's score scale,
+// and the K and V scales fold into the score scale and the output. Every wait
+// is bounded; a give-up is agreed by the softmax warps at the next per-unit
+// vote, and TMEM is freed after a final commit on every path.
 // ---------------------------------------------------------------------------
 constexpr int kU2Tokens = 64;                   // tokens per unit
 constexpr int kU2Cols = 32;                     // query columns per item, at most
@@ -2515,16 +2525,15 @@ constexpr int kU2HalfBytes = kU2Tokens * 128;   // one d-half of a K or V tile: 
 #ifndef PA_U2_STAGES
 #define PA_U2_STAGES 2
 #endif
-constexpr int kU2PBytes = kU2Cols * 128;        // P tile: 32 rows x 64 bf16 tokens
-constexpr int kU2QBytes = 2 * 128 * 128;        // Q tile: 128 rows x 128 bf16, two d-halves
+constexpr int kU2PBytes = kU2Cols * 128;        // P tile: 32 rows x 64 16-bit tokens
+constexpr int kU2QBytes = 2 * 128 * 128;        // Q tile: 128 rows x 128 16-bit, two d-halves
 constexpr int kU2QOff = 2 * kU2PBytes;          // shared memory: [P0][P1][Q][ring][...]
 constexpr int kU2RingOff = kU2QOff + kU2QBytes;
 constexpr uint32_t kU2TmemCols = 256;
 constexpr uint32_t kU2ColO = 0, kU2ColS = 128;  // S buffers at columns 128 and 192
 constexpr float kU2RescaleLog2 = 8.f;
-constexpr uint32_t kU2IdescQK = umma_idesc(128, 64, false);
-constexpr uint32_t kU2IdescPV = umma_idesc(128, 128, true);
 
+// Ring of the bf16 variant: box-major stages with K and V barriers of their own.
 struct U2Geom {
     using T = __nv_bfloat16;
     static constexpr bool kU2 = true;
@@ -2537,26 +2546,45 @@ struct U2Geom {
     static constexpr int kStageBytes = 4 * kU2HalfBytes;  // K halves, then V halves: 32 KB
     static constexpr int kRingBytes = kStages * kStageBytes;
 };
-static_assert(kU2RingOff % 1024 == 0, "ring stages on 1024-byte boundaries");
-// the PV MMA reads 128 rows (16 KB) of a P buffer; rows 32..127 (results never
-// used) come from the shared memory after it
-static_assert(kU2PBytes + 16384 <= kU2RingOff + U2Geom::kRingBytes, "P windows inside the CTA");
 
-// [hdr S][hdr2 S][valid S] then barriers: full_k S, full_v S, empty S, s 2,
-// pv 2, p 2, q, ofree, done, fin; then the TMEM slot and the dead flag; then
-// the slice maxima [2][4][32], give-up flags [2][4] and slice sums [4][32].
-constexpr int kU2ExtHdr = 12 * U2Geom::kStages;
-constexpr int kU2ExtBars = (kU2ExtHdr + 7) & ~7;
-constexpr int kU2NumBars = 3 * U2Geom::kStages + 10;
-constexpr int kU2ExtSlot = kU2ExtBars + 8 * kU2NumBars;
-constexpr int kU2ExtXm = (kU2ExtSlot + 8 + 15) & ~15;
-constexpr int kU2ExtXf = kU2ExtXm + 2 * 4 * 32 * 4;
-constexpr int kU2ExtXl = kU2ExtXf + 2 * 4 * 4;
-constexpr int kU2ExtBytes = kU2ExtXl + 4 * 32 * 4;
-constexpr size_t kU2Smem = (size_t)kU2RingOff + U2Geom::kRingBytes + kU2ExtBytes;
+// Layout of one variant: the ring the producer fills (over codes: stages of
+// [K sub-tiles][V sub-tiles], 16 KB, one barrier), the f16 K and V tiles over
+// codes, and after them [hdr S][hdr2 S][valid S][header slots 3 x 4], the
+// barriers (full_k S, full_v S, empty S, s 2, pv 2, p 2, q, ofree, done, fin,
+// kf_full 4, kf_free, vf_full, vf_free), the TMEM slot and the dead flag, the
+// slice maxima [2][4][32], give-up flags [2][4] and slice sums [4][32].
+template <typename TC>
+struct U2Cfg {
+    static constexpr bool kCodes = !std::is_same<TC, __nv_bfloat16>::value;
+    using Ring = typename std::conditional<
+        kCodes, GroupedRing<TC, 128, kU2Tokens / 16, PA_U2_STAGES * 2 * kU2HalfBytes>, U2Geom>::type;
+    static constexpr int kStages = Ring::kStages;
+    static constexpr int kThreads = kCodes ? 256 : 192;
+    static constexpr int kKfOff = kU2RingOff + Ring::kRingBytes;   // f16 K tile (codes)
+    static constexpr int kVfOff = kKfOff + 2 * kU2HalfBytes;       // f16 V tile (codes)
+    static constexpr int kExtOff = kCodes ? kVfOff + 2 * kU2HalfBytes : kU2RingOff + Ring::kRingBytes;
+    static constexpr int kHdr = 12 * kStages + 48;
+    static constexpr int kBars = (kHdr + 7) & ~7;
+    static constexpr int kNumBars = 3 * kStages + 17;
+    static constexpr int kSlot = kBars + 8 * kNumBars;
+    static constexpr int kXm = (kSlot + 8 + 15) & ~15;
+    static constexpr int kXf = kXm + 2 * 4 * 32 * 4;
+    static constexpr int kXl = kXf + 2 * 4 * 4;
+    static constexpr int kExtBytes = kXl + 4 * 32 * 4;
+    static constexpr size_t kSmem = (size_t)kExtOff + kExtBytes;
+    static constexpr uint32_t kIdescQK = umma_idesc(128, 64, false, kCodes);
+    static constexpr uint32_t kIdescPV = umma_idesc(128, 128, true, kCodes);
+    static_assert(kU2RingOff % 1024 == 0 && kKfOff % 1024 == 0 && kVfOff % 1024 == 0,
+                  "operand tiles on 1024-byte boundaries");
+    // the PV MMA reads 128 rows (16 KB) of a P buffer; rows 32..127 (results
+    // never used) come from the shared memory after it
+    static_assert(kU2PBytes + 16384 <= kExtOff, "P windows inside the CTA");
+    static_assert(kSmem <= 113 * 1024, "two CTAs per SM");
+};
 
 struct U2Bars {
     uint32_t full_k, full_v, empty, s, pv, p, q, ofree, done, fin;  // shared addresses
+    uint32_t kf_full, kf_free, vf_full, vf_free;                    // codes: f16 tiles
     volatile int* dead;
 };
 
@@ -2580,12 +2608,60 @@ __device__ __forceinline__ bool softmax_any(bool pred) {
     return r != 0;
 }
 
-__global__ void __launch_bounds__(192, 2)
+// 16 codes (one 16-byte chunk, in order) -> 16 f16 values in order, exactly:
+// E4M3 by the hardware conversion; int8 as (1024 + code + 128) - 1152 in f16
+// (a byte permute under the exponent of 1024, then one exact subtraction).
+template <typename TC>
+__device__ __forceinline__ void codes_to_f16_exact(const uint4& c, uint4& lo, uint4& hi) {
+    uint32_t h[8];
+    if constexpr (std::is_same<TC, E4M3Code>::value) {
+        codes_to_f16x2<E4M3Code>(c, h);
+    } else {
+        const uint32_t w[4] = {c.x ^ 0x80808080u, c.y ^ 0x80808080u, c.z ^ 0x80808080u,
+                               c.w ^ 0x80808080u};
+        const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t a = __byte_perm(w[i], 0x64646464u, 0x5140);
+            uint32_t b = __byte_perm(w[i], 0x64646464u, 0x5342);
+            __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
+            __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
+            h[2 * i] = *reinterpret_cast<uint32_t*>(&ha);
+            h[2 * i + 1] = *reinterpret_cast<uint32_t*>(&hb);
+        }
+    }
+    lo = make_uint4(h[0], h[1], h[2], h[3]);
+    hi = make_uint4(h[4], h[5], h[6], h[7]);
+}
+
+// 64 rows of 128 codes (rows 128 bytes apart, 128-byte swizzle) -> an f16 tile
+// [2 halves][64 rows][128 B] (128-byte swizzle); rows at or past `zero_from`
+// become zeros. 64 threads (t = 0..63), 8 chunks of 16 codes each.
+template <typename TC>
+__device__ __forceinline__ void convert_tile(uint32_t src, uint32_t dst, int t, int zero_from) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int i = t + 64 * k, r = i >> 3, x = i & 7;
+        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+        if (r < zero_from) codes_to_f16_exact<TC>(lds128(src + swz(r, x)), lo, hi);
+        const uint32_t half = dst + (x >> 2) * kU2HalfBytes;
+        const uint32_t c0 = 2 * (x & 3);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                     :: "r"(half + swz(r, c0)), "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w) : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                     :: "r"(half + swz(r, c0 + 1)), "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w) : "memory");
+    }
+}
+
+template <typename TC>
+__global__ void __launch_bounds__(U2Cfg<TC>::kThreads, 2)
 decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                            const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
                            int num_items, int gs) {
-    using G = U2Geom;
-    constexpr int S_ = G::kStages;
+    using C = U2Cfg<TC>;
+    using G = typename C::Ring;
+    constexpr bool kCodes = C::kCodes;
+    constexpr int S_ = C::kStages;
     constexpr int D = 128;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
@@ -2594,18 +2670,21 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
     const int group = p.num_heads / p.num_kv_heads;
     const int ncols = gs * group;
     const int ipb = 32 / gs;
+    const int DQ = kCodes ? p.head_dim : D;  // q / out head_dim (codes: 64 or 128)
     const uint32_t raw = smem_u32(smem_raw);
     if (raw & 1023u) {
         if (threadIdx.x == 0) atomicOr(&s_status_tma, kStatusSmemAlign);
         return;
     }
     const uint32_t pbuf = raw, qbuf = raw + kU2QOff;
-    uint8_t* ext = smem_raw + kU2RingOff + G::kRingBytes;
+    const uint32_t kfbuf = raw + C::kKfOff, vfbuf = raw + C::kVfOff;
+    uint8_t* ext = smem_raw + C::kExtOff;
     uint32_t* hdr = reinterpret_cast<uint32_t*>(ext);
     uint32_t* hdr2 = hdr + S_;
     int* valid = reinterpret_cast<int*>(hdr2 + S_);
+    uint32_t* hc = reinterpret_cast<uint32_t*>(valid + S_);  // codes: header slots [3][4]
     U2Bars B;
-    B.full_k = smem_u32(ext + kU2ExtBars);
+    B.full_k = smem_u32(ext + C::kBars);
     B.full_v = B.full_k + 8 * S_;
     B.empty = B.full_v + 8 * S_;
     B.s = B.empty + 8 * S_;  // [2]
@@ -2615,11 +2694,15 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
     B.ofree = B.q + 8;
     B.done = B.ofree + 8;
     B.fin = B.done + 8;
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(ext + kU2ExtSlot);
+    B.kf_full = B.fin + 8;   // [4]
+    B.kf_free = B.kf_full + 32;
+    B.vf_full = B.kf_free + 8;
+    B.vf_free = B.vf_full + 8;
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(ext + C::kSlot);
     B.dead = reinterpret_cast<volatile int*>(tslot + 1);
-    float* xm = reinterpret_cast<float*>(ext + kU2ExtXm);  // [2][4][32] slice maxima
-    volatile int* xf = reinterpret_cast<volatile int*>(ext + kU2ExtXf);  // [2][4] give-ups
-    float* xl = reinterpret_cast<float*>(ext + kU2ExtXl);  // [4][32] slice sums
+    float* xm = reinterpret_cast<float*>(ext + C::kXm);  // [2][4][32] slice maxima
+    volatile int* xf = reinterpret_cast<volatile int*>(ext + C::kXf);  // [2][4] give-ups
+    float* xl = reinterpret_cast<float*>(ext + C::kXl);  // [4][32] slice sums
     Ring ring;
     ring.stages = raw + kU2RingOff;
     ring.full = B.full_k;
@@ -2629,7 +2712,9 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         for (int st = 0; st < S_; ++st) {
             mbar_init(B.full_k + 8 * st, 1);
             mbar_init(B.full_v + 8 * st, 1);
-            mbar_init(B.empty + 8 * st, 1);  // the MMA thread's commit after the unit's PV
+            // released by the MMA thread's commit after the unit's PV, or over
+            // codes by the two converter warps once they converted it
+            mbar_init(B.empty + 8 * st, kCodes ? 2 : 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(B.s + 8 * i, 1);
@@ -2640,6 +2725,10 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         mbar_init(B.ofree, 4);
         mbar_init(B.done, 4);
         mbar_init(B.fin, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(B.kf_full + 8 * i, 2);
+        mbar_init(B.kf_free, 1);
+        mbar_init(B.vf_full, 2);
+        mbar_init(B.vf_free, 1);
         *B.dead = 0;
         fence_barrier_init();
     }
@@ -2689,16 +2778,57 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                 for (int u = 0; u < SUB; ++u) phys_cur[m][u] = phys_nxt[m][u];
         }
         if (dead) *B.dead = 1;
-        // drain: the last loads (K and V) of every stage have landed
+        // drain: the last loads of every stage have landed
         if (lane == 0 && issued > 0) {
             const int last = min(issued, S_);
             for (int st = 0; st < last; ++st) {
                 const int it = issued - 1 - ((issued - 1 - st) % S_);
                 const uint32_t par = (uint32_t)(it / S_) & 1u;
                 if (!mbar_wait_bounded(B.full_k + 8 * st, par) ||
-                    !mbar_wait_bounded(B.full_v + 8 * st, par))
+                    (!kCodes && !mbar_wait_bounded(B.full_v + 8 * st, par)))
                     atomicOr(&s_status_tma, kStatusTimeout);
             }
+        }
+        return;
+    }
+
+    if (kCodes && warp >= 6) {  // converters: codes -> f16 K and V tiles
+        const int t = threadIdx.x - 192;
+        int g = 0;
+        bool ok = true;
+        GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
+        while (cur.valid && ok) {
+            for (;;) {
+                const int st = g % S_;
+                if (!u2_wait(B, ring.full + 8 * st, (uint32_t)(g / S_) & 1u)) { ok = false; break; }
+                const uint32_t h = hdr[st], h2 = hdr2[st];
+                const int v = valid[st];
+                const uint32_t cb = ring.stages + st * G::kStageBytes;
+                // the K tile is free once the previous unit's QK is done
+                if (g >= 1 && !u2_wait(B, B.kf_free, (uint32_t)(g - 1) & 1u)) { ok = false; break; }
+                if (v) convert_tile<TC>(cb, kfbuf, t, kU2Tokens);
+                if (t == 0) {
+                    hc[g & 3] = h;
+                    hc[4 + (g & 3)] = h2;
+                    hc[8 + (g & 3)] = (uint32_t)v;
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(B.kf_full + 8 * (g & 3));
+                // the V tile is free once the previous unit's PV is done; rows
+                // past every member's tokens become zeros
+                if (g >= 1 && !u2_wait(B, B.vf_free, (uint32_t)(g - 1) & 1u)) { ok = false; break; }
+                if (v) convert_tile<TC>(cb + G::kSub * G::kSubBytes, vfbuf, t, (int)h2);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(B.vf_full);
+                    mbar_arrive(ring.empty + 8 * st);  // the codes are no longer needed
+                }
+                ++g;
+                if (h & kUnitLast) break;
+            }
+            if (ok) cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
         }
         return;
     }
@@ -2709,27 +2839,32 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         bool prev_valid = false, prev_first = false, o_started = false;
         // PV of unit prev_g: after its P is in shared memory and its V landed
         // (and, for an item's first unit, after the previous item's output left
-        // O); then release its stage.
+        // O); then release its stage (bf16) or its f16 V tile (codes).
         auto issue_pv = [&]() -> bool {
             if (!u2_wait(B, B.p + 8 * (prev_g & 1), (prev_g >> 1) & 1)) return false;
             if (prev_first) {
                 o_started = false;
                 if (prev_item >= 1 && !u2_wait(B, B.ofree, (prev_item - 1) & 1)) return false;
             }
-            if (!u2_wait(B, B.full_v + 8 * prev_st, (uint32_t)(prev_g / S_) & 1u)) return false;
+            if (kCodes) {
+                if (!u2_wait(B, B.vf_full, (uint32_t)prev_g & 1u)) return false;
+            } else if (!u2_wait(B, B.full_v + 8 * prev_st, (uint32_t)(prev_g / S_) & 1u)) {
+                return false;
+            }
             tc_fence_after();
             if (lane == 0) {
                 if (prev_valid) {
                     const uint32_t pa = pbuf + (prev_g & 1) * kU2PBytes;
-                    const uint32_t vb = ring.stages + prev_st * G::kStageBytes + 2 * kU2HalfBytes;
+                    const uint32_t vb =
+                        kCodes ? vfbuf : ring.stages + prev_st * G::kStageBytes + 2 * kU2HalfBytes;
 #pragma unroll
                     for (int k = 0; k < kU2Tokens / 16; ++k)
                         umma_ss(tm + kU2ColO, umma_desc(pa + 32 * k, 16, 1024),
-                                umma_desc(vb + 2048 * k, kU2HalfBytes, 1024), kU2IdescPV,
+                                umma_desc(vb + 2048 * k, kU2HalfBytes, 1024), C::kIdescPV,
                                 o_started || k > 0);
                 }
                 umma_commit(B.pv + 8 * (prev_g & 1));
-                umma_commit(B.empty + 8 * prev_st);
+                umma_commit(kCodes ? B.vf_free : B.empty + 8 * prev_st);
             }
             if (prev_valid) o_started = true;
             __syncwarp();
@@ -2743,21 +2878,32 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             bool first = true;
             for (;;) {
                 const int st = g % S_;
-                if (!u2_wait(B, B.full_k + 8 * st, (uint32_t)(g / S_) & 1u)) { ok = false; break; }
+                uint32_t h;
+                bool v;
+                uint32_t kb;
+                if constexpr (kCodes) {  // the f16 K tile and the unit's header slot
+                    if (!u2_wait(B, B.kf_full + 8 * (g & 3), (uint32_t)(g >> 2) & 1u)) { ok = false; break; }
+                    h = hc[g & 3];
+                    v = hc[8 + (g & 3)] != 0;
+                    kb = kfbuf;
+                } else {
+                    if (!u2_wait(B, B.full_k + 8 * st, (uint32_t)(g / S_) & 1u)) { ok = false; break; }
+                    h = hdr[st];
+                    v = valid[st] != 0;
+                    kb = ring.stages + st * G::kStageBytes;
+                }
                 tc_fence_after();
-                const uint32_t h = hdr[st];
-                const bool v = valid[st] != 0;
                 if (lane == 0) {
                     if (v) {
-                        const uint32_t kb = ring.stages + st * G::kStageBytes;
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
                             umma_ss(tm + kU2ColS + 64 * (g & 1),
                                     umma_desc(qbuf + (k >> 2) * (kU2QBytes / 2) + (k & 3) * 32, 16, 1024),
                                     umma_desc(kb + (k >> 2) * kU2HalfBytes + (k & 3) * 32, 16, 1024),
-                                    kU2IdescQK, k > 0);
+                                    C::kIdescQK, k > 0);
                     }
                     umma_commit(B.s + 8 * (g & 1));
+                    if (kCodes) umma_commit(B.kf_free);
                 }
                 __syncwarp();
                 if (prev_g >= 0 && !issue_pv()) { ok = false; break; }
@@ -2805,27 +2951,54 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             GItem it = gitem_next(walk, p, num_items, gs, ipb, lane, warp == 0, P == 1);
             if (!it.valid || it.tmax > it.t0) return it;
             if (warp == 0 && colv && mem < it.nmem) {
-                uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
-                    ((int64_t)(it.row0 + mem) * p.num_heads + (int64_t)it.kh * group + hd) * D);
-#pragma unroll
-                for (int c = 0; c < D / 8; ++c) o[c] = make_uint4(0u, 0u, 0u, 0u);
+                uint16_t* o = static_cast<uint16_t*>(p.out) +
+                              ((int64_t)(it.row0 + mem) * p.num_heads + (int64_t)it.kh * group + hd) * DQ;
+                for (int c = 0; c < DQ / 8; ++c)
+                    reinterpret_cast<uint4*>(o)[c] = make_uint4(0u, 0u, 0u, 0u);
             }
         }
     };
-    // this thread's Q row (32 warp + lane) := q of its column, 128-byte
-    // swizzled; the softmax takes maxima of unscaled scores, so the sign of the
-    // scale goes into q (an exact negation) and its magnitude is used below
-    const uint32_t qsign = p.scale_log2 < 0.f ? 0x80008000u : 0u;
-    auto stage_q = [&](const GItem& it) {
+    // This thread's Q row (32 warp + lane) := q of its column, 128-byte
+    // swizzled. The softmax takes maxima of unscaled scores, so the sign of the
+    // score scale goes into q (an exact negation) and its magnitude is used;
+    // over codes q is rounded to f16 after its column's power-of-two shift.
+    // Returns the column's score scale (log2 units, positive).
+    auto stage_q = [&](const GItem& it) -> float {
         const int t1 = __shfl_sync(0xffffffffu, it.t1_lane, mem & (kMaxGroupSeqs - 1));
         const bool has = colv && mem < it.nmem && t1 > it.t0;
+        const float sl0 = kCodes ? p.scale_log2 * __ldg(p.k_scale + it.kh) : p.scale_log2;
+        const uint32_t sg = sl0 < 0.f ? 0x80008000u : 0u;
         const uint4* src = reinterpret_cast<const uint4*>(qsrc_base +
-            ((int64_t)(it.row0 + mem) * p.num_heads + (int64_t)it.kh * group + hd) * D * 2);
+            ((int64_t)(it.row0 + mem) * p.num_heads + (int64_t)it.kh * group + hd) * DQ * 2);
         const uint32_t row = 32 * warp + lane;
+        auto ldq = [&](int c) {
+            const uint4 v = has && 8 * c < DQ ? ld_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            return make_uint4(v.x ^ sg, v.y ^ sg, v.z ^ sg, v.w ^ sg);
+        };
+        float slc = fabsf(sl0);
+        float mul = 1.f;
+        if constexpr (kCodes) {
+            uint32_t m = 0;  // largest |q| of the row (bits of a non-negative float)
+#pragma unroll 4
+            for (int c = 0; c < 16; ++c) {
+                const uint4 v = ldq(c);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    m = max(m, max((w[i] << 16) & 0x7fffffffu, w[i] & 0x7fff0000u));
+            }
+            const int sh = m == 0u ? 0 : max(-112, min(113, (int)((m >> 23) & 0xFFu) - 127 - 14));
+            mul = pow2i(-sh);
+            slc *= pow2i(sh);
+        }
+#pragma unroll 4
         for (int c = 0; c < 16; ++c) {
-            uint4 v = has ? ld_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
-            v = make_uint4(v.x ^ qsign, v.y ^ qsign, v.z ^ qsign, v.w ^ qsign);
+            uint4 v = ldq(c);  // (again: a cache hit)
+            if constexpr (kCodes)
+                v = make_uint4(pack_f16x2(bf16_lo(v.x) * mul, bf16_hi(v.x) * mul),
+                               pack_f16x2(bf16_lo(v.y) * mul, bf16_hi(v.y) * mul),
+                               pack_f16x2(bf16_lo(v.z) * mul, bf16_hi(v.z) * mul),
+                               pack_f16x2(bf16_lo(v.w) * mul, bf16_hi(v.w) * mul));
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
                          :: "r"(qbuf + (c >> 3) * (kU2QBytes / 2) + swz(row, c & 7)),
                             "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
@@ -2833,19 +3006,25 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(B.q);
+        return slc;
     };
     GItem cur = next_item();
-    if (cur.valid) stage_q(cur);
+    float sl_next = cur.valid ? stage_q(cur) : 0.f;
     while (cur.valid && ok) {
         const int t1 = __shfl_sync(0xffffffffu, cur.t1_lane, mem & (kMaxGroupSeqs - 1));
-        const float sl = fabsf(p.scale_log2);
+        const float sl = sl_next;
         float m_ref = -INFINITY, l = 0.f;
         for (;;) {
             const int b = g & 1, st = g % S_;
             // S of unit g (and with it every earlier MMA: the PV of unit g - 2
-            // no longer reads P buffer b); the K barrier orders the header reads
+            // no longer reads P buffer b); the K barrier (bf16) or the header
+            // slot's barrier (codes) orders the header reads
             if (healthy) healthy = u2_wait(B, B.s + 8 * b, (g >> 1) & 1);
-            if (healthy) healthy = u2_wait(B, B.full_k + 8 * st, (uint32_t)(g / S_) & 1u);
+            if (kCodes) {
+                if (healthy) healthy = u2_wait(B, B.kf_full + 8 * (g & 3), (uint32_t)(g >> 2) & 1u);
+            } else if (healthy) {
+                healthy = u2_wait(B, B.full_k + 8 * st, (uint32_t)(g / S_) & 1u);
+            }
             uint32_t h = 0;
             int nvmax = 0;
             bool v = false;
@@ -2853,9 +3032,9 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             float mx = -INFINITY;
             if (healthy) {
                 tc_fence_after();
-                h = hdr[st];
-                v = valid[st] != 0;
-                nvmax = (int)hdr2[st];
+                h = kCodes ? hc[g & 3] : hdr[st];
+                v = (kCodes ? hc[8 + (g & 3)] : (uint32_t)valid[st]) != 0;
+                nvmax = (int)(kCodes ? hc[4 + (g & 3)] : hdr2[st]);
                 const int tok0 = cur.t0 + (int)((h >> kUnitSubShift) & kUnitSubMask) * kU2Tokens;
                 uint32_t sr[kU2Slice];
                 tmem_ld16(tm + lane_off + kU2ColS + 64 * b + slice0, sr);
@@ -2914,16 +3093,22 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                     }
                 }
             }
-            // weights of the slice (masked scores give 2^-inf = 0), bf16, summed
-            // as rounded
+            // weights of the slice (masked scores give 2^-inf = 0), bf16 (f16
+            // beside codes), summed as rounded
             const float base = m_ref == -INFINITY ? 0.f : m_ref;
             uint32_t pk[kU2Slice / 2];
             float ps = 0.f;
 #pragma unroll
             for (int j = 0; j < kU2Slice / 2; ++j) {
-                pk[j] = pack_bf16x2(ex2_approx(fmaf(sv[2 * j], sl, -base)),
-                                    ex2_approx(fmaf(sv[2 * j + 1], sl, -base)));
-                ps += bf16_lo(pk[j]) + bf16_hi(pk[j]);
+                const float w0 = ex2_approx(fmaf(sv[2 * j], sl, -base));
+                const float w1 = ex2_approx(fmaf(sv[2 * j + 1], sl, -base));
+                if constexpr (kCodes) {
+                    pk[j] = pack_f16x2(w0, w1);
+                    ps += f16_lo(pk[j]) + f16_hi(pk[j]);
+                } else {
+                    pk[j] = pack_bf16x2(w0, w1);
+                    ps += bf16_lo(pk[j]) + bf16_hi(pk[j]);
+                }
             }
             l += ps;
             // P row `col`, tokens 16 warp .. + 15: 16-byte chunks 2 warp, 2 warp + 1
@@ -2934,9 +3119,10 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
                          :: "r"(prow + swz(col, 2 * warp + 1)), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
                             "r"(pk[7]) : "memory");
-            // V rows of the slice at or past every member's tokens may hold
-            // anything (NaN included): zero them once V has landed
-            if (healthy && v && nvmax < slice0 + kU2Slice) {
+            // bf16: V rows of the slice at or past every member's tokens may hold
+            // anything (NaN included): zero them once V has landed (over codes
+            // the converters wrote those rows as zeros)
+            if (!kCodes && healthy && v && nvmax < slice0 + kU2Slice) {
                 healthy = u2_wait(B, B.full_v + 8 * st, (uint32_t)(g / S_) & 1u);
                 if (healthy) {
                     const uint32_t vb = ring.stages + st * G::kStageBytes + 2 * kU2HalfBytes;
@@ -2963,19 +3149,19 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         const float lt = ((xl[lane] + xl[32 + lane]) + xl[64 + lane]) + xl[96 + lane];
         // the next item's q: every QK of this item is complete (its last S was read)
         const GItem nxt = next_item();
-        if (nxt.valid) stage_q(nxt);
+        if (nxt.valid) sl_next = stage_q(nxt);
         if (warp == 0) {
             if (healthy) healthy = u2_wait(B, B.pv + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1);
             const bool has = colv && mem < cur.nmem && t1 > cur.t0;
             const int64_t row = (int64_t)(cur.row0 + mem) * p.num_heads + (int64_t)cur.kh * group + hd;
-            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            const float inv = (lt > 0.f ? 1.f / lt : 0.f) * (kCodes ? __ldg(p.v_scale + cur.kh) : 1.f);
             if (healthy) {
                 tc_fence_after();
 #pragma unroll 1
                 for (int c0 = 0; c0 < 128; c0 += 32) {
                     uint32_t o[32];
                     tmem_ld32(tm + lane_off + kU2ColO + c0, o);
-                    if (colv && mem < cur.nmem) {
+                    if (colv && mem < cur.nmem && c0 < DQ) {
                         if (P == 1) {
                             uint32_t w[16];
 #pragma unroll
@@ -2983,12 +3169,12 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                                 w[j] = lt > 0.f ? pack_bf16x2(__uint_as_float(o[2 * j]) * inv,
                                                               __uint_as_float(o[2 * j + 1]) * inv)
                                                 : 0u;
-                            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * D + c0);
+                            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * DQ + c0);
 #pragma unroll
                             for (int j = 0; j < 4; ++j)
                                 dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
                         } else if (has) {
-                            float4* dst = reinterpret_cast<float4*>(p.ws_o + (row * P + cur.part) * D + c0);
+                            float4* dst = reinterpret_cast<float4*>(p.ws_o + (row * P + cur.part) * DQ + c0);
 #pragma unroll
                             for (int j = 0; j < 8; ++j)
                                 dst[j] = lt > 0.f ? make_float4(__uint_as_float(o[4 * j]) * inv,
@@ -3064,10 +3250,12 @@ cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUt
     return cudaGetLastError();
 }
 
+template <typename TC>
 cudaError_t launch_umma_grouped(const DecodeParams& p, const CUtensorMap& km,
                                 const CUtensorMap& vm, int gs, cudaStream_t stream) {
-    constexpr size_t smem = kU2Smem;
-    auto kernel = decode_umma_grouped_kernel;
+    using C = U2Cfg<TC>;
+    constexpr size_t smem = C::kSmem;
+    auto kernel = decode_umma_grouped_kernel<TC>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -3079,9 +3267,9 @@ cudaError_t launch_umma_grouped(const DecodeParams& p, const CUtensorMap& km,
     const long groups = p.query_start != nullptr ? (long)p.num_seqs * p.q_chunks
                                                  : (long)(p.num_seqs + gs - 1) / gs;
     const long items = (long)p.num_partitions * p.num_kv_heads * groups;
-    const long slots = 2L * sms;  // two CTAs per SM: 256 TMEM columns and ~106 KB each
+    const long slots = 2L * sms;  // two CTAs per SM: 256 TMEM columns and <= 113 KB each
     const unsigned grid = (unsigned)(items < slots ? items : slots);
-    kernel<<<grid, 192, smem, stream>>>(km, vm, p, (int)items, gs);
+    kernel<<<grid, C::kThreads, smem, stream>>>(km, vm, p, (int)items, gs);
     return cudaGetLastError();
 }
 
@@ -3177,9 +3365,9 @@ bool grouped_supported(int dtype, int head_dim, int group, int gs) {
     return shape && gs >= 1 && gs <= kMaxGroupSeqs && group >= 1 && gs * group <= kGroupedMaxCols;
 }
 
-// The tcgen05 consumer takes bf16 only.
+// The tcgen05 consumer takes bf16 at head_dim 128 and codes at 64 or 128.
 bool grouped_is_tcgen05(int dtype, int head_dim, int gs, int group) {
-    return dtype == 1 && use_umma(head_dim, gs, group);
+    return (dtype == 1 || dtype == 2 || dtype == 3) && use_umma(dtype == 1 ? head_dim : 128, gs, group);
 }
 
 int grouped_ctas_per_sm(int dtype, int head_dim, int gs, int group) {
@@ -3222,8 +3410,11 @@ static cudaError_t launch_grouped_d(const DecodeParams& p, int cw, int nt, int g
 cudaError_t launch_decode_grouped(const DecodeParams& p, int dtype, int head_dim, int gs,
                                   const CUtensorMap& kmap, const CUtensorMap& vmap,
                                   cudaStream_t stream) {
-    if (grouped_is_tcgen05(dtype, head_dim, gs, p.num_heads / p.num_kv_heads))
-        return launch_umma_grouped(p, kmap, vmap, gs, stream);
+    if (grouped_is_tcgen05(dtype, head_dim, gs, p.num_heads / p.num_kv_heads)) {
+        if (dtype == 2) return launch_umma_grouped<E4M3Code>(p, kmap, vmap, gs, stream);
+        if (dtype == 3) return launch_umma_grouped<Int8Code>(p, kmap, vmap, gs, stream);
+        return launch_umma_grouped<__nv_bfloat16>(p, kmap, vmap, gs, stream);
+    }
     int cw = 1, nt = 1;
     grouped_shape(gs, p.num_heads / p.num_kv_heads, &cw, &nt);
     if (dtype == 2) return launch_grouped_d<128, E4M3Code>(p, cw, nt, gs, kmap, vmap, stream);
