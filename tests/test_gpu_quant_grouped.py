@@ -78,7 +78,7 @@ def test_grouped_cow_parity(fmt, gs, ps):
     _append(wl, vals, d)
     out = _grouped(wl, vals, d, gs, ps)
     pa.pa_sync_check()
-    assert G.last_kernel() == pa.PA_KERNEL_GROUPED
+    assert G.last_kernel() in G.kernel_set(pa.PA_KERNEL_GROUPED)
     _oracle_append(wl, host)
     assert np.array_equal(_codes(vals["k_cache"]), host["k_cache"])
     assert np.array_equal(_codes(vals["v_cache"]), host["v_cache"])
@@ -160,7 +160,7 @@ def test_multi_parity(fmt, H, Hkv, d):
                                  max_context_len=wl.max_context_len,
                                  max_query_len=wl.max_query_len, partition_size=ps)
         pa.pa_sync_check()
-        assert G.last_kernel() == pa.PA_KERNEL_GROUPED
+        assert G.last_kernel() in G.kernel_set(pa.PA_KERNEL_GROUPED)
         _oracle_append(wl, host)
         ref = oracle.decode_quant(host["q"], host["k_cache"], host["v_cache"], host["k_scale"],
                                   host["v_scale"], tables_r, ctx_r, wl.scale, fmt,
