@@ -175,7 +175,8 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
             return fail(PA_ERR_INVALID_ARG, "max_query_len %d must be in [1, num_query_tokens %d]",
                         max_query_len, num_query_tokens);
         int gs = max_query_len < 8 ? max_query_len : 8;
-        while (gs > 1 && gs * group > 64) --gs;
+        const int max_cols = pa::grouped_max_cols(c->dtype, c->head_dim, group);
+        while (gs > 1 && gs * group > max_cols) --gs;
         if (pa::grouped_supported(c->dtype, c->head_dim, group, gs)) {
             group_size = gs;
             plan->q_chunks = (max_query_len + gs - 1) / gs;

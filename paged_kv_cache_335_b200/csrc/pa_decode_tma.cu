@@ -270,9 +270,13 @@ __device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t
 #endif
 // Int8 codes widened with a bias of 1152 (one byte permute per two codes, no
 // per-code subtraction); the bias leaves the scores as 1152 x the sum of the
-// lane's q elements and the output as 1152 x the sum of the weights.
+// lane's q elements and the output as 1152 x the sum of the weights. Off: the
+// biased terms are ~10x the true ones, so the fp32 sums lose ~10x more to
+// rounding (visible with |q| ~ 1e6, where scores are ~1e6 and their rounding
+// reaches the gap between the two largest); the codes are widened exactly
+// instead (one f16 subtraction per two codes).
 #ifndef PA_SIMT_INT8_BIASED
-#define PA_SIMT_INT8_BIASED 1
+#define PA_SIMT_INT8_BIASED 0
 #endif
 // Codes as f16 operands of the mixed-precision fma (f16 x f16 + f32 -> f32,
 // one instruction per code, no widening to f32): q is rounded to f16 (exact
@@ -297,8 +301,10 @@ __device__ __forceinline__ void fma2_f16s_f32(uint32_t pp, uint32_t b, float& c0
         : "+f"(c0), "+f"(c1) : "r"(pp), "r"(b));
 }
 
-// 16 codes -> 8 f16x2 words: E4M3 exactly; int8 as 1152 + code (exact).
-template <typename TC>
+// 16 codes -> 8 f16x2 words in order: E4M3 exactly; int8 as 1152 + code
+// (exact), or with kExactInt8 the code itself (one exact f16 subtraction of
+// 1152 per two codes).
+template <typename TC, bool kExactInt8 = false>
 __device__ __forceinline__ void codes_to_f16x2(const uint4& c, uint32_t (&h)[8]) {
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
@@ -311,6 +317,13 @@ __device__ __forceinline__ void codes_to_f16x2(const uint4& c, uint32_t (&h)[8])
             const uint32_t u = w[i] ^ 0x80808080u;
             h[2 * i] = __byte_perm(u, 0x64646464u, 0x5140);
             h[2 * i + 1] = __byte_perm(u, 0x64646464u, 0x5342);
+            if constexpr (kExactInt8) {
+                const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
+                __half2 a = __hsub2(*reinterpret_cast<__half2*>(&h[2 * i]), bias);
+                __half2 b = __hsub2(*reinterpret_cast<__half2*>(&h[2 * i + 1]), bias);
+                h[2 * i] = *reinterpret_cast<uint32_t*>(&a);
+                h[2 * i + 1] = *reinterpret_cast<uint32_t*>(&b);
+            }
         }
     }
 }
@@ -350,7 +363,7 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                                                          std::is_same<T, Int8Code>::value);
     constexpr bool kCodes = std::is_same<T, E4M3Code>::value || std::is_same<T, Int8Code>::value;
     constexpr bool kMixed = PA_SIMT_CODES_MIXED_FMA && kCodes;
-    constexpr bool kBiased = (PA_SIMT_INT8_BIASED || kMixed) && std::is_same<T, Int8Code>::value;
+    constexpr bool kBiased = PA_SIMT_INT8_BIASED && std::is_same<T, Int8Code>::value;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     asm volatile("griddepcontrol.launch_dependents;");
 
@@ -486,7 +499,7 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                     float dot = 0.f;
                     if constexpr (kMixed) {
                         uint32_t kh2[VEC / 2];
-                        codes_to_f16x2<T>(kr[it], kh2);
+                        codes_to_f16x2<T, !kBiased>(kr[it], kh2);
                         float d1 = 0.f;
 #pragma unroll
                         for (int j = 0; j < VEC / 2; ++j) fma2_f16_f32(qh[j], kh2[j], dot, d1);
@@ -530,7 +543,7 @@ decode_tma_simt_kernel(const __grid_constant__ CUtensorMap kmap,
                         l += __half2float(ph);
                         if (tok < t1) {  // slots past the context may hold anything, even NaN
                             uint32_t vh2[VEC / 2];
-                            codes_to_f16x2<T>(vr[it], vh2);
+                            codes_to_f16x2<T, !kBiased>(vr[it], vh2);
                             const uint32_t pp = (uint32_t)__half_as_ushort(ph);
 #pragma unroll
                             for (int j = 0; j < VEC / 2; ++j)
@@ -2614,22 +2627,7 @@ __device__ __forceinline__ bool softmax_any(bool pred) {
 template <typename TC>
 __device__ __forceinline__ void codes_to_f16_exact(const uint4& c, uint4& lo, uint4& hi) {
     uint32_t h[8];
-    if constexpr (std::is_same<TC, E4M3Code>::value) {
-        codes_to_f16x2<E4M3Code>(c, h);
-    } else {
-        const uint32_t w[4] = {c.x ^ 0x80808080u, c.y ^ 0x80808080u, c.z ^ 0x80808080u,
-                               c.w ^ 0x80808080u};
-        const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t a = __byte_perm(w[i], 0x64646464u, 0x5140);
-            uint32_t b = __byte_perm(w[i], 0x64646464u, 0x5342);
-            __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
-            __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
-            h[2 * i] = *reinterpret_cast<uint32_t*>(&ha);
-            h[2 * i + 1] = *reinterpret_cast<uint32_t*>(&hb);
-        }
-    }
+    codes_to_f16x2<TC, true>(c, h);
     lo = make_uint4(h[0], h[1], h[2], h[3]);
     hi = make_uint4(h[4], h[5], h[6], h[7]);
 }
@@ -3363,6 +3361,15 @@ static void grouped_shape(int gs, int group, int* cw, int* nt) {
 bool grouped_supported(int dtype, int head_dim, int group, int gs) {
     const bool shape = (dtype == 1 || dtype == 2 || dtype == 3) && (head_dim == 64 || head_dim == 128);
     return shape && gs >= 1 && gs <= kMaxGroupSeqs && group >= 1 && gs * group <= kGroupedMaxCols;
+}
+
+// Query columns a multi-token item may hold: with the tcgen05 consumer selected
+// and a shape it takes, at most its 32, so every call of that shape runs on it
+// (a token's result is then the same whichever other tokens share the call).
+int grouped_max_cols(int dtype, int head_dim, int group) {
+    const bool capable = (dtype == 1 && head_dim == 128) || dtype == 2 || dtype == 3;
+    return g_grouped_consumer == PA_GROUPED_TCGEN05 && capable && group <= kU2Cols ? kU2Cols
+                                                                                 : kGroupedMaxCols;
 }
 
 // The tcgen05 consumer takes bf16 at head_dim 128 and codes at 64 or 128.

@@ -104,6 +104,8 @@ bool grouped_supported(int dtype, int head_dim, int group, int gs);
 // Select the grouped consumer (PA_GROUPED_MMA_SYNC / PA_GROUPED_TCGEN05);
 // returns the previous one.
 int set_grouped_consumer(int consumer);
+// Most query columns (tokens x heads per kv head) one multi-token item may hold.
+int grouped_max_cols(int dtype, int head_dim, int group);
 // Whether the grouped kernel for (dtype, head_dim, gs, H / Hkv) is the tcgen05 consumer.
 bool grouped_is_tcgen05(int dtype, int head_dim, int gs, int group);
 // CTA slots per SM of the grouped kernel chosen for (dtype, head_dim, gs, H / Hkv).
