@@ -270,13 +270,13 @@ __device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t
 #endif
 // Int8 codes widened with a bias of 1152 (one byte permute per two codes, no
 // per-code subtraction); the bias leaves the scores as 1152 x the sum of the
-// lane's q elements and the output as 1152 x the sum of the weights. Off: the
-// biased terms are ~10x the true ones, so the fp32 sums lose ~10x more to
-// rounding (visible with |q| ~ 1e6, where scores are ~1e6 and their rounding
-// reaches the gap between the two largest); the codes are widened exactly
-// instead (one f16 subtraction per two codes).
+// lane's q elements and the output as 1152 x the sum of the weights. The
+// biased terms are ~10x the true ones, so the fp32 sums carry ~10x the rounding
+// of exactly widened codes (still far inside the bf16 bars). Off: the codes
+// are widened exactly (one f16 subtraction per two codes; 13B int8 step 502 vs
+// 485 us on a B200).
 #ifndef PA_SIMT_INT8_BIASED
-#define PA_SIMT_INT8_BIASED 0
+#define PA_SIMT_INT8_BIASED 1
 #endif
 // Codes as f16 operands of the mixed-precision fma (f16 x f16 + f32 -> f32,
 // one instruction per code, no widening to f32): q is rounded to f16 (exact
