@@ -2831,93 +2831,109 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         return;
     }
 
-    if (warp == 5) {  // MMA issuer: lane 0 issues, the warp walks the items with it
-        int g = 0, n = 0;
-        int prev_g = -1, prev_st = 0, prev_item = 0;
-        bool prev_valid = false, prev_first = false, o_started = false;
-        // PV of unit prev_g: after its P is in shared memory and its V landed
-        // (and, for an item's first unit, after the previous item's output left
-        // O); then release its stage (bf16) or its f16 V tile (codes).
-        auto issue_pv = [&]() -> bool {
-            if (!u2_wait(B, B.p + 8 * (prev_g & 1), (prev_g >> 1) & 1)) return false;
-            if (prev_first) {
-                o_started = false;
-                if (prev_item >= 1 && !u2_wait(B, B.ofree, (prev_item - 1) & 1)) return false;
-            }
-            if (kCodes) {
-                if (!u2_wait(B, B.vf_full, (uint32_t)prev_g & 1u)) return false;
-            } else if (!u2_wait(B, B.full_v + 8 * prev_st, (uint32_t)(prev_g / S_) & 1u)) {
-                return false;
-            }
-            tc_fence_after();
-            if (lane == 0) {
-                if (prev_valid) {
-                    const uint32_t pa = pbuf + (prev_g & 1) * kU2PBytes;
-                    const uint32_t vb =
-                        kCodes ? vfbuf : ring.stages + prev_st * G::kStageBytes + 2 * kU2HalfBytes;
-#pragma unroll
-                    for (int k = 0; k < kU2Tokens / 16; ++k)
-                        umma_ss(tm + kU2ColO, umma_desc(pa + 32 * k, 16, 1024),
-                                umma_desc(vb + 2048 * k, kU2HalfBytes, 1024), C::kIdescPV,
-                                o_started || k > 0);
-                }
-                umma_commit(B.pv + 8 * (prev_g & 1));
-                umma_commit(kCodes ? B.vf_free : B.empty + 8 * prev_st);
-            }
-            if (prev_valid) o_started = true;
-            __syncwarp();
-            return true;
-        };
-        bool ok = true;
+    if (warp == 5) {
+        // MMA issuer, event-driven: lane 0 issues; each turn it issues the next
+        // QK if its K tile has landed (and its S buffer is free: the PV two units
+        // back has been issued), and the next PV if that unit's P is written and
+        // its V landed (for an item's first unit, once the previous item's output
+        // left O). Neither waits behind the other, so a stage is released as soon
+        // as its softmax is done and the next loads go out without a DRAM round
+        // trip behind an unrelated wait.
+        int g_qk = 0, g_pv = 0, n_qk = 0;
+        bool need_q = true, first_qk = true, qk_done = false, o_started = false, ok = true;
+        // per unit g (slot g & 3): stage, valid, first unit of its item, item index
+        int rec_st[4], rec_item[4];
+        bool rec_valid[4], rec_first[4];
         GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
-        while (cur.valid && ok) {
-            if (!u2_wait(B, B.q, n & 1)) { ok = false; break; }
-            tc_fence_after();
-            bool first = true;
-            for (;;) {
-                const int st = g % S_;
-                uint32_t h;
-                bool v;
-                uint32_t kb;
-                if constexpr (kCodes) {  // the f16 K tile and the unit's header slot
-                    if (!u2_wait(B, B.kf_full + 8 * (g & 3), (uint32_t)(g >> 2) & 1u)) { ok = false; break; }
-                    h = hc[g & 3];
-                    v = hc[8 + (g & 3)] != 0;
-                    kb = kfbuf;
-                } else {
-                    if (!u2_wait(B, B.full_k + 8 * st, (uint32_t)(g / S_) & 1u)) { ok = false; break; }
-                    h = hdr[st];
-                    v = valid[st] != 0;
-                    kb = ring.stages + st * G::kStageBytes;
-                }
-                tc_fence_after();
-                if (lane == 0) {
-                    if (v) {
+        if (!cur.valid) qk_done = true;
+        auto lane0 = [&](bool x) { return __shfl_sync(0xffffffffu, x, 0); };
+        uint64_t t_last = global_timer_ns();
+        while (ok && !(qk_done && g_pv == g_qk)) {
+            bool progressed = false;
+            if (*B.dead) { ok = false; break; }
+            // QK of unit g_qk
+            if (!qk_done && g_qk - g_pv <= 1) {
+                if (need_q && lane0(mbar_test_wait(B.q, n_qk & 1))) need_q = false;
+                const int st = g_qk % S_;
+                const bool kready =
+                    !need_q && lane0(kCodes ? mbar_test_wait(B.kf_full + 8 * (g_qk & 3), (uint32_t)(g_qk >> 2) & 1u)
+                                            : mbar_test_wait(B.full_k + 8 * st, (uint32_t)(g_qk / S_) & 1u));
+                if (kready) {
+                    tc_fence_after();
+                    const uint32_t h = kCodes ? hc[g_qk & 3] : hdr[st];
+                    const bool v = (kCodes ? hc[8 + (g_qk & 3)] : (uint32_t)valid[st]) != 0;
+                    if (lane == 0) {
+                        if (v) {
+                            const uint32_t kb = kCodes ? kfbuf : ring.stages + st * G::kStageBytes;
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            umma_ss(tm + kU2ColS + 64 * (g & 1),
-                                    umma_desc(qbuf + (k >> 2) * (kU2QBytes / 2) + (k & 3) * 32, 16, 1024),
-                                    umma_desc(kb + (k >> 2) * kU2HalfBytes + (k & 3) * 32, 16, 1024),
-                                    C::kIdescQK, k > 0);
+                            for (int k = 0; k < 8; ++k)
+                                umma_ss(tm + kU2ColS + 64 * (g_qk & 1),
+                                        umma_desc(qbuf + (k >> 2) * (kU2QBytes / 2) + (k & 3) * 32, 16, 1024),
+                                        umma_desc(kb + (k >> 2) * kU2HalfBytes + (k & 3) * 32, 16, 1024),
+                                        C::kIdescQK, k > 0);
+                        }
+                        umma_commit(B.s + 8 * (g_qk & 1));
+                        if (kCodes) umma_commit(B.kf_free);
                     }
-                    umma_commit(B.s + 8 * (g & 1));
-                    if (kCodes) umma_commit(B.kf_free);
+                    __syncwarp();
+                    const int r = g_qk & 3;
+                    rec_st[r] = st;
+                    rec_valid[r] = v;
+                    rec_first[r] = first_qk;
+                    rec_item[r] = n_qk;
+                    first_qk = false;
+                    ++g_qk;
+                    if (h & kUnitLast) {
+                        ++n_qk;
+                        need_q = true;
+                        first_qk = true;
+                        cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
+                        if (!cur.valid) qk_done = true;
+                    }
+                    progressed = true;
                 }
-                __syncwarp();
-                if (prev_g >= 0 && !issue_pv()) { ok = false; break; }
-                prev_g = g;
-                prev_st = st;
-                prev_valid = v;
-                prev_first = first;
-                prev_item = n;
-                first = false;
-                ++g;
-                if (h & kUnitLast) break;
             }
-            ++n;
-            if (ok) cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
+            // PV of unit g_pv
+            if (g_pv < g_qk) {
+                const int r = g_pv & 3;
+                bool ready = lane0(mbar_test_wait(B.p + 8 * (g_pv & 1), (g_pv >> 1) & 1));
+                ready = ready && lane0(kCodes ? mbar_test_wait(B.vf_full, (uint32_t)g_pv & 1u)
+                                              : mbar_test_wait(B.full_v + 8 * rec_st[r], (uint32_t)(g_pv / S_) & 1u));
+                if (ready && rec_first[r] && rec_item[r] >= 1)
+                    ready = lane0(mbar_test_wait(B.ofree, (rec_item[r] - 1) & 1));
+                if (ready) {
+                    tc_fence_after();
+                    if (rec_first[r]) o_started = false;
+                    if (lane == 0) {
+                        if (rec_valid[r]) {
+                            const uint32_t pa = pbuf + (g_pv & 1) * kU2PBytes;
+                            const uint32_t vb =
+                                kCodes ? vfbuf : ring.stages + rec_st[r] * G::kStageBytes + 2 * kU2HalfBytes;
+#pragma unroll
+                            for (int k = 0; k < kU2Tokens / 16; ++k)
+                                umma_ss(tm + kU2ColO, umma_desc(pa + 32 * k, 16, 1024),
+                                        umma_desc(vb + 2048 * k, kU2HalfBytes, 1024), C::kIdescPV,
+                                        o_started || k > 0);
+                        }
+                        umma_commit(B.pv + 8 * (g_pv & 1));
+                        umma_commit(kCodes ? B.vf_free : B.empty + 8 * rec_st[r]);
+                    }
+                    __syncwarp();
+                    if (rec_valid[r]) o_started = true;
+                    ++g_pv;
+                    progressed = true;
+                }
+            }
+            if (!progressed) __nanosleep(64);  // leave the issue slots to the softmax warp
+            const uint64_t now = global_timer_ns();
+            if (progressed) {
+                t_last = now;
+            } else if (now - t_last > kWaitLimitNs) {  // nothing moved for the wait limit
+                if (lane == 0 && *B.dead == 0) atomicOr(&s_status_tma, kStatusTimeout);
+                if (lane == 0) *B.dead = 1;
+                ok = false;
+            }
         }
-        if (ok && prev_g >= 0) ok = issue_pv();
         // wait for the softmax warps (even after a give-up: they stop touching
         // TMEM before they arrive), then for every issued MMA, then free TMEM
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(B.done, 0)) && lane == 0)
