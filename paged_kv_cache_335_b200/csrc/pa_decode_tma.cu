@@ -2535,8 +2535,19 @@ constexpr int kU2Tokens = 64;                   // tokens per unit
 constexpr int kU2Cols = 32;                     // query columns per item, at most
 constexpr int kU2Slice = kU2Tokens / 4;         // tokens per softmax warp per unit
 constexpr int kU2HalfBytes = kU2Tokens * 128;   // one d-half of a K or V tile: 8 KB
+// Ring depth and CTAs per SM. A stage is busy for the TMA latency of its
+// loads (~2 us for a unit's 16 boxes, measured by timestamps on a B200) plus
+// its use (QK, softmax, PV: ~1.2-1.8 us), so an SM needs about five 32 KB stages
+// in flight to read at HBM rate: one CTA per SM with five bf16 stages (eight
+// 16 KB stages over codes), 200 KB of shared memory.
 #ifndef PA_U2_STAGES
-#define PA_U2_STAGES 2
+#define PA_U2_STAGES 5
+#endif
+#ifndef PA_U2_CODE_STAGES
+#define PA_U2_CODE_STAGES 8
+#endif
+#ifndef PA_U2_CTAS
+#define PA_U2_CTAS 1
 #endif
 constexpr int kU2PBytes = kU2Cols * 128;        // P tile: 32 rows x 64 16-bit tokens
 constexpr int kU2QBytes = 2 * 128 * 128;        // Q tile: 128 rows x 128 16-bit, two d-halves
@@ -2570,7 +2581,7 @@ template <typename TC>
 struct U2Cfg {
     static constexpr bool kCodes = !std::is_same<TC, __nv_bfloat16>::value;
     using Ring = typename std::conditional<
-        kCodes, GroupedRing<TC, 128, kU2Tokens / 16, PA_U2_STAGES * 2 * kU2HalfBytes>, U2Geom>::type;
+        kCodes, GroupedRing<TC, 128, kU2Tokens / 16, PA_U2_CODE_STAGES * 2 * kU2HalfBytes>, U2Geom>::type;
     static constexpr int kStages = Ring::kStages;
     static constexpr int kThreads = kCodes ? 256 : 192;
     static constexpr int kKfOff = kU2RingOff + Ring::kRingBytes;   // f16 K tile (codes)
@@ -2592,7 +2603,8 @@ struct U2Cfg {
     // the PV MMA reads 128 rows (16 KB) of a P buffer; rows 32..127 (results
     // never used) come from the shared memory after it
     static_assert(kU2PBytes + 16384 <= kExtOff, "P windows inside the CTA");
-    static_assert(kSmem <= 113 * 1024, "two CTAs per SM");
+    static_assert(kSmem * PA_U2_CTAS + 1024 * PA_U2_CTAS <= 228 * 1024 && kSmem <= 227 * 1024,
+                  "shared memory of PA_U2_CTAS CTAs per SM");
 };
 
 struct U2Bars {
@@ -2652,7 +2664,7 @@ __device__ __forceinline__ void convert_tile(uint32_t src, uint32_t dst, int t, 
 }
 
 template <typename TC>
-__global__ void __launch_bounds__(U2Cfg<TC>::kThreads, 2)
+__global__ void __launch_bounds__(U2Cfg<TC>::kThreads, PA_U2_CTAS)
 decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                            const __grid_constant__ CUtensorMap vmap, const DecodeParams p,
                            int num_items, int gs) {
@@ -2833,10 +2845,10 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
 
     if (warp == 5) {
         // MMA issuer, event-driven: lane 0 issues; each turn it issues the next
-        // QK if its K tile has landed (and its S buffer is free: the PV two units
-        // back has been issued), and the next PV if that unit's P is written and
-        // its V landed (for an item's first unit, once the previous item's output
-        // left O). Neither waits behind the other, so a stage is released as soon
+        // PV if that unit's P is written and its V landed (for an item's first
+        // unit, once the previous item's output left O), then the next QK if its
+        // K tile has landed (and its S buffer is free: the PV two units back has
+        // been issued). Neither waits behind the other, so a stage is released as soon
         // as its softmax is done and the next loads go out without a DRAM round
         // trip behind an unrelated wait.
         int g_qk = 0, g_pv = 0, n_qk = 0;
@@ -2847,10 +2859,42 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
         if (!cur.valid) qk_done = true;
         auto lane0 = [&](bool x) { return __shfl_sync(0xffffffffu, x, 0); };
-        uint64_t t_last = global_timer_ns();
+        uint64_t t_last = 0;
+        uint32_t idle = 0;  // polls since the last issue
         while (ok && !(qk_done && g_pv == g_qk)) {
             bool progressed = false;
             if (*B.dead) { ok = false; break; }
+            // PV of unit g_pv
+            if (g_pv < g_qk) {
+                const int r = g_pv & 3;
+                bool ready = lane0(mbar_test_wait(B.p + 8 * (g_pv & 1), (g_pv >> 1) & 1));
+                ready = ready && lane0(kCodes ? mbar_test_wait(B.vf_full, (uint32_t)g_pv & 1u)
+                                              : mbar_test_wait(B.full_v + 8 * rec_st[r], (uint32_t)(g_pv / S_) & 1u));
+                if (ready && rec_first[r] && rec_item[r] >= 1)
+                    ready = lane0(mbar_test_wait(B.ofree, (rec_item[r] - 1) & 1));
+                if (ready) {
+                    tc_fence_after();
+                    if (rec_first[r]) o_started = false;
+                    if (lane == 0) {
+                        if (rec_valid[r]) {
+                            const uint32_t pa = pbuf + (g_pv & 1) * kU2PBytes;
+                            const uint32_t vb =
+                                kCodes ? vfbuf : ring.stages + rec_st[r] * G::kStageBytes + 2 * kU2HalfBytes;
+#pragma unroll
+                            for (int k = 0; k < kU2Tokens / 16; ++k)
+                                umma_ss(tm + kU2ColO, umma_desc(pa + 32 * k, 16, 1024),
+                                        umma_desc(vb + 2048 * k, kU2HalfBytes, 1024), C::kIdescPV,
+                                        o_started || k > 0);
+                        }
+                        umma_commit(B.pv + 8 * (g_pv & 1));
+                        umma_commit(kCodes ? B.vf_free : B.empty + 8 * rec_st[r]);
+                    }
+                    __syncwarp();
+                    if (rec_valid[r]) o_started = true;
+                    ++g_pv;
+                    progressed = true;
+                }
+            }
             // QK of unit g_qk
             if (!qk_done && g_qk - g_pv <= 1) {
                 if (need_q && lane0(mbar_test_wait(B.q, n_qk & 1))) need_q = false;
@@ -2893,45 +2937,16 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                     progressed = true;
                 }
             }
-            // PV of unit g_pv
-            if (g_pv < g_qk) {
-                const int r = g_pv & 3;
-                bool ready = lane0(mbar_test_wait(B.p + 8 * (g_pv & 1), (g_pv >> 1) & 1));
-                ready = ready && lane0(kCodes ? mbar_test_wait(B.vf_full, (uint32_t)g_pv & 1u)
-                                              : mbar_test_wait(B.full_v + 8 * rec_st[r], (uint32_t)(g_pv / S_) & 1u));
-                if (ready && rec_first[r] && rec_item[r] >= 1)
-                    ready = lane0(mbar_test_wait(B.ofree, (rec_item[r] - 1) & 1));
-                if (ready) {
-                    tc_fence_after();
-                    if (rec_first[r]) o_started = false;
-                    if (lane == 0) {
-                        if (rec_valid[r]) {
-                            const uint32_t pa = pbuf + (g_pv & 1) * kU2PBytes;
-                            const uint32_t vb =
-                                kCodes ? vfbuf : ring.stages + rec_st[r] * G::kStageBytes + 2 * kU2HalfBytes;
-#pragma unroll
-                            for (int k = 0; k < kU2Tokens / 16; ++k)
-                                umma_ss(tm + kU2ColO, umma_desc(pa + 32 * k, 16, 1024),
-                                        umma_desc(vb + 2048 * k, kU2HalfBytes, 1024), C::kIdescPV,
-                                        o_started || k > 0);
-                        }
-                        umma_commit(B.pv + 8 * (g_pv & 1));
-                        umma_commit(kCodes ? B.vf_free : B.empty + 8 * rec_st[r]);
-                    }
-                    __syncwarp();
-                    if (rec_valid[r]) o_started = true;
-                    ++g_pv;
-                    progressed = true;
-                }
-            }
-            if (!progressed) __nanosleep(64);  // leave the issue slots to the softmax warp
-            const uint64_t now = global_timer_ns();
             if (progressed) {
-                t_last = now;
-            } else if (now - t_last > kWaitLimitNs) {  // nothing moved for the wait limit
-                if (lane == 0 && *B.dead == 0) atomicOr(&s_status_tma, kStatusTimeout);
-                if (lane == 0) *B.dead = 1;
-                ok = false;
+                idle = 0;
+            } else if (__nanosleep(20), ++idle % 32 == 0) {  // the time limit, read now and then
+                const uint64_t now = global_timer_ns();
+                if (idle == 32) t_last = now;
+                if (now - t_last > kWaitLimitNs) {  // nothing moved for the wait limit
+                    if (lane == 0 && *B.dead == 0) atomicOr(&s_status_tma, kStatusTimeout);
+                    if (lane == 0) *B.dead = 1;
+                    ok = false;
+                }
             }
         }
         // wait for the softmax warps (even after a give-up: they stop touching
@@ -3281,7 +3296,7 @@ cudaError_t launch_umma_grouped(const DecodeParams& p, const CUtensorMap& km,
     const long groups = p.query_start != nullptr ? (long)p.num_seqs * p.q_chunks
                                                  : (long)(p.num_seqs + gs - 1) / gs;
     const long items = (long)p.num_partitions * p.num_kv_heads * groups;
-    const long slots = 2L * sms;  // two CTAs per SM: 256 TMEM columns and <= 113 KB each
+    const long slots = (long)PA_U2_CTAS * sms;
     const unsigned grid = (unsigned)(items < slots ? items : slots);
     kernel<<<grid, C::kThreads, smem, stream>>>(km, vm, p, (int)items, gs);
     return cudaGetLastError();
@@ -3394,7 +3409,7 @@ bool grouped_is_tcgen05(int dtype, int head_dim, int gs, int group) {
 }
 
 int grouped_ctas_per_sm(int dtype, int head_dim, int gs, int group) {
-    if (grouped_is_tcgen05(dtype, head_dim, gs, group)) return 2;
+    if (grouped_is_tcgen05(dtype, head_dim, gs, group)) return PA_U2_CTAS;
     int cw = 1, nt = 1;
     grouped_shape(gs, group, &cw, &nt);
     return grouped_min_blocks(head_dim, cw, nt);
