@@ -2419,9 +2419,11 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
 }
 // Instruction descriptor for kind::f16: fp32 accumulator, bf16 (or, with
 // f16, f16) A and B, A K-major, B K-major or MN-major, shape M x N.
-__host__ __device__ constexpr uint32_t umma_idesc(int m, int n, bool b_mn_major, bool f16 = false) {
+__host__ __device__ constexpr uint32_t umma_idesc(int m, int n, bool b_mn_major, bool f16 = false,
+                                                  bool a_mn_major = false) {
     return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) |
-           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+           ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 // D (TMEM) (+)= A (shared) . B (shared)^T, issued by one thread.
 __device__ __forceinline__ void umma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
@@ -2541,20 +2543,21 @@ constexpr int kU2HalfBytes = kU2Tokens * 128;   // one d-half of a K or V tile: 
 // in flight to read at HBM rate: one CTA per SM with five bf16 stages (eight
 // 16 KB stages over codes), 200 KB of shared memory.
 #ifndef PA_U2_STAGES
-#define PA_U2_STAGES 5
+#define PA_U2_STAGES 3
 #endif
 #ifndef PA_U2_CODE_STAGES
-#define PA_U2_CODE_STAGES 8
+#define PA_U2_CODE_STAGES 4
 #endif
 #ifndef PA_U2_CTAS
-#define PA_U2_CTAS 1
+#define PA_U2_CTAS 2
 #endif
 constexpr int kU2PBytes = kU2Cols * 128;        // P tile: 32 rows x 64 16-bit tokens
-constexpr int kU2QBytes = 2 * 128 * 128;        // Q tile: 128 rows x 128 16-bit, two d-halves
-constexpr int kU2QOff = 2 * kU2PBytes;          // shared memory: [P0][P1][Q][ring][...]
-constexpr int kU2RingOff = kU2QOff + kU2QBytes;
+constexpr int kU2RingOff = 2 * kU2PBytes;       // shared memory: [P0][P1][ring][...]
+// TMEM columns: O^T (128 head_dim lanes x 32 query columns, fp32), then Q
+// (128 rows x 128 16-bit values, two per column: the A operand of QK), then S
+// (128 rows x 64 tokens, fp32) twice.
 constexpr uint32_t kU2TmemCols = 256;
-constexpr uint32_t kU2ColO = 0, kU2ColS = 128;  // S buffers at columns 128 and 192
+constexpr uint32_t kU2ColO = 0, kU2ColQ = 32, kU2ColS = 96;
 constexpr float kU2RescaleLog2 = 8.f;
 
 // Ring of the bf16 variant: box-major stages with K and V barriers of their own.
@@ -2596,13 +2599,12 @@ struct U2Cfg {
     static constexpr int kXl = kXf + 2 * 4 * 4;
     static constexpr int kExtBytes = kXl + 4 * 32 * 4;
     static constexpr size_t kSmem = (size_t)kExtOff + kExtBytes;
+    // QK: A = Q from TMEM, B = K K-major; PV (transposed): A = V^T MN-major
+    // (head_dim contiguous in the V tile), B = P K-major (tokens contiguous)
     static constexpr uint32_t kIdescQK = umma_idesc(128, 64, false, kCodes);
-    static constexpr uint32_t kIdescPV = umma_idesc(128, 128, true, kCodes);
+    static constexpr uint32_t kIdescPV = umma_idesc(128, kU2Cols, false, kCodes, true);
     static_assert(kU2RingOff % 1024 == 0 && kKfOff % 1024 == 0 && kVfOff % 1024 == 0,
                   "operand tiles on 1024-byte boundaries");
-    // the PV MMA reads 128 rows (16 KB) of a P buffer; rows 32..127 (results
-    // never used) come from the shared memory after it
-    static_assert(kU2PBytes + 16384 <= kExtOff, "P windows inside the CTA");
     static_assert(kSmem * PA_U2_CTAS + 1024 * PA_U2_CTAS <= 228 * 1024 && kSmem <= 227 * 1024,
                   "shared memory of PA_U2_CTAS CTAs per SM");
 };
@@ -2686,7 +2688,7 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         if (threadIdx.x == 0) atomicOr(&s_status_tma, kStatusSmemAlign);
         return;
     }
-    const uint32_t pbuf = raw, qbuf = raw + kU2QOff;
+    const uint32_t pbuf = raw;
     const uint32_t kfbuf = raw + C::kKfOff, vfbuf = raw + C::kVfOff;
     uint8_t* ext = smem_raw + C::kExtOff;
     uint32_t* hdr = reinterpret_cast<uint32_t*>(ext);
@@ -2882,8 +2884,8 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                                 kCodes ? vfbuf : ring.stages + rec_st[r] * G::kStageBytes + 2 * kU2HalfBytes;
 #pragma unroll
                             for (int k = 0; k < kU2Tokens / 16; ++k)
-                                umma_ss(tm + kU2ColO, umma_desc(pa + 32 * k, 16, 1024),
-                                        umma_desc(vb + 2048 * k, kU2HalfBytes, 1024), C::kIdescPV,
+                                umma_ss(tm + kU2ColO, umma_desc(vb + 2048 * k, kU2HalfBytes, 1024),
+                                        umma_desc(pa + 32 * k, 16, 1024), C::kIdescPV,
                                         o_started || k > 0);
                         }
                         umma_commit(B.pv + 8 * (g_pv & 1));
@@ -2911,8 +2913,7 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                             const uint32_t kb = kCodes ? kfbuf : ring.stages + st * G::kStageBytes;
 #pragma unroll
                             for (int k = 0; k < 8; ++k)
-                                umma_ss(tm + kU2ColS + 64 * (g_qk & 1),
-                                        umma_desc(qbuf + (k >> 2) * (kU2QBytes / 2) + (k & 3) * 32, 16, 1024),
+                                umma_ts(tm + kU2ColS + 64 * (g_qk & 1), tm + kU2ColQ + 8 * k,
                                         umma_desc(kb + (k >> 2) * kU2HalfBytes + (k & 3) * 32, 16, 1024),
                                         C::kIdescQK, k > 0);
                         }
@@ -2999,7 +3000,6 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         const uint32_t sg = sl0 < 0.f ? 0x80008000u : 0u;
         const uint4* src = reinterpret_cast<const uint4*>(qsrc_base +
             ((int64_t)(it.row0 + mem) * p.num_heads + (int64_t)it.kh * group + hd) * DQ * 2);
-        const uint32_t row = 32 * warp + lane;
         auto ldq = [&](int c) {
             const uint4 v = has && 8 * c < DQ ? ld_v4(src + c) : make_uint4(0u, 0u, 0u, 0u);
             return make_uint4(v.x ^ sg, v.y ^ sg, v.z ^ sg, v.w ^ sg);
@@ -3020,19 +3020,27 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             mul = pow2i(-sh);
             slc *= pow2i(sh);
         }
-#pragma unroll 4
-        for (int c = 0; c < 16; ++c) {
-            uint4 v = ldq(c);  // (again: a cache hit)
-            if constexpr (kCodes)
-                v = make_uint4(pack_f16x2(bf16_lo(v.x) * mul, bf16_hi(v.x) * mul),
-                               pack_f16x2(bf16_lo(v.y) * mul, bf16_hi(v.y) * mul),
-                               pack_f16x2(bf16_lo(v.z) * mul, bf16_hi(v.z) * mul),
-                               pack_f16x2(bf16_lo(v.w) * mul, bf16_hi(v.w) * mul));
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
-                         :: "r"(qbuf + (c >> 3) * (kU2QBytes / 2) + swz(row, c & 7)),
-                            "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+        // the row in its TMEM lane: head_dim 2i, 2i + 1 in column i (two halves
+        // of 32 columns)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            uint32_t w[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint4 v = ldq(8 * hf + c);  // (again: a cache hit)
+                if constexpr (kCodes)
+                    v = make_uint4(pack_f16x2(bf16_lo(v.x) * mul, bf16_hi(v.x) * mul),
+                                   pack_f16x2(bf16_lo(v.y) * mul, bf16_hi(v.y) * mul),
+                                   pack_f16x2(bf16_lo(v.z) * mul, bf16_hi(v.z) * mul),
+                                   pack_f16x2(bf16_lo(v.w) * mul, bf16_hi(v.w) * mul));
+                w[4 * c] = v.x;
+                w[4 * c + 1] = v.y;
+                w[4 * c + 2] = v.z;
+                w[4 * c + 3] = v.w;
+            }
+            tmem_st32(tm + lane_off + kU2ColQ + 32 * hf, w);
         }
-        fence_async_smem();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(B.q);
         return slc;
@@ -3105,20 +3113,20 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                     }
                     m_ref = nm;
                 }
-                // warp 0's TMEM lanes hold O's rows: rescale them once the PV of
-                // the previous unit is done
-                if (warp == 0 && __any_sync(0xffffffffu, resc)) {
+                // O^T (lanes: head_dim 32 warp .. + 31, column j: query column j)
+                // is rescaled column by column once the PV of the previous unit is
+                // done; lane j holds column j's factor (every warp holds every
+                // column's state, so all four take the same branch)
+                if (__any_sync(0xffffffffu, resc)) {
                     healthy = u2_wait(B, B.pv + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1);
                     if (healthy) {
                         tc_fence_after();
-#pragma unroll 1
-                        for (int c0 = 0; c0 < 128; c0 += 32) {
-                            uint32_t o[32];
-                            tmem_ld32(tm + lane_off + kU2ColO + c0, o);
+                        uint32_t o[32];
+                        tmem_ld32(tm + lane_off + kU2ColO, o);
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                            tmem_st32(tm + lane_off + kU2ColO + c0, o);
-                        }
+                        for (int j = 0; j < 32; ++j)
+                            o[j] = __float_as_uint(__uint_as_float(o[j]) * __shfl_sync(0xffffffffu, alpha, j));
+                        tmem_st32(tm + lane_off + kU2ColO, o);
                     }
                 }
             }
@@ -3179,42 +3187,34 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         // the next item's q: every QK of this item is complete (its last S was read)
         const GItem nxt = next_item();
         if (nxt.valid) sl_next = stage_q(nxt);
-        if (warp == 0) {
-            if (healthy) healthy = u2_wait(B, B.pv + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1);
+        // O^T: thread (warp, lane) holds head_dim d = 32 warp + lane of every
+        // column; column j's row, normaliser and flags come from lane j
+        if (healthy) healthy = u2_wait(B, B.pv + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1);
+        {
             const bool has = colv && mem < cur.nmem && t1 > cur.t0;
+            const bool wr = colv && mem < cur.nmem;
             const int64_t row = (int64_t)(cur.row0 + mem) * p.num_heads + (int64_t)cur.kh * group + hd;
             const float inv = (lt > 0.f ? 1.f / lt : 0.f) * (kCodes ? __ldg(p.v_scale + cur.kh) : 1.f);
+            const int d = 32 * warp + lane;
             if (healthy) {
                 tc_fence_after();
-#pragma unroll 1
-                for (int c0 = 0; c0 < 128; c0 += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(tm + lane_off + kU2ColO + c0, o);
-                    if (colv && mem < cur.nmem && c0 < DQ) {
+                uint32_t o[32];
+                tmem_ld32(tm + lane_off + kU2ColO, o);
+#pragma unroll
+                for (int j = 0; j < kU2Cols; ++j) {
+                    const bool wr_j = __shfl_sync(0xffffffffu, wr, j);
+                    const bool has_j = __shfl_sync(0xffffffffu, has, j);
+                    const int64_t row_j = __shfl_sync(0xffffffffu, row, j);
+                    const float val = __uint_as_float(o[j]) * __shfl_sync(0xffffffffu, inv, j);
+                    if (d < DQ) {
                         if (P == 1) {
-                            uint32_t w[16];
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                w[j] = lt > 0.f ? pack_bf16x2(__uint_as_float(o[2 * j]) * inv,
-                                                              __uint_as_float(o[2 * j + 1]) * inv)
-                                                : 0u;
-                            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row * DQ + c0);
-#pragma unroll
-                            for (int j = 0; j < 4; ++j)
-                                dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-                        } else if (has) {
-                            float4* dst = reinterpret_cast<float4*>(p.ws_o + (row * P + cur.part) * DQ + c0);
-#pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                dst[j] = lt > 0.f ? make_float4(__uint_as_float(o[4 * j]) * inv,
-                                                                __uint_as_float(o[4 * j + 1]) * inv,
-                                                                __uint_as_float(o[4 * j + 2]) * inv,
-                                                                __uint_as_float(o[4 * j + 3]) * inv)
-                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (wr_j) static_cast<__nv_bfloat16*>(p.out)[row_j * DQ + d] = __float2bfloat16_rn(val);
+                        } else if (has_j) {
+                            p.ws_o[(row_j * P + cur.part) * DQ + d] = val;
                         }
                     }
                 }
-                if (P > 1 && has) {
+                if (warp == 0 && P > 1 && has) {
                     float* ml = p.ws_ml + (row * P + cur.part) * 2;
                     ml[0] = lt > 0.f ? m_ref : -INFINITY;
                     ml[1] = lt;
