@@ -2734,7 +2734,7 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             mbar_init(B.p + 8 * i, 4);
         }
         mbar_init(B.q, 4);
-        mbar_init(B.ofree, 4);
+        mbar_init(B.ofree, 1);  // warp 0's final commit: every PV it issued is complete
         mbar_init(B.done, 4);
         mbar_init(B.fin, 1);
         for (int i = 0; i < 4; ++i) mbar_init(B.kf_full + 8 * i, 2);
@@ -2846,112 +2846,49 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
     }
 
     if (warp == 5) {
-        // MMA issuer, event-driven: lane 0 issues; each turn it issues the next
-        // PV if that unit's P is written and its V landed (for an item's first
-        // unit, once the previous item's output left O), then the next QK if its
-        // K tile has landed (and its S buffer is free: the PV two units back has
-        // been issued). Neither waits behind the other, so a stage is released as soon
-        // as its softmax is done and the next loads go out without a DRAM round
-        // trip behind an unrelated wait.
-        int g_qk = 0, g_pv = 0, n_qk = 0;
-        bool need_q = true, first_qk = true, qk_done = false, o_started = false, ok = true;
-        // per unit g (slot g & 3): stage, valid, first unit of its item, item index
-        int rec_st[4], rec_item[4];
-        bool rec_valid[4], rec_first[4];
+        // QK issuer: lane 0 issues S = Q . K^T of each unit once the item's q is
+        // in TMEM, the unit's K tile has landed and its S buffer is free (the
+        // softmax of the unit two back has read it). The PVs are issued by the
+        // softmax warps themselves, as soon as P is written.
+        int g = 0, n = 0;
+        bool ok = true;
         GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
-        if (!cur.valid) qk_done = true;
-        auto lane0 = [&](bool x) { return __shfl_sync(0xffffffffu, x, 0); };
-        uint64_t t_last = 0;
-        uint32_t idle = 0;  // polls since the last issue
-        while (ok && !(qk_done && g_pv == g_qk)) {
-            bool progressed = false;
-            if (*B.dead) { ok = false; break; }
-            // PV of unit g_pv
-            if (g_pv < g_qk) {
-                const int r = g_pv & 3;
-                bool ready = lane0(mbar_test_wait(B.p + 8 * (g_pv & 1), (g_pv >> 1) & 1));
-                ready = ready && lane0(kCodes ? mbar_test_wait(B.vf_full, (uint32_t)g_pv & 1u)
-                                              : mbar_test_wait(B.full_v + 8 * rec_st[r], (uint32_t)(g_pv / S_) & 1u));
-                if (ready && rec_first[r] && rec_item[r] >= 1)
-                    ready = lane0(mbar_test_wait(B.ofree, (rec_item[r] - 1) & 1));
-                if (ready) {
-                    tc_fence_after();
-                    if (rec_first[r]) o_started = false;
-                    if (lane == 0) {
-                        if (rec_valid[r]) {
-                            const uint32_t pa = pbuf + (g_pv & 1) * kU2PBytes;
-                            const uint32_t vb =
-                                kCodes ? vfbuf : ring.stages + rec_st[r] * G::kStageBytes + 2 * kU2HalfBytes;
-#pragma unroll
-                            for (int k = 0; k < kU2Tokens / 16; ++k)
-                                umma_ss(tm + kU2ColO, umma_desc(vb + 2048 * k, kU2HalfBytes, 1024),
-                                        umma_desc(pa + 32 * k, 16, 1024), C::kIdescPV,
-                                        o_started || k > 0);
-                        }
-                        umma_commit(B.pv + 8 * (g_pv & 1));
-                        umma_commit(kCodes ? B.vf_free : B.empty + 8 * rec_st[r]);
-                    }
-                    __syncwarp();
-                    if (rec_valid[r]) o_started = true;
-                    ++g_pv;
-                    progressed = true;
-                }
-            }
-            // QK of unit g_qk
-            if (!qk_done && g_qk - g_pv <= 1) {
-                if (need_q && lane0(mbar_test_wait(B.q, n_qk & 1))) need_q = false;
-                const int st = g_qk % S_;
-                const bool kready =
-                    !need_q && lane0(kCodes ? mbar_test_wait(B.kf_full + 8 * (g_qk & 3), (uint32_t)(g_qk >> 2) & 1u)
-                                            : mbar_test_wait(B.full_k + 8 * st, (uint32_t)(g_qk / S_) & 1u));
-                if (kready) {
-                    tc_fence_after();
-                    const uint32_t h = kCodes ? hc[g_qk & 3] : hdr[st];
-                    const bool v = (kCodes ? hc[8 + (g_qk & 3)] : (uint32_t)valid[st]) != 0;
-                    if (lane == 0) {
-                        if (v) {
-                            const uint32_t kb = kCodes ? kfbuf : ring.stages + st * G::kStageBytes;
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                umma_ts(tm + kU2ColS + 64 * (g_qk & 1), tm + kU2ColQ + 8 * k,
-                                        umma_desc(kb + (k >> 2) * kU2HalfBytes + (k & 3) * 32, 16, 1024),
-                                        C::kIdescQK, k > 0);
-                        }
-                        umma_commit(B.s + 8 * (g_qk & 1));
-                        if (kCodes) umma_commit(B.kf_free);
-                    }
-                    __syncwarp();
-                    const int r = g_qk & 3;
-                    rec_st[r] = st;
-                    rec_valid[r] = v;
-                    rec_first[r] = first_qk;
-                    rec_item[r] = n_qk;
-                    first_qk = false;
-                    ++g_qk;
-                    if (h & kUnitLast) {
-                        ++n_qk;
-                        need_q = true;
-                        first_qk = true;
-                        cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
-                        if (!cur.valid) qk_done = true;
-                    }
-                    progressed = true;
-                }
-            }
-            if (progressed) {
-                idle = 0;
-            } else if (__nanosleep(20), ++idle % 32 == 0) {  // the time limit, read now and then
-                const uint64_t now = global_timer_ns();
-                if (idle == 32) t_last = now;
-                if (now - t_last > kWaitLimitNs) {  // nothing moved for the wait limit
-                    if (lane == 0 && *B.dead == 0) atomicOr(&s_status_tma, kStatusTimeout);
-                    if (lane == 0) *B.dead = 1;
+        while (cur.valid && ok) {
+            if (!u2_wait(B, B.q, n & 1)) { ok = false; break; }
+            for (;;) {
+                const int st = g % S_;
+                if (g >= 2 && !u2_wait(B, B.p + 8 * (g & 1), ((g - 2) >> 1) & 1)) { ok = false; break; }
+                if (kCodes) {
+                    if (!u2_wait(B, B.kf_full + 8 * (g & 3), (uint32_t)(g >> 2) & 1u)) { ok = false; break; }
+                } else if (!u2_wait(B, B.full_k + 8 * st, (uint32_t)(g / S_) & 1u)) {
                     ok = false;
+                    break;
                 }
+                tc_fence_after();
+                const uint32_t h = kCodes ? hc[g & 3] : hdr[st];
+                const bool v = (kCodes ? hc[8 + (g & 3)] : (uint32_t)valid[st]) != 0;
+                if (lane == 0) {
+                    if (v) {
+                        const uint32_t kb = kCodes ? kfbuf : ring.stages + st * G::kStageBytes;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            umma_ts(tm + kU2ColS + 64 * (g & 1), tm + kU2ColQ + 8 * k,
+                                    umma_desc(kb + (k >> 2) * kU2HalfBytes + (k & 3) * 32, 16, 1024),
+                                    C::kIdescQK, k > 0);
+                    }
+                    umma_commit(B.s + 8 * (g & 1));
+                    if (kCodes) umma_commit(B.kf_free);
+                }
+                __syncwarp();
+                ++g;
+                if (h & kUnitLast) break;
             }
+            ++n;
+            if (ok) cur = gitem_next(walk, p, num_items, gs, ipb, lane, false, false);
         }
         // wait for the softmax warps (even after a give-up: they stop touching
-        // TMEM before they arrive), then for every issued MMA, then free TMEM
+        // TMEM, and their PVs are complete, before they arrive), then for every
+        // QK issued here, then free TMEM
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(B.done, 0)) && lane == 0)
             atomicOr(&s_status_tma, kStatusTimeout);
         if (lane == 0) umma_commit(B.fin);
@@ -3051,6 +2988,7 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
         const int t1 = __shfl_sync(0xffffffffu, cur.t1_lane, mem & (kMaxGroupSeqs - 1));
         const float sl = sl_next;
         float m_ref = -INFINITY, l = 0.f;
+        bool o_started = false;  // warp 0: a PV of this item has written O^T
         for (;;) {
             const int b = g & 1, st = g % S_;
             // S of unit g (and with it every earlier MMA: the PV of unit g - 2
@@ -3148,6 +3086,9 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                 }
             }
             l += ps;
+            // P buffer b is read by the PV of unit g - 2, issued by warp 0 at the
+            // end of that unit: it must be complete before P is rewritten
+            if (g >= 2 && healthy) healthy = u2_wait(B, B.pv + 8 * b, ((g - 2) >> 1) & 1);
             // P row `col`, tokens 16 warp .. + 15: 16-byte chunks 2 warp, 2 warp + 1
             const uint32_t prow = pbuf + b * kU2PBytes;
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
@@ -3175,7 +3116,35 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
+            // S buffer b has been read (the QK issuer may overwrite it)
             if (lane == 0) mbar_arrive(B.p + 8 * b);
+            // O^T += V^T . P^T by warp 0's lane 0 once every warp's P rows are
+            // written (and, over bf16, V has landed); then the stage (bf16) or the
+            // f16 V tile (codes) is released. The first unit of an item overwrites
+            // O^T: the previous item's output was read before this item began.
+            named_barrier(1, 128);
+            if (warp == 0) {
+                if (healthy) {
+                    healthy = kCodes ? u2_wait(B, B.vf_full, (uint32_t)g & 1u)
+                                     : u2_wait(B, B.full_v + 8 * st, (uint32_t)(g / S_) & 1u);
+                }
+                tc_fence_after();
+                if (lane == 0 && healthy) {
+                    if (v) {
+                        const uint32_t vb =
+                            kCodes ? vfbuf : ring.stages + st * G::kStageBytes + 2 * kU2HalfBytes;
+#pragma unroll
+                        for (int k = 0; k < kU2Tokens / 16; ++k)
+                            umma_ss(tm + kU2ColO, umma_desc(vb + 2048 * k, kU2HalfBytes, 1024),
+                                    umma_desc(prow + 32 * k, 16, 1024), C::kIdescPV,
+                                    o_started || k > 0);
+                    }
+                    umma_commit(B.pv + 8 * b);
+                    umma_commit(kCodes ? B.vf_free : B.empty + 8 * st);
+                }
+                if (v) o_started = true;
+                __syncwarp();
+            }
             ++g;
             if (h & kUnitLast) break;
         }
@@ -3221,11 +3190,18 @@ decode_umma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                 }
             }
         }
-        tc_fence_before();
+        tc_fence_before();  // O^T reads done before the next item's first PV (after a barrier)
         __syncwarp();
-        if (lane == 0) mbar_arrive(B.ofree);
         cur = nxt;
         ++n;
+    }
+    // warp 0 issued the PVs: all of them complete before TMEM may be freed
+    if (warp == 0) {
+        if (lane == 0) umma_commit(B.ofree);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(B.ofree, 0)) && lane == 0)
+            atomicOr(&s_status_tma, kStatusTimeout);
+        tc_fence_before();
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(B.done);
