@@ -144,8 +144,10 @@ struct Plan {
     int q_chunks;       // multi: items per (sequence, kv head, partition) = ceil(max_query_len / gs)
     int partition_size;
     int num_partitions;
-    size_t ws_bytes;
+    size_t ws_bytes;      // partial results: the least workspace the call accepts
     size_t ws_ml_offset;
+    size_t sched_offset;  // persistent kernels: the dynamic schedule's counter
+    size_t ws_full;       // the workspace size reported: partials + schedule
 };
 
 int round_up16(int x) { return (x + 15) / 16 * 16; }
@@ -275,6 +277,11 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
         plan->ws_ml_offset = (o_bytes + 255) / 256 * 256;
         plan->ws_bytes = plan->ws_ml_offset + rows * 2 * sizeof(float);
     }
+    // The persistent tensor-core kernel claims its work items from a counter
+    // in the 256 bytes after the partials (zeroed by the call before it
+    // launches); a workspace without them runs the static schedule.
+    plan->sched_offset = (plan->ws_bytes + 255) / 256 * 256;
+    plan->ws_full = plan->use_mma && !plan->grouped ? plan->sched_offset + 256 : plan->ws_bytes;
     return PA_OK;
 }
 
@@ -331,13 +338,18 @@ static int decode_impl(void* out, const void* q, const void* k_cache, const void
         return fail(PA_ERR_INVALID_ARG, "max_context_len %d exceeds block_table_stride %d * "
                     "block_size %d", max_context_len, block_table_stride, cache->block_size);
     if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    const bool ws_aligned = (reinterpret_cast<uintptr_t>(workspace) & 255u) == 0;
     if (plan.ws_bytes > 0) {
         if (!workspace || workspace_bytes < plan.ws_bytes)
             return fail(PA_ERR_WORKSPACE, "pa_decode needs %zu workspace bytes, got %zu at %p",
                         plan.ws_bytes, workspace_bytes, workspace);
-        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-            return fail(PA_ERR_ALIGN, "pa_decode: workspace must be 256-byte aligned");
+        if (!ws_aligned) return fail(PA_ERR_ALIGN, "pa_decode: workspace must be 256-byte aligned");
     }
+    // the dynamic schedule when the workspace holds its counter (the results are
+    // the same bit for bit either way: an item's arithmetic does not depend on
+    // the CTA that runs it)
+    const bool dyn_sched =
+        plan.ws_full > plan.ws_bytes && workspace && ws_aligned && workspace_bytes >= plan.ws_full;
     pa::DecodeParams p;
     p.out = out;
     p.q = q;
@@ -367,7 +379,14 @@ static int decode_impl(void* out, const void* q, const void* k_cache, const void
     p.query_start = plan.multi ? query_start : nullptr;
     p.q_chunks = plan.q_chunks;
     p.num_rows = plan.multi ? num_query_tokens : num_seqs;
+    p.sched = dyn_sched ? reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) +
+                                                          plan.sched_offset)
+                        : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (p.sched) {
+        const cudaError_t me = cudaMemsetAsync(p.sched, 0, sizeof(unsigned int), st);
+        if (me != cudaSuccess) return fail_cuda(me, "pa_decode schedule reset");
+    }
     CUtensorMap kmap, vmap;
     if ((rc = make_cache_map(&kmap, k_cache, cache)) != PA_OK) return rc;
     if ((rc = make_cache_map(&vmap, v_cache, cache)) != PA_OK) return rc;
@@ -523,7 +542,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t max
     Plan plan;
     if (plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan) != PA_OK)
         return 0;
-    return plan.ws_bytes;
+    return plan.ws_full;
 }
 
 int pa_decode_num_partitions(int32_t num_seqs, int32_t num_heads, int32_t max_context_len,
@@ -611,7 +630,7 @@ size_t pa_decode_multi_workspace_size(int32_t num_seqs, int32_t num_query_tokens
         plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan, 1,
                     num_query_tokens, max_query_len) != PA_OK)
         return 0;
-    return plan.ws_bytes;
+    return plan.ws_full;
 }
 
 int pa_decode_multi_num_partitions(int32_t num_seqs, int32_t num_query_tokens,
@@ -633,7 +652,7 @@ size_t pa_decode_grouped_workspace_size(int32_t num_seqs, int32_t num_heads,
     if (plan_decode(num_seqs, num_heads, max_context_len, cache, partition_size, &plan,
                     group_size) != PA_OK)
         return 0;
-    return plan.ws_bytes;
+    return plan.ws_full;
 }
 
 int pa_decode_grouped_num_partitions(int32_t num_seqs, int32_t num_heads,

@@ -65,9 +65,6 @@ namespace {
 #ifndef PA_MMA_SPLIT_QK
 #define PA_MMA_SPLIT_QK 0
 #endif
-#ifndef PA_MMA_PREFETCH_Q
-#define PA_MMA_PREFETCH_Q 1
-#endif
 
 
 constexpr int kBoxBytes = 16 * 128;  // 16 rows x 128 bytes
@@ -1067,6 +1064,125 @@ __device__ __forceinline__ Item item_next(ItemWalk& w, const DecodeParams& p, in
     }
 }
 
+// Dynamic schedule of a persistent CTA: the producer claims work items from
+// the launch's counter in order (so CTAs that stream faster take more items,
+// and every CTA ends within about one item of the others) and hands them to
+// the consumer warps through kItemQ slots with a full / empty mbarrier pair
+// each. The producer keeps one claimed item ahead of the one it issues, so an
+// item is in the queue before any of the previous item's loads wait for ring
+// space: the consumers, which take the next item when they start one (to
+// fetch its q early), never wait for an item the producer cannot yet claim.
+// Slot value -1 ends the stream. Empty items (a partition past the context)
+// are skipped by the producer, except with one partition, where their heads
+// get a zero output from the consumers.
+constexpr int kItemQ = 4;
+constexpr int kItemQBytes = 2 * kItemQ * 8 + 2 * kItemQ * 4;
+
+struct ItemQueue {
+    uint32_t full, empty;  // shared addresses of the barriers, slot i at + 8 i
+    int* u;                // [kItemQ] item index, -1: no more items
+    int* t1;               // [kItemQ] end of the item's tokens
+};
+
+__device__ __forceinline__ ItemQueue item_queue_setup(uint8_t* at, int consumers) {
+    ItemQueue q;
+    q.full = smem_u32(at);
+    q.empty = q.full + 8 * kItemQ;
+    q.u = reinterpret_cast<int*>(at + 16 * kItemQ);
+    q.t1 = q.u + kItemQ;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kItemQ; ++i) {
+            mbar_init(q.full + 8 * i, 1);
+            mbar_init(q.empty + 8 * i, consumers);
+        }
+        fence_barrier_init();
+    }
+    return q;
+}
+
+__device__ __forceinline__ Item item_of(const DecodeParams& p, int u, int t1) {
+    Item it;
+    it.valid = u >= 0;
+    it.part = it.valid ? u % p.num_partitions : 0;
+    const int rest = it.valid ? u / p.num_partitions : 0;
+    it.kh = rest % p.num_kv_heads;
+    it.s = rest / p.num_kv_heads;
+    it.t0 = it.part * p.partition_size;
+    it.t1 = t1;
+    return it;
+}
+
+// Producer side, whole warp: finish a claim whose counter value lane 0 holds
+// in `ticket` (claiming again past empty items). Lane 0 reports context
+// lengths out of range, once per sequence (its first partition).
+__device__ __forceinline__ Item item_claim_finish(const DecodeParams& p, int num_items,
+                                                  unsigned ticket, int lane) {
+    for (;;) {
+        const unsigned u = __shfl_sync(0xffffffffu, ticket, 0);
+        if (u >= (unsigned)num_items) {
+            Item none;
+            none.valid = false;
+            return none;
+        }
+        Item it = item_of(p, (int)u, 0);
+        int ctx = 0;
+        if (lane == 0)
+            ctx = clamp_ctx(__ldg(p.context_lens + it.s), p.max_context_len, it.part == 0);
+        ctx = __shfl_sync(0xffffffffu, ctx, 0);
+        it.t1 = min(ctx, it.t0 + p.partition_size);
+        if (it.t0 < it.t1 || p.num_partitions == 1) return it;
+        if (lane == 0) ticket = atomicAdd(p.sched, 1u);
+    }
+}
+
+// Producer: put the k-th item (or the end of the stream) in its slot. False if
+// the wait for the slot ran out.
+__device__ __forceinline__ bool item_push(const DecodeParams& p, const ItemQueue& q, int k,
+                                          const Item& it, int lane) {
+    const int slot = k % kItemQ;
+    const uint32_t round = (uint32_t)(k / kItemQ);
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(q.empty + 8 * slot, (round & 1u) ^ 1u))) {
+        if (lane == 0) atomicOr(&s_status_tma, kStatusTimeout);
+        return false;
+    }
+    if (lane == 0) {
+        q.u[slot] = it.valid ? it.part + p.num_partitions * (it.kh + p.num_kv_heads * it.s) : -1;
+        q.t1[slot] = it.valid ? it.t1 : 0;
+        mbar_arrive(q.full + 8 * slot);  // release: the slot's words are visible to its readers
+    }
+    __syncwarp();
+    return true;
+}
+
+// Consumer warp: take the k-th item (the end of the stream if `dead` or the
+// wait ran out, which also sets `dead`).
+__device__ __forceinline__ Item item_pop(const DecodeParams& p, const ItemQueue& q, int k,
+                                         int lane, bool& dead) {
+    Item it;
+    it.valid = false;
+    if (dead) return it;
+    const int slot = k % kItemQ;
+    const uint32_t round = (uint32_t)(k / kItemQ);
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(q.full + 8 * slot, round & 1u))) {
+        if (lane == 0) atomicOr(&s_status_tma, kStatusTimeout);
+        dead = true;
+        return it;
+    }
+    const int u = q.u[slot], t1 = q.t1[slot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q.empty + 8 * slot);
+    return item_of(p, u, t1);
+}
+
+// AND of `pred` over the first `threads` threads of the CTA (named barrier 2).
+__device__ __forceinline__ bool consumers_all(bool pred, int threads) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n"
+                 " bar.red.and.pred p, 2, %2, q;\n selp.u32 %0, 1, 0, p;\n}"
+                 : "=r"(r) : "r"((uint32_t)pred), "r"(threads) : "memory");
+    return r != 0;
+}
+
 // Persistent: each CTA walks its work items. The producer streams the items'
 // sub-tiles through the ring without a break between items (block-table
 // entries fetched one 32-sub-tile batch ahead), while the consumers finish one
@@ -1094,17 +1210,19 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
     const int P = p.num_partitions;
     const int group = p.num_heads / p.num_kv_heads;
     Ring ring;
-    uint8_t* base = setup_ring<G>(smem_raw, ring, merge_bytes<D>());
+    uint8_t* base = setup_ring<G>(smem_raw, ring, merge_bytes<D>() + kItemQBytes);
     if (base == nullptr) {
         if (threadIdx.x == 0) atomicOr(&s_status_tma, kStatusSmemAlign);
         return;
     }
     float* merge_buf = reinterpret_cast<float*>(base + G::kRingBytes);
     int merge_sel = 0;  // which half of the double-buffered merge area this item uses
+    const bool dyn = p.sched != nullptr;  // dynamic schedule (else item u to CTA u mod grid)
+    const ItemQueue iq = item_queue_setup(base + G::kRingBytes + merge_bytes<D>(), kConsumerWarps);
     ItemWalk walk;
     walk.k = 0;
     walk.kbase = 0;
-    walk.ctx_lane = item_ctx_load(p, num_items, 0, lane, warp == 0);
+    walk.ctx_lane = dyn ? -1 : item_ctx_load(p, num_items, 0, lane, warp == 0);
     __syncthreads();
 
     if (warp == kConsumerWarps) {  // producer
@@ -1113,9 +1231,19 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
             prefetch_tensormap(&vmap);
         }
         bool dead = false;
-        int g = 0, issued = 0;
-        // batches of up to 32 sub-tiles, the next batch's table entries in flight
-        Item cur = item_next(walk, p, num_items, lane, false, false);
+        int g = 0, issued = 0, kq = 0;
+        // Batches of up to 32 sub-tiles, the next batch's table entries in flight.
+        // Dynamic schedule: an item is claimed (and queued for the consumers) once
+        // every sub-tile of the previous one is issued, so a CTA holds at most the
+        // ring's worth of work ahead of its consumers when the items run out.
+        auto claim = [&]() -> Item {
+            unsigned ticket = 0;
+            if (lane == 0) ticket = atomicAdd(p.sched, 1u);
+            const Item it = item_claim_finish(p, num_items, ticket, lane);
+            if (!item_push(p, iq, kq++, it, lane)) dead = true;
+            return it;
+        };
+        Item cur = dyn ? claim() : item_next(walk, p, num_items, lane, false, false);
         int cur_base = 0;
         int phys_cur = -1;
         if (cur.valid && lane < ((cur.t1 - cur.t0 + 15) >> 4))
@@ -1123,20 +1251,27 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                              ((cur.t0 + (lane << 4)) >> p.log2_block_size));
         while (cur.valid && !dead) {
             const int n_sub = (cur.t1 - cur.t0 + 15) >> 4;
+            const bool last = cur_base + 32 >= n_sub;
             Item nxt = cur;
             int nxt_base = cur_base + 32;
-            if (nxt_base >= n_sub) {
-                nxt = item_next(walk, p, num_items, lane, false, false);
+            if (last) {
+                if (!dyn) nxt = item_next(walk, p, num_items, lane, false, false);
                 nxt_base = 0;
             }
             int phys_nxt = -1;
-            if (nxt.valid && nxt_base + lane < ((nxt.t1 - nxt.t0 + 15) >> 4))
+            if (!(dyn && last) && nxt.valid && nxt_base + lane < ((nxt.t1 - nxt.t0 + 15) >> 4))
                 phys_nxt = __ldg(p.block_tables + (int64_t)nxt.s * p.table_stride +
                                  ((nxt.t0 + ((nxt_base + lane) << 4)) >> p.log2_block_size));
             const int cnt = min(32, n_sub - cur_base);
             issue_batch<G>(&kmap, &vmap, p, ring, g, cnt, phys_cur, cur.kh,
                               cur.t0 + ((cur_base + lane) << 4), lane, issued, dead);
             g += cnt;
+            if (dyn && last && !dead) {
+                nxt = claim();
+                if (nxt.valid && lane < ((nxt.t1 - nxt.t0 + 15) >> 4))
+                    phys_nxt = __ldg(p.block_tables + (int64_t)nxt.s * p.table_stride +
+                                     ((nxt.t0 + (lane << 4)) >> p.log2_block_size));
+            }
             cur = nxt;
             cur_base = nxt_base;
             phys_cur = phys_nxt;
@@ -1171,15 +1306,29 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
             for (int jp = 0; jp < KCH; ++jp) q[jp] = make_uint4(0u, 0u, 0u, 0u);
         }
     };
-    Item cur = item_next(walk, p, num_items, lane, warp == 0, true);
+    // Dynamic schedule: the k-th queued item; the consumer warps take an item
+    // only if every one of them got it (a wait that ran out in one warp ends
+    // the stream for all, so they never split on the merge barriers).
+    int kq = 0;
+    auto next_item = [&]() -> Item {
+        if (!dyn) return item_next(walk, p, num_items, lane, warp == 0, true);
+        Item it = item_pop(p, iq, kq++, lane, dead);
+        if constexpr (kConsumerWarps > 1) {
+            if (!consumers_all(it.valid, kConsumerWarps * 32)) it.valid = false;
+        }
+        return it;
+    };
+    Item cur = next_item();
     uint4 qcur[KCH];
     load_q(cur, qcur);
     while (cur.valid) {
-        Item nxt = item_next(walk, p, num_items, lane, warp == 0, true);
-#if PA_MMA_PREFETCH_Q
+        Item nxt;
         uint4 qnxt[KCH];
-        load_q(nxt, qnxt);  // in flight while this item is processed
-#endif
+        if (!dyn) {
+            // static schedule: the next item is known, its q in flight meanwhile
+            nxt = next_item();
+            load_q(nxt, qnxt);
+        }
         int qsh = 0;  // over codes: this item's q to f16, scaled by 2^-qsh
         if constexpr (kCodes) {
             qsh = q_shift_warp(q_raw_amax(qcur));
@@ -1191,6 +1340,10 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
             if (P == 1)
                 for (int idx = threadIdx.x; idx < group * DQ; idx += kConsumerWarps * 32)
                     Elem<T>::store(p.out, head0 * DQ + idx, 0.f);
+            if (dyn) {
+                nxt = next_item();
+                load_q(nxt, qnxt);
+            }
         } else {
             const int t0 = cur.t0, t1 = cur.t1;
             const int n_sub = (t1 - t0 + 15) >> 4;
@@ -1235,6 +1388,12 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 }
             }
             g += n_sub;
+            if (dyn) {
+                // the next item is queued by now (its loads follow this item's);
+                // its q is in flight during this item's merge and store
+                nxt = next_item();
+                load_q(nxt, qnxt);
+            }
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {
                 l0 += __shfl_xor_sync(0xffffffffu, l0, off);
@@ -1346,12 +1505,8 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
             }
         }
         cur = nxt;
-#if PA_MMA_PREFETCH_Q
 #pragma unroll
         for (int jp = 0; jp < KCH; ++jp) qcur[jp] = qnxt[jp];
-#else
-        load_q(cur, qcur);
-#endif
     }
 }
 
@@ -3228,7 +3383,7 @@ template <int D, typename TC = __nv_bfloat16>
 cudaError_t launch_mma_t(const DecodeParams& p, const CUtensorMap& km, const CUtensorMap& vm,
                          cudaStream_t stream) {
     using G = MmaGeom<D, TC>;
-    constexpr size_t smem = smem_bytes<G>(merge_bytes<D>());
+    constexpr size_t smem = smem_bytes<G>(merge_bytes<D>() + kItemQBytes);
     auto kernel = decode_tma_mma_kernel<D, TC>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

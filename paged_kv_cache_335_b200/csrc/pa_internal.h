@@ -54,6 +54,10 @@ struct DecodeParams {
     // built for 128-code rows and take head_dim 64 pools as rows whose upper
     // half the TMA fills with zero codes (q zero there too, outputs not stored).
     int32_t head_dim;
+    // Dynamic item schedule of the persistent kernels: a counter zeroed before
+    // the launch, from which CTAs claim work items in order (nullptr: static
+    // schedule, item u to CTA u mod grid).
+    unsigned int* sched;
 };
 
 struct CopyParams {

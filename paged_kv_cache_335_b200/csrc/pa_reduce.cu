@@ -30,8 +30,9 @@ __device__ __forceinline__ int clamp_context(int ctx, int max_ctx) {
 //
 // Warp w takes partitions w, w + 4, ...; each lane holds D / 32 consecutive
 // elements of a partial output, and a warp issues the loads of up to kBatch
-// partitions before it uses any of them, so one round trip to memory covers
-// the typical partition count. The warps' sums meet in shared memory.
+// partitions (with the (m, l) loads of the maximum) before it uses any of
+// them, so one round trip to memory covers the typical partition count. The
+// warps' sums meet in shared memory.
 constexpr int kWarps = kThreads / 32;
 constexpr int kBatch = 16;
 
@@ -76,6 +77,22 @@ partition_reduce_kernel(const DecodeParams p) {
     const int64_t out_row = (int64_t)row * p.num_heads + h;
     const float2* ml = reinterpret_cast<const float2*>(p.ws_ml + out_row * p.num_partitions * 2);
     const float* o = p.ws_o + out_row * p.num_partitions * D;
+    // A warp's batch of partials (output rows and their (m, l)) is requested
+    // before the maximum over all partitions is formed, so the first batch and
+    // the maxima share one round trip to memory.
+    Vec ov[kBatch];
+    float2 mlv[kBatch];
+    auto load_batch = [&](int j0) {
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int j = j0 + u * kWarps;
+            if (j < n) {
+                ov[u] = *reinterpret_cast<const Vec*>(o + (int64_t)j * D + lane * V);
+                mlv[u] = ml[j];
+            }
+        }
+    };
+    load_batch(warp);
     // M over all partitions, by every warp (no block barrier needed for it)
     float M = -INFINITY;
     for (int j = lane; j < n; j += 32) M = fmaxf(M, ml[j].x);
@@ -86,16 +103,7 @@ partition_reduce_kernel(const DecodeParams p) {
     for (int k = 0; k < V; ++k) acc[k] = 0.f;
     float L = 0.f;
     for (int j0 = warp; j0 < n; j0 += kWarps * kBatch) {
-        Vec ov[kBatch];
-        float2 mlv[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int j = j0 + u * kWarps;
-            if (j < n) {
-                ov[u] = *reinterpret_cast<const Vec*>(o + (int64_t)j * D + lane * V);
-                mlv[u] = ml[j];
-            }
-        }
+        if (j0 != warp) load_batch(j0);
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int j = j0 + u * kWarps;

@@ -68,7 +68,13 @@ def test_decode_needs_workspace_when_split(lib):
     assert need >= 8 * 8 * (128 + 2) * 4
     rc = _decode_rc(lib, desc, num_seqs=1, num_heads=8, max_ctx=4096, stride=256, ps=512)
     assert rc == pa.PA_ERR_WORKSPACE
-    assert lib.pa_decode_workspace_size(1, 8, 4096, ctypes.byref(desc), -1) == 0
+    # unsplit: no partials, only the 256 bytes of the tensor-core kernel's dynamic
+    # schedule, which a call may omit (it then runs the static schedule)
+    assert lib.pa_decode_workspace_size(1, 8, 4096, ctypes.byref(desc), -1) == 256
+    assert lib.pa_decode_workspace_size(1, 8, 4096, ctypes.byref(desc), 512) == \
+        (8 * 8 * 128 * 4 + 255) // 256 * 256 + (8 * 8 * 2 * 4 + 255) // 256 * 256 + 256
+    d13 = _desc(num_kv_heads=8)  # one query head per kv head: the CUDA-core kernel, no schedule
+    assert lib.pa_decode_workspace_size(1, 8, 4096, ctypes.byref(d13), -1) == 0
 
 
 def test_partition_policy(lib):
@@ -105,8 +111,9 @@ def test_grouped_partition_policy(lib):
         lib.pa_decode_num_partitions(2, 64, 4096, ctypes.byref(f32), 0)
     for bad in (0, 9, -1):
         assert f(128, 64, 2303, ctypes.byref(d70), bad, 0) == pa.PA_ERR_INVALID_ARG
+    # the same partials as pa_decode's split (which adds its 256-byte schedule counter)
     assert lib.pa_decode_grouped_workspace_size(8, 64, 32768, ctypes.byref(d70), 4, 512) == \
-        lib.pa_decode_workspace_size(8, 64, 32768, ctypes.byref(d70), 512)
+        lib.pa_decode_workspace_size(8, 64, 32768, ctypes.byref(d70), 512) - 256
 
 
 def test_grouped_decode_rejects_bad_group_size(lib):
