@@ -135,6 +135,8 @@ constexpr int kMaxPartitions = 4096;
 constexpr int kAutoPartition = 512;    // CUDA-core kernel: partition when splitting
 constexpr double kMmaItemOverhead = 8.0; // tensor-core kernel: per-item cost, in 16-token sub-tiles
 constexpr int kMinPartition = 256;       // tensor-core kernel: smallest partition
+constexpr double kDynItemOverhead = 16.0;  // dynamic schedule: per-item cost, in sub-tiles
+constexpr double kDynTail = 0.25;          // dynamic schedule: tail, in items
 
 struct Plan {
     bool use_mma;
@@ -231,15 +233,24 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
             if (most < 1) most = 1;
             long best_np = 1, best_ps = whole;
             double best_cost = -1.0;
+            // The GQA kernel's dynamic schedule (the workspace holds its counter)
+            // spreads items over the slots as they free up: its time is about
+            //   items * (sub-tiles + overhead) / slots + a tail of a quarter item
+            // (the CTAs still busy when the items run out finish theirs with HBM
+            // to spare). Both models reproduce the measured order of the 70B-GQA
+            // sweep (8 x 32K: 16 partitions 168 us < 32: 172 < 9: 174 < 64: 178).
+            const bool dyn = plan->use_mma && !plan->grouped;
             for (long n = 1; n <= most; ++n) {
                 const int cand_ps = round_up16((int)((max_ctx + n - 1) / n));
                 const long cand_np = (max_ctx + cand_ps - 1) / cand_ps;
                 if (cand_np != n) continue;  // rounding merged two cuts: seen already
                 const long items = units * cand_np;
                 const long waves = (items + slots - 1) / slots;
+                const double sub = (double)(cand_np == 1 ? whole : cand_ps) / 16.0;
                 const double cost =
-                    (double)waves * ((double)(cand_np == 1 ? whole : cand_ps) / 16.0 +
-                                     (cand_np == 1 ? 0.0 : kMmaItemOverhead));
+                    dyn ? (double)items * (sub + (cand_np == 1 ? 0.0 : kDynItemOverhead)) / slots +
+                              kDynTail * sub
+                        : (double)waves * (sub + (cand_np == 1 ? 0.0 : kMmaItemOverhead));
                 if (best_cost < 0.0 || cost < best_cost) {
                     best_cost = cost;
                     best_np = cand_np;
@@ -277,9 +288,13 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
         plan->ws_ml_offset = (o_bytes + 255) / 256 * 256;
         plan->ws_bytes = plan->ws_ml_offset + rows * 2 * sizeof(float);
     }
-    // The persistent tensor-core kernel claims its work items from a counter
+    // The persistent tensor-core GQA kernel claims its work items from a counter
     // in the 256 bytes after the partials (zeroed by the call before it
-    // launches); a workspace without them runs the static schedule.
+    // launches); a workspace without them runs the static schedule. (The
+    // grouped kernel keeps its static schedule: its items are few and long, one
+    // or two per CTA at the measured workloads, so a claim's latency at each
+    // item start cost more than balancing gained: 4-beam CoW 94.9 vs 90.2 us,
+    // 4-token verification 214.5 vs 212 us.)
     plan->sched_offset = (plan->ws_bytes + 255) / 256 * 256;
     plan->ws_full = plan->use_mma && !plan->grouped ? plan->sched_offset + 256 : plan->ws_bytes;
     return PA_OK;

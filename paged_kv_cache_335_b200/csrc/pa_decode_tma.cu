@@ -1672,14 +1672,13 @@ struct GItem {
 // Member m's token limit: its context length, or for query token j of a
 // sequence with n new tokens (the last n of its context_len positions), the
 // causal end ctx - n + j + 1. 0 for members that do not exist.
-__device__ __forceinline__ int gwalk_load(const DecodeParams& p, int num_items, int kbase, int lane,
-                                          int gs, int ipb, bool report) {
-    if (lane >= ipb * gs) return 0;
-    const int u = blockIdx.x + (kbase + lane / gs) * gridDim.x;
-    if (u >= num_items) return 0;
+// Token limit of member m of grouped item u (0 when the member does not exist
+// or reads nothing); `report`: record context lengths out of range (once per
+// member: at its first partition).
+__device__ __forceinline__ int gmember_limit(const DecodeParams& p, int u, int m, int gs,
+                                             bool report) {
     const int part = u % p.num_partitions;
     const int grp = u / p.num_partitions / p.num_kv_heads;
-    const int m = lane % gs;
     if (p.query_start == nullptr) {
         const int s = grp * gs + m;
         if (s >= p.num_seqs) return 0;
@@ -1697,42 +1696,64 @@ __device__ __forceinline__ int gwalk_load(const DecodeParams& p, int num_items, 
     return lim;
 }
 
+__device__ __forceinline__ int gwalk_load(const DecodeParams& p, int num_items, int kbase, int lane,
+                                          int gs, int ipb, bool report) {
+    if (lane >= ipb * gs) return 0;
+    const int u = blockIdx.x + (kbase + lane / gs) * gridDim.x;
+    if (u >= num_items) return 0;
+    return gmember_limit(p, u, lane % gs, gs, report);
+}
+
+// Item u with member limit `lim` on lane l for member l & 7 (any value on lanes
+// whose member does not exist): its fields, tmax included.
+__device__ __forceinline__ GItem gitem_of(const DecodeParams& p, int u, int lim, int gs, int lane) {
+    GItem it;
+    it.valid = u >= 0;
+    it.grp = it.kh = it.part = it.t0 = it.tmax = it.t1_lane = 0;
+    it.row0 = it.nmem = it.tab0 = it.tab_step = 0;
+    if (!it.valid) return it;
+    const int m = lane & (kMaxGroupSeqs - 1);
+    it.part = u % p.num_partitions;
+    const int rest = u / p.num_partitions;
+    it.kh = rest % p.num_kv_heads;
+    it.grp = rest / p.num_kv_heads;
+    it.t0 = it.part * p.partition_size;
+    it.t1_lane = m < gs ? max(it.t0, min(lim, it.t0 + p.partition_size)) : it.t0;
+    it.tmax = __reduce_max_sync(0xffffffffu, it.t1_lane);
+    return it;
+}
+
+// Rows and block-table rows of an item's members.
+__device__ __forceinline__ void gitem_rows(const DecodeParams& p, GItem& it, int gs) {
+    if (p.query_start == nullptr) {
+        it.row0 = it.tab0 = it.grp * gs;
+        it.tab_step = 1;
+        it.nmem = min(gs, p.num_seqs - it.row0);
+    } else {
+        const int sq = it.grp / p.q_chunks, c = it.grp % p.q_chunks;
+        const int q0 = __ldg(p.query_start + sq);
+        it.row0 = q0 + c * gs;
+        it.nmem = min(gs, __ldg(p.query_start + sq + 1) - it.row0);
+        it.tab0 = sq;
+        it.tab_step = 0;
+    }
+}
+
 __device__ __forceinline__ GItem gitem_next(GWalk& w, const DecodeParams& p, int num_items, int gs,
                                             int ipb, int lane, bool report, bool want_empty) {
     for (;;) {
         const int u = blockIdx.x + w.k * gridDim.x;
-        GItem it;
-        it.valid = u < num_items;
-        it.grp = it.kh = it.part = it.t0 = it.tmax = it.t1_lane = 0;
-        it.row0 = it.nmem = it.tab0 = it.tab_step = 0;
-        if (!it.valid) return it;
+        if (u >= num_items) return gitem_of(p, -1, 0, gs, lane);
         if (w.k - w.kbase >= ipb) {
             w.kbase = w.k;
             w.ctx_lane = gwalk_load(p, num_items, w.kbase, lane, gs, ipb, report);
         }
         const int m = lane & (kMaxGroupSeqs - 1);
         const int ctx = __shfl_sync(0xffffffffu, w.ctx_lane, (w.k - w.kbase) * gs + (m < gs ? m : 0));
-        it.part = u % p.num_partitions;
-        const int rest = u / p.num_partitions;
-        it.kh = rest % p.num_kv_heads;
-        it.grp = rest / p.num_kv_heads;
-        it.t0 = it.part * p.partition_size;
-        it.t1_lane = m < gs ? max(it.t0, min(ctx, it.t0 + p.partition_size)) : it.t0;
-        it.tmax = __reduce_max_sync(0xffffffffu, it.t1_lane);
+        GItem it = gitem_of(p, u, ctx, gs, lane);
         ++w.k;
         if (it.tmax > it.t0 || want_empty) {
-            if (p.query_start == nullptr) {
-                it.row0 = it.tab0 = it.grp * gs;
-                it.tab_step = 1;
-                it.nmem = min(gs, p.num_seqs - it.row0);
-            } else {
-                const int sq = it.grp / p.q_chunks, c = it.grp % p.q_chunks;
-                const int q0 = __ldg(p.query_start + sq);
-                it.row0 = q0 + c * gs;
-                it.nmem = min(gs, __ldg(p.query_start + sq + 1) - it.row0);
-                it.tab0 = sq;
-                it.tab_step = 0;
-            }
+            gitem_rows(p, it, gs);
             return it;
         }
     }

@@ -181,3 +181,17 @@ def test_bf16_query_groups_above_64_columns():
     ref = oracle.decode_multi(host["q"], host["k_cache"], host["v_cache"], wl.block_tables,
                               wl.context_lens, wl.query_start, wl.scale, num_threads=G.THREADS)
     G.check_tolerance(G.to_f64(out), ref, "bf16", "128 heads per kv head")
+
+
+def test_large_outputs_of_short_causal_contexts():
+    """Short causal contexts give outputs near single V values (|out| above 4
+    here), where the bf16 output's own rounding exceeds 1e-2: the result must be
+    within the bar of the exact value once that rounding is allowed (measured: a
+    2-token context with exact value -4.20794 returns -4.21875, its correct
+    rounding)."""
+    ctx = [1, 2, 15, 16, 17, 40, 64, 65, 129, 300, 511, 513, 4000, 2500]
+    nq = [1, 2, 15, 3, 9, 8, 1, 17, 4, 300, 0, 33, 4, 7]
+    wl = W.multi_query_case(len(ctx), 64, 8, 128, 16, "bf16", ctx, nq, seed=41)
+    for ps in (-1, 0, 256):
+        errs, out, _ = _step_check(wl, ps)
+        assert errs["max_abs_raw"] > G.BF16_MAX_ABS  # the case this test is for
