@@ -135,8 +135,6 @@ constexpr int kMaxPartitions = 4096;
 constexpr int kAutoPartition = 512;    // CUDA-core kernel: partition when splitting
 constexpr double kMmaItemOverhead = 8.0; // tensor-core kernel: per-item cost, in 16-token sub-tiles
 constexpr int kMinPartition = 256;       // tensor-core kernel: smallest partition
-constexpr double kDynItemOverhead = 16.0;  // dynamic schedule: per-item cost, in sub-tiles
-constexpr double kDynTail = 0.25;          // dynamic schedule: tail, in items
 
 struct Plan {
     bool use_mma;
@@ -233,24 +231,21 @@ int plan_decode(int32_t num_seqs, int32_t num_heads, int32_t max_ctx, const pa_c
             if (most < 1) most = 1;
             long best_np = 1, best_ps = whole;
             double best_cost = -1.0;
-            // The GQA kernel's dynamic schedule (the workspace holds its counter)
-            // spreads items over the slots as they free up: its time is about
-            //   items * (sub-tiles + overhead) / slots + a tail of a quarter item
-            // (the CTAs still busy when the items run out finish theirs with HBM
-            // to spare). Both models reproduce the measured order of the 70B-GQA
-            // sweep (8 x 32K: 16 partitions 168 us < 32: 172 < 9: 174 < 64: 178).
-            const bool dyn = plan->use_mma && !plan->grouped;
+            // (Also under the GQA kernel's dynamic schedule: a model of balanced
+            // items, items x (sub-tiles + overhead) / slots + a tail, ranked the
+            // 70B-GQA sweep well for bf16 (16 partitions 168.4 us vs 9: 170.4) but
+            // not over codes (fp8: 9 partitions 98.8 us, 16: 106.9), and a few
+            // items more than slots leave CTAs running a second item alone at the
+            // end; the waves model picks 9 for both.)
             for (long n = 1; n <= most; ++n) {
                 const int cand_ps = round_up16((int)((max_ctx + n - 1) / n));
                 const long cand_np = (max_ctx + cand_ps - 1) / cand_ps;
                 if (cand_np != n) continue;  // rounding merged two cuts: seen already
                 const long items = units * cand_np;
                 const long waves = (items + slots - 1) / slots;
-                const double sub = (double)(cand_np == 1 ? whole : cand_ps) / 16.0;
                 const double cost =
-                    dyn ? (double)items * (sub + (cand_np == 1 ? 0.0 : kDynItemOverhead)) / slots +
-                              kDynTail * sub
-                        : (double)waves * (sub + (cand_np == 1 ? 0.0 : kMmaItemOverhead));
+                    (double)waves * ((double)(cand_np == 1 ? whole : cand_ps) / 16.0 +
+                                     (cand_np == 1 ? 0.0 : kMmaItemOverhead));
                 if (best_cost < 0.0 || cost < best_cost) {
                     best_cost = cost;
                     best_np = cand_np;

@@ -78,11 +78,12 @@ def test_decode_needs_workspace_when_split(lib):
 
 
 def test_partition_policy(lib):
-    # tensor-core GQA kernel (148 SMs x 4 CTA slots when no GPU is visible), dynamic
-    # schedule: equal partitions, the count minimising items x (sub-tiles + per-item
-    # overhead) / slots + a quarter item of tail
+    # tensor-core GQA kernel (148 SMs x 4 CTA slots when no GPU is visible): equal
+    # partitions, the count minimising waves x (sub-tiles per item + per-item overhead)
     d70 = _desc(num_kv_heads=8)
-    assert lib.pa_decode_num_partitions(8, 64, 32768, ctypes.byref(d70), 0) == 16    # 1024 items
+    assert lib.pa_decode_num_partitions(8, 64, 32768, ctypes.byref(d70), 0) == 9     # 576 items: 1 wave
+    d70q = _desc(num_kv_heads=8, dtype=pa.PA_FP8_E4M3)
+    assert lib.pa_decode_num_partitions(8, 64, 32768, ctypes.byref(d70q), 0) == 9
     assert lib.pa_decode_num_partitions(128, 64, 2303, ctypes.byref(d70), 0) == 1    # 1024 items already
     assert lib.pa_decode_num_partitions(1, 64, 4096, ctypes.byref(d70), 0) == 16     # >= 256 tokens each
     assert lib.pa_decode_num_partitions(1, 64, 300, ctypes.byref(d70), 0) == 2
