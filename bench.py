@@ -494,8 +494,13 @@ def measure_config(w2, device, ps, gs, consumer, args, flush_buf, hbm_peak, read
 
 def e2e_steps(step, steps, warmup):
     """The same step through the Python binding of the C ABI with inputs in
-    pinned HOST memory: H2D of the step's inputs and D2H of the output are
-    inside the timed region."""
+    pinned HOST memory: the H2D copy of every step's inputs and the D2H read of
+    its output are inside the timed region. As a serving loop would issue them,
+    the copies run on two copy streams against double-buffered device inputs and
+    outputs, so step i's inputs cross the link while step i - 1 decodes and its
+    output comes back while step i + 1 decodes; events order every buffer reuse
+    (a buffer is refilled only after the kernels and the read of two steps back
+    are done)."""
     import paged_kv_cache_335_b200 as pa
     torch = step.torch
     wl, v = step.wl, step.vals
@@ -505,14 +510,27 @@ def e2e_steps(step, steps, warmup):
             "slots": step.slots.cpu().pin_memory(), "pairs": step.pairs.cpu().pin_memory()}
     if step.multi:
         host["query_start"] = step.query_start.cpu().pin_memory()
-    dev = {k: torch.empty_like(t, device=v["q"].device) for k, t in host.items()}
-    out_host = torch.empty_like(step.out, device="cpu").pin_memory()
+    devs = [{k: torch.empty_like(t, device=v["q"].device) for k, t in host.items()} for _ in range(2)]
+    outs = [step.out, torch.empty_like(step.out)]
+    outs_host = [torch.empty_like(step.out, device="cpu").pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = outs_host[0].numel() * outs_host[0].element_size()
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_ready, in_free = [ev(), ev()], [ev(), ev()]
+    out_ready, out_free = [ev(), ev()], [ev(), ev()]
 
-    def one():
-        for k in host:
-            dev[k].copy_(host[k], non_blocking=True)
+    def one(i):
+        b = i % 2
+        dev, out = devs[b], outs[b]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(in_free[b])          # the kernels of step i - 2 read these
+            for k in host:
+                dev[k].copy_(host[k], non_blocking=True)
+            in_ready[b].record(s_in)
+        comp.wait_event(in_ready[b])
+        comp.wait_event(out_free[b])             # the read of step i - 2's output is done
         if wl.copy_pairs.shape[0]:
             pa.pa_block_copy(dev["pairs"], v["k_cache"], v["v_cache"])
         if wl.num_tokens and wl.kv_quant:
@@ -521,47 +539,56 @@ def e2e_steps(step, steps, warmup):
         elif wl.num_tokens:
             pa.pa_kv_append(dev["k_new"], dev["v_new"], dev["slots"], v["k_cache"], v["v_cache"])
         if wl.kv_quant and step.multi:
-            pa.pa_decode_multi_quant(step.out, dev["q"], v["k_cache"], v["v_cache"], v["k_scale"],
+            pa.pa_decode_multi_quant(out, dev["q"], v["k_cache"], v["v_cache"], v["k_scale"],
                                      v["v_scale"], dev["tables"], dev["ctx"], dev["query_start"],
                                      wl.scale, max_context_len=wl.max_context_len,
                                      max_query_len=wl.max_query_len, partition_size=step.ps,
                                      workspace=step.ws)
         elif wl.kv_quant and step.group_size > 1:
-            pa.pa_decode_grouped_quant(step.out, dev["q"], v["k_cache"], v["v_cache"],
+            pa.pa_decode_grouped_quant(out, dev["q"], v["k_cache"], v["v_cache"],
                                        v["k_scale"], v["v_scale"], dev["tables"], dev["ctx"],
                                        wl.scale, step.group_size,
                                        max_context_len=wl.max_context_len,
                                        partition_size=step.ps, workspace=step.ws)
         elif wl.kv_quant:
-            pa.pa_decode_quant(step.out, dev["q"], v["k_cache"], v["v_cache"], v["k_scale"],
+            pa.pa_decode_quant(out, dev["q"], v["k_cache"], v["v_cache"], v["k_scale"],
                                v["v_scale"], dev["tables"], dev["ctx"], wl.scale,
                                max_context_len=wl.max_context_len, partition_size=step.ps,
                                workspace=step.ws)
         elif step.multi:
-            pa.pa_decode_multi(step.out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"],
+            pa.pa_decode_multi(out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"],
                                dev["ctx"], dev["query_start"], wl.scale,
                                max_context_len=wl.max_context_len,
                                max_query_len=wl.max_query_len, partition_size=step.ps,
                                workspace=step.ws)
         elif step.group_size > 1:
-            pa.pa_decode_grouped(step.out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"],
+            pa.pa_decode_grouped(out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"],
                                  dev["ctx"], wl.scale, step.group_size,
                                  max_context_len=wl.max_context_len, partition_size=step.ps,
                                  workspace=step.ws)
         else:
-            pa.pa_decode(step.out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"],
+            pa.pa_decode(out, dev["q"], v["k_cache"], v["v_cache"], dev["tables"],
                          dev["ctx"], wl.scale, max_context_len=wl.max_context_len,
                          partition_size=step.ps, workspace=step.ws)
-        out_host.copy_(step.out, non_blocking=True)
+        in_free[b].record(comp)
+        out_ready[b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(out_ready[b])
+            outs_host[b].copy_(out, non_blocking=True)
+            out_free[b].record(s_out)
 
-    for _ in range(warmup):
-        one()
+    for i in range(warmup):
+        one(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
+    e0.record(comp)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(steps):
+        one(i)
+    for b in range(2):
+        comp.wait_event(out_free[b])             # every output is back in host memory
+    e1.record(comp)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     return ms, h2d, d2h
