@@ -806,13 +806,34 @@ __device__ __forceinline__ void code_pairs_f16(uint32_t t, uint32_t& p0, uint32_
             "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
             : "=r"(p0), "=r"(p1) : "r"(t));
     } else {
-        const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
-        uint32_t u0 = __byte_perm(t, 0x64646464u, 0x5140), u1 = __byte_perm(t, 0x64646464u, 0x7362);
-        const __half2 h0 = __hsub2(*reinterpret_cast<__half2*>(&u0), bias);
-        const __half2 h1 = __hsub2(*reinterpret_cast<__half2*>(&u1), bias);
-        p0 = *reinterpret_cast<const uint32_t*>(&h0);
-        p1 = *reinterpret_cast<const uint32_t*>(&h1);
+        // int8 (bytes already offset by 128 in code_word): 1024 + byte = code + 1152,
+        // exact in f16; the consumers take the 1152 out once per sum (kInt8Bias)
+        p0 = __byte_perm(t, 0x64646464u, 0x5140);
+        p1 = __byte_perm(t, 0x64646464u, 0x7362);
     }
+}
+
+// The offset the tensor-core consumers' int8 operands carry (code + 1152): a
+// score over such a K row exceeds the true one by 1152 x the sum of q, an
+// output over such V rows by 1152 (times the V scale) once normalised.
+constexpr float kInt8Bias = 1152.f;
+
+// 1152 x the sum of q over head_dim for query rows 2c and 2c + 1 (b0, b1), from
+// the f16 q fragments thread (r, c) holds for row r (code consumers' B operand):
+// a fixed-order sum over the thread's 32 elements, then over the four threads of
+// the row.
+__device__ __forceinline__ void int8_qk_bias(const uint4 (&q)[4], int c, float& b0, float& b1) {
+    float sum = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sum += f16_lo(w[i]) + f16_hi(w[i]);
+    }
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+    b0 = kInt8Bias * __shfl_sync(0xffffffffu, sum, 4 * (2 * c));
+    b1 = kInt8Bias * __shfl_sync(0xffffffffu, sum, 4 * (2 * c + 1));
 }
 
 template <typename TC>
@@ -952,7 +973,7 @@ template <int D, bool kCodes = false>
 __device__ __forceinline__ void mma_store_item(const DecodeParams& p, int64_t head0, int group,
                                                int part, int r, int c, const float (&acc)[D / 16][4],
                                                float m0, float m1, float l0, float l1,
-                                               float vs = 1.f) {
+                                               float vs = 1.f, float obias = 0.f) {
     constexpr int MT = D / 16;
     const int P = p.num_partitions;
     const int DQ = kCodes ? p.head_dim : D;  // out / workspace row length
@@ -962,6 +983,10 @@ __device__ __forceinline__ void mma_store_item(const DecodeParams& p, int64_t he
         inv0 *= vs;
         inv1 *= vs;
     }
+    // int8 codes: the accumulator carries 1152 x the weights (obias = 1152 x the
+    // V scale), taken out after the normalisation
+    const float ob0 = l0 > 0.f ? obias : 0.f, ob1 = l1 > 0.f ? obias : 0.f;
+    auto nv = [&](float a, float inv, float ob) { return obias != 0.f ? fmaf(a, inv, -ob) : a * inv; };
     const int n0 = 2 * c, n1 = 2 * c + 1;
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
@@ -970,17 +995,17 @@ __device__ __forceinline__ void mma_store_item(const DecodeParams& p, int64_t he
         if (P == 1) {
             if (n0 < group)
                 *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + (head0 + n0) * DQ + d0) =
-                    pack_bf16x2(acc[t][0] * inv0, acc[t][2] * inv0);
+                    pack_bf16x2(nv(acc[t][0], inv0, ob0), nv(acc[t][2], inv0, ob0));
             if (n1 < group)
                 *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + (head0 + n1) * DQ + d0) =
-                    pack_bf16x2(acc[t][1] * inv1, acc[t][3] * inv1);
+                    pack_bf16x2(nv(acc[t][1], inv1, ob1), nv(acc[t][3], inv1, ob1));
         } else {
             if (n0 < group)
                 *reinterpret_cast<float2*>(p.ws_o + ((head0 + n0) * P + part) * DQ + d0) =
-                    make_float2(acc[t][0] * inv0, acc[t][2] * inv0);
+                    make_float2(nv(acc[t][0], inv0, ob0), nv(acc[t][2], inv0, ob0));
             if (n1 < group)
                 *reinterpret_cast<float2*>(p.ws_o + ((head0 + n1) * P + part) * DQ + d0) =
-                    make_float2(acc[t][1] * inv1, acc[t][3] * inv1);
+                    make_float2(nv(acc[t][1], inv1, ob1), nv(acc[t][3], inv1, ob1));
         }
     }
     if (P > 1 && r == 0) {
@@ -1330,9 +1355,11 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
             load_q(nxt, qnxt);
         }
         int qsh = 0;  // over codes: this item's q to f16, scaled by 2^-qsh
+        float qb0 = 0.f, qb1 = 0.f;  // int8: 1152 x sum of q of query rows 2c, 2c + 1
         if constexpr (kCodes) {
             qsh = q_shift_warp(q_raw_amax(qcur));
             q_raw_to_f16(qcur, pow2i(-qsh), qcur);
+            if constexpr (std::is_same<TC, Int8Code>::value) int8_qk_bias(qcur, c, qb0, qb1);
         }
         const int64_t head0 = (int64_t)cur.s * p.num_heads + (int64_t)cur.kh * group;
         if (cur.t0 >= cur.t1) {
@@ -1371,6 +1398,12 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 float sc[4];
                 if constexpr (kCodes) {
                     codes_qk<TC>(kb, qcur, r, c, sc);
+                    if constexpr (std::is_same<TC, Int8Code>::value) {
+                        sc[0] -= qb0;
+                        sc[1] -= qb1;
+                        sc[2] -= qb0;
+                        sc[3] -= qb1;
+                    }
                     uint4 vr[4];
                     codes_load_v(vb, r, c, vr);
                     __syncwarp();
@@ -1439,7 +1472,9 @@ decode_tma_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                 // One warp holds the whole item: normalise and store from registers.
                 if (warp == 0)
                     mma_store_item<D, kCodes>(p, head0, group, cur.part, r, c, acc, m0, m1, l0, l1,
-                                              kCodes ? __ldg(p.v_scale + cur.kh) : 1.f);
+                                              kCodes ? __ldg(p.v_scale + cur.kh) : 1.f,
+                                              std::is_same<TC, Int8Code>::value
+                                                  ? kInt8Bias * __ldg(p.v_scale + cur.kh) : 0.f);
                 if constexpr (kConsumerWarps == 2) named_barrier(1, 64);  // buffer free again
             } else {
                 // Cross-warp merge of this item, in fixed warp order. Buffers alternate
@@ -2321,11 +2356,15 @@ __device__ __forceinline__ void pv_codes(uint32_t vb, int sub_bytes, int lane, i
 template <int D, bool kCodes = false>
 __device__ __forceinline__ void grouped_store_col(const DecodeParams& p, int64_t row, int part, int r,
                                                   int c, int e, const float (&acc)[D / 16][4],
-                                                  float m, float l, float vs = 1.f) {
+                                                  float m, float l, float vs = 1.f,
+                                                  float obias = 0.f) {
     constexpr int MT = D / 16;
     const int P = p.num_partitions;
     const int DQ = kCodes ? p.head_dim : D;  // out / workspace row length
     const float inv = (l > 0.f ? 1.f / l : 0.f) * vs;  // vs: V scale of a quantised cache
+    // int8 codes: 1152 x the weights in the accumulator (obias = 1152 x vs)
+    const float ob = l > 0.f ? obias : 0.f;
+    auto nv = [&](float a) { return obias != 0.f ? fmaf(a, inv, -ob) : a * inv; };
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
         // rows r and r + 8 of m-tile t: head_dim 16t + r and 16t + 8 + r (codes:
@@ -2334,12 +2373,12 @@ __device__ __forceinline__ void grouped_store_col(const DecodeParams& p, int64_t
         if (kCodes && d0 >= DQ) continue;
         if (P == 1) {
             __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + row * DQ;
-            o[d0] = __float2bfloat16_rn(acc[t][e] * inv);
-            o[d1] = __float2bfloat16_rn(acc[t][e + 2] * inv);
+            o[d0] = __float2bfloat16_rn(nv(acc[t][e]));
+            o[d1] = __float2bfloat16_rn(nv(acc[t][e + 2]));
         } else {
             float* o = p.ws_o + (row * P + part) * DQ;
-            o[d0] = acc[t][e] * inv;
-            o[d1] = acc[t][e + 2] * inv;
+            o[d0] = nv(acc[t][e]);
+            o[d1] = nv(acc[t][e + 2]);
         }
     }
     if (P > 1 && r == 0) {
@@ -2482,6 +2521,17 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
     GItem cur = gitem_next(walk, p, num_items, gs, ipb, lane, warp == 0, P == 1);
     uint4 q[NT][KCH];
     float sl = load_q(cur, q);  // the item's score scale (log2 units, positive)
+    // int8 codes: 1152 x the sum of q of the thread's score columns 8j + 2c, + 1
+    constexpr bool kInt8 = std::is_same<TC, Int8Code>::value;
+    float qb[NT][2];
+    auto q_bias = [&]() {
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            qb[j][0] = qb[j][1] = 0.f;
+            if constexpr (kInt8) int8_qk_bias(q[j], c, qb[j][0], qb[j][1]);
+        }
+    };
+    q_bias();
     while (cur.valid && !dead) {
         GItem nxt = gitem_next(walk, p, num_items, gs, ipb, lane, warp == 0, P == 1);
         int t1a[NT], t1b[NT];
@@ -2520,8 +2570,15 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                     for (int u = 0; u < SUB; ++u) {
                         if constexpr (kCodes) {
 #pragma unroll
-                            for (int j = 0; j < NT; ++j)
+                            for (int j = 0; j < NT; ++j) {
                                 codes_qk<TC>(kb + u * G::kSubBytes, q[j], r, c, sc[u][j]);
+                                if constexpr (kInt8) {
+                                    sc[u][j][0] -= qb[j][0];
+                                    sc[u][j][1] -= qb[j][1];
+                                    sc[u][j][2] -= qb[j][0];
+                                    sc[u][j][3] -= qb[j][1];
+                                }
+                            }
                         } else {
                             mma_qk_n<D, NT>(kb + u * G::kSubBytes, q, r, c, sc[u]);
                         }
@@ -2575,12 +2632,14 @@ decode_tma_grouped_kernel(const __grid_constant__ CUtensorMap kmap,
                         (int64_t)(cur.row0 + m) * p.num_heads + (int64_t)cur.kh * group + hd;
                     grouped_store_col<D, kCodes>(p, row, cur.part, r, c, e, acc[j],
                                                  e == 0 ? ma[j] : mb[j], e == 0 ? la[j] : lb[j],
-                                                 kCodes ? __ldg(p.v_scale + cur.kh) : 1.f);
+                                                 kCodes ? __ldg(p.v_scale + cur.kh) : 1.f,
+                                                 kInt8 ? kInt8Bias * __ldg(p.v_scale + cur.kh) : 0.f);
                 }
             }
         }
         cur = nxt;
         sl = load_q(cur, q);
+        q_bias();
     }
 }
 
