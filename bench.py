@@ -123,8 +123,10 @@ def pct(xs, scale=1.0, nd=2):
     return {"p10": round(q(0.1), nd), "p50": round(q(0.5), nd), "p90": round(q(0.9), nd)}
 
 
-def stream_read_gbs(device, reps=10):
-    """Read bandwidth of the library's read-only streaming kernel over 4 GiB."""
+def stream_read_gbs(device, reps=20):
+    """Read bandwidth of the library's read-only streaming kernel over 4 GiB: the
+    best of `reps` back-to-back launches (a roof is the most the hardware gives;
+    decode fractions of it take the decode's typical launch)."""
     import torch
 
     import paged_kv_cache_335_b200 as pa
@@ -136,18 +138,21 @@ def stream_read_gbs(device, reps=10):
     st = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
     args = (ctypes.c_void_p(buf.data_ptr()), ctypes.c_size_t(STREAM_BYTES),
             ctypes.c_void_p(part.data_ptr()), ctas, st)
-    times = []
-    for i in range(reps + 3):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        if lib.pa_stream_read(*args) != 0:
+            raise RuntimeError("pa_stream_read failed")
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for e0, e1 in evs:
         e0.record()
         if lib.pa_stream_read(*args) != 0:
             raise RuntimeError("pa_stream_read failed")
         e1.record()
-        torch.cuda.synchronize()
-        if i >= 3:
-            times.append(e0.elapsed_time(e1))
+    torch.cuda.synchronize()
+    times = [e0.elapsed_time(e1) for e0, e1 in evs]
     del buf
-    return STREAM_BYTES / (statistics.median(times) / 1e3) / 1e9
+    return STREAM_BYTES / (min(times) / 1e3) / 1e9
 
 
 def peaks():

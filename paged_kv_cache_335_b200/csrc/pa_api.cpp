@@ -356,14 +356,17 @@ static int decode_impl(void* out, const void* q, const void* k_cache, const void
         if (!ws_aligned) return fail(PA_ERR_ALIGN, "pa_decode: workspace must be 256-byte aligned");
     }
     // the dynamic schedule when the workspace holds its counter and there are
-    // more items than CTA slots (with one item per CTA a claim only adds its
-    // latency: 70B-GQA at 9 partitions 172.6 us claimed vs 170.5-171.6 static);
-    // the results are the same bit for bit either way: an item's arithmetic
-    // does not depend on the CTA that runs it
+    // at least two items per CTA slot: with fewer there is little to balance and
+    // a claim only adds its latency (measured, claimed vs static: 70B-GQA at 9
+    // partitions, one item per slot, 172.6 vs 170.5-171.6 us; 4-beam CoW per
+    // sequence, 1.7 per slot, 111.0 vs 108.8; 256 x 1K, 3.5 per slot, 163.9 vs
+    // 172.5; 70B at 512-token partitions, 6.9 per slot, 178.6 vs 186.7). The
+    // results are the same bit for bit either way: an item's arithmetic does not
+    // depend on the CTA that runs it.
     const long mma_items = (long)plan.num_partitions * cache->num_kv_heads * num_seqs;
     const bool dyn_sched = plan.ws_full > plan.ws_bytes && workspace && ws_aligned &&
                            workspace_bytes >= plan.ws_full &&
-                           mma_items > (long)sm_count() * pa::mma_ctas_per_sm();
+                           mma_items >= 2L * sm_count() * pa::mma_ctas_per_sm();
     pa::DecodeParams p;
     p.out = out;
     p.q = q;

@@ -4,7 +4,7 @@ With the workspace size that pa_decode_workspace_size reports and more work
 items (partition, kv head, sequence) than CTA slots, the kernel's CTAs claim
 items from a counter in the workspace, so CTAs that stream faster take more
 items; with a workspace that holds only the partial results (or none, unsplit),
-or no more items than slots, they take item u = CTA + k x grid. The cases below
+or fewer than two items per slot, they take item u = CTA + k x grid. The cases below
 with splits have thousands of items, so both schedules run. An item's arithmetic does not depend on the CTA that runs it, so the two
 schedules must give the same output bit for bit, and both must meet the bf16
 bar against the oracle: on ragged contexts (empty sequences and partitions past
