@@ -238,3 +238,33 @@ def test_q_magnitudes_outside_f16_range(fmt):
                 got = decode(qk, wl.scale * 2.0 ** -k, grouped)
                 assert torch.isfinite(got.float()).all()
                 assert G.dev_bits_equal(got, base), f"{fmt} H={H}/{Hkv} grouped={grouped} 2^{k}"
+
+
+@pytest.mark.parametrize("fmt", ["int8", "fp8"])
+def test_same_sign_q_long_context(fmt):
+    """The worst case for the int8 offset the tensor-core consumers take out once
+    per sum (scores minus 1152 x the sum of q): every q element of one sign, so
+    the sum of q and the offset it carries are as large as they can be, over 4K-
+    token contexts, on the GQA consumer (split and unsplit) and the grouped one.
+    Must meet the bars against the oracle like any other q (fp8, which carries no
+    offset, is the control)."""
+    ctx = [4096, 3001, 17, 1]
+    wl = W.quantized(G.custom(len(ctx), 16, 2, 128, 16, "bf16", ctx, seed=37), fmt)
+    vals = W.make_values(wl, DEV, poison=False)
+    vals["q"].copy_(vals["q"].abs())
+    host = _host(vals)
+    d = G.device_tensors(wl, vals)
+    pa.pa_kv_append_quant(vals["k_new"], vals["v_new"], d["slots"], vals["k_cache"], vals["v_cache"],
+                          vals["k_scale"], vals["v_scale"])
+    ref = _oracle_step(wl, host)
+    for grouped, ps in ((False, -1), (False, 512), (True, -1)):
+        out = torch.empty_like(vals["q"])
+        args = (out, vals["q"], vals["k_cache"], vals["v_cache"], vals["k_scale"], vals["v_scale"],
+                d["tables"], d["ctx"], wl.scale)
+        if grouped:
+            pa.pa_decode_grouped_quant(*args, 2, max_context_len=wl.max_context_len, partition_size=ps)
+        else:
+            pa.pa_decode_quant(*args, max_context_len=wl.max_context_len, partition_size=ps)
+        pa.pa_sync_check()
+        assert G.last_kernel() in (pa.PA_KERNEL_MMA,) + G.kernel_set(pa.PA_KERNEL_GROUPED)
+        G.check_tolerance(G.to_f64(out), ref, "bf16", f"{fmt} same-sign q grouped={grouped} ps={ps}")
