@@ -158,8 +158,18 @@ int pa_kv_append(const void* k, const void* v, const int64_t* slot_mapping,
  *   cache         host pointer; cache->num_kv_heads is the kv-head count.
  *   partition_size  0 = library policy; -1 = never split; otherwise the
  *                 tokens per partition, a positive multiple of 16.
- *   workspace     device scratch of at least pa_decode_workspace_size(...)
- *                 bytes (same arguments); may be NULL when that size is 0.
+ *   workspace     device scratch of pa_decode_workspace_size(...) bytes (same
+ *                 arguments), 256-byte aligned; may be NULL when that size is 0.
+ *                 For grouped-query heads (2..8 query heads per kv head) the
+ *                 size includes 256 bytes after the partial results for the
+ *                 tensor-core kernel's work-item counter, which the call zeroes
+ *                 (cudaMemsetAsync on `stream`) before the kernel: with at least
+ *                 two work items per CTA slot, the CTAs claim items from it so
+ *                 that those streaming faster take more. A workspace that holds
+ *                 only the partial results (or none when the call does not
+ *                 split) is accepted and runs the static schedule instead
+ *                 (item u to CTA u mod grid); the results are the same bit for
+ *                 bit. A workspace must not be used by two calls at once.
  * The result does not depend on the physical placement of blocks: the
  * arithmetic order depends only on logical token positions.
  */
@@ -171,10 +181,13 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * pa_decode_workspace_size — bytes of device scratch pa_decode needs for the
- * same (num_seqs, num_heads, max_context_len, cache, partition_size); 0 when
- * the call will not split. Returns 0 and sets the last error on bad
- * arguments. Queries the current device's SM count (cached per device).
+ * pa_decode_workspace_size — bytes of device scratch pa_decode takes for the
+ * same (num_seqs, num_heads, max_context_len, cache, partition_size): the
+ * partial results of a split context, plus 256 bytes for the tensor-core
+ * kernel's work-item counter when the heads are grouped-query (so 256 for an
+ * unsplit grouped-query call, 0 for an unsplit call on the CUDA-core kernel).
+ * Returns 0 and sets the last error on bad arguments. Queries the current
+ * device's SM count (cached per device).
  */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads,
                                 int32_t max_context_len,
