@@ -458,8 +458,9 @@ int pa_block_swap(const int64_t* src_dst_pairs, int32_t num_pairs,
  * cannot call cudaMalloc where they decode (code inside a memory arena sized up
  * front, plug-ins of an engine that owns all device allocations, loops that
  * must never enter an allocator). This entry point computes exactly what
- * pa_decode computes, with the same arguments minus the workspace: when the
- * context is split, the partial results go to a buffer of
+ * pa_decode computes, with the same arguments minus the workspace: the
+ * workspace pa_decode_workspace_size asks for (the partial results of a split
+ * context, the work-item counter of grouped-query heads) is a buffer of
  * PA_NOALLOC_SCRATCH_BYTES inside the library. It allocates nothing.
  *
  * The first call on a device looks up that buffer's device address

@@ -4,11 +4,12 @@
 // Some callers cannot call cudaMalloc (or any allocating routine) where they
 // decode: code that runs inside a memory arena sized up front, plug-ins of a
 // host engine that owns every device allocation, or loops that must never
-// enter an allocator. When a long context is split into partitions, pa_decode
-// needs a workspace for the partial results; this entry point takes that
-// workspace from a buffer inside the library instead: a file-scope device
-// array of PA_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library
-// holds until the process exits. Nothing here allocates.
+// enter an allocator. pa_decode needs a workspace for the partial results of a
+// split context and, for grouped-query heads, for the tensor-core kernel's
+// work-item counter; this entry point takes that workspace from a buffer inside
+// the library instead: a file-scope device array of PA_NOALLOC_SCRATCH_BYTES,
+// which every GPU that loads the library holds until the process exits.
+// Nothing here allocates.
 //
 // On the host, `s_scratch` names a host-side stand-in, not device memory, so
 // its device address is looked up with cudaGetSymbolAddress, with the device
@@ -20,7 +21,7 @@
 // Every call shares the one buffer per device: calls whose kernels overlap on
 // the GPU (different streams, no ordering between them) race on it. The buffer
 // needs no clearing: each call writes every partial result before its merge
-// reads it.
+// reads it, and zeroes the counter before its kernel.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
