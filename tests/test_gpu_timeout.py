@@ -16,22 +16,25 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _decode(wl, vals, d, out, gs):
+def _decode(wl, vals, d, out, gs, ps=0):
     kc, vc = vals["k_cache"], vals["v_cache"]
     if gs > 1:
         pa.pa_decode_grouped(out, vals["q"], kc, vc, d["tables"], d["ctx"], wl.scale, gs,
-                             max_context_len=wl.max_context_len, partition_size=0)
+                             max_context_len=wl.max_context_len, partition_size=ps)
     else:
         pa.pa_decode(out, vals["q"], kc, vc, d["tables"], d["ctx"], wl.scale,
-                     max_context_len=wl.max_context_len, partition_size=0)
+                     max_context_len=wl.max_context_len, partition_size=ps)
 
 
-@pytest.mark.parametrize("name,kw,gs", [
-    ("llama70b_gqa", dict(num_seqs=1, context_len=1024), 1),   # persistent tensor-core kernel
-    ("tiny", {}, 1),                                             # CUDA-core kernel
-    ("cow_beam4", dict(num_prompts=2, prompt_len=300, max_suffix=30), 4),   # grouped kernel
+@pytest.mark.parametrize("name,kw,gs,ps", [
+    ("llama70b_gqa", dict(num_seqs=1, context_len=1024), 1, 0),   # persistent tensor-core kernel
+    # the same kernel under its dynamic item schedule (2048 items claimed from the
+    # workspace's counter: the queue's waits give up too)
+    ("llama70b_gqa", dict(num_seqs=8, context_len=8192), 1, 256),
+    ("tiny", {}, 1, 0),                                             # CUDA-core kernel
+    ("cow_beam4", dict(num_prompts=2, prompt_len=300, max_suffix=30), 4, 0),   # grouped kernel
 ])
-def test_skipped_load_times_out_then_recovers(name, kw, gs):
+def test_skipped_load_times_out_then_recovers(name, kw, gs, ps):
     wl = W.make(name, **kw)
     vals = W.make_values(wl, DEV)
     d = G.device_tensors(wl, vals)
@@ -45,7 +48,7 @@ def test_skipped_load_times_out_then_recovers(name, kw, gs):
     lib.pa_test_skip_load(1)
     try:
         t0 = time.time()
-        _decode(wl, vals, d, out, gs)
+        _decode(wl, vals, d, out, gs, ps)
         with pytest.raises(pa.PAError) as e:
             pa.pa_sync_check()
         assert e.value.code == pa.PA_ERR_TIMEOUT
@@ -54,7 +57,7 @@ def test_skipped_load_times_out_then_recovers(name, kw, gs):
         lib.pa_test_skip_load(-1)
     pa.pa_sync_check()                                  # status was cleared
     out2 = torch.empty_like(vals["q"])
-    _decode(wl, vals, d, out2, gs)
+    _decode(wl, vals, d, out2, gs, ps)
     pa.pa_sync_check()
     if gs > 1:
         assert G.last_kernel() in G.kernel_set(pa.PA_KERNEL_GROUPED)
